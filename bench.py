@@ -1,0 +1,411 @@
+"""Throughput of the two-point ZO probe step on B200 (one JSON line on rank 0).
+
+One step = zo_probe_plan + zo_score (both candidates of every prompt, one
+packed batch) + zo_step (c and the banked update), on the OPT-13B-shaped
+decoder with batch 64 by default (synthetic ragged prompts, random-init bf16
+weights drawn on the device).  The metric is scored tokens/s (prefill tokens
+of the physical batch) with ZO steps/s beside it; the GEMM kernel's live
+roofline, the whole-step roofline fraction, the end-to-end number through
+the public API with host buffers, the oracle on the host cores, the SM
+clocks and the kernel launch count are reported on the same line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload opt-13b-b64]
+    python bench.py --impl reference ...   (the CPU oracle as the reference arm)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from zeroth_order_fine_b200 import workload as wl  # noqa: E402
+
+METRIC = "ZO steps/s & scored tokens/s (OPT-13B shape, batch 64); % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---- algorithmic work of one step ----------------------------------------------------
+
+def step_work(w: wl.Workload, batches, n_slots: int):
+    """Algorithmic FLOPs and HBM bytes of one step over the given per-rank batches."""
+    sh = w.shape
+    es = 2 if sh.dtype == wl.DTYPE_BF16 else 4
+    flops = 0.0
+    bytes_ = 0.0
+    T_all = 0
+    S_all = 0
+    for b in batches:
+        rows = list(b.prompts) * 2 + list(b.fg_prompts)
+        tls = list(b.target_lens) * 2 + list(b.fg_target_lens)
+        T = sum(len(r) for r in rows)
+        S = int(sum(tls))
+        T_all += T
+        S_all += S
+        flops += 2.0 * sh.body_params() * T                      # every decoder linear, all rows
+        flops += 2.0 * sh.vocab * sh.d_model * S                 # lm_head at scored positions only
+        ctx = sum(L * (L + 1) / 2 for L in (len(r) for r in rows))
+        flops += 4.0 * ctx * sh.q_dim * sh.n_layers              # QK^T and PV, causal
+        for m in w.matrices:                                     # shrink + expand of the bank
+            di, do = sh.matrix_dims(m)
+            flops += 2.0 * T * (di + do) * w.rank * (1 + n_slots) * sh.n_layers
+        # bytes: weights once; activations ~ 10 passes of T x d per layer (fp32 residual
+        # read+write twice, bf16 normalised inputs, q/k/v, attention out, FFN act in/out)
+        act = T * (8 * sh.d_model * 4 + (2 * sh.d_model + sh.q_dim + 2 * sh.kv_dim) * es
+                   + 2 * sh.d_ffn * es) * sh.n_layers
+        bytes_ += act + sh.vocab * sh.d_model * es
+    bytes_ += (sh.body_params() + sh.vocab * sh.d_model) * es    # per rank weights, once
+    return flops, bytes_, T_all, S_all
+
+
+# ---- clocks during the timed region -----------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- the oracle on the host cores -------------------------------------------------------
+
+def oracle_sample(w: wl.Workload, n_prompts: int = 2, seed: int = 0):
+    """Time the CPU oracle on a bounded sample of the workload.
+
+    The sample is n_prompts prompts of the workload's batch (both candidate
+    rows each) through ONE decoder layer plus the final norm and the lm_head
+    at their scored positions; the per-layer time is scaled by n_layers.  The
+    weights of the sample are drawn with numpy's generator (their values do
+    not change the oracle's work; the oracle's own counter-stream init of a
+    full-width layer would take longer than the scoring itself).
+    """
+    import torch
+
+    from oracle import model as om
+    from oracle import zo as ozo
+    sh = w.shape
+    one = wl.shrink_shape(sh, n_layers=1)
+    rng = np.random.default_rng(seed)
+
+    def t(*shape, mean=0.0):
+        return torch.from_numpy(rng.standard_normal(shape, dtype=np.float32) * 0.02 + mean).double()
+
+    d = sh.d_model
+    layer = {}
+    for m in sh.matrices():
+        di, do = sh.matrix_dims(m)
+        layer[f"W{m}"] = t(do, di)
+        if sh.arch == wl.ARCH_OPT:
+            layer[f"b{m}"] = t(do)
+    layer["ln1_w"], layer["ln2_w"] = t(d, mean=1.0), t(d, mean=1.0)
+    if sh.arch == wl.ARCH_OPT:
+        layer["ln1_b"], layer["ln2_b"] = t(d), t(d)
+    else:
+        layer["q_norm"], layer["k_norm"] = t(sh.head_dim, mean=1.0), t(sh.head_dim, mean=1.0)
+    tok = t(sh.vocab, d)
+    weights = om.Weights(one, tok, t(sh.max_pos, d) if sh.arch == wl.ARCH_OPT else None,
+                         t(d, mean=1.0), t(d) if sh.arch == wl.ARCH_OPT else None,
+                         tok if sh.tie_lm_head else t(sh.vocab, d), [layer])
+    run = ozo.OracleRun(weights, w.run_seed, w.nu, w.rank, [0], w.matrices, w.scale_mode)
+    batch = wl.make_batch(w, batch=n_prompts, fg_rows=min(w.fg_rows, n_prompts))
+    run.plan(0, w.eps)
+    t0 = time.perf_counter()
+    run.score(batch.prompts, batch.target_lens, batch.fg_prompts, batch.fg_target_lens)
+    run.step(w.lr)
+    secs_one = time.perf_counter() - t0
+    # the lm_head part is already inside secs_one once; scale only the layer part
+    hs = torch.zeros(int(2 * batch.target_lens.sum() + batch.fg_target_lens.sum()), d,
+                     dtype=torch.float64)
+    t1 = time.perf_counter()
+    logits = hs @ weights.lm_head.T
+    torch.logsumexp(logits, dim=-1)
+    secs_head = time.perf_counter() - t1
+    secs_step = (secs_one - secs_head) * sh.n_layers + secs_head
+    T = batch.n_tokens_physical
+    return {"secs_per_sample_step": secs_step, "tokens": T, "tokens_per_s": T / secs_step,
+            "sample": (f"{n_prompts} prompts ({2 * n_prompts} candidate rows, {T} tokens) "
+                       f"through 1 of {sh.n_layers} layers + lm_head at the scored positions, "
+                       f"layer time scaled x{sh.n_layers}; oracle float64 on the host cores"),
+            "cores": torch.get_num_threads()}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w, n_prompts=args.ref_prompts, seed=i)
+        if i >= args.warmup:
+            per_step.append(r)
+    tok = sum(r["tokens"] for r in per_step)
+    secs = sum(r["secs_per_sample_step"] for r in per_step)
+    value = tok / secs
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "scored tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * secs / len(per_step), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "model": w.shape.name, "global_batch": w.batch},
+            "cpu_baseline": {"value": value, "unit": "scored tokens/s", "kind": "oracle",
+                             "cores": per_step[0]["cores"], "sample": per_step[0]["sample"]},
+            "e2e": {"value": value, "unit": "scored tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- the CUDA path ------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="opt-13b-b64", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-prompts", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cuda-cores", action="store_true", help="GEMMs on CUDA cores only")
+    args = ap.parse_args()
+    w = wl.WORKLOADS[args.workload]
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    from zeroth_order_fine_b200 import zo
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    stream = torch.cuda.current_stream()
+
+    sh = w.shape
+    batch = wl.make_batch(w, seed=w.data_seed + 1000 * rank)
+    model = zo.DeviceModel(sh, w.weight_seed)
+    tg = zo.make_targets(sh.n_layers, w.matrices, w.scale_mode)
+    T = batch.n_tokens_physical
+    S = int(2 * batch.target_lens.sum() + batch.fg_target_lens.sum())
+    R = 2 * w.batch + len(batch.fg_prompts)
+    h = zo.Handle(model, w.run_seed, w.nu, w.rank, tg, max_tokens=T, max_rows=R, max_scored=S,
+                  max_slots=8, impl=1 if args.cuda_cores else 0, profile=1)
+    toks = torch.from_numpy(batch.packed()).cuda()
+    ftoks = torch.from_numpy(batch.fg_packed()).cuda() if batch.fg_prompts else None
+    sums = torch.zeros(2, dtype=torch.float64, device="cuda")
+    step_no = [0]
+
+    def one_step(tokens, want_c=False):
+        t = step_no[0]
+        h.zo_probe_plan(t, w.eps)
+        if ftoks is not None:
+            h.zo_score_cobatch(tokens, batch.seq_lens, batch.target_lens, ftoks, batch.fg_seq_lens,
+                               batch.fg_target_lens)
+        else:
+            h.zo_score(tokens, batch.seq_lens, batch.target_lens)
+        if world > 1:
+            h.zo_objective_sums(sums)
+            dist.all_reduce(sums)
+            c = h.zo_step_from_sums(w.lr, sums, want_c=want_c)
+        else:
+            c = h.zo_step(w.lr, want_c=want_c)
+        step_no[0] += 1
+        return c
+
+    for _ in range(args.warmup):
+        one_step(toks)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s0 = h.zo_stats()
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    clk = ClockSampler(gpu_uuid)
+    clk.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        one_step(toks)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = clk.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    s1 = h.zo_stats()
+    if s1["last_error_code"] not in (0,):
+        raise RuntimeError(f"library reported error {s1['last_error_code']} during the run")
+    if world > 1:
+        t_ = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t_, op=dist.ReduceOp.MAX)
+        ms = float(t_.item())
+
+    # e2e: the same steps through the public API with host buffers (pinned), the
+    # H2D copy of the step's tokens and the D2H read of c inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_toks = torch.from_numpy(batch.packed()).pin_memory()
+        dev_buf = torch.empty_like(toks)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            dev_buf.copy_(host_toks, non_blocking=True)
+            one_step(dev_buf, want_c=True)           # zo_step copies c (8 bytes) to the host
+        torch.cuda.synchronize()
+        e2e_s = (time.perf_counter() - t0) / args.steps
+        if world > 1:
+            t_ = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t_, op=dist.ReduceOp.MAX)
+            e2e_s = float(t_.item())
+        e2e = {"value": world * T / e2e_s, "unit": "scored tokens/s",
+               "h2d_bytes_per_step": int(host_toks.numel() * 4), "d2h_bytes_per_step": 8}
+
+    peaks, peak_kind = load_peaks()
+    n_slots = s1["bank_slots"]
+    flops, bytes_, T1, S1 = step_work(w, [batch], n_slots)
+    flops_all = flops * world
+    tok_s = world * T / (ms / 1000.0)
+    steps_s = 1000.0 / ms
+    d_ms = s1["tc_gemm_ms"] - s0["tc_gemm_ms"]
+    d_fl = s1["tc_gemm_flops"] - s0["tc_gemm_flops"]
+    d_n = s1["tc_gemm_launches"] - s0["tc_gemm_launches"]
+    gemm_tflops = d_fl / (d_ms / 1000.0) / 1e12 if d_ms > 0 else None
+    peak_t = peaks["bf16_tflops_sustained"]
+    roof_t = max(flops / (peak_t * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    line = {
+        "metric": METRIC, "value": tok_s, "unit": "scored tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (random-init weights drawn on the device, Zipf(1.1) ragged prompts)",
+        "config": {"workload": w.name, "model": sh.name, "global_batch": w.batch * world,
+                   "prompts_per_gpu": w.batch, "physical_rows_per_gpu": R,
+                   "tokens_per_gpu": T, "scored_positions_per_gpu": S, "rank": w.rank,
+                   "targets": [wl.MATRIX_NAMES[m] for m in w.matrices],
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (weights %.1f GB read every step)" %
+                         ((sh.body_params() + sh.vocab * sh.d_model) * 2 / 1e9),
+                   "gemm_impl": "cuda-cores" if args.cuda_cores else "tcgen05"},
+        "steps_per_s": steps_s,
+        "scored_tokens_per_s": tok_s,
+        "target_tokens_per_s": world * S / (ms / 1000.0),
+        "step_roofline": {"flops": flops_all, "bytes": bytes_ * world,
+                          "roofline_ms": roof_t * 1000.0, "frac": roof_t * 1000.0 / ms,
+                          "peak": f"{peak_kind} bf16 {peak_t} TFLOP/s sustained, "
+                                  f"HBM {peaks['hbm_gbs']} GB/s"},
+        "roofline": {"kernel": "gemm_tc_kernel (tcgen05 GEMM, all epilogues)", "bound": "tensor",
+                     "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": (gemm_tflops / peak_t) if gemm_tflops else None,
+                     "traffic": None, "launches_timed": d_n,
+                     "avg_launch_ms": d_ms / d_n if d_n else None,
+                     "peak_kind": f"{peak_kind} (sustained: the kernel runs inside a long step)",
+                     "share_of_step": (d_ms / args.steps) / ms if d_n else None},
+        "state_transition": {"bytes_per_step": (s1["state_transition_bytes"] -
+                                                s0["state_transition_bytes"]) / args.steps,
+                             "dense_ref_bytes_per_step": (s1["dense_ref_bytes"] -
+                                                          s0["dense_ref_bytes"]) / args.steps,
+                             "dense_ref_targets_per_step": (s1["dense_ref_bytes_targets"] -
+                                                            s0["dense_ref_bytes_targets"]) / args.steps},
+        "phases_ms_per_step": {k: (s1[k] - s0[k]) / args.steps for k in ("ms_plan", "ms_score",
+                                                                         "ms_step")},
+        "gpu_launches": int(s1["kernel_launches"] - s0["kernel_launches"]),
+        "e2e": e2e,
+        "clocks": clocks,
+    }
+    st = line["state_transition"]
+    st["frac_of_dense"] = st["bytes_per_step"] / st["dense_ref_bytes_per_step"]
+    st["frac_of_dense_targets"] = st["bytes_per_step"] / st["dense_ref_targets_per_step"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(w, n_prompts=args.ref_prompts)
+        line["cpu_baseline"] = {"value": cb["tokens_per_s"], "unit": "scored tokens/s",
+                                "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,76 @@
+/*
+ * zo_ops.h -- kernel-level entry points of the B200 ZO library.
+ *
+ * The single operations the probe step is built from, exposed so that each
+ * can be checked and timed on its own.  None of them allocates: every
+ * buffer, including scratch ("workspace"), is the caller's device memory.
+ * All are queued on `stream` (cudaStream_t, NULL = legacy default stream)
+ * and return ZO_OK or a ZO_ERR_* code from zo.h.
+ */
+#ifndef ZO_OPS_H
+#define ZO_OPS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { ZO_ACT_NONE = 0, ZO_ACT_RELU = 1 };
+enum { ZO_IMPL_AUTO = 0, ZO_IMPL_CUDA_CORES = 1, ZO_IMPL_TENSOR_CORES = 2 };
+
+/* One decoder linear layer, y = act(x W^T + b) (the frozen base weights W of
+ * "Inference-Native Zeroth-Order Optimization", abstract; the GEMM is the
+ * batched forward that dominates the step, "Zeroth-Order Fine-Tuning Was an
+ * Inference Workload All Along", section "Why ZO Fine-Tuning Is Really
+ * Scoring").
+ *   x    dev [M x K] dtype, row-major          W  dev [N x K] dtype, row-major
+ *   bias dev float [N] or NULL
+ *   y    accumulate == 0: dev [M x N] dtype; accumulate == 1: dev float [M x N],
+ *        y += x W^T + b (the residual-add form)
+ *   impl ZO_IMPL_TENSOR_CORES needs dtype bf16 and K % 8 == 0 (else
+ *        ZO_ERR_UNSUPPORTED); AUTO picks tensor cores whenever they apply. */
+int zo_op_linear(const void* x, const void* W, const float* bias, void* y, int32_t M,
+                 int32_t N, int32_t K, int32_t dtype, int32_t act, int32_t accumulate,
+                 int32_t impl, void* stream);
+
+/* Bytes of workspace zo_op_lm_head_logprob needs for n_rows rows and vocab. */
+size_t zo_op_lm_head_workspace(int32_t n_rows, int32_t vocab, int32_t impl);
+
+/* Token log-probabilities through the lm_head without writing vocab-sized
+ * logits to memory (the objective is the log-probability of the label
+ * tokens: "Zeroth-Order Fine-Tuning Was an Inference Workload All Along",
+ * sections "Why ZO Fine-Tuning Is Really Scoring" and "The System
+ * Reorganization"):  logprob[i] = (h_i E^T)[target_i] - logsumexp(h_i E^T).
+ *   h        dev [n_rows x d] dtype (final-norm hidden states)
+ *   E        dev [vocab x d] dtype
+ *   targets  dev int32 [n_rows], each in [0, vocab)
+ *   logprob  dev float [n_rows]
+ *   workspace dev, >= zo_op_lm_head_workspace(n_rows, vocab, impl) bytes,
+ *            256-byte aligned; contents are scratch. */
+int zo_op_lm_head_logprob(const void* h, const void* E, const int32_t* targets, int32_t n_rows,
+                          int32_t vocab, int32_t d, int32_t dtype, float* logprob,
+                          void* workspace, size_t workspace_bytes, int32_t impl, void* stream);
+
+/* Packed variable-length causal attention, no padding ("Inference-Native
+ * Zeroth-Order Optimization", abstract: padding elimination and
+ * variable-length packing).
+ *   qkv      dev [T x (H + 2*Hkv)*hd] dtype: q | k | v per token
+ *   out      dev [T x H*hd] dtype
+ *   seq_lens host int32 [n_rows], rows back to back in qkv
+ *   workspace dev >= 4*(n_rows + 1 + T/64 + n_rows + 1) bytes (row offsets and tiles) */
+int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t n_rows,
+                    int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t dtype,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise the device and return the tensor-core kernels' error word:
+ * 0 when clean, bit 0 set when a bounded wait inside a kernel expired (the
+ * kernel then stopped early and its output is invalid), -1 when the device
+ * reported an error. */
+int zo_op_error_word(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ZO_OPS_H */

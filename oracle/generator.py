@@ -35,12 +35,12 @@ M2 = 0x94D049BB133111EB
 
 # Weight tensors use a step' no direction ever has, so their keys never collide.
 WEIGHT_TAG = MASK64
-GLOBAL_LAYER = 0xFFFF
 
-# Tensor ids for weight initialisation (matrix ids 0..6 are shared with the directions).
-T_BIAS0 = 7          # + matrix id: bias of that matrix
-T_LN1_W, T_LN1_B, T_LN2_W, T_LN2_B, T_QNORM, T_KNORM = 14, 15, 16, 17, 18, 19
-T_TOK_EMBED, T_POS_EMBED, T_FINAL_W, T_FINAL_B, T_LM_HEAD = 32, 33, 34, 35, 36
+# Tensor ids of the initial weights are input keys, shared with the library's
+# tests through the workload module (they hold no arithmetic of the method).
+from zeroth_order_fine_b200.workload import (GLOBAL_LAYER, T_BIAS0, T_LN1_W, T_LN1_B,  # noqa: E402
+                                             T_LN2_W, T_LN2_B, T_QNORM, T_KNORM, T_TOK_EMBED,
+                                             T_POS_EMBED, T_FINAL_W, T_FINAL_B, T_LM_HEAD)
 
 F32 = np.float32
 _U64 = np.uint64

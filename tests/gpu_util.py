@@ -1,0 +1,42 @@
+"""Shared set-up of the GPU tests: the same workload on the CUDA path (through the
+C ABI) and in the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from zeroth_order_fine_b200 import workload as wl
+
+needs_gpu = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def gpu_handle(w: wl.Workload, shape=None, batch=None, max_slots=8, impl=0, nu=None,
+               layers=None, start_step=0, fg=0):
+    from zeroth_order_fine_b200 import zo
+    shape = shape or w.shape
+    model = zo.DeviceModel(shape, w.weight_seed)
+    tg = zo.make_targets(shape.n_layers, w.matrices, w.scale_mode, layers)
+    B = batch or w.batch
+    max_len = w.len_hi
+    h = zo.Handle(model, w.run_seed, nu or w.nu, w.rank, tg,
+                  max_tokens=(2 * B + fg) * max_len + 64, max_rows=2 * B + fg,
+                  max_scored=(2 * B + fg) * max(w.tgt_hi, w.fg_tgt_hi if fg else 1),
+                  max_slots=max_slots, start_step=start_step, impl=impl)
+    return model, h
+
+
+def oracle_run(w: wl.Workload, shape=None, nu=None, layers=None, start_step=0):
+    from oracle import model as om
+    from oracle import zo as ozo
+    shape = shape or w.shape
+    weights = om.init_weights(shape, w.weight_seed)
+    ls = range(shape.n_layers) if layers is None else layers
+    return ozo.OracleRun(weights, w.run_seed, nu or w.nu, w.rank, ls, w.matrices, w.scale_mode,
+                         start_step)
+
+
+def dev_tokens(batch: wl.Batch):
+    return torch.from_numpy(batch.packed()).cuda()
+
+
+def dev_fg_tokens(batch: wl.Batch):
+    return torch.from_numpy(batch.fg_packed()).cuda()

@@ -1,0 +1,64 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU and exports every
+symbol include/*.h declares (no compute calls here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[\w\s\*]+?\b(zo_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def built_lib():
+    from zeroth_order_fine_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_every_declared_symbol_is_exported(built_lib):
+    names = declared_functions()
+    assert len(names) >= 20
+    missing = [n for n in sorted(names) if not hasattr(built_lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_the_header():
+    from zeroth_order_fine_b200 import zo
+    assert declared_functions() <= set(zo.EXPORTED)
+
+
+def test_struct_sizes_match_header(built_lib):
+    """The ctypes mirrors have the C layouts (checked against offsets fixed by the header)."""
+    from zeroth_order_fine_b200 import zo
+    assert ctypes.sizeof(zo.zo_model_desc) == 13 * 4
+    assert ctypes.sizeof(zo.zo_targets) == 24
+    assert zo.zo_options.stream.offset == 64 and ctypes.sizeof(zo.zo_options) == 80
+    assert ctypes.sizeof(zo.zo_layer_weights) == 20 * 8
+
+
+def test_library_refuses_bad_create_without_gpu(built_lib):
+    """Argument checks run on the host before any CUDA call."""
+    from zeroth_order_fine_b200 import zo
+    L = zo.lib()
+    out = ctypes.c_void_p()
+    assert L.zo_create(None, None, None, ctypes.byref(out)) == zo.ZO_ERR_ARG
+    assert L.zo_last_error(None)
+
+
+def test_product_path_does_not_import_oracle():
+    for f in glob.glob(os.path.join(ROOT, "zeroth_order_fine_b200", "**", "*.*"), recursive=True):
+        if f.endswith((".py", ".cu", ".cpp", ".cuh", ".h")):
+            txt = open(f).read()
+            assert "import oracle" not in txt and "from oracle" not in txt, f

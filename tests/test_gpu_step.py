@@ -1,0 +1,253 @@
+"""End-to-end parity of the probe step through the C ABI against the oracle,
+and the invariants the pages fix: eps = 0 gives L+ == L-, co-batched
+foreground rows are bit-identical to the same rows scored alone, runs are
+deterministic, a saved state resumes the same trajectory, non-finite
+objectives are refused."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from zeroth_order_fine_b200 import workload as wl
+from gpu_util import dev_fg_tokens, dev_tokens, gpu_handle, needs_gpu, oracle_run
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+TINY = wl.WORKLOADS["tiny"]
+TINY_BF16 = dataclasses.replace(TINY, shape=wl.shrink_shape(wl.TINY, dtype=wl.DTYPE_BF16))
+# A small Qwen3-family model (GQA, q/k RMSNorm, RoPE, SwiGLU) with the MeZO-style
+# factorised direction on all seven matrices.
+Q3_SMALL = wl.ModelShape("qwen3-small", wl.ARCH_QWEN3, 2, 256, 4, 2, 64, 512, 1000, 4096, 1e-6,
+                         1e6, wl.DTYPE_FP32, False)
+QWEN_SMALL = wl.Workload("qwen3-small", Q3_SMALL, 6, 20, 90, 1, 4, True, 8, wl.ALL7,
+                         wl.SCALE_MEZO, 1e-3, 1e-4, 3, fg_rows=4, data_seed=11)
+
+
+def _cat(xs):
+    return np.concatenate([np.asarray(x) for x in xs])
+
+
+@pytest.mark.parametrize("impl", [0, 1])
+def test_tiny_fp32_steps_match_oracle(impl):
+    """Config 1: one probe pair + update, then 10 more steps; fp32 tolerances."""
+    w = TINY
+    batch = wl.make_batch(w)
+    model, h = gpu_handle(w, impl=impl)
+    orc = oracle_run(w)
+    toks = dev_tokens(batch)
+    for t in range(11):
+        h.zo_probe_plan(t, w.eps)
+        orc.plan(t, w.eps)
+        Lp, Lm, lp = h.zo_score(toks, batch.seq_lens, batch.target_lens,
+                                target_ids=torch.from_numpy(batch.target_ids()).cuda(),
+                                want_logprob=True)
+        ref = orc.score(batch.prompts, batch.target_lens)
+        ref_lp = _cat(ref.logprob_plus + ref.logprob_minus)
+        assert np.max(np.abs(lp.cpu().numpy() - ref_lp)) <= 1e-4
+        assert np.max(np.abs(Lp.cpu().numpy() - ref.L_plus)) <= 1e-4
+        assert np.max(np.abs(Lm.cpu().numpy() - ref.L_minus)) <= 1e-4
+        c = h.zo_step(w.lr)
+        c_ref = orc.step(w.lr)
+        assert abs(c - c_ref) <= 1e-2 * max(abs(c_ref), 1.0), (t, c, c_ref)
+    for (l, m) in orc.bank:
+        A = h.zo_read_bank(l, m, 0)
+        Ar = orc.bank[(l, m)][0][0].numpy()
+        assert np.max(np.abs(A - Ar)) <= 1e-2 * max(np.max(np.abs(Ar)), 1e-12) + 1e-9
+
+
+def test_qwen3_mezo_fp32_matches_oracle():
+    w = QWEN_SMALL
+    batch = wl.make_batch(w)
+    model, h = gpu_handle(w, fg=w.fg_rows, max_slots=4)
+    orc = oracle_run(w)
+    toks, ftoks = dev_tokens(batch), dev_fg_tokens(batch)
+    for t in range(4):                        # crosses a window boundary (nu = 3)
+        h.zo_probe_plan(t, w.eps)
+        orc.plan(t, w.eps)
+        Lp, Lm, lp, flp = h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, ftoks,
+                                             batch.fg_seq_lens, batch.fg_target_lens,
+                                             want_logprob=True)
+        ref = orc.score(batch.prompts, batch.target_lens, batch.fg_prompts, batch.fg_target_lens)
+        assert np.max(np.abs(lp.cpu().numpy() - _cat(ref.logprob_plus + ref.logprob_minus))) <= 1e-4
+        assert np.max(np.abs(flp.cpu().numpy() - _cat(ref.fg_logprob))) <= 1e-4
+        c = h.zo_step(w.lr)
+        c_ref = orc.step(w.lr)
+        assert abs(c - c_ref) <= 1e-2 * max(abs(c_ref), 1.0)
+
+
+def test_tiny_bf16_objectives_and_trajectory():
+    """bf16 mode: L+- within 2e-2 and a 100-step loss trajectory within 2 %."""
+    w = TINY_BF16
+    batch = wl.make_batch(w)
+    model, h = gpu_handle(w)
+    orc = oracle_run(w)
+    toks = dev_tokens(batch)
+    traj, traj_ref = [], []
+    for t in range(100):
+        h.zo_probe_plan(t, w.eps)
+        orc.plan(t, w.eps)
+        Lp, Lm, _ = h.zo_score(toks, batch.seq_lens, batch.target_lens)
+        ref = orc.score(batch.prompts, batch.target_lens)
+        if t in (0, 50, 99):
+            assert np.max(np.abs(Lp.cpu().numpy() - ref.L_plus)) <= 2e-2
+            assert np.max(np.abs(Lm.cpu().numpy() - ref.L_minus)) <= 2e-2
+        traj.append(float((Lp.mean() + Lm.mean()).item()) / 2)
+        traj_ref.append(float(ref.L_plus.mean() + ref.L_minus.mean()) / 2)
+        h.zo_step(w.lr * 100, want_c=False)
+        orc.step(w.lr * 100)
+    traj, traj_ref = np.array(traj), np.array(traj_ref)
+    assert np.max(np.abs(traj - traj_ref) / np.abs(traj_ref)) <= 0.02
+
+
+def test_opt13_width_slice_bf16_matches_oracle():
+    """Two full-width OPT-1.3B layers (d=2048, vocab 50272) on the tensor-core path."""
+    w = wl.WORKLOADS["opt-1.3b-b16"]
+    shape = wl.shrink_shape(w.shape, n_layers=2)
+    batch = wl.make_batch(w, batch=4, len_hi=64)
+    model, h = gpu_handle(w, shape=shape, batch=4)
+    orc = oracle_run(w, shape=shape)
+    toks = dev_tokens(batch)
+    for t in range(3):
+        h.zo_probe_plan(t, w.eps)
+        orc.plan(t, w.eps)
+        Lp, Lm, _ = h.zo_score(toks, batch.seq_lens, batch.target_lens)
+        ref = orc.score(batch.prompts, batch.target_lens)
+        assert np.max(np.abs(Lp.cpu().numpy() - ref.L_plus)) <= 2e-2
+        assert np.max(np.abs(Lm.cpu().numpy() - ref.L_minus)) <= 2e-2
+        h.zo_step(w.lr)
+        orc.step(w.lr)
+
+
+@pytest.mark.parametrize("wk", ["tiny", "tiny-bf16"])
+def test_eps_zero_gives_bitwise_equal_objectives(wk):
+    w = TINY if wk == "tiny" else TINY_BF16
+    batch = wl.make_batch(w)
+    model, h = gpu_handle(w)
+    toks = dev_tokens(batch)
+    h.zo_probe_plan(0, 0.0)
+    Lp, Lm, lp = h.zo_score(toks, batch.seq_lens, batch.target_lens, want_logprob=True)
+    assert torch.equal(Lp, Lm)
+    n = lp.numel() // 2
+    assert torch.equal(lp[:n], lp[n:])
+
+
+def _cobatch_vs_alone(w, shape=None, steps=2):
+    batch = wl.make_batch(w, fg_rows=5)
+    model, h = gpu_handle(w, shape=shape, fg=5)
+    toks, ftoks = dev_tokens(batch), dev_fg_tokens(batch)
+    for t in range(steps):
+        h.zo_probe_plan(t, w.eps)
+        _, _, _, flp = h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, ftoks,
+                                          batch.fg_seq_lens, batch.fg_target_lens)
+        alone = h.zo_score_foreground(ftoks, batch.fg_seq_lens, batch.fg_target_lens)
+        assert torch.equal(flp, alone), t
+        # the probe rows' results are not disturbed by the foreground rows either
+        h.zo_score(toks, batch.seq_lens, batch.target_lens)
+        h.zo_step(w.lr)
+
+
+def test_cobatched_foreground_bit_identical_fp32():
+    _cobatch_vs_alone(dataclasses.replace(TINY, fg_rows=5))
+
+
+def test_cobatched_foreground_bit_identical_bf16():
+    _cobatch_vs_alone(dataclasses.replace(TINY_BF16, fg_rows=5))
+
+
+def test_cobatched_foreground_bit_identical_qwen3_bf16():
+    shape = dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16)
+    _cobatch_vs_alone(dataclasses.replace(QWEN_SMALL, shape=shape), steps=4)
+
+
+def test_deterministic_and_resumable():
+    w = TINY_BF16
+    batch = wl.make_batch(w)
+    toks = dev_tokens(batch)
+
+    def run(h, t0, t1):
+        out = []
+        for t in range(t0, t1):
+            h.zo_probe_plan(t, w.eps)
+            Lp, Lm, _ = h.zo_score(toks, batch.seq_lens, batch.target_lens)
+            out.append((Lp.cpu().numpy().copy(), Lm.cpu().numpy().copy(), h.zo_step(w.lr)))
+        return out
+
+    _, h1 = gpu_handle(w, nu=3)
+    a = run(h1, 0, 8)
+    _, h2 = gpu_handle(w, nu=3)
+    b = run(h2, 0, 4)
+    state = h2.zo_save_state()
+    h2.close()
+    _, h3 = gpu_handle(w, nu=3)
+    h3.zo_load_state(state)
+    b += run(h3, 4, 8)
+    for (x1, y1, c1), (x2, y2, c2) in zip(a, b):
+        assert np.array_equal(x1, x2) and np.array_equal(y1, y2) and c1 == c2
+
+
+def test_nonfinite_objective_refused_bank_unchanged():
+    from zeroth_order_fine_b200 import zo
+    w = TINY
+    batch = wl.make_batch(w)
+    model, h = gpu_handle(w)
+    toks = dev_tokens(batch)
+    h.zo_probe_plan(0, w.eps)
+    h.zo_score(toks, batch.seq_lens, batch.target_lens)
+    h.zo_step(w.lr)
+    A0 = h.zo_read_bank(0, wl.MAT_Q, 0)
+    h.zo_probe_plan(1, 0.0)                       # c = 0 / (2 * 0): not finite
+    h.zo_score(toks, batch.seq_lens, batch.target_lens)
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_step(w.lr)
+    assert e.value.code == zo.ZO_ERR_NONFINITE
+    assert np.array_equal(h.zo_read_bank(0, wl.MAT_Q, 0), A0)
+    h.zo_probe_plan(1, w.eps)                     # the step counter did not advance
+    h.zo_score(toks, batch.seq_lens, batch.target_lens)
+    h.zo_step(w.lr)
+
+
+def test_call_order_and_argument_errors():
+    from zeroth_order_fine_b200 import zo
+    w = TINY
+    batch = wl.make_batch(w)
+    model, h = gpu_handle(w)
+    toks = dev_tokens(batch)
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_probe_plan(3, w.eps)
+    assert e.value.code == zo.ZO_ERR_STATE
+    h.zo_probe_plan(0, w.eps)
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_step(w.lr)
+    assert e.value.code == zo.ZO_ERR_STATE
+    bad = batch.target_lens.copy()
+    bad[0] = batch.seq_lens[0]                    # no prefix left
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_score(toks, batch.seq_lens, bad)
+    assert e.value.code == zo.ZO_ERR_ARG
+    wrong = torch.from_numpy(batch.target_ids()).cuda()
+    wrong[0] += 1
+    h.zo_score(toks, batch.seq_lens, batch.target_lens, target_ids=wrong)
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_step(w.lr)
+    assert e.value.code == zo.ZO_ERR_ARG
+
+
+def test_state_transition_bytes_counted():
+    w = TINY
+    batch = wl.make_batch(w)
+    model, h = gpu_handle(w, nu=4)
+    toks = dev_tokens(batch)
+    for t in range(6):
+        h.zo_probe_plan(t, w.eps)
+        h.zo_score(toks, batch.seq_lens, batch.target_lens)
+        h.zo_step(w.lr)
+    s = h.zo_stats()
+    sh = w.shape
+    u = sum(sh.matrix_dims(m)[0] * w.rank for m in w.matrices) * sh.n_layers
+    v = sum(sh.matrix_dims(m)[1] * w.rank for m in w.matrices) * sh.n_layers
+    per_step = 4 * u + (8 * u + 4 * u)
+    per_window = 4 * v + 2 * 4 * v + 4 * u
+    assert s["state_transition_bytes"] == 6 * per_step + 2 * per_window
+    assert s["dense_ref_bytes"] == 6 * 2 * 4 * sh.body_params()
+    assert s["steps"] == 6 and s["bank_slots"] == 2

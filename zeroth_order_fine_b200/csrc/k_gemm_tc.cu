@@ -1,0 +1,554 @@
+// Tensor-core GEMM for sm_100a: C = A B^T (+ A2 B2^T), bf16 in, fp32 accumulate.
+//
+// The batched forward of both candidates is the dominant cost of the probe
+// step ("Zeroth-Order Fine-Tuning Was an Inference Workload All Along",
+// section "Why ZO Fine-Tuning Is Really Scoring": the pair of forward
+// objective evaluations is the expensive operation), so every decoder linear
+// layer -- with the candidate perturbation and the banked updates appended as
+// extra K blocks (A2 = the shrink output S, B2 = the expand factors) -- runs
+// here, and the lm_head runs here with a log-sum-exp epilogue so logits never
+// reach memory.
+//
+// Design (one CTA per SM, persistent):
+//   warp 0      TMA producer: 128x64 A and BNx64 B boxes, 128-byte swizzle,
+//               into a STAGES-deep shared-memory ring (mbarrier complete_tx)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//               (M=128, N=BN, K=16 per instruction, kind::f16, fp32 accumulate)
+//   warps 2..5  epilogue: tcgen05.ld 32x32b from a double-buffered TMEM
+//               accumulator, fused bias / ReLU / residual add / LSE, stores
+// Tiles are walked in M-groups of 8 so concurrent CTAs share B strips in L2.
+// Every mbarrier wait is bounded: on expiry the kernel records
+// ZO_TC_TIMEOUT in the error word, drains what it issued and returns.
+#include <cuda.h>
+#include <float.h>
+
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace zo {
+
+namespace {
+
+constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_BYTES = BN * BK * 2;        // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 512;              // two BN-wide fp32 accumulators
+constexpr int GROUP_M = 8;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t WAIT_LIMIT = 1u << 24;   // ~2 s of polling with back-off
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+
+__device__ int g_tc_error = 0;              // bit 0: a bounded wait expired
+
+struct TcParams {
+    int M, N, kb_main, kb_ext;
+    int n_m_blk, n_n_blk, n_tiles;
+    int epi;
+    const float* bias;
+    void* C; int ldc; int c_type;
+    const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
+    int* err;
+};
+
+// ---- PTX wrappers ------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait; false when the limit expired or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_f,
+                                          int* err) {
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_f) return false;
+        if (i >= WAIT_LIMIT) {
+            *abort_f = 1;
+            atomicOr(err, 1);
+            return false;
+        }
+        if (i > 32) __nanosleep(128);
+    }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+// 32 lanes x 32 consecutive fp32 columns per warp.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes in 8-row groups 1024 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
+    d |= (uint64_t)1u << 16;                           // leading byte offset (unused, 16 B)
+    d |= (uint64_t)(1024u >> 4) << 32;                 // stride byte offset
+    d |= (uint64_t)1u << 46;                           // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                           // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = BN.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void tile_coords(int t, const TcParams& p, int* mb, int* nb) {
+    const int per_group = GROUP_M * p.n_n_blk;
+    const int g = t / per_group;
+    const int first_m = g * GROUP_M;
+    const int gm = min(p.n_m_blk - first_m, GROUP_M);
+    const int in = t - g * per_group;
+    *mb = first_m + in % gm;
+    *nb = in / gm;
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, float* v,
+                                               float* run_max, float* run_sum) {
+    const bool row_ok = m < p.M;
+    if (EPI == EPI_LSE) {
+        float mx = -FLT_MAX;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (n + j < p.N) mx = fmaxf(mx, v[j]);
+        const float nm = fmaxf(*run_max, mx);
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (n + j < p.N) s += expf(v[j] - nm);
+        *run_sum = *run_sum * expf(*run_max - nm) + s;
+        *run_max = nm;
+        if (row_ok) {
+            const int tg = p.targets[m] - n;
+            if (tg >= 0 && tg < 32) {
+                float tv = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (j == tg) tv = v[j];
+                p.tgt_logit[m] = tv;
+            }
+        }
+        return;
+    }
+    if (!row_ok) return;
+    if (p.bias) {
+        if (n + 32 <= p.N) {
+            const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 b = __ldg(b4 + q);
+                v[4 * q] += b.x; v[4 * q + 1] += b.y; v[4 * q + 2] += b.z; v[4 * q + 3] += b.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (n + j < p.N) v[j] += p.bias[n + j];
+        }
+    }
+    if (EPI == EPI_RESID) {
+        float* C = static_cast<float*>(p.C) + (size_t)m * p.ldc + n;
+        if (n + 32 <= p.N) {
+            float4* c4 = reinterpret_cast<float4*>(C);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float4 c = c4[q];
+                c.x += v[4 * q]; c.y += v[4 * q + 1]; c.z += v[4 * q + 2]; c.w += v[4 * q + 3];
+                c4[q] = c;
+            }
+        } else {
+            for (int j = 0; j < 32 && n + j < p.N; ++j) C[j] += v[j];
+        }
+        return;
+    }
+    if (EPI == EPI_STORE_RELU) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
+    }
+    if (p.c_type == E_BF16) {
+        __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + (size_t)m * p.ldc + n;
+        if (n + 32 <= p.N) {
+            uint4* c4 = reinterpret_cast<uint4*>(C);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint4 w;
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * q], v[8 * q + 1]);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * q + 2], v[8 * q + 3]);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 4], v[8 * q + 5]);
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * q + 6], v[8 * q + 7]);
+                w.x = *reinterpret_cast<uint32_t*>(&h0);
+                w.y = *reinterpret_cast<uint32_t*>(&h1);
+                w.z = *reinterpret_cast<uint32_t*>(&h2);
+                w.w = *reinterpret_cast<uint32_t*>(&h3);
+                c4[q] = w;
+            }
+        } else {
+            for (int j = 0; j < 32 && n + j < p.N; ++j) C[j] = __float2bfloat16_rn(v[j]);
+        }
+    } else {
+        float* C = static_cast<float*>(p.C) + (size_t)m * p.ldc + n;
+        for (int j = 0; j < 32 && n + j < p.N; ++j) C[j] = v[j];
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                   const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;           // 1024-aligned for SW128
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+    // barriers: full[S] empty[S] tfull[2] tempty[2] drain
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+    auto tempty = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t drain = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 128);
+    volatile int* abort_f = reinterpret_cast<volatile int*>(gbase + STAGES * STAGE_BYTES + 136);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), 4);
+        }
+        mbar_init(drain, 1);
+        *abort_f = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int kb_total = p.kb_main + p.kb_ext;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int armed_s[STAGES];
+            uint32_t armed_ph[STAGES];
+            int n_armed = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+                int mb, nb;
+                tile_coords(t, p, &mb, &nb);
+                for (int kb = 0; kb < kb_total; ++kb) {
+                    if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                    const uint32_t sa = base + s * STAGE_BYTES;
+                    const uint32_t sb = sa + A_BYTES;
+                    mbar_expect_tx(full(s), STAGE_BYTES);
+                    if (kb < p.kb_main) {
+                        tma_load_2d(sa, &tmA, full(s), kb * BK, mb * BM);
+                        tma_load_2d(sb, &tmB, full(s), kb * BK, nb * BN);
+                    } else {
+                        const int k = (kb - p.kb_main) * BK;
+                        tma_load_2d(sa, &tmA2, full(s), k, mb * BM);
+                        tma_load_2d(sb, &tmB2, full(s), k, nb * BN);
+                    }
+                    armed_s[n_armed % STAGES] = s;
+                    armed_ph[n_armed % STAGES] = ph;
+                    ++n_armed;
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (!ok) {
+                // drain: let every copy this thread issued land before the CTA exits
+                const int n = n_armed < STAGES ? n_armed : STAGES;
+                for (int i = 0; i < n; ++i) {
+                    const int j = (n_armed - 1 - i) % STAGES;
+                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(armed_s[j]), armed_ph[j]); ++it)
+                        __nanosleep(128);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t aph = 0;
+            bool ok = true, issued = false;
+            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+                if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < kb_total; ++kb) {
+                    if (!mbar_wait(full(s), ph, abort_f, p.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = base + s * STAGE_BYTES;
+                    const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), kIdesc,
+                               (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit(empty(s));            // stage free once these MMAs retire
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(tfull(acc));              // accumulator ready for the epilogue
+                if (++acc == 2) { acc = 0; aph ^= 1u; }
+            }
+            if (!ok && issued) {
+                tc_commit(drain);
+                for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(drain, 0); ++it) __nanosleep(128);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int lane_base = 32 * (warp & 3);
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+            int mb, nb;
+            tile_coords(t, p, &mb, &nb);
+            if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
+            tc_fence_after();
+            const int m = mb * BM + lane_base + lane;
+            float run_max = -FLT_MAX, run_sum = 0.f;
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n = nb * BN + c * 32;
+                if (n >= p.N) break;                // whole chunk past N (warp-uniform)
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN + c * 32), v);
+                epilogue_chunk<EPI>(p, m, n, v, &run_max, &run_sum);
+            }
+            if (EPI == EPI_LSE && m < p.M) {
+                p.part_max[(size_t)m * p.n_col_tiles + nb] = run_max;
+                p.part_sum[(size_t)m * p.n_col_tiles + nb] = run_sum;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty(acc));
+            if (++acc == 2) { acc = 0; aph ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---- host side ---------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 map over a row-major [rows x cols] matrix with leading dimension ld,
+// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld,
+              uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {BK, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int EPI>
+int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+               const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES) != cudaSuccess)
+            return 1;
+        attr = true;
+    }
+    const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+    gemm_tc_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(a, b, a2, b2, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const GemmArgs& g) {
+    if (g.a_type != E_BF16 || g.b_type != E_BF16) return false;
+    if (g.K % 8 || g.lda % 8 || g.ldb % 8 || g.K <= 0 || g.M <= 0 || g.N <= 0) return false;
+    if (!aligned16(g.A) || !aligned16(g.B)) return false;
+    if (g.K2 > 0) {
+        if (g.a2_type != E_BF16 || g.b2_type != E_BF16 || g.lda2 % 8 || g.ldb2 % 8 || g.K2 % 8)
+            return false;
+        if (!aligned16(g.A2) || !aligned16(g.B2)) return false;
+    }
+    switch (g.epi) {
+        case EPI_STORE:
+        case EPI_STORE_RELU:
+            if (g.c_type != E_BF16 || g.ldc % 8 || !aligned16(g.C)) return false;
+            if (g.bias && !aligned16(g.bias)) return false;
+            return true;
+        case EPI_RESID:
+            if (g.c_type != E_F32 || g.ldc % 4 || !aligned16(g.C)) return false;
+            if (g.bias && !aligned16(g.bias)) return false;
+            return true;
+        case EPI_LSE:
+            return true;
+        default:
+            return false;
+    }
+}
+
+int gemm_tc_col_tiles(int N) { return (N + BN - 1) / BN; }
+
+int gemm_tc(const GemmArgs& g, cudaStream_t st) {
+    CUtensorMap a, b, a2, b2;
+    if (!make_map(&a, g.A, g.M, g.K, g.lda, BM)) return 1;
+    if (!make_map(&b, g.B, g.N, g.K, g.ldb, BN)) return 1;
+    if (g.K2 > 0) {
+        if (!make_map(&a2, g.A2, g.M, g.K2, g.lda2, BM)) return 1;
+        if (!make_map(&b2, g.B2, g.N, g.K2, g.ldb2, BN)) return 1;
+    } else {
+        a2 = a;
+        b2 = b;
+    }
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = g.M; p.N = g.N;
+    p.kb_main = (g.K + BK - 1) / BK;
+    p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
+    p.n_m_blk = (g.M + BM - 1) / BM;
+    p.n_n_blk = (g.N + BN - 1) / BN;
+    p.n_tiles = p.n_m_blk * p.n_n_blk;
+    p.epi = g.epi;
+    p.bias = g.bias;
+    p.C = g.C; p.ldc = g.ldc; p.c_type = g.c_type;
+    p.targets = g.targets; p.part_max = g.part_max; p.part_sum = g.part_sum;
+    p.tgt_logit = g.tgt_logit; p.n_col_tiles = g.n_col_tiles;
+    int* err = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
+    p.err = err;
+    switch (g.epi) {
+        case EPI_STORE: return launch_epi<EPI_STORE>(a, b, a2, b2, p, st);
+        case EPI_STORE_RELU: return launch_epi<EPI_STORE_RELU>(a, b, a2, b2, p, st);
+        case EPI_RESID: return launch_epi<EPI_RESID>(a, b, a2, b2, p, st);
+        case EPI_LSE: return launch_epi<EPI_LSE>(a, b, a2, b2, p, st);
+        default: return 1;
+    }
+}
+
+int gemm_tc_error_word() {
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_error, sizeof(int)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(int));
+    return v;
+}
+
+}  // namespace zo

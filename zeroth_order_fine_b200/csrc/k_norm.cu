@@ -1,0 +1,137 @@
+// Token metadata, embeddings, LayerNorm / RMSNorm (optionally gathering the
+// scored rows first) and the SwiGLU activation.  All HBM-bound, one CTA per
+// token row; the row is staged in shared memory so it is read once.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace zo {
+
+// One CTA per physical row: token ids / positions / signs of the packed batch
+// and, per scored position, the index of the hidden state that predicts it
+// (the position before the target token) and the target id.
+__global__ void build_tokens_kernel(RowMeta m, const int* __restrict__ probe_src,
+                                    const int* __restrict__ fg_src, int* tok_id, int* tok_pos,
+                                    int* tok_sign, int* tok_row, int* sc_tok, int* sc_tgt,
+                                    const int* tgt_check_probe, const int* tgt_check_fg,
+                                    const int* tgt_check_off, int* err_word) {
+    const int r = blockIdx.x;
+    const int start = m.cu_seqlens[r];
+    const int len = m.cu_seqlens[r + 1] - start;
+    const int* src = (m.row_is_fg[r] ? fg_src : probe_src) + m.row_src[r];
+    const int sign = m.row_sign[r];
+    for (int p = threadIdx.x; p < len; p += blockDim.x) {
+        const int t = start + p;
+        tok_id[t] = src[p];
+        tok_pos[t] = p;
+        tok_sign[t] = sign;
+        tok_row[t] = r;
+    }
+    const int s0 = m.score_off[r];
+    const int tl = m.score_off[r + 1] - s0;
+    const int* chk = m.row_is_fg[r] ? tgt_check_fg : tgt_check_probe;
+    for (int j = threadIdx.x; j < tl; j += blockDim.x) {
+        const int tgt = src[len - tl + j];
+        sc_tok[s0 + j] = start + len - tl + j - 1;
+        sc_tgt[s0 + j] = tgt;
+        if (chk != nullptr && tgt_check_off[r] >= 0 && chk[tgt_check_off[r] + j] != tgt)
+            atomicOr(err_word, 1);
+    }
+}
+
+void launch_build_tokens(RowMeta m, int R, const int* probe_src, const int* fg_src,
+                         int* tok_id, int* tok_pos, int* tok_sign, int* tok_row, int* sc_tok,
+                         int* sc_tgt, const int* tgt_check_probe, const int* tgt_check_fg,
+                         const int* tgt_check_off, int* err_word, cudaStream_t st) {
+    if (R == 0) return;
+    build_tokens_kernel<<<R, 128, 0, st>>>(m, probe_src, fg_src, tok_id, tok_pos, tok_sign,
+                                           tok_row, sc_tok, sc_tgt, tgt_check_probe,
+                                           tgt_check_fg, tgt_check_off, err_word);
+}
+
+// resid[t] = tok_embed[id] (+ pos_embed[pos]) in fp32.
+__global__ void embed_kernel(const int* __restrict__ tok_id, const int* __restrict__ tok_pos,
+                             const void* __restrict__ tok_embed,
+                             const void* __restrict__ pos_embed, int dtype,
+                             float* __restrict__ resid, int d) {
+    const int t = blockIdx.x;
+    const size_t te = (size_t)tok_id[t] * d;
+    const size_t pe = (size_t)tok_pos[t] * d;
+    float* out = resid + (size_t)t * d;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        float v = ld_elem(tok_embed, te + i, dtype);
+        if (pos_embed) v += ld_elem(pos_embed, pe + i, dtype);
+        out[i] = v;
+    }
+}
+
+void launch_embed(const int* tok_id, const int* tok_pos, const void* tok_embed,
+                  const void* pos_embed, int dtype, float* resid, int T, int d, cudaStream_t st) {
+    if (T == 0) return;
+    embed_kernel<<<T, 256, 0, st>>>(tok_id, tok_pos, tok_embed, pos_embed, dtype, resid, d);
+}
+
+// LayerNorm: (x - mean) / sqrt(var + eps) * w + b; RMSNorm: x / sqrt(mean(x^2) + eps) * w.
+// Statistics in fp32 with a two-pass variance over the staged row.
+__global__ void __launch_bounds__(256) norm_kernel(const float* __restrict__ x,
+                                                   const int* __restrict__ rows, int d, int kind,
+                                                   const float* __restrict__ w,
+                                                   const float* __restrict__ b, float eps,
+                                                   void* __restrict__ out, int out_type) {
+    extern __shared__ float srow[];
+    __shared__ float red[32];
+    const int t = blockIdx.x;
+    const int src = rows ? rows[t] : t;
+    const float* xr = x + (size_t)src * d;
+    float s = 0.f;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        const float v = xr[i];
+        srow[i] = v;
+        s += (kind == 0) ? v : v * v;
+    }
+    s = block_sum(s, red);
+    float mean = 0.f, rstd;
+    if (kind == 0) {
+        mean = s / (float)d;
+        float q = 0.f;
+        for (int i = threadIdx.x; i < d; i += blockDim.x) {
+            const float c = srow[i] - mean;
+            q += c * c;
+        }
+        q = block_sum(q, red);
+        rstd = 1.0f / sqrtf(q / (float)d + eps);
+    } else {
+        rstd = 1.0f / sqrtf(s / (float)d + eps);
+    }
+    const size_t o = (size_t)t * d;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        float y = (srow[i] - mean) * rstd * w[i];
+        if (kind == 0) y += b[i];
+        st_elem(out, o + i, out_type, y);
+    }
+}
+
+void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
+                 const float* b, float eps, void* out, int out_type, cudaStream_t st) {
+    if (T == 0) return;
+    norm_kernel<<<T, 256, d * sizeof(float), st>>>(x, rows, d, kind, w, b, eps, out, out_type);
+}
+
+// out[t, j] = silu(gu[t, j]) * gu[t, f + j]; gu = [gate | up] per row.
+__global__ void swiglu_kernel(const void* __restrict__ gu, int f, void* __restrict__ out,
+                              int dtype) {
+    const int t = blockIdx.x;
+    const size_t gi = (size_t)t * 2 * f, oi = (size_t)t * f;
+    for (int j = threadIdx.x; j < f; j += blockDim.x) {
+        const float g = ld_elem(gu, gi + j, dtype);
+        const float u = ld_elem(gu, gi + f + j, dtype);
+        const float si = g / (1.0f + expf(-g));
+        st_elem(out, oi + j, dtype, si * u);
+    }
+}
+
+void launch_swiglu(const void* gu, int T, int f, void* out, int dtype, cudaStream_t st) {
+    if (T == 0) return;
+    swiglu_kernel<<<T, 256, 0, st>>>(gu, f, out, dtype);
+}
+
+}  // namespace zo

@@ -1,0 +1,130 @@
+// Objective, estimator and factored bank update.
+//
+//  * log-sum-exp merge of the lm_head tiles' partials, in fixed tile order;
+//  * per-row objective L = -mean(log p) over the row's target span (fp64);
+//  * c = mean_i (L+_i - L-_i) / (2 eps), no 1/r ("Zeroth-Order Fine-Tuning
+//    Was an Inference Workload All Along", sections "Why ZO Fine-Tuning Is
+//    Really Scoring" and "The System Reorganization"), reduced in a fixed
+//    order in fp64 with warp shuffles;
+//  * A_k <- A_k - lr c U_t for every target in one launch (the U-side
+//    accumulator of the lazy window, same page, "Memory-write reduction"),
+//    refused on the device when c is not finite.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace zo {
+
+// One warp per scored position; lanes take tiles lane, lane+32, ... and the
+// lane results are combined by a fixed xor tree.
+__global__ void lse_merge_kernel(const float* __restrict__ pmax, const float* __restrict__ psum,
+                                 const float* __restrict__ tgt, int S, int n_tiles,
+                                 float* __restrict__ logprob) {
+    const int s = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (s >= S) return;
+    const float* pm = pmax + (size_t)s * n_tiles;
+    const float* ps = psum + (size_t)s * n_tiles;
+    float m = -FLT_MAX;
+    for (int i = lane; i < n_tiles; i += 32) m = fmaxf(m, pm[i]);
+    m = warp_max(m);
+    float z = 0.f;
+    for (int i = lane; i < n_tiles; i += 32) z += ps[i] * expf(pm[i] - m);
+    z = warp_sum(z);
+    if (lane == 0) logprob[s] = tgt[s] - (m + logf(z));
+}
+
+void launch_lse_merge(const float* part_max, const float* part_sum, const float* tgt_logit,
+                      int S, int n_tiles, float* logprob, cudaStream_t st) {
+    if (S == 0) return;
+    lse_merge_kernel<<<cdiv(S, 8), 256, 0, st>>>(part_max, part_sum, tgt_logit, S, n_tiles,
+                                                 logprob);
+}
+
+__global__ void row_objective_kernel(const float* __restrict__ logprob,
+                                     const int* __restrict__ score_off, int R, int B,
+                                     double* __restrict__ L_row, float* L_plus, float* L_minus) {
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= R) return;
+    const int a = score_off[r], b = score_off[r + 1];
+    double s = 0.0;
+    for (int i = a; i < b; ++i) s += (double)logprob[i];
+    const double L = -s / (double)(b - a);
+    L_row[r] = L;
+    if (r < B && L_plus) L_plus[r] = (float)L;
+    else if (r >= B && r < 2 * B && L_minus) L_minus[r - B] = (float)L;
+}
+
+void launch_row_objective(const float* logprob, const int* score_off, int R, int B,
+                          double* L_row, float* L_plus, float* L_minus, cudaStream_t st) {
+    if (R == 0) return;
+    row_objective_kernel<<<cdiv(R, 128), 128, 0, st>>>(logprob, score_off, R, B, L_row, L_plus,
+                                                       L_minus);
+}
+
+// sums[0] = sum_i (L+_i - L-_i), sums[1] = B; one CTA, fixed order.
+__global__ void objective_sums_kernel(const double* __restrict__ L_row, int B, double* sums) {
+    __shared__ double red[32];
+    double s = 0.0;
+    for (int i = threadIdx.x; i < B; i += blockDim.x) s += L_row[i] - L_row[B + i];
+    s = warp_sum_d(s);
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    if (lane == 0) red[w] = s;
+    __syncthreads();
+    if (w == 0) {
+        double v = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0;
+        v = warp_sum_d(v);
+        if (lane == 0) {
+            sums[0] = v;
+            sums[1] = (double)B;
+        }
+    }
+}
+
+void launch_objective_sums(const double* L_row, int B, double* sums, cudaStream_t st) {
+    objective_sums_kernel<<<1, 256, 0, st>>>(L_row, B, sums);
+}
+
+__global__ void estimate_kernel(const double* sums, float eps, double* c, int* flag) {
+    const double v = sums[0] / sums[1] / (2.0 * (double)eps);
+    *c = v;
+    *flag = isfinite(v) ? 0 : 1;
+}
+
+void launch_estimate(const double* sums, float eps, double* c, int* flag, cudaStream_t st) {
+    estimate_kernel<<<1, 1, 0, st>>>(sums, eps, c, flag);
+}
+
+// One launch over every target: blockIdx.y = target, float4 where aligned.
+__global__ void __launch_bounds__(256) bank_update_kernel(const UpdateJob* __restrict__ jobs,
+                                                          const double* __restrict__ c,
+                                                          const int* __restrict__ flag,
+                                                          float lr) {
+    if (*flag) return;                       // non-finite c: bank unchanged
+    const UpdateJob jb = jobs[blockIdx.y];
+    const float coef = (float)((double)lr * *c);
+    const int n4 = jb.n >> 2;
+    float4* A4 = reinterpret_cast<float4*>(jb.A);
+    const float4* U4 = reinterpret_cast<const float4*>(jb.U);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) {
+        float4 a = A4[i];
+        const float4 u = U4[i];
+        a.x -= coef * u.x; a.y -= coef * u.y; a.z -= coef * u.z; a.w -= coef * u.w;
+        A4[i] = a;
+    }
+    for (int i = (n4 << 2) + blockIdx.x * blockDim.x + threadIdx.x; i < jb.n;
+         i += gridDim.x * blockDim.x)
+        jb.A[i] -= coef * jb.U[i];
+}
+
+void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_n, const double* c,
+                        const int* flag, float lr, cudaStream_t st) {
+    if (n_jobs == 0) return;
+    unsigned bx = cdiv(max_n / 4 + 1, 256);
+    if (bx > 32) bx = 32;
+    dim3 grid(bx, n_jobs);
+    bank_update_kernel<<<grid, 256, 0, st>>>(jobs, c, flag, lr);
+}
+
+}  // namespace zo

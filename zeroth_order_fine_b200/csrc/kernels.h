@@ -1,0 +1,115 @@
+// Internal launch interface between the engine (engine.cpp) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace zo {
+
+enum ElemType : int { E_F32 = 0, E_BF16 = 1 };
+
+// ---- generator -------------------------------------------------------------------------
+struct GenJob {
+    float* dst;
+    int layer, matrix, which;   // which: 0 = U, 1 = V
+    int dim, r;                 // factor is [dim x r]
+    int transposed, ld;         // transposed: write element (i, c) at dst[c*ld + i]
+};
+
+struct WindowJob {
+    const float* V;             // [d_out x r] row-major
+    void* EB;                   // extension operand [N x ldb] (model dtype)
+    float* A;                   // new slot's A_k^T rows, r*d_in floats to zero
+    int eb_type, ldb, row0, d_out, d_in, r, col_dir, col_slot;
+};
+
+void launch_init_tensor(void* dst, uint64_t n, uint64_t key, float std_, float mean, int dtype,
+                        cudaStream_t st);
+void launch_gen_factors(const GenJob* d_jobs, int n_jobs, int max_pairs, uint64_t run_seed,
+                        uint64_t step, uint64_t nu, float scale, int apply_scale,
+                        cudaStream_t st);
+void launch_open_window(const WindowJob* d_jobs, int n_jobs, cudaStream_t st);
+
+// ---- token metadata / embeddings / norms -----------------------------------------------
+struct RowMeta {          // device arrays built from the host plan of one score call
+    const int* cu_seqlens;    // [R+1] physical token offsets
+    const int* row_src;       // [R] offset of the row's tokens in its source array
+    const int* row_is_fg;     // [R]
+    const int* row_sign;      // [R] +1 / -1 / 0
+    const int* score_off;     // [R+1] offsets of each row's scored span
+};
+
+void launch_build_tokens(RowMeta m, int R, const int* probe_src, const int* fg_src,
+                         int* tok_id, int* tok_pos, int* tok_sign, int* tok_row, int* sc_tok,
+                         int* sc_tgt, const int* tgt_check_probe, const int* tgt_check_fg,
+                         const int* tgt_check_off, int* err_word, cudaStream_t st);
+void launch_embed(const int* tok_id, const int* tok_pos, const void* tok_embed,
+                  const void* pos_embed, int dtype, float* resid, int T, int d, cudaStream_t st);
+// kind 0: LayerNorm(w, b), 1: RMSNorm(w).  rows: optional gather list (else 0..T-1).
+void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
+                 const float* b, float eps, void* out, int out_type, cudaStream_t st);
+void launch_swiglu(const void* gu, int T, int f, void* out, int dtype, cudaStream_t st);
+
+// ---- GEMM ----------------------------------------------------------------------------
+enum Epi : int {
+    EPI_STORE = 0,       // C = acc + bias (out_type)
+    EPI_STORE_RELU = 1,  // C = relu(acc + bias)
+    EPI_RESID = 2,       // C(fp32) += acc + bias
+    EPI_SHRINK = 3,      // C = acc * (col < scale_cols ? sign[row] * eps : 1)
+    EPI_LSE = 4          // per (row, 64-col tile): max, sum exp(x - max); target logit
+};
+
+struct GemmArgs {
+    const void* A; int lda; int a_type;     // [M x K], K contiguous
+    const void* B; int ldb; int b_type;     // [N x K], K contiguous
+    const void* A2; int lda2;               // optional extension [M x K2] (type a2_type)
+    const void* B2; int ldb2;               // [N x K2] (type b2_type)
+    int a2_type, b2_type, K2;
+    int M, N, K;
+    const float* bias;
+    int epi;
+    void* C; int ldc; int c_type;
+    // EPI_SHRINK
+    const int* row_sign; float eps; int scale_cols;
+    // EPI_LSE
+    const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
+};
+
+void gemm_simt(const GemmArgs& g, cudaStream_t st);
+// tcgen05 / TMEM / TMA path; returns false when the shape is outside its limits.
+bool gemm_tc_supported(const GemmArgs& g);
+int gemm_tc(const GemmArgs& g, cudaStream_t st);   // 0 ok, else 1
+int gemm_lse_col_tiles(int N);                      // LSE column tiles, CUDA-core path (the most)
+int gemm_tc_col_tiles(int N);                       // LSE column tiles, tensor-core path
+int gemm_tc_error_word();                           // bit 0: a bounded wait expired
+
+// ---- attention -----------------------------------------------------------------------
+struct AttnArgs {
+    const void* qkv; int ld_qkv;    // [T x ld_qkv]: q at col 0, k at q_dim, v at q_dim+kv_dim
+    void* out; int ld_out;          // [T x H*hd]
+    int dtype;
+    const int* cu_seqlens;          // [R+1]
+    const int* tiles;               // [n_tiles] packed (row << 16 | q_tile)
+    int n_tiles;
+    int H, Hkv, hd;
+    float scale;
+    // Qwen3: per-head RMSNorm of q, k and rotary positions
+    const float* q_norm; const float* k_norm; float norm_eps; float rope_theta; int rope;
+};
+void launch_attention(const AttnArgs& a, cudaStream_t st);
+
+// ---- objective, estimator, update ------------------------------------------------------
+void launch_lse_merge(const float* part_max, const float* part_sum, const float* tgt_logit,
+                      int S, int n_tiles, float* logprob, cudaStream_t st);
+// per row L = -mean(logprob over its span) (fp64); L+/L- copies for the probe rows.
+void launch_row_objective(const float* logprob, const int* score_off, int R, int B,
+                          double* L_row, float* L_plus, float* L_minus, cudaStream_t st);
+// sums[0] = sum_i (L_row[i] - L_row[B+i]) in a fixed order, sums[1] = B.
+void launch_objective_sums(const double* L_row, int B, double* sums, cudaStream_t st);
+// c = sums[0] / sums[1] / (2 eps); flag = 1 if not finite (update refused).
+void launch_estimate(const double* sums, float eps, double* c, int* flag, cudaStream_t st);
+
+struct UpdateJob { float* A; const float* U; int n; };
+void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_n, const double* c,
+                        const int* flag, float lr, cudaStream_t st);
+
+}  // namespace zo

@@ -1,0 +1,147 @@
+// Kernel-level entry points (include/zo_ops.h): argument checks and launches.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "../../include/zo.h"
+#include "../../include/zo_ops.h"
+#include "kernels.h"
+
+using namespace zo;
+
+namespace {
+bool use_tc(int32_t impl, int dtype) {
+    if (impl == ZO_IMPL_CUDA_CORES) return false;
+    return dtype == ZO_DTYPE_BF16;
+}
+}  // namespace
+
+extern "C" {
+
+int zo_op_linear(const void* x, const void* W, const float* bias, void* y, int32_t M, int32_t N,
+                 int32_t K, int32_t dtype, int32_t act, int32_t accumulate, int32_t impl,
+                 void* stream) {
+    if (!x || !W || !y || M < 0 || N <= 0 || K <= 0) return ZO_ERR_ARG;
+    if (dtype != ZO_DTYPE_FP32 && dtype != ZO_DTYPE_BF16) return ZO_ERR_ARG;
+    if (act != ZO_ACT_NONE && act != ZO_ACT_RELU) return ZO_ERR_ARG;
+    if (accumulate && act != ZO_ACT_NONE) return ZO_ERR_ARG;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    const int t = dtype == ZO_DTYPE_BF16 ? E_BF16 : E_F32;
+    g.A = x; g.lda = K; g.a_type = t;
+    g.B = W; g.ldb = K; g.b_type = t;
+    g.M = M; g.N = N; g.K = K;
+    g.bias = bias;
+    g.epi = accumulate ? EPI_RESID : (act == ZO_ACT_RELU ? EPI_STORE_RELU : EPI_STORE);
+    g.C = y; g.ldc = N; g.c_type = accumulate ? E_F32 : t;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 0) return ZO_OK;
+    if (use_tc(impl, dtype)) {
+        if (gemm_tc_supported(g)) {
+            if (gemm_tc(g, st)) return ZO_ERR_CUDA;
+            return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+        }
+        if (impl == ZO_IMPL_TENSOR_CORES) return ZO_ERR_UNSUPPORTED;
+    } else if (impl == ZO_IMPL_TENSOR_CORES) {
+        return ZO_ERR_UNSUPPORTED;
+    }
+    gemm_simt(g, st);
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
+size_t zo_op_lm_head_workspace(int32_t n_rows, int32_t vocab, int32_t impl) {
+    (void)impl;
+    const size_t tiles = (size_t)gemm_lse_col_tiles(vocab);
+    const size_t part = ((size_t)n_rows * tiles * 4 + 255) / 256 * 256;
+    const size_t tg = ((size_t)n_rows * 4 + 255) / 256 * 256;
+    return 2 * part + tg;
+}
+
+int zo_op_lm_head_logprob(const void* h, const void* E, const int32_t* targets, int32_t n_rows,
+                          int32_t vocab, int32_t d, int32_t dtype, float* logprob,
+                          void* workspace, size_t workspace_bytes, int32_t impl, void* stream) {
+    if (!h || !E || !targets || !logprob || n_rows < 0 || vocab <= 0 || d <= 0) return ZO_ERR_ARG;
+    if (dtype != ZO_DTYPE_FP32 && dtype != ZO_DTYPE_BF16) return ZO_ERR_ARG;
+    if (n_rows == 0) return ZO_OK;
+    const size_t need = zo_op_lm_head_workspace(n_rows, vocab, impl);
+    if (!workspace || workspace_bytes < need) return ZO_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return ZO_ERR_ARG;
+    const int tiles = gemm_lse_col_tiles(vocab);   // the larger count: both paths fit
+    const size_t part = ((size_t)n_rows * tiles * 4 + 255) / 256 * 256;
+    char* ws = static_cast<char*>(workspace);
+    float* pmax = reinterpret_cast<float*>(ws);
+    float* psum = reinterpret_cast<float*>(ws + part);
+    float* tgt = reinterpret_cast<float*>(ws + 2 * part);
+    const int t = dtype == ZO_DTYPE_BF16 ? E_BF16 : E_F32;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.A = h; g.lda = d; g.a_type = t;
+    g.B = E; g.ldb = d; g.b_type = t;
+    g.M = n_rows; g.N = vocab; g.K = d;
+    g.epi = EPI_LSE;
+    g.targets = targets; g.part_max = pmax; g.part_sum = psum; g.tgt_logit = tgt;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool tc = use_tc(impl, dtype) && gemm_tc_supported(g);
+    if (impl == ZO_IMPL_TENSOR_CORES && !tc) return ZO_ERR_UNSUPPORTED;
+    g.n_col_tiles = tc ? gemm_tc_col_tiles(vocab) : tiles;
+    if (tc) {
+        if (gemm_tc(g, st)) return ZO_ERR_CUDA;
+    } else {
+        gemm_simt(g, st);
+    }
+    launch_lse_merge(pmax, psum, tgt, n_rows, g.n_col_tiles, logprob, st);
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
+int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t n_rows,
+                    int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t dtype,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+    if (!qkv || !out || !seq_lens || n_rows < 0 || n_heads <= 0 || n_kv_heads <= 0) return ZO_ERR_ARG;
+    if (n_heads % n_kv_heads) return ZO_ERR_ARG;
+    if (head_dim != 32 && head_dim != 64 && head_dim != 128 && head_dim != 256)
+        return ZO_ERR_UNSUPPORTED;
+    if (dtype != ZO_DTYPE_FP32 && dtype != ZO_DTYPE_BF16) return ZO_ERR_ARG;
+    if (n_rows == 0) return ZO_OK;
+    if (n_rows >= 32768) return ZO_ERR_ARG;
+    std::vector<int> meta(n_rows + 1);
+    meta[0] = 0;
+    std::vector<int> tiles;
+    for (int r = 0; r < n_rows; ++r) {
+        if (seq_lens[r] < 1 || seq_lens[r] > 65535 * 64) return ZO_ERR_ARG;
+        meta[r + 1] = meta[r] + seq_lens[r];
+        for (int q = 0; q < (seq_lens[r] + 63) / 64; ++q) tiles.push_back((r << 16) | q);
+    }
+    const size_t need = (meta.size() + tiles.size()) * 4;
+    if (!workspace || workspace_bytes < need) return ZO_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* w = static_cast<int*>(workspace);
+    meta.insert(meta.end(), tiles.begin(), tiles.end());
+    if (cudaMemcpyAsync(w, meta.data(), meta.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return ZO_ERR_CUDA;
+    // the host vector must outlive the copy
+    if (cudaStreamSynchronize(st) != cudaSuccess) return ZO_ERR_CUDA;
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.qkv = qkv; a.ld_qkv = (n_heads + 2 * n_kv_heads) * head_dim;
+    a.out = out; a.ld_out = n_heads * head_dim;
+    a.dtype = dtype == ZO_DTYPE_BF16 ? E_BF16 : E_F32;
+    a.cu_seqlens = w;
+    a.tiles = w + n_rows + 1;
+    a.n_tiles = (int)tiles.size();
+    a.H = n_heads; a.Hkv = n_kv_heads; a.hd = head_dim;
+    a.scale = (float)(1.0 / std::sqrt((double)head_dim));
+    launch_attention(a, st);
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
+/* Error word of the tensor-core kernels (bit 0: a bounded wait expired);
+ * synchronises the device and clears the word. */
+int zo_op_error_word(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    const int v = gemm_tc_error_word();
+    return v;
+}
+
+}  // extern "C"

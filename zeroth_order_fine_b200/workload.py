@@ -27,6 +27,16 @@ DTYPE_BF16 = 1
 MAT_Q, MAT_K, MAT_V, MAT_O, MAT_GATE, MAT_UP, MAT_DOWN = range(7)
 MATRIX_NAMES = ("q", "k", "v", "o", "gate", "up", "down")
 
+# Keys of the initial-weight tensors in the counter stream (weight_seed, layer, tensor):
+# matrix ids 0..6 name the matrices themselves, 7 + id their biases.
+T_BIAS0 = 7
+T_LN1_W, T_LN1_B, T_LN2_W, T_LN2_B, T_QNORM, T_KNORM = 14, 15, 16, 17, 18, 19
+T_TOK_EMBED, T_POS_EMBED, T_FINAL_W, T_FINAL_B, T_LM_HEAD = 32, 33, 34, 35, 36
+GLOBAL_LAYER = 0xFFFF
+# Initial distributions (a reading: the pages only say "random init"): matrices,
+# embeddings and biases N(0, 0.02); norm scales 1 + N(0, 0.02); LayerNorm shifts N(0, 0.02).
+INIT_STD = 0.02
+
 SCALE_LOZO = 0       # factors unscaled
 SCALE_MEZO = 1       # both factors multiplied by fp32(1/sqrt(r))
 
