@@ -232,7 +232,15 @@ int zo_stats(zo_handle* h, zo_stats_t* out);
 /* Serialise (run seed, step, nu, rank, targets, bank slots A_k) into buf
  * (host).  With buf == NULL only *n is set.  V factors are re-drawn from the
  * counter stream on load, so a resumed run reproduces the trajectory bit for
- * bit. */
+ * bit.  Layout (little endian): an 88-byte header
+ *   uint64 magic 0x5A4F42414E4B3031, version 1, run_seed, step, start_window;
+ *   int32 nu, rank, n_slots, scale_mode; uint32 matrix_mask, 0;
+ *   uint64 layer_mask_lo, layer_mask_hi, payload_floats
+ * then, for each layer, for each fused group in the order [q|k|v], o,
+ * FFN-in (OPT up; Qwen3 gate, up), FFN-out (down), for each slot j, for each
+ * targeted matrix of the group in id order: A_j^T as fp32 [r x d_in].
+ * zo_load_state accepts any buffer in this layout written under the same
+ * options (seed, nu, rank, targets), e.g. a bank trained elsewhere. */
 int zo_save_state(zo_handle* h, void* buf, size_t* n);
 int zo_load_state(zo_handle* h, const void* buf, size_t n);
 

@@ -40,3 +40,34 @@ def dev_tokens(batch: wl.Batch):
 
 def dev_fg_tokens(batch: wl.Batch):
     return torch.from_numpy(batch.fg_packed()).cuda()
+
+
+def oracle_state_blob(orc, w: wl.Workload, shape=None) -> bytes:
+    """The oracle's bank in the library's state layout (zo.h, zo_save_state)."""
+    import struct
+    shape = shape or w.shape
+    r = w.rank
+    groups = ([wl.MAT_Q, wl.MAT_K, wl.MAT_V], [wl.MAT_O],
+              [wl.MAT_UP] if shape.arch == wl.ARCH_OPT else [wl.MAT_GATE, wl.MAT_UP],
+              [wl.MAT_DOWN])
+    n_slots = len(next(iter(orc.bank.values())))
+    payload = []
+    for l in range(shape.n_layers):
+        for g in groups:
+            tg = [m for m in g if m in w.matrices and (l, m) in orc.bank]
+            for j in range(n_slots):
+                for m in tg:
+                    A = orc.bank[(l, m)][j][0].numpy()          # [d_in x r]
+                    payload.append(np.ascontiguousarray(A.T.astype(np.float32)))
+    data = b"".join(a.tobytes() for a in payload)
+    lo = hi = 0
+    for l in range(shape.n_layers):
+        if l < 64:
+            lo |= 1 << l
+        else:
+            hi |= 1 << (l - 64)
+    mm = sum(1 << m for m in w.matrices)
+    start_window = orc.bank[next(iter(orc.bank))][0][2]
+    head = struct.pack("<5Q4i2I3Q", 0x5A4F42414E4B3031, 1, w.run_seed, orc.t, start_window,
+                       orc.nu, r, n_slots, w.scale_mode, mm, 0, lo, hi, len(data) // 4)
+    return head + data

@@ -51,6 +51,7 @@ struct Group {
     int row_off[kMaxTargetsPerGroup] = {0, 0, 0};
     int d_out[kMaxTargetsPerGroup] = {0, 0, 0};
     float* FT = nullptr;         // shrink factors (fp32)
+    void* FTb = nullptr;         // bf16 mirror of FT (bf16 models): the shrink GEMM operand
     void* EB = nullptr;          // expand factors (model dtype)
     float* Vcur[kMaxTargetsPerGroup] = {nullptr, nullptr, nullptr};
 };
@@ -319,7 +320,9 @@ int open_window(zo_handle* h, uint64_t step) {
                 WindowJob w;
                 w.V = G.Vcur[t];
                 w.EB = G.EB;
-                w.A = G.FT + (size_t)(G.n_t * r * (1 + k) + t * r) * G.K;
+                const size_t a_off = (size_t)(G.n_t * r * (1 + k) + t * r) * G.K;
+                w.A = G.FT + a_off;
+                w.A_bf = G.FTb ? static_cast<char*>(G.FTb) + a_off * 2 : nullptr;
                 w.eb_type = h->dt;
                 w.ldb = h->kcap;
                 w.row0 = G.row_off[t];
@@ -332,6 +335,7 @@ int open_window(zo_handle* h, uint64_t step) {
                 UpdateJob u;
                 u.A = w.A;
                 u.U = G.FT + (size_t)(t * r) * G.K;
+                u.A_bf = w.A_bf;
                 u.n = r * G.K;
                 max_n = std::max(max_n, u.n);
                 uj[nu++] = u;
@@ -525,6 +529,11 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
             CRC(dev_alloc(h, &p, ft_rows * G.K * 4));
             G.FT = static_cast<float*>(p);
             CK(h, cudaMemsetAsync(G.FT, 0, ft_rows * G.K * 4, h->st));
+            if (h->dt == E_BF16) {
+                CRC(dev_alloc(h, &p, ft_rows * G.K * 2));
+                G.FTb = p;
+                CK(h, cudaMemsetAsync(G.FTb, 0, ft_rows * G.K * 2, h->st));
+            }
             CRC(dev_alloc(h, &p, (size_t)G.N * h->kcap * es));
             G.EB = p;
             CK(h, cudaMemsetAsync(G.EB, 0, (size_t)G.N * h->kcap * es, h->st));
@@ -581,8 +590,10 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
             for (int t = 0; t < G.n_t; ++t) {
                 int di, dout;
                 matrix_dims(d, G.mats[t], &di, &dout);
-                GenJob ju{G.FT + (size_t)t * r * G.K, l, G.mats[t], 0, di, r, 1, G.K};
-                GenJob jv{G.Vcur[t], l, G.mats[t], 1, dout, r, 0, 0};
+                GenJob ju{G.FT + (size_t)t * r * G.K,
+                          G.FTb ? static_cast<char*>(G.FTb) + (size_t)t * r * G.K * 2 : nullptr,
+                          l, G.mats[t], 0, di, r, 1, G.K};
+                GenJob jv{G.Vcur[t], nullptr, l, G.mats[t], 1, dout, r, 0, 0};
                 gu.push_back(ju);
                 gv.push_back(jv);
                 h->maxU_pairs = std::max(h->maxU_pairs, (di * r + 1) / 2);
@@ -795,7 +806,9 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
             GemmArgs s;
             memset(&s, 0, sizeof(s));
             s.A = X; s.lda = G.K; s.a_type = h->dt;
-            s.B = G.FT; s.ldb = G.K; s.b_type = E_F32;
+            if (G.FTb) { s.B = G.FTb; s.b_type = E_BF16; }
+            else { s.B = G.FT; s.b_type = E_F32; }
+            s.ldb = G.K;
             s.M = Ti; s.N = kext; s.K = G.K;
             s.epi = EPI_SHRINK;
             s.C = h->ext; s.ldc = h->kcap; s.c_type = h->dt;
@@ -1093,8 +1106,11 @@ int zo_load_state(zo_handle* h, const void* buf, size_t n) {
             for (int j = 0; j < hd.n_slots; ++j) {
                 const size_t bytes = (size_t)G.n_t * r * G.K * 4;
                 if (!bytes) continue;
-                CK(h, cudaMemcpyAsync(G.FT + (size_t)G.n_t * r * (1 + j) * G.K, p, bytes,
-                                      cudaMemcpyHostToDevice, h->st));
+                float* dst = G.FT + (size_t)G.n_t * r * (1 + j) * G.K;
+                CK(h, cudaMemcpyAsync(dst, p, bytes, cudaMemcpyHostToDevice, h->st));
+                if (G.FTb)
+                    launch_to_bf16(dst, static_cast<char*>(G.FTb) + (size_t)G.n_t * r * (1 + j) * G.K * 2,
+                                   bytes / 4, h->st);
                 p += bytes;
             }
     CK(h, cudaStreamSynchronize(h->st));

@@ -50,6 +50,7 @@ struct TcParams {
     const float* bias;
     void* C; int ldc; int c_type;
     const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
+    const int* row_sign; float eps; int scale_cols;
     int* err;
 };
 
@@ -225,6 +226,13 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, 
     if (EPI == EPI_STORE_RELU) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
+    }
+    if (EPI == EPI_SHRINK && n < p.scale_cols) {
+        // direction columns carry the row's candidate sign times eps
+        const float rs = (float)p.row_sign[m] * p.eps;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (n + j < p.scale_cols) v[j] *= rs;
     }
     if (p.c_type == E_BF16) {
         __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + (size_t)m * p.ldc + n;
@@ -500,6 +508,9 @@ bool gemm_tc_supported(const GemmArgs& g) {
             return true;
         case EPI_LSE:
             return true;
+        case EPI_SHRINK:
+            if (g.c_type != E_BF16 || g.ldc % 8 || !aligned16(g.C)) return false;
+            return true;
         default:
             return false;
     }
@@ -531,6 +542,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.C = g.C; p.ldc = g.ldc; p.c_type = g.c_type;
     p.targets = g.targets; p.part_max = g.part_max; p.part_sum = g.part_sum;
     p.tgt_logit = g.tgt_logit; p.n_col_tiles = g.n_col_tiles;
+    p.row_sign = g.row_sign; p.eps = g.eps; p.scale_cols = g.scale_cols;
     int* err = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
@@ -539,6 +551,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
         case EPI_STORE_RELU: return launch_epi<EPI_STORE_RELU>(a, b, a2, b2, p, st);
         case EPI_RESID: return launch_epi<EPI_RESID>(a, b, a2, b2, p, st);
         case EPI_LSE: return launch_epi<EPI_LSE>(a, b, a2, b2, p, st);
+        case EPI_SHRINK: return launch_epi<EPI_SHRINK>(a, b, a2, b2, p, st);
         default: return 1;
     }
 }

@@ -71,12 +71,9 @@ __global__ void __launch_bounds__(256) gen_factors_kernel(const GenJob* jobs, in
             if (e >= n) break;
             float v = z[h];
             if (apply_scale) v = __fmul_rn(v, scale);
-            if (jb.transposed) {
-                const uint64_t i = e / jb.r, c = e % jb.r;
-                jb.dst[c * (uint64_t)jb.ld + i] = v;
-            } else {
-                jb.dst[e] = v;
-            }
+            const uint64_t o = jb.transposed ? (e % jb.r) * (uint64_t)jb.ld + e / jb.r : e;
+            jb.dst[o] = v;
+            if (jb.dst_bf) static_cast<__nv_bfloat16*>(jb.dst_bf)[o] = __float2bfloat16_rn(v);
         }
     }
 }
@@ -108,8 +105,24 @@ __global__ void open_window_kernel(const WindowJob* jobs) {
         st_elem(jb.EB, row + jb.col_slot + c, jb.eb_type, v);
     }
     const int na = jb.d_in * jb.r;
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < na; e += gridDim.x * blockDim.x)
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < na; e += gridDim.x * blockDim.x) {
         jb.A[e] = 0.0f;
+        if (jb.A_bf) static_cast<__nv_bfloat16*>(jb.A_bf)[e] = __float2bfloat16_rn(0.0f);
+    }
+}
+
+__global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                               size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+void launch_to_bf16(const float* src, void* dst, size_t n, cudaStream_t st) {
+    if (n == 0) return;
+    unsigned b = cdiv((long long)n, 256);
+    if (b > 148 * 8) b = 148 * 8;
+    to_bf16_kernel<<<b, 256, 0, st>>>(src, static_cast<__nv_bfloat16*>(dst), n);
 }
 
 void launch_open_window(const WindowJob* d_jobs, int n_jobs, cudaStream_t st) {

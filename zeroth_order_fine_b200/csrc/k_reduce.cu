@@ -107,15 +107,22 @@ __global__ void __launch_bounds__(256) bank_update_kernel(const UpdateJob* __res
     const int n4 = jb.n >> 2;
     float4* A4 = reinterpret_cast<float4*>(jb.A);
     const float4* U4 = reinterpret_cast<const float4*>(jb.U);
+    __nv_bfloat162* B2 = static_cast<__nv_bfloat162*>(jb.A_bf);
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) {
         float4 a = A4[i];
         const float4 u = U4[i];
         a.x -= coef * u.x; a.y -= coef * u.y; a.z -= coef * u.z; a.w -= coef * u.w;
         A4[i] = a;
+        if (B2) {
+            B2[2 * i] = __floats2bfloat162_rn(a.x, a.y);
+            B2[2 * i + 1] = __floats2bfloat162_rn(a.z, a.w);
+        }
     }
     for (int i = (n4 << 2) + blockIdx.x * blockDim.x + threadIdx.x; i < jb.n;
-         i += gridDim.x * blockDim.x)
+         i += gridDim.x * blockDim.x) {
         jb.A[i] -= coef * jb.U[i];
+        if (jb.A_bf) static_cast<__nv_bfloat16*>(jb.A_bf)[i] = __float2bfloat16_rn(jb.A[i]);
+    }
 }
 
 void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_n, const double* c,

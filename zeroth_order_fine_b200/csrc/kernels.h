@@ -10,6 +10,7 @@ enum ElemType : int { E_F32 = 0, E_BF16 = 1 };
 // ---- generator -------------------------------------------------------------------------
 struct GenJob {
     float* dst;
+    void* dst_bf;               // optional bf16 mirror written at the same positions
     int layer, matrix, which;   // which: 0 = U, 1 = V
     int dim, r;                 // factor is [dim x r]
     int transposed, ld;         // transposed: write element (i, c) at dst[c*ld + i]
@@ -19,6 +20,7 @@ struct WindowJob {
     const float* V;             // [d_out x r] row-major
     void* EB;                   // extension operand [N x ldb] (model dtype)
     float* A;                   // new slot's A_k^T rows, r*d_in floats to zero
+    void* A_bf;                 // optional bf16 mirror of those rows
     int eb_type, ldb, row0, d_out, d_in, r, col_dir, col_slot;
 };
 
@@ -108,7 +110,8 @@ void launch_objective_sums(const double* L_row, int B, double* sums, cudaStream_
 // c = sums[0] / sums[1] / (2 eps); flag = 1 if not finite (update refused).
 void launch_estimate(const double* sums, float eps, double* c, int* flag, cudaStream_t st);
 
-struct UpdateJob { float* A; const float* U; int n; };
+struct UpdateJob { float* A; const float* U; void* A_bf; int n; };
+void launch_to_bf16(const float* src, void* dst, size_t n, cudaStream_t st);
 void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_n, const double* c,
                         const int* flag, float lr, cudaStream_t st);
 
