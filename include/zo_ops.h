@@ -59,10 +59,12 @@ int zo_op_lm_head_logprob(const void* h, const void* E, const int32_t* targets, 
  *   qkv      dev [T x (H + 2*Hkv)*hd] dtype: q | k | v per token
  *   out      dev [T x H*hd] dtype
  *   seq_lens host int32 [n_rows], rows back to back in qkv
- *   workspace dev >= 4*(n_rows + 1 + T/64 + n_rows + 1) bytes (row offsets and tiles) */
+ *   workspace dev >= 4*(n_rows + 1 + T/64 + n_rows + 1) bytes (row offsets and tiles)
+ *   impl     ZO_IMPL_TENSOR_CORES needs bf16 and head_dim 128; AUTO picks them then.
+ * The call copies the row offsets from the host and synchronises the stream. */
 int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t n_rows,
                     int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t dtype,
-                    void* workspace, size_t workspace_bytes, void* stream);
+                    void* workspace, size_t workspace_bytes, int32_t impl, void* stream);
 
 /* Synchronise the device and return the tensor-core kernels' error word:
  * 0 when clean, bit 0 set when a bounded wait inside a kernel expired (the

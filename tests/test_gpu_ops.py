@@ -105,15 +105,19 @@ def test_lm_head_logprob(S, V, d, dtype, impl):
     assert torch.max((got.double().cpu() - ref).abs()) < 2e-4
 
 
-@pytest.mark.parametrize("lens,H,Hkv,hd,dtype", [([1, 5, 64, 65, 130], 4, 4, 128, torch.float32),
-                                                 ([16, 128, 77, 3], 40, 40, 128, torch.bfloat16),
-                                                 ([200, 1, 64], 8, 2, 64, torch.float32)])
-def test_attention_matches_oracle(lens, H, Hkv, hd, dtype):
+@pytest.mark.parametrize("lens,H,Hkv,hd,dtype,impl", [
+    ([1, 5, 64, 65, 130], 4, 4, 128, torch.float32, 1),
+    ([16, 128, 77, 3], 40, 40, 128, torch.bfloat16, 1),
+    ([16, 128, 77, 3], 40, 40, 128, torch.bfloat16, 2),
+    ([1, 129, 300, 256, 512], 4, 2, 128, torch.bfloat16, 2),
+    ([200, 1, 64], 8, 2, 64, torch.float32, 1)])
+def test_attention_matches_oracle(lens, H, Hkv, hd, dtype, impl):
     from oracle import model as om
     from zeroth_order_fine_b200 import zo
     T = sum(lens)
     qkv = _rand((T, (H + 2 * Hkv) * hd), dtype, 16)
-    out = zo.zo_op_attention(qkv.cuda(), lens, H, Hkv, hd).double().cpu()
+    out = zo.zo_op_attention(qkv.cuda(), lens, H, Hkv, hd, impl=impl).double().cpu()
+    assert zo.zo_op_error_word() == 0
     q = qkv.double()[:, :H * hd].reshape(T, H, hd)
     k = qkv.double()[:, H * hd:(H + Hkv) * hd].reshape(T, Hkv, hd)
     v = qkv.double()[:, (H + Hkv) * hd:].reshape(T, Hkv, hd)

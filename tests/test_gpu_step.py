@@ -18,7 +18,7 @@ TINY = wl.WORKLOADS["tiny"]
 TINY_BF16 = dataclasses.replace(TINY, shape=wl.shrink_shape(wl.TINY, dtype=wl.DTYPE_BF16))
 # A small Qwen3-family model (GQA, q/k RMSNorm, RoPE, SwiGLU) with the MeZO-style
 # factorised direction on all seven matrices.
-Q3_SMALL = wl.ModelShape("qwen3-small", wl.ARCH_QWEN3, 2, 256, 4, 2, 64, 512, 1000, 4096, 1e-6,
+Q3_SMALL = wl.ModelShape("qwen3-small", wl.ARCH_QWEN3, 2, 256, 4, 2, 128, 512, 1000, 4096, 1e-6,
                          1e6, wl.DTYPE_FP32, False)
 QWEN_SMALL = wl.Workload("qwen3-small", Q3_SMALL, 6, 20, 90, 1, 4, True, 8, wl.ALL7,
                          wl.SCALE_MEZO, 1e-3, 1e-4, 3, fg_rows=4, data_seed=11)

@@ -749,6 +749,9 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
     }
     int fo = 0;
     int r = 0, nt = 0;
+    // attention tiles: 128 queries for the tensor-core kernel, 64 for the CUDA-core one
+    const bool tc_attn = h->use_tc && h->dt == E_BF16 && d.head_dim == 128;
+    const int qtile = tc_attn ? 128 : 64;
     for (int pass = 0; pass < 3; ++pass) {
         const int n = pass < 2 ? B : F;
         for (int i = 0; i < n; ++i, ++r) {
@@ -764,7 +767,7 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
             S += tl;
             cu[r + 1] = (int)std::min<long long>(T, 0x7fffffff);
             soff[r + 1] = (int)std::min<long long>(S, 0x7fffffff);
-            for (int q = 0; q < (L + 63) / 64; ++q) {
+            for (int q = 0; q < (L + qtile - 1) / qtile; ++q) {
                 if (nt >= h->max_tiles) FAIL(h, ZO_ERR_ARG, "too many attention tiles");
                 tiles[nt++] = (r << 16) | q;
             }
@@ -850,7 +853,8 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
             a.q_norm = L.w.q_norm; a.k_norm = L.w.k_norm; a.norm_eps = d.norm_eps;
             a.rope = 1; a.rope_theta = d.rope_theta;
         }
-        launch_attention(a, h->st);
+        if (tc_attn && attention_tc_supported(a)) launch_attention_tc(a, h->st);
+        else launch_attention(a, h->st);
         rc = group_gemm(L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32);
         if (rc) return rc;
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps, h->xn,
@@ -1025,6 +1029,8 @@ int zo_stats(zo_handle* h, zo_stats_t* out) {
     out->last_error_code = flag ? ZO_ERR_NONFINITE : h->err_code;
     const int ew = gemm_tc_error_word();
     if (ew > 0 && (ew & 1)) out->last_error_code = ZO_ERR_TIMEOUT;
+    const int aw = attention_tc_error_word();
+    if (aw > 0 && (aw & 1)) out->last_error_code = ZO_ERR_TIMEOUT;
     out->gemm_launches = h->prof.launches;
     out->gemm_ms = h->prof.ms;
     out->gemm_flops = h->prof.fl;

@@ -1,0 +1,371 @@
+// Packed variable-length causal attention on the 5th-generation tensor cores.
+//
+// One CTA (4 warps, 128 threads) takes one 128-query tile of one row for one
+// head; thread i owns query row i, which is also TMEM lane i.  Per 128-key
+// chunk of the row:
+//   S  = Q K^T        tcgen05.mma M=128 N=128 K=128, fp32 accumulator in TMEM
+//   P  = exp(S*scale - m)  (causal and length masks) written as bf16 into the
+//                     K buffer, in the 128-byte-swizzled K-major layout
+//   O += P V^T^T      tcgen05.mma M=128 N=128 K=128 with V staged transposed
+// With one chunk (rows <= 128 tokens, the common case) the row maximum comes
+// from the same S; with several, a first pass over the chunks finds the row
+// maximum so O can accumulate in TMEM without rescaling.  Queries, keys and
+// values are staged with plain coalesced loads (Qwen3 applies the per-head
+// RMSNorm and the rotary positions on the way), so a query's result depends
+// only on its own row: packing never changes a bit.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace zo {
+
+namespace {
+
+constexpr int TQ = 128, TK = 128, HD = 128;
+constexpr int ATOM = TQ * 128;                  // bytes of one 64-column swizzle atom block
+constexpr int BUF = 2 * ATOM;                   // one [128 x 128] bf16 operand
+constexpr int SMEM = 3 * BUF + 1024 + 64;
+constexpr uint32_t WAIT_LIMIT = 1u << 24;
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TK >> 3) << 17) |
+                            ((uint32_t)(TQ >> 4) << 24);
+
+__device__ int g_attn_error = 0;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+// byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] bf16 K-major SW128 operand
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+    return (uint32_t)((c >> 3) * ATOM + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Stage rows [r0, r0 + 128) of one head (column base col) into buf; rows past
+// n_rows are zero.  Plain copy: 16 threads per row, 16 bytes each, coalesced.
+__device__ __forceinline__ void stage_copy(uint8_t* buf, const __nv_bfloat16* base, size_t ld,
+                                           int n_rows) {
+    for (int idx = threadIdx.x; idx < TQ * 16; idx += blockDim.x) {
+        const int r = idx >> 4, c = idx & 15;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < n_rows) v = *reinterpret_cast<const uint4*>(base + (size_t)r * ld + c * 8);
+        *reinterpret_cast<uint4*>(buf + sw_off(r, c)) = v;
+    }
+}
+
+// Stage with the per-head RMSNorm and rotary positions (rotate-half pairs
+// (i, i + 64)); thread t owns row t.
+__device__ __forceinline__ void stage_norm_rope(uint8_t* buf, const __nv_bfloat16* base, size_t ld,
+                                                int n_rows, int pos0, const float* nw, float eps,
+                                                float theta) {
+    const int r = threadIdx.x;
+    const __nv_bfloat16* row = base + (size_t)r * ld;
+    float ss = 0.f;
+    if (r < n_rows)
+        for (int i = 0; i < HD; ++i) {
+            const float x = __bfloat162float(row[i]);
+            ss += x * x;
+        }
+    const float rs = 1.0f / sqrtf(ss / (float)HD + eps);
+    for (int c = 0; c < 8; ++c) {             // chunk c (dims 8c..) pairs with chunk c + 8
+        uint32_t lo[4], hi[4];
+        for (int j = 0; j < 8; j += 2) {
+            float a[2], b[2];
+            for (int u = 0; u < 2; ++u) {
+                const int i = 8 * c + j + u;
+                if (r < n_rows) {
+                    const float x1 = __bfloat162float(row[i]) * rs * nw[i];
+                    const float x2 = __bfloat162float(row[i + 64]) * rs * nw[i + 64];
+                    const double inv = pow((double)theta, -2.0 * i / HD);
+                    double sn, cs;
+                    sincos((double)(pos0 + r) * inv, &sn, &cs);
+                    a[u] = (float)(x1 * cs - x2 * sn);
+                    b[u] = (float)(x2 * cs + x1 * sn);
+                } else {
+                    a[u] = 0.f;
+                    b[u] = 0.f;
+                }
+            }
+            lo[j / 2] = pack_bf2(a[0], a[1]);
+            hi[j / 2] = pack_bf2(b[0], b[1]);
+        }
+        *reinterpret_cast<uint4*>(buf + sw_off(r, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(buf + sw_off(r, c + 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+}
+
+// V^T: row d of the operand holds dimension d over the chunk's 128 keys.
+// Thread t = dimension t; for each key the 128 threads read one contiguous row.
+__device__ __forceinline__ void stage_vt(uint8_t* buf, const __nv_bfloat16* base, size_t ld,
+                                         int n_keys) {
+    const int d = threadIdx.x;
+    const unsigned short* vb = reinterpret_cast<const unsigned short*>(base);
+    for (int kb = 0; kb < 16; ++kb) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const int k0 = kb * 8 + j;
+            const uint32_t a = k0 < n_keys ? vb[(size_t)k0 * ld + d] : 0u;
+            const uint32_t b = k0 + 1 < n_keys ? vb[(size_t)(k0 + 1) * ld + d] : 0u;
+            w[j / 2] = a | (b << 16);
+        }
+        *reinterpret_cast<uint4*>(buf + sw_off(d, kb)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* err) {
+    for (uint32_t i = 0;; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (i >= WAIT_LIMIT) {
+            atomicOr(err, 1);
+            return false;
+        }
+        if (i > 16) __nanosleep(64);
+    }
+}
+
+// 8 MMAs (K = 128 = 2 atoms x 4 steps of 16) into TMEM column d_col, then commit.
+__device__ __forceinline__ void mma_128(uint32_t d_tmem, uint32_t a, uint32_t b, bool accum_first,
+                                        uint32_t bar) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * ATOM + (kk & 3) * 32;
+        const uint32_t acc = (kk > 0 || accum_first) ? 1u : 0u;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(sw128_desc(a + off)), "l"(sw128_desc(b + off)), "r"(kIdesc), "r"(acc)
+            : "memory");
+    }
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* g = smem_raw + (base - raw);
+    uint8_t* Qb = g;
+    uint8_t* KPb = g + BUF;
+    uint8_t* Vb = g + 2 * BUF;
+    const uint32_t bar = base + 3 * BUF;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 3 * BUF + 16);
+
+    const int tile = a.tiles[blockIdx.x];
+    const int row = tile >> 16, qt = tile & 0xFFFF;
+    const int h = blockIdx.y;
+    const int kvh = h / (a.H / a.Hkv);
+    const int start = a.cu_seqlens[row];
+    const int len = a.cu_seqlens[row + 1] - start;
+    const int q0 = qt * TQ;
+    const int nq = min(TQ, len - q0);
+    const int kend = min(len, q0 + TQ);
+    const int n_chunks = (kend + TK - 1) / TK;
+    const int q_dim = a.H * HD, kv_dim = a.Hkv * HD;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const __nv_bfloat16* qkv = static_cast<const __nv_bfloat16*>(a.qkv);
+    const size_t ld = (size_t)a.ld_qkv;
+    int* err = &g_attn_error;
+
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                         smem_u32(tslot))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // queries of this tile
+    const __nv_bfloat16* qbase = qkv + (size_t)(start + q0) * ld + (size_t)h * HD;
+    if (a.rope) stage_norm_rope(Qb, qbase, ld, nq, q0, a.q_norm, a.norm_eps, a.rope_theta);
+    else stage_copy(Qb, qbase, ld, nq);
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tslot;
+    const uint32_t t_s = tmem, t_o = tmem + 128;
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    uint32_t phase = 0;
+    bool ok = true;
+    const int q = q0 + tid;                        // this thread's query position
+    const float sl2 = a.scale * 1.4426950408889634f;   // scale * log2(e)
+
+    auto stage_k = [&](int c0) {
+        const int nk = min(TK, kend - c0);
+        const __nv_bfloat16* kb = qkv + (size_t)(start + c0) * ld + q_dim + (size_t)kvh * HD;
+        if (a.rope) stage_norm_rope(KPb, kb, ld, nk, c0, a.k_norm, a.norm_eps, a.rope_theta);
+        else stage_copy(KPb, kb, ld, nk);
+    };
+    auto s_mma = [&]() {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) mma_128(t_s, smem_u32(Qb), smem_u32(KPb), false, bar);
+        ok = ok && wait_bar(bar, phase, err);
+        phase ^= 1u;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    };
+
+    // pass 1 (several chunks only): row maximum over every chunk
+    float m = -FLT_MAX;
+    if (n_chunks > 1) {
+        for (int ch = 0; ch < n_chunks && ok; ++ch) {
+            stage_k(ch * TK);
+            s_mma();
+            for (int cc = 0; cc < 4; ++cc) {
+                float v[32];
+                tmem_ld32(t_s + lane_addr + cc * 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int key = ch * TK + cc * 32 + j;
+                    if (key <= q && key < kend) m = fmaxf(m, v[j]);
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncthreads();                       // K buffer is restaged next
+        }
+    }
+    // pass 2: P = exp(S - m), O += P V
+    float l = 0.f;
+    for (int ch = 0; ch < n_chunks && ok; ++ch) {
+        const int c0 = ch * TK;
+        const int nk = min(TK, kend - c0);
+        stage_k(c0);
+        stage_vt(Vb, qkv + (size_t)(start + c0) * ld + q_dim + kv_dim + (size_t)kvh * HD, ld, nk);
+        s_mma();
+        if (!ok) break;
+        if (n_chunks == 1) {
+            for (int cc = 0; cc < 4; ++cc) {
+                float v[32];
+                tmem_ld32(t_s + lane_addr + cc * 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int key = cc * 32 + j;
+                    if (key <= q && key < kend) m = fmaxf(m, v[j]);
+                }
+            }
+        }
+        const float ms = m * sl2;
+        for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            tmem_ld32(t_s + lane_addr + cc * 32, v);
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float p2[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int key = c0 + cc * 32 + j + u;
+                    p2[u] = (key <= q && key < kend) ? exp2f(v[j + u] * sl2 - ms) : 0.f;
+                    l += p2[u];
+                }
+                w[j / 2] = pack_bf2(p2[0], p2[1]);
+            }
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+                *reinterpret_cast<uint4*>(KPb + sw_off(tid, cc * 4 + k4)) =
+                    make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) mma_128(t_o, smem_u32(KPb), smem_u32(Vb), ch > 0, bar);
+        ok = ok && wait_bar(bar, phase, err);
+        phase ^= 1u;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    }
+    // O / l -> bf16, one 256-byte row per thread
+    if (ok) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (size_t)(start + q) * a.ld_out +
+                              (size_t)h * HD;
+        for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            tmem_ld32(t_o + lane_addr + cc * 32, v);
+            if (tid < nq) {
+                uint4* o4 = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4)
+                    o4[k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
+                                        pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
+                                        pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
+                                        pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem)
+                     : "memory");
+}
+
+}  // namespace
+
+bool attention_tc_supported(const AttnArgs& a) {
+    return a.dtype == E_BF16 && a.hd == HD && a.ld_qkv % 8 == 0 && a.ld_out % 8 == 0 &&
+           (reinterpret_cast<uintptr_t>(a.qkv) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
+}
+
+void launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
+    if (a.n_tiles == 0) return;
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+        attr = true;
+    }
+    dim3 grid(a.n_tiles, a.H);
+    attention_tc_kernel<<<grid, 128, SMEM, st>>>(a);
+}
+
+int attention_tc_error_word() {
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_error, sizeof(int)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_attn_error, &zero, sizeof(int));
+    return v;
+}
+
+}  // namespace zo

@@ -1,6 +1,6 @@
 // Token metadata, embeddings, LayerNorm / RMSNorm (optionally gathering the
 // scored rows first) and the SwiGLU activation.  All HBM-bound, one CTA per
-// token row; the row is staged in shared memory so it is read once.
+// token row, each row read once.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -110,9 +110,93 @@ __global__ void __launch_bounds__(256) norm_kernel(const float* __restrict__ x,
     }
 }
 
+// Vectorised form for d % 4 == 0, d <= 1024 * VPT: the row stays in registers
+// (VPT float4 per thread), 16-byte loads, 8-byte bf16 stores.
+template <int VPT>
+__global__ void __launch_bounds__(256) norm_vec_kernel(const float* __restrict__ x,
+                                                       const int* __restrict__ rows, int d,
+                                                       int kind, const float* __restrict__ w,
+                                                       const float* __restrict__ b, float eps,
+                                                       void* __restrict__ out, int out_type) {
+    __shared__ float red[32];
+    const int t = blockIdx.x;
+    const int src = rows ? rows[t] : t;
+    const float4* xr = reinterpret_cast<const float4*>(x + (size_t)src * d);
+    const int n4 = d >> 2;
+    float4 v[VPT];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int j = threadIdx.x + i * 256;
+        v[i] = j < n4 ? xr[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+        s += kind == 0 ? (v[i].x + v[i].y) + (v[i].z + v[i].w)
+                       : (v[i].x * v[i].x + v[i].y * v[i].y) + (v[i].z * v[i].z + v[i].w * v[i].w);
+    }
+    s = block_sum(s, red);
+    float mean = 0.f, rstd;
+    if (kind == 0) {
+        mean = s / (float)d;
+        float q = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int j = threadIdx.x + i * 256;
+            if (j < n4) {
+                const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean,
+                            e = v[i].w - mean;
+                q += (a * a + bb * bb) + (c * c + e * e);
+            }
+        }
+        q = block_sum(q, red);
+        rstd = 1.0f / sqrtf(q / (float)d + eps);
+    } else {
+        rstd = 1.0f / sqrtf(s / (float)d + eps);
+    }
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    const float4* b4 = reinterpret_cast<const float4*>(b);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int j = threadIdx.x + i * 256;
+        if (j >= n4) continue;
+        const float4 ww = w4[j];
+        float4 y;
+        y.x = (v[i].x - mean) * rstd * ww.x;
+        y.y = (v[i].y - mean) * rstd * ww.y;
+        y.z = (v[i].z - mean) * rstd * ww.z;
+        y.w = (v[i].w - mean) * rstd * ww.w;
+        if (kind == 0) {
+            const float4 bb = b4[j];
+            y.x += bb.x; y.y += bb.y; y.z += bb.z; y.w += bb.w;
+        }
+        if (out_type == E_F32) {
+            reinterpret_cast<float4*>(out)[(size_t)t * n4 + j] = y;
+        } else {
+            uint2 pk;
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(y.x, y.y), h1 = __floats2bfloat162_rn(y.z, y.w);
+            pk.x = *reinterpret_cast<uint32_t*>(&h0);
+            pk.y = *reinterpret_cast<uint32_t*>(&h1);
+            reinterpret_cast<uint2*>(out)[(size_t)t * n4 + j] = pk;
+        }
+    }
+}
+
 void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
                  const float* b, float eps, void* out, int out_type, cudaStream_t st) {
     if (T == 0) return;
+    const int vpt = (d / 4 + 255) / 256;
+    auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    const bool aligned = al16(x) && al16(w) && (b == nullptr || al16(b)) && al16(out);
+    if (d % 4 == 0 && vpt <= 8 && aligned) {
+        switch (vpt) {
+            case 1: norm_vec_kernel<1><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            case 2: norm_vec_kernel<2><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            case 3: norm_vec_kernel<3><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            case 4: norm_vec_kernel<4><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            case 5: norm_vec_kernel<5><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            case 6: norm_vec_kernel<6><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            case 7: norm_vec_kernel<7><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            default: norm_vec_kernel<8><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+        }
+    }
     norm_kernel<<<T, 256, d * sizeof(float), st>>>(x, rows, d, kind, w, b, eps, out, out_type);
 }
 

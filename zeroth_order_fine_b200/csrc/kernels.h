@@ -97,7 +97,10 @@ struct AttnArgs {
     // Qwen3: per-head RMSNorm of q, k and rotary positions
     const float* q_norm; const float* k_norm; float norm_eps; float rope_theta; int rope;
 };
-void launch_attention(const AttnArgs& a, cudaStream_t st);
+void launch_attention(const AttnArgs& a, cudaStream_t st);          // CUDA cores, 64-query tiles
+bool attention_tc_supported(const AttnArgs& a);                     // bf16, head_dim 128
+void launch_attention_tc(const AttnArgs& a, cudaStream_t st);       // tensor cores, 128-query tiles
+int attention_tc_error_word();
 
 // ---- objective, estimator, update ------------------------------------------------------
 void launch_lse_merge(const float* part_max, const float* part_sum, const float* tgt_logit,

@@ -97,7 +97,7 @@ int zo_op_lm_head_logprob(const void* h, const void* E, const int32_t* targets, 
 
 int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t n_rows,
                     int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t dtype,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+                    void* workspace, size_t workspace_bytes, int32_t impl, void* stream) {
     if (!qkv || !out || !seq_lens || n_rows < 0 || n_heads <= 0 || n_kv_heads <= 0) return ZO_ERR_ARG;
     if (n_heads % n_kv_heads) return ZO_ERR_ARG;
     if (head_dim != 32 && head_dim != 64 && head_dim != 128 && head_dim != 256)
@@ -107,11 +107,14 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     if (n_rows >= 32768) return ZO_ERR_ARG;
     std::vector<int> meta(n_rows + 1);
     meta[0] = 0;
+    const bool tc = use_tc(impl, dtype) && head_dim == 128;
+    if (impl == ZO_IMPL_TENSOR_CORES && !tc) return ZO_ERR_UNSUPPORTED;
+    const int qtile = tc ? 128 : 64;
     std::vector<int> tiles;
     for (int r = 0; r < n_rows; ++r) {
         if (seq_lens[r] < 1 || seq_lens[r] > 65535 * 64) return ZO_ERR_ARG;
         meta[r + 1] = meta[r] + seq_lens[r];
-        for (int q = 0; q < (seq_lens[r] + 63) / 64; ++q) tiles.push_back((r << 16) | q);
+        for (int q = 0; q < (seq_lens[r] + qtile - 1) / qtile; ++q) tiles.push_back((r << 16) | q);
     }
     const size_t need = (meta.size() + tiles.size()) * 4;
     if (!workspace || workspace_bytes < need) return ZO_ERR_ARG;
@@ -132,7 +135,9 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     a.n_tiles = (int)tiles.size();
     a.H = n_heads; a.Hkv = n_kv_heads; a.hd = head_dim;
     a.scale = (float)(1.0 / std::sqrt((double)head_dim));
-    launch_attention(a, st);
+    if (tc && attention_tc_supported(a)) launch_attention_tc(a, st);
+    else if (impl == ZO_IMPL_TENSOR_CORES) return ZO_ERR_UNSUPPORTED;
+    else launch_attention(a, st);
     return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
 }
 
@@ -141,7 +146,9 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
 int zo_op_error_word(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return -1;
     const int v = gemm_tc_error_word();
-    return v;
+    const int w = attention_tc_error_word();
+    if (v < 0 || w < 0) return -1;
+    return v | w;
 }
 
 }  // extern "C"

@@ -116,7 +116,7 @@ _SIGS = {
                                         c_int32, c_void_p, c_void_p, ctypes.c_size_t, c_int32,
                                         c_void_p]),
     "zo_op_attention": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32,
-                                  c_int32, c_int32, c_void_p, ctypes.c_size_t, c_void_p]),
+                                  c_int32, c_int32, c_void_p, ctypes.c_size_t, c_int32, c_void_p]),
     "zo_op_error_word": (c_int32, []),
 }
 
@@ -416,14 +416,14 @@ def zo_op_lm_head_logprob(h: torch.Tensor, E: torch.Tensor, targets: torch.Tenso
 
 
 def zo_op_attention(qkv: torch.Tensor, seq_lens, n_heads: int, n_kv_heads: int,
-                    head_dim: int) -> torch.Tensor:
+                    head_dim: int, impl: int = IMPL_AUTO) -> torch.Tensor:
     sl = _i32(seq_lens)
     T = qkv.shape[0]
     dtype = wl.DTYPE_BF16 if qkv.dtype == torch.bfloat16 else wl.DTYPE_FP32
     out = torch.empty(T, n_heads * head_dim, dtype=qkv.dtype, device=qkv.device)
     ws = torch.empty(4 * (2 * len(sl) + 2 + T // 64 + 1) + 256, dtype=torch.uint8, device=qkv.device)
     _check(lib().zo_op_attention(_ptr(qkv), _ptr(out), _ptr(sl), len(sl), n_heads, n_kv_heads,
-                                 head_dim, dtype, _ptr(ws), ws.numel(), _stream()))
+                                 head_dim, dtype, _ptr(ws), ws.numel(), impl, _stream()))
     return out
 
 
