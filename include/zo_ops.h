@@ -66,6 +66,30 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
                     int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t dtype,
                     void* workspace, size_t workspace_bytes, int32_t impl, void* stream);
 
+/* zo_op_lm_head_logprob without a workspace argument: the same result (same
+ * kernels, same order), with the scratch taken from a 4 MiB array that the
+ * library keeps in device memory (one per GPU, resident until the process
+ * exits; zo_op_lm_head_noalloc_capacity() gives its size in floats).  This
+ * entry point is an addition of this library, not a step of the method, so
+ * no page describes it.  It is for callers that may not allocate device
+ * memory when they call -- e.g. a process whose device memory belongs to
+ * another runtime's pool, or a loop that must not touch the allocator after
+ * start-up -- and that have no spare buffer to pass as workspace.  It never
+ * allocates or frees (no cudaMalloc, no library allocator).
+ *   Limit: 2 * n_rows * tiles + n_rows <= capacity, with tiles = ceil(vocab/256)
+ *   on tensor cores and ceil(vocab/64) on CUDA cores; larger requests return
+ *   ZO_ERR_UNSUPPORTED (nothing is launched).
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture begins.
+ *   All calls share the array: calls whose kernels may overlap on a GPU (other
+ *   streams, no ordering between them) race and give wrong results.  Rows
+ *   whose target is outside [0, vocab) get NaN. */
+size_t zo_op_lm_head_noalloc_capacity(void);
+int zo_op_lm_head_logprob_noalloc(const void* h, const void* E, const int32_t* targets,
+                                  int32_t n_rows, int32_t vocab, int32_t d, int32_t dtype,
+                                  float* logprob, int32_t impl, void* stream);
+
 /* Synchronise the device and return the tensor-core kernels' error word:
  * 0 when clean, bit 0 set when a bounded wait inside a kernel expired (the
  * kernel then stopped early and its output is invalid), -1 when the device

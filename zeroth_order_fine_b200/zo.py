@@ -118,6 +118,9 @@ _SIGS = {
     "zo_op_attention": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                   c_int32, c_int32, c_void_p, ctypes.c_size_t, c_int32, c_void_p]),
     "zo_op_error_word": (c_int32, []),
+    "zo_op_lm_head_noalloc_capacity": (ctypes.c_size_t, []),
+    "zo_op_lm_head_logprob_noalloc": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32,
+                                                c_int32, c_int32, c_void_p, c_int32, c_void_p]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -424,6 +427,17 @@ def zo_op_attention(qkv: torch.Tensor, seq_lens, n_heads: int, n_kv_heads: int,
     ws = torch.empty(4 * (2 * len(sl) + 2 + T // 64 + 1) + 256, dtype=torch.uint8, device=qkv.device)
     _check(lib().zo_op_attention(_ptr(qkv), _ptr(out), _ptr(sl), len(sl), n_heads, n_kv_heads,
                                  head_dim, dtype, _ptr(ws), ws.numel(), impl, _stream()))
+    return out
+
+
+def zo_op_lm_head_logprob_noalloc(h: torch.Tensor, E: torch.Tensor, targets: torch.Tensor,
+                                   out: torch.Tensor, impl: int = IMPL_AUTO) -> torch.Tensor:
+    """The lm_head log-probabilities with the library's own fixed scratch (no
+    workspace, no allocation inside the call); ``out`` is the caller's buffer."""
+    S, d = h.shape
+    dtype = wl.DTYPE_BF16 if h.dtype == torch.bfloat16 else wl.DTYPE_FP32
+    _check(lib().zo_op_lm_head_logprob_noalloc(_ptr(h), _ptr(E), _ptr(targets), S, E.shape[0], d,
+                                               dtype, _ptr(out), impl, _stream()))
     return out
 
 
