@@ -221,6 +221,57 @@ def run_reference(args, w):
     return 0
 
 
+# ---- one op alone ----------------------------------------------------------------------
+
+def run_kernel(args):
+    """Time one op over --launches launches after 3 warm-up launches (CUDA events)."""
+    import torch
+
+    from zeroth_order_fine_b200 import zo
+    g = torch.Generator(device="cuda").manual_seed(0)
+    M, N, K = args.m, args.n, args.k
+    if args.kernel == "gemm":
+        x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+        W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+        fn = lambda: zo.zo_op_linear(x, W, out=y, impl=zo.IMPL_TENSOR_CORES)  # noqa: E731
+        work, unit = 2.0 * M * N * K, "TFLOP/s"
+        bytes_ = (M * K + N * K + M * N) * 2
+    elif args.kernel == "lm_head":
+        h = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+        E = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        tg = torch.randint(0, N, (M,), device="cuda", generator=g, dtype=torch.int32)
+        fn = lambda: zo.zo_op_lm_head_logprob(h, E, tg, impl=zo.IMPL_TENSOR_CORES)  # noqa: E731
+        work, unit = 2.0 * M * N * K, "TFLOP/s"
+        bytes_ = (M * K + N * K) * 2
+    else:
+        w = wl.WORKLOADS["opt-13b-b64"]
+        b = wl.make_batch(w)
+        lens = np.concatenate([b.seq_lens, b.seq_lens])
+        T = int(lens.sum())
+        H = w.shape.n_heads
+        qkv = torch.randn(T, 3 * H * 128, device="cuda", generator=g).to(torch.bfloat16)
+        fn = lambda: zo.zo_op_attention(qkv, lens, H, H, 128, impl=zo.IMPL_TENSOR_CORES)  # noqa
+        work = 4.0 * sum(L * (L + 1) / 2 for L in lens) * H * 128
+        unit = "TFLOP/s"
+        bytes_ = T * 4 * H * 128 * 2
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.launches):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.launches
+    assert zo.zo_op_error_word() == 0
+    print(json.dumps({"kernel": args.kernel, "m": M, "n": N, "k": K, "ms_per_launch": ms,
+                      "achieved": work / (ms / 1e3) / 1e12, "unit": unit,
+                      "gb_per_s": bytes_ / (ms / 1e3) / 1e9}), flush=True)
+    return 0
+
+
 # ---- the CUDA path ------------------------------------------------------------------
 
 def main():
@@ -234,7 +285,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cuda-cores", action="store_true", help="GEMMs on CUDA cores only")
+    ap.add_argument("--kernel", choices=["gemm", "attention", "lm_head"],
+                    help="time one op alone (kernel microbenchmark, used for ncu captures)")
+    ap.add_argument("--m", type=int, default=4096)
+    ap.add_argument("--n", type=int, default=5120)
+    ap.add_argument("--k", type=int, default=5120)
+    ap.add_argument("--launches", type=int, default=10)
     args = ap.parse_args()
+    if args.kernel:
+        return run_kernel(args)
     w = wl.WORKLOADS[args.workload]
     if args.warmup < 3:
         args.warmup = 3
