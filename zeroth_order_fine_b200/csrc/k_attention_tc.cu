@@ -26,7 +26,7 @@ constexpr int TQ = 128, TK = 128, HD = 128;
 constexpr int ATOM = TQ * 128;                  // bytes of one 64-column swizzle atom block
 constexpr int BUF = 2 * ATOM;                   // one [128 x 128] bf16 operand
 constexpr int SMEM = 3 * BUF + 1024 + 64;
-constexpr uint32_t WAIT_LIMIT = 1u << 24;
+constexpr long long WAIT_CYCLES = 4000000000ll;
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TK >> 3) << 17) |
                             ((uint32_t)(TQ >> 4) << 24);
 
@@ -143,6 +143,7 @@ __device__ __forceinline__ void stage_vt(uint8_t* buf, const __nv_bfloat16* base
 }
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* err) {
+    const long long t0 = clock64();
     for (uint32_t i = 0;; ++i) {
         uint32_t ok;
         asm volatile(
@@ -152,11 +153,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* err
             : "r"(bar), "r"(parity)
             : "memory");
         if (ok) return true;
-        if (i >= WAIT_LIMIT) {
+        if ((i & 63u) == 63u && clock64() - t0 > WAIT_CYCLES) {   // ~2 s: never arrives
             atomicOr(err, 1);
             return false;
         }
-        if (i > 16) __nanosleep(64);
     }
 }
 
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
         if (tid == 0) mma_128(t_s, smem_u32(Qb), smem_u32(KPb), false, bar);
-        ok = ok && wait_bar(bar, phase, err);
+        ok = __syncthreads_and(ok && wait_bar(bar, phase, err));   // uniform across the CTA
         phase ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     };
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
         if (tid == 0) mma_128(t_o, smem_u32(KPb), smem_u32(Vb), ch > 0, bar);
-        ok = ok && wait_bar(bar, phase, err);
+        ok = __syncthreads_and(ok && wait_bar(bar, phase, err));
         phase ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     }

@@ -38,7 +38,8 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 512;              // two BN-wide fp32 accumulators
 constexpr int GROUP_M = 8;
 constexpr int NUM_THREADS = 192;
-constexpr uint32_t WAIT_LIMIT = 1u << 24;   // ~2 s of polling with back-off
+constexpr uint32_t WAIT_LIMIT = 1u << 24;   // drain polls (with back-off) after an abort
+constexpr long long WAIT_CYCLES = 4000000000ll;   // ~2 s at 2 GHz: a stage that never arrives
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 __device__ int g_tc_error = 0;              // bit 0: a bounded wait expired
@@ -79,18 +80,23 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait; false when the limit expired or another role aborted.
+// Bounded wait; false when the limit expired or another role aborted.  No
+// sleep between polls: try_wait already suspends the thread in hardware for a
+// short while, and a software back-off would delay the hand-off of every stage.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_f,
                                           int* err) {
-    for (uint32_t i = 0;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort_f) return false;
-        if (i >= WAIT_LIMIT) {
-            *abort_f = 1;
-            atomicOr(err, 1);
-            return false;
+        if ((i & 63u) == 0) {
+            if (*abort_f) return false;
+            if (clock64() - t0 > WAIT_CYCLES) {
+                *abort_f = 1;
+                atomicOr(err, 1);
+                return false;
+            }
         }
-        if (i > 32) __nanosleep(128);
     }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
