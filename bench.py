@@ -303,7 +303,7 @@ def main():
     import torch
     import torch.distributed as dist
 
-    from zeroth_order_fine_b200 import zo
+    from zeroth_order_fine_b200 import dp, zo
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -338,9 +338,7 @@ def main():
         else:
             h.zo_score(tokens, batch.seq_lens, batch.target_lens)
         if world > 1:
-            h.zo_objective_sums(sums)
-            dist.all_reduce(sums)
-            c = h.zo_step_from_sums(w.lr, sums, want_c=want_c)
+            c = dp.dp_step(h, w.lr, sums, want_c=want_c)   # one 16-byte all-reduce per step
         else:
             c = h.zo_step(w.lr, want_c=want_c)
         step_no[0] += 1

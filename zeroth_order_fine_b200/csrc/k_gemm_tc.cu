@@ -43,6 +43,7 @@ constexpr long long WAIT_CYCLES = 4000000000ll;   // ~2 s at 2 GHz: a stage that
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 __device__ int g_tc_error = 0;              // bit 0: a bounded wait expired
+bool g_use_pairs = true;                    // SM-pair kernel for large decoder GEMMs
 
 struct TcParams {
     int M, N, kb_main, kb_ext;
@@ -429,6 +430,244 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
+// ---- 2-SM variant ----------------------------------------------------------------
+// A CTA pair (cluster of 2) computes one 256 x 256 tile: each CTA loads its
+// own 128 rows of A and its own 128 rows (half the N extent) of B, the even
+// CTA issues tcgen05.mma.cta_group::2 (M = 256) over both CTAs' shared
+// memory, and each CTA's TMEM receives its own 128 accumulator rows.  Per SM
+// this moves a third less operand data per FLOP than the 1-SM tile, so six
+// stages fit and the ring hides longer L2 latencies.  Loads carry no
+// multicast: every CTA fetches its own tiles.
+constexpr int BM2 = 256, STAGES2 = 6;
+constexpr int A2B = 128 * BK * 2;                // 16 KB of A per CTA per stage
+constexpr int B2B = 128 * BK * 2;                // 16 KB of B per CTA per stage
+constexpr int STAGE2_BYTES = A2B + B2B;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 256;
+constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                             ((uint32_t)(BM2 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    // arrive on the barrier at this offset in both CTAs of the pair
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n\t}" ::"r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tile_coords2(int t, const TcParams& p, int* mb, int* nb) {
+    const int per_group = GROUP_M * p.n_n_blk;
+    const int g = t / per_group;
+    const int first_m = g * GROUP_M;
+    const int gm = min(p.n_m_blk - first_m, GROUP_M);
+    const int in = t - g * per_group;
+    *mb = first_m + in % gm;
+    *nb = in / gm;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmA2,
+                    const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;     // same offset in both CTAs
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t bar0 = base + STAGES2 * STAGE2_BYTES;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (STAGES2 + s); };
+    auto tfull = [&](int b) { return bar0 + 8u * (2 * STAGES2 + b); };
+    auto tempty = [&](int b) { return bar0 + 8u * (2 * STAGES2 + 2 + b); };
+    const uint32_t drain = bar0 + 8u * (2 * STAGES2 + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES2 * STAGE2_BYTES + 160);
+    volatile int* abort_f = reinterpret_cast<volatile int*>(gbase + STAGES2 * STAGE2_BYTES + 168);
+
+    const uint32_t rank = cluster_rank();
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES2; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), 8);        // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(drain, 1);
+        *abort_f = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                         // both CTAs' barriers exist before any remote use
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int kb_total = p.kb_main + p.kb_ext;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int armed_s[STAGES2];
+            uint32_t armed_ph[STAGES2];
+            int n_armed = 0;
+            bool ok = true;
+            for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
+                int mb, nb;
+                tile_coords2(t, p, &mb, &nb);
+                const int row_a = mb * BM2 + (int)rank * 128;
+                const int row_b = nb * BN + (int)rank * 128;
+                for (int kb = 0; kb < kb_total; ++kb) {
+                    if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                    const uint32_t sa = base + s * STAGE2_BYTES;
+                    const uint32_t sb = sa + A2B;
+                    // the even CTA expects both CTAs' bytes on its barrier
+                    if (rank == 0) mbar_expect_tx(full(s), 2 * STAGE2_BYTES);
+                    const uint32_t lb = map_rank(full(s), 0);
+                    if (kb < p.kb_main) {
+                        tma_load_2d_pair(sa, &tmA, lb, kb * BK, row_a);
+                        tma_load_2d_pair(sb, &tmB, lb, kb * BK, row_b);
+                    } else {
+                        const int k = (kb - p.kb_main) * BK;
+                        tma_load_2d_pair(sa, &tmA2, lb, k, row_a);
+                        tma_load_2d_pair(sb, &tmB2, lb, k, row_b);
+                    }
+                    armed_s[n_armed % STAGES2] = s;
+                    armed_ph[n_armed % STAGES2] = ph;
+                    ++n_armed;
+                    if (++s == STAGES2) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (!ok && rank == 0) {
+                const int n = n_armed < STAGES2 ? n_armed : STAGES2;
+                for (int i = 0; i < n; ++i) {
+                    const int j = (n_armed - 1 - i) % STAGES2;
+                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(armed_s[j]), armed_ph[j]); ++it)
+                        __nanosleep(128);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t aph = 0;
+            bool ok = true, issued = false;
+            for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
+                if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < kb_total; ++kb) {
+                    if (!mbar_wait(full(s), ph, abort_f, p.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = base + s * STAGE2_BYTES;
+                    const uint32_t sb = sa + A2B;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), kIdesc2,
+                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit_pair(empty(s));       // stage free in both CTAs
+                    if (++s == STAGES2) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit_pair(tfull(acc));         // both halves of the accumulator ready
+                if (++acc == 2) { acc = 0; aph ^= 1u; }
+            }
+            if (!ok && issued) {
+                asm volatile(
+                    "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                        drain)
+                    : "memory");
+                for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(drain, 0); ++it) __nanosleep(128);
+            }
+        }
+    } else {
+        const int lane_base = 32 * (warp & 3);
+        const uint32_t leader_tempty0 = map_rank(tempty(0), 0);
+        const uint32_t leader_tempty1 = map_rank(tempty(1), 0);
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int t = pair; t < p.n_tiles; t += n_pairs) {
+            int mb, nb;
+            tile_coords2(t, p, &mb, &nb);
+            if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
+            tc_fence_after();
+            const int m = mb * BM2 + (int)rank * 128 + lane_base + lane;
+            float run_max = -FLT_MAX, run_sum = 0.f;
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n = nb * BN + c * 32;
+                if (n >= p.N) break;
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN + c * 32), v);
+                epilogue_chunk<EPI>(p, m, n, v, &run_max, &run_sum);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0);
+            if (++acc == 2) { acc = 0; aph ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                         // neither CTA leaves while the pair may touch it
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
 // ---- host side ---------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -491,6 +730,39 @@ int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
 
+template <int EPI>
+int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(gemm_tc2_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM2_BYTES) != cudaSuccess)
+            return 1;
+        attr = true;
+    }
+    static int max_pairs = 0;
+    if (!max_pairs) {
+        // SM pairs that can be resident at once (clusters of 2 stay inside a GPC)
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = 2; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = SMEM2_BYTES;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<EPI>, &cfg) != cudaSuccess || n <= 0)
+            n = num_sms() / 2;
+        max_pairs = n;
+    }
+    int pairs = max_pairs;
+    if (p.n_tiles < pairs) pairs = p.n_tiles;
+    gemm_tc2_kernel<EPI><<<2 * pairs, NUM_THREADS, SMEM2_BYTES, st>>>(a, b, a2, b2, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+
 }  // namespace
 
 bool gemm_tc_supported(const GemmArgs& g) {
@@ -525,12 +797,18 @@ bool gemm_tc_supported(const GemmArgs& g) {
 int gemm_tc_col_tiles(int N) { return (N + BN - 1) / BN; }
 
 int gemm_tc(const GemmArgs& g, cudaStream_t st) {
+    // Decoder GEMMs run on SM pairs, the LSE and shrink forms on single SMs.  The
+    // choice never depends on M (the batch): a row's bits must not change with
+    // the company it is scored in.
+    const bool pair = g_use_pairs && g.N > 128 &&
+                      (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID);
+    const uint32_t b_rows = pair ? 128u : (uint32_t)BN;
     CUtensorMap a, b, a2, b2;
     if (!make_map(&a, g.A, g.M, g.K, g.lda, BM)) return 1;
-    if (!make_map(&b, g.B, g.N, g.K, g.ldb, BN)) return 1;
+    if (!make_map(&b, g.B, g.N, g.K, g.ldb, b_rows)) return 1;
     if (g.K2 > 0) {
         if (!make_map(&a2, g.A2, g.M, g.K2, g.lda2, BM)) return 1;
-        if (!make_map(&b2, g.B2, g.N, g.K2, g.ldb2, BN)) return 1;
+        if (!make_map(&b2, g.B2, g.N, g.K2, g.ldb2, b_rows)) return 1;
     } else {
         a2 = a;
         b2 = b;
@@ -540,7 +818,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.M = g.M; p.N = g.N;
     p.kb_main = (g.K + BK - 1) / BK;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
-    p.n_m_blk = (g.M + BM - 1) / BM;
+    p.n_m_blk = pair ? (g.M + BM2 - 1) / BM2 : (g.M + BM - 1) / BM;
     p.n_n_blk = (g.N + BN - 1) / BN;
     p.n_tiles = p.n_m_blk * p.n_n_blk;
     p.epi = g.epi;
@@ -552,6 +830,14 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     int* err = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
+    if (pair) {
+        switch (g.epi) {
+            case EPI_STORE: return launch_epi2<EPI_STORE>(a, b, a2, b2, p, st);
+            case EPI_STORE_RELU: return launch_epi2<EPI_STORE_RELU>(a, b, a2, b2, p, st);
+            case EPI_RESID: return launch_epi2<EPI_RESID>(a, b, a2, b2, p, st);
+            default: return 1;
+        }
+    }
     switch (g.epi) {
         case EPI_STORE: return launch_epi<EPI_STORE>(a, b, a2, b2, p, st);
         case EPI_STORE_RELU: return launch_epi<EPI_STORE_RELU>(a, b, a2, b2, p, st);
@@ -561,6 +847,8 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
         default: return 1;
     }
 }
+
+void gemm_tc_set_pairs(bool on) { g_use_pairs = on; }
 
 int gemm_tc_error_word() {
     int v = 0;
