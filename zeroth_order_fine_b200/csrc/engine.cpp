@@ -849,6 +849,7 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
         a.tiles = tiles_d; a.n_tiles = nt;
         a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
         a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
+        a.n_tokens = Ti;
         if (d.arch == ZO_ARCH_QWEN3) {
             a.q_norm = L.w.q_norm; a.k_norm = L.w.k_norm; a.norm_eps = d.norm_eps;
             a.rope = 1; a.rope_theta = d.rope_theta;

@@ -6,13 +6,15 @@
 //   S  = Q K^T        tcgen05.mma M=128 N=128 K=128, fp32 accumulator in TMEM
 //   P  = exp(S*scale - m)  (causal and length masks) written as bf16 into the
 //                     K buffer, in the 128-byte-swizzled K-major layout
-//   O += P V^T^T      tcgen05.mma M=128 N=128 K=128 with V staged transposed
+//   O += P V          tcgen05.mma M=128 N=128 K=128, V read as an MN-major operand
 // With one chunk (rows <= 128 tokens, the common case) the row maximum comes
 // from the same S; with several, a first pass over the chunks finds the row
 // maximum so O can accumulate in TMEM without rescaling.  Queries, keys and
-// values are staged with plain coalesced loads (Qwen3 applies the per-head
-// RMSNorm and the rotary positions on the way), so a query's result depends
-// only on its own row: packing never changes a bit.
+// values arrive by TMA straight into the 128-byte-swizzled layout (Qwen3 then
+// applies the per-head RMSNorm and the rotary positions in shared memory).
+// Keys past the row's end are masked to zero probability, so a query's result
+// depends only on its own row: packing never changes a bit.
+#include <cuda.h>
 #include <float.h>
 
 #include "common.cuh"
@@ -70,78 +72,6 @@ __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Stage rows [r0, r0 + 128) of one head (column base col) into buf; rows past
-// n_rows are zero.  Plain copy: 16 threads per row, 16 bytes each, coalesced.
-__device__ __forceinline__ void stage_copy(uint8_t* buf, const __nv_bfloat16* base, size_t ld,
-                                           int n_rows) {
-    for (int idx = threadIdx.x; idx < TQ * 16; idx += blockDim.x) {
-        const int r = idx >> 4, c = idx & 15;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < n_rows) v = *reinterpret_cast<const uint4*>(base + (size_t)r * ld + c * 8);
-        *reinterpret_cast<uint4*>(buf + sw_off(r, c)) = v;
-    }
-}
-
-// Stage with the per-head RMSNorm and rotary positions (rotate-half pairs
-// (i, i + 64)); thread t owns row t.
-__device__ __forceinline__ void stage_norm_rope(uint8_t* buf, const __nv_bfloat16* base, size_t ld,
-                                                int n_rows, int pos0, const float* nw, float eps,
-                                                float theta) {
-    const int r = threadIdx.x;
-    const __nv_bfloat16* row = base + (size_t)r * ld;
-    float ss = 0.f;
-    if (r < n_rows)
-        for (int i = 0; i < HD; ++i) {
-            const float x = __bfloat162float(row[i]);
-            ss += x * x;
-        }
-    const float rs = 1.0f / sqrtf(ss / (float)HD + eps);
-    for (int c = 0; c < 8; ++c) {             // chunk c (dims 8c..) pairs with chunk c + 8
-        uint32_t lo[4], hi[4];
-        for (int j = 0; j < 8; j += 2) {
-            float a[2], b[2];
-            for (int u = 0; u < 2; ++u) {
-                const int i = 8 * c + j + u;
-                if (r < n_rows) {
-                    const float x1 = __bfloat162float(row[i]) * rs * nw[i];
-                    const float x2 = __bfloat162float(row[i + 64]) * rs * nw[i + 64];
-                    const double inv = pow((double)theta, -2.0 * i / HD);
-                    double sn, cs;
-                    sincos((double)(pos0 + r) * inv, &sn, &cs);
-                    a[u] = (float)(x1 * cs - x2 * sn);
-                    b[u] = (float)(x2 * cs + x1 * sn);
-                } else {
-                    a[u] = 0.f;
-                    b[u] = 0.f;
-                }
-            }
-            lo[j / 2] = pack_bf2(a[0], a[1]);
-            hi[j / 2] = pack_bf2(b[0], b[1]);
-        }
-        *reinterpret_cast<uint4*>(buf + sw_off(r, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint4*>(buf + sw_off(r, c + 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    }
-}
-
-// V^T: row d of the operand holds dimension d over the chunk's 128 keys.
-// Thread t = dimension t; for each key the 128 threads read one contiguous row.
-__device__ __forceinline__ void stage_vt(uint8_t* buf, const __nv_bfloat16* base, size_t ld,
-                                         int n_keys) {
-    const int d = threadIdx.x;
-    const unsigned short* vb = reinterpret_cast<const unsigned short*>(base);
-    for (int kb = 0; kb < 16; ++kb) {
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-            const int k0 = kb * 8 + j;
-            const uint32_t a = k0 < n_keys ? vb[(size_t)k0 * ld + d] : 0u;
-            const uint32_t b = k0 + 1 < n_keys ? vb[(size_t)(k0 + 1) * ld + d] : 0u;
-            w[j / 2] = a | (b << 16);
-        }
-        *reinterpret_cast<uint4*>(buf + sw_off(d, kb)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* err) {
     const long long t0 = clock64();
     for (uint32_t i = 0;; ++i) {
@@ -179,7 +109,74 @@ __device__ __forceinline__ void mma_128(uint32_t d_tmem, uint32_t a, uint32_t b,
                  : "memory");
 }
 
-__global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
+    // MN-major operand (V as the B operand of P.V): 64-element MN blocks 16 KB
+    // apart (leading byte offset), 8-row K groups 1024 bytes apart (stride byte offset)
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((uint32_t)ATOM >> 4) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+// P.V: A = P (K-major, keys contiguous), B = V as loaded ([keys x dims], MN-major)
+constexpr uint32_t kIdescPV = kIdesc | (1u << 16);
+
+__device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x,
+                                        int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// In place on a TMA-loaded [128 x 128] row tile: per-head RMSNorm and rotary
+// positions (rotate-half pairs (i, i + 64)); thread t owns row t.
+__device__ __forceinline__ void norm_rope_inplace(uint8_t* buf, int pos0, const float* nw, float eps,
+                                                  float theta) {
+    const int r = threadIdx.x;
+    float ss = 0.f;
+    for (int c = 0; c < 16; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(buf + sw_off(r, c));
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(h[j]);
+            ss += f.x * f.x + f.y * f.y;
+        }
+    }
+    const float rs = 1.0f / sqrtf(ss / (float)HD + eps);
+    for (int c = 0; c < 8; ++c) {
+        uint4 lo = *reinterpret_cast<const uint4*>(buf + sw_off(r, c));
+        uint4 hi = *reinterpret_cast<const uint4*>(buf + sw_off(r, c + 8));
+        __nv_bfloat162* hl = reinterpret_cast<__nv_bfloat162*>(&lo);
+        __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&hi);
+        for (int j = 0; j < 4; ++j) {
+            const float2 x1 = __bfloat1622float2(hl[j]);
+            const float2 x2 = __bfloat1622float2(hh[j]);
+            float o1[2], o2[2];
+            const float a1[2] = {x1.x, x1.y}, a2[2] = {x2.x, x2.y};
+            for (int u = 0; u < 2; ++u) {
+                const int i = 8 * c + 2 * j + u;
+                const float y1 = a1[u] * rs * nw[i];
+                const float y2 = a2[u] * rs * nw[i + 64];
+                const double inv = pow((double)theta, -2.0 * i / HD);
+                double sn, cs;
+                sincos((double)(pos0 + r) * inv, &sn, &cs);
+                o1[u] = (float)(y1 * cs - y2 * sn);
+                o2[u] = (float)(y2 * cs + y1 * sn);
+            }
+            hl[j] = __floats2bfloat162_rn(o1[0], o1[1]);
+            hh[j] = __floats2bfloat162_rn(o2[0], o2[1]);
+        }
+        *reinterpret_cast<uint4*>(buf + sw_off(r, c)) = lo;
+        *reinterpret_cast<uint4*>(buf + sw_off(r, c + 8)) = hi;
+    }
+}
+
+__global__ void __launch_bounds__(128, 2)
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -187,7 +184,8 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
     uint8_t* Qb = g;
     uint8_t* KPb = g + BUF;
     uint8_t* Vb = g + 2 * BUF;
-    const uint32_t bar = base + 3 * BUF;
+    const uint32_t bar_mma = base + 3 * BUF;
+    const uint32_t bar_ld = bar_mma + 8;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 3 * BUF + 16);
 
     const int tile = a.tiles[blockIdx.x];
@@ -202,13 +200,13 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
     const int n_chunks = (kend + TK - 1) / TK;
     const int q_dim = a.H * HD, kv_dim = a.Hkv * HD;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const __nv_bfloat16* qkv = static_cast<const __nv_bfloat16*>(a.qkv);
-    const size_t ld = (size_t)a.ld_qkv;
     int* err = &g_attn_error;
 
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ld));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
@@ -216,42 +214,54 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // queries of this tile
-    const __nv_bfloat16* qbase = qkv + (size_t)(start + q0) * ld + (size_t)h * HD;
-    if (a.rope) stage_norm_rope(Qb, qbase, ld, nq, q0, a.q_norm, a.norm_eps, a.rope_theta);
-    else stage_copy(Qb, qbase, ld, nq);
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tslot;
     const uint32_t t_s = tmem, t_o = tmem + 128;
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    uint32_t phase = 0;
+    uint32_t ph_mma = 0, ph_ld = 0;
     bool ok = true;
-    const int q = q0 + tid;                        // this thread's query position
-    const float sl2 = a.scale * 1.4426950408889634f;   // scale * log2(e)
+    const int q = q0 + tid;
+    const float sl2 = a.scale * 1.4426950408889634f;
+    const int kcol = q_dim + kvh * HD, vcol = q_dim + kv_dim + kvh * HD;
 
-    auto stage_k = [&](int c0) {
-        const int nk = min(TK, kend - c0);
-        const __nv_bfloat16* kb = qkv + (size_t)(start + c0) * ld + q_dim + (size_t)kvh * HD;
-        if (a.rope) stage_norm_rope(KPb, kb, ld, nk, c0, a.k_norm, a.norm_eps, a.rope_theta);
-        else stage_copy(KPb, kb, ld, nk);
+    // one TMA round trip: (Q,) K (and V) of chunk ch; rows past the tensor read as zero
+    auto load = [&](int ch, bool with_q, bool with_v) {
+        if (tid == 0) {
+            const uint32_t bytes = (uint32_t)BUF * (1 + (with_q ? 1 : 0) + (with_v ? 1 : 0));
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_ld),
+                         "r"(bytes)
+                         : "memory");
+            const int r0 = start + ch * TK;
+            for (int half = 0; half < 2; ++half) {
+                if (with_q)
+                    tma_box(smem_u32(Qb) + half * ATOM, &tm, bar_ld, h * HD + half * 64, start + q0);
+                tma_box(smem_u32(KPb) + half * ATOM, &tm, bar_ld, kcol + half * 64, r0);
+                if (with_v) tma_box(smem_u32(Vb) + half * ATOM, &tm, bar_ld, vcol + half * 64, r0);
+            }
+        }
+        ok = __syncthreads_and(ok && wait_bar(bar_ld, ph_ld, err));
+        ph_ld ^= 1u;
+        if (a.rope) {
+            if (with_q) norm_rope_inplace(Qb, q0, a.q_norm, a.norm_eps, a.rope_theta);
+            norm_rope_inplace(KPb, ch * TK, a.k_norm, a.norm_eps, a.rope_theta);
+        }
     };
     auto s_mma = [&]() {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
-        if (tid == 0) mma_128(t_s, smem_u32(Qb), smem_u32(KPb), false, bar);
-        ok = __syncthreads_and(ok && wait_bar(bar, phase, err));   // uniform across the CTA
-        phase ^= 1u;
+        if (tid == 0) mma_128(t_s, smem_u32(Qb), smem_u32(KPb), false, bar_mma);
+        ok = __syncthreads_and(ok && wait_bar(bar_mma, ph_mma, err));
+        ph_mma ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     };
 
-    // pass 1 (several chunks only): row maximum over every chunk
     float m = -FLT_MAX;
     if (n_chunks > 1) {
         for (int ch = 0; ch < n_chunks && ok; ++ch) {
-            stage_k(ch * TK);
+            load(ch, ch == 0, false);
             s_mma();
             for (int cc = 0; cc < 4; ++cc) {
                 float v[32];
@@ -263,16 +273,14 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
                 }
             }
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncthreads();                       // K buffer is restaged next
+            __syncthreads();
         }
     }
-    // pass 2: P = exp(S - m), O += P V
     float l = 0.f;
     for (int ch = 0; ch < n_chunks && ok; ++ch) {
         const int c0 = ch * TK;
-        const int nk = min(TK, kend - c0);
-        stage_k(c0);
-        stage_vt(Vb, qkv + (size_t)(start + c0) * ld + q_dim + kv_dim + (size_t)kvh * HD, ld, nk);
+        load(ch, ch == 0 && n_chunks == 1, true);
+        if (!ok) break;
         s_mma();
         if (!ok) break;
         if (n_chunks == 1) {
@@ -310,12 +318,28 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
-        if (tid == 0) mma_128(t_o, smem_u32(KPb), smem_u32(Vb), ch > 0, bar);
-        ok = __syncthreads_and(ok && wait_bar(bar, phase, err));
-        phase ^= 1u;
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t acc = (kk > 0 || ch > 0) ? 1u : 0u;
+                const uint64_t ad = sw128_desc(smem_u32(KPb) + (kk >> 2) * ATOM + (kk & 3) * 32);
+                const uint64_t bd = sw128_desc_mn(smem_u32(Vb) + kk * 2048);
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(t_o),
+                    "l"(ad), "l"(bd), "r"(kIdescPV), "r"(acc)
+                    : "memory");
+            }
+            asm volatile(
+                "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                    bar_mma)
+                : "memory");
+        }
+        ok = __syncthreads_and(ok && wait_bar(bar_mma, ph_mma, err));
+        ph_mma ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     }
-    // O / l -> bf16, one 256-byte row per thread
     if (ok) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (size_t)(start + q) * a.ld_out +
@@ -341,23 +365,54 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a) {
                      : "memory");
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn attn_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
 }  // namespace
 
 bool attention_tc_supported(const AttnArgs& a) {
     return a.dtype == E_BF16 && a.hd == HD && a.ld_qkv % 8 == 0 && a.ld_out % 8 == 0 &&
+           a.n_tokens > 0 && attn_encode_fn() != nullptr &&
            (reinterpret_cast<uintptr_t>(a.qkv) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
 }
 
 void launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
-    if (a.n_tiles == 0) return;
+    if (a.n_tiles == 0 || a.n_tokens <= 0) return;
     static bool attr = false;
     if (!attr) {
         cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         attr = true;
     }
+    // one map over the packed [T x ld_qkv] q|k|v rows: 64-column x 128-row boxes,
+    // 128-byte swizzle, rows past T read as zero
+    CUtensorMap tm;
+    EncodeTiledFn fn = attn_encode_fn();
+    if (!fn) return;
+    const cuuint64_t dims[2] = {(cuuint64_t)a.ld_qkv, (cuuint64_t)a.n_tokens};
+    const cuuint64_t strides[1] = {(cuuint64_t)a.ld_qkv * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t es[2] = {1, 1};
+    if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.qkv), dims, strides, box,
+           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return;
     dim3 grid(a.n_tiles, a.H);
-    attention_tc_kernel<<<grid, 128, SMEM, st>>>(a);
+    attention_tc_kernel<<<grid, 128, SMEM, st>>>(tm, a);
 }
 
 int attention_tc_error_word() {

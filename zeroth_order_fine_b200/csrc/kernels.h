@@ -97,6 +97,7 @@ struct AttnArgs {
     float scale;
     // Qwen3: per-head RMSNorm of q, k and rotary positions
     const float* q_norm; const float* k_norm; float norm_eps; float rope_theta; int rope;
+    int n_tokens;                   // T: rows of qkv (the tensor-core kernel's TMA extent)
 };
 void launch_attention(const AttnArgs& a, cudaStream_t st);          // CUDA cores, 64-query tiles
 bool attention_tc_supported(const AttnArgs& a);                     // bf16, head_dim 128
