@@ -36,6 +36,28 @@ METRIC = "ZO steps/s & scored tokens/s (OPT-13B shape, batch 64); % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def gemm_traffic():
+    """Per-launch DRAM bytes of the tensor-core GEMM from the committed ncu summary,
+    or None when the kernel source changed after the counters were taken."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "gemm_traffic_opt13b_b64.md")
+    src = os.path.join(ROOT, "zeroth_order_fine_b200", "csrc", "k_gemm_tc.cu")
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    fields = {}
+    for line in open(prof):
+        if ":" in line and line.strip().startswith(("source_sha256", "traffic_bytes_per_launch")):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256") != sha:
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -291,6 +313,9 @@ def main():
     ap.add_argument("--n", type=int, default=5120)
     ap.add_argument("--k", type=int, default=5120)
     ap.add_argument("--launches", type=int, default=10)
+    ap.add_argument("--byte-run", type=int, default=0,
+                    help="run this many consecutive steps of the banked run and report the "
+                         "state-transition bytes (1000 on opt-13b-b16 for the pages' comparison)")
     args = ap.parse_args()
     if args.kernel:
         return run_kernel(args)
@@ -322,8 +347,9 @@ def main():
     T = batch.n_tokens_physical
     S = int(2 * batch.target_lens.sum() + batch.fg_target_lens.sum())
     R = 2 * w.batch + len(batch.fg_prompts)
+    slots = max(8, args.byte_run // w.nu + 2)
     h = zo.Handle(model, w.run_seed, w.nu, w.rank, tg, max_tokens=T, max_rows=R, max_scored=S,
-                  max_slots=8, impl=1 if args.cuda_cores else 0, profile=1)
+                  max_slots=slots, impl=1 if args.cuda_cores else 0, profile=0 if args.byte_run else 1)
     toks = torch.from_numpy(batch.packed()).cuda()
     ftoks = torch.from_numpy(batch.fg_packed()).cuda() if batch.fg_prompts else None
     sums = torch.zeros(2, dtype=torch.float64, device="cuda")
@@ -344,6 +370,34 @@ def main():
         step_no[0] += 1
         return c
 
+    if args.byte_run:
+        t0 = time.perf_counter()
+        window_ms = []
+        tw = t0
+        for i in range(args.byte_run):
+            one_step(toks)
+            if (i + 1) % w.nu == 0:
+                torch.cuda.synchronize()
+                now = time.perf_counter()
+                window_ms.append(round(1000 * (now - tw) / w.nu, 2))
+                tw = now
+        torch.cuda.synchronize()
+        secs = time.perf_counter() - t0
+        st = h.zo_stats()
+        if rank == 0:
+            print(json.dumps({"byte_run": args.byte_run, "workload": w.name, "nu": w.nu,
+                              "bank_slots": st["bank_slots"],
+                              "state_transition_bytes": st["state_transition_bytes"],
+                              "dense_ref_bytes": st["dense_ref_bytes"],
+                              "dense_ref_bytes_targets": st["dense_ref_bytes_targets"],
+                              "frac_of_dense": st["state_transition_bytes"] / st["dense_ref_bytes"],
+                              "frac_of_dense_targets": st["state_transition_bytes"] /
+                              st["dense_ref_bytes_targets"],
+                              "seconds": secs, "ms_per_step": 1000 * secs / args.byte_run,
+                              "ms_per_step_by_window": window_ms,
+                              "last_error_code": st["last_error_code"]}), flush=True)
+        h.close()
+        return 0
     for _ in range(args.warmup):
         one_step(toks)
     torch.cuda.synchronize()
@@ -429,10 +483,12 @@ def main():
                           "roofline_ms": roof_t * 1000.0, "frac": roof_t * 1000.0 / ms,
                           "peak": f"{peak_kind} bf16 {peak_t} TFLOP/s sustained, "
                                   f"HBM {peaks['hbm_gbs']} GB/s"},
-        "roofline": {"kernel": "gemm_tc_kernel (tcgen05 GEMM, all epilogues)", "bound": "tensor",
+        "roofline": {"kernel": "tcgen05 GEMM (gemm_tc2_kernel SM pairs + gemm_tc_kernel; all epilogues)",
+                     "bound": "tensor",
                      "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": (gemm_tflops / peak_t) if gemm_tflops else None,
-                     "traffic": None, "launches_timed": d_n,
+                     "traffic": gemm_traffic(), "launches_timed": d_n,
+                     "algorithmic_flops_per_launch": d_fl / d_n if d_n else None,
                      "avg_launch_ms": d_ms / d_n if d_n else None,
                      "peak_kind": f"{peak_kind} (sustained: the kernel runs inside a long step)",
                      "share_of_step": (d_ms / args.steps) / ms if d_n else None},
