@@ -153,6 +153,8 @@ typedef struct zo_stats_t {
     uint64_t tc_gemm_launches;      /* of which on tensor cores                              */
     double   tc_gemm_ms;
     double   tc_gemm_flops;
+    uint64_t cuda_core_gemm_launches;/* GEMMs that ran on CUDA cores (always counted): 0 for
+                                       bf16 models unless options.impl asks for CUDA cores  */
 } zo_stats_t;
 
 /* ---- lifecycle -------------------------------------------------------------------- */

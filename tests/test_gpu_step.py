@@ -281,3 +281,50 @@ def test_state_transition_bytes_counted():
     assert s["state_transition_bytes"] == 6 * per_step + 2 * per_window
     assert s["dense_ref_bytes"] == 6 * 2 * 4 * sh.body_params()
     assert s["steps"] == 6 and s["bank_slots"] == 2
+
+
+@pytest.mark.parametrize("shape", ["tiny-bf16", "qwen3-bf16"])
+def test_bf16_models_never_leave_the_tensor_cores(shape):
+    """Every GEMM of a bf16 model runs on tcgen05 whatever the bank width: a window
+    opens every step (nu = 1), so the extension grows through widths of every residue."""
+    if shape == "tiny-bf16":
+        w = TINY_BF16
+    else:
+        w = dataclasses.replace(QWEN_SMALL, shape=dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16),
+                                fg_rows=0, rank=3)
+    batch = wl.make_batch(w, fg_rows=0)
+    model, h = gpu_handle(w, nu=1, max_slots=9)
+    toks = dev_tokens(batch)
+    for t in range(9):
+        h.zo_probe_plan(t, w.eps)
+        h.zo_score(toks, batch.seq_lens, batch.target_lens)
+        h.zo_step(w.lr)
+    s = h.zo_stats()
+    assert s["bank_slots"] == 9
+    assert s["cuda_core_gemm_launches"] == 0
+
+
+def test_load_state_clears_slots_beyond_the_loaded_bank():
+    """A shorter bank loaded into a handle that held a longer one scores like a fresh load."""
+    w = TINY_BF16
+    batch = wl.make_batch(w)
+    toks = dev_tokens(batch)
+    _, ha = gpu_handle(w, nu=1, max_slots=8)
+    for t in range(2):
+        ha.zo_probe_plan(t, w.eps)
+        ha.zo_score(toks, batch.seq_lens, batch.target_lens)
+        ha.zo_step(w.lr * 1000)
+    short = ha.zo_save_state()
+    for t in range(2, 6):
+        ha.zo_probe_plan(t, w.eps)
+        ha.zo_score(toks, batch.seq_lens, batch.target_lens)
+        ha.zo_step(w.lr * 1000)
+    ha.zo_load_state(short)
+    _, hb = gpu_handle(w, nu=1, max_slots=8)
+    hb.zo_load_state(short)
+    outs = []
+    for h in (ha, hb):
+        h.zo_probe_plan(2, w.eps)
+        Lp, Lm, _ = h.zo_score(toks, batch.seq_lens, batch.target_lens)
+        outs.append((Lp.cpu().numpy(), Lm.cpu().numpy()))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])

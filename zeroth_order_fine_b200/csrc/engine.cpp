@@ -293,6 +293,7 @@ int run_gemm(zo_handle* h, const GemmArgs& g, double algo_flops) {
         if (e) FAIL(h, ZO_ERR_CUDA, "tcgen05 GEMM launch failed");
     } else {
         gemm_simt(g, h->st);
+        h->stats.cuda_core_gemm_launches++;
     }
     prof_end(h, slot, algo_flops, tc);
     h->stats.kernel_launches++;
@@ -524,7 +525,9 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         for (auto& G : L.g) {
             if (G.n_t == 0) continue;
             if (G.K % 4) { h->err = "d_in must be a multiple of 4"; return fail(ZO_ERR_UNSUPPORTED); }
-            const size_t ft_rows = (size_t)G.n_t * r * (1 + options->max_slots);
+            // rows padded to the 64-row K tile: the shrink may read up to the next
+            // multiple of 8 past the live rows, which stay zero
+            const size_t ft_rows = ((size_t)G.n_t * r * (1 + options->max_slots) + 63) / 64 * 64;
             void* p = nullptr;
             CRC(dev_alloc(h, &p, ft_rows * G.K * 4));
             G.FT = static_cast<float*>(p);
@@ -805,7 +808,9 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
         memset(&g, 0, sizeof(g));
         g.M = Ti;
         if (G.n_t > 0) {
-            const int kext = G.n_t * r_ * (1 + h->n_slots);
+            // live extension columns, padded to a multiple of 8 (16-byte TMA rows); the
+            // padding columns of S and E_B are zero
+            const int kext = (G.n_t * r_ * (1 + h->n_slots) + 7) / 8 * 8;
             GemmArgs s;
             memset(&s, 0, sizeof(s));
             s.A = X; s.lda = G.K; s.a_type = h->dt;
@@ -891,6 +896,7 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
         }
         prof_end(h, slot, 2.0 * Si * (double)d.vocab * d.d_model, tc);
         h->stats.kernel_launches++;
+        if (!tc) h->stats.cuda_core_gemm_launches++;
     }
     launch_lse_merge(h->pmax, h->psum, h->tgt, Si, g.n_col_tiles, h->logprob, h->st);
     h->stats.tokens_scored += (uint64_t)T;
@@ -1096,7 +1102,17 @@ int zo_load_state(zo_handle* h, const void* buf, size_t n) {
         FAIL(h, ZO_ERR_ARG, "state was saved under different options");
     if (hd.n_slots > h->opt.max_slots) FAIL(h, ZO_ERR_UNSUPPORTED, "state has more slots than max_slots");
     if (n < sizeof(StateHeader) + hd.payload_floats * 4) FAIL(h, ZO_ERR_ARG, "truncated state");
-    // re-open every window in order (V re-drawn from the counter stream), then restore A
+    // clear the bank (rows past the loaded slots must read as zero), re-open every
+    // window in order (V re-drawn from the counter stream), then restore A
+    const int rr = h->opt.rank;
+    for (auto& L : h->layers)
+        for (auto& G : L.g) {
+            if (G.n_t == 0) continue;
+            const size_t ft_rows = ((size_t)G.n_t * rr * (1 + h->opt.max_slots) + 63) / 64 * 64;
+            CK(h, cudaMemsetAsync(G.FT, 0, ft_rows * G.K * 4, h->st));
+            if (G.FTb) CK(h, cudaMemsetAsync(G.FTb, 0, ft_rows * G.K * 2, h->st));
+            CK(h, cudaMemsetAsync(G.EB, 0, (size_t)G.N * h->kcap * esize(h->dt), h->st));
+        }
     h->n_slots = 0;
     h->slot_window.clear();
     h->have_plan = false;

@@ -48,6 +48,7 @@ bool g_use_pairs = true;                    // SM-pair kernel for large decoder 
 struct TcParams {
     int M, N, kb_main, kb_ext;
     int n_m_blk, n_n_blk, n_tiles;
+    int group_m;                            // M blocks per raster group
     int epi;
     const float* bias;
     void* C; int ldc; int c_type;
@@ -492,10 +493,10 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
 }
 
 __device__ __forceinline__ void tile_coords2(int t, const TcParams& p, int* mb, int* nb) {
-    const int per_group = GROUP_M * p.n_n_blk;
+    const int per_group = p.group_m * p.n_n_blk;
     const int g = t / per_group;
-    const int first_m = g * GROUP_M;
-    const int gm = min(p.n_m_blk - first_m, GROUP_M);
+    const int first_m = g * p.group_m;
+    const int gm = min(p.n_m_blk - first_m, p.group_m);
     const int in = t - g * per_group;
     *mb = first_m + in % gm;
     *nb = in / gm;
@@ -819,6 +820,14 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.kb_main = (g.K + BK - 1) / BK;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
     p.n_m_blk = pair ? (g.M + BM2 - 1) / BM2 : (g.M + BM - 1) / BM;
+    // Raster: an M group whose A strips (256 rows x K) fit in ~48 MB of L2 sweeps all N
+    // blocks, so each weight strip is fetched from DRAM once per group.
+    {
+        const double strip = (double)BM2 * (g.K + g.K2) * 2.0;
+        int gm = (int)(48.0e6 / strip);
+        gm = gm < 4 ? 4 : (gm > 32 ? 32 : gm);
+        p.group_m = pair ? gm : GROUP_M;
+    }
     p.n_n_blk = (g.N + BN - 1) / BN;
     p.n_tiles = p.n_m_blk * p.n_n_blk;
     p.epi = g.epi;

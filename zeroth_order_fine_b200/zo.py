@@ -78,7 +78,8 @@ class zo_stats_t(ctypes.Structure):
                 ("last_error_code", c_int32), ("kernel_launches", c_uint64),
                 ("gemm_launches", c_uint64), ("gemm_ms", ctypes.c_double),
                 ("gemm_flops", ctypes.c_double), ("tc_gemm_launches", c_uint64),
-                ("tc_gemm_ms", ctypes.c_double), ("tc_gemm_flops", ctypes.c_double)]
+                ("tc_gemm_ms", ctypes.c_double), ("tc_gemm_flops", ctypes.c_double),
+                ("cuda_core_gemm_launches", c_uint64)]
 
 
 _I32P = ctypes.POINTER(c_int32)
