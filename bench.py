@@ -429,6 +429,46 @@ def main():
         dist.all_reduce(t_, op=dist.ReduceOp.MAX)
         ms = float(t_.item())
 
+    # matched-query control: the same physical queries (zo_score only, no plan or
+    # update), to set the complete step against the queries it requires
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h.zo_probe_plan(step_no[0], w.eps)
+    c0.record(stream)
+    for _ in range(args.steps):
+        if ftoks is not None:
+            h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, ftoks, batch.fg_seq_lens,
+                               batch.fg_target_lens)
+        else:
+            h.zo_score(toks, batch.seq_lens, batch.target_lens)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    control_ms = c0.elapsed_time(c1) / args.steps
+    h.zo_step(w.lr, want_c=False)
+    step_no[0] += 1
+    cobatch = None
+    if ftoks is not None:
+        # co-serving analogue: probe rows alone and foreground rows alone vs the mixed batch
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h.zo_probe_plan(step_no[0], w.eps)
+        p0.record(stream)
+        for _ in range(args.steps):
+            h.zo_score(toks, batch.seq_lens, batch.target_lens)
+        p1.record(stream)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            h.zo_score_foreground(ftoks, batch.fg_seq_lens, batch.fg_target_lens)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        probe_ms = p0.elapsed_time(p1) / args.steps
+        fg_ms = f0.elapsed_time(f1) / args.steps
+        cobatch = {"mixed_batch_ms": control_ms, "probe_rows_alone_ms": probe_ms,
+                   "foreground_rows_alone_ms": fg_ms,
+                   "mixed_vs_separate": control_ms / (probe_ms + fg_ms)}
+        h.zo_step(w.lr, want_c=False)
+        step_no[0] += 1
+
     # e2e: the same steps through the public API with host buffers (pinned), the
     # H2D copy of the step's tokens and the D2H read of c inside the timed region
     e2e = None
@@ -500,6 +540,8 @@ def main():
                                                             s0["dense_ref_bytes_targets"]) / args.steps},
         "phases_ms_per_step": {k: (s1[k] - s0[k]) / args.steps for k in ("ms_plan", "ms_score",
                                                                          "ms_step")},
+        "matched_query_control": {"score_only_ms": control_ms, "step_over_control": ms / control_ms},
+        "cobatch": cobatch,
         "gpu_launches": int(s1["kernel_launches"] - s0["kernel_launches"]),
         "e2e": e2e,
         "clocks": clocks,

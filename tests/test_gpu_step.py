@@ -276,7 +276,7 @@ def test_state_transition_bytes_counted():
     sh = w.shape
     u = sum(sh.matrix_dims(m)[0] * w.rank for m in w.matrices) * sh.n_layers
     v = sum(sh.matrix_dims(m)[1] * w.rank for m in w.matrices) * sh.n_layers
-    per_step = 4 * u + (8 * u + 4 * u)
+    per_step = 4 * u + (8 * u + 4 * u)              # fp32 model: no bf16 copies
     per_window = 4 * v + 2 * 4 * v + 4 * u
     assert s["state_transition_bytes"] == 6 * per_step + 2 * per_window
     assert s["dense_ref_bytes"] == 6 * 2 * 4 * sh.body_params()

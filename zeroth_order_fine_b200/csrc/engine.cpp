@@ -623,9 +623,11 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
     }
     // state-transition byte model: U written each step; A read+written and U read by the
     // update; at a window start V written (fp32), EB written twice (model dtype), A zeroed.
-    h->bytes_per_U = u_elems * 4;
-    h->bytes_per_update = a_elems * 8 + u_elems * 4;
-    h->bytes_per_window = v_elems * 4 + v_elems * 2 * es + a_elems * 4;
+    // bf16 models also keep bf16 copies of U and A (the shrink GEMM's operand)
+    const uint64_t mirror = h->dt == E_BF16 ? 2 : 0;
+    h->bytes_per_U = u_elems * (4 + mirror);
+    h->bytes_per_update = a_elems * (8 + mirror) + u_elems * 4;
+    h->bytes_per_window = v_elems * 4 + v_elems * 2 * es + a_elems * (4 + mirror);
     // dense mutation reference: 2 * |theta| bytes (model dtype) per step
     uint64_t body = 0, tgt = 0;
     for (int l = 0; l < d.n_layers; ++l)
