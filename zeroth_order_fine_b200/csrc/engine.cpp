@@ -47,6 +47,7 @@ struct Group {
     const void* W = nullptr;     // [N x K]
     const float* bias = nullptr;
     int n_t = 0;                 // targeted matrices in this group
+    int interleave = 0;          // [gate|up] rows interleaved in 128-row blocks (SwiGLU epilogue)
     int mats[kMaxTargetsPerGroup] = {0, 0, 0};
     int row_off[kMaxTargetsPerGroup] = {0, 0, 0};
     int d_out[kMaxTargetsPerGroup] = {0, 0, 0};
@@ -142,6 +143,7 @@ struct zo_handle {
     bool have_plan = false;
     float mezo_scale = 1.f;
     bool use_tc = false;
+    bool swiglu_fused = false;    // Qwen3 FFN-in GEMM writes silu(gate) * up directly
     // stats
     zo_stats_t stats;
     PhaseTimer tm[3];
@@ -287,6 +289,7 @@ void prof_end(zo_handle* h, int slot, double flops, bool tc) {
 // algo_flops: the launch's algorithmic FLOPs (for the live roofline).
 int run_gemm(zo_handle* h, const GemmArgs& g, double algo_flops) {
     const bool tc = h->use_tc && gemm_tc_supported(g);
+    if (g.epi == EPI_SWIGLU && !tc) FAIL(h, ZO_ERR_UNSUPPORTED, "fused SwiGLU needs tensor cores");
     const int slot = prof_begin(h);
     if (tc) {
         int e = gemm_tc(g, h->st);
@@ -332,6 +335,7 @@ int open_window(zo_handle* h, uint64_t step) {
                 w.r = r;
                 w.col_dir = t * r;
                 w.col_slot = G.n_t * r * (1 + k) + t * r;
+                w.interleave = G.interleave;
                 wj[nw++] = w;
                 UpdateJob u;
                 u.A = w.A;
@@ -381,7 +385,13 @@ void build_groups(zo_handle* h, int l, Layer& L) {
         add(in, ZO_MAT_UP, 0);
     } else {
         in.N = 2 * d.d_ffn;
-        add(in, ZO_MAT_GATE, 0); add(in, ZO_MAT_UP, d.d_ffn);
+        if (h->swiglu_fused) {
+            // rows interleaved: gate block b at rows 256 b .. + 128, up block b right after
+            in.interleave = 1;
+            add(in, ZO_MAT_GATE, 0); add(in, ZO_MAT_UP, 128);
+        } else {
+            add(in, ZO_MAT_GATE, 0); add(in, ZO_MAT_UP, d.d_ffn);
+        }
     }
     Group& out = L.g[G_OUT];
     out.N = d.d_model; out.K = d.d_ffn; out.W = w.w[ZO_MAT_DOWN]; out.bias = w.b[ZO_MAT_DOWN];
@@ -461,6 +471,8 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         if (rc__) return fail(rc__);    \
     } while (0)
 
+    h->use_tc = h->dt == E_BF16 && options->impl == 0;
+    h->swiglu_fused = h->use_tc && d.arch == ZO_ARCH_QWEN3 && d.d_ffn % 128 == 0;
     // layers, fused weights and bank buffers
     h->layers.resize(d.n_layers);
     int max_nt = 0;
@@ -510,7 +522,19 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         Layer& L = h->layers[l];
         const int qkv[3] = {ZO_MAT_Q, ZO_MAT_K, ZO_MAT_V};
         CRC(fused_copy(L, L.g[G_QKV], qkv, 3));
-        if (d.arch == ZO_ARCH_QWEN3) {
+        if (d.arch == ZO_ARCH_QWEN3 && h->swiglu_fused) {
+            Group& G = L.g[G_IN];
+            void* W = nullptr;
+            CRC(dev_alloc(h, &W, (size_t)G.N * G.K * es));
+            const size_t blk = (size_t)128 * G.K * es;          // 128 rows of one matrix
+            for (int half = 0; half < 2; ++half) {
+                const void* src = L.w.w[half == 0 ? ZO_MAT_GATE : ZO_MAT_UP];
+                if (!src) { h->err = "missing gate/up weights"; return fail(ZO_ERR_ARG); }
+                CK(h, cudaMemcpy2DAsync(static_cast<char*>(W) + half * blk, 2 * blk, src, blk, blk,
+                                        d.d_ffn / 128, cudaMemcpyDeviceToDevice, h->st));
+            }
+            G.W = W;
+        } else if (d.arch == ZO_ARCH_QWEN3) {
             const int gu[2] = {ZO_MAT_GATE, ZO_MAT_UP};
             CRC(fused_copy(L, L.g[G_IN], gu, 2));
         }
@@ -554,7 +578,8 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
     CRC(dev_alloc(h, &h->qkv, (size_t)maxT * h->n_qkv * es));
     CRC(dev_alloc(h, &h->att, (size_t)maxT * h->q_dim * es));
     CRC(dev_alloc(h, &h->act, (size_t)maxT * d.d_ffn * es));
-    if (d.arch == ZO_ARCH_QWEN3) CRC(dev_alloc(h, &h->gu, (size_t)maxT * ffn_cols * es));
+    if (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused)
+        CRC(dev_alloc(h, &h->gu, (size_t)maxT * ffn_cols * es));
     if (h->kcap) CRC(dev_alloc(h, &h->ext, (size_t)maxT * h->kcap * es));
     CRC(dev_alloc(h, &h->hs, (size_t)maxS * d.d_model * es));
     h->lse_tiles = gemm_lse_col_tiles(d.vocab);
@@ -641,7 +666,6 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         }
     h->dense_bytes = 2 * body * es;
     h->dense_bytes_targets = 2 * tgt * es;
-    h->use_tc = h->dt == E_BF16 && options->impl == 0;
     if (options->profile) {
         GemmProfiler& p = h->prof;
         p.a.resize(GemmProfiler::kRing);
@@ -798,7 +822,8 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
     launch_build_tokens(m, R, ptok, ftok, h->tok_id, h->tok_pos, h->tok_sign, h->tok_row,
                         h->sc_tok, h->sc_tgt, tgt_ids, nullptr, chk_d, h->err_dev, h->st);
     // build_tokens, embed, per layer 2 norms + attention (+ SwiGLU), final norm, LSE merge
-    h->stats.kernel_launches += 2 + (uint64_t)d.n_layers * (3 + (d.arch == ZO_ARCH_QWEN3)) + 2;
+    h->stats.kernel_launches +=
+        2 + (uint64_t)d.n_layers * (3 + (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused)) + 2;
     launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
                  d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
                  d.d_model, h->st);
@@ -869,6 +894,8 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
                     h->dt, h->st);
         if (d.arch == ZO_ARCH_OPT) {
             rc = group_gemm(L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt);
+        } else if (h->swiglu_fused) {
+            rc = group_gemm(L.g[G_IN], h->xn, EPI_SWIGLU, h->act, d.d_ffn, h->dt);
         } else {
             rc = group_gemm(L.g[G_IN], h->xn, EPI_STORE, h->gu, 2 * d.d_ffn, h->dt);
             if (!rc) launch_swiglu(h->gu, Ti, d.d_ffn, h->act, h->dt, h->st);

@@ -7,9 +7,9 @@
 //   P  = exp(S*scale - m)  (causal and length masks) written as bf16 into the
 //                     K buffer, in the 128-byte-swizzled K-major layout
 //   O += P V          tcgen05.mma M=128 N=128 K=128, V read as an MN-major operand
-// With one chunk (rows <= 128 tokens, the common case) the row maximum comes
-// from the same S; with several, a first pass over the chunks finds the row
-// maximum so O can accumulate in TMEM without rescaling.  Queries, keys and
+// Across chunks the softmax is online: the running maximum and sum and the
+// output row live in the thread's registers, and each chunk's P V (fresh in
+// TMEM) is folded in after rescaling by exp(m_old - m_new).  Queries, keys and
 // values arrive by TMA straight into the 128-byte-swizzled layout (Qwen3 then
 // applies the per-head RMSNorm and the rotary positions in shared memory).
 // Keys past the row's end are masked to zero probability, so a query's result
@@ -258,43 +258,33 @@ __global__ void __launch_bounds__(128, 2)
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     };
 
-    float m = -FLT_MAX;
-    if (n_chunks > 1) {
-        for (int ch = 0; ch < n_chunks && ok; ++ch) {
-            load(ch, ch == 0, false);
-            s_mma();
-            for (int cc = 0; cc < 4; ++cc) {
-                float v[32];
-                tmem_ld32(t_s + lane_addr + cc * 32, v);
+    // single pass, online softmax: O and the running (max, sum) live in registers;
+    // each chunk's P.V lands fresh in TMEM and is folded in with the rescale factor
+    float m = -FLT_MAX, l = 0.f;
+    float o[HD];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int key = ch * TK + cc * 32 + j;
-                    if (key <= q && key < kend) m = fmaxf(m, v[j]);
-                }
-            }
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncthreads();
-        }
-    }
-    float l = 0.f;
+    for (int i = 0; i < HD; ++i) o[i] = 0.f;
     for (int ch = 0; ch < n_chunks && ok; ++ch) {
         const int c0 = ch * TK;
-        load(ch, ch == 0 && n_chunks == 1, true);
+        load(ch, ch == 0, true);
         if (!ok) break;
         s_mma();
         if (!ok) break;
-        if (n_chunks == 1) {
-            for (int cc = 0; cc < 4; ++cc) {
-                float v[32];
-                tmem_ld32(t_s + lane_addr + cc * 32, v);
+        float cmax = -FLT_MAX;
+        for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            tmem_ld32(t_s + lane_addr + cc * 32, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int key = cc * 32 + j;
-                    if (key <= q && key < kend) m = fmaxf(m, v[j]);
-                }
+            for (int j = 0; j < 32; ++j) {
+                const int key = c0 + cc * 32 + j;
+                if (key <= q && key < kend) cmax = fmaxf(cmax, v[j]);
             }
         }
-        const float ms = m * sl2;
+        const float m_new = fmaxf(m, cmax);
+        // rows whose every key so far is masked keep m = -FLT_MAX and contribute nothing
+        const float alpha = (m > -FLT_MAX) ? exp2f((m - m_new) * sl2) : 0.f;
+        const float ms = m_new * sl2;
+        float csum = 0.f;
         for (int cc = 0; cc < 4; ++cc) {
             float v[32];
             tmem_ld32(t_s + lane_addr + cc * 32, v);
@@ -306,7 +296,7 @@ __global__ void __launch_bounds__(128, 2)
                 for (int u = 0; u < 2; ++u) {
                     const int key = c0 + cc * 32 + j + u;
                     p2[u] = (key <= q && key < kend) ? exp2f(v[j + u] * sl2 - ms) : 0.f;
-                    l += p2[u];
+                    csum += p2[u];
                 }
                 w[j / 2] = pack_bf2(p2[0], p2[1]);
             }
@@ -315,6 +305,8 @@ __global__ void __launch_bounds__(128, 2)
                 *reinterpret_cast<uint4*>(KPb + sw_off(tid, cc * 4 + k4)) =
                     make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
         }
+        l = l * alpha + csum;
+        m = m_new;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
@@ -322,7 +314,7 @@ __global__ void __launch_bounds__(128, 2)
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t acc = (kk > 0 || ch > 0) ? 1u : 0u;
+                const uint32_t acc = kk > 0 ? 1u : 0u;
                 const uint64_t ad = sw128_desc(smem_u32(KPb) + (kk >> 2) * ATOM + (kk & 3) * 32);
                 const uint64_t bd = sw128_desc_mn(smem_u32(Vb) + kk * 2048);
                 asm volatile(
@@ -339,24 +331,27 @@ __global__ void __launch_bounds__(128, 2)
         ok = __syncthreads_and(ok && wait_bar(bar_mma, ph_mma, err));
         ph_mma ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    }
-    if (ok) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (size_t)(start + q) * a.ld_out +
-                              (size_t)h * HD;
+        if (!ok) break;
+#pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
             float v[32];
             tmem_ld32(t_o + lane_addr + cc * 32, v);
-            if (tid < nq) {
-                uint4* o4 = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4)
-                    o4[k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
-                                        pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
-                                        pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
-                                        pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
-            }
+            for (int j = 0; j < 32; ++j) o[cc * 32 + j] = o[cc * 32 + j] * alpha + v[j];
         }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();                       // S / O columns and the K, V buffers are reused
+    }
+    if (ok && tid < nq) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                             (size_t)(start + q) * a.ld_out + (size_t)h * HD);
+#pragma unroll
+        for (int k4 = 0; k4 < HD / 8; ++k4)
+            o4[k4] = make_uint4(pack_bf2(o[8 * k4] * inv, o[8 * k4 + 1] * inv),
+                                pack_bf2(o[8 * k4 + 2] * inv, o[8 * k4 + 3] * inv),
+                                pack_bf2(o[8 * k4 + 4] * inv, o[8 * k4 + 5] * inv),
+                                pack_bf2(o[8 * k4 + 6] * inv, o[8 * k4 + 7] * inv));
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();

@@ -268,6 +268,51 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, 
     }
 }
 
+// SwiGLU epilogue: the tile's columns 0..127 are gate features nb*128 + j and
+// columns 128..255 the matching up features; out[m, f] = silu(gate) * up.
+__device__ __forceinline__ void epilogue_swiglu(const TcParams& p, int m, int nb, uint32_t taddr) {
+    const int F = p.N >> 1;
+    for (int c = 0; c < 4; ++c) {
+        const int f0 = nb * 128 + c * 32;
+        if (f0 >= F) break;                         // warp-uniform
+        float gv[32], uv[32];
+        tmem_ld32(taddr + (uint32_t)(c * 32), gv);
+        tmem_ld32(taddr + (uint32_t)(128 + c * 32), uv);
+        if (m >= p.M) continue;
+        if (p.bias) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if (f0 + j < F) {
+                    gv[j] += p.bias[nb * 256 + c * 32 + j];
+                    uv[j] += p.bias[nb * 256 + 128 + c * 32 + j];
+                }
+            }
+        }
+        __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + (size_t)m * p.ldc + f0;
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] = gv[j] / (1.0f + expf(-gv[j])) * uv[j];
+        if (f0 + 32 <= F) {
+            uint4* c4 = reinterpret_cast<uint4*>(C);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(y[8 * q], y[8 * q + 1]);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(y[8 * q + 2], y[8 * q + 3]);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(y[8 * q + 4], y[8 * q + 5]);
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(y[8 * q + 6], y[8 * q + 7]);
+                uint4 w;
+                w.x = *reinterpret_cast<uint32_t*>(&h0);
+                w.y = *reinterpret_cast<uint32_t*>(&h1);
+                w.z = *reinterpret_cast<uint32_t*>(&h2);
+                w.w = *reinterpret_cast<uint32_t*>(&h3);
+                c4[q] = w;
+            }
+        } else {
+            for (int j = 0; j < 32 && f0 + j < F; ++j) C[j] = __float2bfloat16_rn(y[j]);
+        }
+    }
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -403,6 +448,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const int m = mb * BM + lane_base + lane;
             float run_max = -FLT_MAX, run_sum = 0.f;
+            if (EPI == EPI_SWIGLU)
+                epilogue_swiglu(p, m, nb, tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN));
+            else
             for (int c = 0; c < BN / 32; ++c) {
                 const int n = nb * BN + c * 32;
                 if (n >= p.N) break;                // whole chunk past N (warp-uniform)
@@ -644,6 +692,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const int m = mb * BM2 + (int)rank * 128 + lane_base + lane;
             float run_max = -FLT_MAX, run_sum = 0.f;
+            if (EPI == EPI_SWIGLU)
+                epilogue_swiglu(p, m, nb, tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN));
+            else
             for (int c = 0; c < BN / 32; ++c) {
                 const int n = nb * BN + c * 32;
                 if (n >= p.N) break;
@@ -790,6 +841,9 @@ bool gemm_tc_supported(const GemmArgs& g) {
         case EPI_SHRINK:
             if (g.c_type != E_BF16 || g.ldc % 8 || !aligned16(g.C)) return false;
             return true;
+        case EPI_SWIGLU:
+            if (g.c_type != E_BF16 || g.ldc % 8 || !aligned16(g.C) || g.N % 256) return false;
+            return true;
         default:
             return false;
     }
@@ -802,7 +856,8 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     // choice never depends on M (the batch): a row's bits must not change with
     // the company it is scored in.
     const bool pair = g_use_pairs && g.N > 128 &&
-                      (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID);
+                      (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
+                       g.epi == EPI_SWIGLU);
     const uint32_t b_rows = pair ? 128u : (uint32_t)BN;
     CUtensorMap a, b, a2, b2;
     if (!make_map(&a, g.A, g.M, g.K, g.lda, BM)) return 1;
@@ -844,6 +899,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
             case EPI_STORE: return launch_epi2<EPI_STORE>(a, b, a2, b2, p, st);
             case EPI_STORE_RELU: return launch_epi2<EPI_STORE_RELU>(a, b, a2, b2, p, st);
             case EPI_RESID: return launch_epi2<EPI_RESID>(a, b, a2, b2, p, st);
+            case EPI_SWIGLU: return launch_epi2<EPI_SWIGLU>(a, b, a2, b2, p, st);
             default: return 1;
         }
     }
@@ -853,6 +909,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
         case EPI_RESID: return launch_epi<EPI_RESID>(a, b, a2, b2, p, st);
         case EPI_LSE: return launch_epi<EPI_LSE>(a, b, a2, b2, p, st);
         case EPI_SHRINK: return launch_epi<EPI_SHRINK>(a, b, a2, b2, p, st);
+        case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(a, b, a2, b2, p, st);
         default: return 1;
     }
 }

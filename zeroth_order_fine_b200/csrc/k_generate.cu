@@ -100,7 +100,8 @@ __global__ void open_window_kernel(const WindowJob* jobs) {
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
         const int i = e / jb.r, c = e % jb.r;
         const float v = jb.V[e];
-        const size_t row = (size_t)(jb.row0 + i) * jb.ldb;
+        const int fr = jb.interleave ? (i / 128) * 256 + jb.row0 + i % 128 : jb.row0 + i;
+        const size_t row = (size_t)fr * jb.ldb;
         st_elem(jb.EB, row + jb.col_dir + c, jb.eb_type, v);
         st_elem(jb.EB, row + jb.col_slot + c, jb.eb_type, v);
     }

@@ -22,6 +22,7 @@ struct WindowJob {
     float* A;                   // new slot's A_k^T rows, r*d_in floats to zero
     void* A_bf;                 // optional bf16 mirror of those rows
     int eb_type, ldb, row0, d_out, d_in, r, col_dir, col_slot;
+    int interleave;             // 1: row i sits at (i / 128) * 256 + row0 + i % 128
 };
 
 void launch_init_tensor(void* dst, uint64_t n, uint64_t key, float std_, float mean, int dtype,
@@ -57,7 +58,9 @@ enum Epi : int {
     EPI_STORE_RELU = 1,  // C = relu(acc + bias)
     EPI_RESID = 2,       // C(fp32) += acc + bias
     EPI_SHRINK = 3,      // C = acc * (col < scale_cols ? sign[row] * eps : 1)
-    EPI_LSE = 4          // per (row, 64-col tile): max, sum exp(x - max); target logit
+    EPI_LSE = 4,         // per (row, 64-col tile): max, sum exp(x - max); target logit
+    EPI_SWIGLU = 5       // fused [gate|up] rows interleaved in 128-row blocks:
+                         // C[m, f] = silu(gate_f) * up_f, f = n_blk * 128 + j (tensor cores)
 };
 
 struct GemmArgs {
