@@ -328,3 +328,40 @@ def test_load_state_clears_slots_beyond_the_loaded_bank():
         Lp, Lm, _ = h.zo_score(toks, batch.seq_lens, batch.target_lens)
         outs.append((Lp.cpu().numpy(), Lm.cpu().numpy()))
     assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("dtype", [wl.DTYPE_FP32, wl.DTYPE_BF16])
+def test_edge_rows_match_oracle(dtype):
+    """The shortest rows (one prefix token), a row at the model's max_pos, a single
+    prompt, and a target span covering all but the first token."""
+    shape = wl.shrink_shape(wl.TINY, dtype=dtype)
+    w = dataclasses.replace(TINY, shape=shape, tgt_hi=8)      # room for 8-token spans
+    rng = np.random.default_rng(7)
+    rows = [rng.integers(0, shape.vocab, size=L).astype(np.int32) for L in (2, shape.max_pos, 9)]
+    tls = np.array([1, 3, 8], dtype=np.int32)
+    batch = wl.Batch(rows, tls, [], np.zeros(0, np.int32))
+    model, h = gpu_handle(w, batch=3)
+    orc = oracle_run(w)
+    tol = 1e-4 if dtype == wl.DTYPE_FP32 else 2e-2
+    for sub in ([0], [0, 1, 2]):
+        b = wl.Batch([rows[i] for i in sub], tls[sub], [], np.zeros(0, np.int32))
+        h.zo_probe_plan(0, w.eps)
+        orc.plan(0, w.eps)
+        Lp, Lm, lp = h.zo_score(dev_tokens(b), b.seq_lens, b.target_lens, want_logprob=True)
+        ref = orc.score(b.prompts, b.target_lens)
+        assert np.max(np.abs(Lp.cpu().numpy() - ref.L_plus)) <= tol
+        assert np.max(np.abs(Lm.cpu().numpy() - ref.L_minus)) <= tol
+        if dtype == wl.DTYPE_FP32:
+            assert np.max(np.abs(lp.cpu().numpy() - _cat(ref.logprob_plus + ref.logprob_minus))) <= 1e-4
+
+
+def test_rows_beyond_max_pos_rejected():
+    from zeroth_order_fine_b200 import zo
+    w = TINY
+    model, h = gpu_handle(w, batch=2)
+    row = np.zeros(w.shape.max_pos + 1, dtype=np.int32)
+    b = wl.Batch([row], np.array([1], np.int32), [], np.zeros(0, np.int32))
+    h.zo_probe_plan(0, w.eps)
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_score(dev_tokens(b), b.seq_lens, b.target_lens)
+    assert e.value.code == zo.ZO_ERR_ARG
