@@ -74,7 +74,7 @@ typedef struct zo_model_desc {
     int32_t head_dim;        /* 128 for the shapes the library is tuned for; <= 256         */
     int32_t d_ffn;
     int32_t vocab;
-    int32_t max_pos;         /* OPT: rows of pos_embed; rows longer than this are rejected  */
+    int32_t max_pos;         /* longest row: OPT rows of pos_embed, Qwen3 rotary table size */
     float   norm_eps;        /* LayerNorm (OPT) / RMSNorm (Qwen3) epsilon                   */
     float   rope_theta;      /* Qwen3 rotary base                                           */
     int32_t dtype;           /* ZO_DTYPE_*: matrices and embeddings                         */

@@ -108,6 +108,7 @@ struct zo_handle {
     std::vector<void*> owned;
     // activations
     float* resid = nullptr;
+    float *rope_cos = nullptr, *rope_sin = nullptr;   // Qwen3 rotary tables [max_pos x hd/2]
     void *xn = nullptr, *qkv = nullptr, *att = nullptr, *act = nullptr, *gu = nullptr;
     void* ext = nullptr;          // shrink output S (model dtype) [max_tokens x kcap]
     int kcap = 0;                 // columns of FT rows / EB / ext allocated
@@ -406,10 +407,11 @@ int check_desc(const zo_model_desc* d, const zo_weights* w, const zo_options* o)
     if (d->head_dim != 32 && d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256)
         return 2;
     if (d->d_model % 8 || d->d_ffn % 8 || (d->n_heads * d->head_dim) % 8) return 2;
+    if (d->arch == ZO_ARCH_QWEN3 && d->head_dim < 64) return 2;     // q/k norm + rotary kernel
     if (d->d_model > 12288) return 2;
     if (d->vocab <= 0 || d->d_ffn <= 0) return 1;
     if (d->dtype != ZO_DTYPE_FP32 && d->dtype != ZO_DTYPE_BF16) return 1;
-    if (d->arch == ZO_ARCH_OPT && (d->max_pos <= 0 || !w->pos_embed)) return 1;
+    if (d->max_pos <= 0 || (d->arch == ZO_ARCH_OPT && !w->pos_embed)) return 1;
     if (!w->tok_embed || !w->final_w || !w->layers) return 1;
     if (!d->tie_lm_head && !w->lm_head) return 1;
     if (o->lazy_interval < 1 || o->rank < 1 || o->rank > 256 || o->max_slots < 1) return 1;
@@ -582,6 +584,13 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         CRC(dev_alloc(h, &h->gu, (size_t)maxT * ffn_cols * es));
     if (h->kcap) CRC(dev_alloc(h, &h->ext, (size_t)maxT * h->kcap * es));
     CRC(dev_alloc(h, &h->hs, (size_t)maxS * d.d_model * es));
+    if (d.arch == ZO_ARCH_QWEN3) {
+        const size_t n = (size_t)d.max_pos * (d.head_dim / 2);
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->rope_cos), n * 4));
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->rope_sin), n * 4));
+        launch_rope_table(h->rope_cos, h->rope_sin, d.max_pos, d.head_dim, (double)d.rope_theta,
+                          h->st);
+    }
     h->lse_tiles = gemm_lse_col_tiles(d.vocab);
     CRC(dev_alloc(h, reinterpret_cast<void**>(&h->pmax), (size_t)maxS * h->lse_tiles * 4));
     CRC(dev_alloc(h, reinterpret_cast<void**>(&h->psum), (size_t)maxS * h->lse_tiles * 4));
@@ -765,7 +774,7 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
     soff[0] = 0;
     auto row_ok = [&](int L, int tl) {
         if (tl < 1 || L < tl + 1) return false;
-        if (d.arch == ZO_ARCH_OPT && L > d.max_pos) return false;
+        if (L > d.max_pos) return false;        // OPT positions / Qwen3 rotary table
         return L <= 65535 * 64;
     };
     std::vector<int> poff(B), toff(B);
@@ -823,7 +832,8 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
                         h->sc_tok, h->sc_tgt, tgt_ids, nullptr, chk_d, h->err_dev, h->st);
     // build_tokens, embed, per layer 2 norms + attention (+ SwiGLU), final norm, LSE merge
     h->stats.kernel_launches +=
-        2 + (uint64_t)d.n_layers * (3 + (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused)) + 2;
+        2 + (uint64_t)d.n_layers * (3 + (d.arch == ZO_ARCH_QWEN3) +
+                                    (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused)) + 2;
     launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
                  d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
                  d.d_model, h->st);
@@ -872,6 +882,10 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
                     h->dt, h->st);
         int rc = group_gemm(L.g[G_QKV], h->xn, EPI_STORE, h->qkv, h->n_qkv, h->dt);
         if (rc) return rc;
+        if (d.arch == ZO_ARCH_QWEN3)
+            launch_qk_norm_rope(h->qkv, h->n_qkv, h->dt, h->tok_pos, Ti, d.n_heads, d.n_kv_heads,
+                                d.head_dim, L.w.q_norm, L.w.k_norm, d.norm_eps, h->rope_cos,
+                                h->rope_sin, h->st);
         AttnArgs a;
         memset(&a, 0, sizeof(a));
         a.qkv = h->qkv; a.ld_qkv = h->n_qkv;
@@ -882,10 +896,6 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
         a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
         a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
         a.n_tokens = Ti;
-        if (d.arch == ZO_ARCH_QWEN3) {
-            a.q_norm = L.w.q_norm; a.k_norm = L.w.k_norm; a.norm_eps = d.norm_eps;
-            a.rope = 1; a.rope_theta = d.rope_theta;
-        }
         if (tc_attn && attention_tc_supported(a)) launch_attention_tc(a, h->st);
         else launch_attention(a, h->st);
         rc = group_gemm(L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32);

@@ -4,9 +4,7 @@
 // are streamed in 64-key chunks from key 0 up to the tile's causal limit with
 // an online softmax, so a query's result depends only on its own row (the
 // ragged batch is a layout, never a change of results).  Scores and the
-// softmax are fp32; q/k/v may be fp32 or bf16.  For Qwen3 the prologue applies
-// the per-head q/k RMSNorm and the rotary positions (rotate-half pairing)
-// while staging q and k.
+// softmax are fp32; q/k/v may be fp32 or bf16.
 #include <float.h>
 
 #include "common.cuh"
@@ -18,46 +16,14 @@ namespace {
 constexpr int QT = 64;   // queries per CTA
 constexpr int KC = 64;   // keys per chunk
 
-// Stage one q or k row of head h into dst (fp32), with optional RMSNorm +
-// rotary positions; executed by one warp.
+// Stage one q or k row of head h into dst (fp32), times mul; executed by one warp.
 template <int HD>
 __device__ __forceinline__ void stage_row(const void* src, size_t base, int dtype, float* dst,
-                                          float mul, const float* nw, float eps, int rope,
-                                          float theta, int pos) {
+                                          float mul) {
     const int lane = threadIdx.x & 31;
-    float v[HD / 32];
-    float ss = 0.f;
 #pragma unroll
-    for (int i = 0; i < HD / 32; ++i) {
-        v[i] = ld_elem(src, base + lane + 32 * i, dtype);
-        ss += v[i] * v[i];
-    }
-    if (nw) {
-        ss = warp_sum(ss);
-        const float r = 1.0f / sqrtf(ss / (float)HD + eps);
-#pragma unroll
-        for (int i = 0; i < HD / 32; ++i) v[i] = v[i] * r * nw[lane + 32 * i];
-    }
-#pragma unroll
-    for (int i = 0; i < HD / 32; ++i) dst[lane + 32 * i] = v[i];
+    for (int i = 0; i < HD / 32; ++i) dst[lane + 32 * i] = ld_elem(src, base + lane + 32 * i, dtype) * mul;
     __syncwarp();
-    if (rope) {
-        constexpr int half = HD / 2;
-        for (int p = lane; p < half; p += 32) {
-            const double inv = pow((double)theta, -2.0 * p / HD);
-            double sn, cs;
-            sincos((double)pos * inv, &sn, &cs);
-            const float x1 = dst[p], x2 = dst[p + half];
-            dst[p] = (float)(x1 * cs - x2 * sn);
-            dst[p + half] = (float)(x2 * cs + x1 * sn);
-        }
-        __syncwarp();
-    }
-    if (mul != 1.f) {
-#pragma unroll
-        for (int i = 0; i < HD / 32; ++i) dst[lane + 32 * i] *= mul;
-        __syncwarp();
-    }
 }
 
 template <int HD>
@@ -80,7 +46,7 @@ __global__ void __launch_bounds__(256) attention_kernel(AttnArgs a) {
 
     for (int i = warp; i < nq; i += 8)
         stage_row<HD>(a.qkv, (size_t)(start + q0 + i) * a.ld_qkv + (size_t)h * HD, a.dtype,
-                      Qs + i * HD, a.scale, a.q_norm, a.norm_eps, a.rope, a.rope_theta, q0 + i);
+                      Qs + i * HD, a.scale);
 
     constexpr int DPL = HD / 32;           // dims per lane in the PV product
     float m_i[8], l_i[8], o[8][DPL];
@@ -97,8 +63,7 @@ __global__ void __launch_bounds__(256) attention_kernel(AttnArgs a) {
         const int nk = min(KC, kend - c0);
         for (int j = warp; j < nk; j += 8) {
             const size_t tb = (size_t)(start + c0 + j) * a.ld_qkv;
-            stage_row<HD>(a.qkv, tb + q_dim + (size_t)kvh * HD, a.dtype, Ks + j * (HD + 1), 1.f,
-                          a.k_norm, a.norm_eps, a.rope, a.rope_theta, c0 + j);
+            stage_row<HD>(a.qkv, tb + q_dim + (size_t)kvh * HD, a.dtype, Ks + j * (HD + 1), 1.f);
 #pragma unroll
             for (int i = 0; i < HD / 32; ++i)
                 Vs[j * HD + lane + 32 * i] =

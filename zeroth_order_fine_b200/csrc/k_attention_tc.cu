@@ -10,8 +10,8 @@
 // Across chunks the softmax is online: the running maximum and sum and the
 // output row live in the thread's registers, and each chunk's P V (fresh in
 // TMEM) is folded in after rescaling by exp(m_old - m_new).  Queries, keys and
-// values arrive by TMA straight into the 128-byte-swizzled layout (Qwen3 then
-// applies the per-head RMSNorm and the rotary positions in shared memory).
+// values arrive by TMA straight into the 128-byte-swizzled layout (Qwen3's
+// q/k norm and rotary positions were applied to the q|k|v rows beforehand).
 // Keys past the row's end are masked to zero probability, so a query's result
 // depends only on its own row: packing never changes a bit.
 #include <cuda.h>
@@ -132,49 +132,6 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, ui
         : "memory");
 }
 
-// In place on a TMA-loaded [128 x 128] row tile: per-head RMSNorm and rotary
-// positions (rotate-half pairs (i, i + 64)); thread t owns row t.
-__device__ __forceinline__ void norm_rope_inplace(uint8_t* buf, int pos0, const float* nw, float eps,
-                                                  float theta) {
-    const int r = threadIdx.x;
-    float ss = 0.f;
-    for (int c = 0; c < 16; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(buf + sw_off(r, c));
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-        for (int j = 0; j < 4; ++j) {
-            const float2 f = __bfloat1622float2(h[j]);
-            ss += f.x * f.x + f.y * f.y;
-        }
-    }
-    const float rs = 1.0f / sqrtf(ss / (float)HD + eps);
-    for (int c = 0; c < 8; ++c) {
-        uint4 lo = *reinterpret_cast<const uint4*>(buf + sw_off(r, c));
-        uint4 hi = *reinterpret_cast<const uint4*>(buf + sw_off(r, c + 8));
-        __nv_bfloat162* hl = reinterpret_cast<__nv_bfloat162*>(&lo);
-        __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&hi);
-        for (int j = 0; j < 4; ++j) {
-            const float2 x1 = __bfloat1622float2(hl[j]);
-            const float2 x2 = __bfloat1622float2(hh[j]);
-            float o1[2], o2[2];
-            const float a1[2] = {x1.x, x1.y}, a2[2] = {x2.x, x2.y};
-            for (int u = 0; u < 2; ++u) {
-                const int i = 8 * c + 2 * j + u;
-                const float y1 = a1[u] * rs * nw[i];
-                const float y2 = a2[u] * rs * nw[i + 64];
-                const double inv = pow((double)theta, -2.0 * i / HD);
-                double sn, cs;
-                sincos((double)(pos0 + r) * inv, &sn, &cs);
-                o1[u] = (float)(y1 * cs - y2 * sn);
-                o2[u] = (float)(y2 * cs + y1 * sn);
-            }
-            hl[j] = __floats2bfloat162_rn(o1[0], o1[1]);
-            hh[j] = __floats2bfloat162_rn(o2[0], o2[1]);
-        }
-        *reinterpret_cast<uint4*>(buf + sw_off(r, c)) = lo;
-        *reinterpret_cast<uint4*>(buf + sw_off(r, c + 8)) = hi;
-    }
-}
-
 __global__ void __launch_bounds__(128, 2)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -243,10 +200,6 @@ __global__ void __launch_bounds__(128, 2)
         }
         ok = __syncthreads_and(ok && wait_bar(bar_ld, ph_ld, err));
         ph_ld ^= 1u;
-        if (a.rope) {
-            if (with_q) norm_rope_inplace(Qb, q0, a.q_norm, a.norm_eps, a.rope_theta);
-            norm_rope_inplace(KPb, ch * TK, a.k_norm, a.norm_eps, a.rope_theta);
-        }
     };
     auto s_mma = [&]() {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

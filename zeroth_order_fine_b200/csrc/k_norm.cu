@@ -213,6 +213,84 @@ __global__ void swiglu_kernel(const void* __restrict__ gu, int f, void* __restri
     }
 }
 
+// Rotary table: cos / sin of pos * theta^(-2i/hd) for i < hd/2, angles in double.
+__global__ void rope_table_kernel(float* cos_t, float* sin_t, int max_pos, int half, int hd,
+                                  double theta) {
+    const int n = max_pos * half;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+        const int pos = e / half, i = e % half;
+        const double ang = (double)pos * pow(theta, -2.0 * i / hd);
+        double sn, cs;
+        sincos(ang, &sn, &cs);
+        cos_t[e] = (float)cs;
+        sin_t[e] = (float)sn;
+    }
+}
+
+void launch_rope_table(float* cos_t, float* sin_t, int max_pos, int hd, double theta,
+                       cudaStream_t st) {
+    const int n = max_pos * (hd / 2);
+    unsigned b = cdiv(n, 256);
+    if (b > 148 * 8) b = 148 * 8;
+    rope_table_kernel<<<b, 256, 0, st>>>(cos_t, sin_t, max_pos, hd / 2, hd, theta);
+}
+
+// Qwen3 q/k per-head RMSNorm then rotary positions (rotate-half pairs (i, i + hd/2)),
+// in place on the q and k columns of the packed [T x ld] q|k|v rows.  One warp per
+// (token, head); the position is the token's index within its row.
+template <int HD>
+__global__ void qk_norm_rope_kernel(void* qkv, int ld, int dtype, const int* __restrict__ tok_pos,
+                                    int H, int Hkv, const float* __restrict__ qn,
+                                    const float* __restrict__ kn, float eps,
+                                    const float* __restrict__ cos_t,
+                                    const float* __restrict__ sin_t, int T) {
+    constexpr int PER = HD / 32, HALF = HD / 2;
+    const int warps = blockDim.x >> 5;
+    const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int heads = H + Hkv;
+    if (gw >= T * heads) return;
+    const int t = gw / heads, hh = gw % heads;
+    const float* nw = hh < H ? qn : kn;
+    const size_t base = (size_t)t * ld + (size_t)hh * HD;
+    // lane holds elements lane + 32 j: pairs (i, i + HD/2) sit in the same lane
+    float x[PER];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        x[j] = ld_elem(qkv, base + lane + 32 * j, dtype);
+        ss += x[j] * x[j];
+    }
+    ss = warp_sum(ss);
+    const float rs = 1.0f / sqrtf(ss / (float)HD + eps);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) x[j] = x[j] * rs * nw[lane + 32 * j];
+    const size_t rb = (size_t)tok_pos[t] * HALF;
+#pragma unroll
+    for (int j = 0; j < PER / 2; ++j) {
+        const int i = lane + 32 * j;                 // i < HD/2, partner at i + HD/2 = j + PER/2
+        const float c = cos_t[rb + i], sn = sin_t[rb + i];
+        const float a = x[j], b = x[j + PER / 2];
+        x[j] = a * c - b * sn;
+        x[j + PER / 2] = b * c + a * sn;
+    }
+#pragma unroll
+    for (int j = 0; j < PER; ++j) st_elem(qkv, base + lane + 32 * j, dtype, x[j]);
+}
+
+void launch_qk_norm_rope(void* qkv, int ld, int dtype, const int* tok_pos, int T, int H, int Hkv,
+                         int hd, const float* qn, const float* kn, float eps, const float* cos_t,
+                         const float* sin_t, cudaStream_t st) {
+    if (T == 0) return;
+    const unsigned blocks = cdiv((long long)T * (H + Hkv), 8);
+    switch (hd) {
+        case 64: qk_norm_rope_kernel<64><<<blocks, 256, 0, st>>>(qkv, ld, dtype, tok_pos, H, Hkv, qn, kn, eps, cos_t, sin_t, T); break;
+        case 128: qk_norm_rope_kernel<128><<<blocks, 256, 0, st>>>(qkv, ld, dtype, tok_pos, H, Hkv, qn, kn, eps, cos_t, sin_t, T); break;
+        case 256: qk_norm_rope_kernel<256><<<blocks, 256, 0, st>>>(qkv, ld, dtype, tok_pos, H, Hkv, qn, kn, eps, cos_t, sin_t, T); break;
+        default: break;
+    }
+}
+
 void launch_swiglu(const void* gu, int T, int f, void* out, int dtype, cudaStream_t st) {
     if (T == 0) return;
     swiglu_kernel<<<T, 256, 0, st>>>(gu, f, out, dtype);

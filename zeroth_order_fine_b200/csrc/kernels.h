@@ -51,6 +51,12 @@ void launch_embed(const int* tok_id, const int* tok_pos, const void* tok_embed,
 void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
                  const float* b, float eps, void* out, int out_type, cudaStream_t st);
 void launch_swiglu(const void* gu, int T, int f, void* out, int dtype, cudaStream_t st);
+void launch_rope_table(float* cos_t, float* sin_t, int max_pos, int hd, double theta,
+                       cudaStream_t st);
+// Qwen3: per-head RMSNorm of q and k, then rotary positions, in place in the q|k|v rows
+void launch_qk_norm_rope(void* qkv, int ld, int dtype, const int* tok_pos, int T, int H, int Hkv,
+                         int hd, const float* qn, const float* kn, float eps, const float* cos_t,
+                         const float* sin_t, cudaStream_t st);
 
 // ---- GEMM ----------------------------------------------------------------------------
 enum Epi : int {
@@ -98,10 +104,10 @@ struct AttnArgs {
     int n_tiles;
     int H, Hkv, hd;
     float scale;
-    // Qwen3: per-head RMSNorm of q, k and rotary positions
-    const float* q_norm; const float* k_norm; float norm_eps; float rope_theta; int rope;
     int n_tokens;                   // T: rows of qkv (the tensor-core kernel's TMA extent)
 };
+// (Qwen3's q/k RMSNorm and rotary positions are applied to the q|k|v rows before
+// attention by launch_qk_norm_rope; the attention kernels take q and k as they are.)
 void launch_attention(const AttnArgs& a, cudaStream_t st);          // CUDA cores, 64-query tiles
 bool attention_tc_supported(const AttnArgs& a);                     // bf16, head_dim 128
 void launch_attention_tc(const AttnArgs& a, cudaStream_t st);       // tensor cores, 128-query tiles
