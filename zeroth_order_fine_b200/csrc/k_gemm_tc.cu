@@ -15,7 +15,9 @@
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (M=128, N=BN, K=16 per instruction, kind::f16, fp32 accumulate)
 //   warps 2..5  epilogue: tcgen05.ld 32x32b from a double-buffered TMEM
-//               accumulator, fused bias / ReLU / residual add / LSE, stores
+//               accumulator, fused bias / ReLU / residual add / SwiGLU / LSE;
+//               the SM-pair kernel hands its tiles to TMA stores (reduce-add for
+//               the residual stream) through swizzled shared-memory staging
 // Tiles are walked in M-groups of 8 so concurrent CTAs share B strips in L2.
 // Every mbarrier wait is bounded: on expiry the kernel records
 // ZO_TC_TIMEOUT in the error word, drains what it issued and returns.
@@ -491,7 +493,9 @@ constexpr int BM2 = 256, STAGES2 = 6;
 constexpr int A2B = 128 * BK * 2;                // 16 KB of A per CTA per stage
 constexpr int B2B = 128 * BK * 2;                // 16 KB of B per CTA per stage
 constexpr int STAGE2_BYTES = A2B + B2B;
-constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 256;
+// epilogue staging: 4 warps x 2 buffers x 4 KB (32 rows x 128 bytes, 128-byte swizzle)
+constexpr int STG_BYTES = 4 * 2 * 4096;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + STG_BYTES + 1024 + 256;
 constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                              ((uint32_t)(BM2 >> 4) << 24);
 
@@ -540,6 +544,135 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                  : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// 16-byte chunk k (0..7) of staging row r (0..31): 128-byte rows, 128-byte swizzle
+__device__ __forceinline__ uint32_t stg_off(int r, int k) {
+    return (uint32_t)(r * 128 + ((k ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Pair-kernel epilogue: each warp stages its 32 rows x (32 fp32 | 64 bf16) columns in
+// shared memory and one lane hands them to the TMA unit -- a store, or for the
+// residual stream an fp32 reduce-add, so the SM never reads the residual.  Two
+// staging buffers per warp alternate; a buffer is rewritten only after the TMA
+// has read it.
+template <int EPI>
+__device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMap* tmC,
+                                             uint32_t stg, uint8_t* stg_ptr, int& buf, int m_base,
+                                             int nb, uint32_t taddr, int lane) {
+    const int r = lane;
+    auto stage_begin = [&]() {
+        if (lane == 0) bulk_wait_read1();
+        __syncwarp();
+    };
+    auto stage_end_store = [&](int x, bool reduce) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+            if (reduce) tma_reduce_add_2d(tmC, stg + buf * 4096, x, m_base);
+            else tma_store_2d(tmC, stg + buf * 4096, x, m_base);
+            bulk_commit();
+        }
+        buf ^= 1;
+    };
+    if (EPI == EPI_RESID) {
+        for (int c = 0; c < BN / 32; ++c) {
+            const int n = nb * BN + c * 32;
+            if (n >= p.N) break;
+            float v[32];
+            tmem_ld32(taddr + (uint32_t)(c * 32), v);
+            if (p.bias) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] += (n + j < p.N) ? __ldg(p.bias + n + j) : 0.f;
+            }
+            stage_begin();
+            uint8_t* b = stg_ptr + buf * 4096;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4*>(b + stg_off(r, k)) =
+                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            stage_end_store(n, true);
+        }
+    } else if (EPI == EPI_SWIGLU) {
+        const int F = p.N >> 1;
+        for (int c = 0; c < 4; c += 2) {
+            const int f0 = nb * 128 + c * 32;
+            if (f0 >= F) break;
+            float y[64];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float gv[32], uv[32];
+                tmem_ld32(taddr + (uint32_t)((c + h) * 32), gv);
+                tmem_ld32(taddr + (uint32_t)(128 + (c + h) * 32), uv);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    float g = gv[j], u = uv[j];
+                    if (p.bias) {
+                        g += __ldg(p.bias + nb * 256 + (c + h) * 32 + j);
+                        u += __ldg(p.bias + nb * 256 + 128 + (c + h) * 32 + j);
+                    }
+                    y[h * 32 + j] = g / (1.0f + expf(-g)) * u;
+                }
+            }
+            stage_begin();
+            uint8_t* b = stg_ptr + buf * 4096;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<uint4*>(b + stg_off(r, k)) =
+                    make_uint4(pack2_bf16(y[8 * k], y[8 * k + 1]), pack2_bf16(y[8 * k + 2], y[8 * k + 3]),
+                               pack2_bf16(y[8 * k + 4], y[8 * k + 5]), pack2_bf16(y[8 * k + 6], y[8 * k + 7]));
+            stage_end_store(f0, false);
+        }
+    } else {   // EPI_STORE, EPI_STORE_RELU: bf16, 64 columns per store
+        for (int c = 0; c < BN / 32; c += 2) {
+            const int n = nb * BN + c * 32;
+            if (n >= p.N) break;
+            float y[64];
+            tmem_ld32(taddr + (uint32_t)(c * 32), y);
+            tmem_ld32(taddr + (uint32_t)((c + 1) * 32), y + 32);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                float v = y[j];
+                if (p.bias) v += (n + j < p.N) ? __ldg(p.bias + n + j) : 0.f;
+                if (EPI == EPI_STORE_RELU) v = fmaxf(v, 0.f);
+                y[j] = v;
+            }
+            stage_begin();
+            uint8_t* b = stg_ptr + buf * 4096;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<uint4*>(b + stg_off(r, k)) =
+                    make_uint4(pack2_bf16(y[8 * k], y[8 * k + 1]), pack2_bf16(y[8 * k + 2], y[8 * k + 3]),
+                               pack2_bf16(y[8 * k + 4], y[8 * k + 5]), pack2_bf16(y[8 * k + 6], y[8 * k + 7]));
+            stage_end_store(n, false);
+        }
+    }
+}
+
 __device__ __forceinline__ void tile_coords2(int t, const TcParams& p, int* mb, int* nb) {
     const int per_group = p.group_m * p.n_n_blk;
     const int g = t / per_group;
@@ -554,19 +687,22 @@ template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2,
-                    const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
+                    const __grid_constant__ CUtensorMap tmB2,
+                    const __grid_constant__ CUtensorMap tmC, const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;     // same offset in both CTAs
     uint8_t* gbase = smem_raw + (base - raw);
-    const uint32_t bar0 = base + STAGES2 * STAGE2_BYTES;
+    const uint32_t stg0 = base + STAGES2 * STAGE2_BYTES;          // epilogue staging (1024-aligned)
+    const uint32_t bar0 = stg0 + STG_BYTES;
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (STAGES2 + s); };
     auto tfull = [&](int b) { return bar0 + 8u * (2 * STAGES2 + b); };
     auto tempty = [&](int b) { return bar0 + 8u * (2 * STAGES2 + 2 + b); };
     const uint32_t drain = bar0 + 8u * (2 * STAGES2 + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES2 * STAGE2_BYTES + 160);
-    volatile int* abort_f = reinterpret_cast<volatile int*>(gbase + STAGES2 * STAGE2_BYTES + 168);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES2 * STAGE2_BYTES + STG_BYTES + 160);
+    volatile int* abort_f =
+        reinterpret_cast<volatile int*>(gbase + STAGES2 * STAGE2_BYTES + STG_BYTES + 168);
 
     const uint32_t rank = cluster_rank();
     const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
@@ -683,6 +819,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int lane_base = 32 * (warp & 3);
         const uint32_t leader_tempty0 = map_rank(tempty(0), 0);
         const uint32_t leader_tempty1 = map_rank(tempty(1), 0);
+        const int ew = warp & 3;
+        const uint32_t stg = stg0 + (uint32_t)ew * 8192u;
+        uint8_t* stg_ptr = gbase + STAGES2 * STAGE2_BYTES + ew * 8192;
+        int buf = 0;
         int acc = 0;
         uint32_t aph = 0;
         for (int t = pair; t < p.n_tiles; t += n_pairs) {
@@ -690,23 +830,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tile_coords2(t, p, &mb, &nb);
             if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
             tc_fence_after();
-            const int m = mb * BM2 + (int)rank * 128 + lane_base + lane;
-            float run_max = -FLT_MAX, run_sum = 0.f;
-            if (EPI == EPI_SWIGLU)
-                epilogue_swiglu(p, m, nb, tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN));
-            else
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n = nb * BN + c * 32;
-                if (n >= p.N) break;
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN + c * 32), v);
-                epilogue_chunk<EPI>(p, m, n, v, &run_max, &run_sum);
-            }
+            const int m_base = mb * BM2 + (int)rank * 128 + lane_base;
+            epilogue_tma<EPI>(p, &tmC, stg, stg_ptr, buf, m_base, nb,
+                              tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN), lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0);
             if (++acc == 2) { acc = 0; aph ^= 1u; }
         }
+        if (lane == 0) bulk_wait_all();    // every store of this warp has landed
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -754,6 +887,24 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output map for the TMA-store epilogue: [rows x cols] with leading dimension ld,
+// bf16 boxes of 64 columns x 32 rows or fp32 boxes of 32 columns x 32 rows (128-byte
+// inner extent, 128-byte swizzle); boxes past the edges are clipped.
+bool make_map_out(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld,
+                  bool f32) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t esz = f32 ? 4 : 2;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * esz};
+    const cuuint32_t box[2] = {f32 ? 32u : 64u, 32u};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int num_sms() {
@@ -784,7 +935,7 @@ int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2
 
 template <int EPI>
 int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
+                const CUtensorMap& b2, const CUtensorMap& c, const TcParams& p, cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(gemm_tc2_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -811,7 +962,7 @@ int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a
     }
     int pairs = max_pairs;
     if (p.n_tiles < pairs) pairs = p.n_tiles;
-    gemm_tc2_kernel<EPI><<<2 * pairs, NUM_THREADS, SMEM2_BYTES, st>>>(a, b, a2, b2, p);
+    gemm_tc2_kernel<EPI><<<2 * pairs, NUM_THREADS, SMEM2_BYTES, st>>>(a, b, a2, b2, c, p);
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
 
@@ -895,11 +1046,16 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
     if (pair) {
+        // output map for the TMA-store epilogue: 32-row boxes, 128-byte inner extent
+        CUtensorMap c;
+        const bool f32 = g.epi == EPI_RESID;
+        const uint64_t cols = g.epi == EPI_SWIGLU ? (uint64_t)(g.N / 2) : (uint64_t)g.N;
+        if (!make_map_out(&c, g.C, (uint64_t)g.M, cols, (uint64_t)g.ldc, f32)) return 1;
         switch (g.epi) {
-            case EPI_STORE: return launch_epi2<EPI_STORE>(a, b, a2, b2, p, st);
-            case EPI_STORE_RELU: return launch_epi2<EPI_STORE_RELU>(a, b, a2, b2, p, st);
-            case EPI_RESID: return launch_epi2<EPI_RESID>(a, b, a2, b2, p, st);
-            case EPI_SWIGLU: return launch_epi2<EPI_SWIGLU>(a, b, a2, b2, p, st);
+            case EPI_STORE: return launch_epi2<EPI_STORE>(a, b, a2, b2, c, p, st);
+            case EPI_STORE_RELU: return launch_epi2<EPI_STORE_RELU>(a, b, a2, b2, c, p, st);
+            case EPI_RESID: return launch_epi2<EPI_RESID>(a, b, a2, b2, c, p, st);
+            case EPI_SWIGLU: return launch_epi2<EPI_SWIGLU>(a, b, a2, b2, c, p, st);
             default: return 1;
         }
     }
