@@ -20,7 +20,9 @@ def _bf16_ulp(x):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 64), (127, 320, 200), (129, 512, 512),
-                                   (300, 1000, 1024), (1000, 768, 5120), (257, 256, 8)])
+                                   (300, 1000, 1024), (1000, 768, 5120), (257, 256, 8),
+                                   (33, 40, 72), (130, 64, 320), (300, 104, 1000),
+                                   (65, 128, 2048)])
 @pytest.mark.parametrize("impl", [1, 2])
 def test_linear_store_bf16(M, N, K, impl):
     from zeroth_order_fine_b200 import zo
@@ -37,7 +39,8 @@ def test_linear_store_bf16(M, N, K, impl):
         assert torch.all(err <= _bf16_ulp(r) + 1e-4 * (K ** 0.5) * 0.05), err.max()
 
 
-@pytest.mark.parametrize("M,N,K", [(5, 256, 64), (200, 640, 520), (513, 5120, 2048)])
+@pytest.mark.parametrize("M,N,K", [(5, 256, 64), (200, 640, 520), (513, 5120, 2048),
+                                   (200, 96, 520), (77, 64, 136)])
 @pytest.mark.parametrize("impl", [1, 2])
 def test_linear_residual_accumulate(M, N, K, impl):
     from zeroth_order_fine_b200 import zo
@@ -110,6 +113,9 @@ def test_lm_head_logprob(S, V, d, dtype, impl):
     ([16, 128, 77, 3], 40, 40, 128, torch.bfloat16, 1),
     ([16, 128, 77, 3], 40, 40, 128, torch.bfloat16, 2),
     ([1, 129, 300, 256, 512], 4, 2, 128, torch.bfloat16, 2),
+    # several items per persistent CTA, 1-5 key chunks each, in mixed order
+    ([int(x) for x in np.random.default_rng(5).integers(1, 600, 40)], 8, 2, 128,
+     torch.bfloat16, 2),
     ([200, 1, 64], 8, 2, 64, torch.float32, 1)])
 def test_attention_matches_oracle(lens, H, Hkv, hd, dtype, impl):
     from oracle import model as om

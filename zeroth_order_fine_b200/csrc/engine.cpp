@@ -145,6 +145,7 @@ struct zo_handle {
     float mezo_scale = 1.f;
     bool use_tc = false;
     bool swiglu_fused = false;    // Qwen3 FFN-in GEMM writes silu(gate) * up directly
+    bool qknr_fused = false;      // Qwen3 q|k|v GEMM applies q/k RMSNorm and RoPE itself
     // stats
     zo_stats_t stats;
     PhaseTimer tm[3];
@@ -291,6 +292,8 @@ void prof_end(zo_handle* h, int slot, double flops, bool tc) {
 int run_gemm(zo_handle* h, const GemmArgs& g, double algo_flops) {
     const bool tc = h->use_tc && gemm_tc_supported(g);
     if (g.epi == EPI_SWIGLU && !tc) FAIL(h, ZO_ERR_UNSUPPORTED, "fused SwiGLU needs tensor cores");
+    if (g.epi == EPI_QKNR && !tc)
+        FAIL(h, ZO_ERR_UNSUPPORTED, "fused q/k norm and rotary positions need the SM-pair kernel");
     const int slot = prof_begin(h);
     if (tc) {
         int e = gemm_tc(g, h->st);
@@ -475,6 +478,15 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
 
     h->use_tc = h->dt == E_BF16 && options->impl == 0;
     h->swiglu_fused = h->use_tc && d.arch == ZO_ARCH_QWEN3 && d.d_ffn % 128 == 0;
+    // the q|k|v GEMM epilogue applies the q/k norm and rotary positions when it can read
+    // the norm weights as 16-byte vectors (head_dim 128, more than one head)
+    h->qknr_fused = h->use_tc && d.arch == ZO_ARCH_QWEN3 && d.head_dim == 128 &&
+                    h->n_qkv > 128;
+    for (int l = 0; l < d.n_layers && h->qknr_fused; ++l) {
+        const zo_layer_weights& lw = weights->layers[l];
+        if ((reinterpret_cast<uintptr_t>(lw.q_norm) & 15) || (reinterpret_cast<uintptr_t>(lw.k_norm) & 15))
+            h->qknr_fused = false;
+    }
     // layers, fused weights and bank buffers
     h->layers.resize(d.n_layers);
     int max_nt = 0;
@@ -811,6 +823,9 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
             }
         }
     }
+    // the persistent tensor-core kernel deals items out in order: longest (most key chunks) first
+    if (tc_attn)
+        std::stable_sort(tiles, tiles + nt, [](int x, int y) { return (x & 0xFFFF) > (y & 0xFFFF); });
     if (T > h->opt.max_tokens) FAIL(h, ZO_ERR_ARG, "more tokens than max_tokens");
     if (S > h->opt.max_scored) FAIL(h, ZO_ERR_ARG, "more scored positions than max_scored");
     if (R >= 32768) FAIL(h, ZO_ERR_ARG, "too many rows");
@@ -832,7 +847,7 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
                         h->sc_tok, h->sc_tgt, tgt_ids, nullptr, chk_d, h->err_dev, h->st);
     // build_tokens, embed, per layer 2 norms + attention (+ SwiGLU), final norm, LSE merge
     h->stats.kernel_launches +=
-        2 + (uint64_t)d.n_layers * (3 + (d.arch == ZO_ARCH_QWEN3) +
+        2 + (uint64_t)d.n_layers * (3 + (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused) +
                                     (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused)) + 2;
     launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
                  d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
@@ -840,9 +855,15 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
 
     const int r_ = h->opt.rank;
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
-    auto group_gemm = [&](Group& G, const void* X, int epi, void* C, int ldc, int ctype) -> int {
+    auto group_gemm = [&](Group& G, const void* X, int epi, void* C, int ldc, int ctype,
+                          const Layer* Lq = nullptr) -> int {
         GemmArgs g;
         memset(&g, 0, sizeof(g));
+        if (epi == EPI_QKNR) {
+            g.tok_pos = h->tok_pos; g.qn = Lq->w.q_norm; g.kn = Lq->w.k_norm;
+            g.rope_cos = h->rope_cos; g.rope_sin = h->rope_sin; g.norm_eps = d.norm_eps;
+            g.n_q_heads = d.n_heads; g.n_qk_heads = d.n_heads + d.n_kv_heads;
+        }
         g.M = Ti;
         if (G.n_t > 0) {
             // live extension columns, padded to a multiple of 8 (16-byte TMA rows); the
@@ -880,9 +901,10 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
         Layer& L = h->layers[l];
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps, h->xn,
                     h->dt, h->st);
-        int rc = group_gemm(L.g[G_QKV], h->xn, EPI_STORE, h->qkv, h->n_qkv, h->dt);
+        int rc = group_gemm(L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
+                            h->n_qkv, h->dt, &L);
         if (rc) return rc;
-        if (d.arch == ZO_ARCH_QWEN3)
+        if (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused)
             launch_qk_norm_rope(h->qkv, h->n_qkv, h->dt, h->tok_pos, Ti, d.n_heads, d.n_kv_heads,
                                 d.head_dim, L.w.q_norm, L.w.k_norm, d.norm_eps, h->rope_cos,
                                 h->rope_sin, h->st);

@@ -1,15 +1,15 @@
 // Packed variable-length causal attention on the 5th-generation tensor cores.
 //
-// One CTA (4 warps, 128 threads) takes one 128-query tile of one row for one
-// head; thread i owns query row i, which is also TMEM lane i.  Per 128-key
-// chunk of the row:
+// Work items are (128-query tile of one row, head) pairs, one CTA (4 warps,
+// 128 threads) each; thread i owns query row i of the tile, which is also TMEM
+// lane i.  Per 128-key chunk of the row:
 //   S  = Q K^T        tcgen05.mma M=128 N=128 K=128, fp32 accumulator in TMEM
 //   P  = exp(S*scale - m)  (causal and length masks) written as bf16 into the
 //                     K buffer, in the 128-byte-swizzled K-major layout
 //   O += P V          tcgen05.mma M=128 N=128 K=128, V read as an MN-major operand
-// Across chunks the softmax is online: the running maximum and sum and the
-// output row live in the thread's registers, and each chunk's P V (fresh in
-// TMEM) is folded in after rescaling by exp(m_old - m_new).  Queries, keys and
+// Across chunks the softmax is online: the running maximum and sum live in the
+// thread's registers, the output row in TMEM, rescaled by exp(m_old - m_new)
+// before each chunk's P V accumulates onto it.  Queries, keys and
 // values arrive by TMA straight into the 128-byte-swizzled layout (Qwen3's
 // q/k norm and rotary positions were applied to the q|k|v rows beforehand).
 // Keys past the row's end are masked to zero probability, so a query's result
@@ -65,6 +65,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
@@ -132,6 +150,33 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, ui
         : "memory");
 }
 
+// One (query tile, head) work item.
+struct Item {
+    int start, len, q0, nq, kend, n_chunks, h, kvh;
+};
+__device__ __forceinline__ Item get_item(const AttnArgs& a, int i) {
+    Item it;
+    const int tile = a.tiles[i / a.H];
+    const int row = tile >> 16, qt = tile & 0xFFFF;
+    it.h = i % a.H;
+    it.kvh = it.h / (a.H / a.Hkv);
+    it.start = a.cu_seqlens[row];
+    it.len = a.cu_seqlens[row + 1] - it.start;
+    it.q0 = qt * TQ;
+    it.nq = min(TQ, it.len - it.q0);
+    it.kend = min(it.len, it.q0 + TQ);
+    it.n_chunks = (it.kend + TK - 1) / TK;
+    return it;
+}
+
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// One CTA per item, two CTAs per SM: while one CTA waits on its TMA loads or
+// its MMAs, the other runs its softmax.  Items are dealt longest first.
 __global__ void __launch_bounds__(128, 2)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -145,16 +190,7 @@ __global__ void __launch_bounds__(128, 2)
     const uint32_t bar_ld = bar_mma + 8;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 3 * BUF + 16);
 
-    const int tile = a.tiles[blockIdx.x];
-    const int row = tile >> 16, qt = tile & 0xFFFF;
-    const int h = blockIdx.y;
-    const int kvh = h / (a.H / a.Hkv);
-    const int start = a.cu_seqlens[row];
-    const int len = a.cu_seqlens[row + 1] - start;
-    const int q0 = qt * TQ;
-    const int nq = min(TQ, len - q0);
-    const int kend = min(len, q0 + TQ);
-    const int n_chunks = (kend + TK - 1) / TK;
+    const Item it = get_item(a, blockIdx.x);
     const int q_dim = a.H * HD, kv_dim = a.Hkv * HD;
     const int tid = threadIdx.x, warp = tid >> 5;
     int* err = &g_attn_error;
@@ -179,87 +215,105 @@ __global__ void __launch_bounds__(128, 2)
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
     uint32_t ph_mma = 0, ph_ld = 0;
     bool ok = true;
-    const int q = q0 + tid;
+    const int q = it.q0 + tid;                         // this thread's query
     const float sl2 = a.scale * 1.4426950408889634f;
-    const int kcol = q_dim + kvh * HD, vcol = q_dim + kv_dim + kvh * HD;
+    const int kcol = q_dim + it.kvh * HD, vcol = q_dim + kv_dim + it.kvh * HD;
 
-    // one TMA round trip: (Q,) K (and V) of chunk ch; rows past the tensor read as zero
-    auto load = [&](int ch, bool with_q, bool with_v) {
+    float m = -FLT_MAX, l = 0.f;
+    for (int c = 0; c < it.n_chunks && ok; ++c) {
+        const int c0 = c * TK;
+        // K and V of chunk c (and Q with the first): rows past the tensor read as zero
         if (tid == 0) {
-            const uint32_t bytes = (uint32_t)BUF * (1 + (with_q ? 1 : 0) + (with_v ? 1 : 0));
+            const uint32_t bytes = (uint32_t)BUF * (c == 0 ? 3u : 2u);
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_ld),
                          "r"(bytes)
                          : "memory");
-            const int r0 = start + ch * TK;
+            const int r0 = it.start + c0;
             for (int half = 0; half < 2; ++half) {
-                if (with_q)
-                    tma_box(smem_u32(Qb) + half * ATOM, &tm, bar_ld, h * HD + half * 64, start + q0);
+                if (c == 0)
+                    tma_box(smem_u32(Qb) + half * ATOM, &tm, bar_ld, it.h * HD + half * 64,
+                            it.start + it.q0);
                 tma_box(smem_u32(KPb) + half * ATOM, &tm, bar_ld, kcol + half * 64, r0);
-                if (with_v) tma_box(smem_u32(Vb) + half * ATOM, &tm, bar_ld, vcol + half * 64, r0);
+                tma_box(smem_u32(Vb) + half * ATOM, &tm, bar_ld, vcol + half * 64, r0);
             }
         }
-        ok = __syncthreads_and(ok && wait_bar(bar_ld, ph_ld, err));
+        ok = __syncthreads_and(wait_bar(bar_ld, ph_ld, err));
         ph_ld ^= 1u;
-    };
-    auto s_mma = [&]() {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!ok) break;
+
+        // S = Q K^T
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
         if (tid == 0) mma_128(t_s, smem_u32(Qb), smem_u32(KPb), false, bar_mma);
-        ok = __syncthreads_and(ok && wait_bar(bar_mma, ph_mma, err));
+        ok = __syncthreads_and(wait_bar(bar_mma, ph_mma, err));
         ph_mma ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    };
+        if (!ok) break;
 
-    // single pass, online softmax: O and the running (max, sum) live in registers;
-    // each chunk's P.V lands fresh in TMEM and is folded in with the rescale factor
-    float m = -FLT_MAX, l = 0.f;
-    float o[HD];
-#pragma unroll
-    for (int i = 0; i < HD; ++i) o[i] = 0.f;
-    for (int ch = 0; ch < n_chunks && ok; ++ch) {
-        const int c0 = ch * TK;
-        load(ch, ch == 0, true);
-        if (!ok) break;
-        s_mma();
-        if (!ok) break;
+        // keys c0 + j with j < lim are visible to this query (causal and row end); column
+        // groups of 32 keys that no query of the warp sees are skipped, and so are warps
+        // whose queries all lie past the row's end (warp-uniform; their P rows are zero)
+        const int lim = min(q + 1, it.kend) - c0;
+        const int wlim = min(it.q0 + warp * 32 + 32, it.kend) - c0;
+        const bool warp_live = it.q0 + warp * 32 < it.len;
+        const int ncc = (!warp_live || wlim <= 0) ? 0 : min(4, (wlim + 31) >> 5);
+        float sv[4][32];
         float cmax = -FLT_MAX;
-        for (int cc = 0; cc < 4; ++cc) {
-            float v[32];
-            tmem_ld32(t_s + lane_addr + cc * 32, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int key = c0 + cc * 32 + j;
-                if (key <= q && key < kend) cmax = fmaxf(cmax, v[j]);
+        for (int cc = 0; cc < 4; ++cc) {
+            if (cc < ncc) {
+                tmem_ld32(t_s + lane_addr + cc * 32, sv[cc]);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    sv[cc][j] = (cc * 32 + j < lim) ? sv[cc][j] : -FLT_MAX;
+                    cmax = fmaxf(cmax, sv[cc][j]);
+                }
             }
         }
         const float m_new = fmaxf(m, cmax);
         // rows whose every key so far is masked keep m = -FLT_MAX and contribute nothing
         const float alpha = (m > -FLT_MAX) ? exp2f((m - m_new) * sl2) : 0.f;
-        const float ms = m_new * sl2;
-        float csum = 0.f;
+        // masked scores are -FLT_MAX, so exp2(s*sl2 - ms) underflows to exactly 0 for them
+        const float ms = (m_new > -FLT_MAX) ? m_new * sl2 : 0.f;
+        float cs0 = 0.f, cs1 = 0.f;
+#pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-            float v[32];
-            tmem_ld32(t_s + lane_addr + cc * 32, v);
             uint32_t w[16];
+            if (cc < ncc) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                float p2[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int key = c0 + cc * 32 + j + u;
-                    p2[u] = (key <= q && key < kend) ? exp2f(v[j + u] * sl2 - ms) : 0.f;
-                    csum += p2[u];
+                for (int j = 0; j < 32; j += 2) {
+                    const float p0 = ex2_ftz(fmaf(sv[cc][j], sl2, -ms));
+                    const float p1 = ex2_ftz(fmaf(sv[cc][j + 1], sl2, -ms));
+                    cs0 += p0;
+                    cs1 += p1;
+                    w[j / 2] = pack_bf2(p0, p1);
                 }
-                w[j / 2] = pack_bf2(p2[0], p2[1]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) w[j] = 0u;
             }
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
                 *reinterpret_cast<uint4*>(KPb + sw_off(tid, cc * 4 + k4)) =
                     make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
         }
-        l = l * alpha + csum;
+        l = l * alpha + (cs0 + cs1);
         m = m_new;
+        if (c > 0) {
+            // the running output stays in TMEM: rescale it by exp(m_old - m_new), then P V
+            // accumulates on top of it
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                float v[32];
+                tmem_ld32(t_o + lane_addr + cc * 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= alpha;
+                tmem_st32(t_o + lane_addr + cc * 32, v);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        }
+
+        // O (+)= P V
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
@@ -267,7 +321,7 @@ __global__ void __launch_bounds__(128, 2)
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t acc = kk > 0 ? 1u : 0u;
+                const uint32_t acc = (kk > 0 || c > 0) ? 1u : 0u;
                 const uint64_t ad = sw128_desc(smem_u32(KPb) + (kk >> 2) * ATOM + (kk & 3) * 32);
                 const uint64_t bd = sw128_desc_mn(smem_u32(Vb) + kk * 2048);
                 asm volatile(
@@ -281,30 +335,29 @@ __global__ void __launch_bounds__(128, 2)
                     bar_mma)
                 : "memory");
         }
-        ok = __syncthreads_and(ok && wait_bar(bar_mma, ph_mma, err));
+        ok = __syncthreads_and(wait_bar(bar_mma, ph_mma, err));
         ph_mma ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (!ok) break;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            float v[32];
-            tmem_ld32(t_o + lane_addr + cc * 32, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[cc * 32 + j] = o[cc * 32 + j] * alpha + v[j];
-        }
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();                       // S / O columns and the K, V buffers are reused
+        // the K/P and V buffers and the S columns are free again
     }
-    if (ok && tid < nq) {
+    if (ok) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
         uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
-                                             (size_t)(start + q) * a.ld_out + (size_t)h * HD);
+                                             (size_t)(it.start + q) * a.ld_out +
+                                             (size_t)it.h * HD);
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            tmem_ld32(t_o + lane_addr + cc * 32, v);          // warp-collective: every lane
+            if (tid < it.nq) {
 #pragma unroll
-        for (int k4 = 0; k4 < HD / 8; ++k4)
-            o4[k4] = make_uint4(pack_bf2(o[8 * k4] * inv, o[8 * k4 + 1] * inv),
-                                pack_bf2(o[8 * k4 + 2] * inv, o[8 * k4 + 3] * inv),
-                                pack_bf2(o[8 * k4 + 4] * inv, o[8 * k4 + 5] * inv),
-                                pack_bf2(o[8 * k4 + 6] * inv, o[8 * k4 + 7] * inv));
+                for (int k4 = 0; k4 < 4; ++k4)
+                    o4[cc * 4 + k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
+                                                 pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
+                                                 pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
+                                                 pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
+            }
+        }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -359,8 +412,9 @@ void launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return;
-    dim3 grid(a.n_tiles, a.H);
-    attention_tc_kernel<<<grid, 128, SMEM, st>>>(tm, a);
+    const long long items = (long long)a.n_tiles * a.H;
+    if (items > 0x7fffffffLL) return;
+    attention_tc_kernel<<<(unsigned)items, 128, SMEM, st>>>(tm, a);
 }
 
 int attention_tc_error_word() {

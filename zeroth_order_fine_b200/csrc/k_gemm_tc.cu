@@ -10,10 +10,10 @@
 // reach memory.
 //
 // Design (one CTA per SM, persistent):
-//   warp 0      TMA producer: 128x64 A and BNx64 B boxes, 128-byte swizzle,
-//               into a STAGES-deep shared-memory ring (mbarrier complete_tx)
+//   warp 0      TMA producer: 128x64 A and Nx64 B boxes, 128-byte swizzle,
+//               into a 192 KB shared-memory ring (mbarrier complete_tx)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//               (M=128, N=BN, K=16 per instruction, kind::f16, fp32 accumulate)
+//               (M=128, N=64/128/256, K=16 per instruction, kind::f16, fp32 accumulate)
 //   warps 2..5  epilogue: tcgen05.ld 32x32b from a double-buffered TMEM
 //               accumulator, fused bias / ReLU / residual add / SwiGLU / LSE;
 //               the SM-pair kernel hands its tiles to TMA stores (reduce-add for
@@ -33,16 +33,34 @@ namespace zo {
 
 namespace {
 
-constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
+constexpr int BM = 128, BK = 64, BN = 256;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
-constexpr int B_BYTES = BN * BK * 2;        // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 512;              // two BN-wide fp32 accumulators
 constexpr int GROUP_M = 8;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t WAIT_LIMIT = 1u << 24;   // drain polls (with back-off) after an abort
 constexpr long long WAIT_CYCLES = 4000000000ll;   // ~2 s at 2 GHz: a stage that never arrives
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+
+// Single-SM kernel geometry for an N tile of BNT columns (64, 128 or 256): the
+// ring holds 192 KB whatever the width, so narrow GEMMs (the bank shrink, whose
+// N is the handful of factor columns) keep as many bytes in flight per SM as the
+// wide ones and do not spend tensor-core time on columns that do not exist.
+template <int BNT>
+struct Tile1 {
+    static_assert(BNT == 64 || BNT == 128 || BNT == 256, "N tile");
+    static constexpr int B_BYTES = BNT * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // multiple of 1024
+    static constexpr int STAGES = (192 * 1024) / STAGE_BYTES;    // 8, 6, 4
+    static constexpr int TMEM_COLS = 2 * BNT;                    // double-buffered accumulator
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+    // bf16 x bf16 -> fp32, both K-major, M = 128, N = BNT
+    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                      ((uint32_t)(BNT >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    // barriers (8 B each: full, empty per stage; tfull, tempty per accumulator; drain)
+    // then the TMEM base and the abort flag, all inside the 256-byte tail
+    static constexpr int SLOT_OFF = 240, ABORT_OFF = 248;
+    static_assert(8 * (2 * STAGES + 5) <= SLOT_OFF, "barrier region");
+};
 
 __device__ int g_tc_error = 0;              // bit 0: a bounded wait expired
 bool g_use_pairs = true;                    // SM-pair kernel for large decoder GEMMs
@@ -56,6 +74,9 @@ struct TcParams {
     void* C; int ldc; int c_type;
     const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
     const int* row_sign; float eps; int scale_cols;
+    const int* tok_pos; const float* qn; const float* kn;
+    const float* rope_cos; const float* rope_sin; float norm_eps;
+    int n_q_heads, n_qk_heads;
     int* err;
 };
 
@@ -161,9 +182,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = BN.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
 
 __device__ __forceinline__ void tile_coords(int t, const TcParams& p, int* mb, int* nb) {
     const int per_group = GROUP_M * p.n_n_blk;
@@ -229,7 +247,9 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, 
                 c4[q] = c;
             }
         } else {
-            for (int j = 0; j < 32 && n + j < p.N; ++j) C[j] += v[j];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (n + j < p.N) C[j] += v[j];
         }
         return;
     }
@@ -262,11 +282,15 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, 
                 c4[q] = w;
             }
         } else {
-            for (int j = 0; j < 32 && n + j < p.N; ++j) C[j] = __float2bfloat16_rn(v[j]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (n + j < p.N) C[j] = __float2bfloat16_rn(v[j]);
         }
     } else {
         float* C = static_cast<float*>(p.C) + (size_t)m * p.ldc + n;
-        for (int j = 0; j < 32 && n + j < p.N; ++j) C[j] = v[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (n + j < p.N) C[j] = v[j];
     }
 }
 
@@ -310,16 +334,21 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, int m, int nb
                 c4[q] = w;
             }
         } else {
-            for (int j = 0; j < 32 && f0 + j < F; ++j) C[j] = __float2bfloat16_rn(y[j]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (f0 + j < F) C[j] = __float2bfloat16_rn(y[j]);
         }
     }
 }
 
-template <int EPI>
+template <int EPI, int BNT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                    const TcParams p) {
+    using T1 = Tile1<BNT>;
+    constexpr int STAGES = T1::STAGES;
+    constexpr int STAGE_BYTES = T1::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;           // 1024-aligned for SW128
@@ -331,8 +360,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto tfull = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
     auto tempty = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
     const uint32_t drain = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 128);
-    volatile int* abort_f = reinterpret_cast<volatile int*>(gbase + STAGES * STAGE_BYTES + 136);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + T1::SLOT_OFF);
+    volatile int* abort_f = reinterpret_cast<volatile int*>(gbase + STAGES * STAGE_BYTES + T1::ABORT_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -352,7 +381,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
-                     "r"(TMEM_COLS)
+                     "r"(T1::TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -367,9 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            int armed_s[STAGES];
-            uint32_t armed_ph[STAGES];
-            int n_armed = 0;
+            int n_armed = 0;                // loads issued; the i-th used stage i % S, phase (i / S) & 1
             bool ok = true;
             for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
                 int mb, nb;
@@ -381,14 +408,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     mbar_expect_tx(full(s), STAGE_BYTES);
                     if (kb < p.kb_main) {
                         tma_load_2d(sa, &tmA, full(s), kb * BK, mb * BM);
-                        tma_load_2d(sb, &tmB, full(s), kb * BK, nb * BN);
+                        tma_load_2d(sb, &tmB, full(s), kb * BK, nb * BNT);
                     } else {
                         const int k = (kb - p.kb_main) * BK;
                         tma_load_2d(sa, &tmA2, full(s), k, mb * BM);
-                        tma_load_2d(sb, &tmB2, full(s), k, nb * BN);
+                        tma_load_2d(sb, &tmB2, full(s), k, nb * BNT);
                     }
-                    armed_s[n_armed % STAGES] = s;
-                    armed_ph[n_armed % STAGES] = ph;
                     ++n_armed;
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
@@ -397,8 +422,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // drain: let every copy this thread issued land before the CTA exits
                 const int n = n_armed < STAGES ? n_armed : STAGES;
                 for (int i = 0; i < n; ++i) {
-                    const int j = (n_armed - 1 - i) % STAGES;
-                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(armed_s[j]), armed_ph[j]); ++it)
+                    const int a = n_armed - 1 - i;
+                    const uint32_t aph = (uint32_t)(a / STAGES) & 1u;
+                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(a % STAGES), aph); ++it)
                         __nanosleep(128);
                 }
             }
@@ -414,7 +440,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
                 if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)(acc * BN);
+                const uint32_t d = tmem + (uint32_t)(acc * BNT);
                 for (int kb = 0; kb < kb_total; ++kb) {
                     if (!mbar_wait(full(s), ph, abort_f, p.err)) { ok = false; break; }
                     tc_fence_after();
@@ -422,7 +448,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t sb = sa + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), kIdesc,
+                        tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
                                (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
@@ -451,13 +477,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int m = mb * BM + lane_base + lane;
             float run_max = -FLT_MAX, run_sum = 0.f;
             if (EPI == EPI_SWIGLU)
-                epilogue_swiglu(p, m, nb, tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN));
+                epilogue_swiglu(p, m, nb, tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BNT));
             else
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n = nb * BN + c * 32;
+            for (int c = 0; c < BNT / 32; ++c) {
+                const int n = nb * BNT + c * 32;
                 if (n >= p.N) break;                // whole chunk past N (warp-uniform)
                 float v[32];
-                tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN + c * 32), v);
+                tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BNT + c * 32), v);
                 epilogue_chunk<EPI>(p, m, n, v, &run_max, &run_sum);
             }
             if (EPI == EPI_LSE && m < p.M) {
@@ -476,7 +502,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     if (warp == 1) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(TMEM_COLS)
+                     "r"(T1::TMEM_COLS)
                      : "memory");
     }
 }
@@ -563,6 +589,9 @@ __device__ __forceinline__ void bulk_commit() {
 __device__ __forceinline__ void bulk_wait_read1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -646,6 +675,87 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
                     make_uint4(pack2_bf16(y[8 * k], y[8 * k + 1]), pack2_bf16(y[8 * k + 2], y[8 * k + 3]),
                                pack2_bf16(y[8 * k + 4], y[8 * k + 5]), pack2_bf16(y[8 * k + 6], y[8 * k + 7]));
             stage_end_store(f0, false);
+        }
+    } else if (EPI == EPI_QKNR) {
+        // one 128-column head at a time.  The accumulator is rounded to bf16 (the value the
+        // unfused path stores); q and k heads then get RMSNorm over the head and the rotary
+        // rotation of the pairs (i, i + 64) at the token's position.  Columns 32c.. and
+        // 64 + 32c.. are handled together, so a head goes out through both staging buffers.
+        const int m = m_base + r;
+        const int pos = m < p.M ? __ldg(p.tok_pos + m) : 0;
+        for (int hb = 0; hb < 2; ++hb) {
+            const int n0 = nb * BN + hb * 128;
+            if (n0 >= p.N) break;                  // warp-uniform
+            const int head = n0 >> 7;
+            const bool qk = head < p.n_qk_heads;
+            const uint32_t th = taddr + (uint32_t)(hb * 128);
+            float rs = 1.f;
+            if (qk) {
+                float ss = 0.f;
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(th + (uint32_t)(c * 32), v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float x = __bfloat162float(__float2bfloat16_rn(v[j]));
+                        ss += x * x;
+                    }
+                }
+                rs = 1.0f / sqrtf(ss / 128.0f + p.norm_eps);
+            }
+            const float* w = head < p.n_q_heads ? p.qn : p.kn;
+            if (lane == 0) bulk_wait_read0();      // both staging buffers free
+            __syncwarp();
+            for (int c = 0; c < 2; ++c) {
+                float lo[32], hi[32];
+                tmem_ld32(th + (uint32_t)(c * 32), lo);
+                tmem_ld32(th + (uint32_t)(64 + c * 32), hi);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    lo[j] = __bfloat162float(__float2bfloat16_rn(lo[j]));
+                    hi[j] = __bfloat162float(__float2bfloat16_rn(hi[j]));
+                }
+                if (qk) {
+                    const float4* wl = reinterpret_cast<const float4*>(w + 32 * c);
+                    const float4* wh = reinterpret_cast<const float4*>(w + 64 + 32 * c);
+                    const float4* c4 = reinterpret_cast<const float4*>(p.rope_cos + (size_t)pos * 64 + 32 * c);
+                    const float4* s4 = reinterpret_cast<const float4*>(p.rope_sin + (size_t)pos * 64 + 32 * c);
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 a4 = __ldg(wl + j4), b4 = __ldg(wh + j4);
+                        const float4 cv = __ldg(c4 + j4), sv = __ldg(s4 + j4);
+                        const float wa[4] = {a4.x, a4.y, a4.z, a4.w};
+                        const float wb[4] = {b4.x, b4.y, b4.z, b4.w};
+                        const float cs[4] = {cv.x, cv.y, cv.z, cv.w};
+                        const float sn[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 4 * j4 + e;
+                            const float a = lo[j] * rs * wa[e], b = hi[j] * rs * wb[e];
+                            lo[j] = a * cs[e] - b * sn[e];
+                            hi[j] = b * cs[e] + a * sn[e];
+                        }
+                    }
+                }
+                uint8_t* b0 = stg_ptr;
+                uint8_t* b1 = stg_ptr + 4096;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    *reinterpret_cast<uint4*>(b0 + stg_off(r, 4 * c + k)) =
+                        make_uint4(pack2_bf16(lo[8 * k], lo[8 * k + 1]), pack2_bf16(lo[8 * k + 2], lo[8 * k + 3]),
+                                   pack2_bf16(lo[8 * k + 4], lo[8 * k + 5]), pack2_bf16(lo[8 * k + 6], lo[8 * k + 7]));
+                    *reinterpret_cast<uint4*>(b1 + stg_off(r, 4 * c + k)) =
+                        make_uint4(pack2_bf16(hi[8 * k], hi[8 * k + 1]), pack2_bf16(hi[8 * k + 2], hi[8 * k + 3]),
+                                   pack2_bf16(hi[8 * k + 4], hi[8 * k + 5]), pack2_bf16(hi[8 * k + 6], hi[8 * k + 7]));
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(tmC, stg, n0, m_base);
+                tma_store_2d(tmC, stg + 4096, n0 + 64, m_base);
+                bulk_commit();
+            }
         }
     } else {   // EPI_STORE, EPI_STORE_RELU: bf16, 64 columns per store
         for (int c = 0; c < BN / 32; c += 2) {
@@ -739,9 +849,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            int armed_s[STAGES2];
-            uint32_t armed_ph[STAGES2];
-            int n_armed = 0;
+            int n_armed = 0;                // loads issued; the i-th used stage i % S, phase (i / S) & 1
             bool ok = true;
             for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
                 int mb, nb;
@@ -763,8 +871,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         tma_load_2d_pair(sa, &tmA2, lb, k, row_a);
                         tma_load_2d_pair(sb, &tmB2, lb, k, row_b);
                     }
-                    armed_s[n_armed % STAGES2] = s;
-                    armed_ph[n_armed % STAGES2] = ph;
                     ++n_armed;
                     if (++s == STAGES2) { s = 0; ph ^= 1u; }
                 }
@@ -772,8 +878,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (!ok && rank == 0) {
                 const int n = n_armed < STAGES2 ? n_armed : STAGES2;
                 for (int i = 0; i < n; ++i) {
-                    const int j = (n_armed - 1 - i) % STAGES2;
-                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(armed_s[j]), armed_ph[j]); ++it)
+                    const int a = n_armed - 1 - i;
+                    const uint32_t aph = (uint32_t)(a / STAGES2) & 1u;
+                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(a % STAGES2), aph); ++it)
                         __nanosleep(128);
                 }
             }
@@ -918,19 +1025,38 @@ int num_sms() {
     return n;
 }
 
-template <int EPI>
+template <int EPI, int BNT>
 int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
+    constexpr int smem = Tile1<BNT>::SMEM_BYTES;
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI, BNT>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return 1;
         attr = true;
     }
     const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
-    gemm_tc_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(a, b, a2, b2, p);
+    gemm_tc_kernel<EPI, BNT><<<grid, NUM_THREADS, smem, st>>>(a, b, a2, b2, p);
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+
+// N tile of the single-SM kernel: the narrowest of 64/128/256 that covers N, for
+// the epilogues that work column chunk by column chunk; the LSE partials and the
+// SwiGLU gate/up interleave are laid out in 256-column tiles.
+int tile1_width(const GemmArgs& g) {
+    if (g.epi == EPI_LSE || g.epi == EPI_SWIGLU) return BN;
+    return g.N <= 64 ? 64 : (g.N <= 128 ? 128 : 256);
+}
+
+template <int EPI>
+int launch_epi_w(int bnt, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                 const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
+    switch (bnt) {
+        case 64: return launch_epi<EPI, 64>(a, b, a2, b2, p, st);
+        case 128: return launch_epi<EPI, 128>(a, b, a2, b2, p, st);
+        default: return launch_epi<EPI, 256>(a, b, a2, b2, p, st);
+    }
 }
 
 template <int EPI>
@@ -995,6 +1121,15 @@ bool gemm_tc_supported(const GemmArgs& g) {
         case EPI_SWIGLU:
             if (g.c_type != E_BF16 || g.ldc % 8 || !aligned16(g.C) || g.N % 256) return false;
             return true;
+        case EPI_QKNR:
+            // SM-pair kernel only; head_dim 128, whole heads per 256-column tile
+            if (!g_use_pairs || g.N <= 128 || g.N % 128) return false;
+            if (g.c_type != E_BF16 || g.ldc % 8 || !aligned16(g.C) || g.bias) return false;
+            if (!g.tok_pos || !g.qn || !g.kn || !g.rope_cos || !g.rope_sin) return false;
+            if (!aligned16(g.qn) || !aligned16(g.kn) || !aligned16(g.rope_cos) ||
+                !aligned16(g.rope_sin))
+                return false;
+            return g.n_qk_heads * 128 <= g.N && g.n_q_heads <= g.n_qk_heads;
         default:
             return false;
     }
@@ -1008,8 +1143,10 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     // the company it is scored in.
     const bool pair = g_use_pairs && g.N > 128 &&
                       (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
-                       g.epi == EPI_SWIGLU);
-    const uint32_t b_rows = pair ? 128u : (uint32_t)BN;
+                       g.epi == EPI_SWIGLU || g.epi == EPI_QKNR);
+    if (g.epi == EPI_QKNR && !pair) return 1;
+    const int bnt = pair ? BN : tile1_width(g);
+    const uint32_t b_rows = pair ? 128u : (uint32_t)bnt;
     CUtensorMap a, b, a2, b2;
     if (!make_map(&a, g.A, g.M, g.K, g.lda, BM)) return 1;
     if (!make_map(&b, g.B, g.N, g.K, g.ldb, b_rows)) return 1;
@@ -1034,7 +1171,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
         gm = gm < 4 ? 4 : (gm > 32 ? 32 : gm);
         p.group_m = pair ? gm : GROUP_M;
     }
-    p.n_n_blk = (g.N + BN - 1) / BN;
+    p.n_n_blk = (g.N + bnt - 1) / bnt;
     p.n_tiles = p.n_m_blk * p.n_n_blk;
     p.epi = g.epi;
     p.bias = g.bias;
@@ -1042,6 +1179,9 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.targets = g.targets; p.part_max = g.part_max; p.part_sum = g.part_sum;
     p.tgt_logit = g.tgt_logit; p.n_col_tiles = g.n_col_tiles;
     p.row_sign = g.row_sign; p.eps = g.eps; p.scale_cols = g.scale_cols;
+    p.tok_pos = g.tok_pos; p.qn = g.qn; p.kn = g.kn;
+    p.rope_cos = g.rope_cos; p.rope_sin = g.rope_sin; p.norm_eps = g.norm_eps;
+    p.n_q_heads = g.n_q_heads; p.n_qk_heads = g.n_qk_heads;
     int* err = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
@@ -1056,16 +1196,17 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
             case EPI_STORE_RELU: return launch_epi2<EPI_STORE_RELU>(a, b, a2, b2, c, p, st);
             case EPI_RESID: return launch_epi2<EPI_RESID>(a, b, a2, b2, c, p, st);
             case EPI_SWIGLU: return launch_epi2<EPI_SWIGLU>(a, b, a2, b2, c, p, st);
+            case EPI_QKNR: return launch_epi2<EPI_QKNR>(a, b, a2, b2, c, p, st);
             default: return 1;
         }
     }
     switch (g.epi) {
-        case EPI_STORE: return launch_epi<EPI_STORE>(a, b, a2, b2, p, st);
-        case EPI_STORE_RELU: return launch_epi<EPI_STORE_RELU>(a, b, a2, b2, p, st);
-        case EPI_RESID: return launch_epi<EPI_RESID>(a, b, a2, b2, p, st);
-        case EPI_LSE: return launch_epi<EPI_LSE>(a, b, a2, b2, p, st);
-        case EPI_SHRINK: return launch_epi<EPI_SHRINK>(a, b, a2, b2, p, st);
-        case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(a, b, a2, b2, p, st);
+        case EPI_STORE: return launch_epi_w<EPI_STORE>(bnt, a, b, a2, b2, p, st);
+        case EPI_STORE_RELU: return launch_epi_w<EPI_STORE_RELU>(bnt, a, b, a2, b2, p, st);
+        case EPI_RESID: return launch_epi_w<EPI_RESID>(bnt, a, b, a2, b2, p, st);
+        case EPI_LSE: return launch_epi<EPI_LSE, BN>(a, b, a2, b2, p, st);
+        case EPI_SHRINK: return launch_epi_w<EPI_SHRINK>(bnt, a, b, a2, b2, p, st);
+        case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, BN>(a, b, a2, b2, p, st);
         default: return 1;
     }
 }

@@ -65,8 +65,11 @@ enum Epi : int {
     EPI_RESID = 2,       // C(fp32) += acc + bias
     EPI_SHRINK = 3,      // C = acc * (col < scale_cols ? sign[row] * eps : 1)
     EPI_LSE = 4,         // per (row, 64-col tile): max, sum exp(x - max); target logit
-    EPI_SWIGLU = 5       // fused [gate|up] rows interleaved in 128-row blocks:
+    EPI_SWIGLU = 5,      // fused [gate|up] rows interleaved in 128-row blocks:
                          // C[m, f] = silu(gate_f) * up_f, f = n_blk * 128 + j (tensor cores)
+    EPI_QKNR = 6         // Qwen3 q|k|v (bf16, head_dim 128, SM-pair tensor-core kernel only):
+                         // the q and k heads (head < n_qk_heads) get per-head RMSNorm and
+                         // rotary positions from the tables; v heads are stored as they are
 };
 
 struct GemmArgs {
@@ -83,6 +86,11 @@ struct GemmArgs {
     const int* row_sign; float eps; int scale_cols;
     // EPI_LSE
     const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
+    // EPI_QKNR: token positions [M], norm weights [128] of q and k, rotary tables
+    // [max_pos x 64]; heads below n_q_heads use qn, the next ones up to n_qk_heads kn
+    const int* tok_pos; const float* qn; const float* kn;
+    const float* rope_cos; const float* rope_sin; float norm_eps;
+    int n_q_heads, n_qk_heads;
 };
 
 void gemm_simt(const GemmArgs& g, cudaStream_t st);

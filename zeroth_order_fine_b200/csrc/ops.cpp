@@ -3,6 +3,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <algorithm>
 #include <vector>
 
 #include "../../include/zo.h"
@@ -116,6 +117,10 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
         meta[r + 1] = meta[r] + seq_lens[r];
         for (int q = 0; q < (seq_lens[r] + qtile - 1) / qtile; ++q) tiles.push_back((r << 16) | q);
     }
+    // the persistent tensor-core kernel deals items out in order: longest (most key chunks) first
+    if (tc)
+        std::stable_sort(tiles.begin(), tiles.end(),
+                         [](int x, int y) { return (x & 0xFFFF) > (y & 0xFFFF); });
     const size_t need = (meta.size() + tiles.size()) * 4;
     if (!workspace || workspace_bytes < need) return ZO_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
