@@ -314,6 +314,7 @@ def main():
     ap.add_argument("--ref-prompts", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the whole-step CUDA graph leg")
     ap.add_argument("--cuda-cores", action="store_true", help="GEMMs on CUDA cores only")
     ap.add_argument("--kernel", choices=["gemm", "attention", "lm_head"],
                     help="time one op alone (kernel microbenchmark, used for ncu captures)")
@@ -477,6 +478,28 @@ def main():
         h.zo_step(w.lr, want_c=False)
         step_no[0] += 1
 
+    # whole-step CUDA graph: the same probe steps, each one graph launch (zo_step_graph)
+    graph = None
+    if world == 1 and ftoks is None and not args.no_graph:
+        for _ in range(2):                              # capture (and a window, if one opens)
+            h.zo_step_graph(toks, batch.seq_lens, batch.target_lens, w.eps, w.lr)
+            step_no[0] += 1
+        torch.cuda.synchronize()
+        g_s = h.zo_stats()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            h.zo_step_graph(toks, batch.seq_lens, batch.target_lens, w.eps, w.lr)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        step_no[0] += args.steps
+        g_e = h.zo_stats()
+        g_ms = g0.elapsed_time(g1) / args.steps
+        graph = {"ms_per_step": g_ms, "scored_tokens_per_s": T / (g_ms / 1000.0),
+                 "eager_over_graph": ms / g_ms,
+                 "captures_in_timed_region": int(g_e["graph_captures"] - g_s["graph_captures"]),
+                 "replays_in_timed_region": int(g_e["graph_replays"] - g_s["graph_replays"])}
+
     # e2e: the same steps through the public API with host buffers (pinned), the
     # H2D copy of the step's tokens and the D2H read of c inside the timed region
     e2e = None
@@ -550,6 +573,7 @@ def main():
                                                                          "ms_step")},
         "matched_query_control": {"score_only_ms": control_ms, "step_over_control": ms / control_ms},
         "cobatch": cobatch,
+        "step_graph": graph,
         "gpu_launches": int(s1["kernel_launches"] - s0["kernel_launches"]),
         "e2e": e2e,
         "clocks": clocks,

@@ -155,6 +155,8 @@ typedef struct zo_stats_t {
     double   tc_gemm_flops;
     uint64_t cuda_core_gemm_launches;/* GEMMs that ran on CUDA cores (always counted): 0 for
                                        bf16 models unless options.impl asks for CUDA cores  */
+    uint64_t graph_captures;        /* zo_step_graph: step graphs captured                  */
+    uint64_t graph_replays;         /* zo_step_graph: step graph launches                   */
 } zo_stats_t;
 
 /* ---- lifecycle -------------------------------------------------------------------- */
@@ -221,6 +223,28 @@ int zo_score_foreground(zo_handle* h, const int32_t* fg_tokens, int32_t n_fg,
  * call synchronises, writes c (host double) and returns ZO_ERR_NONFINITE
  * (and the step counter does not advance). */
 int zo_step(zo_handle* h, float lr, double* c_out);
+
+/* One whole probe step -- zo_probe_plan at the handle's step counter, zo_score
+ * of n_prompts prompts (no target_ids check, no per-token output) and
+ * zo_step(lr, NULL) -- as a single CUDA graph launch on the handle's stream:
+ * the step's ~10 kernels per layer leave the host as one launch ("Zeroth-Order
+ * Fine-Tuning Was an Inference Workload All Along", section "Why ZO
+ * Fine-Tuning Is Really Scoring": the step is the pair of forward evaluations
+ * plus an update that is cheap, so nothing else should cost time).
+ *   packed_tokens  dev  int32 [sum(seq_lens)]; seq_lens, target_lens host int32
+ *   [n_prompts]; L_plus, L_minus dev float [n_prompts] or NULL.
+ * The graph is captured on first use and again whenever the batch layout
+ * (n_prompts, seq_lens, target_lens), eps, lr, the token or output pointers,
+ * or the bank's slot count changes; otherwise it is replayed, reading the
+ * current contents of packed_tokens.  A step that opens a lazy window does the
+ * window's host-side set-up eagerly first.  The direction draws and results
+ * are bit-identical to the eager calls.  Never synchronises: a non-finite c
+ * refuses the update on the device (bank unchanged) and the step counter
+ * advances, as zo_step with c_out == NULL.  ZO_ERR_STATE if a plan from
+ * zo_probe_plan is still open. */
+int zo_step_graph(zo_handle* h, const int32_t* packed_tokens, int32_t n_prompts,
+                  const int32_t* seq_lens, const int32_t* target_lens, float eps, float lr,
+                  float* L_plus, float* L_minus);
 
 /* Data-parallel split of zo_step: write {sum_i (L+_i - L-_i), n_prompts}
  * (dev double[2]) for this replica's prompts; after the caller has summed

@@ -365,3 +365,76 @@ def test_rows_beyond_max_pos_rejected():
     with pytest.raises(zo.ZoError) as e:
         h.zo_score(dev_tokens(b), b.seq_lens, b.target_lens)
     assert e.value.code == zo.ZO_ERR_ARG
+
+
+def _graph_workload(shape):
+    if shape == "tiny-bf16":
+        return TINY_BF16
+    return dataclasses.replace(QWEN_SMALL, shape=dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16),
+                               fg_rows=0)
+
+
+@pytest.mark.parametrize("shape", ["tiny-bf16", "qwen3-bf16"])
+def test_step_graph_is_bit_identical_to_eager_steps(shape):
+    """zo_step_graph replays one captured graph per window; L+/L- of every step and the
+    final bank equal those of plan/score/step called one by one, across window
+    boundaries (nu = 3) and with eager steps interleaved (the device step counter is
+    re-seeded)."""
+    w = _graph_workload(shape)
+    batch = wl.make_batch(w, fg_rows=0)
+    toks = dev_tokens(batch)
+    _, he = gpu_handle(w, nu=3)
+    _, hg = gpu_handle(w, nu=3)
+    eager, graphed = [], []
+    for t in range(8):
+        he.zo_probe_plan(t, w.eps)
+        Lp, Lm, _ = he.zo_score(toks, batch.seq_lens, batch.target_lens)
+        eager.append((Lp.cpu().numpy().copy(), Lm.cpu().numpy().copy()))
+        he.zo_step(w.lr, want_c=False)
+        if t == 5:                                   # an eager step in the middle
+            hg.zo_probe_plan(t, w.eps)
+            Lp, Lm, _ = hg.zo_score(toks, batch.seq_lens, batch.target_lens)
+            hg.zo_step(w.lr, want_c=False)
+        else:
+            Lp, Lm = hg.zo_step_graph(toks, batch.seq_lens, batch.target_lens, w.eps, w.lr)
+        graphed.append((Lp.cpu().numpy().copy(), Lm.cpu().numpy().copy()))
+    for (a, b), (c, d) in zip(eager, graphed):
+        assert np.array_equal(a, c) and np.array_equal(b, d)
+    assert he.zo_save_state() == hg.zo_save_state()
+    s = hg.zo_stats()
+    # windows open at steps 0, 3, 6: one capture each; the other graph steps replay
+    assert s["graph_captures"] == 3 and s["graph_replays"] == 7
+    assert s["steps"] == 8 and s["last_error_code"] == 0
+
+
+def test_step_graph_follows_new_token_contents():
+    """The graph reads the current contents of the token buffer: new prompts of the same
+    layout give the same L+/L- as the eager path on those prompts."""
+    w = TINY_BF16
+    b0 = wl.make_batch(w)
+    rng = np.random.default_rng(3)
+    b1 = wl.Batch([rng.integers(0, w.shape.vocab, len(p)).astype(np.int32) for p in b0.prompts],
+                  b0.target_lens, [], np.zeros(0, dtype=np.int32))
+    toks = dev_tokens(b0)
+    _, he = gpu_handle(w, nu=50)
+    _, hg = gpu_handle(w, nu=50)
+    for t, b in enumerate([b0, b1, b0]):
+        toks.copy_(torch.from_numpy(b.packed()).cuda())
+        he.zo_probe_plan(t, w.eps)
+        Lp, Lm, _ = he.zo_score(toks, b.seq_lens, b.target_lens)
+        he.zo_step(w.lr, want_c=False)
+        Gp, Gm = hg.zo_step_graph(toks, b.seq_lens, b.target_lens, w.eps, w.lr)
+        assert torch.equal(Lp, Gp) and torch.equal(Lm, Gm)
+    assert hg.zo_stats()["graph_captures"] == 1
+
+
+def test_step_graph_refuses_an_open_plan():
+    from zeroth_order_fine_b200 import zo
+    w = TINY_BF16
+    batch = wl.make_batch(w)
+    toks = dev_tokens(batch)
+    _, h = gpu_handle(w)
+    h.zo_probe_plan(0, w.eps)
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_step_graph(toks, batch.seq_lens, batch.target_lens, w.eps, w.lr)
+    assert e.value.code == zo.ZO_ERR_STATE

@@ -146,6 +146,24 @@ struct zo_handle {
     bool use_tc = false;
     bool swiglu_fused = false;    // Qwen3 FFN-in GEMM writes silu(gate) * up directly
     bool qknr_fused = false;      // Qwen3 q|k|v GEMM applies q/k RMSNorm and RoPE itself
+    // whole-step CUDA graph (zo_step_graph): captured for one batch layout, eps, lr,
+    // set of buffers and bank slot count; replayed while those stay the same
+    struct StepGraph {
+        cudaStream_t cap = nullptr;           // capture stream (the handle's may be the legacy one)
+        cudaGraphExec_t exec = nullptr;
+        int* meta = nullptr;                  // device metadata of the captured layout
+        uint64_t* step_dev = nullptr;         // the step the next replay generates U for
+        uint64_t step_next = ~0ull;           // value *step_dev holds once queued work has run
+        std::vector<int> lens, tls;
+        const void* tok = nullptr;
+        float *Lp = nullptr, *Lm = nullptr;
+        float eps = 0.f, lr = 0.f;
+        int slots = -1;
+        long long T = 0, S = 0;
+        uint64_t launches = 0;                // kernels per replay
+        uint64_t captures = 0, replays = 0;
+    } graph;
+    bool capturing = false;       // launches are being recorded into a graph
     // stats
     zo_stats_t stats;
     PhaseTimer tm[3];
@@ -271,7 +289,7 @@ void timer_end(zo_handle* h, int ph) {
 
 int prof_begin(zo_handle* h) {
     GemmProfiler& p = h->prof;
-    if (!p.on) return -1;
+    if (!p.on || h->capturing) return -1;
     if (p.head - p.tail >= GemmProfiler::kRing) prof_harvest(p, true);
     const int i = (int)(p.head % GemmProfiler::kRing);
     cudaEventRecord(p.a[i], h->st);
@@ -314,7 +332,7 @@ int open_window(zo_handle* h, uint64_t step) {
         FAIL(h, ZO_ERR_UNSUPPORTED, "bank full: more lazy windows than max_slots");
     const int r = h->opt.rank;
     // V of the window for every target
-    launch_gen_factors(h->genV_d, h->n_genV, h->maxV_pairs, h->opt.run_seed, step,
+    launch_gen_factors(h->genV_d, h->n_genV, h->maxV_pairs, h->opt.run_seed, step, nullptr,
                        (uint64_t)h->opt.lazy_interval, h->mezo_scale,
                        h->opt.targets.scale_mode == ZO_SCALE_MEZO, h->st);
     // staging: window jobs then update jobs
@@ -708,6 +726,8 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
 void zo_destroy(zo_handle* h) {
     if (!h) return;
     cudaStreamSynchronize(h->st);
+    if (h->graph.exec) cudaGraphExecDestroy(h->graph.exec);
+    if (h->graph.cap) cudaStreamDestroy(h->graph.cap);
     for (void* p : h->owned) cudaFree(p);
     if (h->meta_h) cudaFreeHost(h->meta_h);
     if (h->jobs_h) cudaFreeHost(h->jobs_h);
@@ -743,7 +763,7 @@ int zo_probe_plan(zo_handle* h, uint64_t step, int32_t rank, float eps, const zo
         int rc = open_window(h, step);
         if (rc) { timer_end(h, 0); return rc; }
     }
-    launch_gen_factors(h->genU_d, h->n_genU, h->maxU_pairs, h->opt.run_seed, step, nu,
+    launch_gen_factors(h->genU_d, h->n_genU, h->maxU_pairs, h->opt.run_seed, step, nullptr, nu,
                        h->mezo_scale, h->opt.targets.scale_mode == ZO_SCALE_MEZO, h->st);
     if (h->n_genU) h->stats.kernel_launches++;
     timer_end(h, 0);
@@ -761,19 +781,21 @@ int zo_probe_plan(zo_handle* h, uint64_t step, int32_t rank, float eps, const zo
 
 namespace {
 
-// The packed physical batch: + rows, - rows, then foreground rows.
-int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_t* lens,
-               const int32_t* tls, const int32_t* tgt_ids, const int32_t* ftok, int F,
-               const int32_t* flens, const int32_t* ftls) {
+// Host layout of one packed physical batch (+ rows, - rows, then foreground rows):
+// the metadata ints cu[R+1] src[R] fg[R] sign[R] soff[R+1] chk[R] tiles[nt] are
+// written to `host`; the kernels of a score read the same layout from device memory.
+struct BatchPlan {
+    int R = 0, B = 0, F = 0, nt = 0;
+    long long T = 0, S = 0;
+    size_t nints = 0;
+};
+
+int prepare_batch(zo_handle* h, int B, const int32_t* lens, const int32_t* tls,
+                  const int32_t* tgt_ids, int F, const int32_t* flens, const int32_t* ftls,
+                  int* host, BatchPlan* bp) {
     const zo_model_desc& d = h->desc;
-    if (B < 0 || F < 0 || (B > 0 && (!ptok || !lens || !tls)) || (F > 0 && (!ftok || !flens || !ftls)))
-        FAIL(h, ZO_ERR_ARG, "missing score arguments");
     const int R = 2 * B + F;
-    if (R == 0) FAIL(h, ZO_ERR_ARG, "empty batch");
-    if (R > h->opt.max_rows) FAIL(h, ZO_ERR_ARG, "more rows than max_rows");
-    // host metadata
-    CK(h, cudaEventSynchronize(h->meta_ev));
-    int* cu = h->meta_h;
+    int* cu = host;
     int* src = cu + (R + 1);
     int* isfg = src + R;
     int* sign = isfg + R;
@@ -823,16 +845,26 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
             }
         }
     }
-    // the persistent tensor-core kernel deals items out in order: longest (most key chunks) first
+    // attention CTAs are issued in item order: longest (most key chunks) first
     if (tc_attn)
         std::stable_sort(tiles, tiles + nt, [](int x, int y) { return (x & 0xFFFF) > (y & 0xFFFF); });
     if (T > h->opt.max_tokens) FAIL(h, ZO_ERR_ARG, "more tokens than max_tokens");
     if (S > h->opt.max_scored) FAIL(h, ZO_ERR_ARG, "more scored positions than max_scored");
     if (R >= 32768) FAIL(h, ZO_ERR_ARG, "too many rows");
-    const size_t nints = (size_t)(tiles - cu) + nt;
-    int* md = h->meta;
-    CK(h, cudaMemcpyAsync(md, cu, nints * 4, cudaMemcpyHostToDevice, h->st));
-    CK(h, cudaEventRecord(h->meta_ev, h->st));
+    bp->R = R; bp->B = B; bp->F = F; bp->nt = nt; bp->T = T; bp->S = S;
+    bp->nints = (size_t)(tiles - cu) + nt;
+    return ZO_OK;
+}
+
+// Every kernel of one score over a batch laid out by prepare_batch, whose metadata
+// is already in device memory at md.  Enqueues only (no host synchronisation), so
+// it can be captured into a CUDA graph.
+int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
+                 const int32_t* ptok, const int32_t* ftok, const int32_t* tgt_ids) {
+    const zo_model_desc& d = h->desc;
+    const int R = bp.R, nt = bp.nt;
+    const long long T = bp.T, S = bp.S;
+    const bool tc_attn = h->use_tc && h->dt == E_BF16 && d.head_dim == 128;
     RowMeta m;
     m.cu_seqlens = md;
     m.row_src = md + (R + 1);
@@ -967,6 +999,24 @@ int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_
     return ZO_OK;
 }
 
+int score_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_t* lens,
+               const int32_t* tls, const int32_t* tgt_ids, const int32_t* ftok, int F,
+               const int32_t* flens, const int32_t* ftls) {
+    if (B < 0 || F < 0 || (B > 0 && (!ptok || !lens || !tls)) || (F > 0 && (!ftok || !flens || !ftls)))
+        FAIL(h, ZO_ERR_ARG, "missing score arguments");
+    const int R = 2 * B + F;
+    if (R == 0) FAIL(h, ZO_ERR_ARG, "empty batch");
+    if (R > h->opt.max_rows) FAIL(h, ZO_ERR_ARG, "more rows than max_rows");
+    // the pinned staging buffer is reused once the previous score's copy has left it
+    CK(h, cudaEventSynchronize(h->meta_ev));
+    BatchPlan bp;
+    int rc = prepare_batch(h, B, lens, tls, tgt_ids, F, flens, ftls, h->meta_h, &bp);
+    if (rc) return rc;
+    CK(h, cudaMemcpyAsync(h->meta, h->meta_h, bp.nints * 4, cudaMemcpyHostToDevice, h->st));
+    CK(h, cudaEventRecord(h->meta_ev, h->st));
+    return launch_batch(h, eps, h->meta, bp, ptok, ftok, tgt_ids);
+}
+
 }  // namespace
 
 static int score_common(zo_plan* plan, zo_handle* h, const int32_t* ptok, int32_t B,
@@ -1082,6 +1132,119 @@ int zo_step(zo_handle* h, float lr, double* c_out) {
     return zo_step_from_sums(h, lr, h->sums, c_out);
 }
 
+int zo_step_graph(zo_handle* h, const int32_t* packed_tokens, int32_t n_prompts,
+                  const int32_t* seq_lens, const int32_t* target_lens, float eps, float lr,
+                  float* L_plus, float* L_minus) {
+    if (!h) return ZO_ERR_ARG;
+    if (!packed_tokens || !seq_lens || !target_lens || n_prompts < 1)
+        FAIL(h, ZO_ERR_ARG, "missing step arguments");
+    if (!std::isfinite(eps) || !std::isfinite(lr)) FAIL(h, ZO_ERR_ARG, "eps and lr must be finite");
+    if (h->have_plan) FAIL(h, ZO_ERR_STATE, "a plan is open: finish it with zo_step first");
+    const int B = n_prompts, R = 2 * B;
+    if (R > h->opt.max_rows) FAIL(h, ZO_ERR_ARG, "more rows than max_rows");
+    auto& G = h->graph;
+    const uint64_t step = h->step;
+    // a window boundary changes the bank's layout on the host: it runs eagerly, and the
+    // graph is captured again below for the new slot count
+    const uint64_t nu = (uint64_t)h->opt.lazy_interval;
+    const int64_t window = (int64_t)(step / nu);
+    if (h->n_genU && (h->n_slots == 0 || h->slot_window.back() != window)) {
+        int rc = open_window(h, step);
+        if (rc) return rc;
+    }
+    const bool same = G.exec && G.tok == packed_tokens && G.Lp == L_plus && G.Lm == L_minus &&
+                      G.eps == eps && G.lr == lr && G.slots == h->n_slots &&
+                      (int)G.lens.size() == B &&
+                      std::equal(G.lens.begin(), G.lens.end(), seq_lens) &&
+                      std::equal(G.tls.begin(), G.tls.end(), target_lens);
+    if (!same) {
+        if (G.exec) {
+            CK(h, cudaStreamSynchronize(h->st));
+            cudaGraphExecDestroy(G.exec);
+            G.exec = nullptr;
+        }
+        if (!G.cap) CK(h, cudaStreamCreateWithFlags(&G.cap, cudaStreamNonBlocking));
+        if (!G.meta) {
+            const int rc = dev_alloc(h, reinterpret_cast<void**>(&G.meta), h->meta_ints * 4);
+            if (rc) return rc;
+        }
+        if (!G.step_dev) {
+            const int rc = dev_alloc(h, reinterpret_cast<void**>(&G.step_dev), 8);
+            if (rc) return rc;
+        }
+        // the layout is fixed for the graph's life: its metadata goes to the device once
+        std::vector<int> host(h->meta_ints);
+        BatchPlan bp;
+        int rc = prepare_batch(h, B, seq_lens, target_lens, nullptr, 0, nullptr, nullptr,
+                               host.data(), &bp);
+        if (rc) return rc;
+        CK(h, cudaMemcpyAsync(G.meta, host.data(), bp.nints * 4, cudaMemcpyHostToDevice, h->st));
+        CK(h, cudaStreamSynchronize(h->st));
+        const zo_stats_t saved = h->stats;
+        cudaStream_t user_st = h->st;
+        cudaGraph_t graph = nullptr;
+        CK(h, cudaStreamBeginCapture(G.cap, cudaStreamCaptureModeRelaxed));
+        h->st = G.cap;
+        h->capturing = true;
+        const uint64_t k0 = h->stats.kernel_launches;
+        launch_gen_factors(h->genU_d, h->n_genU, h->maxU_pairs, h->opt.run_seed, 0, G.step_dev,
+                           nu, h->mezo_scale, h->opt.targets.scale_mode == ZO_SCALE_MEZO, h->st);
+        rc = launch_batch(h, eps, G.meta, bp, packed_tokens, nullptr, nullptr);
+        if (!rc) {
+            const int* soff_d = G.meta + (R + 1) + 3 * R;
+            launch_row_objective(h->logprob, soff_d, R, B, h->L_row, L_plus, L_minus, h->st);
+            launch_objective_sums(h->L_row, B, h->sums, h->st);
+            launch_estimate(h->sums, eps, h->c_dev, h->flag_dev, h->st);
+            launch_bank_update(h->upd_d, h->n_genU, h->max_upd, h->c_dev, h->flag_dev, lr, h->st);
+            launch_advance_step(G.step_dev, h->st);
+        }
+        const uint64_t launched = h->stats.kernel_launches - k0;
+        h->capturing = false;
+        h->st = user_st;
+        const cudaError_t ce = cudaStreamEndCapture(G.cap, &graph);
+        h->stats = saved;
+        if (rc) {
+            if (graph) cudaGraphDestroy(graph);
+            return rc;
+        }
+        if (ce != cudaSuccess || !graph) FAIL(h, ZO_ERR_CUDA, "step graph capture failed");
+        const cudaError_t ie = cudaGraphInstantiate(&G.exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (ie != cudaSuccess) {
+            G.exec = nullptr;
+            FAIL(h, ZO_ERR_CUDA, "step graph instantiation failed");
+        }
+        G.tok = packed_tokens; G.Lp = L_plus; G.Lm = L_minus; G.eps = eps; G.lr = lr;
+        G.slots = h->n_slots;
+        G.lens.assign(seq_lens, seq_lens + B);
+        G.tls.assign(target_lens, target_lens + B);
+        G.T = bp.T; G.S = bp.S;
+        // gen_factors, the score's kernels, objective, sums, estimate, update, step counter
+        G.launches = launched + (h->n_genU ? 1 : 0) + 4 + (h->n_genU > 0);
+        G.step_next = ~0ull;
+        G.captures++;
+    }
+    // the device step counter is re-seeded when eager steps or a reload moved the host's
+    if (G.step_next != step) {
+        launch_set_step(G.step_dev, step, h->st);
+        h->stats.kernel_launches++;
+    }
+    CK(h, cudaGraphLaunch(G.exec, h->st));
+    G.step_next = step + 1;
+    G.replays++;
+    h->stats.kernel_launches += G.launches;
+    h->stats.tokens_scored += (uint64_t)G.T;
+    h->stats.positions_scored += (uint64_t)G.S;
+    h->stats.score_calls++;
+    h->stats.state_transition_bytes += h->bytes_per_U + h->bytes_per_update;
+    h->stats.dense_ref_bytes += h->dense_bytes;
+    h->stats.dense_ref_bytes_targets += h->dense_bytes_targets;
+    h->stats.steps++;
+    h->step++;
+    CK(h, cudaGetLastError());
+    return ZO_OK;
+}
+
 int zo_stats(zo_handle* h, zo_stats_t* out) {
     if (!h || !out) return ZO_ERR_ARG;
     CK(h, cudaStreamSynchronize(h->st));
@@ -1105,6 +1268,8 @@ int zo_stats(zo_handle* h, zo_stats_t* out) {
     out->tc_gemm_launches = h->prof.tc_launches;
     out->tc_gemm_ms = h->prof.tc_ms;
     out->tc_gemm_flops = h->prof.tc_fl;
+    out->graph_captures = h->graph.captures;
+    out->graph_replays = h->graph.replays;
     return ZO_OK;
 }
 

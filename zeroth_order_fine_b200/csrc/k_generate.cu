@@ -55,10 +55,13 @@ void launch_init_tensor(void* dst, uint64_t n, uint64_t key, float std_, float m
 // reads) or dst[e] (V: row-major, kept for the window).
 __global__ void __launch_bounds__(256) gen_factors_kernel(const GenJob* jobs, int n_jobs,
                                                           uint64_t run_seed, uint64_t step,
+                                                          const uint64_t* step_dev,
                                                           uint64_t nu, float scale,
                                                           int apply_scale) {
     const GenJob jb = jobs[blockIdx.y];
-    const uint64_t key = factor_key(run_seed, step, nu, jb.layer, jb.matrix, jb.which);
+    // a captured step graph reads the step from device memory, an eager launch takes it by value
+    const uint64_t t = step_dev ? *step_dev : step;
+    const uint64_t key = factor_key(run_seed, t, nu, jb.layer, jb.matrix, jb.which);
     const uint64_t n = (uint64_t)jb.dim * jb.r;
     const uint64_t npairs = (n + 1) / 2;
     for (uint64_t j = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; j < npairs;
@@ -79,15 +82,27 @@ __global__ void __launch_bounds__(256) gen_factors_kernel(const GenJob* jobs, in
 }
 
 void launch_gen_factors(const GenJob* d_jobs, int n_jobs, int max_pairs, uint64_t run_seed,
-                        uint64_t step, uint64_t nu, float scale, int apply_scale,
-                        cudaStream_t st) {
+                        uint64_t step, const uint64_t* step_dev, uint64_t nu, float scale,
+                        int apply_scale, cudaStream_t st) {
     if (n_jobs == 0) return;
     unsigned bx = cdiv(max_pairs, 256);
     if (bx > 64) bx = 64;
     if (bx == 0) bx = 1;
     dim3 grid(bx, n_jobs);
-    gen_factors_kernel<<<grid, 256, 0, st>>>(d_jobs, n_jobs, run_seed, step, nu, scale,
+    gen_factors_kernel<<<grid, 256, 0, st>>>(d_jobs, n_jobs, run_seed, step, step_dev, nu, scale,
                                              apply_scale);
+}
+
+__global__ void set_step_kernel(uint64_t* step_dev, uint64_t v, int add) {
+    *step_dev = add ? *step_dev + v : v;
+}
+
+void launch_set_step(uint64_t* step_dev, uint64_t v, cudaStream_t st) {
+    set_step_kernel<<<1, 1, 0, st>>>(step_dev, v, 0);
+}
+
+void launch_advance_step(uint64_t* step_dev, cudaStream_t st) {
+    set_step_kernel<<<1, 1, 0, st>>>(step_dev, 1, 1);
 }
 
 // Window opening: write the new window's V (row-major [d_out x r], fp32) into

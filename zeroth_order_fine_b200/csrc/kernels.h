@@ -27,9 +27,12 @@ struct WindowJob {
 
 void launch_init_tensor(void* dst, uint64_t n, uint64_t key, float std_, float mean, int dtype,
                         cudaStream_t st);
+// step_dev (may be null): read the step from device memory instead of `step`
 void launch_gen_factors(const GenJob* d_jobs, int n_jobs, int max_pairs, uint64_t run_seed,
-                        uint64_t step, uint64_t nu, float scale, int apply_scale,
-                        cudaStream_t st);
+                        uint64_t step, const uint64_t* step_dev, uint64_t nu, float scale,
+                        int apply_scale, cudaStream_t st);
+void launch_set_step(uint64_t* step_dev, uint64_t v, cudaStream_t st);   // *step_dev = v
+void launch_advance_step(uint64_t* step_dev, cudaStream_t st);           // *step_dev += 1
 void launch_open_window(const WindowJob* d_jobs, int n_jobs, cudaStream_t st);
 
 // ---- token metadata / embeddings / norms -----------------------------------------------

@@ -117,7 +117,7 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
         meta[r + 1] = meta[r] + seq_lens[r];
         for (int q = 0; q < (seq_lens[r] + qtile - 1) / qtile; ++q) tiles.push_back((r << 16) | q);
     }
-    // the persistent tensor-core kernel deals items out in order: longest (most key chunks) first
+    // attention CTAs are issued in item order: longest (most key chunks) first
     if (tc)
         std::stable_sort(tiles.begin(), tiles.end(),
                          [](int x, int y) { return (x & 0xFFFF) > (y & 0xFFFF); });

@@ -79,7 +79,8 @@ class zo_stats_t(ctypes.Structure):
                 ("gemm_launches", c_uint64), ("gemm_ms", ctypes.c_double),
                 ("gemm_flops", ctypes.c_double), ("tc_gemm_launches", c_uint64),
                 ("tc_gemm_ms", ctypes.c_double), ("tc_gemm_flops", ctypes.c_double),
-                ("cuda_core_gemm_launches", c_uint64)]
+                ("cuda_core_gemm_launches", c_uint64), ("graph_captures", c_uint64),
+                ("graph_replays", c_uint64)]
 
 
 _I32P = ctypes.POINTER(c_int32)
@@ -101,6 +102,8 @@ _SIGS = {
                                    c_void_p, c_void_p]),
     "zo_score_foreground": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
     "zo_step": (c_int32, [c_void_p, ctypes.c_float, c_void_p]),
+    "zo_step_graph": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, ctypes.c_float,
+                                ctypes.c_float, c_void_p, c_void_p]),
     "zo_objective_sums": (c_int32, [c_void_p, c_void_p]),
     "zo_step_from_sums": (c_int32, [c_void_p, ctypes.c_float, c_void_p, c_void_p]),
     "zo_stats": (c_int32, [c_void_p, ctypes.POINTER(zo_stats_t)]),
@@ -351,6 +354,21 @@ class Handle:
         c = ctypes.c_double(0.0)
         _check(lib().zo_step(self.h, lr, ctypes.byref(c) if want_c else None), self.h)
         return c.value if want_c else None
+
+    # zo_step_graph: the library bakes the output pointers into its graph, so the
+    # handle keeps one pair of L+/L- buffers per batch size; the returned tensors are
+    # overwritten by the next step of the same size
+    def zo_step_graph(self, tokens, seq_lens, target_lens, eps: float, lr: float):
+        sl, tl = _i32(seq_lens), _i32(target_lens)
+        B = len(sl)
+        bufs = self.__dict__.setdefault("_graph_out", {})
+        if B not in bufs:
+            bufs[B] = (torch.empty(B, dtype=torch.float32, device=tokens.device),
+                       torch.empty(B, dtype=torch.float32, device=tokens.device))
+        Lp, Lm = bufs[B]
+        _check(lib().zo_step_graph(self.h, _ptr(tokens), B, _ptr(sl), _ptr(tl), eps, lr,
+                                   _ptr(Lp), _ptr(Lm)), self.h)
+        return Lp, Lm
 
     def zo_objective_sums(self, dev_sums: torch.Tensor) -> None:
         _check(lib().zo_objective_sums(self.h, _ptr(dev_sums)), self.h)
