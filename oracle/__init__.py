@@ -21,6 +21,9 @@ Parts and what pins them (see tests/test_oracle_*.py):
 * model      -- OPT and Qwen3 forwards checked against the HuggingFace
   ``transformers`` implementations of the same architectures (a library
   routine), causality and packing invariants.
+* fp8        -- the E4M3 cast against the format decoded bit by bit (all 256
+  codes; nearest value, ties to even, saturation), the per-row quantiser's
+  scale equivariance and error bound.
 * zo         -- the estimator against its closed form and an exact quadratic
   toy, its epsilon -> 0 limit against autograd, the factored perturbation
   against a dense brute force with W +/- eps*U V^T materialised, the bank

@@ -44,6 +44,7 @@ import numpy as np
 import torch
 
 from zeroth_order_fine_b200 import workload as wl
+from . import fp8 as fp8q
 from . import generator as gen
 
 f64 = torch.float64
@@ -129,14 +130,30 @@ class MatrixPerturbation:
 Perturb = Dict[Tuple[int, int], MatrixPerturbation]
 
 
+# Matrices whose base product runs in FP8 in the fp8 mode: the ones fed by a norm
+# (q, k, v and the FFN input projections), whose inputs have a per-token scale.
+FP8_MATRICES = (wl.MAT_Q, wl.MAT_K, wl.MAT_V, wl.MAT_GATE, wl.MAT_UP)
+
+
+def base_product(x: torch.Tensor, W: torch.Tensor, fp8: bool) -> torch.Tensor:
+    """x W^T; with fp8, of the per-row E4M3 quantised x and W (oracle/fp8.py)."""
+    if not fp8:
+        return x @ W.T
+    return (fp8q.dequant_rows(x.to(torch.float32).numpy()) @
+            fp8q.dequant_rows(W.to(torch.float32).numpy()).T)
+
+
 def perturbed_linear(x: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor],
                      pert: Optional[MatrixPerturbation], sign_eps: torch.Tensor,
-                     dense: bool) -> torch.Tensor:
-    """y = x (W^T + sum_j A_j V_j^T + s eps U V^T) + b, row-wise signs in sign_eps [T]."""
+                     dense: bool, fp8: bool = False) -> torch.Tensor:
+    """y = x (W^T + sum_j A_j V_j^T + s eps U V^T) + b, row-wise signs in sign_eps [T].
+
+    With fp8 the base term x W^T is taken between the E4M3-quantised x and W; the
+    bank and direction terms keep the exact x."""
     if pert is None:
-        y = x @ W.T
+        y = base_product(x, W, fp8)
     elif not dense:
-        y = x @ W.T
+        y = base_product(x, W, fp8)
         for A, Vj in pert.bank:
             y = y + (x @ A) @ Vj.T
         if pert.U is not None:
@@ -144,7 +161,7 @@ def perturbed_linear(x: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor]
     else:
         # brute force: one dense theta per distinct sign value
         y = torch.empty(x.shape[0], W.shape[0], dtype=f64)
-        base = W.T.clone()
+        base = torch.zeros_like(W.T) if fp8 else W.T.clone()
         for A, Vj in pert.bank:
             base = base + A @ Vj.T
         for se in torch.unique(sign_eps):
@@ -153,6 +170,8 @@ def perturbed_linear(x: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor]
                 theta = theta + se * (pert.U @ pert.V.T)
             rows = sign_eps == se
             y[rows] = x[rows] @ theta
+        if fp8:
+            y = y + base_product(x, W, True)
     if b is not None:
         y = y + b
     return y
@@ -196,8 +215,10 @@ def causal_attention(q, k, v, n_rep: int) -> torch.Tensor:
 
 def hidden_states(w: Weights, rows: Sequence[np.ndarray], signs: Sequence[float], eps,
                   perturb: Optional[Perturb], dense: bool = False,
-                  layer_ids: Optional[Sequence[int]] = None) -> torch.Tensor:
-    """Final-norm hidden states [T, d] of the concatenated rows (float64)."""
+                  layer_ids: Optional[Sequence[int]] = None, fp8: bool = False) -> torch.Tensor:
+    """Final-norm hidden states [T, d] of the concatenated rows (float64).
+
+    fp8: the base products of FP8_MATRICES use E4M3 inputs (oracle/fp8.py)."""
     sh = w.shape
     bf = sh.dtype == wl.DTYPE_BF16
     rnd = bf16_round if bf else (lambda t: t)
@@ -216,7 +237,8 @@ def hidden_states(w: Weights, rows: Sequence[np.ndarray], signs: Sequence[float]
     for li, p in zip(ids, w.layers):
         def lin(x, m):
             pm = perturb.get((li, m)) if perturb else None
-            return perturbed_linear(x, p[f"W{m}"], p.get(f"b{m}"), pm, sign_eps, dense)
+            return perturbed_linear(x, p[f"W{m}"], p.get(f"b{m}"), pm, sign_eps, dense,
+                                    fp8 and m in FP8_MATRICES)
 
         if sh.arch == wl.ARCH_OPT:
             x = rnd(layer_norm(h, p["ln1_w"], p["ln1_b"], sh.norm_eps))

@@ -64,8 +64,9 @@ class OracleRun:
 
     def __init__(self, weights: om.Weights, run_seed: int, nu: int, rank: int,
                  layers: Sequence[int], matrices: Sequence[int], scale_mode: int,
-                 start_step: int = 0):
+                 start_step: int = 0, fp8: bool = False):
         self.w = weights
+        self.fp8 = fp8                  # E4M3 base products of the norm-fed matrices
         self.sh = weights.shape
         self.run_seed = run_seed
         self.nu = nu
@@ -121,7 +122,7 @@ class OracleRun:
         signs = [1.0] * B + [-1.0] * B + [0.0] * len(fg_prompts)
         tls = list(target_lens) + list(target_lens) + list(fg_target_lens)
         hs = om.hidden_states(self.w, rows, signs, self.eps, self.perturbation(), dense,
-                              layer_ids=layer_ids)
+                              layer_ids=layer_ids, fp8=self.fp8)
         lps = om.token_logprobs(self.w, hs, rows, tls)
         Lp = np.array([row_objective(x) for x in lps[:B]])
         Lm = np.array([row_objective(x) for x in lps[B:2 * B]])
