@@ -100,6 +100,15 @@ def step_work(w: wl.Workload, batches, n_slots: int):
     return flops, bytes_, T_all, S_all
 
 
+def fp8_flops(w: wl.Workload, batches) -> float:
+    """The part of step_work's FLOPs that the fp8 option runs in E4M3: the base products of
+    q|k|v and the FFN input projections (the norm-fed matrices)."""
+    sh = w.shape
+    n_in = 2 * sh.d_ffn if sh.arch == wl.ARCH_QWEN3 else sh.d_ffn
+    per_tok = 2.0 * sh.d_model * (sh.q_dim + 2 * sh.kv_dim + n_in) * sh.n_layers
+    return per_tok * sum(b.n_tokens_physical for b in batches)
+
+
 # ---- clocks during the timed region -----------------------------------------------------
 
 class ClockSampler:
@@ -315,6 +324,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the whole-step CUDA graph leg")
+    ap.add_argument("--fp8", action="store_true",
+                    help="E4M3 base products for q|k|v and the FFN input (zo_options.fp8)")
     ap.add_argument("--cuda-cores", action="store_true", help="GEMMs on CUDA cores only")
     ap.add_argument("--kernel", choices=["gemm", "attention", "lm_head"],
                     help="time one op alone (kernel microbenchmark, used for ncu captures)")
@@ -358,7 +369,8 @@ def main():
     R = 2 * w.batch + len(batch.fg_prompts)
     slots = max(8, args.byte_run // w.nu + 2)
     h = zo.Handle(model, w.run_seed, w.nu, w.rank, tg, max_tokens=T, max_rows=R, max_scored=S,
-                  max_slots=slots, impl=1 if args.cuda_cores else 0, profile=0 if args.byte_run else 1)
+                  max_slots=slots, impl=1 if args.cuda_cores else 0, profile=0 if args.byte_run else 1,
+                  fp8=1 if args.fp8 else 0)
     toks = torch.from_numpy(batch.packed()).cuda()
     ftoks = torch.from_numpy(batch.fg_packed()).cuda() if batch.fg_prompts else None
     sums = torch.zeros(2, dtype=torch.float64, device="cuda")
@@ -533,11 +545,22 @@ def main():
     d_n = s1["tc_gemm_launches"] - s0["tc_gemm_launches"]
     gemm_tflops = d_fl / (d_ms / 1000.0) / 1e12 if d_ms > 0 else None
     peak_t = peaks["bf16_tflops_sustained"]
-    roof_t = max(flops / (peak_t * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    if args.fp8:
+        # E4M3 share at twice the measured bf16 rate (the nominal dense ratio), the rest at it
+        f8 = fp8_flops(w, [batch])
+        t_fl = (flops - f8) / (peak_t * 1e12) + f8 / (2 * peak_t * 1e12)
+    else:
+        t_fl = flops / (peak_t * 1e12)
+    roof_t = max(t_fl, bytes_ / (peaks["hbm_gbs"] * 1e9))
+    peak_g = peak_t
+    if args.fp8 and d_fl > 0:
+        f8g = fp8_flops(w, [batch]) * args.steps          # E4M3 FLOPs among the timed GEMMs
+        peak_g = d_fl / ((d_fl - f8g) / peak_t + f8g / (2 * peak_t))
     line = {
         "metric": METRIC, "value": tok_s, "unit": "scored tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 (q|k|v, FFN-in) + bf16" if args.fp8 else "bf16",
         "data": "synthetic (random-init weights drawn on the device, Zipf(1.1) ragged prompts)",
         "config": {"workload": w.name, "model": sh.name, "global_batch": w.batch * world,
                    "prompts_per_gpu": w.batch, "physical_rows_per_gpu": R,
@@ -546,22 +569,25 @@ def main():
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (weights %.1f GB read every step)" %
                          ((sh.body_params() + sh.vocab * sh.d_model) * 2 / 1e9),
-                   "gemm_impl": "cuda-cores" if args.cuda_cores else "tcgen05"},
+                   "gemm_impl": "cuda-cores" if args.cuda_cores else "tcgen05",
+                   "fp8": bool(args.fp8)},
         "steps_per_s": steps_s,
         "scored_tokens_per_s": tok_s,
         "target_tokens_per_s": world * S / (ms / 1000.0),
         "step_roofline": {"flops": flops_all, "bytes": bytes_ * world,
                           "roofline_ms": roof_t * 1000.0, "frac": roof_t * 1000.0 / ms,
-                          "peak": f"{peak_kind} bf16 {peak_t} TFLOP/s sustained, "
-                                  f"HBM {peaks['hbm_gbs']} GB/s"},
+                          "peak": f"{peak_kind} bf16 {peak_t} TFLOP/s sustained"
+                                  + (" (E4M3 share at 2x)" if args.fp8 else "")
+                                  + f", HBM {peaks['hbm_gbs']} GB/s"},
         "roofline": {"kernel": "tcgen05 GEMM (gemm_tc2_kernel SM pairs + gemm_tc_kernel; all epilogues)",
                      "bound": "tensor",
-                     "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": (gemm_tflops / peak_t) if gemm_tflops else None,
+                     "achieved": gemm_tflops, "peak": peak_g, "unit": "TFLOP/s",
+                     "frac": (gemm_tflops / peak_g) if gemm_tflops else None,
                      "traffic": gemm_traffic(), "launches_timed": d_n,
                      "algorithmic_flops_per_launch": d_fl / d_n if d_n else None,
                      "avg_launch_ms": d_ms / d_n if d_n else None,
-                     "peak_kind": f"{peak_kind} (sustained: the kernel runs inside a long step)",
+                     "peak_kind": f"{peak_kind} (sustained: the kernel runs inside a long step)"
+                                  + ("; E4M3 launches at 2x the bf16 figure" if args.fp8 else ""),
                      "share_of_step": (d_ms / args.steps) / ms if d_n else None},
         "state_transition": {"bytes_per_step": (s1["state_transition_bytes"] -
                                                 s0["state_transition_bytes"]) / args.steps,

@@ -129,6 +129,14 @@ typedef struct zo_options {
     void*      stream;       /* cudaStream_t; NULL = legacy default stream                  */
     int32_t    impl;         /* 0: tensor cores wherever they apply (bf16), 1: CUDA cores only */
     int32_t    profile;      /* 1: time every GEMM launch with CUDA events (zo_stats gemm_*) */
+    int32_t    fp8;          /* 1: the base products fed by a norm (q|k|v and the FFN input
+                                projections) run in E4M3 on the tensor cores ("Inference-Native
+                                Zeroth-Order Optimization", abstract: the queries inherit the
+                                runtime's quantisation): weights quantised once per output
+                                channel at zo_create, activations per token by the norm kernel
+                                (scale = amax / 448, round to nearest even, saturated).  The
+                                direction, bank and every other GEMM stay in the model dtype.
+                                bf16 models with impl 0 only, else ZO_ERR_UNSUPPORTED.  0: off */
 } zo_options;
 
 typedef struct zo_handle zo_handle;

@@ -20,6 +20,28 @@ extern "C" {
 enum { ZO_ACT_NONE = 0, ZO_ACT_RELU = 1 };
 enum { ZO_IMPL_AUTO = 0, ZO_IMPL_CUDA_CORES = 1, ZO_IMPL_TENSOR_CORES = 2 };
 
+/* E4M3 quantisation of the rows of x, the format zo_options.fp8 runs the
+ * norm-fed base GEMMs in ("Inference-Native Zeroth-Order Optimization",
+ * abstract: the queries inherit the runtime's quantisation):
+ * scale[r] = amax_r / 448 and q[r, :] = E4M3(x[r, :] * (448 / amax_r)),
+ * both quotients and the product rounded to nearest in fp32, the cast
+ * round-to-nearest-even and saturated at +-448; an all-zero row has scale 1.
+ *   x     dev [rows x cols] dtype (fp32 or bf16), row-major
+ *   q     dev uint8 [rows x cols] E4M3 codes;  scale dev float [rows]
+ * ZO_ERR_ARG on NULL pointers or negative sizes.  Asynchronous on stream. */
+int zo_op_quantize_rows_e4m3(const void* x, int32_t dtype, int32_t rows, int32_t cols,
+                             uint8_t* q, float* scale, void* stream);
+
+/* The E4M3 base GEMM: y = act((q_x * s_x) (q_W * s_W)^T + b) on the SM-pair
+ * tcgen05 kernel (kind::f8f6f4, fp32 accumulate, dequantised in the
+ * epilogue), the form zo_options.fp8 uses for q|k|v and the FFN input.
+ *   xq dev uint8 [M x K], sx dev float [M]; wq dev uint8 [N x K], sw dev float [N]
+ *   bias dev float [N] or NULL;  y dev bf16 [M x N];  act ZO_ACT_*
+ * Needs K % 16 == 0 and N > 128 (the SM-pair tile), else ZO_ERR_UNSUPPORTED. */
+int zo_op_linear_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                     const float* bias, void* y, int32_t M, int32_t N, int32_t K, int32_t act,
+                     void* stream);
+
 /* One decoder linear layer, y = act(x W^T + b) (the frozen base weights W of
  * "Inference-Native Zeroth-Order Optimization", abstract; the GEMM is the
  * batched forward that dominates the step, "Zeroth-Order Fine-Tuning Was an

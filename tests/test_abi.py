@@ -44,8 +44,38 @@ def test_struct_sizes_match_header(built_lib):
     from zeroth_order_fine_b200 import zo
     assert ctypes.sizeof(zo.zo_model_desc) == 13 * 4
     assert ctypes.sizeof(zo.zo_targets) == 24
-    assert zo.zo_options.stream.offset == 64 and ctypes.sizeof(zo.zo_options) == 80
+    assert zo.zo_options.stream.offset == 64 and ctypes.sizeof(zo.zo_options) == 88
     assert ctypes.sizeof(zo.zo_layer_weights) == 20 * 8
+
+
+def test_struct_layouts_match_the_c_compiler(tmp_path):
+    """sizeof/offsetof of every ABI struct from gcc on include/zo.h equal the ctypes mirrors."""
+    import os
+    import shutil
+    import subprocess
+    from zeroth_order_fine_b200 import zo
+    if not shutil.which("gcc"):
+        pytest.skip("gcc not available")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    structs = {"zo_model_desc": zo.zo_model_desc, "zo_layer_weights": zo.zo_layer_weights,
+               "zo_weights": zo.zo_weights, "zo_targets": zo.zo_targets,
+               "zo_options": zo.zo_options, "zo_stats_t": zo.zo_stats_t}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zo.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'printf("{name} %zu\\n", sizeof({name}));')
+        for f, _ in cls._fields_:
+            lines.append(f'printf("{name}.{f} %zu\\n", offsetof({name}, {f}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = dict(l.rsplit(" ", 1) for l in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                        check=True).stdout.splitlines())
+    for name, cls in structs.items():
+        assert int(got[name]) == ctypes.sizeof(cls), name
+        for f, _ in cls._fields_:
+            assert int(got[f"{name}.{f}"]) == getattr(cls, f).offset, f"{name}.{f}"
 
 
 def test_library_refuses_bad_create_without_gpu(built_lib):

@@ -76,12 +76,12 @@ def test_qwen3_mezo_fp32_matches_oracle():
         assert abs(c - c_ref) <= 1e-2 * max(abs(c_ref), 1.0)
 
 
-def _bf16_same_state_parity(w, shape, batch, pre_steps):
+def _bf16_same_state_parity(w, shape, batch, pre_steps, fp8=False):
     """L+- of the GPU and the oracle on the same state: step 0, then after the
     oracle's own pre_steps updates, its bank loaded into the library."""
     from gpu_util import oracle_state_blob
-    model, h = gpu_handle(w, shape=shape, batch=len(batch.prompts))
-    orc = oracle_run(w, shape=shape)
+    model, h = gpu_handle(w, shape=shape, batch=len(batch.prompts), fp8=int(fp8))
+    orc = oracle_run(w, shape=shape, fp8=fp8)
     toks = dev_tokens(batch)
     errs = []
     h.zo_probe_plan(0, w.eps)

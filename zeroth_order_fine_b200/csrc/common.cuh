@@ -48,6 +48,17 @@ __device__ __forceinline__ float block_sum(float v, float* red /* >= 32 floats *
     return warp_sum(s);
 }
 
+// Block-wide max, same contract as block_sum.
+__device__ __forceinline__ float block_max(float v, float* red /* >= 32 floats */) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_max(v);
+    __syncthreads();
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    float s = lane < nw ? red[lane] : -3.0e38f;
+    return warp_max(s);
+}
+
 inline unsigned cdiv(long long a, long long b) { return (unsigned)((a + b - 1) / b); }
 
 }  // namespace zo

@@ -55,6 +55,8 @@ struct Group {
     void* FTb = nullptr;         // bf16 mirror of FT (bf16 models): the shrink GEMM operand
     void* EB = nullptr;          // expand factors (model dtype)
     float* Vcur[kMaxTargetsPerGroup] = {nullptr, nullptr, nullptr};
+    uint8_t* Wq = nullptr;       // E4M3 copy of W (fp8 option, norm-fed groups)
+    float* sw = nullptr;         // its per-row (output channel) scales
 };
 
 struct Layer {
@@ -146,6 +148,9 @@ struct zo_handle {
     bool use_tc = false;
     bool swiglu_fused = false;    // Qwen3 FFN-in GEMM writes silu(gate) * up directly
     bool qknr_fused = false;      // Qwen3 q|k|v GEMM applies q/k RMSNorm and RoPE itself
+    bool fp8 = false;             // norm-fed base GEMMs in E4M3 (zo_options.fp8)
+    uint8_t* xq = nullptr;        // E4M3 rows of the norm output
+    float* sx = nullptr;          // their per-token scales
     // whole-step CUDA graph (zo_step_graph): captured for one batch layout, eps, lr,
     // set of buffers and bank slot count; replayed while those stay the same
     struct StepGraph {
@@ -358,6 +363,7 @@ int open_window(zo_handle* h, uint64_t step) {
                 w.col_dir = t * r;
                 w.col_slot = G.n_t * r * (1 + k) + t * r;
                 w.interleave = G.interleave;
+                w.row_div = G.sw;               // E4M3 groups: V / s_w per expand row
                 wj[nw++] = w;
                 UpdateJob u;
                 u.A = w.A;
@@ -441,6 +447,11 @@ int check_desc(const zo_model_desc* d, const zo_weights* w, const zo_options* o)
     if (o->targets.matrix_mask & ~0x7Fu) return 1;
     if (o->impl != 0 && o->impl != 1) return 1;
     if (o->profile != 0 && o->profile != 1) return 1;
+    if (o->fp8 != 0 && o->fp8 != 1) return 1;
+    if (o->fp8 && (d->dtype != ZO_DTYPE_BF16 || o->impl != 0 || !norm_fp8_supported(d->d_model) ||
+                   d->d_model % 16 || (d->n_heads + 2 * d->n_kv_heads) * d->head_dim <= 128 ||
+                   d->d_ffn <= 64))
+        return 2;
     if (d->arch == ZO_ARCH_OPT && (o->targets.matrix_mask & (1u << ZO_MAT_GATE))) return 1;
     return 0;
 }
@@ -495,6 +506,7 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
     } while (0)
 
     h->use_tc = h->dt == E_BF16 && options->impl == 0;
+    h->fp8 = options->fp8 == 1;
     h->swiglu_fused = h->use_tc && d.arch == ZO_ARCH_QWEN3 && d.d_ffn % 128 == 0;
     // the q|k|v GEMM epilogue applies the q/k norm and rotary positions when it can read
     // the norm weights as 16-byte vectors (head_dim 128, more than one head)
@@ -578,6 +590,19 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
             h->err = "missing LayerNorm shift";
             return fail(ZO_ERR_ARG);
         }
+        if (h->fp8) {
+            // E4M3 copies of the norm-fed matrices, one scale per output channel
+            for (int gi : {(int)G_QKV, (int)G_IN}) {
+                Group& G = L.g[gi];
+                void* p = nullptr;
+                CRC(dev_alloc(h, &p, (size_t)G.N * G.K));
+                G.Wq = static_cast<uint8_t*>(p);
+                CRC(dev_alloc(h, &p, (size_t)G.N * 4));
+                G.sw = static_cast<float*>(p);
+                launch_quant_rows_e4m3(G.W, E_BF16, G.N, G.K, (size_t)G.K, G.Wq, (size_t)G.K, G.sw,
+                                       h->st);
+            }
+        }
         for (auto& G : L.g) {
             if (G.n_t == 0) continue;
             if (G.K % 4) { h->err = "d_in must be a multiple of 4"; return fail(ZO_ERR_UNSUPPORTED); }
@@ -607,6 +632,10 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
     const int ffn_cols = d.arch == ZO_ARCH_QWEN3 ? 2 * d.d_ffn : d.d_ffn;
     CRC(dev_alloc(h, reinterpret_cast<void**>(&h->resid), (size_t)maxT * d.d_model * 4));
     CRC(dev_alloc(h, &h->xn, (size_t)maxT * d.d_model * es));
+    if (h->fp8) {
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->xq), (size_t)maxT * d.d_model));
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->sx), (size_t)maxT * 4));
+    }
     CRC(dev_alloc(h, &h->qkv, (size_t)maxT * h->n_qkv * es));
     CRC(dev_alloc(h, &h->att, (size_t)maxT * h->q_dim * es));
     CRC(dev_alloc(h, &h->act, (size_t)maxT * d.d_ffn * es));
@@ -911,6 +940,7 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
             s.epi = EPI_SHRINK;
             s.C = h->ext; s.ldc = h->kcap; s.c_type = h->dt;
             s.row_sign = h->tok_sign; s.eps = eps; s.scale_cols = G.n_t * r_;
+            if (G.Wq) s.a_scale = h->sx;      // S / s_x: the base GEMM accumulates in E4M3 units
             int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
             if (rc) return rc;
             g.A2 = h->ext; g.lda2 = h->kcap; g.a2_type = h->dt;
@@ -919,6 +949,12 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
         }
         g.A = X; g.lda = G.K; g.a_type = h->dt;
         g.B = G.W; g.ldb = G.K; g.b_type = h->dt;
+        if (G.Wq) {
+            // E4M3 rows of the same norm output and of W; dequantised in the epilogue
+            g.A = h->xq; g.a_type = E_FP8;
+            g.B = G.Wq; g.b_type = E_FP8;
+            g.a_scale = h->sx; g.b_scale = G.sw;
+        }
         g.N = G.N; g.K = G.K;
         g.bias = G.bias;
         g.epi = epi;
@@ -932,7 +968,7 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
     for (int l = 0; l < d.n_layers; ++l) {
         Layer& L = h->layers[l];
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps, h->xn,
-                    h->dt, h->st);
+                    h->dt, h->st, h->xq, h->sx);
         int rc = group_gemm(L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
                             h->n_qkv, h->dt, &L);
         if (rc) return rc;
@@ -955,7 +991,7 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
         rc = group_gemm(L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32);
         if (rc) return rc;
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps, h->xn,
-                    h->dt, h->st);
+                    h->dt, h->st, h->xq, h->sx);
         if (d.arch == ZO_ARCH_OPT) {
             rc = group_gemm(L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt);
         } else if (h->swiglu_fused) {

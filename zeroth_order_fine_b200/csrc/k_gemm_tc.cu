@@ -77,6 +77,8 @@ struct TcParams {
     const int* tok_pos; const float* qn; const float* kn;
     const float* rope_cos; const float* rope_sin; float norm_eps;
     int n_q_heads, n_qk_heads;
+    int fp8;                                // main K blocks are E4M3 (SM-pair kernel)
+    const float* a_scale; const float* b_scale;
     int* err;
 };
 
@@ -263,6 +265,12 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, 
 #pragma unroll
         for (int j = 0; j < 32; ++j)
             if (n + j < p.scale_cols) v[j] *= rs;
+    }
+    if (EPI == EPI_SHRINK && p.a_scale) {
+        // the group's base GEMM runs in E4M3: its accumulator is in units of 1 / a_scale[m]
+        const float sa = __ldg(p.a_scale + m);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = v[j] / sa;
     }
     if (p.c_type == E_BF16) {
         __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + (size_t)m * p.ldc + n;
@@ -524,6 +532,11 @@ constexpr int STG_BYTES = 4 * 2 * 4096;
 constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + STG_BYTES + 1024 + 256;
 constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                              ((uint32_t)(BM2 >> 4) << 24);
+// kind::f8f6f4, A and B both E4M3 (format code 0), fp32 accumulate, M = 256, N = 256.  A
+// stage holds the same 128-byte rows, so 128 K elements instead of 64 and each of the
+// four MMAs per stage covers K = 32.
+constexpr uint32_t kIdesc2F8 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM2 >> 4) << 24);
+constexpr int BK8 = 128;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -554,6 +567,15 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
         "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
         " [%0], m;\n\t}" ::"r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
         : "memory");
 }
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -602,6 +624,14 @@ __device__ __forceinline__ uint32_t stg_off(int r, int k) {
 __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// E4M3 accumulators back to real units: v[j] *= a_scale[m] * b_scale[n + j].
+template <int W>
+__device__ __forceinline__ void dequant_chunk(const TcParams& p, int m, int n, float* v) {
+    const float sa = m < p.M ? __ldg(p.a_scale + m) : 0.f;
+#pragma unroll
+    for (int j = 0; j < W; ++j) v[j] = v[j] * sa * ((n + j < p.N) ? __ldg(p.b_scale + n + j) : 0.f);
 }
 
 // Pair-kernel epilogue: each warp stages its 32 rows x (32 fp32 | 64 bf16) columns in
@@ -657,6 +687,10 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
                 float gv[32], uv[32];
                 tmem_ld32(taddr + (uint32_t)((c + h) * 32), gv);
                 tmem_ld32(taddr + (uint32_t)(128 + (c + h) * 32), uv);
+                if (p.a_scale) {
+                    dequant_chunk<32>(p, m_base + r, nb * 256 + (c + h) * 32, gv);
+                    dequant_chunk<32>(p, m_base + r, nb * 256 + 128 + (c + h) * 32, uv);
+                }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     float g = gv[j], u = uv[j];
@@ -695,6 +729,7 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
                 for (int c = 0; c < 4; ++c) {
                     float v[32];
                     tmem_ld32(th + (uint32_t)(c * 32), v);
+                    if (p.a_scale) dequant_chunk<32>(p, m, n0 + c * 32, v);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float x = __bfloat162float(__float2bfloat16_rn(v[j]));
@@ -710,6 +745,10 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
                 float lo[32], hi[32];
                 tmem_ld32(th + (uint32_t)(c * 32), lo);
                 tmem_ld32(th + (uint32_t)(64 + c * 32), hi);
+                if (p.a_scale) {
+                    dequant_chunk<32>(p, m, n0 + c * 32, lo);
+                    dequant_chunk<32>(p, m, n0 + 64 + c * 32, hi);
+                }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     lo[j] = __bfloat162float(__float2bfloat16_rn(lo[j]));
@@ -764,6 +803,7 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
             float y[64];
             tmem_ld32(taddr + (uint32_t)(c * 32), y);
             tmem_ld32(taddr + (uint32_t)((c + 1) * 32), y + 32);
+            if (p.a_scale) dequant_chunk<64>(p, m_base + r, n, y);
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
                 float v = y[j];
@@ -864,8 +904,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (rank == 0) mbar_expect_tx(full(s), 2 * STAGE2_BYTES);
                     const uint32_t lb = map_rank(full(s), 0);
                     if (kb < p.kb_main) {
-                        tma_load_2d_pair(sa, &tmA, lb, kb * BK, row_a);
-                        tma_load_2d_pair(sb, &tmB, lb, kb * BK, row_b);
+                        const int k = kb * (p.fp8 ? BK8 : BK);
+                        tma_load_2d_pair(sa, &tmA, lb, k, row_a);
+                        tma_load_2d_pair(sb, &tmB, lb, k, row_b);
                     } else {
                         const int k = (kb - p.kb_main) * BK;
                         tma_load_2d_pair(sa, &tmA2, lb, k, row_a);
@@ -901,10 +942,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     tc_fence_after();
                     const uint32_t sa = base + s * STAGE2_BYTES;
                     const uint32_t sb = sa + A2B;
+                    if (p.fp8 && kb < p.kb_main) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), kIdesc2,
-                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_pair_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
+                                           kIdesc2F8, (kb > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
+                                        kIdesc2, (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     tc_commit_pair(empty(s));       // stage free in both CTAs
@@ -982,14 +1029,16 @@ EncodeTiledFn encode_fn() {
 // 2-D bf16 map over a row-major [rows x cols] matrix with leading dimension ld,
 // box = 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld,
-              uint32_t box_rows) {
+              uint32_t box_rows, bool fp8 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    // 128-byte box rows either way: 64 bf16 or 128 E4M3 elements
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {ld * 2};
-    const cuuint32_t box[2] = {BK, box_rows};
+    const cuuint64_t strides[1] = {ld * (fp8 ? 1 : 2)};
+    const cuuint32_t box[2] = {fp8 ? (cuuint32_t)BK8 : (cuuint32_t)BK, box_rows};
     const cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+    return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void*>(ptr), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1095,8 +1144,18 @@ int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a
 }  // namespace
 
 bool gemm_tc_supported(const GemmArgs& g) {
-    if (g.a_type != E_BF16 || g.b_type != E_BF16) return false;
-    if (g.K % 8 || g.lda % 8 || g.ldb % 8 || g.K <= 0 || g.M <= 0 || g.N <= 0) return false;
+    if (g.a_type == E_FP8 || g.b_type == E_FP8) {
+        // E4M3 main operands: SM-pair kernel, 16-byte rows, scales for both sides
+        if (g.a_type != E_FP8 || g.b_type != E_FP8 || !g_use_pairs || g.N <= 128) return false;
+        if (g.K % 16 || g.lda % 16 || g.ldb % 16 || g.K <= 0 || g.M <= 0) return false;
+        if (!g.a_scale || !g.b_scale) return false;
+        if (g.epi != EPI_STORE && g.epi != EPI_STORE_RELU && g.epi != EPI_QKNR &&
+            g.epi != EPI_SWIGLU)
+            return false;
+    } else {
+        if (g.a_type != E_BF16 || g.b_type != E_BF16) return false;
+        if (g.K % 8 || g.lda % 8 || g.ldb % 8 || g.K <= 0 || g.M <= 0 || g.N <= 0) return false;
+    }
     if (!aligned16(g.A) || !aligned16(g.B)) return false;
     if (g.K2 > 0) {
         if (g.a2_type != E_BF16 || g.b2_type != E_BF16 || g.lda2 % 8 || g.ldb2 % 8 || g.K2 % 8)
@@ -1148,8 +1207,10 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     const int bnt = pair ? BN : tile1_width(g);
     const uint32_t b_rows = pair ? 128u : (uint32_t)bnt;
     CUtensorMap a, b, a2, b2;
-    if (!make_map(&a, g.A, g.M, g.K, g.lda, BM)) return 1;
-    if (!make_map(&b, g.B, g.N, g.K, g.ldb, b_rows)) return 1;
+    const bool f8 = g.a_type == E_FP8;
+    if (f8 && !pair) return 1;
+    if (!make_map(&a, g.A, g.M, g.K, g.lda, BM, f8)) return 1;
+    if (!make_map(&b, g.B, g.N, g.K, g.ldb, b_rows, f8)) return 1;
     if (g.K2 > 0) {
         if (!make_map(&a2, g.A2, g.M, g.K2, g.lda2, BM)) return 1;
         if (!make_map(&b2, g.B2, g.N, g.K2, g.ldb2, b_rows)) return 1;
@@ -1160,13 +1221,15 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     TcParams p;
     memset(&p, 0, sizeof(p));
     p.M = g.M; p.N = g.N;
-    p.kb_main = (g.K + BK - 1) / BK;
+    p.kb_main = f8 ? (g.K + BK8 - 1) / BK8 : (g.K + BK - 1) / BK;
+    p.fp8 = f8 ? 1 : 0;
+    p.a_scale = g.a_scale; p.b_scale = g.b_scale;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
     p.n_m_blk = pair ? (g.M + BM2 - 1) / BM2 : (g.M + BM - 1) / BM;
     // Raster: an M group whose A strips (256 rows x K) fit in ~48 MB of L2 sweeps all N
     // blocks, so each weight strip is fetched from DRAM once per group.
     {
-        const double strip = (double)BM2 * (g.K + g.K2) * 2.0;
+        const double strip = (double)BM2 * ((double)g.K * (f8 ? 1.0 : 2.0) + g.K2 * 2.0);
         int gm = (int)(48.0e6 / strip);
         gm = gm < 4 ? 4 : (gm > 32 ? 32 : gm);
         p.group_m = pair ? gm : GROUP_M;

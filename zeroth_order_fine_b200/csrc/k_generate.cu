@@ -114,8 +114,8 @@ __global__ void open_window_kernel(const WindowJob* jobs) {
     const int n = jb.d_out * jb.r;
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
         const int i = e / jb.r, c = e % jb.r;
-        const float v = jb.V[e];
         const int fr = jb.interleave ? (i / 128) * 256 + jb.row0 + i % 128 : jb.row0 + i;
+        const float v = jb.row_div ? jb.V[e] / jb.row_div[fr] : jb.V[e];
         const size_t row = (size_t)fr * jb.ldb;
         st_elem(jb.EB, row + jb.col_dir + c, jb.eb_type, v);
         st_elem(jb.EB, row + jb.col_slot + c, jb.eb_type, v);

@@ -1,6 +1,8 @@
 // Token metadata, embeddings, LayerNorm / RMSNorm (optionally gathering the
 // scored rows first) and the SwiGLU activation.  All HBM-bound, one CTA per
 // token row, each row read once.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -112,12 +114,16 @@ __global__ void __launch_bounds__(256) norm_kernel(const float* __restrict__ x,
 
 // Vectorised form for d % 4 == 0, d <= 1024 * VPT: the row stays in registers
 // (VPT float4 per thread), 16-byte loads, 8-byte bf16 stores.
+// With q8: the bf16 output row is also quantised to E4M3 with one scale per row
+// (amax / 448), from the bf16-rounded values, for the FP8 base GEMMs.
 template <int VPT>
 __global__ void __launch_bounds__(256) norm_vec_kernel(const float* __restrict__ x,
                                                        const int* __restrict__ rows, int d,
                                                        int kind, const float* __restrict__ w,
                                                        const float* __restrict__ b, float eps,
-                                                       void* __restrict__ out, int out_type) {
+                                                       void* __restrict__ out, int out_type,
+                                                       uint8_t* __restrict__ q8,
+                                                       float* __restrict__ s8) {
     __shared__ float red[32];
     const int t = blockIdx.x;
     const int src = rows ? rows[t] : t;
@@ -175,29 +181,85 @@ __global__ void __launch_bounds__(256) norm_vec_kernel(const float* __restrict__
             pk.x = *reinterpret_cast<uint32_t*>(&h0);
             pk.y = *reinterpret_cast<uint32_t*>(&h1);
             reinterpret_cast<uint2*>(out)[(size_t)t * n4 + j] = pk;
+            v[i] = make_float4(__low2float(h0), __high2float(h0), __low2float(h1), __high2float(h1));
         }
+    }
+    if (q8 == nullptr) return;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int j = threadIdx.x + i * 256;
+        if (j < n4)
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)),
+                                     fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+    }
+    amax = block_max(amax, red);
+    const float inv = amax > 0.f ? 448.0f / amax : 1.0f;
+    if (threadIdx.x == 0) s8[t] = amax > 0.f ? amax / 448.0f : 1.0f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int j = threadIdx.x + i * 256;
+        if (j >= n4) continue;
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[i].x * inv, v[i].y * inv),
+                                                     __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v[i].z * inv, v[i].w * inv),
+                                                     __NV_SATFINITE, __NV_E4M3);
+        reinterpret_cast<uint32_t*>(q8)[(size_t)t * n4 + j] = lo | (hi << 16);
     }
 }
 
+// One CTA per row: amax, then the codes (used for the frozen weights at set-up).
+__global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const void* __restrict__ x,
+                                                              int x_type, int cols, size_t ldx,
+                                                              uint8_t* __restrict__ q, size_t ldq,
+                                                              float* __restrict__ scale) {
+    __shared__ float red[32];
+    const size_t r = blockIdx.x;
+    float amax = 0.f;
+    for (int i = threadIdx.x; i < cols; i += blockDim.x)
+        amax = fmaxf(amax, fabsf(ld_elem(x, r * ldx + i, x_type)));
+    amax = block_max(amax, red);
+    const float inv = amax > 0.f ? 448.0f / amax : 1.0f;
+    if (threadIdx.x == 0) scale[r] = amax > 0.f ? amax / 448.0f : 1.0f;
+    for (int i = 2 * threadIdx.x; i < cols; i += 2 * blockDim.x) {
+        const float a = ld_elem(x, r * ldx + i, x_type) * inv;
+        const float b = i + 1 < cols ? ld_elem(x, r * ldx + i + 1, x_type) * inv : 0.f;
+        const uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+        q[r * ldq + i] = (uint8_t)(c & 0xFFu);
+        if (i + 1 < cols) q[r * ldq + i + 1] = (uint8_t)(c >> 8);
+    }
+}
+
+void launch_quant_rows_e4m3(const void* x, int x_type, int rows, int cols, size_t ldx,
+                            uint8_t* q, size_t ldq, float* scale, cudaStream_t st) {
+    if (rows == 0) return;
+    quant_rows_e4m3_kernel<<<rows, 256, 0, st>>>(x, x_type, cols, ldx, q, ldq, scale);
+}
+
+bool norm_fp8_supported(int d) { return d % 4 == 0 && (d / 4 + 255) / 256 <= 8; }
+
 void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
-                 const float* b, float eps, void* out, int out_type, cudaStream_t st) {
+                 const float* b, float eps, void* out, int out_type, cudaStream_t st,
+                 uint8_t* q8, float* s8) {
     if (T == 0) return;
     const int vpt = (d / 4 + 255) / 256;
     auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
     const bool aligned = al16(x) && al16(w) && (b == nullptr || al16(b)) && al16(out);
     if (d % 4 == 0 && vpt <= 8 && aligned) {
         switch (vpt) {
-            case 1: norm_vec_kernel<1><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
-            case 2: norm_vec_kernel<2><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
-            case 3: norm_vec_kernel<3><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
-            case 4: norm_vec_kernel<4><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
-            case 5: norm_vec_kernel<5><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
-            case 6: norm_vec_kernel<6><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
-            case 7: norm_vec_kernel<7><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
-            default: norm_vec_kernel<8><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type); return;
+            case 1: norm_vec_kernel<1><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 2: norm_vec_kernel<2><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 3: norm_vec_kernel<3><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 4: norm_vec_kernel<4><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 5: norm_vec_kernel<5><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 6: norm_vec_kernel<6><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 7: norm_vec_kernel<7><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            default: norm_vec_kernel<8><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
         }
     }
     norm_kernel<<<T, 256, d * sizeof(float), st>>>(x, rows, d, kind, w, b, eps, out, out_type);
+    // the E4M3 rows of the bf16 output, when the vectorised form could not write them
+    if (q8) launch_quant_rows_e4m3(out, out_type, T, d, (size_t)d, q8, (size_t)d, s8, st);
 }
 
 // out[t, j] = silu(gu[t, j]) * gu[t, f + j]; gu = [gate | up] per row.

@@ -5,7 +5,7 @@
 
 namespace zo {
 
-enum ElemType : int { E_F32 = 0, E_BF16 = 1 };
+enum ElemType : int { E_F32 = 0, E_BF16 = 1, E_FP8 = 2 };   // E_FP8: E4M3 bytes
 
 // ---- generator -------------------------------------------------------------------------
 struct GenJob {
@@ -23,6 +23,8 @@ struct WindowJob {
     void* A_bf;                 // optional bf16 mirror of those rows
     int eb_type, ldb, row0, d_out, d_in, r, col_dir, col_slot;
     int interleave;             // 1: row i sits at (i / 128) * 256 + row0 + i % 128
+    const float* row_div;       // optional: E_B row fr holds V / row_div[fr] (the fused
+                                // matrix's FP8 weight scales), so one accumulator serves both
 };
 
 void launch_init_tensor(void* dst, uint64_t n, uint64_t key, float std_, float mean, int dtype,
@@ -51,8 +53,15 @@ void launch_build_tokens(RowMeta m, int R, const int* probe_src, const int* fg_s
 void launch_embed(const int* tok_id, const int* tok_pos, const void* tok_embed,
                   const void* pos_embed, int dtype, float* resid, int T, int d, cudaStream_t st);
 // kind 0: LayerNorm(w, b), 1: RMSNorm(w).  rows: optional gather list (else 0..T-1).
+// E4M3 per-row quantisation: scale[r] = amax / 448, q = E4M3(x * (448 / amax)), RN, saturated;
+// an all-zero row has scale 1.  x is fp32 or bf16 [rows x ldx], q [rows x ldq] bytes.
+void launch_quant_rows_e4m3(const void* x, int x_type, int rows, int cols, size_t ldx,
+                            uint8_t* q, size_t ldq, float* scale, cudaStream_t st);
+// q8/s8 (optional, vectorised path only): also the E4M3 quantisation of the bf16 output rows
 void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
-                 const float* b, float eps, void* out, int out_type, cudaStream_t st);
+                 const float* b, float eps, void* out, int out_type, cudaStream_t st,
+                 uint8_t* q8 = nullptr, float* s8 = nullptr);
+bool norm_fp8_supported(int d);
 void launch_swiglu(const void* gu, int T, int f, void* out, int dtype, cudaStream_t st);
 void launch_rope_table(float* cos_t, float* sin_t, int max_pos, int hd, double theta,
                        cudaStream_t st);
@@ -89,6 +98,10 @@ struct GemmArgs {
     const int* row_sign; float eps; int scale_cols;
     // EPI_LSE
     const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
+    // E_FP8 operands: dequantisation scales per row of A [M] and of B [N]; the epilogue
+    // multiplies the accumulator by a_scale[m] * b_scale[n] (the extension operands must
+    // be pre-divided accordingly).  EPI_SHRINK with a_scale divides its output rows by it.
+    const float* a_scale; const float* b_scale;
     // EPI_QKNR: token positions [M], norm weights [128] of q and k, rotary tables
     // [max_pos x 64]; heads below n_q_heads use qn, the next ones up to n_qk_heads kn
     const int* tok_pos; const float* qn; const float* kn;

@@ -21,6 +21,35 @@ bool use_tc(int32_t impl, int dtype) {
 
 extern "C" {
 
+int zo_op_quantize_rows_e4m3(const void* x, int32_t dtype, int32_t rows, int32_t cols,
+                             uint8_t* q, float* scale, void* stream) {
+    if (!x || !q || !scale || rows < 0 || cols <= 0) return ZO_ERR_ARG;
+    if (dtype != ZO_DTYPE_FP32 && dtype != ZO_DTYPE_BF16) return ZO_ERR_ARG;
+    launch_quant_rows_e4m3(x, dtype == ZO_DTYPE_BF16 ? E_BF16 : E_F32, rows, cols, (size_t)cols, q,
+                           (size_t)cols, scale, static_cast<cudaStream_t>(stream));
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
+int zo_op_linear_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                     const float* bias, void* y, int32_t M, int32_t N, int32_t K, int32_t act,
+                     void* stream) {
+    if (!xq || !sx || !wq || !sw || !y || M < 0 || N <= 0 || K <= 0) return ZO_ERR_ARG;
+    if (act != ZO_ACT_NONE && act != ZO_ACT_RELU) return ZO_ERR_ARG;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.A = xq; g.lda = K; g.a_type = E_FP8;
+    g.B = wq; g.ldb = K; g.b_type = E_FP8;
+    g.a_scale = sx; g.b_scale = sw;
+    g.M = M; g.N = N; g.K = K;
+    g.bias = bias;
+    g.epi = act == ZO_ACT_RELU ? EPI_STORE_RELU : EPI_STORE;
+    g.C = y; g.ldc = N; g.c_type = E_BF16;
+    if (M == 0) return ZO_OK;
+    if (!gemm_tc_supported(g)) return ZO_ERR_UNSUPPORTED;
+    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return ZO_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
 int zo_op_linear(const void* x, const void* W, const float* bias, void* y, int32_t M, int32_t N,
                  int32_t K, int32_t dtype, int32_t act, int32_t accumulate, int32_t impl,
                  void* stream) {

@@ -66,7 +66,7 @@ class zo_options(ctypes.Structure):
     _fields_ = [("run_seed", c_uint64), ("lazy_interval", c_int32), ("rank", c_int32),
                 ("targets", zo_targets), ("max_tokens", c_int32), ("max_rows", c_int32),
                 ("max_scored", c_int32), ("max_slots", c_int32), ("start_step", c_uint64),
-                ("stream", c_void_p), ("impl", c_int32), ("profile", c_int32)]
+                ("stream", c_void_p), ("impl", c_int32), ("profile", c_int32), ("fp8", c_int32)]
 
 
 class zo_stats_t(ctypes.Structure):
@@ -115,6 +115,10 @@ _SIGS = {
                                  ctypes.c_float, ctypes.c_float, c_int32, c_void_p]),
     "zo_op_linear": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                c_int32, c_int32, c_int32, c_int32, c_void_p]),
+    "zo_op_quantize_rows_e4m3": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                           c_void_p, c_void_p]),
+    "zo_op_linear_fp8": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   c_int32, c_int32, c_int32, c_int32, c_void_p]),
     "zo_op_lm_head_workspace": (ctypes.c_size_t, [c_int32, c_int32, c_int32]),
     "zo_op_lm_head_logprob": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                         c_int32, c_void_p, c_void_p, ctypes.c_size_t, c_int32,
@@ -277,7 +281,7 @@ class Handle:
     def __init__(self, model: DeviceModel, run_seed: int, nu: int, rank: int,
                  targets: zo_targets, max_tokens: int, max_rows: int, max_scored: int,
                  max_slots: int = 32, start_step: int = 0, stream=None, impl: int = 0,
-                 profile: int = 0):
+                 profile: int = 0, fp8: int = 0):
         self.model = model
         self.targets = targets
         self.rank = rank
@@ -285,7 +289,7 @@ class Handle:
         self._desc = model.desc()
         self._w = model.weights()
         opt = zo_options(run_seed, nu, rank, targets, max_tokens, max_rows, max_scored, max_slots,
-                         start_step, _stream(self.stream), impl, profile)
+                         start_step, _stream(self.stream), impl, profile, fp8)
         h = c_void_p()
         rc = lib().zo_create(ctypes.byref(self._desc), ctypes.byref(self._w), ctypes.byref(opt),
                              ctypes.byref(h))
@@ -422,6 +426,27 @@ def zo_op_linear(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] 
     _check(lib().zo_op_linear(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, dtype, act,
                               int(accumulate), impl, _stream()))
     return out
+
+
+def zo_op_quantize_rows_e4m3(x: torch.Tensor):
+    """(codes uint8 [rows, cols], scale float [rows]) of the E4M3 row quantiser."""
+    rows, cols = x.shape
+    dtype = wl.DTYPE_BF16 if x.dtype == torch.bfloat16 else wl.DTYPE_FP32
+    q = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    sc = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib().zo_op_quantize_rows_e4m3(_ptr(x), dtype, rows, cols, _ptr(q), _ptr(sc),
+                                          _stream()))
+    return q, sc
+
+
+def zo_op_linear_fp8(xq: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                     bias: Optional[torch.Tensor] = None, act: int = 0) -> torch.Tensor:
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
+    _check(lib().zo_op_linear_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y),
+                                  M, N, K, act, _stream()))
+    return y
 
 
 def zo_op_lm_head_logprob(h: torch.Tensor, E: torch.Tensor, targets: torch.Tensor,
