@@ -269,7 +269,15 @@ def run_kernel(args):
     from zeroth_order_fine_b200 import zo
     g = torch.Generator(device="cuda").manual_seed(0)
     M, N, K = args.m, args.n, args.k
-    if args.kernel == "gemm":
+    if args.kernel == "gemm" and args.fp8:
+        x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+        W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        xq, sx = zo.zo_op_quantize_rows_e4m3(x)
+        wq, sw = zo.zo_op_quantize_rows_e4m3(W)
+        fn = lambda: zo.zo_op_linear_fp8(xq, sx, wq, sw)  # noqa: E731
+        work, unit = 2.0 * M * N * K, "TFLOP/s"
+        bytes_ = M * K + N * K + M * N * 2
+    elif args.kernel == "gemm":
         x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
         W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
         y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
@@ -305,7 +313,8 @@ def run_kernel(args):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.launches
     assert zo.zo_op_error_word() == 0
-    print(json.dumps({"kernel": args.kernel, "m": M, "n": N, "k": K, "ms_per_launch": ms,
+    print(json.dumps({"kernel": args.kernel + ("-e4m3" if args.fp8 else ""), "m": M, "n": N,
+                      "k": K, "ms_per_launch": ms,
                       "achieved": work / (ms / 1e3) / 1e12, "unit": unit,
                       "gb_per_s": bytes_ / (ms / 1e3) / 1e9}), flush=True)
     return 0

@@ -630,8 +630,21 @@ __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
 template <int W>
 __device__ __forceinline__ void dequant_chunk(const TcParams& p, int m, int n, float* v) {
     const float sa = m < p.M ? __ldg(p.a_scale + m) : 0.f;
+    if (n + W <= p.N) {                     // n is a multiple of 32: 16-byte aligned scales
+        const float4* b4 = reinterpret_cast<const float4*>(p.b_scale + n);
 #pragma unroll
-    for (int j = 0; j < W; ++j) v[j] = v[j] * sa * ((n + j < p.N) ? __ldg(p.b_scale + n + j) : 0.f);
+        for (int q = 0; q < W / 4; ++q) {
+            const float4 sb = __ldg(b4 + q);
+            v[4 * q] = v[4 * q] * sa * sb.x;
+            v[4 * q + 1] = v[4 * q + 1] * sa * sb.y;
+            v[4 * q + 2] = v[4 * q + 2] * sa * sb.z;
+            v[4 * q + 3] = v[4 * q + 3] * sa * sb.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < W; ++j)
+            v[j] = v[j] * sa * ((n + j < p.N) ? __ldg(p.b_scale + n + j) : 0.f);
+    }
 }
 
 // Pair-kernel epilogue: each warp stages its 32 rows x (32 fp32 | 64 bf16) columns in
