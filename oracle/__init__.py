@@ -24,6 +24,8 @@ Parts and what pins them (see tests/test_oracle_*.py):
 * fp8        -- the E4M3 cast against the format decoded bit by bit (all 256
   codes; nearest value, ties to even, saturation), the per-row quantiser's
   scale equivariance and error bound.
+* generation -- greedy decoding (one full forward per token) against teacher-forced
+  scoring of the generated tokens, eps = 0 symmetry, the dense brute force.
 * zo         -- the estimator against its closed form and an exact quadratic
   toy, its epsilon -> 0 limit against autograd, the factored perturbation
   against a dense brute force with W +/- eps*U V^T materialised, the bank

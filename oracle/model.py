@@ -267,6 +267,24 @@ def hidden_states(w: Weights, rows: Sequence[np.ndarray], signs: Sequence[float]
     return rms_norm(h, w.final_w, sh.norm_eps)
 
 
+def span_logits(w: Weights, hs: torch.Tensor, rows: Sequence[np.ndarray],
+                target_lens: Sequence[int]) -> List[torch.Tensor]:
+    """Per row, the full-vocabulary logits [tl, V] at the positions that predict its last
+    tl tokens (positions L - tl - 1 .. L - 2)."""
+    bf = w.shape.dtype == wl.DTYPE_BF16
+    out = []
+    off = 0
+    for r, tl in zip(rows, target_lens):
+        L = len(r)
+        idx = torch.arange(off + L - tl - 1, off + L - 1)
+        hsel = hs[idx]
+        if bf:
+            hsel = bf16_round(hsel)
+        out.append(hsel @ w.lm_head.T)
+        off += L
+    return out
+
+
 def token_logprobs(w: Weights, hs: torch.Tensor, rows: Sequence[np.ndarray],
                    target_lens: Sequence[int]) -> List[torch.Tensor]:
     """Per row, log p(target token | prefix) for each of its last target_lens tokens.
@@ -277,18 +295,20 @@ def token_logprobs(w: Weights, hs: torch.Tensor, rows: Sequence[np.ndarray],
     of the label tokens: page 1, "Why ZO Fine-Tuning Is Really Scoring" and
     "The System Reorganization").
     """
-    bf = w.shape.dtype == wl.DTYPE_BF16
     out = []
-    off = 0
-    for r, tl in zip(rows, target_lens):
+    for r, tl, logits in zip(rows, target_lens, span_logits(w, hs, rows, target_lens)):
         L = len(r)
-        idx = torch.arange(off + L - tl - 1, off + L - 1)
-        hsel = hs[idx]
-        if bf:
-            hsel = bf16_round(hsel)
-        logits = hsel @ w.lm_head.T
         lse = torch.logsumexp(logits, dim=-1)
         tgt = torch.from_numpy(np.asarray(r[L - tl:], dtype=np.int64))
         out.append(logits[torch.arange(tl), tgt] - lse)
-        off += L
     return out
+
+
+def last_logits(w: Weights, hs: torch.Tensor, rows: Sequence[np.ndarray]) -> torch.Tensor:
+    """Logits [rows, V] at each row's last position: the prediction of its next token."""
+    bf = w.shape.dtype == wl.DTYPE_BF16
+    ends = torch.from_numpy(np.cumsum([len(r) for r in rows]) - 1)
+    hsel = hs[ends]
+    if bf:
+        hsel = bf16_round(hsel)
+    return hsel @ w.lm_head.T

@@ -131,6 +131,37 @@ class OracleRun:
         self.last = res
         return res
 
+    # -- generation queries -------------------------------------------------------------
+    def generate(self, prompts: Sequence[np.ndarray], n_new: int, dense: bool = False):
+        """Greedy generation under theta + eps z (rows 0..B-1) and theta - eps z (rows
+        B..2B-1): n_new tokens per row, each the largest logit of the full forward of the
+        row so far (ties: lowest id); objective per row = mean -log p of its new tokens.
+
+        A reading of "Inference-Native Zeroth-Order Optimization" (abstract: the same
+        ProbePlan covers autoregressive generation); written as the plain definition, one
+        full forward per new token, no cache.  Returns (L_plus, L_minus, tokens [2B, n_new],
+        logprobs [2B, n_new]) and records the result for step()."""
+        B = len(prompts)
+        seqs = [list(np.asarray(prompts[r % B])) for r in range(2 * B)]   # one list per row
+        signs = [1.0] * B + [-1.0] * B
+        pert = self.perturbation()
+        toks = np.zeros((2 * B, n_new), dtype=np.int64)
+        lps = np.zeros((2 * B, n_new), dtype=np.float64)
+        for g in range(n_new):
+            rows = [np.asarray(x, dtype=np.int64) for x in seqs]
+            hs = om.hidden_states(self.w, rows, signs, self.eps, pert, dense, fp8=self.fp8)
+            logits = om.last_logits(self.w, hs, rows)
+            lse = torch.logsumexp(logits, dim=-1)
+            for r in range(2 * B):
+                t = int(torch.argmax(logits[r]).item())
+                toks[r, g] = t
+                lps[r, g] = float(logits[r, t] - lse[r])
+                seqs[r].append(t)
+        L = -lps.mean(axis=1)
+        res = ScoreResult(L[:B], L[B:], list(lps[:B]), list(lps[B:]), [])
+        self.last = res
+        return L[:B], L[B:], toks, lps
+
     # -- step ---------------------------------------------------------------------------
     def step(self, lr: float) -> float:
         """c from the last score; A_k <- A_k - lr c U_t for every target; t <- t + 1.
