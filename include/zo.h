@@ -137,6 +137,9 @@ typedef struct zo_options {
                                 (scale = amax / 448, round to nearest even, saturated).  The
                                 direction, bank and every other GEMM stay in the model dtype.
                                 bf16 models with impl 0 only, else ZO_ERR_UNSUPPORTED.  0: off */
+    int32_t    max_new;      /* most tokens zo_generate decodes per row (0: no generation);
+                                sizes the KV cache: n_layers x (max_tokens + max_rows * max_new)
+                                rows of 2 * n_kv_heads * head_dim elements                   */
 } zo_options;
 
 typedef struct zo_handle zo_handle;
@@ -205,6 +208,27 @@ int zo_probe_plan(zo_handle* h, uint64_t step, int32_t rank, float eps,
 int zo_score(zo_plan* plan, const int32_t* packed_tokens, int32_t n_prompts,
              const int32_t* seq_lens, const int32_t* target_lens, const int32_t* target_ids,
              float* L_plus, float* L_minus, float* tok_logprob);
+
+/* Generation queries ("Inference-Native Zeroth-Order Optimization", abstract:
+ * the same ProbePlan covers autoregressive generation as well as token
+ * scoring).  Each prompt becomes a + row and a - row (all +, then all -, as in
+ * zo_score); each row decodes n_new tokens greedily under its own candidate
+ * state theta +- eps z: the prompt runs once as a packed prefill whose keys and
+ * values are kept in a per-layer cache, then one decode step per further token
+ * appends to it.  Greedy = the largest logit, ties to the lowest token id.  The
+ * row's objective is the mean of -log p(token | prefix) over its generated
+ * tokens; L+/L- go to L_plus/L_minus as in zo_score, and zo_step then applies
+ * the update.
+ *   packed_tokens dev int32 [sum(seq_lens)], seq_lens host int32 [n_prompts], each >= 2
+ *     and seq_len + n_new <= max_pos
+ *   gen_tokens  dev int32 [2 n_prompts x n_new] or NULL: row r's tokens at r * n_new
+ *   gen_logprob dev float [2 n_prompts x n_new] or NULL: their log-probabilities
+ *   L_plus, L_minus dev float [n_prompts] or NULL
+ * ZO_ERR_UNSUPPORTED when options.max_new is 0; ZO_ERR_ARG when n_new is outside
+ * 1..max_new or the batch exceeds max_tokens / max_rows. */
+int zo_generate(zo_plan* plan, const int32_t* packed_tokens, int32_t n_prompts,
+                const int32_t* seq_lens, int32_t n_new, int32_t* gen_tokens,
+                float* gen_logprob, float* L_plus, float* L_minus);
 
 /* zo_score with n_fg unperturbed foreground rows appended to the same
  * physical batch (co-batching: "Inference-Native Zeroth-Order Optimization",

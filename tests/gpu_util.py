@@ -10,7 +10,7 @@ needs_gpu = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CU
 
 
 def gpu_handle(w: wl.Workload, shape=None, batch=None, max_slots=8, impl=0, nu=None,
-               layers=None, start_step=0, fg=0, fp8=0):
+               layers=None, start_step=0, fg=0, fp8=0, max_new=0):
     from zeroth_order_fine_b200 import zo
     shape = shape or w.shape
     model = zo.DeviceModel(shape, w.weight_seed)
@@ -20,7 +20,8 @@ def gpu_handle(w: wl.Workload, shape=None, batch=None, max_slots=8, impl=0, nu=N
     h = zo.Handle(model, w.run_seed, nu or w.nu, w.rank, tg,
                   max_tokens=(2 * B + fg) * max_len + 64, max_rows=2 * B + fg,
                   max_scored=(2 * B + fg) * max(w.tgt_hi, w.fg_tgt_hi if fg else 1),
-                  max_slots=max_slots, start_step=start_step, impl=impl, fp8=fp8)
+                  max_slots=max_slots, start_step=start_step, impl=impl, fp8=fp8,
+                  max_new=max_new)
     return model, h
 
 

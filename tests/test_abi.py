@@ -44,7 +44,7 @@ def test_struct_sizes_match_header(built_lib):
     from zeroth_order_fine_b200 import zo
     assert ctypes.sizeof(zo.zo_model_desc) == 13 * 4
     assert ctypes.sizeof(zo.zo_targets) == 24
-    assert zo.zo_options.stream.offset == 64 and ctypes.sizeof(zo.zo_options) == 88
+    assert zo.zo_options.stream.offset == 64 and ctypes.sizeof(zo.zo_options) == 88   # 84 bytes of fields, 8-aligned
     assert ctypes.sizeof(zo.zo_layer_weights) == 20 * 8
 
 

@@ -1,0 +1,116 @@
+"""Generation queries through the C ABI (zo_generate): greedy decoding of both candidates
+with the KV cache, checked against the oracle teacher-forced on the GPU's own tokens (each
+token must be a largest logit there, within the mode's tolerance, and its log-probability
+must match), the eps = 0 symmetry, the GPU's own prefill scoring of the generated rows, and
+the update that follows."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from zeroth_order_fine_b200 import workload as wl
+from gpu_util import dev_tokens, gpu_handle, needs_gpu, oracle_run
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+TINY = wl.WORKLOADS["tiny"]
+TINY_BF16 = dataclasses.replace(TINY, shape=wl.shrink_shape(wl.TINY, dtype=wl.DTYPE_BF16))
+Q3_SMALL_BF16 = wl.ModelShape("qwen3-small", wl.ARCH_QWEN3, 2, 256, 4, 2, 128, 512, 1000, 4096,
+                              1e-6, 1e6, wl.DTYPE_BF16, False)
+QWEN_SMALL = wl.Workload("qwen3-small", Q3_SMALL_BF16, 6, 20, 90, 1, 4, True, 8, wl.ALL7,
+                         wl.SCALE_MEZO, 1e-3, 1e-4, 3, fg_rows=0, data_seed=11)
+G = 6
+
+
+def _check_against_oracle(w, fp8, logit_tol, lp_tol, L_tol, impl=0):
+    from oracle import model as om
+    batch = wl.make_batch(w, fg_rows=0)
+    B = len(batch.prompts)
+    _, h = gpu_handle(w, max_new=G, fp8=int(fp8), impl=impl)
+    toks = dev_tokens(batch)
+    h.zo_probe_plan(0, w.eps)
+    Lp, Lm, gt, gl = h.zo_generate(toks, batch.seq_lens, G)
+    gt, gl = gt.cpu().numpy(), gl.cpu().numpy()
+    orc = oracle_run(w, fp8=fp8)
+    orc.plan(0, w.eps)
+    rows = [np.concatenate([p, gt[r]]).astype(np.int64)
+            for r, p in enumerate(list(batch.prompts) * 2)]
+    hs = om.hidden_states(orc.w, rows, [1.0] * B + [-1.0] * B, orc.eps, orc.perturbation(),
+                          fp8=fp8)
+    logits = om.span_logits(orc.w, hs, rows, [G] * (2 * B))
+    ref_lp = om.token_logprobs(orc.w, hs, rows, [G] * (2 * B))
+    for r in range(2 * B):
+        lg = logits[r].numpy()
+        chosen = lg[np.arange(G), gt[r]]
+        assert np.all(chosen >= lg.max(axis=1) - logit_tol), (r, lg.max(axis=1) - chosen)
+        assert np.max(np.abs(gl[r] - ref_lp[r].numpy())) <= lp_tol, r
+    ref_L = np.array([-x.numpy().mean() for x in ref_lp])
+    assert np.max(np.abs(Lp.cpu().numpy() - ref_L[:B])) <= L_tol
+    assert np.max(np.abs(Lm.cpu().numpy() - ref_L[B:])) <= L_tol
+    c = h.zo_step(w.lr)
+    assert np.isfinite(c) and h.zo_stats()["steps"] == 1
+    return h, batch, gt
+
+
+@pytest.mark.parametrize("impl", [0, 1])
+def test_tiny_fp32_generation_matches_oracle(impl):
+    _check_against_oracle(TINY, False, 1e-4, 1e-4, 1e-4, impl=impl)
+
+
+def test_tiny_bf16_generation_matches_oracle():
+    _check_against_oracle(TINY_BF16, False, 5e-2, 3e-2, 2e-2)
+
+
+def test_qwen3_bf16_generation_matches_oracle():
+    _check_against_oracle(QWEN_SMALL, False, 5e-2, 3e-2, 2e-2)
+
+
+def test_qwen3_fp8_generation_matches_oracle():
+    _check_against_oracle(QWEN_SMALL, True, 5e-2, 3e-2, 2e-2)
+
+
+@pytest.mark.parametrize("w", [TINY, TINY_BF16, QWEN_SMALL], ids=["fp32", "bf16", "qwen3-bf16"])
+def test_generation_eps_zero_is_symmetric(w):
+    batch = wl.make_batch(w, fg_rows=0)
+    B = len(batch.prompts)
+    _, h = gpu_handle(w, max_new=G)
+    h.zo_probe_plan(0, 0.0)
+    Lp, Lm, gt, gl = h.zo_generate(dev_tokens(batch), batch.seq_lens, G)
+    assert torch.equal(gt[:B], gt[B:]) and torch.equal(gl[:B], gl[B:]) and torch.equal(Lp, Lm)
+
+
+@pytest.mark.parametrize("w,tol", [(TINY, 1e-4), (QWEN_SMALL, 2e-2)], ids=["fp32", "qwen3-bf16"])
+def test_decode_agrees_with_prefill_scoring_of_the_generated_rows(w, tol):
+    """The KV-cache decode path and the packed prefill path give the same log-probs for the
+    generated tokens (the + rows scored under the + candidate as target spans)."""
+    batch = wl.make_batch(w, fg_rows=0)
+    B = len(batch.prompts)
+    _, h = gpu_handle(w, max_new=G)
+    h.zo_probe_plan(0, w.eps)
+    _, _, gt, gl = h.zo_generate(dev_tokens(batch), batch.seq_lens, G)
+    gt_h = gt.cpu().numpy()
+    rows = [np.concatenate([p, gt_h[r]]).astype(np.int32) for r, p in enumerate(batch.prompts)]
+    full = wl.Batch(rows, np.full(B, G, dtype=np.int32), [], np.zeros(0, dtype=np.int32))
+    _, h2 = gpu_handle(dataclasses.replace(w, len_hi=w.len_hi + G, tgt_hi=G), max_new=0, batch=B)
+    h2.zo_probe_plan(0, w.eps)
+    _, _, lp = h2.zo_score(dev_tokens(full), full.seq_lens, full.target_lens, want_logprob=True)
+    plus = lp[:B * G].cpu().numpy().reshape(B, G)
+    assert np.max(np.abs(plus - gl[:B].cpu().numpy())) <= tol
+
+
+def test_generation_argument_checks():
+    from zeroth_order_fine_b200 import zo
+    w = TINY
+    batch = wl.make_batch(w, fg_rows=0)
+    toks = dev_tokens(batch)
+    _, h0 = gpu_handle(w)
+    h0.zo_probe_plan(0, w.eps)
+    with pytest.raises(zo.ZoError) as e:
+        h0.zo_generate(toks, batch.seq_lens, 2)
+    assert e.value.code == zo.ZO_ERR_UNSUPPORTED
+    _, h = gpu_handle(w, max_new=4)
+    h.zo_probe_plan(0, w.eps)
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_generate(toks, batch.seq_lens, 5)
+    assert e.value.code == zo.ZO_ERR_ARG

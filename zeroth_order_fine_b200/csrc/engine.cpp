@@ -27,6 +27,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <string>
 #include <vector>
 
@@ -115,6 +116,12 @@ struct zo_handle {
     void* ext = nullptr;          // shrink output S (model dtype) [max_tokens x kcap]
     int kcap = 0;                 // columns of FT rows / EB / ext allocated
     void* hs = nullptr;           // scored hidden states
+    // generation queries (options.max_new > 0)
+    void* kv_cache = nullptr;     // per layer [kv_rows x 2 kv_dim] in the model dtype
+    size_t kv_rows = 0;
+    int* part_arg = nullptr;      // LSE partials: argmax column per (row, tile)
+    int *gen_tok = nullptr, *gen_last = nullptr, *gen_lens = nullptr;
+    float* gen_lp = nullptr;
     float *pmax = nullptr, *psum = nullptr, *tgt = nullptr, *logprob = nullptr;
     int lse_tiles = 0;
     double* L_row = nullptr;
@@ -448,6 +455,7 @@ int check_desc(const zo_model_desc* d, const zo_weights* w, const zo_options* o)
     if (o->impl != 0 && o->impl != 1) return 1;
     if (o->profile != 0 && o->profile != 1) return 1;
     if (o->fp8 != 0 && o->fp8 != 1) return 1;
+    if (o->max_new < 0 || o->max_new > 4096) return 1;
     if (o->fp8 && (d->dtype != ZO_DTYPE_BF16 || o->impl != 0 || !norm_fp8_supported(d->d_model) ||
                    d->d_model % 16 || (d->n_heads + 2 * d->n_kv_heads) * d->head_dim <= 128 ||
                    d->d_ffn <= 64))
@@ -642,7 +650,18 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
     if (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused)
         CRC(dev_alloc(h, &h->gu, (size_t)maxT * ffn_cols * es));
     if (h->kcap) CRC(dev_alloc(h, &h->ext, (size_t)maxT * h->kcap * es));
-    CRC(dev_alloc(h, &h->hs, (size_t)maxS * d.d_model * es));
+    // scored rows: the target positions of a score, or one row per candidate of a generation
+    const int maxSR = options->max_new > 0 ? std::max(maxS, maxR) : maxS;
+    CRC(dev_alloc(h, &h->hs, (size_t)maxSR * d.d_model * es));
+    if (options->max_new > 0) {
+        h->kv_rows = (size_t)maxT + (size_t)maxR * options->max_new;
+        CRC(dev_alloc(h, &h->kv_cache,
+                      (size_t)d.n_layers * h->kv_rows * 2 * h->kv_dim * es));
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_tok), (size_t)maxR * options->max_new * 4));
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_lp), (size_t)maxR * options->max_new * 4));
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_last), (size_t)maxR * 4));
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_lens), (size_t)maxR * 4));
+    }
     if (d.arch == ZO_ARCH_QWEN3) {
         const size_t n = (size_t)d.max_pos * (d.head_dim / 2);
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->rope_cos), n * 4));
@@ -651,9 +670,11 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
                           h->st);
     }
     h->lse_tiles = gemm_lse_col_tiles(d.vocab);
-    CRC(dev_alloc(h, reinterpret_cast<void**>(&h->pmax), (size_t)maxS * h->lse_tiles * 4));
-    CRC(dev_alloc(h, reinterpret_cast<void**>(&h->psum), (size_t)maxS * h->lse_tiles * 4));
-    CRC(dev_alloc(h, reinterpret_cast<void**>(&h->tgt), (size_t)maxS * 4));
+    CRC(dev_alloc(h, reinterpret_cast<void**>(&h->pmax), (size_t)maxSR * h->lse_tiles * 4));
+    CRC(dev_alloc(h, reinterpret_cast<void**>(&h->psum), (size_t)maxSR * h->lse_tiles * 4));
+    CRC(dev_alloc(h, reinterpret_cast<void**>(&h->tgt), (size_t)maxSR * 4));
+    if (options->max_new > 0)
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->part_arg), (size_t)maxSR * h->lse_tiles * 4));
     CRC(dev_alloc(h, reinterpret_cast<void**>(&h->logprob), (size_t)maxS * 4));
     CRC(dev_alloc(h, reinterpret_cast<void**>(&h->L_row), (size_t)maxR * 8));
     for (int** p : {&h->tok_id, &h->tok_pos, &h->tok_sign, &h->tok_row})
@@ -888,6 +909,97 @@ int prepare_batch(zo_handle* h, int B, const int32_t* lens, const int32_t* tls,
 // Every kernel of one score over a batch laid out by prepare_batch, whose metadata
 // is already in device memory at md.  Enqueues only (no host synchronisation), so
 // it can be captured into a CUDA graph.
+// One fused GEMM group of a layer over Ti token rows: the bank shrink (when the group
+// carries targets) and the base GEMM with the extension K blocks, epilogue epi.
+int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc, int ctype,
+               int Ti, float eps, const Layer* Lq = nullptr) {
+    const zo_model_desc& d = h->desc;
+    const int r_ = h->opt.rank;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    if (epi == EPI_QKNR) {
+        g.tok_pos = h->tok_pos; g.qn = Lq->w.q_norm; g.kn = Lq->w.k_norm;
+        g.rope_cos = h->rope_cos; g.rope_sin = h->rope_sin; g.norm_eps = d.norm_eps;
+        g.n_q_heads = d.n_heads; g.n_qk_heads = d.n_heads + d.n_kv_heads;
+    }
+    g.M = Ti;
+    if (G.n_t > 0) {
+        // live extension columns, padded to a multiple of 8 (16-byte TMA rows); the
+        // padding columns of S and E_B are zero
+        const int kext = (G.n_t * r_ * (1 + h->n_slots) + 7) / 8 * 8;
+        GemmArgs s;
+        memset(&s, 0, sizeof(s));
+        s.A = X; s.lda = G.K; s.a_type = h->dt;
+        if (G.FTb) { s.B = G.FTb; s.b_type = E_BF16; }
+        else { s.B = G.FT; s.b_type = E_F32; }
+        s.ldb = G.K;
+        s.M = Ti; s.N = kext; s.K = G.K;
+        s.epi = EPI_SHRINK;
+        s.C = h->ext; s.ldc = h->kcap; s.c_type = h->dt;
+        s.row_sign = h->tok_sign; s.eps = eps; s.scale_cols = G.n_t * r_;
+        if (G.Wq) s.a_scale = h->sx;      // S / s_x: the base GEMM accumulates in E4M3 units
+        int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
+        if (rc) return rc;
+        g.A2 = h->ext; g.lda2 = h->kcap; g.a2_type = h->dt;
+        g.B2 = G.EB; g.ldb2 = h->kcap; g.b2_type = h->dt;
+        g.K2 = kext;
+    }
+    g.A = X; g.lda = G.K; g.a_type = h->dt;
+    g.B = G.W; g.ldb = G.K; g.b_type = h->dt;
+    if (G.Wq) {
+        // E4M3 rows of the same norm output and of W; dequantised in the epilogue
+        g.A = h->xq; g.a_type = E_FP8;
+        g.B = G.Wq; g.b_type = E_FP8;
+        g.a_scale = h->sx; g.b_scale = G.sw;
+    }
+    g.N = G.N; g.K = G.K;
+    g.bias = G.bias;
+    g.epi = epi;
+    g.C = C; g.ldc = ldc; g.c_type = ctype;
+    // algorithmic work: the base GEMM plus, per target, its own expand columns
+    double fl = 2.0 * Ti * (double)G.N * G.K;
+    for (int t = 0; t < G.n_t; ++t) fl += 2.0 * Ti * (double)G.d_out[t] * r_ * (1 + h->n_slots);
+    return run_gemm(h, g, fl);
+}
+
+// Every decoder layer over the Ti token rows whose ids, positions, signs and embeddings are
+// in place (h->tok_*, h->resid).  attn(l) enqueues layer l's attention: it reads the q|k|v
+// rows in h->qkv (q/k normalised and rotated for Qwen3) and writes h->att.
+int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)>& attn) {
+    const zo_model_desc& d = h->desc;
+    const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
+    for (int l = 0; l < d.n_layers; ++l) {
+        Layer& L = h->layers[l];
+        launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps, h->xn,
+                    h->dt, h->st, h->xq, h->sx);
+        int rc = group_gemm(h, L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
+                            h->n_qkv, h->dt, Ti, eps, &L);
+        if (rc) return rc;
+        if (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused)
+            launch_qk_norm_rope(h->qkv, h->n_qkv, h->dt, h->tok_pos, Ti, d.n_heads, d.n_kv_heads,
+                                d.head_dim, L.w.q_norm, L.w.k_norm, d.norm_eps, h->rope_cos,
+                                h->rope_sin, h->st);
+        rc = attn(l);
+        if (rc) return rc;
+        rc = group_gemm(h, L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps);
+        if (rc) return rc;
+        launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps, h->xn,
+                    h->dt, h->st, h->xq, h->sx);
+        if (d.arch == ZO_ARCH_OPT) {
+            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt, Ti, eps);
+        } else if (h->swiglu_fused) {
+            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_SWIGLU, h->act, d.d_ffn, h->dt, Ti, eps);
+        } else {
+            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE, h->gu, 2 * d.d_ffn, h->dt, Ti, eps);
+            if (!rc) launch_swiglu(h->gu, Ti, d.d_ffn, h->act, h->dt, h->st);
+        }
+        if (rc) return rc;
+        rc = group_gemm(h, L.g[G_OUT], h->act, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps);
+        if (rc) return rc;
+    }
+    return ZO_OK;
+}
+
 int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
                  const int32_t* ptok, const int32_t* ftok, const int32_t* tgt_ids) {
     const zo_model_desc& d = h->desc;
@@ -914,96 +1026,23 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
                  d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
                  d.d_model, h->st);
 
-    const int r_ = h->opt.rank;
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
-    auto group_gemm = [&](Group& G, const void* X, int epi, void* C, int ldc, int ctype,
-                          const Layer* Lq = nullptr) -> int {
-        GemmArgs g;
-        memset(&g, 0, sizeof(g));
-        if (epi == EPI_QKNR) {
-            g.tok_pos = h->tok_pos; g.qn = Lq->w.q_norm; g.kn = Lq->w.k_norm;
-            g.rope_cos = h->rope_cos; g.rope_sin = h->rope_sin; g.norm_eps = d.norm_eps;
-            g.n_q_heads = d.n_heads; g.n_qk_heads = d.n_heads + d.n_kv_heads;
-        }
-        g.M = Ti;
-        if (G.n_t > 0) {
-            // live extension columns, padded to a multiple of 8 (16-byte TMA rows); the
-            // padding columns of S and E_B are zero
-            const int kext = (G.n_t * r_ * (1 + h->n_slots) + 7) / 8 * 8;
-            GemmArgs s;
-            memset(&s, 0, sizeof(s));
-            s.A = X; s.lda = G.K; s.a_type = h->dt;
-            if (G.FTb) { s.B = G.FTb; s.b_type = E_BF16; }
-            else { s.B = G.FT; s.b_type = E_F32; }
-            s.ldb = G.K;
-            s.M = Ti; s.N = kext; s.K = G.K;
-            s.epi = EPI_SHRINK;
-            s.C = h->ext; s.ldc = h->kcap; s.c_type = h->dt;
-            s.row_sign = h->tok_sign; s.eps = eps; s.scale_cols = G.n_t * r_;
-            if (G.Wq) s.a_scale = h->sx;      // S / s_x: the base GEMM accumulates in E4M3 units
-            int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
-            if (rc) return rc;
-            g.A2 = h->ext; g.lda2 = h->kcap; g.a2_type = h->dt;
-            g.B2 = G.EB; g.ldb2 = h->kcap; g.b2_type = h->dt;
-            g.K2 = kext;
-        }
-        g.A = X; g.lda = G.K; g.a_type = h->dt;
-        g.B = G.W; g.ldb = G.K; g.b_type = h->dt;
-        if (G.Wq) {
-            // E4M3 rows of the same norm output and of W; dequantised in the epilogue
-            g.A = h->xq; g.a_type = E_FP8;
-            g.B = G.Wq; g.b_type = E_FP8;
-            g.a_scale = h->sx; g.b_scale = G.sw;
-        }
-        g.N = G.N; g.K = G.K;
-        g.bias = G.bias;
-        g.epi = epi;
-        g.C = C; g.ldc = ldc; g.c_type = ctype;
-        // algorithmic work: the base GEMM plus, per target, its own expand columns
-        double fl = 2.0 * Ti * (double)G.N * G.K;
-        for (int t = 0; t < G.n_t; ++t) fl += 2.0 * Ti * (double)G.d_out[t] * r_ * (1 + h->n_slots);
-        return run_gemm(h, g, fl);
-    };
-
-    for (int l = 0; l < d.n_layers; ++l) {
-        Layer& L = h->layers[l];
-        launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps, h->xn,
-                    h->dt, h->st, h->xq, h->sx);
-        int rc = group_gemm(L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
-                            h->n_qkv, h->dt, &L);
-        if (rc) return rc;
-        if (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused)
-            launch_qk_norm_rope(h->qkv, h->n_qkv, h->dt, h->tok_pos, Ti, d.n_heads, d.n_kv_heads,
-                                d.head_dim, L.w.q_norm, L.w.k_norm, d.norm_eps, h->rope_cos,
-                                h->rope_sin, h->st);
-        AttnArgs a;
-        memset(&a, 0, sizeof(a));
-        a.qkv = h->qkv; a.ld_qkv = h->n_qkv;
-        a.out = h->att; a.ld_out = h->q_dim;
-        a.dtype = h->dt;
-        a.cu_seqlens = m.cu_seqlens;
-        a.tiles = tiles_d; a.n_tiles = nt;
-        a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
-        a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
-        a.n_tokens = Ti;
-        if (tc_attn && attention_tc_supported(a)) launch_attention_tc(a, h->st);
-        else launch_attention(a, h->st);
-        rc = group_gemm(L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32);
-        if (rc) return rc;
-        launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps, h->xn,
-                    h->dt, h->st, h->xq, h->sx);
-        if (d.arch == ZO_ARCH_OPT) {
-            rc = group_gemm(L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt);
-        } else if (h->swiglu_fused) {
-            rc = group_gemm(L.g[G_IN], h->xn, EPI_SWIGLU, h->act, d.d_ffn, h->dt);
-        } else {
-            rc = group_gemm(L.g[G_IN], h->xn, EPI_STORE, h->gu, 2 * d.d_ffn, h->dt);
-            if (!rc) launch_swiglu(h->gu, Ti, d.d_ffn, h->act, h->dt, h->st);
-        }
-        if (rc) return rc;
-        rc = group_gemm(L.g[G_OUT], h->act, EPI_RESID, h->resid, d.d_model, E_F32);
-        if (rc) return rc;
-    }
+    int rc = decoder_layers(h, Ti, eps, [&](int l) -> int {
+            AttnArgs a;
+            memset(&a, 0, sizeof(a));
+            a.qkv = h->qkv; a.ld_qkv = h->n_qkv;
+            a.out = h->att; a.ld_out = h->q_dim;
+            a.dtype = h->dt;
+            a.cu_seqlens = m.cu_seqlens;
+            a.tiles = tiles_d; a.n_tiles = nt;
+            a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
+            a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
+            a.n_tokens = Ti;
+            if (tc_attn && attention_tc_supported(a)) launch_attention_tc(a, h->st);
+            else launch_attention(a, h->st);
+            return ZO_OK;
+        });
+    if (rc) return rc;
     // scored positions: gather + final norm, then lm_head with log-sum-exp
     launch_norm(h->resid, h->sc_tok, Si, d.d_model, nk, h->wts.final_w, h->wts.final_b,
                 d.norm_eps, h->hs, h->dt, h->st);
@@ -1031,6 +1070,126 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
     h->stats.tokens_scored += (uint64_t)T;
     h->stats.positions_scored += (uint64_t)S;
     h->stats.score_calls++;
+    CK(h, cudaGetLastError());
+    return ZO_OK;
+}
+
+// lm_head over M rows of h->hs with the LSE epilogue recording each tile's argmax, then
+// the greedy choice per row into tok[r * stride], lp[r * stride].
+int lm_head_greedy(zo_handle* h, int M, int* tok, float* lp, int stride) {
+    const zo_model_desc& d = h->desc;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.A = h->hs; g.lda = d.d_model; g.a_type = h->dt;
+    g.B = d.tie_lm_head ? h->wts.tok_embed : h->wts.lm_head; g.ldb = d.d_model; g.b_type = h->dt;
+    g.M = M; g.N = d.vocab; g.K = d.d_model;
+    g.epi = EPI_LSE;
+    g.targets = h->gen_last;            // any valid ids: the target logit is not used here
+    g.part_max = h->pmax; g.part_sum = h->psum; g.tgt_logit = h->tgt; g.part_arg = h->part_arg;
+    const bool tc = h->use_tc && gemm_tc_supported(g);
+    g.n_col_tiles = tc ? gemm_tc_col_tiles(d.vocab) : h->lse_tiles;
+    if (tc) {
+        if (gemm_tc(g, h->st)) FAIL(h, ZO_ERR_CUDA, "tcgen05 lm_head launch failed");
+    } else {
+        gemm_simt(g, h->st);
+        h->stats.cuda_core_gemm_launches++;
+    }
+    launch_lse_argmax_merge(h->pmax, h->psum, h->part_arg, M, g.n_col_tiles, tok, lp, stride,
+                            h->st);
+    h->stats.kernel_launches += 2;
+    return ZO_OK;
+}
+
+// Generation queries: packed prefill into the KV cache, then greedy decode steps.
+int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int32_t* lens,
+                  int G) {
+    const zo_model_desc& d = h->desc;
+    const int R = 2 * B;
+    std::vector<int> tls(B, 1);
+    CK(h, cudaEventSynchronize(h->meta_ev));
+    BatchPlan bp;
+    int rc = prepare_batch(h, B, lens, tls.data(), nullptr, 0, nullptr, nullptr, h->meta_h, &bp);
+    if (rc) return rc;
+    if ((size_t)bp.T + (size_t)R * G > h->kv_rows) FAIL(h, ZO_ERR_ARG, "generation exceeds the KV cache");
+    CK(h, cudaMemcpyAsync(h->meta, h->meta_h, bp.nints * 4, cudaMemcpyHostToDevice, h->st));
+    CK(h, cudaEventRecord(h->meta_ev, h->st));
+    const int* md = h->meta;
+    RowMeta m;
+    m.cu_seqlens = md;
+    m.row_src = md + (R + 1);
+    m.row_is_fg = m.row_src + R;
+    m.row_sign = m.row_is_fg + R;
+    m.score_off = m.row_sign + R;
+    const int* chk_d = m.score_off + (R + 1);
+    const int* tiles_d = chk_d + R;
+    const int Ti = (int)bp.T, nt = bp.nt;
+    const int kv2 = 2 * h->kv_dim;
+    const size_t layer_elems = h->kv_rows * (size_t)kv2;
+    const size_t es = esize(h->dt);
+    auto cache = [&](int l) { return static_cast<char*>(h->kv_cache) + (size_t)l * layer_elems * es; };
+    const bool tc_attn = h->use_tc && h->dt == E_BF16 && d.head_dim == 128;
+    const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;
+    const float scale = (float)(1.0 / std::sqrt((double)d.head_dim));
+
+    // prefill: the prompts of both candidates as one packed batch, k|v kept per layer
+    launch_build_tokens(m, R, ptok, nullptr, h->tok_id, h->tok_pos, h->tok_sign, h->tok_row,
+                        h->sc_tok, h->sc_tgt, nullptr, nullptr, chk_d, h->err_dev, h->st);
+    launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
+                 d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
+                 d.d_model, h->st);
+    rc = decoder_layers(h, Ti, eps, [&](int l) -> int {
+        launch_kv_scatter(h->qkv, h->n_qkv, h->q_dim, kv2, h->tok_row, Ti, G, cache(l), h->dt,
+                          h->st);
+        AttnArgs a;
+        memset(&a, 0, sizeof(a));
+        a.qkv = h->qkv; a.ld_qkv = h->n_qkv;
+        a.out = h->att; a.ld_out = h->q_dim;
+        a.dtype = h->dt;
+        a.cu_seqlens = m.cu_seqlens;
+        a.tiles = tiles_d; a.n_tiles = nt;
+        a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
+        a.scale = scale;
+        a.n_tokens = Ti;
+        if (tc_attn && attention_tc_supported(a)) launch_attention_tc(a, h->st);
+        else launch_attention(a, h->st);
+        h->stats.kernel_launches += 2;
+        return ZO_OK;
+    });
+    if (rc) return rc;
+    launch_last_tokens(md, R, h->gen_last, h->gen_lens, h->st);
+    launch_norm(h->resid, h->gen_last, R, d.d_model, nk, h->wts.final_w, h->wts.final_b,
+                d.norm_eps, h->hs, h->dt, h->st);
+    rc = lm_head_greedy(h, R, h->gen_tok, h->gen_lp, G);
+    if (rc) return rc;
+    h->stats.kernel_launches += 4 + (uint64_t)d.n_layers * (2 + (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused) +
+                                                             (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused));
+    h->stats.tokens_scored += (uint64_t)Ti;
+
+    // decode: token g of every row at position len + g, attending over its row's cache
+    for (int g = 0; g + 1 < G; ++g) {
+        launch_decode_prep(h->gen_tok, G, g, h->gen_lens, R, B, h->tok_id, h->tok_pos,
+                           h->tok_sign, h->tok_row, h->st);
+        launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
+                     d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, R,
+                     d.d_model, h->st);
+        rc = decoder_layers(h, R, eps, [&](int l) -> int {
+            launch_kv_append(h->qkv, h->n_qkv, h->q_dim, kv2, md, h->gen_lens, R, g, G, cache(l),
+                             h->dt, h->st);
+            launch_decode_attention(h->qkv, h->n_qkv, cache(l), kv2, md, h->gen_lens, R, g, G,
+                                    d.n_heads, d.n_kv_heads, d.head_dim, scale, h->att, h->q_dim,
+                                    h->dt, h->st);
+            h->stats.kernel_launches += 2;
+            return ZO_OK;
+        });
+        if (rc) return rc;
+        launch_norm(h->resid, nullptr, R, d.d_model, nk, h->wts.final_w, h->wts.final_b,
+                    d.norm_eps, h->hs, h->dt, h->st);
+        rc = lm_head_greedy(h, R, h->gen_tok + g + 1, h->gen_lp + g + 1, G);
+        if (rc) return rc;
+        h->stats.kernel_launches += 3 + (uint64_t)d.n_layers * (2 + (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused) +
+                                                                 (d.arch == ZO_ARCH_QWEN3 && !h->swiglu_fused));
+        h->stats.tokens_scored += (uint64_t)R;
+    }
     CK(h, cudaGetLastError());
     return ZO_OK;
 }
@@ -1108,6 +1267,40 @@ int zo_score_cobatch(zo_plan* plan, const int32_t* packed_tokens, int32_t n_prom
     return score_common(plan, h, packed_tokens, n_prompts, seq_lens, target_lens, target_ids,
                         L_plus, L_minus, tok_logprob, fg_tokens, n_fg, fg_seq_lens,
                         fg_target_lens, fg_tok_logprob);
+}
+
+int zo_generate(zo_plan* plan, const int32_t* packed_tokens, int32_t n_prompts,
+                const int32_t* seq_lens, int32_t n_new, int32_t* gen_tokens,
+                float* gen_logprob, float* L_plus, float* L_minus) {
+    if (!plan || !plan->h) return ZO_ERR_ARG;
+    zo_handle* h = plan->h;
+    if (!h->have_plan || plan != &h->plan) FAIL(h, ZO_ERR_STATE, "stale plan");
+    if (h->opt.max_new < 1) FAIL(h, ZO_ERR_UNSUPPORTED, "generation needs options.max_new >= 1");
+    if (n_prompts < 1 || !packed_tokens || !seq_lens) FAIL(h, ZO_ERR_ARG, "missing generation arguments");
+    if (n_new < 1 || n_new > h->opt.max_new) FAIL(h, ZO_ERR_ARG, "n_new outside 1..max_new");
+    if (2 * n_prompts > h->opt.max_rows) FAIL(h, ZO_ERR_ARG, "more rows than max_rows");
+    for (int i = 0; i < n_prompts; ++i)
+        if (seq_lens[i] < 2 || (long long)seq_lens[i] + n_new > h->desc.max_pos)
+            FAIL(h, ZO_ERR_ARG, "seq_len must be >= 2 and seq_len + n_new <= max_pos");
+    timer_begin(h, 1);
+    int rc = generate_impl(h, plan->eps, packed_tokens, n_prompts, seq_lens, n_new);
+    if (rc) { timer_end(h, 1); return rc; }
+    const int R = 2 * n_prompts;
+    launch_gen_objective(h->gen_lp, R, n_prompts, n_new, h->L_row, L_plus, L_minus, h->st);
+    if (gen_tokens)
+        CK(h, cudaMemcpyAsync(gen_tokens, h->gen_tok, (size_t)R * n_new * 4,
+                              cudaMemcpyDeviceToDevice, h->st));
+    if (gen_logprob)
+        CK(h, cudaMemcpyAsync(gen_logprob, h->gen_lp, (size_t)R * n_new * 4,
+                              cudaMemcpyDeviceToDevice, h->st));
+    timer_end(h, 1);
+    h->stats.kernel_launches++;
+    h->stats.positions_scored += (uint64_t)R * n_new;
+    h->stats.score_calls++;
+    plan->scored = true;
+    plan->B = n_prompts;
+    CK(h, cudaGetLastError());
+    return ZO_OK;
 }
 
 int zo_score_foreground(zo_handle* h, const int32_t* fg_tokens, int32_t n_fg,

@@ -80,10 +80,19 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
                 if (n0 + tx * 4 + j < g.N) s += expf(v[j] - mx);
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            int arg = 0x7fffffff;                  // lowest column holding the tile max
+            if (g.part_arg) {
+#pragma unroll
+                for (int j = 3; j >= 0; --j)
+                    if (n0 + tx * 4 + j < g.N && v[j] == mx) arg = n0 + tx * 4 + j;
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) arg = min(arg, __shfl_xor_sync(0xffffffffu, arg, o));
+            }
             if (m < g.M) {
                 if (tx == 0) {
                     g.part_max[(size_t)m * g.n_col_tiles + blockIdx.x] = mx;
                     g.part_sum[(size_t)m * g.n_col_tiles + blockIdx.x] = s;
+                    if (g.part_arg) g.part_arg[(size_t)m * g.n_col_tiles + blockIdx.x] = arg;
                 }
                 const int tgt = g.targets[m] - (n0 + tx * 4);
                 if (tgt >= 0 && tgt < 4) g.tgt_logit[m] = v[tgt];

@@ -73,6 +73,7 @@ struct TcParams {
     const float* bias;
     void* C; int ldc; int c_type;
     const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
+    int* part_arg;
     const int* row_sign; float eps; int scale_cols;
     const int* tok_pos; const float* qn; const float* kn;
     const float* rope_cos; const float* rope_sin; float norm_eps;
@@ -197,13 +198,21 @@ __device__ __forceinline__ void tile_coords(int t, const TcParams& p, int* mb, i
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, float* v,
-                                               float* run_max, float* run_sum) {
+                                               float* run_max, float* run_sum, int* run_arg) {
     const bool row_ok = m < p.M;
     if (EPI == EPI_LSE) {
         float mx = -FLT_MAX;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
             if (n + j < p.N) mx = fmaxf(mx, v[j]);
+        if (p.part_arg && mx > *run_max) {
+            // the lowest column of this chunk that holds its maximum
+            int a = n;
+#pragma unroll
+            for (int j = 31; j >= 0; --j)
+                if (n + j < p.N && v[j] == mx) a = n + j;
+            *run_arg = a;
+        }
         const float nm = fmaxf(*run_max, mx);
         float s = 0.f;
 #pragma unroll
@@ -484,6 +493,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const int m = mb * BM + lane_base + lane;
             float run_max = -FLT_MAX, run_sum = 0.f;
+            int run_arg = nb * BNT;
             if (EPI == EPI_SWIGLU)
                 epilogue_swiglu(p, m, nb, tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BNT));
             else
@@ -492,11 +502,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (n >= p.N) break;                // whole chunk past N (warp-uniform)
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BNT + c * 32), v);
-                epilogue_chunk<EPI>(p, m, n, v, &run_max, &run_sum);
+                epilogue_chunk<EPI>(p, m, n, v, &run_max, &run_sum, &run_arg);
             }
             if (EPI == EPI_LSE && m < p.M) {
                 p.part_max[(size_t)m * p.n_col_tiles + nb] = run_max;
                 p.part_sum[(size_t)m * p.n_col_tiles + nb] = run_sum;
+                if (p.part_arg) p.part_arg[(size_t)m * p.n_col_tiles + nb] = run_arg;
             }
             tc_fence_before();
             __syncwarp();
@@ -1254,6 +1265,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.C = g.C; p.ldc = g.ldc; p.c_type = g.c_type;
     p.targets = g.targets; p.part_max = g.part_max; p.part_sum = g.part_sum;
     p.tgt_logit = g.tgt_logit; p.n_col_tiles = g.n_col_tiles;
+    p.part_arg = g.part_arg;
     p.row_sign = g.row_sign; p.eps = g.eps; p.scale_cols = g.scale_cols;
     p.tok_pos = g.tok_pos; p.qn = g.qn; p.kn = g.kn;
     p.rope_cos = g.rope_cos; p.rope_sin = g.rope_sin; p.norm_eps = g.norm_eps;

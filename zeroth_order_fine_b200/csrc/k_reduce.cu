@@ -42,6 +42,40 @@ void launch_lse_merge(const float* part_max, const float* part_sum, const float*
                                                  logprob);
 }
 
+__global__ void lse_argmax_merge_kernel(const float* __restrict__ pmax, const float* __restrict__ psum,
+                                        const int* __restrict__ parg, int S, int n_tiles,
+                                        int* __restrict__ token, float* __restrict__ logprob,
+                                        int stride) {
+    const int s = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (s >= S) return;
+    const float* pm = pmax + (size_t)s * n_tiles;
+    const float* ps = psum + (size_t)s * n_tiles;
+    float m = -FLT_MAX;
+    for (int i = lane; i < n_tiles; i += 32) m = fmaxf(m, pm[i]);
+    m = warp_max(m);
+    int first = 0x7fffffff;                  // the lowest tile holding the maximum
+    for (int i = lane; i < n_tiles; i += 32)
+        if (pm[i] == m) first = min(first, i);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    float z = 0.f;
+    for (int i = lane; i < n_tiles; i += 32) z += ps[i] * expf(pm[i] - m);
+    z = warp_sum(z);
+    if (lane == 0) {
+        token[(size_t)s * stride] = parg[(size_t)s * n_tiles + first];
+        logprob[(size_t)s * stride] = m - (m + logf(z));
+    }
+}
+
+void launch_lse_argmax_merge(const float* part_max, const float* part_sum, const int* part_arg,
+                             int S, int n_tiles, int* token, float* logprob, int stride,
+                             cudaStream_t st) {
+    if (S == 0) return;
+    lse_argmax_merge_kernel<<<cdiv(S, 8), 256, 0, st>>>(part_max, part_sum, part_arg, S, n_tiles,
+                                                        token, logprob, stride);
+}
+
 __global__ void row_objective_kernel(const float* __restrict__ logprob,
                                      const int* __restrict__ score_off, int R, int B,
                                      double* __restrict__ L_row, float* L_plus, float* L_minus) {

@@ -96,8 +96,9 @@ struct GemmArgs {
     void* C; int ldc; int c_type;
     // EPI_SHRINK
     const int* row_sign; float eps; int scale_cols;
-    // EPI_LSE
+    // EPI_LSE (part_arg optional: per (row, column tile) the lowest column of the tile max)
     const int* targets; float* part_max; float* part_sum; float* tgt_logit; int n_col_tiles;
+    int* part_arg;
     // E_FP8 operands: dequantisation scales per row of A [M] and of B [N]; the epilogue
     // multiplies the accumulator by a_scale[m] * b_scale[n] (the extension operands must
     // be pre-divided accordingly).  EPI_SHRINK with a_scale divides its output rows by it.
@@ -140,6 +141,36 @@ int attention_tc_error_word();
 // ---- objective, estimator, update ------------------------------------------------------
 void launch_lse_merge(const float* part_max, const float* part_sum, const float* tgt_logit,
                       int S, int n_tiles, float* logprob, cudaStream_t st);
+// Greedy choice per row from the LSE partials: token = the lowest column holding the
+// largest logit, logprob = that logit - logsumexp; written at row * stride.
+void launch_lse_argmax_merge(const float* part_max, const float* part_sum, const int* part_arg,
+                             int S, int n_tiles, int* token, float* logprob, int stride,
+                             cudaStream_t st);
+
+// ---- generation queries (KV cache) --------------------------------------------------------
+// Cache layout per layer: [rows of (k | v)], row r's tokens at cu[r] + r * G + p, where cu
+// are the prompt offsets and G the new tokens per row; a cache row is 2 * kv_dim wide.
+// Prefill: copy each token's k|v columns of the packed q|k|v rows into the cache.
+void launch_kv_scatter(const void* qkv, int ld_qkv, int q_dim, int kv2, const int* tok_row,
+                       int T, int G, void* cache, int dtype, cudaStream_t st);
+// Decode step g (g >= 0): row r's new token sits at prompt length + g.
+void launch_decode_prep(const int* gen_tok, int G, int g, const int* lens, int R, int B,
+                        int* tok_id, int* tok_pos, int* tok_sign, int* tok_row, cudaStream_t st);
+void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int* cu,
+                      const int* lens, int R, int g, int G, void* cache, int dtype,
+                      cudaStream_t st);
+// One query per row (its q heads in qkv row r) against the row's n = lens[r] + g + 1 cached
+// keys; softmax(q k^T * scale) v into out [R x H*hd].  CUDA cores (memory-bound).
+void launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int kv2,
+                             const int* cu, const int* lens, int R, int g, int G, int H, int Hkv,
+                             int hd, float scale, void* out, int ld_out, int dtype,
+                             cudaStream_t st);
+// Last prompt token of each row (the hidden state that predicts the first new token) and
+// the rows' prompt lengths.
+void launch_last_tokens(const int* cu, int R, int* out, int* lens, cudaStream_t st);
+// Generation objective: L_row[r] = -mean_g logprob[r * G + g] (fp64, fixed order); L+/L-.
+void launch_gen_objective(const float* logprob, int R, int B, int G, double* L_row,
+                          float* L_plus, float* L_minus, cudaStream_t st);
 // per row L = -mean(logprob over its span) (fp64); L+/L- copies for the probe rows.
 void launch_row_objective(const float* logprob, const int* score_off, int R, int B,
                           double* L_row, float* L_plus, float* L_minus, cudaStream_t st);

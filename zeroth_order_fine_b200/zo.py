@@ -66,7 +66,8 @@ class zo_options(ctypes.Structure):
     _fields_ = [("run_seed", c_uint64), ("lazy_interval", c_int32), ("rank", c_int32),
                 ("targets", zo_targets), ("max_tokens", c_int32), ("max_rows", c_int32),
                 ("max_scored", c_int32), ("max_slots", c_int32), ("start_step", c_uint64),
-                ("stream", c_void_p), ("impl", c_int32), ("profile", c_int32), ("fp8", c_int32)]
+                ("stream", c_void_p), ("impl", c_int32), ("profile", c_int32), ("fp8", c_int32),
+                ("max_new", c_int32)]
 
 
 class zo_stats_t(ctypes.Structure):
@@ -101,6 +102,8 @@ _SIGS = {
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
                                    c_void_p, c_void_p]),
     "zo_score_foreground": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
+    "zo_generate": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_int32, c_void_p, c_void_p,
+                              c_void_p, c_void_p]),
     "zo_step": (c_int32, [c_void_p, ctypes.c_float, c_void_p]),
     "zo_step_graph": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, ctypes.c_float,
                                 ctypes.c_float, c_void_p, c_void_p]),
@@ -281,7 +284,7 @@ class Handle:
     def __init__(self, model: DeviceModel, run_seed: int, nu: int, rank: int,
                  targets: zo_targets, max_tokens: int, max_rows: int, max_scored: int,
                  max_slots: int = 32, start_step: int = 0, stream=None, impl: int = 0,
-                 profile: int = 0, fp8: int = 0):
+                 profile: int = 0, fp8: int = 0, max_new: int = 0):
         self.model = model
         self.targets = targets
         self.rank = rank
@@ -289,7 +292,7 @@ class Handle:
         self._desc = model.desc()
         self._w = model.weights()
         opt = zo_options(run_seed, nu, rank, targets, max_tokens, max_rows, max_scored, max_slots,
-                         start_step, _stream(self.stream), impl, profile, fp8)
+                         start_step, _stream(self.stream), impl, profile, fp8, max_new)
         h = c_void_p()
         rc = lib().zo_create(ctypes.byref(self._desc), ctypes.byref(self._w), ctypes.byref(opt),
                              ctypes.byref(h))
@@ -344,6 +347,19 @@ class Handle:
                                       _ptr(Lp), _ptr(Lm), _ptr(lp), _ptr(fg_tokens), F,
                                       _ptr(fsl), _ptr(ftl), _ptr(flp)), self.h)
         return Lp, Lm, lp, flp
+
+    # zo_generate: greedy generation queries of both candidates
+    def zo_generate(self, tokens, seq_lens, n_new: int):
+        sl = _i32(seq_lens)
+        B = len(sl)
+        dev = tokens.device
+        Lp = torch.empty(B, dtype=torch.float32, device=dev)
+        Lm = torch.empty(B, dtype=torch.float32, device=dev)
+        gt = torch.empty(2 * B, n_new, dtype=torch.int32, device=dev)
+        gl = torch.empty(2 * B, n_new, dtype=torch.float32, device=dev)
+        _check(lib().zo_generate(self.plan, _ptr(tokens), B, _ptr(sl), n_new, _ptr(gt), _ptr(gl),
+                                 _ptr(Lp), _ptr(Lm)), self.h)
+        return Lp, Lm, gt, gl
 
     # zo_score_foreground
     def zo_score_foreground(self, fg_tokens, fg_seq_lens, fg_target_lens):
