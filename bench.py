@@ -322,6 +322,68 @@ def run_kernel(args):
 
 # ---- the CUDA path ------------------------------------------------------------------
 
+def run_generate(args, w: wl.Workload):
+    """Generation-query steps (zo_probe_plan + zo_generate + zo_step) on one GPU: greedy
+    decoding of --generate tokens per candidate row with the KV cache."""
+    import torch
+
+    from zeroth_order_fine_b200 import zo
+    G = args.generate
+    sh = w.shape
+    batch = wl.make_batch(w, fg_rows=0)
+    model = zo.DeviceModel(sh, w.weight_seed)
+    tg = zo.make_targets(sh.n_layers, w.matrices, w.scale_mode)
+    T = batch.n_tokens_physical
+    B = len(batch.prompts)
+    h = zo.Handle(model, w.run_seed, w.nu, w.rank, tg, max_tokens=T, max_rows=2 * B,
+                  max_scored=2 * B, max_slots=8, fp8=1 if args.fp8 else 0, max_new=G)
+    toks = torch.from_numpy(batch.packed()).cuda()
+    t = [0]
+
+    def step():
+        h.zo_probe_plan(t[0], w.eps)
+        h.zo_generate(toks, batch.seq_lens, G)
+        h.zo_step(w.lr, want_c=False)
+        t[0] += 1
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, peak_kind = load_peaks()
+    es = 2 if sh.dtype == wl.DTYPE_BF16 else 4
+    # prefill: the scoring step's FLOPs at its own roofline; every decode step reads the
+    # weights (and lm_head) once and each row's cache once
+    flops, _, _, _ = step_work(w, [batch], 1)
+    w_bytes = (sh.body_params() + sh.vocab * sh.d_model) * es
+    kv_row = 2 * sh.kv_dim * sh.n_layers * es
+    lens = np.concatenate([batch.seq_lens, batch.seq_lens]).astype(np.float64)
+    kv_bytes = sum(float(np.sum(lens + g + 1)) * kv_row for g in range(G - 1))
+    t_prefill = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_decode = ((G - 1) * w_bytes + kv_bytes) / (peaks["hbm_gbs"] * 1e9)
+    roof_ms = (t_prefill + t_decode) * 1000.0
+    s = h.zo_stats()
+    print(json.dumps({
+        "mode": "generate", "workload": w.name, "new_tokens_per_row": G, "rows": 2 * B,
+        "prompt_tokens": T, "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+        "generated_tokens_per_s": 2 * B * G / (ms / 1000.0),
+        "dtype": "e4m3 (q|k|v, FFN-in) + bf16" if args.fp8 else "bf16",
+        "roofline": {"prefill_ms": t_prefill * 1000.0, "decode_ms": t_decode * 1000.0,
+                     "roofline_ms": roof_ms, "frac": roof_ms / ms,
+                     "peak": f"{peak_kind} bf16 {peaks['bf16_tflops_sustained']} TFLOP/s sustained "
+                             f"(prefill), HBM {peaks['hbm_gbs']} GB/s (decode: weights + cache "
+                             f"once per token)"},
+        "last_error_code": s["last_error_code"]}), flush=True)
+    h.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -333,6 +395,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the whole-step CUDA graph leg")
+    ap.add_argument("--generate", type=int, default=0,
+                    help="generation-query steps: greedy tokens per candidate row (zo_generate)")
     ap.add_argument("--fp8", action="store_true",
                     help="E4M3 base products for q|k|v and the FFN input (zo_options.fp8)")
     ap.add_argument("--cuda-cores", action="store_true", help="GEMMs on CUDA cores only")
@@ -353,6 +417,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.generate:
+        return run_generate(args, w)
 
     import torch
     import torch.distributed as dist

@@ -912,7 +912,7 @@ int prepare_batch(zo_handle* h, int B, const int32_t* lens, const int32_t* tls,
 // One fused GEMM group of a layer over Ti token rows: the bank shrink (when the group
 // carries targets) and the base GEMM with the extension K blocks, epilogue epi.
 int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc, int ctype,
-               int Ti, float eps, const Layer* Lq = nullptr) {
+               int Ti, float eps, const Layer* Lq = nullptr, bool decode = false) {
     const zo_model_desc& d = h->desc;
     const int r_ = h->opt.rank;
     GemmArgs g;
@@ -938,8 +938,16 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
         s.C = h->ext; s.ldc = h->kcap; s.c_type = h->dt;
         s.row_sign = h->tok_sign; s.eps = eps; s.scale_cols = G.n_t * r_;
         if (G.Wq) s.a_scale = h->sx;      // S / s_x: the base GEMM accumulates in E4M3 units
-        int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
-        if (rc) return rc;
+        if (decode) {
+            // a decode step's handful of rows: a CUDA-core dot per (row, factor column)
+            // beats one tensor-core CTA walking the whole K range
+            launch_shrink_rows(s.A, s.a_type, s.B, s.b_type, Ti, kext, G.K, s.C, s.ldc, s.c_type,
+                               s.row_sign, eps, s.scale_cols, s.a_scale, h->st);
+            h->stats.kernel_launches++;
+        } else {
+            int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
+            if (rc) return rc;
+        }
         g.A2 = h->ext; g.lda2 = h->kcap; g.a2_type = h->dt;
         g.B2 = G.EB; g.ldb2 = h->kcap; g.b2_type = h->dt;
         g.K2 = kext;
@@ -965,7 +973,8 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
 // Every decoder layer over the Ti token rows whose ids, positions, signs and embeddings are
 // in place (h->tok_*, h->resid).  attn(l) enqueues layer l's attention: it reads the q|k|v
 // rows in h->qkv (q/k normalised and rotated for Qwen3) and writes h->att.
-int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)>& attn) {
+int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)>& attn,
+                   bool decode = false) {
     const zo_model_desc& d = h->desc;
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
     for (int l = 0; l < d.n_layers; ++l) {
@@ -973,7 +982,7 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps, h->xn,
                     h->dt, h->st, h->xq, h->sx);
         int rc = group_gemm(h, L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
-                            h->n_qkv, h->dt, Ti, eps, &L);
+                            h->n_qkv, h->dt, Ti, eps, &L, decode);
         if (rc) return rc;
         if (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused)
             launch_qk_norm_rope(h->qkv, h->n_qkv, h->dt, h->tok_pos, Ti, d.n_heads, d.n_kv_heads,
@@ -981,20 +990,20 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
                                 h->rope_sin, h->st);
         rc = attn(l);
         if (rc) return rc;
-        rc = group_gemm(h, L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps);
+        rc = group_gemm(h, L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr, decode);
         if (rc) return rc;
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps, h->xn,
                     h->dt, h->st, h->xq, h->sx);
         if (d.arch == ZO_ARCH_OPT) {
-            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt, Ti, eps);
+            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt, Ti, eps, nullptr, decode);
         } else if (h->swiglu_fused) {
-            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_SWIGLU, h->act, d.d_ffn, h->dt, Ti, eps);
+            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_SWIGLU, h->act, d.d_ffn, h->dt, Ti, eps, nullptr, decode);
         } else {
-            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE, h->gu, 2 * d.d_ffn, h->dt, Ti, eps);
+            rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE, h->gu, 2 * d.d_ffn, h->dt, Ti, eps, nullptr, decode);
             if (!rc) launch_swiglu(h->gu, Ti, d.d_ffn, h->act, h->dt, h->st);
         }
         if (rc) return rc;
-        rc = group_gemm(h, L.g[G_OUT], h->act, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps);
+        rc = group_gemm(h, L.g[G_OUT], h->act, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr, decode);
         if (rc) return rc;
     }
     return ZO_OK;
@@ -1180,7 +1189,7 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
                                     h->dt, h->st);
             h->stats.kernel_launches += 2;
             return ZO_OK;
-        });
+        }, true);
         if (rc) return rc;
         launch_norm(h->resid, nullptr, R, d.d_model, nk, h->wts.final_w, h->wts.final_b,
                     d.norm_eps, h->hs, h->dt, h->st);

@@ -6,7 +6,8 @@
 // once as a packed prefill whose k|v rows are kept per layer, then every new token is one
 // row of a decode step that attends over its own row's cache.  Everything is memory-bound
 // (a decode step reads every weight once for all rows and each row's cache once), so these
-// kernels are plain 16-byte copies and CUDA-core reductions; the GEMMs stay on tcgen05.
+// kernels are plain 16-byte copies and coalesced CUDA-core reductions; the GEMMs stay on
+// tcgen05.
 #include <float.h>
 
 #include "common.cuh"
@@ -57,98 +58,125 @@ __global__ void kv_append_kernel(const char* __restrict__ qkv, int ld_qkv, int q
     copy_row(qkv + ((size_t)r * ld_qkv + q_dim) * es, cache + crow * kv2 * es, kv2, es);
 }
 
-// One CTA per (row, kv head): the n_rep query heads that share the kv head, keys streamed in
-// chunks of 128 (one key per thread for the scores, one dimension per thread for P V), with
-// an online softmax across chunks in fp32.
-constexpr int DEC_THREADS = 128, DEC_CHUNK = 128, DEC_MAX_REP = 8, DEC_MAX_HD = 256;
+// One CTA per (row, kv head): the n_rep query heads that share the kv head.  Each warp takes
+// every 4th key; its 32 lanes split the head dimension (hd / 32 consecutive elements each), so
+// a key's k and v rows are read as one coalesced warp access.  Per warp an online softmax
+// (fp32) over its keys, then the four warps' partial results are merged.
+constexpr int DEC_WARPS = 4, DEC_MAX_REP = 8, DEC_MAX_DPL = 8;      // hd <= 256
 
-__global__ void __launch_bounds__(DEC_THREADS) decode_attention_kernel(
+template <int DPL>
+__device__ __forceinline__ void load_dims(const void* base, size_t off, int dtype, float* v) {
+    if (dtype == E_F32) {
+        const float* p = static_cast<const float*>(base) + off;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) v[i] = p[i];
+    } else {
+        const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(base) + off;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) v[i] = __bfloat162float(p[i]);
+    }
+}
+
+template <int DPL>
+__global__ void __launch_bounds__(DEC_WARPS * 32) decode_attention_kernel(
     const void* __restrict__ qkv, int ld_qkv, const void* __restrict__ cache, int kv2,
-    const int* __restrict__ cu, const int* __restrict__ lens, int g, int G, int H, int Hkv, int hd,
+    const int* __restrict__ cu, const int* __restrict__ lens, int g, int G, int H, int Hkv,
     float scale, void* __restrict__ out, int ld_out, int dtype) {
-    __shared__ float qs[DEC_MAX_REP][DEC_MAX_HD];
-    __shared__ float ps[DEC_MAX_REP][DEC_CHUNK];
-    __shared__ float red[32];
-    __shared__ float m_sh[DEC_MAX_REP], l_sh[DEC_MAX_REP], a_sh[DEC_MAX_REP];
+    constexpr int HD = DPL * 32;
+    __shared__ float sm_m[DEC_WARPS][DEC_MAX_REP], sm_l[DEC_WARPS][DEC_MAX_REP];
+    __shared__ float sm_o[DEC_WARPS][DEC_MAX_REP][HD];
     const int r = blockIdx.x, kvh = blockIdx.y;
     const int n_rep = H / Hkv;
-    const int tid = threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t base = (size_t)cu[r] + (size_t)r * G;
     const int n = lens[r] + g + 1;
     const int kv_dim = kv2 / 2;
-    for (int i = tid; i < n_rep * hd; i += DEC_THREADS) {
-        const int hh = i / hd, dd = i % hd;
-        qs[hh][dd] = ld_elem(qkv, (size_t)r * ld_qkv + (size_t)(kvh * n_rep + hh) * hd + dd, dtype);
-    }
-    if (tid < n_rep) {
-        m_sh[tid] = -FLT_MAX;
-        l_sh[tid] = 0.f;
-    }
-    float acc[DEC_MAX_REP][2];
+    const int d0 = lane * DPL;
+    float q[DEC_MAX_REP][DPL], o[DEC_MAX_REP][DPL], m[DEC_MAX_REP], l[DEC_MAX_REP];
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAX_REP; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
+    for (int hh = 0; hh < DEC_MAX_REP; ++hh) {
+        m[hh] = -FLT_MAX;
+        l[hh] = 0.f;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) o[hh][i] = q[hh][i] = 0.f;
+        if (hh < n_rep)
+            load_dims<DPL>(qkv, (size_t)r * ld_qkv + (size_t)(kvh * n_rep + hh) * HD + d0, dtype,
+                           q[hh]);
+    }
+    for (int j = warp; j < n; j += DEC_WARPS) {
+        const size_t kr = (base + j) * kv2 + (size_t)kvh * HD + d0;
+        float k[DPL], v[DPL];
+        load_dims<DPL>(cache, kr, dtype, k);
+        load_dims<DPL>(cache, kr + kv_dim, dtype, v);
+#pragma unroll
+        for (int hh = 0; hh < DEC_MAX_REP; ++hh) {
+            if (hh >= n_rep) break;
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) s = fmaf(q[hh][i], k[i], s);
+            s = warp_sum(s) * scale;
+            const float m_new = fmaxf(m[hh], s);
+            const float alpha = m[hh] > -FLT_MAX ? expf(m[hh] - m_new) : 0.f;
+            const float p = expf(s - m_new);
+            l[hh] = l[hh] * alpha + p;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) o[hh][i] = fmaf(p, v[i], o[hh][i] * alpha);
+            m[hh] = m_new;
+        }
+    }
+#pragma unroll
+    for (int hh = 0; hh < DEC_MAX_REP; ++hh) {
+        if (hh >= n_rep) break;
+        if (lane == 0) {
+            sm_m[warp][hh] = m[hh];
+            sm_l[warp][hh] = l[hh];
+        }
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) sm_o[warp][hh][d0 + i] = o[hh][i];
+    }
     __syncthreads();
-    for (int c0 = 0; c0 < n; c0 += DEC_CHUNK) {
-        const int j = c0 + tid;
-        // scores of this thread's key for every query head of the group
-        float sc[DEC_MAX_REP];
-#pragma unroll
-        for (int hh = 0; hh < DEC_MAX_REP; ++hh) sc[hh] = -FLT_MAX;
-        if (j < n) {
-            const size_t kb = (base + j) * kv2 + (size_t)kvh * hd;
-            for (int hh = 0; hh < n_rep; ++hh) sc[hh] = 0.f;
-            for (int dd = 0; dd < hd; ++dd) {
-                const float kv = ld_elem(cache, kb + dd, dtype);
-#pragma unroll
-                for (int hh = 0; hh < DEC_MAX_REP; ++hh)
-                    if (hh < n_rep) sc[hh] = fmaf(qs[hh][dd], kv, sc[hh]);
-            }
-#pragma unroll
-            for (int hh = 0; hh < DEC_MAX_REP; ++hh)
-                if (hh < n_rep) sc[hh] *= scale;
+    // merge the warps' partial softmaxes in a fixed order
+    for (int idx = threadIdx.x; idx < n_rep * HD; idx += DEC_WARPS * 32) {
+        const int hh = idx / HD, dd = idx % HD;
+        float mm = -FLT_MAX;
+        for (int w = 0; w < DEC_WARPS; ++w) mm = fmaxf(mm, sm_m[w][hh]);
+        float ll = 0.f, acc = 0.f;
+        for (int w = 0; w < DEC_WARPS; ++w) {
+            const float f = sm_m[w][hh] > -FLT_MAX ? expf(sm_m[w][hh] - mm) : 0.f;
+            ll += sm_l[w][hh] * f;
+            acc += sm_o[w][hh][dd] * f;
         }
-        for (int hh = 0; hh < n_rep; ++hh) {
-            const float cmax = block_max(sc[hh], red);
-            const float m_old = m_sh[hh];
-            const float m_new = fmaxf(m_old, cmax);
-            const float p = j < n ? expf(sc[hh] - m_new) : 0.f;
-            ps[hh][tid] = p;
-            const float csum = block_sum(p, red);
-            if (tid == 0) {
-                const float alpha = m_old > -FLT_MAX ? expf(m_old - m_new) : 0.f;
-                a_sh[hh] = alpha;
-                l_sh[hh] = l_sh[hh] * alpha + csum;
-                m_sh[hh] = m_new;
-            }
-        }
-        __syncthreads();
-        const int nk = min(DEC_CHUNK, n - c0);
-        for (int dd0 = 0; dd0 < 2; ++dd0) {
-            const int dd = tid + dd0 * DEC_THREADS;
-            if (dd >= hd) continue;
-            float part[DEC_MAX_REP];
-#pragma unroll
-            for (int hh = 0; hh < DEC_MAX_REP; ++hh) part[hh] = 0.f;
-            for (int jj = 0; jj < nk; ++jj) {
-                const float v = ld_elem(cache, (base + c0 + jj) * kv2 + kv_dim + (size_t)kvh * hd + dd,
-                                        dtype);
-#pragma unroll
-                for (int hh = 0; hh < DEC_MAX_REP; ++hh)
-                    if (hh < n_rep) part[hh] = fmaf(ps[hh][jj], v, part[hh]);
-            }
-#pragma unroll
-            for (int hh = 0; hh < DEC_MAX_REP; ++hh)
-                if (hh < n_rep) acc[hh][dd0] = acc[hh][dd0] * a_sh[hh] + part[hh];
-        }
-        __syncthreads();                       // ps and a_sh are rewritten by the next chunk
+        st_elem(out, (size_t)r * ld_out + (size_t)(kvh * n_rep + hh) * HD + dd, dtype,
+                ll > 0.f ? acc / ll : 0.f);
     }
-    for (int dd0 = 0; dd0 < 2; ++dd0) {
-        const int dd = tid + dd0 * DEC_THREADS;
-        if (dd >= hd) continue;
-        for (int hh = 0; hh < n_rep; ++hh) {
-            const float inv = l_sh[hh] > 0.f ? 1.f / l_sh[hh] : 0.f;
-            st_elem(out, (size_t)r * ld_out + (size_t)(kvh * n_rep + hh) * hd + dd, dtype,
-                    acc[hh][dd0] * inv);
+}
+
+// grid (ceil(N / 8), M): one row against 8 factor rows, K split over the block (512
+// threads, four K steps in flight per thread)
+__global__ void __launch_bounds__(512) shrink_rows_kernel(
+    const void* __restrict__ x, int x_type, const void* __restrict__ FT, int ft_type, int N, int K,
+    void* __restrict__ C, int ldc, int c_type, const int* __restrict__ row_sign, float eps,
+    int scale_cols, const float* __restrict__ a_scale) {
+    __shared__ float red[32];
+    const int m = blockIdx.y, j0 = blockIdx.x * 8;
+    float acc[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.f;
+#pragma unroll 4
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        const float xv = ld_elem(x, (size_t)m * K + k, x_type);
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+            if (j0 + jj < N) acc[jj] = fmaf(xv, ld_elem(FT, (size_t)(j0 + jj) * K + k, ft_type), acc[jj]);
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+        const float v = block_sum(acc[jj], red);
+        const int j = j0 + jj;
+        if (threadIdx.x == 0 && j < N) {
+            float y = j < scale_cols ? v * ((float)row_sign[m] * eps) : v;
+            if (a_scale) y = y / a_scale[m];
+            st_elem(C, (size_t)m * ldc + j, c_type, y);
         }
     }
 }
@@ -202,10 +230,24 @@ void launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
                              const int* cu, const int* lens, int R, int g, int G, int H, int Hkv,
                              int hd, float scale, void* out, int ld_out, int dtype,
                              cudaStream_t st) {
-    if (R == 0 || H / Hkv > DEC_MAX_REP || hd > DEC_MAX_HD) return;
+    if (R == 0 || H / Hkv > DEC_MAX_REP || hd % 32 || hd / 32 > DEC_MAX_DPL) return;
     dim3 grid(R, Hkv);
-    decode_attention_kernel<<<grid, DEC_THREADS, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G,
-                                                          H, Hkv, hd, scale, out, ld_out, dtype);
+    switch (hd / 32) {
+        case 1: decode_attention_kernel<1><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
+        case 2: decode_attention_kernel<2><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
+        case 4: decode_attention_kernel<4><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
+        case 8: decode_attention_kernel<8><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
+        default: break;
+    }
+}
+
+void launch_shrink_rows(const void* x, int x_type, const void* FT, int ft_type, int M, int N,
+                        int K, void* C, int ldc, int c_type, const int* row_sign, float eps,
+                        int scale_cols, const float* a_scale, cudaStream_t st) {
+    if (M == 0 || N == 0) return;
+    dim3 grid(cdiv(N, 8), M);
+    shrink_rows_kernel<<<grid, 512, 0, st>>>(x, x_type, FT, ft_type, N, K, C, ldc, c_type,
+                                             row_sign, eps, scale_cols, a_scale);
 }
 
 void launch_last_tokens(const int* cu, int R, int* out, int* lens, cudaStream_t st) {

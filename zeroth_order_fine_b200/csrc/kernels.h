@@ -165,6 +165,12 @@ void launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
                              const int* cu, const int* lens, int R, int g, int G, int H, int Hkv,
                              int hd, float scale, void* out, int ld_out, int dtype,
                              cudaStream_t st);
+// Bank shrink for a few rows (decode steps), on CUDA cores: C[m, j] = (x[m] . FT[j]) *
+// (j < scale_cols ? row_sign[m] * eps : 1) / (a_scale ? a_scale[m] : 1); x [M x K] in
+// x_type, FT [N x K] in ft_type, C [M x ldc] in c_type.
+void launch_shrink_rows(const void* x, int x_type, const void* FT, int ft_type, int M, int N,
+                        int K, void* C, int ldc, int c_type, const int* row_sign, float eps,
+                        int scale_cols, const float* a_scale, cudaStream_t st);
 // Last prompt token of each row (the hidden state that predicts the first new token) and
 // the rows' prompt lengths.
 void launch_last_tokens(const int* cu, int R, int* out, int* lens, cudaStream_t st);
