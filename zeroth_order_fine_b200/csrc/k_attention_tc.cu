@@ -187,8 +187,9 @@ __global__ void __launch_bounds__(128, 2)
     uint8_t* KPb = g + BUF;
     uint8_t* Vb = g + 2 * BUF;
     const uint32_t bar_mma = base + 3 * BUF;
-    const uint32_t bar_ld = bar_mma + 8;
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 3 * BUF + 16);
+    const uint32_t bar_ld = bar_mma + 8;               // Q and K of a chunk
+    const uint32_t bar_v = bar_mma + 16;               // V of a chunk: lands under QK^T + softmax
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 3 * BUF + 32);
 
     const Item it = get_item(a, blockIdx.x);
     const int q_dim = a.H * HD, kv_dim = a.Hkv * HD;
@@ -198,6 +199,7 @@ __global__ void __launch_bounds__(128, 2)
     if (tid == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ld));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_v));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -213,8 +215,8 @@ __global__ void __launch_bounds__(128, 2)
     const uint32_t tmem = *tslot;
     const uint32_t t_s = tmem, t_o = tmem + 128;
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    uint32_t ph_mma = 0, ph_ld = 0;
-    bool ok = true;
+    uint32_t ph_mma = 0, ph_ld = 0, ph_v = 0;
+    bool ok = true, v_pending = false;
     const int q = it.q0 + tid;                         // this thread's query
     const float sl2 = a.scale * 1.4426950408889634f;
     const int kcol = q_dim + it.kvh * HD, vcol = q_dim + kv_dim + it.kvh * HD;
@@ -224,9 +226,12 @@ __global__ void __launch_bounds__(128, 2)
         const int c0 = c * TK;
         // K and V of chunk c (and Q with the first): rows past the tensor read as zero
         if (tid == 0) {
-            const uint32_t bytes = (uint32_t)BUF * (c == 0 ? 3u : 2u);
+            const uint32_t bytes = (uint32_t)BUF * (c == 0 ? 2u : 1u);
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_ld),
                          "r"(bytes)
+                         : "memory");
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_v),
+                         "r"((uint32_t)BUF)
                          : "memory");
             const int r0 = it.start + c0;
             for (int half = 0; half < 2; ++half) {
@@ -234,9 +239,11 @@ __global__ void __launch_bounds__(128, 2)
                     tma_box(smem_u32(Qb) + half * ATOM, &tm, bar_ld, it.h * HD + half * 64,
                             it.start + it.q0);
                 tma_box(smem_u32(KPb) + half * ATOM, &tm, bar_ld, kcol + half * 64, r0);
-                tma_box(smem_u32(Vb) + half * ATOM, &tm, bar_ld, vcol + half * 64, r0);
             }
+            for (int half = 0; half < 2; ++half)
+                tma_box(smem_u32(Vb) + half * ATOM, &tm, bar_v, vcol + half * 64, r0);
         }
+        v_pending = true;
         ok = __syncthreads_and(wait_bar(bar_ld, ph_ld, err));
         ph_ld ^= 1u;
         if (!ok) break;
@@ -313,10 +320,13 @@ __global__ void __launch_bounds__(128, 2)
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         }
 
-        // O (+)= P V
+        // O (+)= P V, once V has landed
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
+        ok = __syncthreads_and(wait_bar(bar_v, ph_v, err));
+        if (!ok) break;
+        ph_v ^= 1u;
+        v_pending = false;
         if (tid == 0) {
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll
@@ -357,6 +367,20 @@ __global__ void __launch_bounds__(128, 2)
                                                  pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
                                                  pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
             }
+        }
+    }
+    if (v_pending && tid == 0) {
+        // an aborted CTA lets its V copy land before its shared memory goes away
+        const long long t0 = clock64();
+        for (;;) {
+            uint32_t done;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(done)
+                : "r"(bar_v), "r"(ph_v)
+                : "memory");
+            if (done || clock64() - t0 > WAIT_CYCLES) break;
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");

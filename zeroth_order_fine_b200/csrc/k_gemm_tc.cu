@@ -18,7 +18,8 @@
 //               accumulator, fused bias / ReLU / residual add / SwiGLU / LSE;
 //               the SM-pair kernel hands its tiles to TMA stores (reduce-add for
 //               the residual stream) through swizzled shared-memory staging
-// Tiles are walked in M-groups of 8 so concurrent CTAs share B strips in L2.
+// Tiles are walked in M-groups (8 blocks single-SM, 12 for SM pairs) so concurrent CTAs
+// share B strips in L2.
 // Every mbarrier wait is bounded: on expiry the kernel records
 // ZO_TC_TIMEOUT in the error word, drains what it issued and returns.
 #include <cuda.h>
@@ -78,8 +79,7 @@ struct TcParams {
     const int* tok_pos; const float* qn; const float* kn;
     const float* rope_cos; const float* rope_sin; float norm_eps;
     int n_q_heads, n_qk_heads;
-    int fp8;                                // main K blocks are E4M3 (SM-pair kernel)
-    const float* a_scale; const float* b_scale;
+    const float* a_scale; const float* b_scale;   // E4M3 dequantisation (F8 kernels)
     int* err;
 };
 
@@ -663,7 +663,7 @@ __device__ __forceinline__ void dequant_chunk(const TcParams& p, int m, int n, f
 // residual stream an fp32 reduce-add, so the SM never reads the residual.  Two
 // staging buffers per warp alternate; a buffer is rewritten only after the TMA
 // has read it.
-template <int EPI>
+template <int EPI, bool F8>
 __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMap* tmC,
                                              uint32_t stg, uint8_t* stg_ptr, int& buf, int m_base,
                                              int nb, uint32_t taddr, int lane) {
@@ -711,7 +711,7 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
                 float gv[32], uv[32];
                 tmem_ld32(taddr + (uint32_t)((c + h) * 32), gv);
                 tmem_ld32(taddr + (uint32_t)(128 + (c + h) * 32), uv);
-                if (p.a_scale) {
+                if (F8) {
                     dequant_chunk<32>(p, m_base + r, nb * 256 + (c + h) * 32, gv);
                     dequant_chunk<32>(p, m_base + r, nb * 256 + 128 + (c + h) * 32, uv);
                 }
@@ -753,7 +753,7 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
                 for (int c = 0; c < 4; ++c) {
                     float v[32];
                     tmem_ld32(th + (uint32_t)(c * 32), v);
-                    if (p.a_scale) dequant_chunk<32>(p, m, n0 + c * 32, v);
+                    if (F8) dequant_chunk<32>(p, m, n0 + c * 32, v);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float x = __bfloat162float(__float2bfloat16_rn(v[j]));
@@ -769,7 +769,7 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
                 float lo[32], hi[32];
                 tmem_ld32(th + (uint32_t)(c * 32), lo);
                 tmem_ld32(th + (uint32_t)(64 + c * 32), hi);
-                if (p.a_scale) {
+                if (F8) {
                     dequant_chunk<32>(p, m, n0 + c * 32, lo);
                     dequant_chunk<32>(p, m, n0 + 64 + c * 32, hi);
                 }
@@ -827,7 +827,7 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
             float y[64];
             tmem_ld32(taddr + (uint32_t)(c * 32), y);
             tmem_ld32(taddr + (uint32_t)((c + 1) * 32), y + 32);
-            if (p.a_scale) dequant_chunk<64>(p, m_base + r, n, y);
+            if (F8) dequant_chunk<64>(p, m_base + r, n, y);
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
                 float v = y[j];
@@ -857,7 +857,9 @@ __device__ __forceinline__ void tile_coords2(int t, const TcParams& p, int* mb, 
     *nb = in / gm;
 }
 
-template <int EPI>
+// F8: the main K blocks are E4M3 (kind::f8f6f4) and the epilogue dequantises; a separate
+// instantiation, so the bf16 kernels carry none of it.
+template <int EPI, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2,
@@ -928,7 +930,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (rank == 0) mbar_expect_tx(full(s), 2 * STAGE2_BYTES);
                     const uint32_t lb = map_rank(full(s), 0);
                     if (kb < p.kb_main) {
-                        const int k = kb * (p.fp8 ? BK8 : BK);
+                        const int k = kb * (F8 ? BK8 : BK);
                         tma_load_2d_pair(sa, &tmA, lb, k, row_a);
                         tma_load_2d_pair(sb, &tmB, lb, k, row_b);
                     } else {
@@ -966,7 +968,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     tc_fence_after();
                     const uint32_t sa = base + s * STAGE2_BYTES;
                     const uint32_t sb = sa + A2B;
-                    if (p.fp8 && kb < p.kb_main) {
+                    if (F8 && kb < p.kb_main) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             tc_mma_pair_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
@@ -1009,7 +1011,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
             tc_fence_after();
             const int m_base = mb * BM2 + (int)rank * 128 + lane_base;
-            epilogue_tma<EPI>(p, &tmC, stg, stg_ptr, buf, m_base, nb,
+            epilogue_tma<EPI, F8>(p, &tmC, stg, stg_ptr, buf, m_base, nb,
                               tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN), lane);
             tc_fence_before();
             __syncwarp();
@@ -1132,12 +1134,12 @@ int launch_epi_w(int bnt, const CUtensorMap& a, const CUtensorMap& b, const CUte
     }
 }
 
-template <int EPI>
+template <int EPI, bool F8>
 int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                 const CUtensorMap& b2, const CUtensorMap& c, const TcParams& p, cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(gemm_tc2_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_tc2_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SMEM2_BYTES) != cudaSuccess)
             return 1;
         attr = true;
@@ -1155,13 +1157,13 @@ int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a
         cfg.attrs = at;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<EPI>, &cfg) != cudaSuccess || n <= 0)
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<EPI, F8>, &cfg) != cudaSuccess || n <= 0)
             n = num_sms() / 2;
         max_pairs = n;
     }
     int pairs = max_pairs;
     if (p.n_tiles < pairs) pairs = p.n_tiles;
-    gemm_tc2_kernel<EPI><<<2 * pairs, NUM_THREADS, SMEM2_BYTES, st>>>(a, b, a2, b2, c, p);
+    gemm_tc2_kernel<EPI, F8><<<2 * pairs, NUM_THREADS, SMEM2_BYTES, st>>>(a, b, a2, b2, c, p);
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
 
@@ -1246,18 +1248,14 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     memset(&p, 0, sizeof(p));
     p.M = g.M; p.N = g.N;
     p.kb_main = f8 ? (g.K + BK8 - 1) / BK8 : (g.K + BK - 1) / BK;
-    p.fp8 = f8 ? 1 : 0;
     p.a_scale = g.a_scale; p.b_scale = g.b_scale;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
     p.n_m_blk = pair ? (g.M + BM2 - 1) / BM2 : (g.M + BM - 1) / BM;
-    // Raster: an M group whose A strips (256 rows x K) fit in ~48 MB of L2 sweeps all N
-    // blocks, so each weight strip is fetched from DRAM once per group.
-    {
-        const double strip = (double)BM2 * ((double)g.K * (f8 ? 1.0 : 2.0) + g.K2 * 2.0);
-        int gm = (int)(48.0e6 / strip);
-        gm = gm < 4 ? 4 : (gm > 32 ? 32 : gm);
-        p.group_m = pair ? gm : GROUP_M;
-    }
+    // Raster: the SM pairs walk M groups of 12 blocks of 256 rows, each sweeping every N
+    // block, so a weight strip is fetched once per group while the group's A strips stay in
+    // L2.  12 was the fastest of 4..24 for both the fc1 (K = 5120) and fc2 (K = 20480) shapes
+    // of the OPT-13B step, timed on B200 under the power cap.
+    p.group_m = pair ? 12 : GROUP_M;
     p.n_n_blk = (g.N + bnt - 1) / bnt;
     p.n_tiles = p.n_m_blk * p.n_n_blk;
     p.epi = g.epi;
@@ -1280,11 +1278,19 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
         const uint64_t cols = g.epi == EPI_SWIGLU ? (uint64_t)(g.N / 2) : (uint64_t)g.N;
         if (!make_map_out(&c, g.C, (uint64_t)g.M, cols, (uint64_t)g.ldc, f32)) return 1;
         switch (g.epi) {
-            case EPI_STORE: return launch_epi2<EPI_STORE>(a, b, a2, b2, c, p, st);
-            case EPI_STORE_RELU: return launch_epi2<EPI_STORE_RELU>(a, b, a2, b2, c, p, st);
-            case EPI_RESID: return launch_epi2<EPI_RESID>(a, b, a2, b2, c, p, st);
-            case EPI_SWIGLU: return launch_epi2<EPI_SWIGLU>(a, b, a2, b2, c, p, st);
-            case EPI_QKNR: return launch_epi2<EPI_QKNR>(a, b, a2, b2, c, p, st);
+            case EPI_STORE:
+                return f8 ? launch_epi2<EPI_STORE, true>(a, b, a2, b2, c, p, st)
+                          : launch_epi2<EPI_STORE, false>(a, b, a2, b2, c, p, st);
+            case EPI_STORE_RELU:
+                return f8 ? launch_epi2<EPI_STORE_RELU, true>(a, b, a2, b2, c, p, st)
+                          : launch_epi2<EPI_STORE_RELU, false>(a, b, a2, b2, c, p, st);
+            case EPI_RESID: return f8 ? 1 : launch_epi2<EPI_RESID, false>(a, b, a2, b2, c, p, st);
+            case EPI_SWIGLU:
+                return f8 ? launch_epi2<EPI_SWIGLU, true>(a, b, a2, b2, c, p, st)
+                          : launch_epi2<EPI_SWIGLU, false>(a, b, a2, b2, c, p, st);
+            case EPI_QKNR:
+                return f8 ? launch_epi2<EPI_QKNR, true>(a, b, a2, b2, c, p, st)
+                          : launch_epi2<EPI_QKNR, false>(a, b, a2, b2, c, p, st);
             default: return 1;
         }
     }
