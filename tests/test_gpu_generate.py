@@ -58,6 +58,14 @@ def test_tiny_fp32_generation_matches_oracle(impl):
     _check_against_oracle(TINY, False, 1e-4, 1e-4, 1e-4, impl=impl)
 
 
+def test_opt_width_bf16_generation_matches_oracle():
+    """Two full-width OPT-1.3B layers (d = 2048, vocab 50272): the decode GEMMs have few
+    output tiles for their 8 rows and split K over the SM pairs."""
+    w = wl.WORKLOADS["opt-1.3b-b16"]
+    w = dataclasses.replace(w, shape=wl.shrink_shape(w.shape, n_layers=2), batch=4, len_hi=48)
+    _check_against_oracle(w, False, 5e-2, 3e-2, 2e-2)
+
+
 def test_tiny_bf16_generation_matches_oracle():
     _check_against_oracle(TINY_BF16, False, 5e-2, 3e-2, 2e-2)
 
@@ -80,7 +88,13 @@ def test_generation_eps_zero_is_symmetric(w):
     assert torch.equal(gt[:B], gt[B:]) and torch.equal(gl[:B], gl[B:]) and torch.equal(Lp, Lm)
 
 
-@pytest.mark.parametrize("w,tol", [(TINY, 1e-4), (QWEN_SMALL, 2e-2)], ids=["fp32", "qwen3-bf16"])
+OPT_WIDTH = dataclasses.replace(wl.WORKLOADS["opt-1.3b-b16"],
+                                shape=wl.shrink_shape(wl.WORKLOADS["opt-1.3b-b16"].shape, n_layers=2),
+                                batch=4, len_hi=48)
+
+
+@pytest.mark.parametrize("w,tol", [(TINY, 1e-4), (QWEN_SMALL, 2e-2), (OPT_WIDTH, 2e-2)],
+                         ids=["fp32", "qwen3-bf16", "opt-width-bf16"])
 def test_decode_agrees_with_prefill_scoring_of_the_generated_rows(w, tol):
     """The KV-cache decode path and the packed prefill path give the same log-probs for the
     generated tokens (the + rows scored under the + candidate as target spans)."""

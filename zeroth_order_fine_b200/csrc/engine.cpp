@@ -120,6 +120,8 @@ struct zo_handle {
     void* kv_cache = nullptr;     // per layer [kv_rows x 2 kv_dim] in the model dtype
     size_t kv_rows = 0;
     int* part_arg = nullptr;      // LSE partials: argmax column per (row, tile)
+    float* splitk_ws = nullptr;   // decode GEMMs' split-K slices
+    size_t splitk_floats = 0;
     int *gen_tok = nullptr, *gen_last = nullptr, *gen_lens = nullptr;
     float* gen_lp = nullptr;
     float *pmax = nullptr, *psum = nullptr, *tgt = nullptr, *logprob = nullptr;
@@ -661,6 +663,10 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_lp), (size_t)maxR * options->max_new * 4));
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_last), (size_t)maxR * 4));
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_lens), (size_t)maxR * 4));
+        // up to 8 K splits of the widest store / ReLU / residual GEMM over a decode step's rows
+        const size_t widest = std::max<size_t>({(size_t)h->n_qkv, (size_t)d.d_ffn, (size_t)d.d_model});
+        h->splitk_floats = 8 * (size_t)maxR * widest;
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->splitk_ws), h->splitk_floats * 4));
     }
     if (d.arch == ZO_ARCH_QWEN3) {
         const size_t n = (size_t)d.max_pos * (d.head_dim / 2);
@@ -964,6 +970,10 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
     g.bias = G.bias;
     g.epi = epi;
     g.C = C; g.ldc = ldc; g.c_type = ctype;
+    if (decode) {                         // few rows: the GEMM may split K over the SM pairs
+        g.ws = h->splitk_ws;
+        g.ws_floats = h->splitk_floats;
+    }
     // algorithmic work: the base GEMM plus, per target, its own expand columns
     double fl = 2.0 * Ti * (double)G.N * G.K;
     for (int t = 0; t < G.n_t; ++t) fl += 2.0 * Ti * (double)G.d_out[t] * r_ * (1 + h->n_slots);

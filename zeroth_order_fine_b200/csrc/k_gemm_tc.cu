@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <float.h>
 
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
@@ -80,6 +81,7 @@ struct TcParams {
     const float* rope_cos; const float* rope_sin; float norm_eps;
     int n_q_heads, n_qk_heads;
     const float* a_scale; const float* b_scale;   // E4M3 dequantisation (F8 kernels)
+    int ksplit, kbs;                        // split-K (SPLIT kernels): splits, main blocks each
     int* err;
 };
 
@@ -609,6 +611,14 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                  "r"(src), "r"(x), "r"(y)
                  : "memory");
 }
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y,
+                                             int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
     asm volatile(
         "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -663,10 +673,10 @@ __device__ __forceinline__ void dequant_chunk(const TcParams& p, int m, int n, f
 // residual stream an fp32 reduce-add, so the SM never reads the residual.  Two
 // staging buffers per warp alternate; a buffer is rewritten only after the TMA
 // has read it.
-template <int EPI, bool F8>
+template <int EPI, bool F8, bool SPLIT>
 __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMap* tmC,
                                              uint32_t stg, uint8_t* stg_ptr, int& buf, int m_base,
-                                             int nb, uint32_t taddr, int lane) {
+                                             int nb, uint32_t taddr, int lane, int split) {
     const int r = lane;
     auto stage_begin = [&]() {
         if (lane == 0) bulk_wait_read1();
@@ -682,7 +692,29 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
         }
         buf ^= 1;
     };
-    if (EPI == EPI_RESID) {
+    if (SPLIT) {
+        // one K split's raw fp32 accumulator into its slice of the workspace; the split
+        // reduction applies bias and the epilogue afterwards, summing the slices in order
+        for (int c = 0; c < BN / 32; ++c) {
+            const int n = nb * BN + c * 32;
+            if (n >= p.N) break;
+            float v[32];
+            tmem_ld32(taddr + (uint32_t)(c * 32), v);
+            stage_begin();
+            uint8_t* b = stg_ptr + buf * 4096;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4*>(b + stg_off(r, k)) =
+                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(tmC, stg + buf * 4096, n, m_base, split);
+                bulk_commit();
+            }
+            buf ^= 1;
+        }
+    } else if (EPI == EPI_RESID) {
         for (int c = 0; c < BN / 32; ++c) {
             const int n = nb * BN + c * 32;
             if (n >= p.N) break;
@@ -859,7 +891,7 @@ __device__ __forceinline__ void tile_coords2(int t, const TcParams& p, int* mb, 
 
 // F8: the main K blocks are E4M3 (kind::f8f6f4) and the epilogue dequantises; a separate
 // instantiation, so the bf16 kernels carry none of it.
-template <int EPI, bool F8>
+template <int EPI, bool F8, bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2,
@@ -909,7 +941,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     cluster_sync();                         // both CTAs' barriers exist before any remote use
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int kb_total = p.kb_main + p.kb_ext;
+    // work items: tiles, or (tile, K split) pairs; a split takes kbs main K blocks and the
+    // last split also the extension blocks
+    const int n_items = SPLIT ? p.n_tiles * p.ksplit : p.n_tiles;
+    auto item_blocks = [&](int sp, int* kb0, int* n_main, int* n_kb) {
+        if (!SPLIT) {
+            *kb0 = 0;
+            *n_main = p.kb_main;
+            *n_kb = p.kb_main + p.kb_ext;
+            return;
+        }
+        *kb0 = sp * p.kbs;
+        *n_main = max(0, min(p.kbs, p.kb_main - *kb0));
+        *n_kb = *n_main + (sp == p.ksplit - 1 ? p.kb_ext : 0);
+    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -917,12 +962,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             uint32_t ph = 0;
             int n_armed = 0;                // loads issued; the i-th used stage i % S, phase (i / S) & 1
             bool ok = true;
-            for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
+            for (int t = pair; t < n_items && ok; t += n_pairs) {
                 int mb, nb;
-                tile_coords2(t, p, &mb, &nb);
+                tile_coords2(SPLIT ? t / p.ksplit : t, p, &mb, &nb);
                 const int row_a = mb * BM2 + (int)rank * 128;
                 const int row_b = nb * BN + (int)rank * 128;
-                for (int kb = 0; kb < kb_total; ++kb) {
+                int kb0, n_main, n_kb;
+                item_blocks(SPLIT ? t % p.ksplit : 0, &kb0, &n_main, &n_kb);
+                for (int i = 0; i < n_kb; ++i) {
+                    const int kb = i < n_main ? kb0 + i : p.kb_main + (i - n_main);
                     if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err)) { ok = false; break; }
                     const uint32_t sa = base + s * STAGE2_BYTES;
                     const uint32_t sb = sa + A2B;
@@ -959,11 +1007,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int acc = 0;
             uint32_t aph = 0;
             bool ok = true, issued = false;
-            for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
+            for (int t = pair; t < n_items && ok; t += n_pairs) {
                 if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < kb_total; ++kb) {
+                int kb0, n_main, n_kb;
+                item_blocks(SPLIT ? t % p.ksplit : 0, &kb0, &n_main, &n_kb);
+                for (int i = 0; i < n_kb; ++i) {
+                    const int kb = i < n_main ? kb0 + i : p.kb_main + (i - n_main);
                     if (!mbar_wait(full(s), ph, abort_f, p.err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = base + s * STAGE2_BYTES;
@@ -972,12 +1023,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             tc_mma_pair_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
-                                           kIdesc2F8, (kb > 0 || kk > 0) ? 1u : 0u);
+                                           kIdesc2F8, (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
                             tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
-                                        kIdesc2, (kb > 0 || kk > 0) ? 1u : 0u);
+                                        kIdesc2, (i > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     tc_commit_pair(empty(s));       // stage free in both CTAs
@@ -1005,14 +1056,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         int buf = 0;
         int acc = 0;
         uint32_t aph = 0;
-        for (int t = pair; t < p.n_tiles; t += n_pairs) {
+        for (int t = pair; t < n_items; t += n_pairs) {
             int mb, nb;
-            tile_coords2(t, p, &mb, &nb);
+            tile_coords2(SPLIT ? t / p.ksplit : t, p, &mb, &nb);
             if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
             tc_fence_after();
             const int m_base = mb * BM2 + (int)rank * 128 + lane_base;
-            epilogue_tma<EPI, F8>(p, &tmC, stg, stg_ptr, buf, m_base, nb,
-                              tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN), lane);
+            epilogue_tma<EPI, F8, SPLIT>(p, &tmC, stg, stg_ptr, buf, m_base, nb,
+                                         tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN),
+                                         lane, SPLIT ? t % p.ksplit : 0);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0);
@@ -1134,12 +1186,12 @@ int launch_epi_w(int bnt, const CUtensorMap& a, const CUtensorMap& b, const CUte
     }
 }
 
-template <int EPI, bool F8>
+template <int EPI, bool F8, bool SPLIT = false>
 int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                 const CUtensorMap& b2, const CUtensorMap& c, const TcParams& p, cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(gemm_tc2_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_tc2_kernel<EPI, F8, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SMEM2_BYTES) != cudaSuccess)
             return 1;
         attr = true;
@@ -1157,14 +1209,61 @@ int launch_epi2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a
         cfg.attrs = at;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<EPI, F8>, &cfg) != cudaSuccess || n <= 0)
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<EPI, F8, SPLIT>, &cfg) != cudaSuccess || n <= 0)
             n = num_sms() / 2;
         max_pairs = n;
     }
     int pairs = max_pairs;
-    if (p.n_tiles < pairs) pairs = p.n_tiles;
-    gemm_tc2_kernel<EPI, F8><<<2 * pairs, NUM_THREADS, SMEM2_BYTES, st>>>(a, b, a2, b2, c, p);
+    const int items = SPLIT ? p.n_tiles * p.ksplit : p.n_tiles;
+    if (items < pairs) pairs = items;
+    gemm_tc2_kernel<EPI, F8, SPLIT><<<2 * pairs, NUM_THREADS, SMEM2_BYTES, st>>>(a, b, a2, b2, c, p);
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+
+}  // namespace
+
+namespace {
+
+// y[m, n] = sum_s ws[s, m, n] (in s order) + bias[n], then the epilogue: bf16 store / ReLU,
+// or the fp32 residual add.  One thread per 4 columns.
+__global__ void splitk_epilogue_kernel(const float* __restrict__ ws, int ks, int M, int N,
+                                       const float* __restrict__ bias, int epi, void* C, int ldc) {
+    const int m = blockIdx.y;
+    const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (n >= N) return;
+    float y[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) y[j] = 0.f;
+    for (int s = 0; s < ks; ++s) {
+        const float* w = ws + ((size_t)s * M + m) * N + n;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (n + j < N) y[j] += w[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (n + j >= N) break;
+        float v = y[j] + (bias ? bias[n + j] : 0.f);
+        if (epi == EPI_RESID) {
+            static_cast<float*>(C)[(size_t)m * ldc + n + j] += v;
+        } else {
+            if (epi == EPI_STORE_RELU) v = fmaxf(v, 0.f);
+            static_cast<__nv_bfloat16*>(C)[(size_t)m * ldc + n + j] = __float2bfloat16_rn(v);
+        }
+    }
+}
+
+// [ks][M][N] fp32 workspace, 32 x 32 boxes (128-byte rows, 128-byte swizzle)
+bool make_map_ws(CUtensorMap* m, const float* ws, int ks, int M, int N) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)ks};
+    const cuuint64_t strides[2] = {(cuuint64_t)N * 4, (cuuint64_t)M * N * 4};
+    const cuuint32_t box[3] = {32u, 32u, 1u};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ws), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -1271,6 +1370,31 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     int* err = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
+    if (pair && g.ws && !f8 && g.N % 4 == 0 &&
+        (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID)) {
+        // too few output tiles to keep the SM pairs streaming the weights: split K so that
+        // about two items per pair exist, each split keeping at least 4 main K blocks
+        const int pairs = num_sms() / 2;
+        int ks = (2 * pairs + p.n_tiles - 1) / p.n_tiles;
+        ks = std::min(ks, std::min(8, p.kb_main / 4));
+        while (ks > 1 && (size_t)ks * g.M * g.N > g.ws_floats) --ks;
+        if (ks > 1) {
+            p.ksplit = ks;
+            p.kbs = (p.kb_main + ks - 1) / ks;
+            CUtensorMap c;
+            if (!make_map_ws(&c, g.ws, ks, g.M, g.N)) return 1;
+            int rc = 1;
+            switch (g.epi) {
+                case EPI_STORE: rc = launch_epi2<EPI_STORE, false, true>(a, b, a2, b2, c, p, st); break;
+                case EPI_STORE_RELU: rc = launch_epi2<EPI_STORE_RELU, false, true>(a, b, a2, b2, c, p, st); break;
+                default: rc = launch_epi2<EPI_RESID, false, true>(a, b, a2, b2, c, p, st); break;
+            }
+            if (rc) return rc;
+            dim3 grid((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M);
+            splitk_epilogue_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias, g.epi, g.C, g.ldc);
+            return cudaGetLastError() == cudaSuccess ? 0 : 1;
+        }
+    }
     if (pair) {
         // output map for the TMA-store epilogue: 32-row boxes, 128-byte inner extent
         CUtensorMap c;

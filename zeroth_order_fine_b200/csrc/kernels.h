@@ -108,6 +108,10 @@ struct GemmArgs {
     const int* tok_pos; const float* qn; const float* kn;
     const float* rope_cos; const float* rope_sin; float norm_eps;
     int n_q_heads, n_qk_heads;
+    // optional fp32 workspace (ws_floats floats): lets a bf16 store / ReLU / residual GEMM
+    // with too few output tiles for the SMs split K over the SM pairs (decode steps), the
+    // slices summed in order by a reduction that applies the epilogue
+    float* ws; size_t ws_floats;
 };
 
 void gemm_simt(const GemmArgs& g, cudaStream_t st);
