@@ -458,6 +458,7 @@ int check_desc(const zo_model_desc* d, const zo_weights* w, const zo_options* o)
     if (o->profile != 0 && o->profile != 1) return 1;
     if (o->fp8 != 0 && o->fp8 != 1) return 1;
     if (o->max_new < 0 || o->max_new > 4096) return 1;
+    if (o->max_new > 0 && d->n_heads / d->n_kv_heads > 8) return 2;   // decode attention groups
     if (o->fp8 && (d->dtype != ZO_DTYPE_BF16 || o->impl != 0 || !norm_fp8_supported(d->d_model) ||
                    d->d_model % 16 || (d->n_heads + 2 * d->n_kv_heads) * d->head_dim <= 128 ||
                    d->d_ffn <= 64))
@@ -1057,8 +1058,11 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
             a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
             a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
             a.n_tokens = Ti;
-            if (tc_attn && attention_tc_supported(a)) launch_attention_tc(a, h->st);
-            else launch_attention(a, h->st);
+            if (tc_attn && attention_tc_supported(a)) {
+                if (!launch_attention_tc(a, h->st)) FAIL(h, ZO_ERR_CUDA, "attention tensor map failed");
+            } else {
+                launch_attention(a, h->st);
+            }
             return ZO_OK;
         });
     if (rc) return rc;
@@ -1169,8 +1173,11 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
         a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
         a.scale = scale;
         a.n_tokens = Ti;
-        if (tc_attn && attention_tc_supported(a)) launch_attention_tc(a, h->st);
-        else launch_attention(a, h->st);
+        if (tc_attn && attention_tc_supported(a)) {
+            if (!launch_attention_tc(a, h->st)) FAIL(h, ZO_ERR_CUDA, "attention tensor map failed");
+        } else {
+            launch_attention(a, h->st);
+        }
         h->stats.kernel_launches += 2;
         return ZO_OK;
     });
@@ -1194,9 +1201,10 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
         rc = decoder_layers(h, R, eps, [&](int l) -> int {
             launch_kv_append(h->qkv, h->n_qkv, h->q_dim, kv2, md, h->gen_lens, R, g, G, cache(l),
                              h->dt, h->st);
-            launch_decode_attention(h->qkv, h->n_qkv, cache(l), kv2, md, h->gen_lens, R, g, G,
-                                    d.n_heads, d.n_kv_heads, d.head_dim, scale, h->att, h->q_dim,
-                                    h->dt, h->st);
+            if (!launch_decode_attention(h->qkv, h->n_qkv, cache(l), kv2, md, h->gen_lens, R, g, G,
+                                         d.n_heads, d.n_kv_heads, d.head_dim, scale, h->att,
+                                         h->q_dim, h->dt, h->st))
+                FAIL(h, ZO_ERR_UNSUPPORTED, "decode attention: more than 8 query heads per kv head");
             h->stats.kernel_launches += 2;
             return ZO_OK;
         }, true);

@@ -416,8 +416,8 @@ bool attention_tc_supported(const AttnArgs& a) {
            (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
 }
 
-void launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
-    if (a.n_tiles == 0 || a.n_tokens <= 0) return;
+bool launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
+    if (a.n_tiles == 0 || a.n_tokens <= 0) return true;
     static bool attr = false;
     if (!attr) {
         cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
@@ -427,7 +427,7 @@ void launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
     // 128-byte swizzle, rows past T read as zero
     CUtensorMap tm;
     EncodeTiledFn fn = attn_encode_fn();
-    if (!fn) return;
+    if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)a.ld_qkv, (cuuint64_t)a.n_tokens};
     const cuuint64_t strides[1] = {(cuuint64_t)a.ld_qkv * 2};
     const cuuint32_t box[2] = {64, 128};
@@ -435,10 +435,11 @@ void launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
     if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.qkv), dims, strides, box,
            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return;
+        return false;
     const long long items = (long long)a.n_tiles * a.H;
-    if (items > 0x7fffffffLL) return;
+    if (items > 0x7fffffffLL) return false;
     attention_tc_kernel<<<(unsigned)items, 128, SMEM, st>>>(tm, a);
+    return true;
 }
 
 int attention_tc_error_word() {

@@ -226,19 +226,21 @@ void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int
                                         dtype == E_F32 ? 4 : 2);
 }
 
-void launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int kv2,
+bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int kv2,
                              const int* cu, const int* lens, int R, int g, int G, int H, int Hkv,
                              int hd, float scale, void* out, int ld_out, int dtype,
                              cudaStream_t st) {
-    if (R == 0 || H / Hkv > DEC_MAX_REP || hd % 32 || hd / 32 > DEC_MAX_DPL) return;
+    if (H / Hkv > DEC_MAX_REP || hd % 32 || hd / 32 > DEC_MAX_DPL) return false;
+    if (R == 0) return true;
     dim3 grid(R, Hkv);
     switch (hd / 32) {
         case 1: decode_attention_kernel<1><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
         case 2: decode_attention_kernel<2><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
         case 4: decode_attention_kernel<4><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
         case 8: decode_attention_kernel<8><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu, lens, g, G, H, Hkv, scale, out, ld_out, dtype); break;
-        default: break;
+        default: return false;
     }
+    return true;
 }
 
 void launch_shrink_rows(const void* x, int x_type, const void* FT, int ft_type, int M, int N,

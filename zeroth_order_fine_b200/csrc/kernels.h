@@ -139,7 +139,8 @@ struct AttnArgs {
 // attention by launch_qk_norm_rope; the attention kernels take q and k as they are.)
 void launch_attention(const AttnArgs& a, cudaStream_t st);          // CUDA cores, 64-query tiles
 bool attention_tc_supported(const AttnArgs& a);                     // bf16, head_dim 128
-void launch_attention_tc(const AttnArgs& a, cudaStream_t st);       // tensor cores, 128-query tiles
+bool launch_attention_tc(const AttnArgs& a, cudaStream_t st);       // tensor cores, 128-query tiles;
+                                                                    // false if the tensor map fails
 int attention_tc_error_word();
 
 // ---- objective, estimator, update ------------------------------------------------------
@@ -164,8 +165,9 @@ void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int
                       const int* lens, int R, int g, int G, void* cache, int dtype,
                       cudaStream_t st);
 // One query per row (its q heads in qkv row r) against the row's n = lens[r] + g + 1 cached
-// keys; softmax(q k^T * scale) v into out [R x H*hd].  CUDA cores (memory-bound).
-void launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int kv2,
+// keys; softmax(q k^T * scale) v into out [R x H*hd].  CUDA cores (memory-bound).  false
+// when H / Hkv > 8 or hd is not 32, 64, 128 or 256.
+bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int kv2,
                              const int* cu, const int* lens, int R, int g, int G, int H, int Hkv,
                              int hd, float scale, void* out, int ld_out, int dtype,
                              cudaStream_t st);

@@ -170,9 +170,13 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     a.H = n_heads; a.Hkv = n_kv_heads; a.hd = head_dim;
     a.scale = (float)(1.0 / std::sqrt((double)head_dim));
     a.n_tokens = meta[n_rows];
-    if (tc && attention_tc_supported(a)) launch_attention_tc(a, st);
-    else if (impl == ZO_IMPL_TENSOR_CORES) return ZO_ERR_UNSUPPORTED;
-    else launch_attention(a, st);
+    if (tc && attention_tc_supported(a)) {
+        if (!launch_attention_tc(a, st)) return ZO_ERR_CUDA;
+    } else if (impl == ZO_IMPL_TENSOR_CORES) {
+        return ZO_ERR_UNSUPPORTED;
+    } else {
+        launch_attention(a, st);
+    }
     return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
 }
 
