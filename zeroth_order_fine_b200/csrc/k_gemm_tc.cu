@@ -65,7 +65,7 @@ struct Tile1 {
 };
 
 __device__ int g_tc_error = 0;              // bit 0: a bounded wait expired
-bool g_use_pairs = true;                    // SM-pair kernel for large decoder GEMMs
+constexpr bool g_use_pairs = true;          // SM-pair kernel for large decoder GEMMs
 
 struct TcParams {
     int M, N, kb_main, kb_ext;
@@ -1429,7 +1429,6 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     }
 }
 
-void gemm_tc_set_pairs(bool on) { g_use_pairs = on; }
 
 int gemm_tc_error_word() {
     int v = 0;

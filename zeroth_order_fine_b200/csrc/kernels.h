@@ -121,7 +121,6 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st);   // 0 ok, else 1
 int gemm_lse_col_tiles(int N);                      // LSE column tiles, CUDA-core path (the most)
 int gemm_tc_col_tiles(int N);                       // LSE column tiles, tensor-core path
 int gemm_tc_error_word();                           // bit 0: a bounded wait expired
-void gemm_tc_set_pairs(bool on);                    // SM-pair (cta_group::2) kernel on/off
 
 // ---- attention -----------------------------------------------------------------------
 struct AttnArgs {
