@@ -74,6 +74,17 @@ def test_qwen3_bf16_generation_matches_oracle():
     _check_against_oracle(QWEN_SMALL, False, 5e-2, 3e-2, 2e-2)
 
 
+Q3_WIDE = wl.ModelShape("qwen3-wide", wl.ARCH_QWEN3, 2, 1024, 8, 2, 128, 2048, 4096, 4096, 1e-6,
+                        1e6, wl.DTYPE_BF16, False)
+QWEN_WIDE = dataclasses.replace(QWEN_SMALL, shape=Q3_WIDE)
+
+
+def test_qwen3_wide_bf16_generation_matches_oracle():
+    """d = 1024: every decode GEMM splits K, including the q/k-norm + RoPE and SwiGLU forms
+    whose epilogues then run in the split reduction."""
+    _check_against_oracle(QWEN_WIDE, False, 5e-2, 3e-2, 2e-2)
+
+
 def test_qwen3_fp8_generation_matches_oracle():
     _check_against_oracle(QWEN_SMALL, True, 5e-2, 3e-2, 2e-2)
 
@@ -93,8 +104,9 @@ OPT_WIDTH = dataclasses.replace(wl.WORKLOADS["opt-1.3b-b16"],
                                 batch=4, len_hi=48)
 
 
-@pytest.mark.parametrize("w,tol", [(TINY, 1e-4), (QWEN_SMALL, 2e-2), (OPT_WIDTH, 2e-2)],
-                         ids=["fp32", "qwen3-bf16", "opt-width-bf16"])
+@pytest.mark.parametrize("w,tol", [(TINY, 1e-4), (QWEN_SMALL, 2e-2), (OPT_WIDTH, 2e-2),
+                                   (QWEN_WIDE, 2e-2)],
+                         ids=["fp32", "qwen3-bf16", "opt-width-bf16", "qwen3-wide-bf16"])
 def test_decode_agrees_with_prefill_scoring_of_the_generated_rows(w, tol):
     """The KV-cache decode path and the packed prefill path give the same log-probs for the
     generated tokens (the + rows scored under the + candidate as target spans)."""

@@ -664,8 +664,9 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_lp), (size_t)maxR * options->max_new * 4));
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_last), (size_t)maxR * 4));
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->gen_lens), (size_t)maxR * 4));
-        // up to 8 K splits of the widest store / ReLU / residual GEMM over a decode step's rows
-        const size_t widest = std::max<size_t>({(size_t)h->n_qkv, (size_t)d.d_ffn, (size_t)d.d_model});
+        // up to 8 K splits of the widest decode GEMM over a decode step's rows
+        const size_t ffn_in = (size_t)d.d_ffn * (d.arch == ZO_ARCH_QWEN3 ? 2 : 1);
+        const size_t widest = std::max<size_t>({(size_t)h->n_qkv, ffn_in, (size_t)d.d_model});
         h->splitk_floats = 8 * (size_t)maxR * widest;
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->splitk_ws), h->splitk_floats * 4));
     }
@@ -949,7 +950,8 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
             // a decode step's handful of rows: a CUDA-core dot per (row, factor column)
             // beats one tensor-core CTA walking the whole K range
             launch_shrink_rows(s.A, s.a_type, s.B, s.b_type, Ti, kext, G.K, s.C, s.ldc, s.c_type,
-                               s.row_sign, eps, s.scale_cols, s.a_scale, h->st);
+                               s.row_sign, eps, s.scale_cols, s.a_scale, h->splitk_ws,
+                               h->splitk_floats, h->st);
             h->stats.kernel_launches++;
         } else {
             int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
@@ -1192,6 +1194,8 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
     h->stats.tokens_scored += (uint64_t)Ti;
 
     // decode: token g of every row at position len + g, attending over its row's cache
+    int max_len = 0;
+    for (int i = 0; i < B; ++i) max_len = std::max(max_len, (int)lens[i]);
     for (int g = 0; g + 1 < G; ++g) {
         launch_decode_prep(h->gen_tok, G, g, h->gen_lens, R, B, h->tok_id, h->tok_pos,
                            h->tok_sign, h->tok_row, h->st);
@@ -1203,7 +1207,8 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
                              h->dt, h->st);
             if (!launch_decode_attention(h->qkv, h->n_qkv, cache(l), kv2, md, h->gen_lens, R, g, G,
                                          d.n_heads, d.n_kv_heads, d.head_dim, scale, h->att,
-                                         h->q_dim, h->dt, h->st))
+                                         h->q_dim, h->dt, max_len + g + 1, h->splitk_ws,
+                                         h->splitk_floats, h->st))
                 FAIL(h, ZO_ERR_UNSUPPORTED, "decode attention: more than 8 query heads per kv head");
             h->stats.kernel_launches += 2;
             return ZO_OK;

@@ -1253,6 +1253,70 @@ __global__ void splitk_epilogue_kernel(const float* __restrict__ ws, int ks, int
     }
 }
 
+// SwiGLU from the split slices: gate/up rows interleaved in 128-row blocks, so output f
+// reads column (f / 128) * 256 + f % 128 (gate) and the one 128 after it (up).
+__global__ void splitk_swiglu_kernel(const float* __restrict__ ws, int ks, int M, int N,
+                                     const float* __restrict__ bias, __nv_bfloat16* C, int ldc) {
+    const int m = blockIdx.y;
+    const int f = blockIdx.x * blockDim.x + threadIdx.x;
+    const int F = N / 2;
+    if (f >= F) return;
+    const int gc = (f / 128) * 256 + f % 128, uc = gc + 128;
+    float g = 0.f, u = 0.f;
+    for (int s = 0; s < ks; ++s) {
+        const float* w = ws + ((size_t)s * M + m) * N;
+        g += w[gc];
+        u += w[uc];
+    }
+    if (bias) {
+        g += bias[gc];
+        u += bias[uc];
+    }
+    C[(size_t)m * ldc + f] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+}
+
+// Qwen3 q|k|v from the split slices, one warp per (row, head): the summed head is rounded
+// to bf16, then q and k heads get RMSNorm over the head and the rotary rotation of the
+// pairs (i, i + 64) at the token's position; lane l holds columns 4l..4l+3, its partner
+// columns sit in lane l ^ 16.
+__global__ void splitk_qknr_kernel(const float* __restrict__ ws, int ks, int M, int N, TcParams p,
+                                   __nv_bfloat16* C, int ldc) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int heads = N / 128;
+    if (warp >= M * heads) return;
+    const int m = warp / heads, head = warp % heads;
+    const int c0 = head * 128 + 4 * lane;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < ks; ++s) {
+        const float4 w = *reinterpret_cast<const float4*>(ws + ((size_t)s * M + m) * N + c0);
+        x[0] += w.x; x[1] += w.y; x[2] += w.z; x[3] += w.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+    if (head < p.n_qk_heads) {
+        float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+        ss = warp_sum(ss);
+        const float rs = 1.0f / sqrtf(ss / 128.0f + p.norm_eps);
+        const float* w = head < p.n_q_heads ? p.qn : p.kn;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = x[e] * rs * w[4 * lane + e];
+        const int pos = p.tok_pos[m];
+        const int i0 = (4 * lane) & 63;
+        float partner[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) partner[e] = __shfl_xor_sync(0xffffffffu, x[e], 16);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float cs = p.rope_cos[(size_t)pos * 64 + i0 + e];
+            const float sn = p.rope_sin[(size_t)pos * 64 + i0 + e];
+            // lanes 0..15 hold a = x[i], lanes 16..31 hold b = x[i + 64]
+            x[e] = lane < 16 ? x[e] * cs - partner[e] * sn : x[e] * cs + partner[e] * sn;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) C[(size_t)m * ldc + c0 + e] = __float2bfloat16_rn(x[e]);
+}
+
 // [ks][M][N] fp32 workspace, 32 x 32 boxes (128-byte rows, 128-byte swizzle)
 bool make_map_ws(CUtensorMap* m, const float* ws, int ks, int M, int N) {
     EncodeTiledFn fn = encode_fn();
@@ -1371,7 +1435,8 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
     if (pair && g.ws && !f8 && g.N % 4 == 0 &&
-        (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID)) {
+        (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
+         g.epi == EPI_SWIGLU || g.epi == EPI_QKNR)) {
         // too few output tiles to keep the SM pairs streaming the weights: split K so that
         // about two items per pair exist, each split keeping at least 4 main K blocks
         const int pairs = num_sms() / 2;
@@ -1383,15 +1448,22 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
             p.kbs = (p.kb_main + ks - 1) / ks;
             CUtensorMap c;
             if (!make_map_ws(&c, g.ws, ks, g.M, g.N)) return 1;
-            int rc = 1;
-            switch (g.epi) {
-                case EPI_STORE: rc = launch_epi2<EPI_STORE, false, true>(a, b, a2, b2, c, p, st); break;
-                case EPI_STORE_RELU: rc = launch_epi2<EPI_STORE_RELU, false, true>(a, b, a2, b2, c, p, st); break;
-                default: rc = launch_epi2<EPI_RESID, false, true>(a, b, a2, b2, c, p, st); break;
-            }
+            // the split kernels' epilogue only stores fp32 slices: one instantiation serves all
+            const int rc = launch_epi2<EPI_STORE, false, true>(a, b, a2, b2, c, p, st);
             if (rc) return rc;
-            dim3 grid((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M);
-            splitk_epilogue_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias, g.epi, g.C, g.ldc);
+            if (g.epi == EPI_SWIGLU) {
+                dim3 grid((unsigned)((g.N / 2 + 127) / 128), (unsigned)g.M);
+                splitk_swiglu_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias,
+                                                           static_cast<__nv_bfloat16*>(g.C), g.ldc);
+            } else if (g.epi == EPI_QKNR) {
+                const long long warps = (long long)g.M * (g.N / 128);
+                splitk_qknr_kernel<<<(unsigned)((warps + 3) / 4), 128, 0, st>>>(
+                    g.ws, ks, g.M, g.N, p, static_cast<__nv_bfloat16*>(g.C), g.ldc);
+            } else {
+                dim3 grid((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M);
+                splitk_epilogue_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias, g.epi,
+                                                             g.C, g.ldc);
+            }
             return cudaGetLastError() == cudaSuccess ? 0 : 1;
         }
     }

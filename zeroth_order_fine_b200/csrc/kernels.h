@@ -166,16 +166,20 @@ void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int
 // One query per row (its q heads in qkv row r) against the row's n = lens[r] + g + 1 cached
 // keys; softmax(q k^T * scale) v into out [R x H*hd].  CUDA cores (memory-bound).  false
 // when H / Hkv > 8 or hd is not 32, 64, 128 or 256.
+// max_n: the most keys any row has at this step; ws (ws_floats floats) holds the partials
+// when the keys split over several CTAs.
 bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int kv2,
                              const int* cu, const int* lens, int R, int g, int G, int H, int Hkv,
-                             int hd, float scale, void* out, int ld_out, int dtype,
-                             cudaStream_t st);
+                             int hd, float scale, void* out, int ld_out, int dtype, int max_n,
+                             float* ws, size_t ws_floats, cudaStream_t st);
 // Bank shrink for a few rows (decode steps), on CUDA cores: C[m, j] = (x[m] . FT[j]) *
 // (j < scale_cols ? row_sign[m] * eps : 1) / (a_scale ? a_scale[m] : 1); x [M x K] in
 // x_type, FT [N x K] in ft_type, C [M x ldc] in c_type.
+// ws (optional, ws_floats floats): lets K split over more CTAs, the parts summed in order.
 void launch_shrink_rows(const void* x, int x_type, const void* FT, int ft_type, int M, int N,
                         int K, void* C, int ldc, int c_type, const int* row_sign, float eps,
-                        int scale_cols, const float* a_scale, cudaStream_t st);
+                        int scale_cols, const float* a_scale, float* ws, size_t ws_floats,
+                        cudaStream_t st);
 // Last prompt token of each row (the hidden state that predicts the first new token) and
 // the rows' prompt lengths.
 void launch_last_tokens(const int* cu, int R, int* out, int* lens, cudaStream_t st);
