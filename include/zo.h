@@ -225,7 +225,8 @@ int zo_score(zo_plan* plan, const int32_t* packed_tokens, int32_t n_prompts,
  *   gen_logprob dev float [2 n_prompts x n_new] or NULL: their log-probabilities
  *   L_plus, L_minus dev float [n_prompts] or NULL
  * ZO_ERR_UNSUPPORTED when options.max_new is 0; ZO_ERR_ARG when n_new is outside
- * 1..max_new or the batch exceeds max_tokens / max_rows. */
+ * 1..max_new or the batch exceeds max_tokens (prompt tokens of both candidates),
+ * max_rows (2 n_prompts) or max_scored (2 n_prompts). */
 int zo_generate(zo_plan* plan, const int32_t* packed_tokens, int32_t n_prompts,
                 const int32_t* seq_lens, int32_t n_new, int32_t* gen_tokens,
                 float* gen_logprob, float* L_plus, float* L_minus);
