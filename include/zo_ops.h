@@ -57,6 +57,25 @@ int zo_op_linear(const void* x, const void* W, const float* bias, void* y, int32
                  int32_t N, int32_t K, int32_t dtype, int32_t act, int32_t accumulate,
                  int32_t impl, void* stream);
 
+/* The decode-step form of zo_op_linear (bf16 only): the few token rows of one
+ * generation step ("Inference-Native Zeroth-Order Optimization", abstract:
+ * ProbePlan queries may be autoregressive generation) against a whole weight
+ * matrix, which makes the GEMM a stream of the weights.  With M <= 128 the
+ * weights take the 128-row side of a single-SM tcgen05 GEMM and the tokens the
+ * narrow N side (32, 64 or 128 columns); K is split over the SMs, each split
+ * stores its fp32 slice in ws, and a reduction adds the slices in split order
+ * and applies bias, ReLU or the residual add, so the result does not depend on
+ * scheduling.  Larger M splits K on the SM-pair kernel instead.
+ *   x, W, bias, y, M, N, K, act, accumulate: as zo_op_linear (dtype bf16)
+ *   ws   dev float [ws_floats], caller-owned scratch; at least M x N floats
+ *        (room for up to 16 slices lets more splits run)
+ * M = 0 is a no-op.  ZO_ERR_ARG on NULL pointers, negative sizes or ws_floats < M x N;
+ * ZO_ERR_UNSUPPORTED when K % 8 is not 0, or N % 8 (N % 4 with accumulate), or a
+ * pointer is not 16-byte aligned.  Asynchronous on stream. */
+int zo_op_linear_decode(const void* x, const void* W, const float* bias, void* y, int32_t M,
+                        int32_t N, int32_t K, int32_t act, int32_t accumulate, float* ws,
+                        size_t ws_floats, void* stream);
+
 /* Bytes of workspace zo_op_lm_head_logprob needs for n_rows rows and vocab. */
 size_t zo_op_lm_head_workspace(int32_t n_rows, int32_t vocab, int32_t impl);
 

@@ -55,6 +55,55 @@ def test_linear_residual_accumulate(M, N, K, impl):
     assert torch.max((y.double().cpu() - ref).abs()) < 2e-4
 
 
+# decode-step GEMMs: swapped single-SM tiles for M <= 128 (N tile 32 / 64 / 128, ragged
+# weight-row tiles, K not a multiple of the 64-wide block, 1..16 K splits), the SM-pair split
+# for M > 128; the slices are summed in split order
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (17, 392, 1000), (32, 5120, 5120),
+                                   (40, 1280, 2048), (64, 640, 776), (100, 4096, 4096),
+                                   (128, 15360, 5120), (32, 5120, 20480), (160, 2048, 1024),
+                                   (0, 256, 64)])
+def test_linear_decode(M, N, K):
+    from zeroth_order_fine_b200 import zo
+    x = _rand((M, K), torch.bfloat16, 31)
+    W = _rand((N, K), torch.bfloat16, 32, 0.05)
+    b = _rand((N,), torch.float32, 33)
+    ref = x.double() @ W.double().T + b.double()
+    for act in (0, 1):
+        y = zo.zo_op_linear_decode(x.cuda(), W.cuda(), b.cuda(), act=act)
+        assert zo.zo_op_error_word() == 0
+        r = torch.relu(ref) if act else ref
+        err = (y.double().cpu() - r).abs()
+        assert torch.all(err <= _bf16_ulp(r) + 1e-4 * (K ** 0.5) * 0.05), err.max()
+    y0 = _rand((M, N), torch.float32, 34)
+    y = y0.cuda().clone()
+    zo.zo_op_linear_decode(x.cuda(), W.cuda(), b.cuda(), out=y, accumulate=True)
+    assert zo.zo_op_error_word() == 0
+    if M:
+        # fp32 accumulation over K products and the split slices: rounding grows like sqrt(K)
+        # ulps of the running sum
+        r = y0.double() + ref
+        err = (y.double().cpu() - r).abs()
+        assert torch.all(err <= 1e-6 * (K ** 0.5) * torch.clamp(r.abs(), min=1.0)), err.max()
+
+
+def test_linear_decode_is_deterministic_and_checks_its_workspace():
+    from zeroth_order_fine_b200 import zo
+    x = _rand((32, 5120), torch.bfloat16, 35).cuda()
+    W = _rand((5120, 5120), torch.bfloat16, 36, 0.05).cuda()
+    y1 = zo.zo_op_linear_decode(x, W)
+    y2 = zo.zo_op_linear_decode(x, W)
+    assert torch.equal(y1, y2)
+    # a single-slice workspace forces one split: the same values up to the fp32 summation
+    # order, so both sit within the bound against the float64 product
+    y3 = zo.zo_op_linear_decode(x, W, ws=torch.empty(32 * 5120, device="cuda"))
+    ref = x.double().cpu() @ W.double().cpu().T
+    for y in (y1, y3):
+        err = (y.double().cpu() - ref).abs()
+        assert torch.all(err <= _bf16_ulp(ref) + 1e-4 * (5120 ** 0.5) * 0.05), err.max()
+    with pytest.raises(RuntimeError):
+        zo.zo_op_linear_decode(x, W, ws=torch.empty(100, device="cuda"))
+
+
 def test_tensor_cores_match_cuda_cores_closely():
     from zeroth_order_fine_b200 import zo
     x = _rand((700, 2048), torch.bfloat16, 8)

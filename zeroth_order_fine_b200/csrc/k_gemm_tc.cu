@@ -49,10 +49,10 @@ constexpr long long WAIT_CYCLES = 4000000000ll;   // ~2 s at 2 GHz: a stage that
 // wide ones and do not spend tensor-core time on columns that do not exist.
 template <int BNT>
 struct Tile1 {
-    static_assert(BNT == 64 || BNT == 128 || BNT == 256, "N tile");
+    static_assert(BNT == 32 || BNT == 64 || BNT == 128 || BNT == 256, "N tile");
     static constexpr int B_BYTES = BNT * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // multiple of 1024
-    static constexpr int STAGES = (192 * 1024) / STAGE_BYTES;    // 8, 6, 4
+    static constexpr int STAGES = (192 * 1024) / STAGE_BYTES;    // 9, 8, 6, 4
     static constexpr int TMEM_COLS = 2 * BNT;                    // double-buffered accumulator
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
     // bf16 x bf16 -> fp32, both K-major, M = 128, N = BNT
@@ -63,6 +63,12 @@ struct Tile1 {
     static constexpr int SLOT_OFF = 240, ABORT_OFF = 248;
     static_assert(8 * (2 * STAGES + 5) <= SLOT_OFF, "barrier region");
 };
+
+// Decode steps (a few dozen token rows): the operands are swapped, so the weight rows fill
+// the 128-row MMA side and the tokens are the narrow N side, and each (128 weight rows, K
+// split) item stores its raw fp32 accumulator transposed, as rows of tokens, into its slice
+// of a [ks][tokens][features] workspace; the split reduction applies bias and the epilogue.
+constexpr int EPI_SPLIT_T = 16;
 
 __device__ int g_tc_error = 0;              // bit 0: a bounded wait expired
 constexpr bool g_use_pairs = true;          // SM-pair kernel for large decoder GEMMs
@@ -408,7 +414,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int kb_total = p.kb_main + p.kb_ext;
+    // work items: tiles, or (tile, K split) pairs for EPI_SPLIT_T; a split takes kbs main K
+    // blocks and the last split also the extension blocks
+    constexpr bool SPLIT = EPI == EPI_SPLIT_T;
+    const int ks = SPLIT ? p.ksplit : 1;
+    const int n_items = p.n_tiles * ks;
+    auto item_blocks = [&](int sp, int* kb0, int* n_main, int* n_kb) {
+        if (!SPLIT) {
+            *kb0 = 0;
+            *n_main = p.kb_main;
+            *n_kb = p.kb_main + p.kb_ext;
+            return;
+        }
+        *kb0 = sp * p.kbs;
+        *n_main = max(0, min(p.kbs, p.kb_main - *kb0));
+        *n_kb = *n_main + (sp == ks - 1 ? p.kb_ext : 0);
+    };
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -417,10 +438,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t ph = 0;
             int n_armed = 0;                // loads issued; the i-th used stage i % S, phase (i / S) & 1
             bool ok = true;
-            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+            for (int t = blockIdx.x; t < n_items && ok; t += gridDim.x) {
                 int mb, nb;
-                tile_coords(t, p, &mb, &nb);
-                for (int kb = 0; kb < kb_total; ++kb) {
+                tile_coords(t / ks, p, &mb, &nb);
+                int kb0, n_main, n_kb;
+                item_blocks(t % ks, &kb0, &n_main, &n_kb);
+                for (int i = 0; i < n_kb; ++i) {
+                    const int kb = i < n_main ? kb0 + i : p.kb_main + (i - n_main);
                     if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err)) { ok = false; break; }
                     const uint32_t sa = base + s * STAGE_BYTES;
                     const uint32_t sb = sa + A_BYTES;
@@ -456,11 +480,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int acc = 0;
             uint32_t aph = 0;
             bool ok = true, issued = false;
-            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+            for (int t = blockIdx.x; t < n_items && ok; t += gridDim.x) {
                 if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * BNT);
-                for (int kb = 0; kb < kb_total; ++kb) {
+                int kb0, n_main, n_kb;
+                item_blocks(t % ks, &kb0, &n_main, &n_kb);
+                for (int i = 0; i < n_kb; ++i) {
                     if (!mbar_wait(full(s), ph, abort_f, p.err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = base + s * STAGE_BYTES;
@@ -468,7 +494,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
-                               (kb > 0 || kk > 0) ? 1u : 0u);
+                               (i > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     tc_commit(empty(s));            // stage free once these MMAs retire
@@ -488,15 +514,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int lane_base = 32 * (warp & 3);
         int acc = 0;
         uint32_t aph = 0;
-        for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+        for (int t = blockIdx.x; t < n_items; t += gridDim.x) {
             int mb, nb;
-            tile_coords(t, p, &mb, &nb);
+            tile_coords(t / ks, p, &mb, &nb);
             if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
             tc_fence_after();
             const int m = mb * BM + lane_base + lane;
             float run_max = -FLT_MAX, run_sum = 0.f;
             int run_arg = nb * BNT;
-            if (EPI == EPI_SWIGLU)
+            if (EPI == EPI_SPLIT_T) {
+                // lane = feature m, columns = tokens: for each token the warp's 32 lanes
+                // write 32 consecutive features
+                float* slice = static_cast<float*>(p.C) + (size_t)(t % ks) * p.N * p.M;
+                for (int c = 0; c < BNT / 32; ++c) {
+                    const int n = nb * BNT + c * 32;
+                    if (n >= p.N) break;            // warp-uniform
+                    float v[32];
+                    tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BNT + c * 32), v);
+                    if (m < p.M) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (n + j < p.N) slice[(size_t)(n + j) * p.M + m] = v[j];
+                    }
+                }
+            } else if (EPI == EPI_SWIGLU)
                 epilogue_swiglu(p, m, nb, tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BNT));
             else
             for (int c = 0; c < BNT / 32; ++c) {
@@ -1163,7 +1204,8 @@ int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2
             return 1;
         attr = true;
     }
-    const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+    const int items = EPI == EPI_SPLIT_T ? p.n_tiles * p.ksplit : p.n_tiles;
+    const int grid = items < num_sms() ? items : num_sms();
     gemm_tc_kernel<EPI, BNT><<<grid, NUM_THREADS, smem, st>>>(a, b, a2, b2, p);
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
@@ -1330,6 +1372,98 @@ bool make_map_ws(CUtensorMap* m, const float* ws, int ks, int M, int N) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The split reduction of a [ks][M][N] workspace into g.C with g's epilogue.
+int launch_split_reduce(const GemmArgs& g, const TcParams& p, int ks, cudaStream_t st) {
+    if (g.epi == EPI_SWIGLU) {
+        dim3 grid((unsigned)((g.N / 2 + 127) / 128), (unsigned)g.M);
+        splitk_swiglu_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias,
+                                                   static_cast<__nv_bfloat16*>(g.C), g.ldc);
+    } else if (g.epi == EPI_QKNR) {
+        const long long warps = (long long)g.M * (g.N / 128);
+        splitk_qknr_kernel<<<(unsigned)((warps + 3) / 4), 128, 0, st>>>(
+            g.ws, ks, g.M, g.N, p, static_cast<__nv_bfloat16*>(g.C), g.ldc);
+    } else {
+        dim3 grid((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M);
+        splitk_epilogue_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias, g.epi, g.C,
+                                                     g.ldc);
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+
+// Splits of kb_main K blocks into ks parts of kbs blocks: the number of non-empty parts.
+int effective_splits(int kb_main, int ks, int* kbs) {
+    *kbs = (kb_main + ks - 1) / ks;
+    return (kb_main + *kbs - 1) / *kbs;
+}
+
+// Decode-step GEMM on single SMs with the operands swapped: A = the weights [N x K] (128-row
+// tiles), B = the M <= 128 token rows (one N tile of 32, 64 or 128), likewise for the
+// extension blocks.  Each (weight tile, K split) item writes its fp32 slice transposed into
+// the workspace, then the split reduction applies g's epilogue.
+int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
+    const int bnt = g.M <= 32 ? 32 : (g.M <= 64 ? 64 : 128);
+    CUtensorMap a, b, a2, b2;
+    if (!make_map(&a, g.B, g.N, g.K, g.ldb, BM)) return 1;
+    if (!make_map(&b, g.A, g.M, g.K, g.lda, bnt)) return 1;
+    if (g.K2 > 0) {
+        if (!make_map(&a2, g.B2, g.N, g.K2, g.ldb2, BM)) return 1;
+        if (!make_map(&b2, g.A2, g.M, g.K2, g.lda2, bnt)) return 1;
+    } else {
+        a2 = a;
+        b2 = b;
+    }
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = g.N; p.N = g.M;
+    p.kb_main = (g.K + BK - 1) / BK;
+    p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
+    p.n_m_blk = (g.N + BM - 1) / BM;
+    p.n_n_blk = 1;
+    p.n_tiles = p.n_m_blk;
+    p.group_m = GROUP_M;
+    p.epi = EPI_SPLIT_T;
+    p.C = g.ws; p.ldc = g.N; p.c_type = E_F32;
+    p.tok_pos = g.tok_pos; p.qn = g.qn; p.kn = g.kn;
+    p.rope_cos = g.rope_cos; p.rope_sin = g.rope_sin; p.norm_eps = g.norm_eps;
+    p.n_q_heads = g.n_q_heads; p.n_qk_heads = g.n_qk_heads;
+    int* err = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
+    p.err = err;
+    // K splits: the weight stream is the cost.  In units of one 128 x 64 weight block, the
+    // busiest SM streams rounds x (kbs + slice) blocks at up to SM_BW_REL times its fair share
+    // of HBM, and all SMs together stream the weights plus the slices written and read back;
+    // take the split count with the smaller bound, every split keeping at least 2 blocks.
+    const int sms = num_sms();
+    constexpr double SM_BW_REL = 1.25;
+    const double slice = g.M / 32.0;                 // 128 x M fp32 = M / 32 weight blocks
+    int ks = 1;
+    double best = 1e300;
+    for (int k = 1; k <= 16 && k <= std::max(1, p.kb_main / 2); ++k) {
+        int kbs;
+        if (effective_splits(p.kb_main, k, &kbs) != k) continue;
+        if ((size_t)k * g.M * g.N > g.ws_floats) break;
+        const long long items = (long long)p.n_tiles * k;
+        const long long rounds = (items + sms - 1) / sms;
+        const double t_sm = (double)rounds * (kbs + slice) / SM_BW_REL;
+        const double t_hbm = ((double)p.n_tiles * p.kb_main + 2.0 * items * slice) / sms;
+        const double cost = std::max(t_sm, t_hbm);
+        if (cost < best * 0.98) {                    // a clear gain for each extra split
+            best = cost;
+            ks = k;
+        }
+    }
+    ks = effective_splits(p.kb_main, ks, &p.kbs);
+    p.ksplit = ks;
+    int rc;
+    switch (bnt) {
+        case 32: rc = launch_epi<EPI_SPLIT_T, 32>(a, b, a2, b2, p, st); break;
+        case 64: rc = launch_epi<EPI_SPLIT_T, 64>(a, b, a2, b2, p, st); break;
+        default: rc = launch_epi<EPI_SPLIT_T, 128>(a, b, a2, b2, p, st); break;
+    }
+    if (rc) return rc;
+    return launch_split_reduce(g, p, ks, st);
+}
+
 }  // namespace
 
 bool gemm_tc_supported(const GemmArgs& g) {
@@ -1388,7 +1522,12 @@ int gemm_tc_col_tiles(int N) { return (N + BN - 1) / BN; }
 int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     // Decoder GEMMs run on SM pairs, the LSE and shrink forms on single SMs.  The
     // choice never depends on M (the batch): a row's bits must not change with
-    // the company it is scored in.
+    // the company it is scored in.  Decode steps (a workspace given) are the exception:
+    // their few token rows take the swapped single-SM form.
+    if (g.ws && g.M <= 128 && g.a_type == E_BF16 && g.b_type == E_BF16 && g.N % 4 == 0 &&
+        (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
+         g.epi == EPI_SWIGLU || g.epi == EPI_QKNR))
+        return gemm_tc_swapped(g, st);
     const bool pair = g_use_pairs && g.N > 128 &&
                       (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
                        g.epi == EPI_SWIGLU || g.epi == EPI_QKNR);
@@ -1443,28 +1582,15 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
         int ks = (2 * pairs + p.n_tiles - 1) / p.n_tiles;
         ks = std::min(ks, std::min(8, p.kb_main / 4));
         while (ks > 1 && (size_t)ks * g.M * g.N > g.ws_floats) --ks;
+        if (ks > 1) ks = effective_splits(p.kb_main, ks, &p.kbs);   // no split without K blocks
         if (ks > 1) {
             p.ksplit = ks;
-            p.kbs = (p.kb_main + ks - 1) / ks;
             CUtensorMap c;
             if (!make_map_ws(&c, g.ws, ks, g.M, g.N)) return 1;
             // the split kernels' epilogue only stores fp32 slices: one instantiation serves all
             const int rc = launch_epi2<EPI_STORE, false, true>(a, b, a2, b2, c, p, st);
             if (rc) return rc;
-            if (g.epi == EPI_SWIGLU) {
-                dim3 grid((unsigned)((g.N / 2 + 127) / 128), (unsigned)g.M);
-                splitk_swiglu_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias,
-                                                           static_cast<__nv_bfloat16*>(g.C), g.ldc);
-            } else if (g.epi == EPI_QKNR) {
-                const long long warps = (long long)g.M * (g.N / 128);
-                splitk_qknr_kernel<<<(unsigned)((warps + 3) / 4), 128, 0, st>>>(
-                    g.ws, ks, g.M, g.N, p, static_cast<__nv_bfloat16*>(g.C), g.ldc);
-            } else {
-                dim3 grid((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M);
-                splitk_epilogue_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias, g.epi,
-                                                             g.C, g.ldc);
-            }
-            return cudaGetLastError() == cudaSuccess ? 0 : 1;
+            return launch_split_reduce(g, p, ks, st);
         }
     }
     if (pair) {

@@ -108,9 +108,10 @@ struct GemmArgs {
     const int* tok_pos; const float* qn; const float* kn;
     const float* rope_cos; const float* rope_sin; float norm_eps;
     int n_q_heads, n_qk_heads;
-    // optional fp32 workspace (ws_floats floats): lets a bf16 store / ReLU / residual GEMM
-    // with too few output tiles for the SMs split K over the SM pairs (decode steps), the
-    // slices summed in order by a reduction that applies the epilogue
+    // optional fp32 workspace (ws_floats floats) for decode steps: the bf16 store / ReLU /
+    // residual / SwiGLU / q-k-norm GEMMs split K, over single SMs with the operands swapped
+    // (M <= 128 token rows as the narrow N side) or over the SM pairs (larger M), and a
+    // reduction sums the slices in order and applies the epilogue
     float* ws; size_t ws_floats;
 };
 

@@ -81,6 +81,29 @@ int zo_op_linear(const void* x, const void* W, const float* bias, void* y, int32
     return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
 }
 
+int zo_op_linear_decode(const void* x, const void* W, const float* bias, void* y, int32_t M,
+                        int32_t N, int32_t K, int32_t act, int32_t accumulate, float* ws,
+                        size_t ws_floats, void* stream) {
+    if (M < 0 || N <= 0 || K <= 0) return ZO_ERR_ARG;
+    if (act != ZO_ACT_NONE && act != ZO_ACT_RELU) return ZO_ERR_ARG;
+    if (accumulate && act != ZO_ACT_NONE) return ZO_ERR_ARG;
+    if (M == 0) return ZO_OK;
+    if (!x || !W || !y || !ws || ws_floats < (size_t)M * N) return ZO_ERR_ARG;
+    if (K % 8 || N % 4) return ZO_ERR_UNSUPPORTED;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.A = x; g.lda = K; g.a_type = E_BF16;
+    g.B = W; g.ldb = K; g.b_type = E_BF16;
+    g.M = M; g.N = N; g.K = K;
+    g.bias = bias;
+    g.epi = accumulate ? EPI_RESID : (act == ZO_ACT_RELU ? EPI_STORE_RELU : EPI_STORE);
+    g.C = y; g.ldc = N; g.c_type = accumulate ? E_F32 : E_BF16;
+    g.ws = ws; g.ws_floats = ws_floats;
+    if (!gemm_tc_supported(g)) return ZO_ERR_UNSUPPORTED;
+    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return ZO_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
 size_t zo_op_lm_head_workspace(int32_t n_rows, int32_t vocab, int32_t impl) {
     (void)impl;
     const size_t tiles = (size_t)gemm_lse_col_tiles(vocab);

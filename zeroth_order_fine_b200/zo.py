@@ -118,6 +118,9 @@ _SIGS = {
                                  ctypes.c_float, ctypes.c_float, c_int32, c_void_p]),
     "zo_op_linear": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                c_int32, c_int32, c_int32, c_int32, c_void_p]),
+    "zo_op_linear_decode": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
+                                      c_int32, c_int32, c_int32, c_void_p, ctypes.c_size_t,
+                                      c_void_p]),
     "zo_op_quantize_rows_e4m3": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                            c_void_p, c_void_p]),
     "zo_op_linear_fp8": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -441,6 +444,21 @@ def zo_op_linear(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] 
         out = torch.empty(M, N, dtype=torch.float32 if accumulate else x.dtype, device=x.device)
     _check(lib().zo_op_linear(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, dtype, act,
                               int(accumulate), impl, _stream()))
+    return out
+
+
+def zo_op_linear_decode(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, act: int = 0, accumulate: bool = False,
+                        ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The decode-step linear (bf16): split-K tensor-core GEMM through an fp32 workspace."""
+    M, K = x.shape
+    N = W.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float32 if accumulate else x.dtype, device=x.device)
+    if ws is None:
+        ws = torch.empty(max(1, 16 * M * N), dtype=torch.float32, device=x.device)
+    _check(lib().zo_op_linear_decode(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, act,
+                                     int(accumulate), _ptr(ws), ws.numel(), _stream()))
     return out
 
 
