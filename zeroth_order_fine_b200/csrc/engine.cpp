@@ -947,12 +947,20 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
         s.row_sign = h->tok_sign; s.eps = eps; s.scale_cols = G.n_t * r_;
         if (G.Wq) s.a_scale = h->sx;      // S / s_x: the base GEMM accumulates in E4M3 units
         if (decode) {
-            // a decode step's handful of rows: a CUDA-core dot per (row, factor column)
-            // beats one tensor-core CTA walking the whole K range
-            launch_shrink_rows(s.A, s.a_type, s.B, s.b_type, Ti, kext, G.K, s.C, s.ldc, s.c_type,
-                               s.row_sign, eps, s.scale_cols, s.a_scale, h->splitk_ws,
-                               h->splitk_floats, h->st);
-            h->stats.kernel_launches++;
+            // a decode step's handful of rows: the factor rows take the 128-row side of the
+            // swapped tensor-core GEMM with K split over the SMs (bf16 factors), else a tiled
+            // CUDA-core dot per (row, factor column)
+            s.ws = h->splitk_ws;
+            s.ws_floats = h->splitk_floats;
+            if (h->use_tc && Ti <= 128 && gemm_tc_supported(s)) {
+                int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
+                if (rc) return rc;
+            } else {
+                launch_shrink_rows(s.A, s.a_type, s.B, s.b_type, Ti, kext, G.K, s.C, s.ldc,
+                                   s.c_type, s.row_sign, eps, s.scale_cols, s.a_scale,
+                                   h->splitk_ws, h->splitk_floats, h->st);
+                h->stats.kernel_launches++;
+            }
         } else {
             int rc = run_gemm(h, s, 2.0 * Ti * (double)G.K * kext);
             if (rc) return rc;

@@ -60,128 +60,210 @@ __global__ void kv_append_kernel(const char* __restrict__ qkv, int ld_qkv, int q
     copy_row(qkv + ((size_t)r * ld_qkv + q_dim) * es, cache + crow * kv2 * es, kv2, es);
 }
 
-// One CTA per (row, kv head): the n_rep query heads that share the kv head.  The 4 warps
-// take rounds of 4 consecutive keys in turn; a warp's 32 lanes split the head dimension
-// (hd / 32 consecutive elements each), so a key's k and v rows are read as one coalesced warp
-// access.  Per warp an online softmax (fp32) over its keys, then the four warps' partial
-// results are merged.
-constexpr int DEC_WARPS = 4, DEC_MAX_REP = 8, DEC_MAX_DPL = 8;      // hd <= 256
-
-// DPL consecutive elements at off (a multiple of DPL): 8/16-byte loads when DPL % 4 == 0
-template <int DPL>
-__device__ __forceinline__ void load_dims(const void* base, size_t off, int dtype, float* v) {
-    if (dtype == E_F32) {
-        const float* p = static_cast<const float*>(base) + off;
-        if (DPL % 4 == 0) {
+__device__ __forceinline__ void bf16x8(const uint4& u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-            for (int i = 0; i < DPL; i += 4) {
-                const float4 t = *reinterpret_cast<const float4*>(p + i);
-                v[i] = t.x; v[i + 1] = t.y; v[i + 2] = t.z; v[i + 3] = t.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) v[i] = p[i];
-        }
-    } else {
-        const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(base) + off;
-        if (DPL % 4 == 0) {
-#pragma unroll
-            for (int i = 0; i < DPL; i += 4) {
-                const uint2 t = *reinterpret_cast<const uint2*>(p + i);
-                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&t.x));
-                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&t.y));
-                v[i] = a.x; v[i + 1] = a.y; v[i + 2] = b.x; v[i + 3] = b.y;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) v[i] = __bfloat162float(p[i]);
-        }
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
     }
 }
 
-// blockIdx.z takes keys [z * kps, (z + 1) * kps) of the row.  With part == nullptr (one
-// split) the CTA writes the output; else it writes its (max, sum, unnormalised output) per
-// query head to part, and decode_merge_kernel combines the splits in order.
-template <int DPL>
-__global__ void __launch_bounds__(DEC_WARPS * 32) decode_attention_kernel(
+// 8 consecutive elements at off (a multiple of 8): one 16-byte load (bf16) or two (fp32)
+__device__ __forceinline__ void load8(const void* base, size_t off, int dtype, float* v) {
+    if (dtype == E_F32) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
+        const float4 a = p[0], b = p[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + off), v);
+    }
+}
+
+// One CTA per (row, kv head, key split): the n_rep query heads that share the kv head (NREP =
+// n_rep rounded up to a power of two; the padding heads have q = 0 and are not written), over
+// the keys [kbeg, kend) of the row, in tiles of kt keys.  Per tile:
+//   0. the tile's k and v rows of this head go to shared memory by asynchronous 16-byte
+//      copies, all issued at once, so the whole tile is in flight together;
+//   1. scores s[h][j] = scale * q_h . k_j: a key row is read by LPK = HD/8 adjacent lanes (8
+//      elements each), the dot finished by xor shuffles over those lanes;
+//   2. one warp per head: tile max, running max m, p = exp(s - m), running sum l, and the
+//      rescale factor of the older keys;
+//   3. o[h] += sum_j p[h][j] v_j, each lane accumulating its 8 dims over its key slot's keys.
+// The key slots' partial outputs are added in slot order at the end.  With part == nullptr
+// (one split) the CTA writes o / l; else (m, l, unnormalised o) per head for
+// decode_merge_kernel, which combines the splits in split order.
+constexpr int DEC_THREADS = 128, DEC_WARPS = DEC_THREADS / 32, DEC_KT_MAX = 128;
+constexpr int DEC_MAX_REP = 8;
+
+// keys per tile: the tile's k and v rows fill 64 KB of shared memory, at most DEC_KT_MAX
+inline int dec_tile_keys(int hd, int es) { return std::min(DEC_KT_MAX, 65536 / (2 * hd * es)); }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// 8 consecutive elements of a shared-memory row (bf16 or fp32)
+__device__ __forceinline__ void smem8(const uint8_t* p, int es, float* v) {
+    if (es == 4) {
+        const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        bf16x8(*reinterpret_cast<const uint4*>(p), v);
+    }
+}
+
+template <int HD, int NREP>
+__global__ void __launch_bounds__(DEC_THREADS) decode_attention_kernel(
     const void* __restrict__ qkv, int ld_qkv, const void* __restrict__ cache, int kv2,
-    const int* __restrict__ cu, const int* __restrict__ lens, int g, int G, int H, int Hkv,
-    float scale, void* __restrict__ out, int ld_out, int dtype, int kps, float* __restrict__ part) {
-    constexpr int HD = DPL * 32;
-    __shared__ float sm_m[DEC_WARPS][DEC_MAX_REP], sm_l[DEC_WARPS][DEC_MAX_REP];
-    __shared__ float sm_o[DEC_WARPS][DEC_MAX_REP][HD];
+    const int* __restrict__ cu, const int* __restrict__ lens, int g, int G, int Hkv, int n_rep,
+    float scale, void* __restrict__ out, int ld_out, int dtype, int kps, int kt,
+    float* __restrict__ part) {
+    constexpr int LPK = HD / 8;                        // lanes per key
+    constexpr int KPW = 32 / LPK;                      // keys per warp-wide access
+    constexpr int SLOTS = DEC_WARPS * KPW;             // keys per CTA-wide access
+    constexpr int U = NREP >= 8 ? 2 : 4;               // keys per lane per round
+    extern __shared__ __align__(16) uint8_t dsm[];
+    const int es = dtype == E_F32 ? 4 : 2;
+    const int row_bytes = HD * es;
+    uint8_t* Ks = dsm;                                 // [kt][HD] elements
+    uint8_t* Vs = dsm + (size_t)kt * row_bytes;        // [kt][HD]
+    float* so = reinterpret_cast<float*>(dsm);         // [SLOTS][NREP][HD], after the last tile
+    const size_t kv_bytes = (size_t)2 * kt * row_bytes, so_bytes = (size_t)SLOTS * NREP * HD * 4;
+    const size_t tiles_bytes = kv_bytes > so_bytes ? kv_bytes : so_bytes;
+    float* sp = reinterpret_cast<float*>(dsm + tiles_bytes);   // [NREP][kt]
+    __shared__ float s_alpha[NREP], s_m[NREP], s_l[NREP];
     const int r = blockIdx.x, kvh = blockIdx.y;
-    const int n_rep = H / Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / LPK, slot = warp * KPW + sub, d0 = (lane % LPK) * 8;
     const size_t base = (size_t)cu[r] + (size_t)r * G;
     const int n = lens[r] + g + 1;
     const int kbeg = blockIdx.z * kps, kend = min(n, kbeg + kps);
     const int kv_dim = kv2 / 2;
-    const int d0 = lane * DPL;
-    float q[DEC_MAX_REP][DPL], o[DEC_MAX_REP][DPL], m[DEC_MAX_REP], l[DEC_MAX_REP];
+    float q[NREP][8], o[NREP][8];
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAX_REP; ++hh) {
-        m[hh] = -FLT_MAX;
-        l[hh] = 0.f;
+    for (int h = 0; h < NREP; ++h) {
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) o[hh][i] = q[hh][i] = 0.f;
-        if (hh < n_rep)
-            load_dims<DPL>(qkv, (size_t)r * ld_qkv + (size_t)(kvh * n_rep + hh) * HD + d0, dtype,
-                           q[hh]);
+        for (int e = 0; e < 8; ++e) o[h][e] = q[h][e] = 0.f;
+        if (h < n_rep)
+            load8(qkv, (size_t)r * ld_qkv + (size_t)(kvh * n_rep + h) * HD + d0, dtype, q[h]);
     }
-    for (int j = kbeg + warp; j < kend; j += DEC_WARPS) {
-        const size_t kr = (base + j) * kv2 + (size_t)kvh * HD + d0;
-        float k[DPL], v[DPL];
-        load_dims<DPL>(cache, kr, dtype, k);
-        load_dims<DPL>(cache, kr + kv_dim, dtype, v);
-#pragma unroll
-        for (int hh = 0; hh < DEC_MAX_REP; ++hh) {
-            if (hh >= n_rep) break;
-            float s_ = 0.f;
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) s_ = fmaf(q[hh][i], k[i], s_);
-            s_ = warp_sum(s_) * scale;
-            const float m_new = fmaxf(m[hh], s_);
-            const float alpha = m[hh] > -FLT_MAX ? expf(m[hh] - m_new) : 0.f;
-            const float p = expf(s_ - m_new);
-            l[hh] = l[hh] * alpha + p;
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) o[hh][i] = fmaf(p, v[i], o[hh][i] * alpha);
-            m[hh] = m_new;
+    if (threadIdx.x < NREP) {
+        s_m[threadIdx.x] = -FLT_MAX;
+        s_l[threadIdx.x] = 0.f;
+    }
+    const char* cbase = static_cast<const char*>(cache);
+    const int chunks = row_bytes / 16;                 // 16-byte pieces per row
+    const uint32_t ks_addr = static_cast<uint32_t>(__cvta_generic_to_shared(Ks));
+    const uint32_t vs_addr = static_cast<uint32_t>(__cvta_generic_to_shared(Vs));
+    for (int t0 = kbeg; t0 < kend; t0 += kt) {
+        const int nt = min(kt, kend - t0);
+        // 0. the tile's k and v rows of this head
+        for (int c = threadIdx.x; c < nt * chunks; c += DEC_THREADS) {
+            const int row = c / chunks, pc = c - row * chunks;
+            const char* src = cbase + ((base + t0 + row) * kv2 + (size_t)kvh * HD) * es + pc * 16;
+            cp_async16(ks_addr + row * row_bytes + pc * 16, src);
+            cp_async16(vs_addr + row * row_bytes + pc * 16, src + (size_t)kv_dim * es);
         }
-    }
+        cp_async_wait_all();
+        __syncthreads();
+        // 1. scores; the loop bounds are uniform over the warp (the shuffles need every lane)
+        for (int i0 = warp * KPW; i0 < nt; i0 += U * SLOTS) {
+            float k[U][8];
 #pragma unroll
-    for (int hh = 0; hh < DEC_MAX_REP; ++hh) {
-        if (hh >= n_rep) break;
-        if (lane == 0) {
-            sm_m[warp][hh] = m[hh];
-            sm_l[warp][hh] = l[hh];
+            for (int u = 0; u < U; ++u) {
+                const int j = i0 + sub + u * SLOTS;
+                if (j < nt) {
+                    smem8(Ks + j * row_bytes + d0 * es, es, k[u]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) k[u][e] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = i0 + sub + u * SLOTS;
+#pragma unroll
+                for (int h = 0; h < NREP; ++h) {
+                    float s_ = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s_ = fmaf(q[h][e], k[u][e], s_);
+#pragma unroll
+                    for (int x = LPK / 2; x > 0; x >>= 1) s_ += __shfl_xor_sync(0xffffffffu, s_, x);
+                    if (d0 == 0 && j < nt) sp[h * kt + j] = s_ * scale;
+                }
+            }
         }
+        __syncthreads();
+        // 2. softmax statistics, one warp per head
+        for (int h = warp; h < NREP; h += DEC_WARPS) {
+            float mx = -FLT_MAX;
+            for (int j = lane; j < nt; j += 32) mx = fmaxf(mx, sp[h * kt + j]);
+            mx = warp_max(mx);
+            const float m_old = s_m[h];
+            const float m_new = fmaxf(m_old, mx);
+            float sum = 0.f;
+            for (int j = lane; j < nt; j += 32) {
+                const float pj = expf(sp[h * kt + j] - m_new);
+                sp[h * kt + j] = pj;
+                sum += pj;
+            }
+            sum = warp_sum(sum);
+            if (lane == 0) {
+                const float alpha = m_old > -FLT_MAX ? expf(m_old - m_new) : 0.f;
+                s_alpha[h] = alpha;
+                s_m[h] = m_new;
+                s_l[h] = s_l[h] * alpha + sum;
+            }
+        }
+        __syncthreads();
+        // 3. o = alpha * o + P V
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) sm_o[warp][hh][d0 + i] = o[hh][i];
+        for (int h = 0; h < NREP; ++h) {
+            const float a = s_alpha[h];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[h][e] *= a;
+        }
+        for (int j = slot; j < nt; j += SLOTS) {
+            float v[8];
+            smem8(Vs + j * row_bytes + d0 * es, es, v);
+#pragma unroll
+            for (int h = 0; h < NREP; ++h) {
+                const float pj = sp[h * kt + j];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pj, v[e], o[h][e]);
+            }
+        }
+        __syncthreads();                               // the tile buffers are refilled next
     }
+    // add the key slots' partial outputs in slot order (so reuses the tile buffers)
+#pragma unroll
+    for (int h = 0; h < NREP; ++h)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) so[(slot * NREP + h) * HD + d0 + e] = o[h][e];
     __syncthreads();
-    // merge the warps' partial softmaxes in a fixed order
     const int S = gridDim.z;
     float* pr = part ? part + ((size_t)(r * Hkv + kvh) * S + blockIdx.z) * n_rep * (HD + 2) : nullptr;
-    for (int idx = threadIdx.x; idx < n_rep * HD; idx += DEC_WARPS * 32) {
-        const int hh = idx / HD, dd = idx % HD;
-        float mm = -FLT_MAX;
-        for (int w = 0; w < DEC_WARPS; ++w) mm = fmaxf(mm, sm_m[w][hh]);
-        float ll = 0.f, acc = 0.f;
-        for (int w = 0; w < DEC_WARPS; ++w) {
-            const float f = sm_m[w][hh] > -FLT_MAX ? expf(sm_m[w][hh] - mm) : 0.f;
-            ll += sm_l[w][hh] * f;
-            acc += sm_o[w][hh][dd] * f;
-        }
+    for (int idx = threadIdx.x; idx < n_rep * HD; idx += DEC_THREADS) {
+        const int h = idx / HD, dd = idx % HD;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int sl = 0; sl < SLOTS; ++sl) acc += so[(sl * NREP + h) * HD + dd];
+        const float ll = s_l[h];
         if (pr) {
-            pr[hh * (HD + 2) + dd] = acc;
+            pr[h * (HD + 2) + dd] = acc;
             if (dd == 0) {
-                pr[hh * (HD + 2) + HD] = mm;
-                pr[hh * (HD + 2) + HD + 1] = ll;
+                pr[h * (HD + 2) + HD] = s_m[h];
+                pr[h * (HD + 2) + HD + 1] = ll;
             }
         } else {
-            st_elem(out, (size_t)r * ld_out + (size_t)(kvh * n_rep + hh) * HD + dd, dtype,
+            st_elem(out, (size_t)r * ld_out + (size_t)(kvh * n_rep + h) * HD + dd, dtype,
                     ll > 0.f ? acc / ll : 0.f);
         }
     }
@@ -213,16 +295,6 @@ __global__ void decode_merge_kernel(const float* __restrict__ part, int S, int n
 // memory (fp32), each of the 256 threads owning one (row, column) dot product, so every
 // factor row is read once per 32 rows and every x row once per 8 columns.
 constexpr int SR_ROWS = 32, SR_COLS = 8, SR_KC = 128;
-
-__device__ __forceinline__ void bf16x8(const uint4& u, float* f) {
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 t = __bfloat1622float2(h[i]);
-        f[2 * i] = t.x;
-        f[2 * i + 1] = t.y;
-    }
-}
 
 // With part != nullptr, blockIdx.z takes K range [z * kspan, (z + 1) * kspan) and writes its
 // raw partial to part[z][m][j]; shrink_rows_sum then adds the parts in z order.
@@ -309,6 +381,7 @@ __global__ void shrink_rows_sum_kernel(const float* __restrict__ part, int ks, i
                                        void* __restrict__ C, int ldc, int c_type,
                                        const int* __restrict__ row_sign, float eps, int scale_cols,
                                        const float* __restrict__ a_scale) {
+    grid_dep_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= M * N) return;
     const int m = i / N, j = i % N;
@@ -364,35 +437,67 @@ void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int
                                         dtype == E_F32 ? 4 : 2);
 }
 
+template <int HD, int NR>
+bool launch_dec(dim3 grid, size_t smem, cudaStream_t st, const void* qkv, int ld_qkv,
+                const void* cache, int kv2, const int* cu, const int* lens, int g, int G, int Hkv,
+                int n_rep, float scale, void* out, int ld_out, int dtype, int kps, int kt,
+                float* part) {
+    static size_t attr = 48 * 1024;
+    if (smem > attr) {
+        if (cudaFuncSetAttribute(decode_attention_kernel<HD, NR>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return false;
+        attr = smem;
+    }
+    decode_attention_kernel<HD, NR><<<grid, DEC_THREADS, smem, st>>>(
+        qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt,
+        part);
+    return cudaGetLastError() == cudaSuccess;
+}
+
+template <int HD>
+bool launch_dec_hd(int nrep_p, dim3 grid, size_t smem, cudaStream_t st, const void* qkv,
+                   int ld_qkv, const void* cache, int kv2, const int* cu, const int* lens, int g,
+                   int G, int Hkv, int n_rep, float scale, void* out, int ld_out, int dtype,
+                   int kps, int kt, float* part) {
+    switch (nrep_p) {
+        case 1: return launch_dec<HD, 1>(grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part);
+        case 2: return launch_dec<HD, 2>(grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part);
+        case 4: return launch_dec<HD, 4>(grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part);
+        default: return launch_dec<HD, 8>(grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part);
+    }
+}
+
 bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int kv2,
                              const int* cu, const int* lens, int R, int g, int G, int H, int Hkv,
                              int hd, float scale, void* out, int ld_out, int dtype, int max_n,
                              float* ws, size_t ws_floats, cudaStream_t st) {
-    if (H / Hkv > DEC_MAX_REP || hd % 32 || hd / 32 > DEC_MAX_DPL) return false;
+    if (Hkv <= 0 || H % Hkv || H / Hkv > DEC_MAX_REP) return false;
+    if (hd != 32 && hd != 64 && hd != 128 && hd != 256) return false;
     if (R == 0) return true;
     const int n_rep = H / Hkv;
-    // with fewer than ~4 (row, kv head) CTAs per SM, split the keys into chunks of 64 so
-    // enough warps stay in flight; the splits' partial softmaxes are combined in order by the
-    // merge kernel
-    constexpr int KPS = 64;
-    int S = (long long)R * Hkv >= 4 * 148 ? 1 : (max_n + KPS - 1) / KPS;
+    const int es = dtype == E_F32 ? 4 : 2;
+    const int kt = dec_tile_keys(hd, es);
+    // with fewer than ~4 (row, kv head) CTAs per SM, split the keys into tiles so enough
+    // copies stay in flight; the splits' partial softmaxes are combined in order by the merge
+    // kernel
+    int S = (long long)R * Hkv >= 4 * 148 ? 1 : (max_n + kt - 1) / kt;
     if (S < 1) S = 1;
     if ((size_t)R * Hkv * S * n_rep * (hd + 2) > ws_floats) S = 1;
-    const int kps = S == 1 ? max_n : KPS;
+    const int kps = S == 1 ? max_n : kt;
     float* part = S > 1 ? ws : nullptr;
+    const int nrep_p = n_rep == 1 ? 1 : n_rep == 2 ? 2 : n_rep <= 4 ? 4 : 8;
+    const size_t slots_bytes = (size_t)(1024 / hd) * nrep_p * hd * 4;
+    const size_t smem = std::max((size_t)2 * kt * hd * es, slots_bytes) + (size_t)nrep_p * kt * 4;
     dim3 grid(R, Hkv, S);
-#define ZO_DEC(DPL)                                                                              \
-    decode_attention_kernel<DPL><<<grid, DEC_WARPS * 32, 0, st>>>(qkv, ld_qkv, cache, kv2, cu,    \
-                                                                 lens, g, G, H, Hkv, scale, out, \
-                                                                 ld_out, dtype, kps, part)
-    switch (hd / 32) {
-        case 1: ZO_DEC(1); break;
-        case 2: ZO_DEC(2); break;
-        case 4: ZO_DEC(4); break;
-        case 8: ZO_DEC(8); break;
-        default: return false;
+    bool ok;
+    switch (hd) {
+        case 32: ok = launch_dec_hd<32>(nrep_p, grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part); break;
+        case 64: ok = launch_dec_hd<64>(nrep_p, grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part); break;
+        case 128: ok = launch_dec_hd<128>(nrep_p, grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part); break;
+        default: ok = launch_dec_hd<256>(nrep_p, grid, smem, st, qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt, part); break;
     }
-#undef ZO_DEC
+    if (!ok) return false;
     if (S > 1) {
         dim3 mg(R, Hkv);
         switch (hd) {
@@ -402,7 +507,7 @@ bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
             default: decode_merge_kernel<256><<<mg, 128, 0, st>>>(part, S, n_rep, Hkv, out, ld_out, dtype); break;
         }
     }
-    return true;
+    return cudaGetLastError() == cudaSuccess;
 }
 
 void launch_shrink_rows(const void* x, int x_type, const void* FT, int ft_type, int M, int N,
@@ -432,6 +537,20 @@ void launch_shrink_rows(const void* x, int x_type, const void* FT, int ft_type, 
     shrink_rows_kernel<<<grid, SR_ROWS * SR_COLS, 0, st>>>(x, x_type, FT, ft_type, M, N, K, C, ldc,
                                                            c_type, row_sign, eps, scale_cols,
                                                            a_scale, nullptr, 0);
+}
+
+void launch_shrink_rows_sum(const float* part, int ks, int M, int N, void* C, int ldc, int c_type,
+                            const int* row_sign, float eps, int scale_cols, const float* a_scale,
+                            cudaStream_t st, bool pdl) {
+    if (M == 0 || N == 0) return;
+    const dim3 grid(cdiv((long long)M * N, 256));
+    if (pdl) {
+        launch_pdl(shrink_rows_sum_kernel, grid, dim3(256), 0, st, part, ks, M, N, C, ldc, c_type,
+                   row_sign, eps, scale_cols, a_scale);
+        return;
+    }
+    shrink_rows_sum_kernel<<<grid, 256, 0, st>>>(part, ks, M, N, C, ldc, c_type, row_sign, eps,
+                                                 scale_cols, a_scale);
 }
 
 void launch_last_tokens(const int* cu, int R, int* out, int* lens, cudaStream_t st) {

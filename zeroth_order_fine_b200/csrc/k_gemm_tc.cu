@@ -374,6 +374,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     using T1 = Tile1<BNT>;
     constexpr int STAGES = T1::STAGES;
     constexpr int STAGE_BYTES = T1::STAGE_BYTES;
+    if (EPI == EPI_SPLIT_T) {
+        // launched as a dependent of the kernel that wrote its operands; its split reduction
+        // is launched as a dependent of this one
+        grid_dep_wait();
+        grid_dep_launch();
+    }
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;           // 1024-aligned for SW128
@@ -1206,6 +1212,9 @@ int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2
     }
     const int items = EPI == EPI_SPLIT_T ? p.n_tiles * p.ksplit : p.n_tiles;
     const int grid = items < num_sms() ? items : num_sms();
+    if (EPI == EPI_SPLIT_T)
+        return launch_pdl(gemm_tc_kernel<EPI, BNT>, dim3(grid), dim3(NUM_THREADS), smem, st, a, b,
+                          a2, b2, p) == cudaSuccess ? 0 : 1;
     gemm_tc_kernel<EPI, BNT><<<grid, NUM_THREADS, smem, st>>>(a, b, a2, b2, p);
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
@@ -1270,6 +1279,7 @@ namespace {
 // or the fp32 residual add.  One thread per 4 columns.
 __global__ void splitk_epilogue_kernel(const float* __restrict__ ws, int ks, int M, int N,
                                        const float* __restrict__ bias, int epi, void* C, int ldc) {
+    grid_dep_wait();
     const int m = blockIdx.y;
     const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (n >= N) return;
@@ -1299,6 +1309,7 @@ __global__ void splitk_epilogue_kernel(const float* __restrict__ ws, int ks, int
 // reads column (f / 128) * 256 + f % 128 (gate) and the one 128 after it (up).
 __global__ void splitk_swiglu_kernel(const float* __restrict__ ws, int ks, int M, int N,
                                      const float* __restrict__ bias, __nv_bfloat16* C, int ldc) {
+    grid_dep_wait();
     const int m = blockIdx.y;
     const int f = blockIdx.x * blockDim.x + threadIdx.x;
     const int F = N / 2;
@@ -1323,6 +1334,7 @@ __global__ void splitk_swiglu_kernel(const float* __restrict__ ws, int ks, int M
 // columns sit in lane l ^ 16.
 __global__ void splitk_qknr_kernel(const float* __restrict__ ws, int ks, int M, int N, TcParams p,
                                    __nv_bfloat16* C, int ldc) {
+    grid_dep_wait();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int heads = N / 128;
     if (warp >= M * heads) return;
@@ -1372,22 +1384,34 @@ bool make_map_ws(CUtensorMap* m, const float* ws, int ks, int M, int N) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The split reduction of a [ks][M][N] workspace into g.C with g's epilogue.
-int launch_split_reduce(const GemmArgs& g, const TcParams& p, int ks, cudaStream_t st) {
-    if (g.epi == EPI_SWIGLU) {
-        dim3 grid((unsigned)((g.N / 2 + 127) / 128), (unsigned)g.M);
-        splitk_swiglu_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias,
-                                                   static_cast<__nv_bfloat16*>(g.C), g.ldc);
+// The split reduction of a [ks][M][N] workspace into g.C with g's epilogue; with pdl it is
+// launched as a programmatic dependent of the GEMM that wrote the slices.
+int launch_split_reduce(const GemmArgs& g, const TcParams& p, int ks, cudaStream_t st, bool pdl) {
+    cudaError_t e = cudaSuccess;
+    auto go = [&](auto kernel, dim3 grid, auto... args) {
+        if (pdl) {
+            e = launch_pdl(kernel, grid, dim3(128), 0, st, args...);
+        } else {
+            kernel<<<grid, 128, 0, st>>>(args...);
+            e = cudaGetLastError();
+        }
+    };
+    if (g.epi == EPI_SHRINK) {
+        launch_shrink_rows_sum(g.ws, ks, g.M, g.N, g.C, g.ldc, g.c_type, g.row_sign, g.eps,
+                               g.scale_cols, g.a_scale, st, pdl);
+        e = cudaGetLastError();
+    } else if (g.epi == EPI_SWIGLU) {
+        go(splitk_swiglu_kernel, dim3((unsigned)((g.N / 2 + 127) / 128), (unsigned)g.M),
+           (const float*)g.ws, ks, g.M, g.N, g.bias, static_cast<__nv_bfloat16*>(g.C), g.ldc);
     } else if (g.epi == EPI_QKNR) {
         const long long warps = (long long)g.M * (g.N / 128);
-        splitk_qknr_kernel<<<(unsigned)((warps + 3) / 4), 128, 0, st>>>(
-            g.ws, ks, g.M, g.N, p, static_cast<__nv_bfloat16*>(g.C), g.ldc);
+        go(splitk_qknr_kernel, dim3((unsigned)((warps + 3) / 4)), (const float*)g.ws, ks, g.M, g.N,
+           p, static_cast<__nv_bfloat16*>(g.C), g.ldc);
     } else {
-        dim3 grid((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M);
-        splitk_epilogue_kernel<<<grid, 128, 0, st>>>(g.ws, ks, g.M, g.N, g.bias, g.epi, g.C,
-                                                     g.ldc);
+        go(splitk_epilogue_kernel, dim3((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M),
+           (const float*)g.ws, ks, g.M, g.N, g.bias, g.epi, g.C, g.ldc);
     }
-    return cudaGetLastError() == cudaSuccess ? 0 : 1;
+    return e == cudaSuccess ? 0 : 1;
 }
 
 // Splits of kb_main K blocks into ks parts of kbs blocks: the number of non-empty parts.
@@ -1461,7 +1485,7 @@ int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
         default: rc = launch_epi<EPI_SPLIT_T, 128>(a, b, a2, b2, p, st); break;
     }
     if (rc) return rc;
-    return launch_split_reduce(g, p, ks, st);
+    return launch_split_reduce(g, p, ks, st, true);
 }
 
 }  // namespace
@@ -1526,7 +1550,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     // their few token rows take the swapped single-SM form.
     if (g.ws && g.M <= 128 && g.a_type == E_BF16 && g.b_type == E_BF16 && g.N % 4 == 0 &&
         (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
-         g.epi == EPI_SWIGLU || g.epi == EPI_QKNR))
+         g.epi == EPI_SWIGLU || g.epi == EPI_QKNR || g.epi == EPI_SHRINK))
         return gemm_tc_swapped(g, st);
     const bool pair = g_use_pairs && g.N > 128 &&
                       (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
@@ -1590,7 +1614,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
             // the split kernels' epilogue only stores fp32 slices: one instantiation serves all
             const int rc = launch_epi2<EPI_STORE, false, true>(a, b, a2, b2, c, p, st);
             if (rc) return rc;
-            return launch_split_reduce(g, p, ks, st);
+            return launch_split_reduce(g, p, ks, st, false);
         }
     }
     if (pair) {

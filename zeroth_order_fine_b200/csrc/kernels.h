@@ -177,6 +177,12 @@ bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
 // (j < scale_cols ? row_sign[m] * eps : 1) / (a_scale ? a_scale[m] : 1); x [M x K] in
 // x_type, FT [N x K] in ft_type, C [M x ldc] in c_type.
 // ws (optional, ws_floats floats): lets K split over more CTAs, the parts summed in order.
+// The ordered sum of ks fp32 slices part[z][M][N] with the bank-shrink epilogue (columns below
+// scale_cols times row_sign[m] * eps, then / a_scale[m] when given), stored to C (c_type);
+// pdl: launched as a programmatic dependent of the kernel that wrote part.
+void launch_shrink_rows_sum(const float* part, int ks, int M, int N, void* C, int ldc, int c_type,
+                            const int* row_sign, float eps, int scale_cols, const float* a_scale,
+                            cudaStream_t st, bool pdl);
 void launch_shrink_rows(const void* x, int x_type, const void* FT, int ft_type, int M, int N,
                         int K, void* C, int ldc, int c_type, const int* row_sign, float eps,
                         int scale_cols, const float* a_scale, float* ws, size_t ws_floats,
