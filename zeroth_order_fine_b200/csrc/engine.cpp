@@ -1001,7 +1001,7 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
     for (int l = 0; l < d.n_layers; ++l) {
         Layer& L = h->layers[l];
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps, h->xn,
-                    h->dt, h->st, h->xq, h->sx);
+                    h->dt, h->st, h->xq, h->sx, decode);
         int rc = group_gemm(h, L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
                             h->n_qkv, h->dt, Ti, eps, &L, decode);
         if (rc) return rc;
@@ -1014,7 +1014,7 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
         rc = group_gemm(h, L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr, decode);
         if (rc) return rc;
         launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps, h->xn,
-                    h->dt, h->st, h->xq, h->sx);
+                    h->dt, h->st, h->xq, h->sx, decode);
         if (d.arch == ZO_ARCH_OPT) {
             rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt, Ti, eps, nullptr, decode);
         } else if (h->swiglu_fused) {

@@ -55,6 +55,8 @@ __global__ void decode_prep_kernel(const int* __restrict__ gen_tok, int G, int g
 __global__ void kv_append_kernel(const char* __restrict__ qkv, int ld_qkv, int q_dim, int kv2,
                                  const int* __restrict__ cu, const int* __restrict__ lens, int g,
                                  int G, char* __restrict__ cache, int es) {
+    grid_dep_wait();                    // launched as a programmatic dependent
+    grid_dep_launch();
     const int r = blockIdx.x;
     const size_t crow = (size_t)cu[r] + (size_t)r * G + lens[r] + g;
     copy_row(qkv + ((size_t)r * ld_qkv + q_dim) * es, cache + crow * kv2 * es, kv2, es);
@@ -129,6 +131,8 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_attention_kernel(
     constexpr int KPW = 32 / LPK;                      // keys per warp-wide access
     constexpr int SLOTS = DEC_WARPS * KPW;             // keys per CTA-wide access
     constexpr int U = NREP >= 8 ? 2 : 4;               // keys per lane per round
+    grid_dep_wait();                                   // launched as a programmatic dependent
+    grid_dep_launch();
     extern __shared__ __align__(16) uint8_t dsm[];
     const int es = dtype == E_F32 ? 4 : 2;
     const int row_bytes = HD * es;
@@ -273,6 +277,8 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_attention_kernel(
 template <int HD>
 __global__ void decode_merge_kernel(const float* __restrict__ part, int S, int n_rep, int Hkv,
                                     void* __restrict__ out, int ld_out, int dtype) {
+    grid_dep_wait();                    // launched as a programmatic dependent
+    grid_dep_launch();
     const int r = blockIdx.x, kvh = blockIdx.y;
     const float* pr = part + (size_t)(r * Hkv + kvh) * S * n_rep * (HD + 2);
     for (int idx = threadIdx.x; idx < n_rep * HD; idx += blockDim.x) {
@@ -432,9 +438,8 @@ void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int
                       const int* lens, int R, int g, int G, void* cache, int dtype,
                       cudaStream_t st) {
     if (R == 0) return;
-    kv_append_kernel<<<R, 128, 0, st>>>(static_cast<const char*>(qkv), ld_qkv, q_dim, kv2, cu,
-                                        lens, g, G, static_cast<char*>(cache),
-                                        dtype == E_F32 ? 4 : 2);
+    launch_pdl(kv_append_kernel, dim3(R), dim3(128), 0, st, static_cast<const char*>(qkv), ld_qkv,
+               q_dim, kv2, cu, lens, g, G, static_cast<char*>(cache), dtype == E_F32 ? 4 : 2);
 }
 
 template <int HD, int NR>
@@ -449,10 +454,9 @@ bool launch_dec(dim3 grid, size_t smem, cudaStream_t st, const void* qkv, int ld
             return false;
         attr = smem;
     }
-    decode_attention_kernel<HD, NR><<<grid, DEC_THREADS, smem, st>>>(
-        qkv, ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps, kt,
-        part);
-    return cudaGetLastError() == cudaSuccess;
+    return launch_pdl(decode_attention_kernel<HD, NR>, grid, dim3(DEC_THREADS), smem, st, qkv,
+                      ld_qkv, cache, kv2, cu, lens, g, G, Hkv, n_rep, scale, out, ld_out, dtype, kps,
+                      kt, part) == cudaSuccess;
 }
 
 template <int HD>
@@ -501,10 +505,10 @@ bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
     if (S > 1) {
         dim3 mg(R, Hkv);
         switch (hd) {
-            case 32: decode_merge_kernel<32><<<mg, 128, 0, st>>>(part, S, n_rep, Hkv, out, ld_out, dtype); break;
-            case 64: decode_merge_kernel<64><<<mg, 128, 0, st>>>(part, S, n_rep, Hkv, out, ld_out, dtype); break;
-            case 128: decode_merge_kernel<128><<<mg, 128, 0, st>>>(part, S, n_rep, Hkv, out, ld_out, dtype); break;
-            default: decode_merge_kernel<256><<<mg, 128, 0, st>>>(part, S, n_rep, Hkv, out, ld_out, dtype); break;
+            case 32: launch_pdl(decode_merge_kernel<32>, mg, dim3(128), 0, st, (const float*)part, S, n_rep, Hkv, out, ld_out, dtype); break;
+            case 64: launch_pdl(decode_merge_kernel<64>, mg, dim3(128), 0, st, (const float*)part, S, n_rep, Hkv, out, ld_out, dtype); break;
+            case 128: launch_pdl(decode_merge_kernel<128>, mg, dim3(128), 0, st, (const float*)part, S, n_rep, Hkv, out, ld_out, dtype); break;
+            default: launch_pdl(decode_merge_kernel<256>, mg, dim3(128), 0, st, (const float*)part, S, n_rep, Hkv, out, ld_out, dtype); break;
         }
     }
     return cudaGetLastError() == cudaSuccess;

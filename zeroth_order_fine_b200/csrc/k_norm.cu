@@ -124,6 +124,8 @@ __global__ void __launch_bounds__(256) norm_vec_kernel(const float* __restrict__
                                                        void* __restrict__ out, int out_type,
                                                        uint8_t* __restrict__ q8,
                                                        float* __restrict__ s8) {
+    grid_dep_wait();                    // a no-op unless launched as a programmatic dependent
+    grid_dep_launch();
     __shared__ float red[32];
     const int t = blockIdx.x;
     const int src = rows ? rows[t] : t;
@@ -238,23 +240,34 @@ void launch_quant_rows_e4m3(const void* x, int x_type, int rows, int cols, size_
 
 bool norm_fp8_supported(int d) { return d % 4 == 0 && (d / 4 + 255) / 256 <= 8; }
 
+template <int VPT>
+void norm_vec_go(bool pdl, int T, cudaStream_t st, const float* x, const int* rows, int d, int kind,
+                 const float* w, const float* b, float eps, void* out, int out_type, uint8_t* q8,
+                 float* s8) {
+    if (pdl)
+        launch_pdl(norm_vec_kernel<VPT>, dim3(T), dim3(256), 0, st, x, rows, d, kind, w, b, eps,
+                   out, out_type, q8, s8);
+    else
+        norm_vec_kernel<VPT><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8);
+}
+
 void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
                  const float* b, float eps, void* out, int out_type, cudaStream_t st,
-                 uint8_t* q8, float* s8) {
+                 uint8_t* q8, float* s8, bool pdl) {
     if (T == 0) return;
     const int vpt = (d / 4 + 255) / 256;
     auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
     const bool aligned = al16(x) && al16(w) && (b == nullptr || al16(b)) && al16(out);
     if (d % 4 == 0 && vpt <= 8 && aligned) {
         switch (vpt) {
-            case 1: norm_vec_kernel<1><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
-            case 2: norm_vec_kernel<2><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
-            case 3: norm_vec_kernel<3><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
-            case 4: norm_vec_kernel<4><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
-            case 5: norm_vec_kernel<5><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
-            case 6: norm_vec_kernel<6><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
-            case 7: norm_vec_kernel<7><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
-            default: norm_vec_kernel<8><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 1: norm_vec_go<1>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 2: norm_vec_go<2>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 3: norm_vec_go<3>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 4: norm_vec_go<4>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 5: norm_vec_go<5>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 6: norm_vec_go<6>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            case 7: norm_vec_go<7>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
+            default: norm_vec_go<8>(pdl, T, st, x, rows, d, kind, w, b, eps, out, out_type, q8, s8); return;
         }
     }
     norm_kernel<<<T, 256, d * sizeof(float), st>>>(x, rows, d, kind, w, b, eps, out, out_type);

@@ -57,10 +57,11 @@ void launch_embed(const int* tok_id, const int* tok_pos, const void* tok_embed,
 // an all-zero row has scale 1.  x is fp32 or bf16 [rows x ldx], q [rows x ldq] bytes.
 void launch_quant_rows_e4m3(const void* x, int x_type, int rows, int cols, size_t ldx,
                             uint8_t* q, size_t ldq, float* scale, cudaStream_t st);
-// q8/s8 (optional, vectorised path only): also the E4M3 quantisation of the bf16 output rows
+// q8/s8 (optional, vectorised path only): also the E4M3 quantisation of the bf16 output rows;
+// pdl: the vectorised form is launched as a programmatic dependent of the kernel before it
 void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,
                  const float* b, float eps, void* out, int out_type, cudaStream_t st,
-                 uint8_t* q8 = nullptr, float* s8 = nullptr);
+                 uint8_t* q8 = nullptr, float* s8 = nullptr, bool pdl = false);
 bool norm_fp8_supported(int d);
 void launch_swiglu(const void* gu, int T, int f, void* out, int dtype, cudaStream_t st);
 void launch_rope_table(float* cos_t, float* sin_t, int max_pos, int hd, double theta,
