@@ -15,6 +15,7 @@ clocks and the kernel launch count are reported on the same line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -329,6 +330,9 @@ def run_generate(args, w: wl.Workload):
 
     from zeroth_order_fine_b200 import zo
     G = args.generate
+    if args.layers:
+        # fewer decoder layers of the same shapes: small device footprint for profiler captures
+        w = dataclasses.replace(w, shape=dataclasses.replace(w.shape, n_layers=args.layers))
     sh = w.shape
     batch = wl.make_batch(w, fg_rows=0)
     model = zo.DeviceModel(sh, w.weight_seed)
@@ -370,7 +374,8 @@ def run_generate(args, w: wl.Workload):
     roof_ms = (t_prefill + t_decode) * 1000.0
     s = h.zo_stats()
     print(json.dumps({
-        "mode": "generate", "workload": w.name, "new_tokens_per_row": G, "rows": 2 * B,
+        "mode": "generate", "workload": w.name, "layers": sh.n_layers, "new_tokens_per_row": G,
+        "rows": 2 * B,
         "prompt_tokens": T, "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
         "generated_tokens_per_s": 2 * B * G / (ms / 1000.0),
         "dtype": "e4m3 (q|k|v, FFN-in) + bf16" if args.fp8 else "bf16",
@@ -395,6 +400,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the whole-step CUDA graph leg")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="with --generate: run only this many decoder layers of the workload's "
+                         "shapes (profiler captures; not a bench line)")
     ap.add_argument("--generate", type=int, default=0,
                     help="generation-query steps: greedy tokens per candidate row (zo_generate)")
     ap.add_argument("--fp8", action="store_true",
