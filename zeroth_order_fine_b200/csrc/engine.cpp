@@ -981,7 +981,7 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
     g.bias = G.bias;
     g.epi = epi;
     g.C = C; g.ldc = ldc; g.c_type = ctype;
-    if (decode) {                         // few rows: the GEMM may split K over the SM pairs
+    if (decode) {                         // few rows: the GEMM splits K (swapped operands)
         g.ws = h->splitk_ws;
         g.ws_floats = h->splitk_floats;
     }
