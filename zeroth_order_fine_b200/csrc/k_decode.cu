@@ -481,13 +481,16 @@ bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
     if (R == 0) return true;
     const int n_rep = H / Hkv;
     const int es = dtype == E_F32 ? 4 : 2;
-    const int kt = dec_tile_keys(hd, es);
+    int kt = dec_tile_keys(hd, es);
     // with fewer than ~4 (row, kv head) CTAs per SM, split the keys into tiles so enough
     // copies stay in flight; the splits' partial softmaxes are combined in order by the merge
-    // kernel
-    int S = (long long)R * Hkv >= 4 * 148 ? 1 : (max_n + kt - 1) / kt;
+    // kernel.  Without a split a CTA walks its keys in half-size tiles: twice the CTAs fit on
+    // an SM (2.7% faster OPT-13B b16 generation steps; with splits the full tile was faster).
+    const bool many = (long long)R * Hkv >= 4 * 148;
+    int S = many ? 1 : (max_n + kt - 1) / kt;
     if (S < 1) S = 1;
     if ((size_t)R * Hkv * S * n_rep * (hd + 2) > ws_floats) S = 1;
+    if (S == 1) kt = std::max(16, kt / 2);
     const int kps = S == 1 ? max_n : kt;
     float* part = S > 1 ? ws : nullptr;
     const int nrep_p = n_rep == 1 ? 1 : n_rep == 2 ? 2 : n_rep <= 4 ? 4 : 8;
