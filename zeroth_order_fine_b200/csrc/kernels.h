@@ -112,7 +112,8 @@ struct GemmArgs {
     // optional fp32 workspace (ws_floats floats) for decode steps: the bf16 store / ReLU /
     // residual / SwiGLU / q-k-norm GEMMs split K, over single SMs with the operands swapped
     // (M <= 128 token rows as the narrow N side) or over the SM pairs (larger M), and a
-    // reduction sums the slices in order and applies the epilogue
+    // reduction sums the slices in order and applies the epilogue.  Callers give at least
+    // M x N floats (one slice); more room allows more splits.
     float* ws; size_t ws_floats;
 };
 
