@@ -59,8 +59,8 @@ def test_tiny_fp32_generation_matches_oracle(impl):
 
 
 def test_opt_width_bf16_generation_matches_oracle():
-    """Two full-width OPT-1.3B layers (d = 2048, vocab 50272): the decode GEMMs have few
-    output tiles for their 8 rows and split K over the SM pairs."""
+    """Two full-width OPT-1.3B layers (d = 2048, vocab 50272): the decode GEMMs stream the
+    weights for their 8 rows on the swapped single-SM kernel with K split over the SMs."""
     w = wl.WORKLOADS["opt-1.3b-b16"]
     w = dataclasses.replace(w, shape=wl.shrink_shape(w.shape, n_layers=2), batch=4, len_hi=48)
     _check_against_oracle(w, False, 5e-2, 3e-2, 2e-2)
@@ -87,6 +87,22 @@ def test_qwen3_wide_bf16_generation_matches_oracle():
 
 def test_qwen3_fp8_generation_matches_oracle():
     _check_against_oracle(QWEN_SMALL, True, 5e-2, 3e-2, 2e-2)
+
+
+@pytest.mark.parametrize("heads,kv_heads", [(6, 2), (8, 1)], ids=["group3", "group8"])
+def test_qwen3_query_group_sizes_generation_matches_oracle(heads, kv_heads):
+    """Query-head groups of 3 (the decode attention pads them to 4 with zero queries) and of
+    8 per kv head."""
+    shape = dataclasses.replace(Q3_SMALL_BF16, name=f"qwen3-group{heads // kv_heads}",
+                                n_heads=heads, n_kv_heads=kv_heads)
+    _check_against_oracle(dataclasses.replace(QWEN_SMALL, shape=shape), False, 5e-2, 3e-2, 2e-2)
+
+
+def test_qwen3_long_prompts_generation_matches_oracle():
+    """Prompts of 150-300 tokens: with few (row, kv head) pairs the decode attention splits
+    each row's keys over several CTAs and merges the partial softmaxes in order."""
+    w = dataclasses.replace(QWEN_SMALL, len_lo=150, len_hi=300)
+    _check_against_oracle(w, False, 5e-2, 3e-2, 2e-2)
 
 
 @pytest.mark.parametrize("w", [TINY, TINY_BF16, QWEN_SMALL], ids=["fp32", "bf16", "qwen3-bf16"])
