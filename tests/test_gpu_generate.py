@@ -89,6 +89,14 @@ def test_qwen3_fp8_generation_matches_oracle():
     _check_against_oracle(QWEN_SMALL, True, 5e-2, 3e-2, 2e-2)
 
 
+def test_opt_width_fp8_generation_matches_oracle():
+    """E4M3 q|k|v and fc1 at OPT-1.3B width: the decode steps run them on the swapped
+    single-SM kernel with kind::f8f6f4 main blocks and the bf16 bank extension."""
+    w = wl.WORKLOADS["opt-1.3b-b16"]
+    w = dataclasses.replace(w, shape=wl.shrink_shape(w.shape, n_layers=2), batch=4, len_hi=48)
+    _check_against_oracle(w, True, 5e-2, 3e-2, 2e-2)
+
+
 @pytest.mark.parametrize("heads,kv_heads", [(6, 2), (8, 1)], ids=["group3", "group8"])
 def test_qwen3_query_group_sizes_generation_matches_oracle(heads, kv_heads):
     """Query-head groups of 3 (the decode attention pads them to 4 with zero queries) and of

@@ -36,6 +36,7 @@ namespace zo {
 namespace {
 
 constexpr int BM = 128, BK = 64, BN = 256;
+constexpr int BK8 = 128;                    // E4M3 K block: the same 128-byte rows
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int TMEM_COLS = 512;              // two BN-wide fp32 accumulators
 constexpr int GROUP_M = 8;
@@ -58,6 +59,9 @@ struct Tile1 {
     // bf16 x bf16 -> fp32, both K-major, M = 128, N = BNT
     static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
                                       ((uint32_t)(BNT >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    // kind::f8f6f4, A and B both E4M3 (format code 0), fp32 accumulate, M = 128, N = BNT
+    static constexpr uint32_t IDESC_F8 = (1u << 4) | ((uint32_t)(BNT >> 3) << 17) |
+                                         ((uint32_t)(BM >> 4) << 24);
     // barriers (8 B each: full, empty per stage; tfull, tempty per accumulator; drain)
     // then the TMEM base and the abort flag, all inside the 256-byte tail
     static constexpr int SLOT_OFF = 240, ABORT_OFF = 248;
@@ -160,6 +164,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
         : "memory");
 }
@@ -366,7 +379,9 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, int m, int nb
     }
 }
 
-template <int EPI, int BNT>
+// F8 (EPI_SPLIT_T only): the main K blocks are E4M3 (kind::f8f6f4, 128 elements per block),
+// the extension blocks bf16, into the same accumulator; the epilogue dequantises.
+template <int EPI, int BNT, bool F8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
@@ -456,8 +471,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t sb = sa + A_BYTES;
                     mbar_expect_tx(full(s), STAGE_BYTES);
                     if (kb < p.kb_main) {
-                        tma_load_2d(sa, &tmA, full(s), kb * BK, mb * BM);
-                        tma_load_2d(sb, &tmB, full(s), kb * BK, nb * BNT);
+                        tma_load_2d(sa, &tmA, full(s), kb * (F8 ? BK8 : BK), mb * BM);
+                        tma_load_2d(sb, &tmB, full(s), kb * (F8 ? BK8 : BK), nb * BNT);
                     } else {
                         const int k = (kb - p.kb_main) * BK;
                         tma_load_2d(sa, &tmA2, full(s), k, mb * BM);
@@ -497,10 +512,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tc_fence_after();
                     const uint32_t sa = base + s * STAGE_BYTES;
                     const uint32_t sb = sa + A_BYTES;
+                    if (F8 && i < n_main) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
-                               (i > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)   // K = 32 E4M3 elements = 32 bytes each
+                            tc_mma_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
+                                      T1::IDESC_F8, (i > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
+                                   (i > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     issued = true;
                     tc_commit(empty(s));            // stage free once these MMAs retire
@@ -538,6 +560,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     float v[32];
                     tmem_ld32(tmem + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BNT + c * 32), v);
                     if (m < p.M) {
+                        if (F8) {
+                            // E4M3 units back to real ones: times the token's scale (N side),
+                            // then the weight row's (M side), the order the SM-pair kernel uses
+                            const float sw = __ldg(p.a_scale + m);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (n + j < p.N) v[j] = v[j] * __ldg(p.b_scale + n + j) * sw;
+                        }
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             if (n + j < p.N) slice[(size_t)(n + j) * p.M + m] = v[j];
@@ -596,7 +626,6 @@ constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN
 // stage holds the same 128-byte rows, so 128 K elements instead of 64 and each of the
 // four MMAs per stage covers K = 32.
 constexpr uint32_t kIdesc2F8 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM2 >> 4) << 24);
-constexpr int BK8 = 128;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -1199,13 +1228,13 @@ int num_sms() {
     return n;
 }
 
-template <int EPI, int BNT>
+template <int EPI, int BNT, bool F8 = false>
 int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
     constexpr int smem = Tile1<BNT>::SMEM_BYTES;
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI, BNT>,
+        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI, BNT, F8>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return 1;
         attr = true;
@@ -1213,9 +1242,9 @@ int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2
     const int items = EPI == EPI_SPLIT_T ? p.n_tiles * p.ksplit : p.n_tiles;
     const int grid = items < num_sms() ? items : num_sms();
     if (EPI == EPI_SPLIT_T)
-        return launch_pdl(gemm_tc_kernel<EPI, BNT>, dim3(grid), dim3(NUM_THREADS), smem, st, a, b,
+        return launch_pdl(gemm_tc_kernel<EPI, BNT, F8>, dim3(grid), dim3(NUM_THREADS), smem, st, a, b,
                           a2, b2, p) == cudaSuccess ? 0 : 1;
-    gemm_tc_kernel<EPI, BNT><<<grid, NUM_THREADS, smem, st>>>(a, b, a2, b2, p);
+    gemm_tc_kernel<EPI, BNT, F8><<<grid, NUM_THREADS, smem, st>>>(a, b, a2, b2, p);
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
 
@@ -1426,9 +1455,10 @@ int effective_splits(int kb_main, int ks, int* kbs) {
 // the workspace, then the split reduction applies g's epilogue.
 int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
     const int bnt = g.M <= 32 ? 32 : (g.M <= 64 ? 64 : 128);
+    const bool f8 = g.a_type == E_FP8;                // E4M3 main blocks (both operands)
     CUtensorMap a, b, a2, b2;
-    if (!make_map(&a, g.B, g.N, g.K, g.ldb, BM)) return 1;
-    if (!make_map(&b, g.A, g.M, g.K, g.lda, bnt)) return 1;
+    if (!make_map(&a, g.B, g.N, g.K, g.ldb, BM, f8)) return 1;
+    if (!make_map(&b, g.A, g.M, g.K, g.lda, bnt, f8)) return 1;
     if (g.K2 > 0) {
         if (!make_map(&a2, g.B2, g.N, g.K2, g.ldb2, BM)) return 1;
         if (!make_map(&b2, g.A2, g.M, g.K2, g.lda2, bnt)) return 1;
@@ -1439,8 +1469,10 @@ int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
     TcParams p;
     memset(&p, 0, sizeof(p));
     p.M = g.N; p.N = g.M;
-    p.kb_main = (g.K + BK - 1) / BK;
+    p.kb_main = f8 ? (g.K + BK8 - 1) / BK8 : (g.K + BK - 1) / BK;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
+    // swapped sides: the weight rows' scales are the kernel's M side, the tokens' its N side
+    p.a_scale = g.b_scale; p.b_scale = g.a_scale;
     p.n_m_blk = (g.N + BM - 1) / BM;
     p.n_n_blk = 1;
     p.n_tiles = p.n_m_blk;
@@ -1479,10 +1511,13 @@ int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
     ks = effective_splits(p.kb_main, ks, &p.kbs);
     p.ksplit = ks;
     int rc;
-    switch (bnt) {
+    switch (bnt + (f8 ? 1 : 0)) {
         case 32: rc = launch_epi<EPI_SPLIT_T, 32>(a, b, a2, b2, p, st); break;
         case 64: rc = launch_epi<EPI_SPLIT_T, 64>(a, b, a2, b2, p, st); break;
-        default: rc = launch_epi<EPI_SPLIT_T, 128>(a, b, a2, b2, p, st); break;
+        case 128: rc = launch_epi<EPI_SPLIT_T, 128>(a, b, a2, b2, p, st); break;
+        case 33: rc = launch_epi<EPI_SPLIT_T, 32, true>(a, b, a2, b2, p, st); break;
+        case 65: rc = launch_epi<EPI_SPLIT_T, 64, true>(a, b, a2, b2, p, st); break;
+        default: rc = launch_epi<EPI_SPLIT_T, 128, true>(a, b, a2, b2, p, st); break;
     }
     if (rc) return rc;
     return launch_split_reduce(g, p, ks, st, true);
@@ -1548,7 +1583,9 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     // choice never depends on M (the batch): a row's bits must not change with
     // the company it is scored in.  Decode steps (a workspace given) are the exception:
     // their few token rows take the swapped single-SM form.
-    if (g.ws && g.M <= 128 && g.a_type == E_BF16 && g.b_type == E_BF16 && g.N % 4 == 0 &&
+    const bool bf16_ops = g.a_type == E_BF16 && g.b_type == E_BF16;
+    const bool e4m3_ops = g.a_type == E_FP8 && g.b_type == E_FP8 && g.a_scale && g.b_scale;
+    if (g.ws && g.M <= 128 && (bf16_ops || e4m3_ops) && g.N % 4 == 0 &&
         (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
          g.epi == EPI_SWIGLU || g.epi == EPI_QKNR || g.epi == EPI_SHRINK))
         return gemm_tc_swapped(g, st);
