@@ -101,6 +101,21 @@ def step_work(w: wl.Workload, batches, n_slots: int):
     return flops, bytes_, T_all, S_all
 
 
+def generate_work(w: wl.Workload, batch, G: int):
+    """(prefill FLOPs, decode bytes) of one generation step of G new tokens per row: the
+    prompts of both candidates as one packed prefill (the scoring step's FLOPs), then G - 1
+    decode steps that each read every weight and the lm_head once and each row's k|v cache
+    (its prompt plus the tokens generated so far) once."""
+    sh = w.shape
+    es = 2 if sh.dtype == wl.DTYPE_BF16 else 4
+    flops, _, _, _ = step_work(w, [batch], 1)
+    w_bytes = (sh.body_params() + sh.vocab * sh.d_model) * es
+    kv_row = 2 * sh.kv_dim * sh.n_layers * es
+    lens = np.concatenate([batch.seq_lens, batch.seq_lens]).astype(np.float64)
+    kv_bytes = sum(float(np.sum(lens + g + 1)) * kv_row for g in range(G - 1))
+    return flops, (G - 1) * w_bytes + kv_bytes
+
+
 def fp8_flops(w: wl.Workload, batches) -> float:
     """The part of step_work's FLOPs that the fp8 option runs in E4M3: the base products of
     q|k|v and the FFN input projections (the norm-fed matrices)."""
@@ -361,16 +376,9 @@ def run_generate(args, w: wl.Workload):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     peaks, peak_kind = load_peaks()
-    es = 2 if sh.dtype == wl.DTYPE_BF16 else 4
-    # prefill: the scoring step's FLOPs at its own roofline; every decode step reads the
-    # weights (and lm_head) once and each row's cache once
-    flops, _, _, _ = step_work(w, [batch], 1)
-    w_bytes = (sh.body_params() + sh.vocab * sh.d_model) * es
-    kv_row = 2 * sh.kv_dim * sh.n_layers * es
-    lens = np.concatenate([batch.seq_lens, batch.seq_lens]).astype(np.float64)
-    kv_bytes = sum(float(np.sum(lens + g + 1)) * kv_row for g in range(G - 1))
+    flops, decode_bytes = generate_work(w, batch, G)
     t_prefill = flops / (peaks["bf16_tflops_sustained"] * 1e12)
-    t_decode = ((G - 1) * w_bytes + kv_bytes) / (peaks["hbm_gbs"] * 1e9)
+    t_decode = decode_bytes / (peaks["hbm_gbs"] * 1e9)
     roof_ms = (t_prefill + t_decode) * 1000.0
     s = h.zo_stats()
     print(json.dumps({

@@ -79,3 +79,19 @@ def test_fp8_share_is_the_norm_fed_base_products():
         ref = 2.0 * T * sh.n_layers * sh.d_model * (sh.q_dim + 2 * sh.kv_dim + n_in * sh.d_ffn)
         assert abs(f8 - ref) <= 1e-9 * ref
         assert 0.3 < f8 / total < 0.8
+
+
+@pytest.mark.parametrize("name,G", [("tiny", 5), ("qwen3-8b-cobatch", 8)])
+def test_generation_work_counts_weights_and_cache_per_decode_step(name, G):
+    w = wl.WORKLOADS[name]
+    sh = w.shape
+    batch = wl.make_batch(w, batch=3, fg_rows=0, len_hi=20)
+    flops, decode_bytes = bench.generate_work(w, batch, G)
+    assert flops == bench.step_work(w, [batch], 1)[0]          # the prefill is a scoring step
+    es = 2 if sh.dtype == wl.DTYPE_BF16 else 4
+    ref = 0
+    for s in range(1, G):              # token s + 1 of each row: the prefill gave the first
+        ref += (sh.body_params() + sh.vocab * sh.d_model) * es
+        for p in list(batch.prompts) * 2:
+            ref += (len(p) + s) * 2 * sh.kv_dim * sh.n_layers * es    # k and v of every key
+    assert abs(decode_bytes - ref) <= 1e-9 * ref
