@@ -92,3 +92,23 @@ def test_product_path_does_not_import_oracle():
         if f.endswith((".py", ".cu", ".cpp", ".cuh", ".h")):
             txt = open(f).read()
             assert "import oracle" not in txt and "from oracle" not in txt, f
+
+
+def test_decode_linear_argument_checks_without_gpu(built_lib):
+    """zo_op_linear_decode validates sizes, pointers and the workspace on the host, before
+    any CUDA call (placeholder addresses are never dereferenced on these paths)."""
+    from zeroth_order_fine_b200 import zo
+    L = zo.lib()
+    p = ctypes.c_void_p(0x10000)
+    call = lambda x, W, y, M, N, K, act, acc, ws, n: L.zo_op_linear_decode(
+        x, W, None, y, M, N, K, act, acc, ws, n, None)
+    assert call(p, p, p, -1, 256, 64, 0, 0, p, 1 << 20) == zo.ZO_ERR_ARG      # negative M
+    assert call(p, p, p, 4, 0, 64, 0, 0, p, 1 << 20) == zo.ZO_ERR_ARG         # empty N
+    assert call(p, p, p, 4, 256, 64, 2, 0, p, 1 << 20) == zo.ZO_ERR_ARG       # unknown act
+    assert call(p, p, p, 4, 256, 64, 1, 1, p, 1 << 20) == zo.ZO_ERR_ARG       # ReLU + accumulate
+    assert call(None, None, None, 0, 256, 64, 0, 0, None, 0) == zo.ZO_OK       # M = 0: no-op
+    assert call(None, p, p, 4, 256, 64, 0, 0, p, 1 << 20) == zo.ZO_ERR_ARG    # NULL x
+    assert call(p, p, p, 4, 256, 64, 0, 0, None, 1 << 20) == zo.ZO_ERR_ARG    # NULL workspace
+    assert call(p, p, p, 4, 256, 64, 0, 0, p, 4 * 256 - 1) == zo.ZO_ERR_ARG   # < one slice
+    assert call(p, p, p, 4, 256, 60, 0, 0, p, 1 << 20) == zo.ZO_ERR_UNSUPPORTED  # K % 8
+    assert call(p, p, p, 4, 258, 64, 0, 0, p, 1 << 20) == zo.ZO_ERR_UNSUPPORTED  # N % 4
