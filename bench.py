@@ -183,33 +183,29 @@ class ClockSampler:
 # ---- the oracle on the host cores -------------------------------------------------------
 
 _SAMPLE_WEIGHTS = {}
+# Workloads whose whole step (every layer, every prompt) the oracle runs in the CPU baseline;
+# the larger ones are timed on one layer and scaled by the layer count ("extrapolated").
+FULL_ORACLE = ("tiny", "opt-1.3b-b16")
 
 
-def oracle_sample(w: wl.Workload, n_prompts: int = 2, seed: int = 0):
-    """Time the CPU oracle on a bounded sample of the workload.
-
-    The sample is n_prompts prompts of the workload's batch (both candidate
-    rows each) through ONE decoder layer plus the final norm and the lm_head
-    at their scored positions; the per-layer time is scaled by n_layers.  The
-    weights of the sample are drawn with numpy's generator (their values do
-    not change the oracle's work; the oracle's own counter-stream init of a
-    full-width layer would take longer than the scoring itself).
-    """
+def _sample_weights(sh: wl.ModelShape, n_layers: int):
+    """Weights of the oracle's timing sample, drawn with numpy's generator (their values do
+    not change the oracle's work; the oracle's own counter-stream init of full-width layers
+    would take longer than the scoring itself)."""
     import torch
 
     from oracle import model as om
-    from oracle import zo as ozo
-    sh = w.shape
-    one = wl.shrink_shape(sh, n_layers=1)
+    key = (sh.name, n_layers)
+    if key in _SAMPLE_WEIGHTS:
+        return _SAMPLE_WEIGHTS[key]
     rng = np.random.default_rng(0)
 
     def t(*shape, mean=0.0):
         return torch.from_numpy(rng.standard_normal(shape, dtype=np.float32) * 0.02 + mean).double()
 
     d = sh.d_model
-    if sh.name in _SAMPLE_WEIGHTS:
-        weights = _SAMPLE_WEIGHTS[sh.name]
-    else:
+    layers = []
+    for _ in range(n_layers):
         layer = {}
         for m in sh.matrices():
             di, do = sh.matrix_dims(m)
@@ -221,33 +217,67 @@ def oracle_sample(w: wl.Workload, n_prompts: int = 2, seed: int = 0):
             layer["ln1_b"], layer["ln2_b"] = t(d), t(d)
         else:
             layer["q_norm"], layer["k_norm"] = t(sh.head_dim, mean=1.0), t(sh.head_dim, mean=1.0)
-        tok = t(sh.vocab, d)
-        weights = om.Weights(one, tok, t(sh.max_pos, d) if sh.arch == wl.ARCH_OPT else None,
-                             t(d, mean=1.0), t(d) if sh.arch == wl.ARCH_OPT else None,
-                             tok if sh.tie_lm_head else t(sh.vocab, d), [layer])
-        _SAMPLE_WEIGHTS[sh.name] = weights
-    run = ozo.OracleRun(weights, w.run_seed, w.nu, w.rank, [0], w.matrices, w.scale_mode)
-    batch = wl.make_batch(w, batch=n_prompts, fg_rows=min(w.fg_rows, n_prompts),
-                          seed=w.data_seed + 7919 * seed)
-    run.plan(0, w.eps)
+        layers.append(layer)
+    tok = t(sh.vocab, d)
+    one = wl.shrink_shape(sh, n_layers=n_layers)
+    weights = om.Weights(one, tok, t(sh.max_pos, d) if sh.arch == wl.ARCH_OPT else None,
+                         t(d, mean=1.0), t(d) if sh.arch == wl.ARCH_OPT else None,
+                         tok if sh.tie_lm_head else t(sh.vocab, d), layers)
+    _SAMPLE_WEIGHTS[key] = weights
+    return weights
+
+
+def oracle_sample(w: wl.Workload, n_prompts: int = 2, seed: int = 0):
+    """Time the CPU oracle on a bounded sample of the workload.
+
+    For the small workloads (FULL_ORACLE) the sample is the whole step: every prompt of the
+    seeded batch (both candidate rows) through every layer, plan + score + update.  For
+    the others it is n_prompts prompts through ONE decoder layer plus the final norm and
+    the lm_head at their scored positions, and the layer time is scaled by n_layers; the
+    result says so ("extrapolated": true, with the measured seconds and the scale).
+    """
+    import torch
+
+    from oracle import zo as ozo
+    sh = w.shape
+    full = w.name in FULL_ORACLE
+    n_lay = sh.n_layers if full else 1
+    weights = _sample_weights(sh, n_lay)
+    run = ozo.OracleRun(weights, w.run_seed, w.nu, w.rank, range(n_lay), w.matrices, w.scale_mode)
+    if full:
+        batch = wl.make_batch(w, seed=w.data_seed + 7919 * seed)
+    else:
+        batch = wl.make_batch(w, batch=n_prompts, fg_rows=min(w.fg_rows, n_prompts),
+                              seed=w.data_seed + 7919 * seed)
     t0 = time.perf_counter()
+    run.plan(0, w.eps)
     run.score(batch.prompts, batch.target_lens, batch.fg_prompts, batch.fg_target_lens)
     run.step(w.lr)
-    secs_one = time.perf_counter() - t0
-    # the lm_head part is already inside secs_one once; scale only the layer part
-    hs = torch.zeros(int(2 * batch.target_lens.sum() + batch.fg_target_lens.sum()), d,
-                     dtype=torch.float64)
-    t1 = time.perf_counter()
-    logits = hs @ weights.lm_head.T
-    torch.logsumexp(logits, dim=-1)
-    secs_head = time.perf_counter() - t1
-    secs_step = (secs_one - secs_head) * sh.n_layers + secs_head
+    secs_sample = time.perf_counter() - t0
     T = batch.n_tokens_physical
+    P = len(batch.prompts)
+    if full:
+        secs_step = secs_sample
+        sample = (f"the whole step: {P} prompts ({2 * P} candidate rows, {T} tokens) through "
+                  f"all {sh.n_layers} layers + lm_head, plan + score + update; oracle float64 "
+                  f"on the host cores")
+        scale = 1
+    else:
+        # the lm_head part is already inside secs_sample once; scale only the layer part
+        hs = torch.zeros(int(2 * batch.target_lens.sum() + batch.fg_target_lens.sum()),
+                         sh.d_model, dtype=torch.float64)
+        t1 = time.perf_counter()
+        logits = hs @ weights.lm_head.T
+        torch.logsumexp(logits, dim=-1)
+        secs_head = time.perf_counter() - t1
+        secs_step = (secs_sample - secs_head) * sh.n_layers + secs_head
+        scale = sh.n_layers
+        sample = (f"{P} prompts ({2 * P} candidate rows, {T} tokens) through 1 of "
+                  f"{sh.n_layers} layers + lm_head at the scored positions, layer time scaled "
+                  f"x{sh.n_layers} (extrapolated); oracle float64 on the host cores")
     return {"secs_per_sample_step": secs_step, "tokens": T, "tokens_per_s": T / secs_step,
-            "sample": (f"{n_prompts} prompts ({2 * n_prompts} candidate rows, {T} tokens) "
-                       f"through 1 of {sh.n_layers} layers + lm_head at the scored positions, "
-                       f"layer time scaled x{sh.n_layers}; oracle float64 on the host cores"),
-            "cores": torch.get_num_threads()}
+            "sample": sample, "extrapolated": not full, "sample_seconds": secs_sample,
+            "layer_scale": scale, "cores": torch.get_num_threads()}
 
 
 def run_reference(args, w):
@@ -267,9 +297,14 @@ def run_reference(args, w):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * secs / len(per_step), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "extrapolated": per_step[0]["extrapolated"],
             "config": {"workload": w.name, "model": w.shape.name, "global_batch": w.batch},
             "cpu_baseline": {"value": value, "unit": "scored tokens/s", "kind": "oracle",
-                             "cores": per_step[0]["cores"], "sample": per_step[0]["sample"]},
+                             "cores": per_step[0]["cores"], "sample": per_step[0]["sample"],
+                             "extrapolated": per_step[0]["extrapolated"],
+                             "layer_scale": per_step[0]["layer_scale"],
+                             "sample_seconds_per_step": [round(r["sample_seconds"], 3)
+                                                         for r in per_step]},
             "e2e": {"value": value, "unit": "scored tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -397,6 +432,64 @@ def run_generate(args, w: wl.Workload):
     return 0
 
 
+def cobatch_leg(steps: int, warmup: int = 2):
+    """Co-serving analogue on the co-batching workload (Qwen3-8B shape, 16 prompts as 32
+    probe rows plus 32 unperturbed foreground rows, lengths 64..512, MeZO-style r = 64 on all
+    seven matrices): the mixed physical batch against the probe rows alone and the foreground
+    rows alone, timed on one handle with CUDA events on the launching stream."""
+    import torch
+
+    from zeroth_order_fine_b200 import zo
+    w = wl.WORKLOADS["qwen3-8b-cobatch"]
+    sh = w.shape
+    batch = wl.make_batch(w)
+    model = zo.DeviceModel(sh, w.weight_seed)
+    T = batch.n_tokens_physical
+    S = int(2 * batch.target_lens.sum() + batch.fg_target_lens.sum())
+    R = 2 * w.batch + len(batch.fg_prompts)
+    h = zo.Handle(model, w.run_seed, w.nu, w.rank,
+                  zo.make_targets(sh.n_layers, w.matrices, w.scale_mode),
+                  max_tokens=T, max_rows=R, max_scored=S, max_slots=4)
+    stream = torch.cuda.current_stream()
+    toks = torch.from_numpy(batch.packed()).cuda()
+    ftoks = torch.from_numpy(batch.fg_packed()).cuda()
+    args_fg = (ftoks, batch.fg_seq_lens, batch.fg_target_lens)
+    t = 0
+    for _ in range(warmup):
+        h.zo_probe_plan(t, w.eps)
+        h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, *args_fg)
+        h.zo_step(w.lr, want_c=False)
+        t += 1
+    h.zo_probe_plan(t, w.eps)
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    mixed = timed(lambda: h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, *args_fg))
+    probe = timed(lambda: h.zo_score(toks, batch.seq_lens, batch.target_lens))
+    fg = timed(lambda: h.zo_score_foreground(*args_fg))
+    h.zo_step(w.lr, want_c=False)
+    err = h.zo_stats()["last_error_code"]
+    h.close()
+    del model
+    torch.cuda.empty_cache()
+    fg_T = int(batch.fg_seq_lens.sum())
+    return {"workload": w.name, "probe_rows": 2 * w.batch, "foreground_rows": len(batch.fg_prompts),
+            "tokens": T, "foreground_tokens": fg_T, "mixed_batch_ms": mixed,
+            "probe_rows_alone_ms": probe, "foreground_rows_alone_ms": fg,
+            "mixed_vs_separate": mixed / (probe + fg),
+            "mixed_tokens_per_s": T / (mixed / 1000.0),
+            "separate_tokens_per_s": T / ((probe + fg) / 1000.0),
+            "steps": steps, "last_error_code": err}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -408,6 +501,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the whole-step CUDA graph leg")
+    ap.add_argument("--no-cobatch", action="store_true",
+                    help="skip the co-batching leg (Qwen3-8B probe + foreground rows)")
     ap.add_argument("--layers", type=int, default=0,
                     help="with --generate: run only this many decoder layers of the workload's "
                          "shapes (profiler captures; not a bench line)")
@@ -698,10 +793,19 @@ def main():
     st = line["state_transition"]
     st["frac_of_dense"] = st["bytes_per_step"] / st["dense_ref_bytes_per_step"]
     st["frac_of_dense_targets"] = st["bytes_per_step"] / st["dense_ref_targets_per_step"]
+    if cobatch is None and world == 1 and not args.no_cobatch:
+        # the co-serving analogue on the co-batching workload, measured in the same run
+        h.close()
+        del model
+        torch.cuda.empty_cache()
+        line["cobatch"] = cobatch_leg(args.steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample(w, n_prompts=args.ref_prompts)
         line["cpu_baseline"] = {"value": cb["tokens_per_s"], "unit": "scored tokens/s",
-                                "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
+                                "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"],
+                                "extrapolated": cb["extrapolated"],
+                                "sample_seconds": cb["sample_seconds"],
+                                "layer_scale": cb["layer_scale"]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     h.close()

@@ -175,7 +175,12 @@ typedef struct zo_stats_t {
 /* Validate desc, borrow the weights, allocate the bank, activations and
  * scratch for the given maxima (all device memory the library uses is
  * allocated here), and repack the attention projections into one fused
- * [q|k|v] matrix (a copy; the caller's tensors stay untouched). */
+ * [q|k|v] matrix (a copy; the caller's tensors stay untouched).
+ * On any failure everything allocated so far is freed, *out stays NULL and
+ * zo_last_error(NULL) says why; an allocation that fails gives ZO_ERR_OOM.
+ * Failure injection for tests: with the environment variable
+ * ZO_FAIL_ALLOC_AT=n set when zo_create is called, the handle's n-th device
+ * allocation (counted from 1) fails as if the device were out of memory. */
 int zo_create(const zo_model_desc* desc, const zo_weights* weights,
               const zo_options* options, zo_handle** out);
 void zo_destroy(zo_handle* h);

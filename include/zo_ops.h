@@ -76,6 +76,70 @@ int zo_op_linear_decode(const void* x, const void* W, const float* bias, void* y
                         int32_t N, int32_t K, int32_t act, int32_t accumulate, float* ws,
                         size_t ws_floats, void* stream);
 
+/* Epilogues of zo_op_linear_ext. */
+enum { ZO_EPI_STORE = 0, ZO_EPI_RELU = 1, ZO_EPI_RESID = 2, ZO_EPI_SWIGLU = 5,
+       ZO_EPI_QK_NORM_ROPE = 6 };
+
+/* Qwen3's per-head q/k RMSNorm and rotary positions, applied by the q|k|v GEMM's
+ * epilogue (ZO_EPI_QK_NORM_ROPE). */
+typedef struct zo_qk_norm_rope_args {
+    const int32_t* tok_pos;   /* dev int32 [M]: each row's position within its sequence      */
+    const float* q_norm;      /* dev float [128]: RMSNorm scales of the query heads, 16-B aligned */
+    const float* k_norm;      /* dev float [128]: the key heads'                              */
+    const float* rope_cos;    /* dev float [max_pos x 64]: cos(pos * theta^(-2i/128)), i < 64  */
+    const float* rope_sin;    /* dev float [max_pos x 64]: the matching sines                 */
+    float eps;                /* RMSNorm epsilon                                               */
+    int32_t n_q_heads;        /* query heads (columns [0, 128 n_q_heads) of y)                */
+    int32_t n_kv_heads;       /* key heads follow, then as many value heads (passed through)  */
+} zo_qk_norm_rope_args;
+
+/* The perturbed linear layer as the probe step runs it, on the tensor cores (bf16 only):
+ *   acc = x W^T + x2 W2^T + b
+ * where x2 W2^T is the extension that carries the candidate perturbation and the banked
+ * slots (x2 = the shrink output s eps (x U) | x A_j, W2 = the expand factors V | V_j), run
+ * as extra K blocks of the same tcgen05 GEMM so that no dense W + eps U V^T is formed
+ * ("Zeroth-Order Fine-Tuning Was an Inference Workload All Along", section "The System
+ * Reorganization"; "Inference-Native Zeroth-Order Optimization", abstract: factorised side
+ * states over frozen base weights).  Then the epilogue:
+ *   ZO_EPI_STORE  y = bf16(acc)                 ZO_EPI_RELU  y = bf16(max(acc, 0))
+ *   ZO_EPI_RESID  y (fp32) += acc               (the residual stream)
+ *   ZO_EPI_SWIGLU the rows of W (and W2, bias) hold gate and up features interleaved in
+ *                 blocks of 128: rows 256 b .. 256 b + 127 are gate features 128 b .., the
+ *                 next 128 rows the up features of the same indices; y [M x N/2] bf16 =
+ *                 silu(gate) * up.  N % 256 == 0.
+ *   ZO_EPI_QK_NORM_ROPE  acc rounded to bf16; each 128-column query and key head then gets
+ *                 RMSNorm over the head (scale q_norm / k_norm) and the rotate-half rotary
+ *                 rotation of the pairs (i, i + 64) at tok_pos[m]; value heads are stored as
+ *                 they are.  N == 128 (n_q_heads + 2 n_kv_heads); no bias.
+ *   x  dev bf16 [M x K], W dev bf16 [N x K]; x2 dev bf16 [M x K2], W2 dev bf16 [N x K2] (or
+ *   K2 = 0 and both NULL); bias dev float [N] or NULL; y dev, row stride ldy elements.
+ * Rows never interact: the result of a row does not depend on M or on the other rows.
+ * ZO_ERR_ARG on NULL pointers, negative sizes, ldy too small or an unknown epilogue;
+ * ZO_ERR_UNSUPPORTED when K, K2 or ldy is not a multiple of 8 (ldy: 4 for ZO_EPI_RESID),
+ * a pointer is not 16-byte aligned, or the epilogue needs N > 128 (SwiGLU, q/k norm) and
+ * does not get it.
+ * Asynchronous on stream. */
+int zo_op_linear_ext(const void* x, const void* W, const float* bias, const void* x2,
+                     const void* W2, int32_t K2, void* y, int32_t ldy, int32_t M, int32_t N,
+                     int32_t K, int32_t epi, const zo_qk_norm_rope_args* qk, void* stream);
+
+/* The rotary tables zo_create builds for Qwen3 models: cos_t[pos * hd/2 + i] =
+ * cos(pos * theta^(-2 i / head_dim)) and sin_t likewise, evaluated in double and rounded
+ * to float.  cos_t, sin_t dev float [max_pos x head_dim / 2].  Asynchronous on stream. */
+int zo_op_rope_table(float* cos_t, float* sin_t, int32_t max_pos, int32_t head_dim,
+                     double theta, void* stream);
+
+/* Test hook for the failure path of the tensor-core GEMM kernels.  Every mbarrier wait in
+ * them gives up after `cycles` SM clock cycles: the kernel then sets bit 0 of the error
+ * word (zo_op_error_word), stops issuing work, waits (again with a bound) for the copies
+ * and MMAs it has already issued, frees its tensor memory and returns; its output is
+ * invalid.  The default bound, about 2 s, is far beyond any wait of a healthy launch; a
+ * bound of a few hundred cycles makes an ordinary launch give up at its first wait for
+ * data, without any barrier being broken.  cycles <= 0 restores the default.  Applies to
+ * launches queued after the call, process-wide (not synchronised with other threads).
+ * Returns the previous bound. */
+int64_t zo_op_set_wait_limit(int64_t cycles);
+
 /* Bytes of workspace zo_op_lm_head_logprob needs for n_rows rows and vocab. */
 size_t zo_op_lm_head_workspace(int32_t n_rows, int32_t vocab, int32_t impl);
 

@@ -1,0 +1,107 @@
+"""Failure paths on the GPU, made without faulting or hanging it.
+
+* A bounded wait that runs out: every mbarrier wait of the tensor-core GEMM gives up after a
+  bound (about 2 s by default), records bit 0 of the error word, drains what it issued,
+  frees its tensor memory and returns.  Setting the bound to a few hundred cycles makes an
+  ordinary, healthy launch give up at its first wait for data -- no barrier is broken,
+  nothing traps -- and the next launch with the default bound must be clean and correct.
+  Only the single-SM kernel is used here (N = 128).
+* An allocation that fails: ZO_FAIL_ALLOC_AT=n makes the n-th device allocation of
+  zo_create fail; the call returns ZO_ERR_OOM, says why, and frees everything it had taken.
+"""
+import os
+
+import pytest
+import torch
+
+from zeroth_order_fine_b200 import workload as wl
+from gpu_util import needs_gpu
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+def _bf16_ulp(x):
+    return torch.clamp(torch.abs(x), min=1e-30) * 2.0 ** -7
+
+
+def test_expired_wait_reports_timeout_then_the_next_launch_is_clean():
+    from zeroth_order_fine_b200 import zo
+    g = torch.Generator().manual_seed(21)
+    M, N, K = 256, 128, 4096                      # single-SM kernel, 64 K blocks per tile
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    ref = x.double() @ W.double().T
+    xd, Wd = x.cuda(), W.cuda()
+    y = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    zo.zo_op_linear(xd, Wd, out=y, impl=zo.IMPL_TENSOR_CORES)
+    assert zo.zo_op_error_word() == 0
+    model = zo.DeviceModel(wl.WORKLOADS["tiny"].shape)
+    w = wl.WORKLOADS["tiny"]
+    h = zo.Handle(model, w.run_seed, w.nu, w.rank, zo.make_targets(2, w.matrices, w.scale_mode),
+                  max_tokens=64, max_rows=2, max_scored=2)
+    old = zo.zo_op_set_wait_limit(300)
+    try:
+        zo.zo_op_linear(xd, Wd, out=y, impl=zo.IMPL_TENSOR_CORES)     # queued: returns ZO_OK
+        torch.cuda.synchronize()
+        # the handle reports the expired wait as ZO_ERR_TIMEOUT (and clears the word)
+        assert h.zo_stats()["last_error_code"] == zo.ZO_ERR_TIMEOUT
+        zo.zo_op_linear(xd, Wd, out=y, impl=zo.IMPL_TENSOR_CORES)
+        assert zo.zo_op_error_word() & 1
+    finally:
+        restored = zo.zo_op_set_wait_limit(0)
+    assert restored == 300 and old > 10 ** 9
+    assert zo.zo_op_error_word() == 0
+    # the same launch with the default bound: clean, correct, and the context still usable
+    for _ in range(2):
+        y2 = zo.zo_op_linear(xd, Wd, impl=zo.IMPL_TENSOR_CORES)
+        assert zo.zo_op_error_word() == 0
+        err = (y2.double().cpu() - ref).abs()
+        assert torch.all(err <= _bf16_ulp(ref) + 1e-4 * (K ** 0.5) * 0.05), err.max()
+    assert h.zo_stats()["last_error_code"] == 0
+    h.close()
+
+
+def _create(w, shape):
+    from zeroth_order_fine_b200 import zo
+    model = zo.DeviceModel(shape, w.weight_seed)
+    h = zo.Handle(model, w.run_seed, w.nu, w.rank,
+                  zo.make_targets(shape.n_layers, w.matrices, w.scale_mode),
+                  max_tokens=512, max_rows=16, max_scored=16)
+    return model, h
+
+
+@pytest.mark.parametrize("wk", ["tiny", "tiny-bf16"])
+def test_injected_allocation_failure_returns_oom_and_leaks_nothing(wk):
+    """Every device allocation of zo_create in turn is made to fail (n = 1, 2, ... until a
+    create goes through): each time the call returns ZO_ERR_OOM naming the allocation, and
+    the device's free memory is back where it was."""
+    from zeroth_order_fine_b200 import zo
+    w = wl.WORKLOADS["tiny"]
+    shape = w.shape if wk == "tiny" else wl.shrink_shape(w.shape, dtype=wl.DTYPE_BF16)
+    model, h = _create(w, shape)                    # warm-up: modules loaded, then freed
+    h.close()
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    tg = zo.make_targets(shape.n_layers, w.matrices, w.scale_mode)
+    n = 0
+    try:
+        while True:
+            n += 1
+            assert n < 1000
+            os.environ["ZO_FAIL_ALLOC_AT"] = str(n)
+            try:
+                h2 = zo.Handle(model, w.run_seed, w.nu, w.rank, tg, max_tokens=512,
+                               max_rows=16, max_scored=16)
+            except zo.ZoError as e:
+                assert e.code == zo.ZO_ERR_OOM, (n, str(e))
+                assert f"allocation {n} refused" in str(e), str(e)
+                torch.cuda.synchronize()
+                assert torch.cuda.mem_get_info()[0] == free0, n
+                continue
+            h2.close()                               # n is past the last allocation
+            break
+    finally:
+        os.environ.pop("ZO_FAIL_ALLOC_AT", None)
+    assert n > 20, n                                # every allocation point was visited
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0

@@ -120,21 +120,40 @@ def test_opt_1_3b_width_slice_bf16_same_state_parity():
     _bf16_same_state_parity(w, shape, wl.make_batch(w, batch=4, len_hi=64), pre_steps=2)
 
 
+def test_opt_13b_width_layer_full_batch_64_bf16_same_state_parity():
+    """One full-width OPT-13B layer (d = 5120, vocab 50272) over the whole seeded batch-64
+    step: 128 physical rows, 9196 packed tokens, so every GEMM runs the SM-pair schedule of
+    the headline step (36 row blocks in raster groups of 12, many tiles per pair) and the
+    attention kernel its full tile list; L+- against the oracle at step 0 and after the
+    oracle's first update (its bank loaded)."""
+    w = wl.WORKLOADS["opt-13b-b64"]
+    shape = wl.shrink_shape(w.shape, n_layers=1)
+    batch = wl.make_batch(w)
+    assert batch.n_tokens_physical > 12 * 256
+    _bf16_same_state_parity(w, shape, batch, pre_steps=1)
+
+
 def test_qwen3_bf16_same_state_parity():
     shape = dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16)
     w = dataclasses.replace(QWEN_SMALL, shape=shape, fg_rows=0)
     _bf16_same_state_parity(w, shape, wl.make_batch(w, fg_rows=0), pre_steps=4)
 
 
-def test_tiny_bf16_loss_trajectory_100_steps():
-    """bf16 mode: the 100-step loss trajectory (each side on its own c) within 2 %."""
-    w = TINY_BF16
-    batch = wl.make_batch(w)
-    model, h = gpu_handle(w)
-    orc = oracle_run(w)
+# The bf16 trajectory workloads: each side follows its own c for 100 steps, so the check
+# is only meaningful when 100 steps move the loss far beyond the 2 % band.  The tiny model
+# with the direction on q and v alone hardly moves (3.5 % at eta = 1e-4); with the direction
+# on all six OPT matrices and eta = 1e-3 the oracle's loss falls by ~13 %.
+ALL6_OPT = (wl.MAT_Q, wl.MAT_K, wl.MAT_V, wl.MAT_O, wl.MAT_UP, wl.MAT_DOWN)
+TRAJ_TINY = dataclasses.replace(TINY_BF16, matrices=ALL6_OPT, lr=1e-3)
+
+
+def _trajectory_vs_oracle(w, shape, batch, steps=100):
+    """Mean objective (L+ + L-)/2 of every step, GPU and oracle each on its own c."""
+    model, h = gpu_handle(w, shape=shape, batch=len(batch.prompts))
+    orc = oracle_run(w, shape=shape)
     toks = dev_tokens(batch)
     traj, traj_ref = [], []
-    for t in range(100):
+    for t in range(steps):
         h.zo_probe_plan(t, w.eps)
         orc.plan(t, w.eps)
         Lp, Lm, _ = h.zo_score(toks, batch.seq_lens, batch.target_lens)
@@ -143,10 +162,31 @@ def test_tiny_bf16_loss_trajectory_100_steps():
         traj_ref.append(float(ref.L_plus.mean() + ref.L_minus.mean()) / 2)
         h.zo_step(w.lr, want_c=False)
         orc.step(w.lr)
-    traj, traj_ref = np.array(traj), np.array(traj_ref)
+    h.close()
+    return np.array(traj), np.array(traj_ref)
+
+
+def _check_trajectory(traj, traj_ref):
+    # the oracle's own movement is at least 5x the band, so an update of half (or twice)
+    # the right strength cannot stay inside it
+    move = abs(traj_ref[-1] - traj_ref[0]) / abs(traj_ref[0])
+    assert move >= 0.10, move
     rel = np.abs(traj - traj_ref) / np.abs(traj_ref)
-    assert np.max(rel) <= 0.02, (np.max(rel), traj[-1], traj_ref[-1])
-    assert abs(traj[-1] - traj[0]) > 0 and abs(traj_ref[-1] - traj_ref[0]) > 0
+    assert np.max(rel) <= 0.02, (np.max(rel), int(np.argmax(rel)), traj[-1], traj_ref[-1])
+
+
+def test_tiny_bf16_loss_trajectory_100_steps():
+    """bf16 mode: the 100-step loss trajectory of the tiny model within 2 % of the oracle's."""
+    w = TRAJ_TINY
+    _check_trajectory(*_trajectory_vs_oracle(w, w.shape, wl.make_batch(w)))
+
+
+def test_opt_1_3b_width_slice_bf16_loss_trajectory_100_steps():
+    """bf16 mode: 100 steps of two full-width OPT-1.3B layers (d = 2048, vocab 50272,
+    q and v targets, eta = 1e-4 as configured), trajectory within 2 % of the oracle's."""
+    w = wl.WORKLOADS["opt-1.3b-b16"]
+    shape = wl.shrink_shape(w.shape, n_layers=2)
+    _check_trajectory(*_trajectory_vs_oracle(w, shape, wl.make_batch(w, batch=4, len_hi=64)))
 
 
 @pytest.mark.parametrize("wk", ["tiny", "tiny-bf16"])

@@ -26,6 +26,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <functional>
 #include <string>
@@ -186,6 +187,9 @@ struct zo_handle {
     uint64_t dense_bytes = 0, dense_bytes_targets = 0;
     std::string err;
     int err_code = 0;
+    // allocation failure injection (ZO_FAIL_ALLOC_AT): device allocations made so far and
+    // the 1-based index of the one to fail (0: none)
+    long long n_allocs = 0, fail_alloc_at = 0;
 };
 
 static std::string g_create_err = kNoErr;
@@ -218,6 +222,13 @@ bool layer_targeted(const zo_targets& t, int l) {
 
 int dev_alloc(zo_handle* h, void** p, size_t bytes) {
     if (bytes == 0) bytes = 16;
+    if (++h->n_allocs == h->fail_alloc_at) {
+        *p = nullptr;
+        h->err = "device allocation " + std::to_string(h->n_allocs) +
+                 " refused by ZO_FAIL_ALLOC_AT (injected out-of-memory)";
+        h->err_code = ZO_ERR_OOM;
+        return ZO_ERR_OOM;
+    }
     cudaError_t e = cudaMalloc(p, bytes);
     if (e != cudaSuccess) {
         h->err = std::string("cudaMalloc: ") + cudaGetErrorString(e);
@@ -487,6 +498,7 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
         return chk == 2 ? ZO_ERR_UNSUPPORTED : ZO_ERR_ARG;
     }
     zo_handle* h = new zo_handle();
+    if (const char* fa = std::getenv("ZO_FAIL_ALLOC_AT")) h->fail_alloc_at = std::atoll(fa);
     h->desc = *desc;
     h->opt = *options;
     h->wts = *weights;

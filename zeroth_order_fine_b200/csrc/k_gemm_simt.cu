@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
                     if (g.part_arg) g.part_arg[(size_t)m * g.n_col_tiles + blockIdx.x] = arg;
                 }
                 const int tgt = g.targets[m] - (n0 + tx * 4);
-                if (tgt >= 0 && tgt < 4) g.tgt_logit[m] = v[tgt];
+                if (tgt >= 0 && tgt < 4 && g.targets[m] < g.N) g.tgt_logit[m] = v[tgt];
             }
         }
         return;

@@ -43,6 +43,7 @@ constexpr int GROUP_M = 8;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t WAIT_LIMIT = 1u << 24;   // drain polls (with back-off) after an abort
 constexpr long long WAIT_CYCLES = 4000000000ll;   // ~2 s at 2 GHz: a stage that never arrives
+long long g_wait_cycles = WAIT_CYCLES;             // host copy handed to every launch
 
 // Single-SM kernel geometry for an N tile of BNT columns (64, 128 or 256): the
 // ring holds 192 KB whatever the width, so narrow GEMMs (the bank shrink, whose
@@ -93,6 +94,7 @@ struct TcParams {
     const float* a_scale; const float* b_scale;   // E4M3 dequantisation (F8 kernels)
     int ksplit, kbs;                        // split-K (SPLIT kernels): splits, main blocks each
     int* err;
+    long long wait_cycles;                  // bound of every mbarrier wait (clock64 cycles)
 };
 
 // ---- PTX wrappers ------------------------------------------------------------------
@@ -120,22 +122,34 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait that suspends the thread for at most ~1 us (suspendTimeHint, in ns) when the
+// phase is not complete, so a waiting thread looks at its clock regularly.
+__device__ __forceinline__ bool mbar_try_bounded(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000u)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait; false when the limit expired or another role aborted.  No
-// sleep between polls: try_wait already suspends the thread in hardware for a
-// short while, and a software back-off would delay the hand-off of every stage.
+// sleep between polls: try_wait already suspends the thread in hardware (until
+// the phase completes, or ~1 us at most), and a software back-off would delay
+// the hand-off of every stage.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_f,
-                                          int* err) {
+                                          int* err, long long limit) {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*abort_f) return false;
-            if (clock64() - t0 > WAIT_CYCLES) {
-                *abort_f = 1;
-                atomicOr(err, 1);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_bounded(bar, parity)) return true;
+        if (*abort_f) return false;
+        if (clock64() - t0 > limit) {
+            *abort_f = 1;
+            atomicOr(err, 1);
+            return false;
         }
     }
 }
@@ -243,7 +257,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int m, int n, 
         *run_max = nm;
         if (row_ok) {
             const int tg = p.targets[m] - n;
-            if (tg >= 0 && tg < 32) {
+            if (tg >= 0 && tg < 32 && n + tg < p.N) {     // padding columns are no target
                 float tv = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
@@ -466,7 +480,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 item_blocks(t % ks, &kb0, &n_main, &n_kb);
                 for (int i = 0; i < n_kb; ++i) {
                     const int kb = i < n_main ? kb0 + i : p.kb_main + (i - n_main);
-                    if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                    if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                     const uint32_t sa = base + s * STAGE_BYTES;
                     const uint32_t sb = sa + A_BYTES;
                     mbar_expect_tx(full(s), STAGE_BYTES);
@@ -502,13 +516,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t aph = 0;
             bool ok = true, issued = false;
             for (int t = blockIdx.x; t < n_items && ok; t += gridDim.x) {
-                if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * BNT);
                 int kb0, n_main, n_kb;
                 item_blocks(t % ks, &kb0, &n_main, &n_kb);
                 for (int i = 0; i < n_kb; ++i) {
-                    if (!mbar_wait(full(s), ph, abort_f, p.err)) { ok = false; break; }
+                    if (!mbar_wait(full(s), ph, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = base + s * STAGE_BYTES;
                     const uint32_t sb = sa + A_BYTES;
@@ -545,7 +559,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = blockIdx.x; t < n_items; t += gridDim.x) {
             int mb, nb;
             tile_coords(t / ks, p, &mb, &nb);
-            if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
+            if (!mbar_wait(tfull(acc), aph, abort_f, p.err, p.wait_cycles)) break;
             tc_fence_after();
             const int m = mb * BM + lane_base + lane;
             float run_max = -FLT_MAX, run_sum = 0.f;
@@ -1047,7 +1061,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 item_blocks(SPLIT ? t % p.ksplit : 0, &kb0, &n_main, &n_kb);
                 for (int i = 0; i < n_kb; ++i) {
                     const int kb = i < n_main ? kb0 + i : p.kb_main + (i - n_main);
-                    if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                    if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                     const uint32_t sa = base + s * STAGE2_BYTES;
                     const uint32_t sb = sa + A2B;
                     // the even CTA expects both CTAs' bytes on its barrier
@@ -1084,14 +1098,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             uint32_t aph = 0;
             bool ok = true, issued = false;
             for (int t = pair; t < n_items && ok; t += n_pairs) {
-                if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err)) { ok = false; break; }
+                if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * BN);
                 int kb0, n_main, n_kb;
                 item_blocks(SPLIT ? t % p.ksplit : 0, &kb0, &n_main, &n_kb);
                 for (int i = 0; i < n_kb; ++i) {
                     const int kb = i < n_main ? kb0 + i : p.kb_main + (i - n_main);
-                    if (!mbar_wait(full(s), ph, abort_f, p.err)) { ok = false; break; }
+                    if (!mbar_wait(full(s), ph, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = base + s * STAGE2_BYTES;
                     const uint32_t sb = sa + A2B;
@@ -1135,7 +1149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         for (int t = pair; t < n_items; t += n_pairs) {
             int mb, nb;
             tile_coords2(SPLIT ? t / p.ksplit : t, p, &mb, &nb);
-            if (!mbar_wait(tfull(acc), aph, abort_f, p.err)) break;
+            if (!mbar_wait(tfull(acc), aph, abort_f, p.err, p.wait_cycles)) break;
             tc_fence_after();
             const int m_base = mb * BM2 + (int)rank * 128 + lane_base;
             epilogue_tma<EPI, F8, SPLIT>(p, &tmC, stg, stg_ptr, buf, m_base, nb,
@@ -1485,6 +1499,7 @@ int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
     int* err = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
+    p.wait_cycles = g_wait_cycles;
     // K splits: the weight stream is the cost.  In units of one 128 x 64 weight block, the
     // busiest SM streams rounds x (kbs + slice) blocks at up to SM_BW_REL times its fair share
     // of HBM, and all SMs together stream the weights plus the slices written and read back;
@@ -1634,6 +1649,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     int* err = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
+    p.wait_cycles = g_wait_cycles;
     if (pair && g.ws && !f8 && g.N % 4 == 0 &&
         (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
          g.epi == EPI_SWIGLU || g.epi == EPI_QKNR)) {
@@ -1688,6 +1704,12 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     }
 }
 
+
+long long gemm_tc_set_wait_cycles(long long cycles) {
+    const long long old = g_wait_cycles;
+    g_wait_cycles = cycles > 0 ? cycles : WAIT_CYCLES;
+    return old;
+}
 
 int gemm_tc_error_word() {
     int v = 0;

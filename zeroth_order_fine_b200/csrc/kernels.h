@@ -124,6 +124,9 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st);   // 0 ok, else 1
 int gemm_lse_col_tiles(int N);                      // LSE column tiles, CUDA-core path (the most)
 int gemm_tc_col_tiles(int N);                       // LSE column tiles, tensor-core path
 int gemm_tc_error_word();                           // bit 0: a bounded wait expired
+// Bound of every mbarrier wait in the tensor-core GEMM kernels launched from now on, in
+// clock64 cycles (<= 0: the default, about 2 s); returns the previous bound.
+long long gemm_tc_set_wait_cycles(long long cycles);
 
 // ---- attention -----------------------------------------------------------------------
 struct AttnArgs {

@@ -203,6 +203,64 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
 }
 
+int zo_op_linear_ext(const void* x, const void* W, const float* bias, const void* x2,
+                     const void* W2, int32_t K2, void* y, int32_t ldy, int32_t M, int32_t N,
+                     int32_t K, int32_t epi, const zo_qk_norm_rope_args* qk, void* stream) {
+    if (!x || !W || !y || M < 0 || N <= 0 || K <= 0 || K2 < 0 || ldy <= 0) return ZO_ERR_ARG;
+    if (K2 > 0 && (!x2 || !W2)) return ZO_ERR_ARG;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    switch (epi) {
+        case ZO_EPI_STORE: g.epi = EPI_STORE; g.c_type = E_BF16; break;
+        case ZO_EPI_RELU: g.epi = EPI_STORE_RELU; g.c_type = E_BF16; break;
+        case ZO_EPI_RESID: g.epi = EPI_RESID; g.c_type = E_F32; break;
+        case ZO_EPI_SWIGLU:
+            if (N % 256) return ZO_ERR_UNSUPPORTED;
+            g.epi = EPI_SWIGLU; g.c_type = E_BF16;
+            if (ldy < N / 2) return ZO_ERR_ARG;
+            break;
+        case ZO_EPI_QK_NORM_ROPE:
+            if (!qk || !qk->tok_pos || !qk->q_norm || !qk->k_norm || !qk->rope_cos ||
+                !qk->rope_sin || qk->n_q_heads <= 0 || qk->n_kv_heads <= 0)
+                return ZO_ERR_ARG;
+            if (bias) return ZO_ERR_UNSUPPORTED;
+            g.epi = EPI_QKNR; g.c_type = E_BF16;
+            g.tok_pos = qk->tok_pos; g.qn = qk->q_norm; g.kn = qk->k_norm;
+            g.rope_cos = qk->rope_cos; g.rope_sin = qk->rope_sin; g.norm_eps = qk->eps;
+            g.n_q_heads = qk->n_q_heads; g.n_qk_heads = qk->n_q_heads + qk->n_kv_heads;
+            if ((int64_t)(g.n_qk_heads + qk->n_kv_heads) * 128 != N) return ZO_ERR_ARG;
+            break;
+        default: return ZO_ERR_ARG;
+    }
+    if (epi != ZO_EPI_SWIGLU && ldy < N) return ZO_ERR_ARG;
+    g.A = x; g.lda = K; g.a_type = E_BF16;
+    g.B = W; g.ldb = K; g.b_type = E_BF16;
+    if (K2 > 0) {
+        g.A2 = x2; g.lda2 = K2; g.a2_type = E_BF16;
+        g.B2 = W2; g.ldb2 = K2; g.b2_type = E_BF16;
+        g.K2 = K2;
+    }
+    g.M = M; g.N = N; g.K = K;
+    g.bias = bias;
+    g.C = y; g.ldc = ldy;
+    if (M == 0) return ZO_OK;
+    if (!gemm_tc_supported(g)) return ZO_ERR_UNSUPPORTED;
+    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return ZO_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
+int zo_op_rope_table(float* cos_t, float* sin_t, int32_t max_pos, int32_t head_dim, double theta,
+                     void* stream) {
+    if (!cos_t || !sin_t || max_pos <= 0 || head_dim <= 0 || head_dim % 2 || !(theta > 0.0))
+        return ZO_ERR_ARG;
+    launch_rope_table(cos_t, sin_t, max_pos, head_dim, theta, static_cast<cudaStream_t>(stream));
+    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+}
+
+int64_t zo_op_set_wait_limit(int64_t cycles) {
+    return (int64_t)gemm_tc_set_wait_cycles((long long)cycles);
+}
+
 /* Error word of the tensor-core kernels (bit 0: a bounded wait expired);
  * synchronises the device and clears the word. */
 int zo_op_error_word(void) {

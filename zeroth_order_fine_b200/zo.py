@@ -84,6 +84,12 @@ class zo_stats_t(ctypes.Structure):
                 ("graph_replays", c_uint64)]
 
 
+class zo_qk_norm_rope_args(ctypes.Structure):
+    _fields_ = [("tok_pos", c_void_p), ("q_norm", c_void_p), ("k_norm", c_void_p),
+                ("rope_cos", c_void_p), ("rope_sin", c_void_p), ("eps", ctypes.c_float),
+                ("n_q_heads", c_int32), ("n_kv_heads", c_int32)]
+
+
 _I32P = ctypes.POINTER(c_int32)
 _F32P = ctypes.POINTER(ctypes.c_float)
 _F64P = ctypes.POINTER(ctypes.c_double)
@@ -121,6 +127,12 @@ _SIGS = {
     "zo_op_linear_decode": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
                                       c_int32, c_int32, c_int32, c_void_p, ctypes.c_size_t,
                                       c_void_p]),
+    "zo_op_linear_ext": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32,
+                                   c_void_p, c_int32, c_int32, c_int32, c_int32, c_int32,
+                                   ctypes.POINTER(zo_qk_norm_rope_args), c_void_p]),
+    "zo_op_rope_table": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, ctypes.c_double,
+                                   c_void_p]),
+    "zo_op_set_wait_limit": (ctypes.c_int64, [ctypes.c_int64]),
     "zo_op_quantize_rows_e4m3": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p,
                                            c_void_p, c_void_p]),
     "zo_op_linear_fp8": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -462,6 +474,49 @@ def zo_op_linear_decode(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.T
     return out
 
 
+EPI_STORE, EPI_RELU, EPI_RESID, EPI_SWIGLU, EPI_QK_NORM_ROPE = 0, 1, 2, 5, 6
+
+
+def zo_op_linear_ext(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                     x2: Optional[torch.Tensor] = None, W2: Optional[torch.Tensor] = None,
+                     epi: int = EPI_STORE, out: Optional[torch.Tensor] = None,
+                     qk: Optional[dict] = None) -> torch.Tensor:
+    """The perturbed linear of one fused group on the tensor cores (bf16): x W^T + x2 W2^T
+    + b with the group's epilogue (store, ReLU, residual add, SwiGLU, q/k norm + RoPE).
+    ``qk`` holds the ZO_EPI_QK_NORM_ROPE arguments: tok_pos, q_norm, k_norm, rope_cos,
+    rope_sin (device tensors), eps, n_q_heads, n_kv_heads."""
+    M, K = x.shape
+    N = W.shape[0]
+    K2 = 0 if x2 is None else x2.shape[1]
+    if out is None:
+        cols = N // 2 if epi == EPI_SWIGLU else N
+        out = torch.empty(M, cols, dtype=torch.float32 if epi == EPI_RESID else torch.bfloat16,
+                          device=x.device)
+    args = None
+    if qk is not None:
+        args = zo_qk_norm_rope_args(_ptr(qk["tok_pos"]), _ptr(qk["q_norm"]), _ptr(qk["k_norm"]),
+                                    _ptr(qk["rope_cos"]), _ptr(qk["rope_sin"]), qk["eps"],
+                                    qk["n_q_heads"], qk["n_kv_heads"])
+    _check(lib().zo_op_linear_ext(_ptr(x), _ptr(W), _ptr(bias), _ptr(x2), _ptr(W2), K2, _ptr(out),
+                                  out.stride(0), M, N, K, epi,
+                                  ctypes.byref(args) if args is not None else None, _stream()))
+    return out
+
+
+def zo_op_rope_table(max_pos: int, head_dim: int, theta: float, device="cuda"):
+    """(cos, sin) rotary tables [max_pos x head_dim/2] as zo_create builds them."""
+    c = torch.empty(max_pos, head_dim // 2, dtype=torch.float32, device=device)
+    s = torch.empty(max_pos, head_dim // 2, dtype=torch.float32, device=device)
+    _check(lib().zo_op_rope_table(_ptr(c), _ptr(s), max_pos, head_dim, theta, _stream()))
+    return c, s
+
+
+def zo_op_set_wait_limit(cycles: int) -> int:
+    """Bound of every mbarrier wait in the tensor-core GEMMs (<= 0: the default); returns
+    the previous bound."""
+    return int(lib().zo_op_set_wait_limit(cycles))
+
+
 def zo_op_quantize_rows_e4m3(x: torch.Tensor):
     """(codes uint8 [rows, cols], scale float [rows]) of the E4M3 row quantiser."""
     rows, cols = x.shape
@@ -513,6 +568,17 @@ def zo_op_lm_head_logprob_noalloc(h: torch.Tensor, E: torch.Tensor, targets: tor
     """The lm_head log-probabilities with the library's own fixed scratch (no
     workspace, no allocation inside the call); ``out`` is the caller's buffer."""
     S, d = h.shape
+    for name, t in (("h", h), ("E", E), ("targets", targets), ("out", out)):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if t.device != h.device:
+            raise ValueError(f"{name} is on {t.device}, h on {h.device}")
+    if E.dtype != h.dtype or E.dim() != 2 or E.shape[1] != d:
+        raise ValueError("E must be [vocab x d] in h's dtype")
+    if targets.dtype != torch.int32 or targets.numel() != S:
+        raise ValueError("targets must be int32 with one entry per row of h")
+    if out.dtype != torch.float32 or out.numel() < S:
+        raise ValueError("out must be float32 with room for one value per row of h")
     dtype = wl.DTYPE_BF16 if h.dtype == torch.bfloat16 else wl.DTYPE_FP32
     _check(lib().zo_op_lm_head_logprob_noalloc(_ptr(h), _ptr(E), _ptr(targets), S, E.shape[0], d,
                                                dtype, _ptr(out), impl, _stream()))
