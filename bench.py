@@ -504,8 +504,8 @@ def main():
     ap.add_argument("--no-cobatch", action="store_true",
                     help="skip the co-batching leg (Qwen3-8B probe + foreground rows)")
     ap.add_argument("--layers", type=int, default=0,
-                    help="with --generate: run only this many decoder layers of the workload's "
-                         "shapes (profiler captures; not a bench line)")
+                    help="run only this many decoder layers of the workload's shapes (small "
+                         "device footprint for profiler captures; not a bench line)")
     ap.add_argument("--generate", type=int, default=0,
                     help="generation-query steps: greedy tokens per candidate row (zo_generate)")
     ap.add_argument("--fp8", action="store_true",
@@ -546,6 +546,10 @@ def main():
                                 device_id=torch.device("cuda", local))
     stream = torch.cuda.current_stream()
 
+    if args.layers:
+        # fewer decoder layers of the same shapes (per-launch GEMM shapes unchanged): for
+        # profiler captures only, and the line says so
+        w = dataclasses.replace(w, shape=dataclasses.replace(w.shape, n_layers=args.layers))
     sh = w.shape
     batch = wl.make_batch(w, seed=w.data_seed + 1000 * rank)
     model = zo.DeviceModel(sh, w.weight_seed)
@@ -756,7 +760,9 @@ def main():
                    "l2": "inputs larger than L2 (weights %.1f GB read every step)" %
                          ((sh.body_params() + sh.vocab * sh.d_model) * 2 / 1e9),
                    "gemm_impl": "cuda-cores" if args.cuda_cores else "tcgen05",
-                   "fp8": bool(args.fp8)},
+                   "fp8": bool(args.fp8),
+                   **({"layers_slice": args.layers, "note": "layer slice for profiling, not a "
+                       "bench line"} if args.layers else {})},
         "steps_per_s": steps_s,
         "scored_tokens_per_s": tok_s,
         "target_tokens_per_s": world * S / (ms / 1000.0),

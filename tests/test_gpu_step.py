@@ -133,6 +133,26 @@ def test_opt_13b_width_layer_full_batch_64_bf16_same_state_parity():
     _bf16_same_state_parity(w, shape, batch, pre_steps=1)
 
 
+def test_tiny_bf16_many_rows_parity_and_cobatching():
+    """160 physical rows of ~62 tokens (~9900 tokens, more 128-row tiles than CTA pairs): the
+    bank shrink's CTA pairs each take a second tile, handing the split halves over twice;
+    L+- against the oracle, and co-batched foreground rows bit-identical to scored alone."""
+    w = dataclasses.replace(TINY_BF16, batch=80, len_lo=60, len_hi=64, fg_rows=6)
+    batch = wl.make_batch(w)
+    assert batch.n_tokens_physical - int(batch.fg_seq_lens.sum()) > 74 * 128
+    _bf16_same_state_parity(w, w.shape, wl.Batch(batch.prompts, batch.target_lens, [],
+                                                 np.zeros(0, np.int32)), pre_steps=2)
+    model, h = gpu_handle(w, fg=6)
+    toks, ftoks = dev_tokens(batch), dev_fg_tokens(batch)
+    for t in range(2):
+        h.zo_probe_plan(t, w.eps)
+        _, _, _, flp = h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, ftoks,
+                                          batch.fg_seq_lens, batch.fg_target_lens)
+        alone = h.zo_score_foreground(ftoks, batch.fg_seq_lens, batch.fg_target_lens)
+        assert torch.equal(flp, alone), t
+        h.zo_step(w.lr)
+
+
 def test_qwen3_bf16_same_state_parity():
     shape = dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16)
     w = dataclasses.replace(QWEN_SMALL, shape=shape, fg_rows=0)
@@ -303,8 +323,13 @@ def test_call_order_and_argument_errors():
     assert e.value.code == zo.ZO_ERR_ARG
 
 
-def test_state_transition_bytes_counted():
-    w = TINY
+@pytest.mark.parametrize("dtype", [wl.DTYPE_FP32, wl.DTYPE_BF16])
+def test_state_transition_bytes_counted(dtype):
+    """The byte model of the state change: U written each step (fp32, or bf16 only for bf16
+    models); the update writes the slot's accumulator (and its bf16 mirror) without reading
+    it, rebuilding it from the window's coefficients (their history read, this step's
+    written); a window writes V, its two copies in the extension operand and a zeroed slot."""
+    w = dataclasses.replace(TINY, shape=wl.shrink_shape(wl.TINY, dtype=dtype))
     batch = wl.make_batch(w)
     model, h = gpu_handle(w, nu=4)
     toks = dev_tokens(batch)
@@ -314,13 +339,46 @@ def test_state_transition_bytes_counted():
         h.zo_step(w.lr)
     s = h.zo_stats()
     sh = w.shape
+    es = 2 if dtype == wl.DTYPE_BF16 else 4
+    mirror = 2 if dtype == wl.DTYPE_BF16 else 0
     u = sum(sh.matrix_dims(m)[0] * w.rank for m in w.matrices) * sh.n_layers
     v = sum(sh.matrix_dims(m)[1] * w.rank for m in w.matrices) * sh.n_layers
-    per_step = 4 * u + (8 * u + 4 * u)              # fp32 model: no bf16 copies
-    per_window = 4 * v + 2 * 4 * v + 4 * u
-    assert s["state_transition_bytes"] == 6 * per_step + 2 * per_window
-    assert s["dense_ref_bytes"] == 6 * 2 * 4 * sh.body_params()
+    per_step_u = (2 if dtype == wl.DTYPE_BF16 else 4) * u
+    replay_lens = [1, 2, 3, 4, 1, 2]                   # steps since the slot opened (nu = 4)
+    updates = sum((4 + mirror) * u + 4 * n for n in replay_lens)
+    per_window = 4 * v + 2 * es * v + (4 + mirror) * u
+    assert s["state_transition_bytes"] == 6 * per_step_u + updates + 2 * per_window
+    assert s["dense_ref_bytes"] == 6 * 2 * es * sh.body_params()
     assert s["steps"] == 6 and s["bank_slots"] == 2
+
+
+@pytest.mark.parametrize("shape", ["tiny-bf16", "qwen3-bf16"])
+def test_bank_replay_equals_read_modify_write(shape, monkeypatch):
+    """The update that rebuilds the slot from its coefficients and the one that reads it back
+    give the same bank and the same objectives, bit for bit, across windows (nu = 3)."""
+    if shape == "tiny-bf16":
+        w = TINY_BF16
+    else:
+        w = dataclasses.replace(QWEN_SMALL, shape=dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16),
+                                fg_rows=0)
+    batch = wl.make_batch(w, fg_rows=0)
+    toks = dev_tokens(batch)
+    runs = []
+    for mode in ("1", "0"):
+        monkeypatch.setenv("ZO_BANK_REPLAY", mode)
+        _, h = gpu_handle(w, nu=3)
+        out = []
+        for t in range(8):
+            h.zo_probe_plan(t, w.eps)
+            Lp, Lm, _ = h.zo_score(toks, batch.seq_lens, batch.target_lens)
+            out.append((Lp.cpu().numpy().copy(), Lm.cpu().numpy().copy(), h.zo_step(w.lr)))
+        runs.append((out, h.zo_save_state(), h.zo_stats()["state_transition_bytes"]))
+        h.close()
+    (a, sa, ba), (b, sb, bb) = runs
+    for (x1, y1, c1), (x2, y2, c2) in zip(a, b):
+        assert np.array_equal(x1, x2) and np.array_equal(y1, y2) and c1 == c2
+    assert sa == sb
+    assert ba < bb                                     # the replay reads no accumulator
 
 
 @pytest.mark.parametrize("shape", ["tiny-bf16", "qwen3-bf16"])

@@ -142,6 +142,13 @@ struct zo_handle {
     int* err_dev = nullptr;
     // generator / window / update job tables
     GenJob* genU_d = nullptr; int n_genU = 0; int maxU_pairs = 0;
+    GenJob* genU32_d = nullptr;   // bf16 models: fp32 U jobs, run only by zo_read_factors
+    // bank update: coefficients of the current slot since replay_from (its opening step), or
+    // replay_from = -1 when the slot must be read-modify-written (loaded state, or replay
+    // judged too costly for the factor sizes: replay_enabled)
+    float* coef_hist = nullptr;
+    long long replay_from = -1;
+    bool replay_enabled = false;
     GenJob* genV_d = nullptr; int n_genV = 0; int maxV_pairs = 0;
     WindowJob* win_d = nullptr; int n_win = 0;
     UpdateJob* upd_d = nullptr; int n_upd = 0; int max_upd = 0;
@@ -174,6 +181,7 @@ struct zo_handle {
         float *Lp = nullptr, *Lm = nullptr;
         float eps = 0.f, lr = 0.f;
         int slots = -1;
+        long long replay_from = -2;           // the bank update's mode baked into the graph
         long long T = 0, S = 0;
         uint64_t launches = 0;                // kernels per replay
         uint64_t captures = 0, replays = 0;
@@ -183,7 +191,8 @@ struct zo_handle {
     zo_stats_t stats;
     PhaseTimer tm[3];
     GemmProfiler prof;
-    uint64_t bytes_per_U = 0, bytes_per_window = 0, bytes_per_update = 0;
+    uint64_t bytes_per_U = 0, bytes_per_window = 0;
+    uint64_t a_elems = 0;         // accumulator elements updated per step (all targets)
     uint64_t dense_bytes = 0, dense_bytes_targets = 0;
     std::string err;
     int err_code = 0;
@@ -350,6 +359,16 @@ int run_gemm(zo_handle* h, const GemmArgs& g, double algo_flops) {
     return ZO_OK;
 }
 
+// State-transition bytes of the bank update at step t: the accumulator written in fp32 (and
+// its bf16 mirror); read as well unless it is rebuilt from the slot's coefficients, whose
+// history is then read and this step's written.
+uint64_t update_bytes(const zo_handle* h, uint64_t t) {
+    const uint64_t mirror = h->dt == E_BF16 ? 2 : 0;
+    if (h->replay_from >= 0)
+        return h->a_elems * (4 + mirror) + 4 * (t - (uint64_t)h->replay_from + 1);
+    return h->a_elems * (8 + mirror);
+}
+
 // ---- window opening: V of the window into EB, slot accumulator zeroed ------------------
 int open_window(zo_handle* h, uint64_t step) {
     const int k = h->n_slots;
@@ -365,8 +384,8 @@ int open_window(zo_handle* h, uint64_t step) {
     WindowJob* wj = static_cast<WindowJob*>(h->jobs_h);
     UpdateJob* uj = reinterpret_cast<UpdateJob*>(wj + h->n_win);
     int nw = 0, nu = 0, max_n = 0;
-    for (auto& L : h->layers)
-        for (auto& G : L.g)
+    for (int l = 0; l < (int)h->layers.size(); ++l)
+        for (auto& G : h->layers[l].g)
             for (int t = 0; t < G.n_t; ++t) {
                 WindowJob w;
                 w.V = G.Vcur[t];
@@ -387,10 +406,13 @@ int open_window(zo_handle* h, uint64_t step) {
                 wj[nw++] = w;
                 UpdateJob u;
                 u.A = w.A;
-                u.U = G.FT + (size_t)(t * r) * G.K;
                 u.A_bf = w.A_bf;
-                u.n = r * G.K;
-                max_n = std::max(max_n, u.n);
+                u.layer = l;
+                u.matrix = G.mats[t];
+                u.dim = G.K;
+                u.r = r;
+                u.ld = G.K;
+                max_n = std::max(max_n, (r * G.K + 1) / 2);
                 uj[nu++] = u;
             }
     CK(h, cudaMemcpyAsync(h->win_d, wj, sizeof(WindowJob) * nw, cudaMemcpyHostToDevice, h->st));
@@ -401,6 +423,8 @@ int open_window(zo_handle* h, uint64_t step) {
     h->stats.kernel_launches += 2;
     h->n_slots = k + 1;
     h->slot_window.push_back((int64_t)(step / (uint64_t)h->opt.lazy_interval));
+    // the new slot starts at zero: from here its updates can be replayed from coefficients
+    h->replay_from = h->replay_enabled ? (long long)step : -1;
     h->stats.state_transition_bytes += h->bytes_per_window;
     return ZO_OK;
 }
@@ -720,18 +744,22 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
     CK(h, cudaMemsetAsync(h->flag_dev, 0, 4, h->st));
 
     // generator job tables (constant for the run) and the job staging area
-    std::vector<GenJob> gu, gv;
+    std::vector<GenJob> gu, gv, gu32;
     uint64_t u_elems = 0, v_elems = 0, a_elems = 0;
     for (int l = 0; l < d.n_layers; ++l)
         for (auto& G : h->layers[l].g)
             for (int t = 0; t < G.n_t; ++t) {
                 int di, dout;
                 matrix_dims(d, G.mats[t], &di, &dout);
-                GenJob ju{G.FT + (size_t)t * r * G.K,
+                // bf16 models keep U in bf16 only: the shrink reads the bf16 rows and the
+                // bank update regenerates U in fp32 from the counter stream
+                GenJob ju{G.FTb ? nullptr : G.FT + (size_t)t * r * G.K,
                           G.FTb ? static_cast<char*>(G.FTb) + (size_t)t * r * G.K * 2 : nullptr,
                           l, G.mats[t], 0, di, r, 1, G.K};
+                GenJob ju32{G.FT + (size_t)t * r * G.K, nullptr, l, G.mats[t], 0, di, r, 1, G.K};
                 GenJob jv{G.Vcur[t], nullptr, l, G.mats[t], 1, dout, r, 0, 0};
                 gu.push_back(ju);
+                gu32.push_back(ju32);
                 gv.push_back(jv);
                 h->maxU_pairs = std::max(h->maxU_pairs, (di * r + 1) / 2);
                 h->maxV_pairs = std::max(h->maxV_pairs, (dout * r + 1) / 2);
@@ -749,19 +777,36 @@ int zo_create(const zo_model_desc* desc, const zo_weights* weights, const zo_opt
                               cudaMemcpyHostToDevice, h->st));
         CK(h, cudaMemcpyAsync(h->genV_d, gv.data(), sizeof(GenJob) * gv.size(),
                               cudaMemcpyHostToDevice, h->st));
+        if (h->dt == E_BF16) {
+            CRC(dev_alloc(h, reinterpret_cast<void**>(&h->genU32_d), sizeof(GenJob) * gu32.size()));
+            CK(h, cudaMemcpyAsync(h->genU32_d, gu32.data(), sizeof(GenJob) * gu32.size(),
+                                  cudaMemcpyHostToDevice, h->st));
+        }
+        CRC(dev_alloc(h, reinterpret_cast<void**>(&h->coef_hist),
+                      (size_t)options->lazy_interval * 4));
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->win_d), sizeof(WindowJob) * gu.size()));
         CRC(dev_alloc(h, reinterpret_cast<void**>(&h->upd_d), sizeof(UpdateJob) * gu.size()));
         h->jobs_bytes = (sizeof(WindowJob) + sizeof(UpdateJob)) * gu.size();
         cudaError_t e = cudaHostAlloc(&h->jobs_h, h->jobs_bytes, cudaHostAllocDefault);
         if (e != cudaSuccess) { h->err = "pinned staging allocation failed"; return fail(ZO_ERR_OOM); }
     }
-    // state-transition byte model: U written each step; A read+written and U read by the
-    // update; at a window start V written (fp32), EB written twice (model dtype), A zeroed.
-    // bf16 models also keep bf16 copies of U and A (the shrink GEMM's operand)
+    // state-transition byte model: U written each step (fp32, or bf16 only for bf16 models);
+    // the update writes A (and its bf16 mirror) and reads it unless it replays the slot's
+    // coefficients (update_bytes); at a window start V written (fp32), EB written twice
+    // (model dtype), A and its mirror zeroed
     const uint64_t mirror = h->dt == E_BF16 ? 2 : 0;
-    h->bytes_per_U = u_elems * (4 + mirror);
-    h->bytes_per_update = a_elems * (8 + mirror) + u_elems * 4;
+    h->bytes_per_U = u_elems * (h->dt == E_BF16 ? 2 : 4);
+    h->a_elems = a_elems;
     h->bytes_per_window = v_elems * 4 + v_elems * 2 * es + a_elems * (4 + mirror);
+    // Rebuilding the slot from its coefficients regenerates one normal per element for every
+    // step of the window so far: worth it while that stays small next to the step (low-rank
+    // factors); high-rank factorised directions read-modify-write instead.  ZO_BANK_REPLAY=0|1
+    // forces the choice (both give the same bits).
+    h->replay_enabled = u_elems * (uint64_t)options->lazy_interval <= (1ull << 26);
+    if (const char* rp = std::getenv("ZO_BANK_REPLAY")) {
+        if (rp[0] == '0') h->replay_enabled = false;
+        if (rp[0] == '1') h->replay_enabled = true;
+    }
     // dense mutation reference: 2 * |theta| bytes (model dtype) per step
     uint64_t body = 0, tgt = 0;
     for (int l = 0; l < d.n_layers; ++l)
@@ -1379,7 +1424,10 @@ int zo_step_from_sums(zo_handle* h, float lr, const double* dev_sums, double* c_
     if (!std::isfinite(lr)) FAIL(h, ZO_ERR_ARG, "lr must be finite");
     timer_begin(h, 2);
     launch_estimate(dev_sums, h->plan.eps, h->c_dev, h->flag_dev, h->st);
-    launch_bank_update(h->upd_d, h->n_genU, h->max_upd, h->c_dev, h->flag_dev, lr, h->st);
+    launch_bank_update(h->upd_d, h->n_genU, h->max_upd, h->c_dev, h->flag_dev, lr,
+                       h->opt.run_seed, h->step, nullptr, (uint64_t)h->opt.lazy_interval,
+                       h->mezo_scale, h->opt.targets.scale_mode == ZO_SCALE_MEZO,
+                       h->replay_from, h->coef_hist, h->st);
     h->stats.kernel_launches += 1 + (h->n_genU > 0);
     timer_end(h, 2);
     CK(h, cudaGetLastError());
@@ -1395,7 +1443,7 @@ int zo_step_from_sums(zo_handle* h, float lr, const double* dev_sums, double* c_
         }
         if (flag) FAIL(h, ZO_ERR_NONFINITE, "non-finite objective: update refused");
     }
-    h->stats.state_transition_bytes += h->bytes_per_update;
+    h->stats.state_transition_bytes += update_bytes(h, h->step);
     h->stats.dense_ref_bytes += h->dense_bytes;
     h->stats.dense_ref_bytes_targets += h->dense_bytes_targets;
     h->stats.steps++;
@@ -1435,6 +1483,7 @@ int zo_step_graph(zo_handle* h, const int32_t* packed_tokens, int32_t n_prompts,
     }
     const bool same = G.exec && G.tok == packed_tokens && G.Lp == L_plus && G.Lm == L_minus &&
                       G.eps == eps && G.lr == lr && G.slots == h->n_slots &&
+                      G.replay_from == h->replay_from &&
                       (int)G.lens.size() == B &&
                       std::equal(G.lens.begin(), G.lens.end(), seq_lens) &&
                       std::equal(G.tls.begin(), G.tls.end(), target_lens);
@@ -1476,7 +1525,10 @@ int zo_step_graph(zo_handle* h, const int32_t* packed_tokens, int32_t n_prompts,
             launch_row_objective(h->logprob, soff_d, R, B, h->L_row, L_plus, L_minus, h->st);
             launch_objective_sums(h->L_row, B, h->sums, h->st);
             launch_estimate(h->sums, eps, h->c_dev, h->flag_dev, h->st);
-            launch_bank_update(h->upd_d, h->n_genU, h->max_upd, h->c_dev, h->flag_dev, lr, h->st);
+            launch_bank_update(h->upd_d, h->n_genU, h->max_upd, h->c_dev, h->flag_dev, lr,
+                               h->opt.run_seed, 0, G.step_dev, nu, h->mezo_scale,
+                               h->opt.targets.scale_mode == ZO_SCALE_MEZO, h->replay_from,
+                               h->coef_hist, h->st);
             launch_advance_step(G.step_dev, h->st);
         }
         const uint64_t launched = h->stats.kernel_launches - k0;
@@ -1497,6 +1549,7 @@ int zo_step_graph(zo_handle* h, const int32_t* packed_tokens, int32_t n_prompts,
         }
         G.tok = packed_tokens; G.Lp = L_plus; G.Lm = L_minus; G.eps = eps; G.lr = lr;
         G.slots = h->n_slots;
+        G.replay_from = h->replay_from;
         G.lens.assign(seq_lens, seq_lens + B);
         G.tls.assign(target_lens, target_lens + B);
         G.T = bp.T; G.S = bp.S;
@@ -1517,7 +1570,7 @@ int zo_step_graph(zo_handle* h, const int32_t* packed_tokens, int32_t n_prompts,
     h->stats.tokens_scored += (uint64_t)G.T;
     h->stats.positions_scored += (uint64_t)G.S;
     h->stats.score_calls++;
-    h->stats.state_transition_bytes += h->bytes_per_U + h->bytes_per_update;
+    h->stats.state_transition_bytes += h->bytes_per_U + update_bytes(h, step);
     h->stats.dense_ref_bytes += h->dense_bytes;
     h->stats.dense_ref_bytes_targets += h->dense_bytes_targets;
     h->stats.steps++;
@@ -1645,6 +1698,7 @@ int zo_load_state(zo_handle* h, const void* buf, size_t n) {
             }
     CK(h, cudaStreamSynchronize(h->st));
     h->step = hd.step;
+    h->replay_from = -1;     // the loaded accumulator has no coefficient history here
     return ZO_OK;
 }
 
@@ -1666,6 +1720,10 @@ int zo_read_factors(zo_plan* plan, int32_t layer, int32_t matrix, float* U_host,
     if (!G) FAIL(h, ZO_ERR_ARG, "not a target matrix");
     const int r = h->opt.rank;
     if (U_host) {
+        if (h->genU32_d)      // bf16 models keep U in bf16: draw the fp32 rows for the copy
+            launch_gen_factors(h->genU32_d, h->n_genU, h->maxU_pairs, h->opt.run_seed,
+                               plan->step, nullptr, (uint64_t)h->opt.lazy_interval,
+                               h->mezo_scale, h->opt.targets.scale_mode == ZO_SCALE_MEZO, h->st);
         std::vector<float> ut((size_t)r * G->K);
         CK(h, cudaMemcpyAsync(ut.data(), G->FT + (size_t)t * r * G->K, ut.size() * 4,
                               cudaMemcpyDeviceToHost, h->st));

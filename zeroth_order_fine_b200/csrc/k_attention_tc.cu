@@ -1,19 +1,24 @@
 // Packed variable-length causal attention on the 5th-generation tensor cores.
 //
-// Work items are (128-query tile of one row, head) pairs, one CTA (4 warps,
-// 128 threads) each; thread i owns query row i of the tile, which is also TMEM
-// lane i.  Per 128-key chunk of the row:
-//   S  = Q K^T        tcgen05.mma M=128 N=128 K=128, fp32 accumulator in TMEM
-//   P  = exp(S*scale - m)  (causal and length masks) written as bf16 into the
-//                     K buffer, in the 128-byte-swizzled K-major layout
-//   O += P V          tcgen05.mma M=128 N=128 K=128, V read as an MN-major operand
-// Across chunks the softmax is online: the running maximum and sum live in the
-// thread's registers, the output row in TMEM, rescaled by exp(m_old - m_new)
-// before each chunk's P V accumulates onto it.  Queries, keys and
-// values arrive by TMA straight into the 128-byte-swizzled layout (Qwen3's
-// q/k norm and rotary positions were applied to the q|k|v rows beforehand).
-// Keys past the row's end are masked to zero probability, so a query's result
-// depends only on its own row: packing never changes a bit.
+// Work items are (128-query tile of one row, head) pairs.  One persistent CTA per
+// SM walks its items in turn with its warps specialised:
+//   warp 0      TMA producer: Q of an item, then K and V of each 128-key chunk,
+//               into two stages of 128-byte-swizzled shared-memory buffers
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
+//                 S = Q K^T      M=128 N=128 K=128 into one of two TMEM S buffers
+//                 O (+)= P V     into one of two TMEM O buffers (one per item in flight)
+//               S of the next chunk is issued while the softmax works on this one
+//   warps 2..5  softmax and epilogue, one query row per thread (= its TMEM lane):
+//               P = exp(S*scale - m) with the causal and row-end masks, written as
+//               bf16 over the chunk's K buffer in the swizzled K-major layout; across
+//               chunks the softmax is online (running max and sum in registers, the
+//               output rescaled in TMEM); at the item's end O / l goes to memory
+// So the next item's loads and its Q K^T overlap this item's softmax and store.
+// Queries, keys and values arrive by TMA straight from the packed q|k|v rows (Qwen3's
+// q/k norm and rotary positions were applied beforehand).  Keys past the row's end
+// get zero probability, so a query's result depends only on its own row: packing
+// never changes a bit.  Every wait is bounded; on expiry the kernel records the error
+// word, drains what it issued, frees its tensor memory and returns.
 #include <cuda.h>
 #include <float.h>
 
@@ -27,8 +32,11 @@ namespace {
 constexpr int TQ = 128, TK = 128, HD = 128;
 constexpr int ATOM = TQ * 128;                  // bytes of one 64-column swizzle atom block
 constexpr int BUF = 2 * ATOM;                   // one [128 x 128] bf16 operand
-constexpr int SMEM = 3 * BUF + 1024 + 64;
+// Q[2] K[2] V[2] buffers, then 19 mbarriers, the TMEM base and the abort flag
+constexpr int SMEM = 6 * BUF + 1024 + 256;
+constexpr int NTHREADS = 192;
 constexpr long long WAIT_CYCLES = 4000000000ll;
+constexpr uint32_t DRAIN_POLLS = 1u << 24;      // drain polls (with back-off) after an abort
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TK >> 3) << 17) |
                             ((uint32_t)(TQ >> 4) << 24);
 
@@ -90,41 +98,75 @@ __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* err) {
+__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// try_wait suspending at most ~1 us, so a waiting thread looks at its clock regularly
+__device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000u)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait; false when the bound expired (recorded in the error word) or another role
+// of the CTA aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_f,
+                                         int* err) {
+    if (bar_test(bar, parity)) return true;
     const long long t0 = clock64();
-    for (uint32_t i = 0;; ++i) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        if ((i & 63u) == 63u && clock64() - t0 > WAIT_CYCLES) {   // ~2 s: never arrives
+    for (;;) {
+        if (bar_try(bar, parity)) return true;
+        if (*abort_f) return false;
+        if (clock64() - t0 > WAIT_CYCLES) {   // ~2 s: never arrives
+            *abort_f = 1;
             atomicOr(err, 1);
             return false;
         }
     }
 }
-
-// 8 MMAs (K = 128 = 2 atoms x 4 steps of 16) into TMEM column d_col, then commit.
-__device__ __forceinline__ void mma_128(uint32_t d_tmem, uint32_t a, uint32_t b, bool accum_first,
-                                        uint32_t bar) {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * ATOM + (kk & 3) * 32;
-        const uint32_t acc = (kk > 0 || accum_first) ? 1u : 0u;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-            "l"(sw128_desc(a + off)), "l"(sw128_desc(b + off)), "r"(kIdesc), "r"(acc)
-            : "memory");
-    }
+// Drain after an abort: let an issued copy or MMA land before shared memory goes away.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < DRAIN_POLLS && !bar_test(bar, parity); ++i) __nanosleep(128);
+}
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      bar)
                  : "memory");
+}
+
+// S = Q K^T: 8 MMAs (K = 128 = 2 swizzle atoms x 4 steps of 16) into TMEM at d_tmem.
+__device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint32_t q, uint32_t k) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * ATOM + (kk & 3) * 32;
+        const uint32_t acc = kk > 0 ? 1u : 0u;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(sw128_desc(q + off)), "l"(sw128_desc(k + off)), "r"(kIdesc), "r"(acc)
+            : "memory");
+    }
 }
 
 __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
@@ -175,36 +217,73 @@ __device__ __forceinline__ float ex2_ftz(float x) {
     return y;
 }
 
-// One CTA per item, two CTAs per SM: while one CTA waits on its TMA loads or
-// its MMAs, the other runs its softmax.  Items are dealt longest first.
-__global__ void __launch_bounds__(128, 2)
+// O (+)= P V: A = P (K-major, keys contiguous) over the chunk's K buffer, B = V as loaded
+// ([keys x dims], MN-major); 8 MMAs of K = 16 keys.
+__device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t pb, uint32_t vb, bool accum) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = (kk > 0 || accum) ? 1u : 0u;
+        const uint64_t ad = sw128_desc(pb + (kk >> 2) * ATOM + (kk & 3) * 32);
+        const uint64_t bd = sw128_desc_mn(vb + kk * 2048);
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(ad), "l"(bd), "r"(kIdescPV), "r"(acc)
+            : "memory");
+    }
+}
+
+// Persistent: CTA b takes items b, b + gridDim.x, ... (dealt longest first by the host).
+// Chunks are numbered g = 0, 1, ... across the CTA's items: chunk g uses K/V stage g & 1
+// and S buffer g & 1; item k uses Q buffer and O buffer k & 1.  Phases follow from the
+// counters: the n-th use of a two-slot resource waits parity (n >> 1) & 1.
+__global__ void __launch_bounds__(NTHREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* g = smem_raw + (base - raw);
-    uint8_t* Qb = g;
-    uint8_t* KPb = g + BUF;
-    uint8_t* Vb = g + 2 * BUF;
-    const uint32_t bar_mma = base + 3 * BUF;
-    const uint32_t bar_ld = bar_mma + 8;               // Q and K of a chunk
-    const uint32_t bar_v = bar_mma + 16;               // V of a chunk: lands under QK^T + softmax
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 3 * BUF + 32);
+    auto Qb = [&](int i) { return base + (uint32_t)(i * BUF); };
+    auto Kb = [&](int i) { return base + (uint32_t)((2 + i) * BUF); };
+    auto Vb = [&](int i) { return base + (uint32_t)((4 + i) * BUF); };
+    const uint32_t bar0 = base + 6 * BUF;
+    auto q_full = [&](int i) { return bar0 + 8u * (0 + i); };
+    auto q_empty = [&](int i) { return bar0 + 8u * (2 + i); };
+    auto k_full = [&](int i) { return bar0 + 8u * (4 + i); };
+    auto v_full = [&](int i) { return bar0 + 8u * (6 + i); };
+    auto kv_empty = [&](int i) { return bar0 + 8u * (8 + i); };
+    auto s_full = [&](int i) { return bar0 + 8u * (10 + i); };
+    auto p_full = [&](int i) { return bar0 + 8u * (12 + i); };
+    auto o_full = [&](int i) { return bar0 + 8u * (14 + i); };
+    auto o_free = [&](int i) { return bar0 + 8u * (16 + i); };
+    const uint32_t drain = bar0 + 8u * 18;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 6 * BUF + 160);
+    volatile int* abort_f = reinterpret_cast<volatile int*>(g + 6 * BUF + 168);
 
-    const Item it = get_item(a, blockIdx.x);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_items = a.n_tiles * a.H;
     const int q_dim = a.H * HD, kv_dim = a.Hkv * HD;
-    const int tid = threadIdx.x, warp = tid >> 5;
     int* err = &g_attn_error;
 
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ld));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_v));
+        for (int i = 0; i < 2; ++i) {
+            bar_init(q_full(i), 1);
+            bar_init(q_empty(i), 1);
+            bar_init(k_full(i), 1);
+            bar_init(v_full(i), 1);
+            bar_init(kv_empty(i), 1);
+            bar_init(s_full(i), 1);
+            bar_init(p_full(i), 4);            // one arrival per softmax warp
+            bar_init(o_full(i), 1);
+            bar_init(o_free(i), 4);
+        }
+        bar_init(drain, 1);
+        *abort_f = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                          smem_u32(tslot))
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -213,180 +292,241 @@ __global__ void __launch_bounds__(128, 2)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tslot;
-    const uint32_t t_s = tmem, t_o = tmem + 128;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    uint32_t ph_mma = 0, ph_ld = 0, ph_v = 0;
-    bool ok = true, v_pending = false;
-    const int q = it.q0 + tid;                         // this thread's query
-    const float sl2 = a.scale * 1.4426950408889634f;
-    const int kcol = q_dim + it.kvh * HD, vcol = q_dim + kv_dim + it.kvh * HD;
+    auto t_s = [&](int i) { return tmem + (uint32_t)(i * 128); };         // S buffers: cols 0, 128
+    auto t_o = [&](int i) { return tmem + (uint32_t)(256 + i * 128); };   // O buffers: 256, 384
 
-    float m = -FLT_MAX, l = 0.f;
-    for (int c = 0; c < it.n_chunks && ok; ++c) {
-        const int c0 = c * TK;
-        // K and V of chunk c (and Q with the first): rows past the tensor read as zero
-        if (tid == 0) {
-            const uint32_t bytes = (uint32_t)BUF * (c == 0 ? 2u : 1u);
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_ld),
-                         "r"(bytes)
-                         : "memory");
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_v),
-                         "r"((uint32_t)BUF)
-                         : "memory");
-            const int r0 = it.start + c0;
-            for (int half = 0; half < 2; ++half) {
-                if (c == 0)
-                    tma_box(smem_u32(Qb) + half * ATOM, &tm, bar_ld, it.h * HD + half * 64,
+    int gq = 0, gcl = 0;                         // producer: Q loads and K/V chunk loads issued
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int& gc = gcl;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int idx = blockIdx.x + k * gridDim.x;
+                if (idx >= n_items) break;
+                const Item it = get_item(a, idx);
+                const int qs = k & 1;
+                if (!wait_bar(q_empty(qs), ((k >> 1) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
+                bar_expect_tx(q_full(qs), BUF);
+                for (int half = 0; half < 2; ++half)
+                    tma_box(Qb(qs) + half * ATOM, &tm, q_full(qs), it.h * HD + half * 64,
                             it.start + it.q0);
-                tma_box(smem_u32(KPb) + half * ATOM, &tm, bar_ld, kcol + half * 64, r0);
-            }
-            for (int half = 0; half < 2; ++half)
-                tma_box(smem_u32(Vb) + half * ATOM, &tm, bar_v, vcol + half * 64, r0);
-        }
-        v_pending = true;
-        ok = __syncthreads_and(wait_bar(bar_ld, ph_ld, err));
-        ph_ld ^= 1u;
-        if (!ok) break;
-
-        // S = Q K^T
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
-        if (tid == 0) mma_128(t_s, smem_u32(Qb), smem_u32(KPb), false, bar_mma);
-        ok = __syncthreads_and(wait_bar(bar_mma, ph_mma, err));
-        ph_mma ^= 1u;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (!ok) break;
-
-        // keys c0 + j with j < lim are visible to this query (causal and row end); column
-        // groups of 32 keys that no query of the warp sees are skipped, and so are warps
-        // whose queries all lie past the row's end (warp-uniform; their P rows are zero)
-        const int lim = min(q + 1, it.kend) - c0;
-        const int wlim = min(it.q0 + warp * 32 + 32, it.kend) - c0;
-        const bool warp_live = it.q0 + warp * 32 < it.len;
-        const int ncc = (!warp_live || wlim <= 0) ? 0 : min(4, (wlim + 31) >> 5);
-        float sv[4][32];
-        float cmax = -FLT_MAX;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            if (cc < ncc) {
-                tmem_ld32(t_s + lane_addr + cc * 32, sv[cc]);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    sv[cc][j] = (cc * 32 + j < lim) ? sv[cc][j] : -FLT_MAX;
-                    cmax = fmaxf(cmax, sv[cc][j]);
+                ++gq;
+                const int kcol = q_dim + it.kvh * HD, vcol = q_dim + kv_dim + it.kvh * HD;
+                for (int c = 0; c < it.n_chunks; ++c) {
+                    const int st = gc & 1;
+                    if (!wait_bar(kv_empty(st), ((gc >> 1) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
+                    const int r0 = it.start + c * TK;
+                    bar_expect_tx(k_full(st), BUF);
+                    for (int half = 0; half < 2; ++half)
+                        tma_box(Kb(st) + half * ATOM, &tm, k_full(st), kcol + half * 64, r0);
+                    bar_expect_tx(v_full(st), BUF);
+                    for (int half = 0; half < 2; ++half)
+                        tma_box(Vb(st) + half * ATOM, &tm, v_full(st), vcol + half * 64, r0);
+                    ++gc;
                 }
             }
         }
-        const float m_new = fmaxf(m, cmax);
-        // rows whose every key so far is masked keep m = -FLT_MAX and contribute nothing
-        const float alpha = (m > -FLT_MAX) ? exp2f((m - m_new) * sl2) : 0.f;
-        // masked scores are -FLT_MAX, so exp2(s*sl2 - ms) underflows to exactly 0 for them
-        const float ms = (m_new > -FLT_MAX) ? m_new * sl2 : 0.f;
-        float cs0 = 0.f, cs1 = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            uint32_t w[16];
-            if (cc < ncc) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const float p0 = ex2_ftz(fmaf(sv[cc][j], sl2, -ms));
-                    const float p1 = ex2_ftz(fmaf(sv[cc][j + 1], sl2, -ms));
-                    cs0 += p0;
-                    cs1 += p1;
-                    w[j / 2] = pack_bf2(p0, p1);
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            // S may run one chunk ahead of P V: chunk gs's S reuses the S buffer of chunk
+            // gs - 2, whose P (so its S was read) arrived before P V of gs - 2 was issued
+            int sk = 0, sc = 0, gs = 0;          // next S: item counter, chunk, global chunk
+            int pk = 0, pc = 0, gp = 0;          // next P V
+            Item s_it, p_it;
+            bool s_more = blockIdx.x < n_items, p_more = s_more;
+            if (s_more) { s_it = get_item(a, blockIdx.x); p_it = s_it; }
+            bool ok = true, issued = false;
+            long long t0 = clock64();
+            while (p_more && ok) {
+                bool progress = false;
+                if (s_more && gs <= gp + 1 && (sc > 0 || bar_test(q_full(sk & 1), (sk >> 1) & 1)) &&
+                    bar_test(k_full(gs & 1), (gs >> 1) & 1)) {
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    mma_qk(t_s(gs & 1), Qb(sk & 1), Kb(gs & 1));
+                    tc_commit(s_full(gs & 1));
+                    issued = progress = true;
+                    ++gs;
+                    if (++sc == s_it.n_chunks) {
+                        sc = 0;
+                        ++sk;
+                        const int idx = blockIdx.x + sk * gridDim.x;
+                        s_more = idx < n_items;
+                        if (s_more) s_it = get_item(a, idx);
+                    }
                 }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) w[j] = 0u;
+                if (gp < gs && bar_test(p_full(gp & 1), (gp >> 1) & 1) &&
+                    bar_test(v_full(gp & 1), (gp >> 1) & 1) &&
+                    (pc > 0 || bar_test(o_free(pk & 1), ((pk >> 1) & 1) ^ 1u))) {
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    mma_pv(t_o(pk & 1), Kb(gp & 1), Vb(gp & 1), pc > 0);
+                    tc_commit(kv_empty(gp & 1));         // K/P and V of the chunk are free
+                    issued = progress = true;
+                    ++gp;
+                    if (++pc == p_it.n_chunks) {
+                        tc_commit(o_full(pk & 1));       // the item's output is complete
+                        tc_commit(q_empty(pk & 1));      // and its Q buffer free
+                        pc = 0;
+                        ++pk;
+                        const int idx = blockIdx.x + pk * gridDim.x;
+                        p_more = idx < n_items;
+                        if (p_more) p_it = get_item(a, idx);
+                    }
+                }
+                if (progress) {
+                    t0 = clock64();
+                } else {
+                    __nanosleep(32);                     // leave the issue slots to the softmax
+                    if (*abort_f) {
+                        ok = false;
+                    } else if (clock64() - t0 > WAIT_CYCLES) {
+                        *abort_f = 1;
+                        atomicOr(err, 1);
+                        ok = false;
+                    }
+                }
             }
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-                *reinterpret_cast<uint4*>(KPb + sw_off(tid, cc * 4 + k4)) =
-                    make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
+            if (issued) {
+                // every MMA retired before the CTA moves on (and before TMEM is freed)
+                tc_commit(drain);
+                drain_bar(drain, 0);
+            }
         }
-        l = l * alpha + (cs0 + cs1);
-        m = m_new;
-        if (c > 0) {
-            // the running output stays in TMEM: rescale it by exp(m_old - m_new), then P V
-            // accumulates on top of it
+    } else {
+        // ---------------- softmax and epilogue (warps 2..5) ----------------
+        const int wq = warp & 3;                 // TMEM lane quarter this warp may access
+        const int row = wq * 32 + lane;          // query row of the tile = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+        const float sl2 = a.scale * 1.4426950408889634f;
+        uint8_t* kbuf[2] = {g + 2 * BUF, g + 3 * BUF};
+        int gc = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            const int idx = blockIdx.x + k * gridDim.x;
+            if (idx >= n_items) break;
+            const Item it = get_item(a, idx);
+            const int q = it.q0 + row;
+            const int os = k & 1;
+            float m = -FLT_MAX, l = 0.f;
+            for (int c = 0; c < it.n_chunks; ++c, ++gc) {
+                const int st = gc & 1;
+                if (!wait_bar(s_full(st), (gc >> 1) & 1, abort_f, err)) { ok = false; break; }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const int c0 = c * TK;
+                // keys c0 + j with j < lim are visible to this query (causal and row end);
+                // column groups of 32 keys that no query of the warp sees are skipped, and so
+                // are warps whose queries all lie past the row's end (their P rows are zero)
+                const int lim = min(q + 1, it.kend) - c0;
+                const int wlim = min(it.q0 + wq * 32 + 32, it.kend) - c0;
+                const bool warp_live = it.q0 + wq * 32 < it.len;
+                const int ncc = (!warp_live || wlim <= 0) ? 0 : min(4, (wlim + 31) >> 5);
+                float sv[4][32];
+                float cmax = -FLT_MAX;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    if (cc < ncc) {
+                        tmem_ld32(t_s(st) + lane_addr + cc * 32, sv[cc]);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            sv[cc][j] = (cc * 32 + j < lim) ? sv[cc][j] : -FLT_MAX;
+                            cmax = fmaxf(cmax, sv[cc][j]);
+                        }
+                    }
+                }
+                const float m_new = fmaxf(m, cmax);
+                // rows whose every key so far is masked keep m = -FLT_MAX and add nothing
+                const float alpha = (m > -FLT_MAX) ? exp2f((m - m_new) * sl2) : 0.f;
+                // masked scores are -FLT_MAX, so exp2(s*sl2 - ms) underflows to exactly 0
+                const float ms = (m_new > -FLT_MAX) ? m_new * sl2 : 0.f;
+                float cs0 = 0.f, cs1 = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t w[16];
+                    if (cc < ncc) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            const float p0 = ex2_ftz(fmaf(sv[cc][j], sl2, -ms));
+                            const float p1 = ex2_ftz(fmaf(sv[cc][j + 1], sl2, -ms));
+                            cs0 += p0;
+                            cs1 += p1;
+                            w[j / 2] = pack_bf2(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) w[j] = 0u;
+                    }
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        *reinterpret_cast<uint4*>(kbuf[st] + sw_off(row, cc * 4 + k4)) =
+                            make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
+                }
+                l = l * alpha + (cs0 + cs1);
+                m = m_new;
+                if (c > 0) {
+                    // the running output stays in TMEM: once the previous chunk's P V has
+                    // retired, rescale it by exp(m_old - m_new); this chunk's P V adds on top
+                    const int pv = gc - 1;
+                    if (!wait_bar(kv_empty(pv & 1), (pv >> 1) & 1, abort_f, err)) { ok = false; break; }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll 1
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float v[32];
+                        tmem_ld32(t_o(os) + lane_addr + cc * 32, v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] *= alpha;
+                        tmem_st32(t_o(os) + lane_addr + cc * 32, v);
+                    }
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                }
+                // P is in shared memory (generic proxy -> the tensor core's async proxy)
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) bar_arrive(p_full(st));
+            }
+            if (!ok) break;
+            // epilogue: O / l of this thread's query row, once the item's last P V retired
+            if (!wait_bar(o_full(os), (k >> 1) & 1, abort_f, err)) { ok = false; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                 (size_t)(it.start + q) * a.ld_out +
+                                                 (size_t)it.h * HD);
+            const bool store = row < it.nq;
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
                 float v[32];
-                tmem_ld32(t_o + lane_addr + cc * 32, v);
+                tmem_ld32(t_o(os) + lane_addr + cc * 32, v);     // warp-collective: every lane
+                if (store) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= alpha;
-                tmem_st32(t_o + lane_addr + cc * 32, v);
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        o4[cc * 4 + k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
+                                                     pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
+                                                     pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
+                                                     pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
+                }
             }
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        }
-
-        // O (+)= P V, once V has landed
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        ok = __syncthreads_and(wait_bar(bar_v, ph_v, err));
-        if (!ok) break;
-        ph_v ^= 1u;
-        v_pending = false;
-        if (tid == 0) {
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t acc = (kk > 0 || c > 0) ? 1u : 0u;
-                const uint64_t ad = sw128_desc(smem_u32(KPb) + (kk >> 2) * ATOM + (kk & 3) * 32);
-                const uint64_t bd = sw128_desc_mn(smem_u32(Vb) + kk * 2048);
-                asm volatile(
-                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(t_o),
-                    "l"(ad), "l"(bd), "r"(kIdescPV), "r"(acc)
-                    : "memory");
-            }
-            asm volatile(
-                "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                    bar_mma)
-                : "memory");
-        }
-        ok = __syncthreads_and(wait_bar(bar_mma, ph_mma, err));
-        ph_mma ^= 1u;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // the K/P and V buffers and the S columns are free again
-    }
-    if (ok) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
-                                             (size_t)(it.start + q) * a.ld_out +
-                                             (size_t)it.h * HD);
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-            float v[32];
-            tmem_ld32(t_o + lane_addr + cc * 32, v);          // warp-collective: every lane
-            if (tid < it.nq) {
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4)
-                    o4[cc * 4 + k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
-                                                 pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
-                                                 pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
-                                                 pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
-            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) bar_arrive(o_free(os));
         }
     }
-    if (v_pending && tid == 0) {
-        // an aborted CTA lets its V copy land before its shared memory goes away
-        const long long t0 = clock64();
-        for (;;) {
-            uint32_t done;
-            asm volatile(
-                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                "selp.u32 %0, 1, 0, p;\n\t}"
-                : "=r"(done)
-                : "r"(bar_v), "r"(ph_v)
-                : "memory");
-            if (done || clock64() - t0 > WAIT_CYCLES) break;
+    __syncthreads();                             // every role has left its loop
+    if (*abort_f && warp == 0 && lane == 0) {
+        // an aborted CTA lets every copy still in flight land before its shared memory goes
+        // away: the two newest loads of each kind (older ones were consumed, so had landed)
+        for (int i = gq - 1; i >= 0 && i >= gq - 2; --i) drain_bar(q_full(i & 1), (i >> 1) & 1);
+        for (int i = gcl - 1; i >= 0 && i >= gcl - 2; --i) {
+            drain_bar(k_full(i & 1), (i >> 1) & 1);
+            drain_bar(v_full(i & 1), (i >> 1) & 1);
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem)
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
                      : "memory");
 }
 
@@ -438,7 +578,15 @@ bool launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
         return false;
     const long long items = (long long)a.n_tiles * a.H;
     if (items > 0x7fffffffLL) return false;
-    attention_tc_kernel<<<(unsigned)items, 128, SMEM, st>>>(tm, a);
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    const unsigned grid = (unsigned)(items < sms ? items : sms);
+    attention_tc_kernel<<<grid, NTHREADS, SMEM, st>>>(tm, a);
     return true;
 }
 

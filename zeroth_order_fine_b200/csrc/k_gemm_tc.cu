@@ -95,6 +95,8 @@ struct TcParams {
     int ksplit, kbs;                        // split-K (SPLIT kernels): splits, main blocks each
     int* err;
     long long wait_cycles;                  // bound of every mbarrier wait (clock64 cycles)
+    int k2_last_steps;                      // 16-column MMA steps holding data in the last
+                                            // extension block (its tail is zero padding)
 };
 
 // ---- PTX wrappers ------------------------------------------------------------------
@@ -466,12 +468,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         *n_kb = *n_main + (sp == ks - 1 ? p.kb_ext : 0);
     };
 
+    int n_armed = 0;                        // producer: loads issued; the i-th used stage i % S,
+                                            // phase (i / S) & 1
+    bool issued = false;                    // MMA issuer: any MMA issued
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            int n_armed = 0;                // loads issued; the i-th used stage i % S, phase (i / S) & 1
             bool ok = true;
             for (int t = blockIdx.x; t < n_items && ok; t += gridDim.x) {
                 int mb, nb;
@@ -496,16 +500,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
             }
-            if (!ok) {
-                // drain: let every copy this thread issued land before the CTA exits
-                const int n = n_armed < STAGES ? n_armed : STAGES;
-                for (int i = 0; i < n; ++i) {
-                    const int a = n_armed - 1 - i;
-                    const uint32_t aph = (uint32_t)(a / STAGES) & 1u;
-                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(a % STAGES), aph); ++it)
-                        __nanosleep(128);
-                }
-            }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -514,7 +508,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t ph = 0;
             int acc = 0;
             uint32_t aph = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             for (int t = blockIdx.x; t < n_items && ok; t += gridDim.x) {
                 if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                 tc_fence_after();
@@ -532,10 +526,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             tc_mma_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
                                       T1::IDESC_F8, (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
+                        // the last extension block stops after its last 16 columns of data
+                        const int nk = (i == n_kb - 1 && n_kb > n_main) ? p.k2_last_steps : BK / 16;
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
-                            tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
-                                   (i > 0 || kk > 0) ? 1u : 0u);
+                            if (kk < nk)
+                                tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
+                                       (i > 0 || kk > 0) ? 1u : 0u);
                         }
                     }
                     issued = true;
@@ -545,10 +542,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (!ok) break;
                 tc_commit(tfull(acc));              // accumulator ready for the epilogue
                 if (++acc == 2) { acc = 0; aph ^= 1u; }
-            }
-            if (!ok && issued) {
-                tc_commit(drain);
-                for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(drain, 0); ++it) __nanosleep(128);
             }
         }
     } else {
@@ -609,6 +602,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     }
 
+    tc_fence_before();
+    __syncthreads();                        // every role has left its loop
+    if (*abort_f && lane == 0) {
+        // an aborted CTA lets what it issued finish before its shared and tensor memory go
+        // away, whichever role gave up: the newest copies (older ones were consumed, so had
+        // landed), then every MMA
+        if (warp == 0) {
+            const int n = n_armed < STAGES ? n_armed : STAGES;
+            for (int i = 0; i < n; ++i) {
+                const int a = n_armed - 1 - i;
+                const uint32_t aph = (uint32_t)(a / STAGES) & 1u;
+                for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(a % STAGES), aph); ++it)
+                    __nanosleep(128);
+            }
+        } else if (warp == 1 && issued) {
+            tc_commit(drain);
+            for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(drain, 0); ++it) __nanosleep(128);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1046,11 +1058,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         *n_kb = *n_main + (sp == p.ksplit - 1 ? p.kb_ext : 0);
     };
 
+    int n_armed = 0;                        // producer: loads issued; the i-th used stage i % S,
+                                            // phase (i / S) & 1
+    bool issued = false;                    // MMA issuer (even CTA): any MMA issued
     if (warp == 0) {
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            int n_armed = 0;                // loads issued; the i-th used stage i % S, phase (i / S) & 1
             bool ok = true;
             for (int t = pair; t < n_items && ok; t += n_pairs) {
                 int mb, nb;
@@ -1080,15 +1094,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (++s == STAGES2) { s = 0; ph ^= 1u; }
                 }
             }
-            if (!ok && rank == 0) {
-                const int n = n_armed < STAGES2 ? n_armed : STAGES2;
-                for (int i = 0; i < n; ++i) {
-                    const int a = n_armed - 1 - i;
-                    const uint32_t aph = (uint32_t)(a / STAGES2) & 1u;
-                    for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(a % STAGES2), aph); ++it)
-                        __nanosleep(128);
-                }
-            }
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
@@ -1096,7 +1101,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             uint32_t ph = 0;
             int acc = 0;
             uint32_t aph = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             for (int t = pair; t < n_items && ok; t += n_pairs) {
                 if (!mbar_wait(tempty(acc), aph ^ 1u, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
                 tc_fence_after();
@@ -1115,10 +1120,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                             tc_mma_pair_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
                                            kIdesc2F8, (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
+                        // the last extension block stops after its last 16 columns of data
+                        const int nk = (i == n_kb - 1 && n_kb > n_main) ? p.k2_last_steps : BK / 16;
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
-                                        kIdesc2, (i > 0 || kk > 0) ? 1u : 0u);
+                            if (kk < nk)
+                                tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
+                                            kIdesc2, (i > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     tc_commit_pair(empty(s));       // stage free in both CTAs
@@ -1127,13 +1135,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 if (!ok) break;
                 tc_commit_pair(tfull(acc));         // both halves of the accumulator ready
                 if (++acc == 2) { acc = 0; aph ^= 1u; }
-            }
-            if (!ok && issued) {
-                asm volatile(
-                    "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                        drain)
-                    : "memory");
-                for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(drain, 0); ++it) __nanosleep(128);
             }
         }
     } else {
@@ -1165,12 +1166,281 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
 
     tc_fence_before();
+    __syncthreads();                        // every role of this CTA has left its loop
+    if (*abort_f && lane == 0 && rank == 0) {
+        // an aborted pair lets what it issued finish first, whichever role gave up: both
+        // CTAs' copies complete on the even CTA's barriers, and its thread issued the MMAs
+        if (warp == 0) {
+            const int n = n_armed < STAGES2 ? n_armed : STAGES2;
+            for (int i = 0; i < n; ++i) {
+                const int a = n_armed - 1 - i;
+                const uint32_t aph = (uint32_t)(a / STAGES2) & 1u;
+                for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(a % STAGES2), aph); ++it)
+                    __nanosleep(128);
+            }
+        } else if (warp == 1 && issued) {
+            asm volatile(
+                "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                    drain)
+                : "memory");
+            for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(drain, 0); ++it) __nanosleep(128);
+        }
+    }
+    tc_fence_before();
     __syncthreads();
     cluster_sync();                         // neither CTA leaves while the pair may touch it
     tc_fence_after();
     if (warp == 1) {
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---- bank shrink with K split over a CTA pair ---------------------------------------
+// The shrink S = x FT^T has M = the batch's token rows and N = the bank's few columns, so it
+// has one 128-row tile per 128 tokens (72 for 9196 rows: half the SMs) and is bound by
+// reading x once.  A cluster of two CTAs computes each tile: each streams its half of K
+// into its own TMEM accumulator, the odd CTA hands its fp32 half to the even CTA through
+// distributed shared memory, and the even CTA adds the halves and applies the shrink
+// epilogue.  The split is the same for every M, so a row's bits never depend on the batch.
+template <int BNT>
+struct TileS {
+    static_assert(BNT == 64 || BNT == 128, "shrink N tile");
+    static constexpr int B_BYTES = BNT * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // multiple of 1024
+    static constexpr int STAGES = BNT == 64 ? 7 : 4;
+    static constexpr int PART_LD = BNT + 4;                      // padded rows: no bank clash
+    static constexpr int PART_BYTES = BM * PART_LD * 4;          // the odd CTA's accumulator
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + PART_BYTES + 1024 + 256;
+    static constexpr uint32_t IDESC = Tile1<BNT>::IDESC;
+    // barriers: full, empty per stage; tfull, tempty, part_full, part_free, drain
+    static constexpr int SLOT_OFF = 200, ABORT_OFF = 208;
+    static_assert(8 * (2 * STAGES + 5) <= SLOT_OFF, "barrier region");
+};
+
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000u)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for an arrival from the other CTA of the pair (acquire at cluster scope,
+// so the stores it released are visible).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort_f, int* err,
+                                                  long long limit) {
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_try_cluster(bar, parity)) return true;
+        if (*abort_f) return false;
+        if (clock64() - t0 > limit) {
+            *abort_f = 1;
+            atomicOr(err, 1);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+template <int BNT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    shrink_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    using TS = TileS<BNT>;
+    constexpr int STAGES = TS::STAGES;
+    constexpr int STAGE_BYTES = TS::STAGE_BYTES;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;           // same offset in both CTAs
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t part0 = base + STAGES * STAGE_BYTES;
+    float* part = reinterpret_cast<float*>(gbase + STAGES * STAGE_BYTES);
+    const uint32_t bar0 = part0 + TS::PART_BYTES;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    const uint32_t tfull = bar0 + 8u * (2 * STAGES);
+    const uint32_t tempty = bar0 + 8u * (2 * STAGES + 1);
+    const uint32_t part_full = bar0 + 8u * (2 * STAGES + 2);   // even CTA: the odd half landed
+    const uint32_t part_free = bar0 + 8u * (2 * STAGES + 3);   // odd CTA: the even one read it
+    const uint32_t drain = bar0 + 8u * (2 * STAGES + 4);
+    uint8_t* tail = gbase + STAGES * STAGE_BYTES + TS::PART_BYTES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + TS::SLOT_OFF);
+    volatile int* abort_f = reinterpret_cast<volatile int*>(tail + TS::ABORT_OFF);
+
+    const uint32_t rank = cluster_rank();
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // K blocks of this CTA: the even CTA the first half, the odd one the rest
+    const int half = (p.kb_main + 1) / 2;
+    const int kb0 = rank == 0 ? 0 : half;
+    const int n_kb = rank == 0 ? half : p.kb_main - half;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 4);
+        mbar_init(part_full, 4);            // one arrival per epilogue warp of the odd CTA
+        mbar_init(part_free, 4);            // one per epilogue warp of the even CTA
+        mbar_init(drain, 1);
+        *abort_f = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(BNT)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                          // both CTAs' barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    int n_armed = 0;                         // producer: loads issued
+    bool issued = false;                     // MMA issuer: any MMA issued
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
+                for (int i = 0; i < n_kb; ++i) {
+                    if (!mbar_wait(empty(s), ph ^ 1u, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
+                    const uint32_t sa = base + s * STAGE_BYTES;
+                    mbar_expect_tx(full(s), STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, full(s), (kb0 + i) * BK, t * BM);
+                    tma_load_2d(sa + A_BYTES, &tmB, full(s), (kb0 + i) * BK, 0);
+                    ++n_armed;
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0, tph = 0;
+            bool ok = true;
+            for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
+                if (!mbar_wait(tempty, tph ^ 1u, abort_f, p.err, p.wait_cycles)) break;
+                tc_fence_after();
+                for (int i = 0; i < n_kb; ++i) {
+                    if (!mbar_wait(full(s), ph, abort_f, p.err, p.wait_cycles)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = base + s * STAGE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc_mma(tmem, sw128_desc(sa + kk * 32), sw128_desc(sa + A_BYTES + kk * 32),
+                               TS::IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+                    issued = true;
+                    tc_commit(empty(s));
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(tfull);
+                tph ^= 1u;
+            }
+        }
+    } else {
+        // epilogue: thread = accumulator row (TMEM lane), 32-column chunks
+        const int lane_base = 32 * (warp & 3);
+        const int r = lane_base + lane;
+        const uint32_t t_row = tmem + ((uint32_t)lane_base << 16);
+        const uint32_t part_row = map_rank(part0 + (uint32_t)(r * TS::PART_LD * 4), 0);
+        const uint32_t peer_full = map_rank(part_full, 0);
+        const uint32_t peer_free = map_rank(part_free, 1);
+        uint32_t tph = 0;
+        int i = 0;
+        for (int t = pair; t < p.n_tiles; t += n_pairs, ++i) {
+            if (!mbar_wait(tfull, tph, abort_f, p.err, p.wait_cycles)) break;
+            tc_fence_after();
+            const int m = t * BM + r;
+            bool ok = true;
+            if (rank == 1) {
+                // the previous tile's half has been read before this one overwrites it
+                if (i > 0 && !mbar_wait_cluster(part_free, (uint32_t)((i - 1) & 1), abort_f, p.err,
+                                                p.wait_cycles))
+                    ok = false;
+                if (ok) {
+                    for (int c = 0; c < BNT / 32; ++c) {
+                        float v[32];
+                        tmem_ld32(t_row + (uint32_t)(c * 32), v);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            st_cluster_v4(part_row + (uint32_t)((c * 32 + 4 * q) * 4), v[4 * q],
+                                          v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    }
+                    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(peer_full);
+                }
+            } else {
+                if (!mbar_wait_cluster(part_full, (uint32_t)(i & 1), abort_f, p.err, p.wait_cycles))
+                    ok = false;
+                if (ok) {
+                    const float* pr = part + (size_t)r * TS::PART_LD;
+                    float dummy_max = 0.f, dummy_sum = 0.f;
+                    int dummy_arg = 0;
+                    for (int c = 0; c < BNT / 32; ++c) {
+                        const int n = c * 32;
+                        if (n >= p.N) break;                 // warp-uniform
+                        float v[32];
+                        tmem_ld32(t_row + (uint32_t)n, v);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 o = *reinterpret_cast<const float4*>(pr + n + 4 * q);
+                            v[4 * q] += o.x; v[4 * q + 1] += o.y; v[4 * q + 2] += o.z; v[4 * q + 3] += o.w;
+                        }
+                        epilogue_chunk<EPI_SHRINK>(p, m, n, v, &dummy_max, &dummy_sum, &dummy_arg);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(peer_free);
+                }
+            }
+            if (!ok) break;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty);
+            tph ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();                         // every role of this CTA has left its loop
+    if (*abort_f && lane == 0) {
+        if (warp == 0) {
+            const int n = n_armed < STAGES ? n_armed : STAGES;
+            for (int k = 0; k < n; ++k) {
+                const int a = n_armed - 1 - k;
+                const uint32_t aph = (uint32_t)(a / STAGES) & 1u;
+                for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(full(a % STAGES), aph); ++it)
+                    __nanosleep(128);
+            }
+        } else if (warp == 1 && issued) {
+            tc_commit(drain);
+            for (uint32_t it = 0; it < WAIT_LIMIT && !mbar_try(drain, 0); ++it) __nanosleep(128);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                          // neither CTA leaves while the other may write to it
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BNT)
                      : "memory");
     }
 }
@@ -1278,6 +1548,23 @@ int launch_epi_w(int bnt, const CUtensorMap& a, const CUtensorMap& b, const CUte
         case 128: return launch_epi<EPI, 128>(a, b, a2, b2, p, st);
         default: return launch_epi<EPI, 256>(a, b, a2, b2, p, st);
     }
+}
+
+template <int BNT>
+int launch_shrink_pair(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p,
+                       cudaStream_t st) {
+    constexpr int smem = TileS<BNT>::SMEM_BYTES;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(shrink_pair_kernel<BNT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess)
+            return 1;
+        attr = true;
+    }
+    int pairs = num_sms() / 2;
+    if (p.n_tiles < pairs) pairs = p.n_tiles;
+    shrink_pair_kernel<BNT><<<2 * pairs, NUM_THREADS, smem, st>>>(a, b, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
 
 template <int EPI, bool F8, bool SPLIT = false>
@@ -1485,6 +1772,7 @@ int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
     p.M = g.N; p.N = g.M;
     p.kb_main = f8 ? (g.K + BK8 - 1) / BK8 : (g.K + BK - 1) / BK;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
+    p.k2_last_steps = g.K2 > 0 ? (g.K2 - (p.kb_ext - 1) * BK + 15) / 16 : BK / 16;
     // swapped sides: the weight rows' scales are the kernel's M side, the tokens' its N side
     p.a_scale = g.b_scale; p.b_scale = g.a_scale;
     p.n_m_blk = (g.N + BM - 1) / BM;
@@ -1628,6 +1916,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.kb_main = f8 ? (g.K + BK8 - 1) / BK8 : (g.K + BK - 1) / BK;
     p.a_scale = g.a_scale; p.b_scale = g.b_scale;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
+    p.k2_last_steps = g.K2 > 0 ? (g.K2 - (p.kb_ext - 1) * BK + 15) / 16 : BK / 16;
     p.n_m_blk = pair ? (g.M + BM2 - 1) / BM2 : (g.M + BM - 1) / BM;
     // Raster: the SM pairs walk M groups of 12 blocks of 256 rows, each sweeping every N
     // block, so a weight strip is fetched once per group while the group's A strips stay in
@@ -1650,6 +1939,11 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_error) != cudaSuccess) return 1;
     p.err = err;
     p.wait_cycles = g_wait_cycles;
+    if (g.epi == EPI_SHRINK && !g.ws && !f8 && g.K2 == 0 && bnt <= 128 && p.kb_main >= 2) {
+        // the bank shrink of a scoring batch: K split over a CTA pair so that every SM streams
+        // rows of x (chosen by N and K only, never by M)
+        return bnt == 64 ? launch_shrink_pair<64>(a, b, p, st) : launch_shrink_pair<128>(a, b, p, st);
+    }
     if (pair && g.ws && !f8 && g.N % 4 == 0 &&
         (g.epi == EPI_STORE || g.epi == EPI_STORE_RELU || g.epi == EPI_RESID ||
          g.epi == EPI_SWIGLU || g.epi == EPI_QKNR)) {

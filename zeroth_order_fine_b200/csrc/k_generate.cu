@@ -52,7 +52,8 @@ void launch_init_tensor(void* dst, uint64_t n, uint64_t key, float std_, float m
 // ---- directions ---------------------------------------------------------------------
 // One job per (target, factor).  Element e = i*r + c of the row-major [dim x r]
 // factor is written to dst[c * ld + i] (U: the transposed rows the shrink GEMM
-// reads) or dst[e] (V: row-major, kept for the window).
+// reads) or dst[e] (V: row-major, kept for the window); dst or its bf16 mirror
+// dst_bf may be null (bf16 models keep U in bf16 only).
 __global__ void __launch_bounds__(256) gen_factors_kernel(const GenJob* jobs, int n_jobs,
                                                           uint64_t run_seed, uint64_t step,
                                                           const uint64_t* step_dev,
@@ -75,7 +76,7 @@ __global__ void __launch_bounds__(256) gen_factors_kernel(const GenJob* jobs, in
             float v = z[h];
             if (apply_scale) v = __fmul_rn(v, scale);
             const uint64_t o = jb.transposed ? (e % jb.r) * (uint64_t)jb.ld + e / jb.r : e;
-            jb.dst[o] = v;
+            if (jb.dst) jb.dst[o] = v;
             if (jb.dst_bf) static_cast<__nv_bfloat16*>(jb.dst_bf)[o] = __float2bfloat16_rn(v);
         }
     }

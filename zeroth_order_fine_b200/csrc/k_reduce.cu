@@ -8,11 +8,15 @@
 //    order in fp64 with warp shuffles;
 //  * A_k <- A_k - lr c U_t for every target in one launch (the U-side
 //    accumulator of the lazy window, same page, "Memory-write reduction"),
-//    refused on the device when c is not finite.
+//    refused on the device when c is not finite.  U_t is regenerated from the
+//    counter stream rather than read, and while the slot's coefficients since
+//    it opened are known the slot is rebuilt from them rather than read, so a
+//    step writes the accumulator without reading it.
 #include <float.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "rng.cuh"
 
 namespace zo {
 
@@ -130,42 +134,60 @@ void launch_estimate(const double* sums, float eps, double* c, int* flag, cudaSt
     estimate_kernel<<<1, 1, 0, st>>>(sums, eps, c, flag);
 }
 
-// One launch over every target: blockIdx.y = target, float4 where aligned.
-__global__ void __launch_bounds__(256) bank_update_kernel(const UpdateJob* __restrict__ jobs,
-                                                          const double* __restrict__ c,
-                                                          const int* __restrict__ flag,
-                                                          float lr) {
-    if (*flag) return;                       // non-finite c: bank unchanged
+// One launch over every target: blockIdx.y = target, one thread per N(0,1) pair of U_t.
+__global__ void __launch_bounds__(256) bank_update_kernel(
+    const UpdateJob* __restrict__ jobs, const double* __restrict__ c, const int* __restrict__ flag,
+    float lr, uint64_t run_seed, uint64_t step, const uint64_t* __restrict__ step_dev, uint64_t nu,
+    float scale, int apply_scale, long long replay_from, float* __restrict__ coef_hist) {
     const UpdateJob jb = jobs[blockIdx.y];
-    const float coef = (float)((double)lr * *c);
-    const int n4 = jb.n >> 2;
-    float4* A4 = reinterpret_cast<float4*>(jb.A);
-    const float4* U4 = reinterpret_cast<const float4*>(jb.U);
-    __nv_bfloat162* B2 = static_cast<__nv_bfloat162*>(jb.A_bf);
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) {
-        float4 a = A4[i];
-        const float4 u = U4[i];
-        a.x -= coef * u.x; a.y -= coef * u.y; a.z -= coef * u.z; a.w -= coef * u.w;
-        A4[i] = a;
-        if (B2) {
-            B2[2 * i] = __floats2bfloat162_rn(a.x, a.y);
-            B2[2 * i + 1] = __floats2bfloat162_rn(a.z, a.w);
+    const uint64_t t = step_dev ? *step_dev : step;
+    const float coef_t = *flag ? 0.0f : (float)((double)lr * *c);   // non-finite c: refused
+    const bool replay = replay_from >= 0;
+    const uint64_t s0 = replay ? (uint64_t)replay_from : t;
+    if (replay && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        coef_hist[t - s0] = coef_t;                 // later steps replay it; read below only for s < t
+    const uint64_t n = (uint64_t)jb.dim * jb.r;
+    const uint64_t npairs = (n + 1) / 2;
+    for (uint64_t j = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; j < npairs;
+         j += (uint64_t)gridDim.x * blockDim.x) {
+        const uint64_t e0 = 2 * j, e1 = 2 * j + 1;
+        const bool has1 = e1 < n;
+        const uint64_t o0 = (e0 % jb.r) * (uint64_t)jb.ld + e0 / jb.r;
+        const uint64_t o1 = has1 ? (e1 % jb.r) * (uint64_t)jb.ld + e1 / jb.r : o0;
+        float a0 = replay ? 0.0f : jb.A[o0];
+        float a1 = (replay || !has1) ? 0.0f : jb.A[o1];
+        for (uint64_t s = s0; s <= t; ++s) {
+            const float cf = s < t ? coef_hist[s - s0] : coef_t;
+            float z0, z1;
+            normal_pair(factor_key(run_seed, s, nu, (uint32_t)jb.layer, (uint32_t)jb.matrix, 0), j,
+                        &z0, &z1);
+            if (apply_scale) {
+                z0 = __fmul_rn(z0, scale);
+                z1 = __fmul_rn(z1, scale);
+            }
+            a0 = __fmaf_rn(-cf, z0, a0);
+            a1 = __fmaf_rn(-cf, z1, a1);
         }
-    }
-    for (int i = (n4 << 2) + blockIdx.x * blockDim.x + threadIdx.x; i < jb.n;
-         i += gridDim.x * blockDim.x) {
-        jb.A[i] -= coef * jb.U[i];
-        if (jb.A_bf) static_cast<__nv_bfloat16*>(jb.A_bf)[i] = __float2bfloat16_rn(jb.A[i]);
+        jb.A[o0] = a0;
+        if (jb.A_bf) static_cast<__nv_bfloat16*>(jb.A_bf)[o0] = __float2bfloat16_rn(a0);
+        if (has1) {
+            jb.A[o1] = a1;
+            if (jb.A_bf) static_cast<__nv_bfloat16*>(jb.A_bf)[o1] = __float2bfloat16_rn(a1);
+        }
     }
 }
 
-void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_n, const double* c,
-                        const int* flag, float lr, cudaStream_t st) {
+void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_pairs, const double* c,
+                        const int* flag, float lr, uint64_t run_seed, uint64_t step,
+                        const uint64_t* step_dev, uint64_t nu, float scale, int apply_scale,
+                        long long replay_from, float* coef_hist, cudaStream_t st) {
     if (n_jobs == 0) return;
-    unsigned bx = cdiv(max_n / 4 + 1, 256);
-    if (bx > 32) bx = 32;
+    unsigned bx = cdiv(max_pairs, 256);
+    if (bx > 64) bx = 64;
+    if (bx == 0) bx = 1;
     dim3 grid(bx, n_jobs);
-    bank_update_kernel<<<grid, 256, 0, st>>>(jobs, c, flag, lr);
+    bank_update_kernel<<<grid, 256, 0, st>>>(jobs, c, flag, lr, run_seed, step, step_dev, nu, scale,
+                                             apply_scale, replay_from, coef_hist);
 }
 
 }  // namespace zo

@@ -9,7 +9,7 @@ enum ElemType : int { E_F32 = 0, E_BF16 = 1, E_FP8 = 2 };   // E_FP8: E4M3 bytes
 
 // ---- generator -------------------------------------------------------------------------
 struct GenJob {
-    float* dst;
+    float* dst;                 // fp32 factor, or null
     void* dst_bf;               // optional bf16 mirror written at the same positions
     int layer, matrix, which;   // which: 0 = U, 1 = V
     int dim, r;                 // factor is [dim x r]
@@ -206,9 +206,22 @@ void launch_objective_sums(const double* L_row, int B, double* sums, cudaStream_
 // c = sums[0] / sums[1] / (2 eps); flag = 1 if not finite (update refused).
 void launch_estimate(const double* sums, float eps, double* c, int* flag, cudaStream_t st);
 
-struct UpdateJob { float* A; const float* U; void* A_bf; int n; };
+// Bank update of every target's current slot, A <- A - coef_t U_t with coef_t = (float)(lr c)
+// (0 when flag is set: a refused update leaves A as it was).  U_t is regenerated from the
+// counter stream (key (run_seed, t, layer, matrix, U)), never read.  A is [r x ld] fp32, the
+// transposed rows of the [dim x r] factor (element (i, c) at A[c * ld + i]), with an optional
+// bf16 mirror at the same positions.
+//   replay_from < 0: read-modify-write of A.
+//   replay_from >= 0: A is not read.  It is rebuilt from zero by the slot's coefficients
+//     coef_s, s = replay_from .. t, kept in coef_hist[s - replay_from] (this step's written
+//     there): the same fused multiply-adds in the same order as the read-modify-write steps
+//     since the slot opened, so both give the same bits.
+// step_dev (may be null): read t from device memory instead of `step`.
+struct UpdateJob { float* A; void* A_bf; int layer, matrix, dim, r, ld; };
 void launch_to_bf16(const float* src, void* dst, size_t n, cudaStream_t st);
-void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_n, const double* c,
-                        const int* flag, float lr, cudaStream_t st);
+void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_pairs, const double* c,
+                        const int* flag, float lr, uint64_t run_seed, uint64_t step,
+                        const uint64_t* step_dev, uint64_t nu, float scale, int apply_scale,
+                        long long replay_from, float* coef_hist, cudaStream_t st);
 
 }  // namespace zo
