@@ -170,3 +170,28 @@ def test_bf16_mode_trajectory_close_to_fp32():
     a, b = r32.score(rows, tls), r16.score(rows, tls)
     # different weights (bf16-rounded), same model: objectives agree to bf16 level
     assert np.max(np.abs(a.L_plus - b.L_plus)) < 2e-2
+
+
+def test_trajectory_workload_discriminates_the_update_strength():
+    """The bf16 100-step trajectory check (2 % band) can tell a wrong update strength: on its
+    workload the oracle's loss moves by more than five times the band, and the oracle run
+    with half (or twice) the learning rate leaves the band."""
+    w = wl.TRAJ_TINY_BF16
+    weights = om.init_weights(w.shape, w.weight_seed)
+    batch = wl.make_batch(w)
+
+    def trajectory(lr):
+        run = zo.OracleRun(weights, w.run_seed, w.nu, w.rank, range(w.shape.n_layers),
+                           w.matrices, w.scale_mode)
+        out = []
+        for t in range(100):
+            run.plan(t, w.eps)
+            res = run.score(batch.prompts, batch.target_lens)
+            out.append(float(res.L_plus.mean() + res.L_minus.mean()) / 2)
+            run.step(lr)
+        return np.array(out)
+
+    ref = trajectory(w.lr)
+    assert abs(ref[-1] - ref[0]) / ref[0] >= 0.10
+    for wrong in (w.lr / 2, w.lr * 2):
+        assert np.max(np.abs(trajectory(wrong) - ref) / ref) > 0.025, wrong

@@ -143,6 +143,16 @@ WORKLOADS = {
 }
 
 
+# bf16 100-step trajectory workload: the tiny model in bf16 with the direction on all six
+# OPT matrices, eta = 2e-4 and eps = 1e-2.  100 steps move its loss by ~13 % (with q and v
+# alone it moves 2.5-7 % at any eta), and at eps = 1e-3 the bf16 rounding of L is comparable
+# to the paired difference 2 eps c, so two runs drift apart by several per cent.
+TRAJ_TINY_BF16 = dataclasses.replace(
+    WORKLOADS["tiny"], name="tiny-bf16-trajectory",
+    shape=dataclasses.replace(TINY, name="tiny-opt-bf16", dtype=DTYPE_BF16),
+    matrices=(MAT_Q, MAT_K, MAT_V, MAT_O, MAT_UP, MAT_DOWN), lr=2e-4, eps=1e-2)
+
+
 def shrink_shape(shape: ModelShape, n_layers: Optional[int] = None, **kw) -> ModelShape:
     """The same family at another size (used for full-width layer slices)."""
     fields = dataclasses.asdict(shape)
