@@ -400,6 +400,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sl2 = a.scale * 1.4426950408889634f;
         uint8_t* kbuf[2] = {g + 2 * BUF, g + 3 * BUF};
+        // epilogue of item ke: O / l of this thread's query row, once its last P V retired
+        auto store_item = [&](int ke, const Item& it, float l) -> bool {
+            const int os = ke & 1;
+            if (!wait_bar(o_full(os), (ke >> 1) & 1, abort_f, err)) return false;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                 (size_t)(it.start + it.q0 + row) * a.ld_out +
+                                                 (size_t)it.h * HD);
+            const bool store = row < it.nq;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                float v[32];
+                tmem_ld32(t_o(os) + lane_addr + cc * 32, v);     // warp-collective: every lane
+                if (store) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        o4[cc * 4 + k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
+                                                     pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
+                                                     pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
+                                                     pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) bar_arrive(o_free(os));
+            return true;
+        };
+        int pk = -1;                             // item whose output is still to be stored
+        Item pit;
+        float pl = 0.f;
         int gc = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
@@ -486,31 +517,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) bar_arrive(p_full(st));
             }
             if (!ok) break;
-            // epilogue: O / l of this thread's query row, once the item's last P V retired
-            if (!wait_bar(o_full(os), (k >> 1) & 1, abort_f, err)) { ok = false; break; }
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
-                                                 (size_t)(it.start + q) * a.ld_out +
-                                                 (size_t)it.h * HD);
-            const bool store = row < it.nq;
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-                float v[32];
-                tmem_ld32(t_o(os) + lane_addr + cc * 32, v);     // warp-collective: every lane
-                if (store) {
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4)
-                        o4[cc * 4 + k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
-                                                     pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
-                                                     pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
-                                                     pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
-                }
-            }
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) bar_arrive(o_free(os));
+            // the previous item's output goes out now, after this item's softmax: its P V ran
+            // meanwhile, so the wait below rarely stalls
+            if (pk >= 0 && !store_item(pk, pit, pl)) { ok = false; break; }
+            pk = k;
+            pit = it;
+            pl = l;
         }
+        if (ok && pk >= 0) store_item(pk, pit, pl);
     }
     __syncthreads();                             // every role has left its loop
     if (*abort_f && warp == 0 && lane == 0) {

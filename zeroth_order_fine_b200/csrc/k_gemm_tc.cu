@@ -95,8 +95,6 @@ struct TcParams {
     int ksplit, kbs;                        // split-K (SPLIT kernels): splits, main blocks each
     int* err;
     long long wait_cycles;                  // bound of every mbarrier wait (clock64 cycles)
-    int k2_last_steps;                      // 16-column MMA steps holding data in the last
-                                            // extension block (its tail is zero padding)
 };
 
 // ---- PTX wrappers ------------------------------------------------------------------
@@ -526,13 +524,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             tc_mma_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
                                       T1::IDESC_F8, (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
-                        // the last extension block stops after its last 16 columns of data
-                        const int nk = (i == n_kb - 1 && n_kb > n_main) ? p.k2_last_steps : BK / 16;
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
-                            if (kk < nk)
-                                tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
-                                       (i > 0 || kk > 0) ? 1u : 0u);
+                            tc_mma(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), T1::IDESC,
+                                   (i > 0 || kk > 0) ? 1u : 0u);
                         }
                     }
                     issued = true;
@@ -1120,13 +1115,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                             tc_mma_pair_f8(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
                                            kIdesc2F8, (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
-                        // the last extension block stops after its last 16 columns of data
-                        const int nk = (i == n_kb - 1 && n_kb > n_main) ? p.k2_last_steps : BK / 16;
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            if (kk < nk)
-                                tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
-                                            kIdesc2, (i > 0 || kk > 0) ? 1u : 0u);
+                            tc_mma_pair(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
+                                        kIdesc2, (i > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     tc_commit_pair(empty(s));       // stage free in both CTAs
@@ -1772,7 +1764,6 @@ int gemm_tc_swapped(const GemmArgs& g, cudaStream_t st) {
     p.M = g.N; p.N = g.M;
     p.kb_main = f8 ? (g.K + BK8 - 1) / BK8 : (g.K + BK - 1) / BK;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
-    p.k2_last_steps = g.K2 > 0 ? (g.K2 - (p.kb_ext - 1) * BK + 15) / 16 : BK / 16;
     // swapped sides: the weight rows' scales are the kernel's M side, the tokens' its N side
     p.a_scale = g.b_scale; p.b_scale = g.a_scale;
     p.n_m_blk = (g.N + BM - 1) / BM;
@@ -1916,7 +1907,6 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.kb_main = f8 ? (g.K + BK8 - 1) / BK8 : (g.K + BK - 1) / BK;
     p.a_scale = g.a_scale; p.b_scale = g.b_scale;
     p.kb_ext = g.K2 > 0 ? (g.K2 + BK - 1) / BK : 0;
-    p.k2_last_steps = g.K2 > 0 ? (g.K2 - (p.kb_ext - 1) * BK + 15) / 16 : BK / 16;
     p.n_m_blk = pair ? (g.M + BM2 - 1) / BM2 : (g.M + BM - 1) / BM;
     // Raster: the SM pairs walk M groups of 12 blocks of 256 rows, each sweeping every N
     // block, so a weight strip is fetched once per group while the group's A strips stay in
