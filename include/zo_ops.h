@@ -5,7 +5,8 @@
  * can be checked and timed on its own.  None of them allocates: every
  * buffer, including scratch ("workspace"), is the caller's device memory.
  * All are queued on `stream` (cudaStream_t, NULL = legacy default stream)
- * and return ZO_OK or a ZO_ERR_* code from zo.h.
+ * and return ZO_OK or a ZO_ERR_* code from zo.h.  After ZO_ERR_CUDA,
+ * zo_op_last_error() names what failed and the CUDA error.
  */
 #ifndef ZO_OPS_H
 #define ZO_OPS_H
@@ -200,6 +201,12 @@ int zo_op_lm_head_logprob_noalloc(const void* h, const void* E, const int32_t* t
  * kernel then stopped early and its output is invalid), -1 when the device
  * reported an error. */
 int zo_op_error_word(void);
+
+/* What the calling thread's last zo_op_* call that returned ZO_ERR_CUDA ran
+ * into: the step that failed and the CUDA error's name and text ("" before
+ * any failure).  The string is the library's, valid until that thread's next
+ * failing call. */
+const char* zo_op_last_error(void);
 
 #ifdef __cplusplus
 }

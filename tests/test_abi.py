@@ -112,3 +112,8 @@ def test_decode_linear_argument_checks_without_gpu(built_lib):
     assert call(p, p, p, 4, 256, 64, 0, 0, p, 4 * 256 - 1) == zo.ZO_ERR_ARG   # < one slice
     assert call(p, p, p, 4, 256, 60, 0, 0, p, 1 << 20) == zo.ZO_ERR_UNSUPPORTED  # K % 8
     assert call(p, p, p, 4, 258, 64, 0, 0, p, 1 << 20) == zo.ZO_ERR_UNSUPPORTED  # N % 4
+
+
+def test_op_error_text_is_empty_before_any_failure(built_lib):
+    built_lib.zo_op_last_error.restype = ctypes.c_char_p
+    assert built_lib.zo_op_last_error() == b""

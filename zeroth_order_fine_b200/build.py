@@ -1,7 +1,7 @@
 """Build libzo_b200.so in-tree for sm_100a (nvcc; no JIT, no torch extension).
 
 Each translation unit under csrc/ is compiled to an object under _build/
-(rebuilt only when it or a header changed) and linked into
+(rebuilt only when it or a header changed, earlier builds kept by content) and linked into
 zeroth_order_fine_b200/libzo_b200.so, which the Python binding loads.
 """
 from __future__ import annotations
@@ -56,9 +56,14 @@ def build(verbose: bool = False) -> str:
     hdr = _headers_digest()
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(lambda s: _compile(s, hdr, verbose), srcs))
-    newest = max(os.path.getmtime(o) for o in objs)
-    if os.path.exists(OUT) and os.path.getmtime(OUT) >= newest:
-        return OUT
+    # relink whenever the set of objects differs from the one the library was linked from
+    # (going back to an earlier source picks up its cached, older object)
+    stamp = os.path.join(BUILD, os.path.basename(OUT) + ".objects")
+    linked = "\n".join(os.path.basename(o) for o in objs) + "\n"
+    if os.path.exists(OUT) and os.path.exists(stamp):
+        with open(stamp) as fh:
+            if fh.read() == linked:
+                return OUT
     cmd = [NVCC] + ARCH + ["-shared", "-o", OUT + ".tmp"] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
     if verbose:
         print(" ".join(cmd), flush=True)
@@ -66,6 +71,8 @@ def build(verbose: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(OUT + ".tmp", OUT)
+    with open(stamp, "w") as fh:
+        fh.write(linked)
     return OUT
 
 

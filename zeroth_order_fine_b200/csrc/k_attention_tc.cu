@@ -32,9 +32,10 @@ namespace {
 constexpr int TQ = 128, TK = 128, HD = 128;
 constexpr int ATOM = TQ * 128;                  // bytes of one 64-column swizzle atom block
 constexpr int BUF = 2 * ATOM;                   // one [128 x 128] bf16 operand
-// Q[2] K[2] V[2] buffers, then 19 mbarriers, the TMEM base and the abort flag
-constexpr int SMEM = 6 * BUF + 1024 + 256;
-constexpr int NTHREADS = 192;
+// Q[3] K[2] V[2] buffers, then 23 mbarriers, the TMEM base and the abort flag
+constexpr int SMEM = 7 * BUF + 1024 + 256;
+constexpr int NTHREADS = 224;                   // Q/K producer, MMA issuer, 4 softmax warps,
+                                                // V producer
 constexpr long long WAIT_CYCLES = 4000000000ll;
 constexpr uint32_t DRAIN_POLLS = 1u << 24;      // drain polls (with back-off) after an abort
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TK >> 3) << 17) |
@@ -196,20 +197,69 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, ui
 struct Item {
     int start, len, q0, nq, kend, n_chunks, h, kvh;
 };
-__device__ __forceinline__ Item get_item(const AttnArgs& a, int i) {
+__device__ __forceinline__ Item make_item(const AttnArgs& a, int i, int tile, int start, int end) {
     Item it;
-    const int tile = a.tiles[i / a.H];
-    const int row = tile >> 16, qt = tile & 0xFFFF;
+    const int qt = tile & 0xFFFF;
     it.h = i % a.H;
     it.kvh = it.h / (a.H / a.Hkv);
-    it.start = a.cu_seqlens[row];
-    it.len = a.cu_seqlens[row + 1] - it.start;
+    it.start = start;
+    it.len = end - start;
     it.q0 = qt * TQ;
     it.nq = min(TQ, it.len - it.q0);
     it.kend = min(it.len, it.q0 + TQ);
     it.n_chunks = (it.kend + TK - 1) / TK;
     return it;
 }
+__device__ __forceinline__ Item get_item(const AttnArgs& a, int i) {
+    const int tile = a.tiles[i / a.H];
+    const int row = tile >> 16;
+    return make_item(a, i, tile, a.cu_seqlens[row], a.cu_seqlens[row + 1]);
+}
+
+// The items of this CTA in order (k-th: blockIdx.x + k * gridDim.x), with their metadata
+// fetched two items ahead: the tile of item k + 2 and the row offsets of item k + 1 are
+// loaded while item k is being worked on, so no role waits on the dependent loads
+// (tile, then the row's offsets) when it moves to its next item.
+struct ItemFeed {
+    const int* tiles;
+    const int* cu;
+    AttnArgs shape;             // only H and Hkv are read (make_item)
+    int n_items;
+    int k;                      // index of cur among this CTA's items
+    bool has;                   // cur exists
+    Item cur;
+    int tile1, s1, e1;          // item k + 1: tile and row offsets (valid when k + 1 exists)
+    int tile2;                  // item k + 2: tile
+    __device__ __forceinline__ int idx(int kk) const { return blockIdx.x + kk * gridDim.x; }
+    __device__ __forceinline__ void init(const AttnArgs& args, int n) {
+        tiles = args.tiles;
+        cu = args.cu_seqlens;
+        shape.H = args.H;
+        shape.Hkv = args.Hkv;
+        n_items = n;
+        k = 0;
+        has = idx(0) < n;
+        if (has) cur = get_item(args, idx(0));
+        tile1 = s1 = e1 = tile2 = 0;
+        if (idx(1) < n) {
+            tile1 = tiles[idx(1) / shape.H];
+            s1 = cu[tile1 >> 16];
+            e1 = cu[(tile1 >> 16) + 1];
+        }
+        if (idx(2) < n) tile2 = tiles[idx(2) / shape.H];
+    }
+    __device__ __forceinline__ void advance() {
+        ++k;
+        has = idx(k) < n_items;
+        if (has) cur = make_item(shape, idx(k), tile1, s1, e1);   // loaded an item ago
+        if (idx(k + 1) < n_items) {
+            tile1 = tile2;
+            s1 = cu[tile1 >> 16];                                  // used at the next advance
+            e1 = cu[(tile1 >> 16) + 1];
+        }
+        if (idx(k + 2) < n_items) tile2 = tiles[idx(k + 2) / shape.H];
+    }
+};
 
 __device__ __forceinline__ float ex2_ftz(float x) {
     float y;
@@ -243,22 +293,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* g = smem_raw + (base - raw);
-    auto Qb = [&](int i) { return base + (uint32_t)(i * BUF); };
-    auto Kb = [&](int i) { return base + (uint32_t)((2 + i) * BUF); };
-    auto Vb = [&](int i) { return base + (uint32_t)((4 + i) * BUF); };
-    const uint32_t bar0 = base + 6 * BUF;
+    auto Qb = [&](int i) { return base + (uint32_t)(i * BUF); };          // i < 3
+    auto Kb = [&](int i) { return base + (uint32_t)((3 + i) * BUF); };
+    auto Vb = [&](int i) { return base + (uint32_t)((5 + i) * BUF); };
+    const uint32_t bar0 = base + 7 * BUF;
     auto q_full = [&](int i) { return bar0 + 8u * (0 + i); };
-    auto q_empty = [&](int i) { return bar0 + 8u * (2 + i); };
-    auto k_full = [&](int i) { return bar0 + 8u * (4 + i); };
-    auto v_full = [&](int i) { return bar0 + 8u * (6 + i); };
-    auto kv_empty = [&](int i) { return bar0 + 8u * (8 + i); };
-    auto s_full = [&](int i) { return bar0 + 8u * (10 + i); };
-    auto p_full = [&](int i) { return bar0 + 8u * (12 + i); };
-    auto o_full = [&](int i) { return bar0 + 8u * (14 + i); };
-    auto o_free = [&](int i) { return bar0 + 8u * (16 + i); };
-    const uint32_t drain = bar0 + 8u * 18;
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 6 * BUF + 160);
-    volatile int* abort_f = reinterpret_cast<volatile int*>(g + 6 * BUF + 168);
+    auto q_empty = [&](int i) { return bar0 + 8u * (3 + i); };
+    auto k_full = [&](int i) { return bar0 + 8u * (6 + i); };
+    auto v_full = [&](int i) { return bar0 + 8u * (8 + i); };
+    auto k_empty = [&](int i) { return bar0 + 8u * (10 + i); };
+    auto v_empty = [&](int i) { return bar0 + 8u * (12 + i); };
+    auto s_full = [&](int i) { return bar0 + 8u * (14 + i); };
+    auto p_full = [&](int i) { return bar0 + 8u * (16 + i); };
+    auto o_full = [&](int i) { return bar0 + 8u * (18 + i); };
+    auto o_free = [&](int i) { return bar0 + 8u * (20 + i); };
+    const uint32_t drain = bar0 + 8u * 22;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 7 * BUF + 192);
+    volatile int* abort_f = reinterpret_cast<volatile int*>(g + 7 * BUF + 200);
+    // P of a chunk goes over its K buffer, except for an item's last chunk: over the item's
+    // Q buffer, whose last reader (that chunk's S) has retired by then.  So the K buffer of an
+    // item's last chunk is free as soon as its S retires, and the next K load overlaps the
+    // softmax instead of waiting for P V.
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = a.n_tiles * a.H;
@@ -266,12 +321,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int* err = &g_attn_error;
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 3; ++i) {
             bar_init(q_full(i), 1);
             bar_init(q_empty(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             bar_init(k_full(i), 1);
             bar_init(v_full(i), 1);
-            bar_init(kv_empty(i), 1);
+            bar_init(k_empty(i), 1);
+            bar_init(v_empty(i), 1);
             bar_init(s_full(i), 1);
             bar_init(p_full(i), 4);            // one arrival per softmax warp
             bar_init(o_full(i), 1);
@@ -295,34 +353,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     auto t_s = [&](int i) { return tmem + (uint32_t)(i * 128); };         // S buffers: cols 0, 128
     auto t_o = [&](int i) { return tmem + (uint32_t)(256 + i * 128); };   // O buffers: 256, 384
 
-    int gq = 0, gcl = 0;                         // producer: Q loads and K/V chunk loads issued
-    if (warp == 0) {
-        // ---------------- TMA producer ----------------
+    int gq = 0, gcl = 0;                         // producers: Q loads, K (warp 0) or V (warp 6)
+                                                 // chunk loads issued
+    if (warp == 0 || warp == 6) {
+        // ---------------- TMA producers: Q and K (warp 0), V (warp 6) ----------------
         if (lane == 0) {
+            const bool vk = warp == 6;
             int& gc = gcl;
             bool ok = true;
-            for (int k = 0; ok; ++k) {
-                const int idx = blockIdx.x + k * gridDim.x;
-                if (idx >= n_items) break;
-                const Item it = get_item(a, idx);
-                const int qs = k & 1;
-                if (!wait_bar(q_empty(qs), ((k >> 1) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
-                bar_expect_tx(q_full(qs), BUF);
-                for (int half = 0; half < 2; ++half)
-                    tma_box(Qb(qs) + half * ATOM, &tm, q_full(qs), it.h * HD + half * 64,
-                            it.start + it.q0);
-                ++gq;
-                const int kcol = q_dim + it.kvh * HD, vcol = q_dim + kv_dim + it.kvh * HD;
+            ItemFeed feed;
+            feed.init(a, n_items);
+            for (int k = 0; ok && feed.has; ++k, feed.advance()) {
+                const Item it = feed.cur;
+                if (!vk) {
+                    const int qs = k % 3;
+                    if (!wait_bar(q_empty(qs), ((k / 3) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
+                    bar_expect_tx(q_full(qs), BUF);
+                    for (int half = 0; half < 2; ++half)
+                        tma_box(Qb(qs) + half * ATOM, &tm, q_full(qs), it.h * HD + half * 64,
+                                it.start + it.q0);
+                    ++gq;
+                }
+                const int col = vk ? q_dim + kv_dim + it.kvh * HD : q_dim + it.kvh * HD;
                 for (int c = 0; c < it.n_chunks; ++c) {
                     const int st = gc & 1;
-                    if (!wait_bar(kv_empty(st), ((gc >> 1) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
-                    const int r0 = it.start + c * TK;
-                    bar_expect_tx(k_full(st), BUF);
+                    const uint32_t e = vk ? v_empty(st) : k_empty(st);
+                    const uint32_t f = vk ? v_full(st) : k_full(st);
+                    if (!wait_bar(e, ((gc >> 1) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
+                    bar_expect_tx(f, BUF);
                     for (int half = 0; half < 2; ++half)
-                        tma_box(Kb(st) + half * ATOM, &tm, k_full(st), kcol + half * 64, r0);
-                    bar_expect_tx(v_full(st), BUF);
-                    for (int half = 0; half < 2; ++half)
-                        tma_box(Vb(st) + half * ATOM, &tm, v_full(st), vcol + half * 64, r0);
+                        tma_box((vk ? Vb(st) : Kb(st)) + half * ATOM, &tm, f, col + half * 64,
+                                it.start + c * TK);
                     ++gc;
                 }
             }
@@ -334,44 +395,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // gs - 2, whose P (so its S was read) arrived before P V of gs - 2 was issued
             int sk = 0, sc = 0, gs = 0;          // next S: item counter, chunk, global chunk
             int pk = 0, pc = 0, gp = 0;          // next P V
-            Item s_it, p_it;
-            bool s_more = blockIdx.x < n_items, p_more = s_more;
-            if (s_more) { s_it = get_item(a, blockIdx.x); p_it = s_it; }
+            ItemFeed s_feed, p_feed;             // the items of the next S and the next P V
+            s_feed.init(a, n_items);
+            p_feed.init(a, n_items);
+            bool s_more = s_feed.has, p_more = p_feed.has;
             bool ok = true, issued = false;
             long long t0 = clock64();
             while (p_more && ok) {
                 bool progress = false;
-                if (s_more && gs <= gp + 1 && (sc > 0 || bar_test(q_full(sk & 1), (sk >> 1) & 1)) &&
+                if (s_more && gs <= gp + 1 && (sc > 0 || bar_test(q_full(sk % 3), (sk / 3) & 1)) &&
                     bar_test(k_full(gs & 1), (gs >> 1) & 1)) {
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                    mma_qk(t_s(gs & 1), Qb(sk & 1), Kb(gs & 1));
+                    mma_qk(t_s(gs & 1), Qb(sk % 3), Kb(gs & 1));
                     tc_commit(s_full(gs & 1));
+                    // the item's last chunk keeps its P in the Q buffer: its K is free now
+                    if (sc == s_feed.cur.n_chunks - 1) tc_commit(k_empty(gs & 1));
                     issued = progress = true;
                     ++gs;
-                    if (++sc == s_it.n_chunks) {
+                    if (++sc == s_feed.cur.n_chunks) {
                         sc = 0;
                         ++sk;
-                        const int idx = blockIdx.x + sk * gridDim.x;
-                        s_more = idx < n_items;
-                        if (s_more) s_it = get_item(a, idx);
+                        s_feed.advance();
+                        s_more = s_feed.has;
                     }
                 }
                 if (gp < gs && bar_test(p_full(gp & 1), (gp >> 1) & 1) &&
                     bar_test(v_full(gp & 1), (gp >> 1) & 1) &&
                     (pc > 0 || bar_test(o_free(pk & 1), ((pk >> 1) & 1) ^ 1u))) {
+                    const bool last = pc == p_feed.cur.n_chunks - 1;
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                    mma_pv(t_o(pk & 1), Kb(gp & 1), Vb(gp & 1), pc > 0);
-                    tc_commit(kv_empty(gp & 1));         // K/P and V of the chunk are free
+                    mma_pv(t_o(pk & 1), last ? Qb(pk % 3) : Kb(gp & 1), Vb(gp & 1), pc > 0);
+                    tc_commit(v_empty(gp & 1));          // V of the chunk is free
+                    if (!last) tc_commit(k_empty(gp & 1));   // and its K buffer (held P)
                     issued = progress = true;
                     ++gp;
-                    if (++pc == p_it.n_chunks) {
+                    if (++pc == p_feed.cur.n_chunks) {
                         tc_commit(o_full(pk & 1));       // the item's output is complete
-                        tc_commit(q_empty(pk & 1));      // and its Q buffer free
+                        tc_commit(q_empty(pk % 3));      // and its Q buffer (P) free
                         pc = 0;
                         ++pk;
-                        const int idx = blockIdx.x + pk * gridDim.x;
-                        p_more = idx < n_items;
-                        if (p_more) p_it = get_item(a, idx);
+                        p_feed.advance();
+                        p_more = p_feed.has;
                     }
                 }
                 if (progress) {
@@ -399,7 +463,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int row = wq * 32 + lane;          // query row of the tile = TMEM lane
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sl2 = a.scale * 1.4426950408889634f;
-        uint8_t* kbuf[2] = {g + 2 * BUF, g + 3 * BUF};
         // epilogue of item ke: O / l of this thread's query row, once its last P V retired
         auto store_item = [&](int ke, const Item& it, float l) -> bool {
             const int os = ke & 1;
@@ -433,15 +496,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float pl = 0.f;
         int gc = 0;
         bool ok = true;
-        for (int k = 0; ok; ++k) {
-            const int idx = blockIdx.x + k * gridDim.x;
-            if (idx >= n_items) break;
-            const Item it = get_item(a, idx);
+        ItemFeed feed;
+        feed.init(a, n_items);
+        for (int k = 0; ok && feed.has; ++k, feed.advance()) {
+            const Item it = feed.cur;
             const int q = it.q0 + row;
             const int os = k & 1;
             float m = -FLT_MAX, l = 0.f;
             for (int c = 0; c < it.n_chunks; ++c, ++gc) {
                 const int st = gc & 1;
+                // P over the chunk's K buffer, or over the item's Q buffer for its last chunk
+                uint8_t* pbuf = c == it.n_chunks - 1 ? g + (k % 3) * BUF : g + (3 + st) * BUF;
                 if (!wait_bar(s_full(st), (gc >> 1) & 1, abort_f, err)) { ok = false; break; }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const int c0 = c * TK;
@@ -453,7 +518,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const bool warp_live = it.q0 + wq * 32 < it.len;
                 const int ncc = (!warp_live || wlim <= 0) ? 0 : min(4, (wlim + 31) >> 5);
                 float sv[4][32];
-                float cmax = -FLT_MAX;
+                // four running maxima: short dependency chains
+                float cm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     if (cc < ncc) {
@@ -461,16 +527,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             sv[cc][j] = (cc * 32 + j < lim) ? sv[cc][j] : -FLT_MAX;
-                            cmax = fmaxf(cmax, sv[cc][j]);
+                            cm[j & 3] = fmaxf(cm[j & 3], sv[cc][j]);
                         }
                     }
                 }
+                const float cmax = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
                 const float m_new = fmaxf(m, cmax);
                 // rows whose every key so far is masked keep m = -FLT_MAX and add nothing
                 const float alpha = (m > -FLT_MAX) ? exp2f((m - m_new) * sl2) : 0.f;
                 // masked scores are -FLT_MAX, so exp2(s*sl2 - ms) underflows to exactly 0
                 const float ms = (m_new > -FLT_MAX) ? m_new * sl2 : 0.f;
-                float cs0 = 0.f, cs1 = 0.f;
+                // eight running sums, added in a fixed tree: short dependency chains
+                float cs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     uint32_t w[16];
@@ -479,8 +547,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         for (int j = 0; j < 32; j += 2) {
                             const float p0 = ex2_ftz(fmaf(sv[cc][j], sl2, -ms));
                             const float p1 = ex2_ftz(fmaf(sv[cc][j + 1], sl2, -ms));
-                            cs0 += p0;
-                            cs1 += p1;
+                            cs[j & 7] += p0;
+                            cs[(j + 1) & 7] += p1;
                             w[j / 2] = pack_bf2(p0, p1);
                         }
                     } else {
@@ -489,16 +557,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                        *reinterpret_cast<uint4*>(kbuf[st] + sw_off(row, cc * 4 + k4)) =
+                        *reinterpret_cast<uint4*>(pbuf + sw_off(row, cc * 4 + k4)) =
                             make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
                 }
-                l = l * alpha + (cs0 + cs1);
+                l = l * alpha + (((cs[0] + cs[1]) + (cs[2] + cs[3])) + ((cs[4] + cs[5]) + (cs[6] + cs[7])));
                 m = m_new;
                 if (c > 0) {
                     // the running output stays in TMEM: once the previous chunk's P V has
                     // retired, rescale it by exp(m_old - m_new); this chunk's P V adds on top
                     const int pv = gc - 1;
-                    if (!wait_bar(kv_empty(pv & 1), (pv >> 1) & 1, abort_f, err)) { ok = false; break; }
+                    if (!wait_bar(v_empty(pv & 1), (pv >> 1) & 1, abort_f, err)) { ok = false; break; }
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll 1
                     for (int cc = 0; cc < 4; ++cc) {
@@ -527,14 +595,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok && pk >= 0) store_item(pk, pit, pl);
     }
     __syncthreads();                             // every role has left its loop
-    if (*abort_f && warp == 0 && lane == 0) {
+    if (*abort_f && (warp == 0 || warp == 6) && lane == 0) {
         // an aborted CTA lets every copy still in flight land before its shared memory goes
-        // away: the two newest loads of each kind (older ones were consumed, so had landed)
-        for (int i = gq - 1; i >= 0 && i >= gq - 2; --i) drain_bar(q_full(i & 1), (i >> 1) & 1);
-        for (int i = gcl - 1; i >= 0 && i >= gcl - 2; --i) {
-            drain_bar(k_full(i & 1), (i >> 1) & 1);
-            drain_bar(v_full(i & 1), (i >> 1) & 1);
-        }
+        // away: the newest loads of each kind (older ones were consumed, so had landed)
+        if (warp == 0)
+            for (int i = gq - 1; i >= 0 && i >= gq - 3; --i) drain_bar(q_full(i % 3), (i / 3) & 1);
+        for (int i = gcl - 1; i >= 0 && i >= gcl - 2; --i)
+            drain_bar(warp == 0 ? k_full(i & 1) : v_full(i & 1), (i >> 1) & 1);
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -572,11 +639,11 @@ bool attention_tc_supported(const AttnArgs& a) {
 
 bool launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
     if (a.n_tiles == 0 || a.n_tokens <= 0) return true;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-        attr = true;
-    }
+    static cudaError_t attr = cudaErrorNotReady;
+    if (attr == cudaErrorNotReady)
+        attr = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    SMEM);
+    if (attr != cudaSuccess) return false;
     // one map over the packed [T x ld_qkv] q|k|v rows: 64-column x 128-row boxes,
     // 128-byte swizzle, rows past T read as zero
     CUtensorMap tm;

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstring>
 #include <algorithm>
+#include <string>
 #include <vector>
 
 #include "../../include/zo.h"
@@ -13,6 +14,23 @@
 using namespace zo;
 
 namespace {
+thread_local std::string t_op_err;
+
+// ZO_OK, or ZO_ERR_CUDA with the CUDA error (a failed launch, or an earlier asynchronous
+// error the launch ran into) kept for zo_op_last_error
+int op_status() {
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return ZO_OK;
+    t_op_err = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
+    return ZO_ERR_CUDA;
+}
+int op_fail(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    t_op_err = what;
+    if (e != cudaSuccess) t_op_err += std::string(" (") + cudaGetErrorName(e) + ")";
+    return ZO_ERR_CUDA;
+}
+
 bool use_tc(int32_t impl, int dtype) {
     if (impl == ZO_IMPL_CUDA_CORES) return false;
     return dtype == ZO_DTYPE_BF16;
@@ -27,7 +45,7 @@ int zo_op_quantize_rows_e4m3(const void* x, int32_t dtype, int32_t rows, int32_t
     if (dtype != ZO_DTYPE_FP32 && dtype != ZO_DTYPE_BF16) return ZO_ERR_ARG;
     launch_quant_rows_e4m3(x, dtype == ZO_DTYPE_BF16 ? E_BF16 : E_F32, rows, cols, (size_t)cols, q,
                            (size_t)cols, scale, static_cast<cudaStream_t>(stream));
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    return op_status();
 }
 
 int zo_op_linear_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
@@ -46,8 +64,8 @@ int zo_op_linear_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, cons
     g.C = y; g.ldc = N; g.c_type = E_BF16;
     if (M == 0) return ZO_OK;
     if (!gemm_tc_supported(g)) return ZO_ERR_UNSUPPORTED;
-    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return ZO_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return op_fail("tensor-core GEMM launch failed");
+    return op_status();
 }
 
 int zo_op_linear(const void* x, const void* W, const float* bias, void* y, int32_t M, int32_t N,
@@ -70,15 +88,15 @@ int zo_op_linear(const void* x, const void* W, const float* bias, void* y, int32
     if (M == 0) return ZO_OK;
     if (use_tc(impl, dtype)) {
         if (gemm_tc_supported(g)) {
-            if (gemm_tc(g, st)) return ZO_ERR_CUDA;
-            return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+            if (gemm_tc(g, st)) return op_fail("tensor-core GEMM launch failed");
+            return op_status();
         }
         if (impl == ZO_IMPL_TENSOR_CORES) return ZO_ERR_UNSUPPORTED;
     } else if (impl == ZO_IMPL_TENSOR_CORES) {
         return ZO_ERR_UNSUPPORTED;
     }
     gemm_simt(g, st);
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    return op_status();
 }
 
 int zo_op_linear_decode(const void* x, const void* W, const float* bias, void* y, int32_t M,
@@ -100,8 +118,8 @@ int zo_op_linear_decode(const void* x, const void* W, const float* bias, void* y
     g.C = y; g.ldc = N; g.c_type = accumulate ? E_F32 : E_BF16;
     g.ws = ws; g.ws_floats = ws_floats;
     if (!gemm_tc_supported(g)) return ZO_ERR_UNSUPPORTED;
-    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return ZO_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return op_fail("tensor-core GEMM launch failed");
+    return op_status();
 }
 
 size_t zo_op_lm_head_workspace(int32_t n_rows, int32_t vocab, int32_t impl) {
@@ -140,12 +158,12 @@ int zo_op_lm_head_logprob(const void* h, const void* E, const int32_t* targets, 
     if (impl == ZO_IMPL_TENSOR_CORES && !tc) return ZO_ERR_UNSUPPORTED;
     g.n_col_tiles = tc ? gemm_tc_col_tiles(vocab) : tiles;
     if (tc) {
-        if (gemm_tc(g, st)) return ZO_ERR_CUDA;
+        if (gemm_tc(g, st)) return op_fail("tensor-core GEMM launch failed");
     } else {
         gemm_simt(g, st);
     }
     launch_lse_merge(pmax, psum, tgt, n_rows, g.n_col_tiles, logprob, st);
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    return op_status();
 }
 
 int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t n_rows,
@@ -179,9 +197,9 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     int* w = static_cast<int*>(workspace);
     meta.insert(meta.end(), tiles.begin(), tiles.end());
     if (cudaMemcpyAsync(w, meta.data(), meta.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
-        return ZO_ERR_CUDA;
+        return op_fail("copy of the row metadata failed");
     // the host vector must outlive the copy
-    if (cudaStreamSynchronize(st) != cudaSuccess) return ZO_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return op_fail("stream synchronisation failed");
     AttnArgs a;
     memset(&a, 0, sizeof(a));
     a.qkv = qkv; a.ld_qkv = (n_heads + 2 * n_kv_heads) * head_dim;
@@ -194,13 +212,13 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     a.scale = (float)(1.0 / std::sqrt((double)head_dim));
     a.n_tokens = meta[n_rows];
     if (tc && attention_tc_supported(a)) {
-        if (!launch_attention_tc(a, st)) return ZO_ERR_CUDA;
+        if (!launch_attention_tc(a, st)) return op_fail("tensor-core attention setup failed");
     } else if (impl == ZO_IMPL_TENSOR_CORES) {
         return ZO_ERR_UNSUPPORTED;
     } else {
         launch_attention(a, st);
     }
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    return op_status();
 }
 
 int zo_op_linear_ext(const void* x, const void* W, const float* bias, const void* x2,
@@ -245,8 +263,8 @@ int zo_op_linear_ext(const void* x, const void* W, const float* bias, const void
     g.C = y; g.ldc = ldy;
     if (M == 0) return ZO_OK;
     if (!gemm_tc_supported(g)) return ZO_ERR_UNSUPPORTED;
-    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return ZO_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    if (gemm_tc(g, static_cast<cudaStream_t>(stream))) return op_fail("tensor-core GEMM launch failed");
+    return op_status();
 }
 
 int zo_op_rope_table(float* cos_t, float* sin_t, int32_t max_pos, int32_t head_dim, double theta,
@@ -254,7 +272,7 @@ int zo_op_rope_table(float* cos_t, float* sin_t, int32_t max_pos, int32_t head_d
     if (!cos_t || !sin_t || max_pos <= 0 || head_dim <= 0 || head_dim % 2 || !(theta > 0.0))
         return ZO_ERR_ARG;
     launch_rope_table(cos_t, sin_t, max_pos, head_dim, theta, static_cast<cudaStream_t>(stream));
-    return cudaGetLastError() == cudaSuccess ? ZO_OK : ZO_ERR_CUDA;
+    return op_status();
 }
 
 int64_t zo_op_set_wait_limit(int64_t cycles) {
@@ -270,5 +288,7 @@ int zo_op_error_word(void) {
     if (v < 0 || w < 0) return -1;
     return v | w;
 }
+
+const char* zo_op_last_error(void) { return t_op_err.c_str(); }
 
 }  // extern "C"

@@ -100,6 +100,7 @@ _SIGS = {
                             ctypes.POINTER(zo_options), ctypes.POINTER(c_void_p)]),
     "zo_destroy": (None, [c_void_p]),
     "zo_last_error": (ctypes.c_char_p, [c_void_p]),
+    "zo_op_last_error": (ctypes.c_char_p, []),
     "zo_probe_plan": (c_int32, [c_void_p, c_uint64, c_int32, ctypes.c_float,
                                 ctypes.POINTER(zo_targets), ctypes.POINTER(c_void_p)]),
     "zo_score": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -188,6 +189,12 @@ def _stream(stream=None) -> int:
 def _check(rc: int, handle=None) -> None:
     if rc != ZO_OK:
         msg = lib().zo_last_error(handle)
+        raise ZoError(rc, msg.decode() if msg else "")
+
+
+def _check_op(rc: int) -> None:
+    if rc != ZO_OK:
+        msg = lib().zo_op_last_error() if rc == ZO_ERR_CUDA else b""
         raise ZoError(rc, msg.decode() if msg else "")
 
 
@@ -454,7 +461,7 @@ def zo_op_linear(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] 
     dtype = wl.DTYPE_BF16 if x.dtype == torch.bfloat16 else wl.DTYPE_FP32
     if out is None:
         out = torch.empty(M, N, dtype=torch.float32 if accumulate else x.dtype, device=x.device)
-    _check(lib().zo_op_linear(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, dtype, act,
+    _check_op(lib().zo_op_linear(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, dtype, act,
                               int(accumulate), impl, _stream()))
     return out
 
@@ -469,7 +476,7 @@ def zo_op_linear_decode(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.T
         out = torch.empty(M, N, dtype=torch.float32 if accumulate else x.dtype, device=x.device)
     if ws is None:
         ws = torch.empty(max(1, 16 * M * N), dtype=torch.float32, device=x.device)
-    _check(lib().zo_op_linear_decode(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, act,
+    _check_op(lib().zo_op_linear_decode(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, act,
                                      int(accumulate), _ptr(ws), ws.numel(), _stream()))
     return out
 
@@ -497,7 +504,7 @@ def zo_op_linear_ext(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tens
         args = zo_qk_norm_rope_args(_ptr(qk["tok_pos"]), _ptr(qk["q_norm"]), _ptr(qk["k_norm"]),
                                     _ptr(qk["rope_cos"]), _ptr(qk["rope_sin"]), qk["eps"],
                                     qk["n_q_heads"], qk["n_kv_heads"])
-    _check(lib().zo_op_linear_ext(_ptr(x), _ptr(W), _ptr(bias), _ptr(x2), _ptr(W2), K2, _ptr(out),
+    _check_op(lib().zo_op_linear_ext(_ptr(x), _ptr(W), _ptr(bias), _ptr(x2), _ptr(W2), K2, _ptr(out),
                                   out.stride(0), M, N, K, epi,
                                   ctypes.byref(args) if args is not None else None, _stream()))
     return out
@@ -507,7 +514,7 @@ def zo_op_rope_table(max_pos: int, head_dim: int, theta: float, device="cuda"):
     """(cos, sin) rotary tables [max_pos x head_dim/2] as zo_create builds them."""
     c = torch.empty(max_pos, head_dim // 2, dtype=torch.float32, device=device)
     s = torch.empty(max_pos, head_dim // 2, dtype=torch.float32, device=device)
-    _check(lib().zo_op_rope_table(_ptr(c), _ptr(s), max_pos, head_dim, theta, _stream()))
+    _check_op(lib().zo_op_rope_table(_ptr(c), _ptr(s), max_pos, head_dim, theta, _stream()))
     return c, s
 
 
@@ -523,7 +530,7 @@ def zo_op_quantize_rows_e4m3(x: torch.Tensor):
     dtype = wl.DTYPE_BF16 if x.dtype == torch.bfloat16 else wl.DTYPE_FP32
     q = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
     sc = torch.empty(rows, dtype=torch.float32, device=x.device)
-    _check(lib().zo_op_quantize_rows_e4m3(_ptr(x), dtype, rows, cols, _ptr(q), _ptr(sc),
+    _check_op(lib().zo_op_quantize_rows_e4m3(_ptr(x), dtype, rows, cols, _ptr(q), _ptr(sc),
                                           _stream()))
     return q, sc
 
@@ -533,7 +540,7 @@ def zo_op_linear_fp8(xq: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: t
     M, K = xq.shape
     N = wq.shape[0]
     y = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
-    _check(lib().zo_op_linear_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y),
+    _check_op(lib().zo_op_linear_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y),
                                   M, N, K, act, _stream()))
     return y
 
@@ -546,7 +553,7 @@ def zo_op_lm_head_logprob(h: torch.Tensor, E: torch.Tensor, targets: torch.Tenso
     ws_bytes = lib().zo_op_lm_head_workspace(S, V, impl)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=h.device)
     out = torch.empty(S, dtype=torch.float32, device=h.device)
-    _check(lib().zo_op_lm_head_logprob(_ptr(h), _ptr(E), _ptr(targets), S, V, d, dtype, _ptr(out),
+    _check_op(lib().zo_op_lm_head_logprob(_ptr(h), _ptr(E), _ptr(targets), S, V, d, dtype, _ptr(out),
                                        _ptr(ws), ws.numel(), impl, _stream()))
     return out
 
@@ -558,7 +565,7 @@ def zo_op_attention(qkv: torch.Tensor, seq_lens, n_heads: int, n_kv_heads: int,
     dtype = wl.DTYPE_BF16 if qkv.dtype == torch.bfloat16 else wl.DTYPE_FP32
     out = torch.empty(T, n_heads * head_dim, dtype=qkv.dtype, device=qkv.device)
     ws = torch.empty(4 * (2 * len(sl) + 2 + T // 64 + 1) + 256, dtype=torch.uint8, device=qkv.device)
-    _check(lib().zo_op_attention(_ptr(qkv), _ptr(out), _ptr(sl), len(sl), n_heads, n_kv_heads,
+    _check_op(lib().zo_op_attention(_ptr(qkv), _ptr(out), _ptr(sl), len(sl), n_heads, n_kv_heads,
                                  head_dim, dtype, _ptr(ws), ws.numel(), impl, _stream()))
     return out
 
@@ -580,7 +587,7 @@ def zo_op_lm_head_logprob_noalloc(h: torch.Tensor, E: torch.Tensor, targets: tor
     if out.dtype != torch.float32 or out.numel() < S:
         raise ValueError("out must be float32 with room for one value per row of h")
     dtype = wl.DTYPE_BF16 if h.dtype == torch.bfloat16 else wl.DTYPE_FP32
-    _check(lib().zo_op_lm_head_logprob_noalloc(_ptr(h), _ptr(E), _ptr(targets), S, E.shape[0], d,
+    _check_op(lib().zo_op_lm_head_logprob_noalloc(_ptr(h), _ptr(E), _ptr(targets), S, E.shape[0], d,
                                                dtype, _ptr(out), impl, _stream()))
     return out
 
