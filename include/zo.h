@@ -202,7 +202,10 @@ int zo_probe_plan(zo_handle* h, uint64_t step, int32_t rank, float eps,
  * Fine-Tuning Is Really Scoring": the pair of forward objective
  * evaluations).  Each prompt becomes a + row and a - row of one packed
  * variable-length batch (all + rows, then all - rows; no padding).
- *   packed_tokens  dev  int32 [sum(seq_lens)]   prompts back to back
+ *   packed_tokens  dev  int32 [sum(seq_lens)]   prompts back to back; ids
+ *                  outside [0, vocab) are checked on the device and never used
+ *                  as an index: the row's objective becomes NaN and zo_step
+ *                  returns ZO_ERR_ARG with the bank unchanged
  *   seq_lens       host int32 [n_prompts]
  *   target_lens    host int32 [n_prompts]       1 <= t < seq_len
  *   target_ids     dev  int32 [sum(target_lens)] or NULL; when given it must

@@ -11,6 +11,8 @@
 """
 import os
 
+import numpy as np
+
 import pytest
 import torch
 
@@ -105,3 +107,43 @@ def test_injected_allocation_failure_returns_oom_and_leaks_nothing(wk):
     assert n > 20, n                                # every allocation point was visited
     torch.cuda.synchronize()
     assert torch.cuda.mem_get_info()[0] == free0
+
+
+@pytest.mark.parametrize("bad", ["vocab", "negative", "last-target"])
+def test_out_of_range_token_ids_are_rejected_on_the_device(bad):
+    """A token id outside [0, vocab) is never used as an index: build_tokens replaces it
+    (its embedding row becomes NaN; a target's logit NaN), so only that prompt's L+- turn
+    NaN, the other prompts score exactly as in a clean batch, zo_step reports ZO_ERR_ARG
+    naming the id and leaves the bank as it was, and the next clean step goes through."""
+    from zeroth_order_fine_b200 import zo
+    from gpu_util import dev_tokens, gpu_handle
+    w = wl.WORKLOADS["tiny"]
+    batch = wl.make_batch(w)
+    clean = batch.packed()
+    _, h = gpu_handle(w)
+    h.zo_probe_plan(0, w.eps)
+    Lp0, Lm0, _ = h.zo_score(dev_tokens(batch), batch.seq_lens, batch.target_lens)
+    Lp0, Lm0 = Lp0.cpu().numpy(), Lm0.cpu().numpy()
+    state0 = h.zo_save_state()
+    toks = clean.copy()
+    starts = np.concatenate([[0], np.cumsum(batch.seq_lens)])
+    i = 1                                                 # the prompt that gets the bad id
+    pos = {"vocab": starts[i] + 1, "negative": starts[i] + 2,
+           "last-target": starts[i + 1] - 1}[bad]
+    toks[pos] = {"vocab": w.shape.vocab, "negative": -5, "last-target": w.shape.vocab + 7}[bad]
+    h.zo_probe_plan(0, w.eps)
+    Lp, Lm, _ = h.zo_score(torch.from_numpy(toks).cuda(), batch.seq_lens, batch.target_lens)
+    Lp, Lm = Lp.cpu().numpy(), Lm.cpu().numpy()
+    assert np.isnan(Lp[i]) and np.isnan(Lm[i])
+    others = [j for j in range(len(batch.seq_lens)) if j != i]
+    assert np.array_equal(Lp[others], Lp0[others]) and np.array_equal(Lm[others], Lm0[others])
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_step(w.lr)
+    assert e.value.code == zo.ZO_ERR_ARG and "token id" in str(e.value)
+    assert h.zo_save_state() == state0                    # update refused, bank unchanged
+    h.zo_probe_plan(0, w.eps)
+    Lp1, Lm1, _ = h.zo_score(dev_tokens(batch), batch.seq_lens, batch.target_lens)
+    assert np.array_equal(Lp1.cpu().numpy(), Lp0) and np.array_equal(Lm1.cpu().numpy(), Lm0)
+    c = h.zo_step(w.lr)
+    assert np.isfinite(c)
+    h.close()

@@ -1103,8 +1103,9 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
     const int* tiles_d = chk_d + R;
     const int Ti = (int)T, Si = (int)S;
 
-    launch_build_tokens(m, R, ptok, ftok, h->tok_id, h->tok_pos, h->tok_sign, h->tok_row,
-                        h->sc_tok, h->sc_tgt, tgt_ids, nullptr, chk_d, h->err_dev, h->st);
+    launch_build_tokens(m, R, ptok, ftok, d.vocab, h->tok_id, h->tok_pos, h->tok_sign,
+                        h->tok_row, h->sc_tok, h->sc_tgt, h->tgt, tgt_ids, nullptr, chk_d,
+                        h->err_dev, h->st);
     // build_tokens, embed, per layer 2 norms + attention (+ SwiGLU), final norm, LSE merge
     h->stats.kernel_launches +=
         2 + (uint64_t)d.n_layers * (3 + (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused) +
@@ -1222,8 +1223,9 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
     const float scale = (float)(1.0 / std::sqrt((double)d.head_dim));
 
     // prefill: the prompts of both candidates as one packed batch, k|v kept per layer
-    launch_build_tokens(m, R, ptok, nullptr, h->tok_id, h->tok_pos, h->tok_sign, h->tok_row,
-                        h->sc_tok, h->sc_tgt, nullptr, nullptr, chk_d, h->err_dev, h->st);
+    launch_build_tokens(m, R, ptok, nullptr, d.vocab, h->tok_id, h->tok_pos, h->tok_sign,
+                        h->tok_row, h->sc_tok, h->sc_tgt, h->tgt, nullptr, nullptr, chk_d,
+                        h->err_dev, h->st);
     launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
                  d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
                  d.d_model, h->st);
@@ -1439,6 +1441,7 @@ int zo_step_from_sums(zo_handle* h, float lr, const double* dev_sums, double* c_
         CK(h, cudaStreamSynchronize(h->st));
         if (err) {
             CK(h, cudaMemsetAsync(h->err_dev, 0, 4, h->st));
+            if (err & 2) FAIL(h, ZO_ERR_ARG, "a token id lies outside [0, vocab): update refused");
             FAIL(h, ZO_ERR_ARG, "target_ids differ from the rows' last tokens");
         }
         if (flag) FAIL(h, ZO_ERR_NONFINITE, "non-finite objective: update refused");

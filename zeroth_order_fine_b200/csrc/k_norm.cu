@@ -12,10 +12,11 @@ namespace zo {
 // and, per scored position, the index of the hidden state that predicts it
 // (the position before the target token) and the target id.
 __global__ void build_tokens_kernel(RowMeta m, const int* __restrict__ probe_src,
-                                    const int* __restrict__ fg_src, int* tok_id, int* tok_pos,
-                                    int* tok_sign, int* tok_row, int* sc_tok, int* sc_tgt,
-                                    const int* tgt_check_probe, const int* tgt_check_fg,
-                                    const int* tgt_check_off, int* err_word) {
+                                    const int* __restrict__ fg_src, int vocab, int* tok_id,
+                                    int* tok_pos, int* tok_sign, int* tok_row, int* sc_tok,
+                                    int* sc_tgt, float* tgt_logit, const int* tgt_check_probe,
+                                    const int* tgt_check_fg, const int* tgt_check_off,
+                                    int* err_word) {
     const int r = blockIdx.x;
     const int start = m.cu_seqlens[r];
     const int len = m.cu_seqlens[r + 1] - start;
@@ -23,7 +24,14 @@ __global__ void build_tokens_kernel(RowMeta m, const int* __restrict__ probe_src
     const int sign = m.row_sign[r];
     for (int p = threadIdx.x; p < len; p += blockDim.x) {
         const int t = start + p;
-        tok_id[t] = src[p];
+        int id = src[p];
+        // an id outside the vocabulary is never used as an index: -1 makes the embedding
+        // row NaN, and bit 1 of the error word reports it
+        if ((unsigned)id >= (unsigned)vocab) {
+            id = -1;
+            atomicOr(err_word, 2);
+        }
+        tok_id[t] = id;
         tok_pos[t] = p;
         tok_sign[t] = sign;
         tok_row[t] = r;
@@ -34,31 +42,39 @@ __global__ void build_tokens_kernel(RowMeta m, const int* __restrict__ probe_src
     for (int j = threadIdx.x; j < tl; j += blockDim.x) {
         const int tgt = src[len - tl + j];
         sc_tok[s0 + j] = start + len - tl + j - 1;
+        // the lm_head epilogue writes the logit of an in-range target only; an out-of-range
+        // one keeps this NaN, so its log-prob is NaN
         sc_tgt[s0 + j] = tgt;
+        if ((unsigned)tgt >= (unsigned)vocab) tgt_logit[s0 + j] = __int_as_float(0x7fc00000);
         if (chk != nullptr && tgt_check_off[r] >= 0 && chk[tgt_check_off[r] + j] != tgt)
             atomicOr(err_word, 1);
     }
 }
 
-void launch_build_tokens(RowMeta m, int R, const int* probe_src, const int* fg_src,
+void launch_build_tokens(RowMeta m, int R, const int* probe_src, const int* fg_src, int vocab,
                          int* tok_id, int* tok_pos, int* tok_sign, int* tok_row, int* sc_tok,
-                         int* sc_tgt, const int* tgt_check_probe, const int* tgt_check_fg,
-                         const int* tgt_check_off, int* err_word, cudaStream_t st) {
+                         int* sc_tgt, float* tgt_logit, const int* tgt_check_probe,
+                         const int* tgt_check_fg, const int* tgt_check_off, int* err_word,
+                         cudaStream_t st) {
     if (R == 0) return;
-    build_tokens_kernel<<<R, 128, 0, st>>>(m, probe_src, fg_src, tok_id, tok_pos, tok_sign,
-                                           tok_row, sc_tok, sc_tgt, tgt_check_probe,
+    build_tokens_kernel<<<R, 128, 0, st>>>(m, probe_src, fg_src, vocab, tok_id, tok_pos, tok_sign,
+                                           tok_row, sc_tok, sc_tgt, tgt_logit, tgt_check_probe,
                                            tgt_check_fg, tgt_check_off, err_word);
 }
 
-// resid[t] = tok_embed[id] (+ pos_embed[pos]) in fp32.
+// resid[t] = tok_embed[id] (+ pos_embed[pos]) in fp32; NaN for a rejected id (-1).
 __global__ void embed_kernel(const int* __restrict__ tok_id, const int* __restrict__ tok_pos,
                              const void* __restrict__ tok_embed,
                              const void* __restrict__ pos_embed, int dtype,
                              float* __restrict__ resid, int d) {
     const int t = blockIdx.x;
+    float* out = resid + (size_t)t * d;
+    if (tok_id[t] < 0) {                         // rejected id: the row is NaN throughout
+        for (int i = threadIdx.x; i < d; i += blockDim.x) out[i] = __int_as_float(0x7fc00000);
+        return;
+    }
     const size_t te = (size_t)tok_id[t] * d;
     const size_t pe = (size_t)tok_pos[t] * d;
-    float* out = resid + (size_t)t * d;
     for (int i = threadIdx.x; i < d; i += blockDim.x) {
         float v = ld_elem(tok_embed, te + i, dtype);
         if (pos_embed) v += ld_elem(pos_embed, pe + i, dtype);

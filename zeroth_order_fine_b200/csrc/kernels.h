@@ -46,10 +46,13 @@ struct RowMeta {          // device arrays built from the host plan of one score
     const int* score_off;     // [R+1] offsets of each row's scored span
 };
 
-void launch_build_tokens(RowMeta m, int R, const int* probe_src, const int* fg_src,
+// Token ids outside [0, vocab) become -1 (a NaN embedding row; an out-of-range target gets
+// a NaN logit) and set bit 1 of err_word; target_ids that differ set bit 0.
+void launch_build_tokens(RowMeta m, int R, const int* probe_src, const int* fg_src, int vocab,
                          int* tok_id, int* tok_pos, int* tok_sign, int* tok_row, int* sc_tok,
-                         int* sc_tgt, const int* tgt_check_probe, const int* tgt_check_fg,
-                         const int* tgt_check_off, int* err_word, cudaStream_t st);
+                         int* sc_tgt, float* tgt_logit, const int* tgt_check_probe,
+                         const int* tgt_check_fg, const int* tgt_check_off, int* err_word,
+                         cudaStream_t st);
 void launch_embed(const int* tok_id, const int* tok_pos, const void* tok_embed,
                   const void* pos_embed, int dtype, float* resid, int T, int d, cudaStream_t st);
 // kind 0: LayerNorm(w, b), 1: RMSNorm(w).  rows: optional gather list (else 0..T-1).
