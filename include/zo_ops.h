@@ -202,6 +202,22 @@ int zo_op_lm_head_logprob_noalloc(const void* h, const void* E, const int32_t* t
  * reported an error. */
 int zo_op_error_word(void);
 
+/* The debug build (libzo_b200_debug.so, compiled with ZO_DEBUG) checks, on the
+ * device, the indices its kernels derive from the host-built row metadata:
+ * the attention work tiles (row and query tile), the key/value cache rows
+ * of generation, and each row's scored span.  A failed check sets a bit of
+ * a device word (1: attention tile, 2: cache row, 4: scored span) and the
+ * access is skipped (an empty attention item, no cache copy, a NaN
+ * objective); nothing traps.  The release build compiles the checks away.
+ * zo_debug_build() is 1 in the debug build, else 0.  zo_debug_word(clear)
+ * returns the bits set since the last clear (always 0 in the release build)
+ * and clears them when clear != 0.  Synchronous (reads device memory).
+ * In the debug build only, ZO_DEBUG_PLANT=attention_tile in the environment
+ * makes zo_op_attention point its last work tile at a row past the batch,
+ * so that a test can see the check fire. */
+int zo_debug_build(void);
+uint32_t zo_debug_word(int32_t clear);
+
 /* What the calling thread's last zo_op_* call that returned ZO_ERR_CUDA ran
  * into: the step that failed and the CUDA error's name and text ("" before
  * any failure).  The string is the library's, valid until that thread's next

@@ -117,3 +117,13 @@ def test_decode_linear_argument_checks_without_gpu(built_lib):
 def test_op_error_text_is_empty_before_any_failure(built_lib):
     built_lib.zo_op_last_error.restype = ctypes.c_char_p
     assert built_lib.zo_op_last_error() == b""
+
+
+def test_debug_build_exports_the_same_symbols_and_says_so(built_lib):
+    """libzo_b200_debug.so (ZO_DEBUG: device bounds checks) links from the same sources:
+    every declared symbol is there, and zo_debug_build tells the two builds apart."""
+    from zeroth_order_fine_b200 import build
+    dbg = ctypes.CDLL(build.build(debug=True))
+    missing = [n for n in sorted(declared_functions()) if not hasattr(dbg, n)]
+    assert not missing, missing
+    assert dbg.zo_debug_build() == 1 and built_lib.zo_debug_build() == 0

@@ -2,7 +2,9 @@
 
 Each translation unit under csrc/ is compiled to an object under _build/
 (rebuilt only when it or a header changed, earlier builds kept by content) and linked into
-zeroth_order_fine_b200/libzo_b200.so, which the Python binding loads.
+zeroth_order_fine_b200/libzo_b200.so, which the Python binding loads.  `--debug` builds
+libzo_b200_debug.so instead: the same sources with ZO_DEBUG defined (device bounds checks),
+loaded when ZO_LIB=debug.
 """
 from __future__ import annotations
 
@@ -17,6 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libzo_b200.so")
+OUT_DEBUG = os.path.join(HERE, "libzo_b200_debug.so")
 BUILD = os.path.join(ROOT, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -33,15 +36,15 @@ def _headers_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def _compile(src: str, hdr: str, verbose: bool) -> str:
+def _compile(src: str, hdr: str, flags: list, verbose: bool) -> str:
     with open(src, "rb") as fh:
-        tag = hashlib.sha256(fh.read() + hdr.encode() + " ".join(FLAGS).encode()).hexdigest()[:16]
+        tag = hashlib.sha256(fh.read() + hdr.encode() + " ".join(flags).encode()).hexdigest()[:16]
     obj = os.path.join(BUILD, os.path.basename(src) + "." + tag + ".o")
     if os.path.exists(obj):
         return obj
-    cmd = [NVCC] + ARCH + FLAGS + ["-c", src, "-o", obj]
+    cmd = [NVCC] + ARCH + flags + ["-c", src, "-o", obj]
     if src.endswith(".cpp"):
-        cmd = [NVCC] + FLAGS + ["-x", "cu"] + ARCH + ["-c", src, "-o", obj]
+        cmd = [NVCC] + flags + ["-x", "cu"] + ARCH + ["-c", src, "-o", obj]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -50,31 +53,33 @@ def _compile(src: str, hdr: str, verbose: bool) -> str:
     return obj
 
 
-def build(verbose: bool = False) -> str:
+def build(verbose: bool = False, debug: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
     hdr = _headers_digest()
+    flags = FLAGS + (["-DZO_DEBUG"] if debug else [])
+    out = OUT_DEBUG if debug else OUT
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, hdr, verbose), srcs))
+        objs = list(ex.map(lambda s: _compile(s, hdr, flags, verbose), srcs))
     # relink whenever the set of objects differs from the one the library was linked from
     # (going back to an earlier source picks up its cached, older object)
-    stamp = os.path.join(BUILD, os.path.basename(OUT) + ".objects")
+    stamp = os.path.join(BUILD, os.path.basename(out) + ".objects")
     linked = "\n".join(os.path.basename(o) for o in objs) + "\n"
-    if os.path.exists(OUT) and os.path.exists(stamp):
+    if os.path.exists(out) and os.path.exists(stamp):
         with open(stamp) as fh:
             if fh.read() == linked:
-                return OUT
-    cmd = [NVCC] + ARCH + ["-shared", "-o", OUT + ".tmp"] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
+                return out
+    cmd = [NVCC] + ARCH + ["-shared", "-o", out + ".tmp"] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(OUT + ".tmp", OUT)
+    os.replace(out + ".tmp", out)
     with open(stamp, "w") as fh:
         fh.write(linked)
-    return OUT
+    return out
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -61,6 +61,31 @@ __device__ __forceinline__ float block_max(float v, float* red /* >= 32 floats *
 
 inline unsigned cdiv(long long a, long long b) { return (unsigned)((a + b - 1) / b); }
 
+// ---- debug build (ZO_DEBUG): device bounds checks -------------------------------------
+// ZO_DCHECK(cond, bit) is `cond` in the debug build, where a failed check also ORs `bit` into
+// the translation unit's debug word and the caller skips the access; in the release build it
+// is `true` and compiles away.  No check traps.  A translation unit that checks places
+// ZO_DEBUG_WORD(reader) at namespace scope before its kernels: the word, and a host function
+// `unsigned reader(bool clear)` that returns it (0 in the release build).
+#ifdef ZO_DEBUG
+#define ZO_DCHECK(cond, bit) ((cond) ? true : (atomicOr(&g_zo_debug_word, (unsigned)(bit)), false))
+#define ZO_DEBUG_WORD(reader)                                                               \
+    static __device__ unsigned int g_zo_debug_word = 0;                                     \
+    unsigned reader(bool clear) {                                                           \
+        unsigned v = 0;                                                                     \
+        if (cudaMemcpyFromSymbol(&v, g_zo_debug_word, sizeof(v)) != cudaSuccess) return ~0u; \
+        if (clear) {                                                                        \
+            const unsigned z = 0;                                                           \
+            cudaMemcpyToSymbol(g_zo_debug_word, &z, sizeof(z));                             \
+        }                                                                                   \
+        return v;                                                                           \
+    }
+#else
+#define ZO_DCHECK(cond, bit) true
+#define ZO_DEBUG_WORD(reader) \
+    unsigned reader(bool) { return 0; }
+#endif
+
 // Programmatic dependent launch: a kernel launched with launch_pdl may be scheduled while the
 // kernel before it on the stream still runs; grid_dep_wait() blocks until that kernel has
 // finished and its writes are visible (a no-op for an ordinary launch), grid_dep_launch()

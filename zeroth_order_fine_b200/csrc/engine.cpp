@@ -1126,6 +1126,7 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
             a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
             a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
             a.n_tokens = Ti;
+            a.n_rows = R;
             if (tc_attn && attention_tc_supported(a)) {
                 if (!launch_attention_tc(a, h->st)) FAIL(h, ZO_ERR_CUDA, "attention tensor map failed");
             } else {
@@ -1230,8 +1231,8 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
                  d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
                  d.d_model, h->st);
     rc = decoder_layers(h, Ti, eps, [&](int l) -> int {
-        launch_kv_scatter(h->qkv, h->n_qkv, h->q_dim, kv2, h->tok_row, Ti, G, cache(l), h->dt,
-                          h->st);
+        launch_kv_scatter(h->qkv, h->n_qkv, h->q_dim, kv2, h->tok_row, Ti, G, cache(l),
+                          h->kv_rows, h->dt, h->st);
         AttnArgs a;
         memset(&a, 0, sizeof(a));
         a.qkv = h->qkv; a.ld_qkv = h->n_qkv;
@@ -1242,6 +1243,7 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
         a.H = d.n_heads; a.Hkv = d.n_kv_heads; a.hd = d.head_dim;
         a.scale = scale;
         a.n_tokens = Ti;
+        a.n_rows = R;
         if (tc_attn && attention_tc_supported(a)) {
             if (!launch_attention_tc(a, h->st)) FAIL(h, ZO_ERR_CUDA, "attention tensor map failed");
         } else {
@@ -1271,7 +1273,7 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
                      d.d_model, h->st);
         rc = decoder_layers(h, R, eps, [&](int l) -> int {
             launch_kv_append(h->qkv, h->n_qkv, h->q_dim, kv2, md, h->gen_lens, R, g, G, cache(l),
-                             h->dt, h->st);
+                             h->kv_rows, h->dt, h->st);
             if (!launch_decode_attention(h->qkv, h->n_qkv, cache(l), kv2, md, h->gen_lens, R, g, G,
                                          d.n_heads, d.n_kv_heads, d.head_dim, scale, h->att,
                                          h->q_dim, h->dt, max_len + g + 1, h->splitk_ws,
@@ -1324,11 +1326,11 @@ static int score_common(zo_plan* plan, zo_handle* h, const int32_t* ptok, int32_
     const int R = 2 * B + F;
     // score_off sits after cu[R+1], src[R], fg[R], sign[R] in the device metadata
     const int* soff_d = h->meta + (R + 1) + 3 * R;
-    launch_row_objective(h->logprob, soff_d, R, B, h->L_row, Lp, Lm, h->st);
-    h->stats.kernel_launches++;
     long long Sp = 0, Sf = 0;
     for (int i = 0; i < B; ++i) Sp += tls[i];
     for (int i = 0; i < F; ++i) Sf += ftls[i];
+    launch_row_objective(h->logprob, soff_d, R, B, 2 * Sp + Sf, h->L_row, Lp, Lm, h->st);
+    h->stats.kernel_launches++;
     if (tok_lp && Sp)
         CK(h, cudaMemcpyAsync(tok_lp, h->logprob, 2 * Sp * 4, cudaMemcpyDeviceToDevice, h->st));
     if (fg_lp && Sf)
@@ -1525,7 +1527,8 @@ int zo_step_graph(zo_handle* h, const int32_t* packed_tokens, int32_t n_prompts,
         rc = launch_batch(h, eps, G.meta, bp, packed_tokens, nullptr, nullptr);
         if (!rc) {
             const int* soff_d = G.meta + (R + 1) + 3 * R;
-            launch_row_objective(h->logprob, soff_d, R, B, h->L_row, L_plus, L_minus, h->st);
+            launch_row_objective(h->logprob, soff_d, R, B, bp.S, h->L_row, L_plus, L_minus,
+                                 h->st);
             launch_objective_sums(h->L_row, B, h->sums, h->st);
             launch_estimate(h->sums, eps, h->c_dev, h->flag_dev, h->st);
             launch_bank_update(h->upd_d, h->n_genU, h->max_upd, h->c_dev, h->flag_dev, lr,

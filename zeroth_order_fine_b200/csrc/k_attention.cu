@@ -12,6 +12,8 @@
 
 namespace zo {
 
+ZO_DEBUG_WORD(debug_word_attention)
+
 namespace {
 constexpr int QT = 64;   // queries per CTA
 constexpr int KC = 64;   // keys per chunk
@@ -34,11 +36,14 @@ __global__ void __launch_bounds__(256) attention_kernel(AttnArgs a) {
     float* Vs = Ks + KC * (HD + 1);        // [KC][HD]
     const int tile = a.tiles[blockIdx.x];
     const int row = tile >> 16, qt = tile & 0xFFFF;
+    // (debug build) a tile naming a row or query tile that is not there is skipped whole
+    if (!ZO_DCHECK((unsigned)row < (unsigned)a.n_rows, ZO_DBG_ATTN_TILE)) return;
     const int h = blockIdx.y;
     const int kvh = h / (a.H / a.Hkv);
     const int start = a.cu_seqlens[row];
     const int len = a.cu_seqlens[row + 1] - start;
     const int q0 = qt * QT;
+    if (!ZO_DCHECK(q0 < len, ZO_DBG_ATTN_TILE)) return;
     const int nq = min(QT, len - q0);
     const int kend = min(len, q0 + QT);    // keys needed by this tile
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

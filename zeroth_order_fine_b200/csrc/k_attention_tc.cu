@@ -27,6 +27,8 @@
 
 namespace zo {
 
+ZO_DEBUG_WORD(debug_word_attention_tc)
+
 namespace {
 
 constexpr int TQ = 128, TK = 128, HD = 128;
@@ -208,12 +210,30 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i, int tile, in
     it.nq = min(TQ, it.len - it.q0);
     it.kend = min(it.len, it.q0 + TQ);
     it.n_chunks = (it.kend + TK - 1) / TK;
+    // (debug build) a query tile past its row's end, an empty span included, becomes an empty
+    // item: one fully masked key chunk at token 0 and nothing stored
+    if (!ZO_DCHECK(it.q0 < it.len, ZO_DBG_ATTN_TILE)) {
+        it.start = it.len = it.q0 = it.nq = it.kend = 0;
+        it.n_chunks = 1;
+    }
     return it;
+}
+// Token offsets of the row a tile names; (debug build) a row that is not there is not read
+// and gives an empty span
+__device__ __forceinline__ void row_span(const int* cu, int n_rows, int tile, int& s, int& e) {
+    const int row = tile >> 16;
+    if (ZO_DCHECK((unsigned)row < (unsigned)n_rows, ZO_DBG_ATTN_TILE)) {
+        s = cu[row];
+        e = cu[row + 1];
+    } else {
+        s = e = 0;
+    }
 }
 __device__ __forceinline__ Item get_item(const AttnArgs& a, int i) {
     const int tile = a.tiles[i / a.H];
-    const int row = tile >> 16;
-    return make_item(a, i, tile, a.cu_seqlens[row], a.cu_seqlens[row + 1]);
+    int s, e;
+    row_span(a.cu_seqlens, a.n_rows, tile, s, e);
+    return make_item(a, i, tile, s, e);
 }
 
 // The items of this CTA in order (k-th: blockIdx.x + k * gridDim.x), with their metadata
@@ -223,7 +243,7 @@ __device__ __forceinline__ Item get_item(const AttnArgs& a, int i) {
 struct ItemFeed {
     const int* tiles;
     const int* cu;
-    AttnArgs shape;             // only H and Hkv are read (make_item)
+    AttnArgs shape;             // only H, Hkv and n_rows are read
     int n_items;
     int k;                      // index of cur among this CTA's items
     bool has;                   // cur exists
@@ -236,6 +256,7 @@ struct ItemFeed {
         cu = args.cu_seqlens;
         shape.H = args.H;
         shape.Hkv = args.Hkv;
+        shape.n_rows = args.n_rows;
         n_items = n;
         k = 0;
         has = idx(0) < n;
@@ -243,8 +264,7 @@ struct ItemFeed {
         tile1 = s1 = e1 = tile2 = 0;
         if (idx(1) < n) {
             tile1 = tiles[idx(1) / shape.H];
-            s1 = cu[tile1 >> 16];
-            e1 = cu[(tile1 >> 16) + 1];
+            row_span(cu, shape.n_rows, tile1, s1, e1);
         }
         if (idx(2) < n) tile2 = tiles[idx(2) / shape.H];
     }
@@ -254,8 +274,7 @@ struct ItemFeed {
         if (has) cur = make_item(shape, idx(k), tile1, s1, e1);   // loaded an item ago
         if (idx(k + 1) < n_items) {
             tile1 = tile2;
-            s1 = cu[tile1 >> 16];                                  // used at the next advance
-            e1 = cu[(tile1 >> 16) + 1];
+            row_span(cu, shape.n_rows, tile1, s1, e1);             // used at the next advance
         }
         if (idx(k + 2) < n_items) tile2 = tiles[idx(k + 2) / shape.H];
     }

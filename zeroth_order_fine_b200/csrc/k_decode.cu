@@ -17,6 +17,8 @@
 
 namespace zo {
 
+ZO_DEBUG_WORD(debug_word_decode)
+
 namespace {
 
 // 16-byte copies when both rows allow it, else element by element
@@ -35,9 +37,10 @@ __device__ __forceinline__ void copy_row(const void* src, void* dst, int n_elem,
 
 __global__ void kv_scatter_kernel(const char* __restrict__ qkv, int ld_qkv, int q_dim, int kv2,
                                   const int* __restrict__ tok_row, int G, char* __restrict__ cache,
-                                  int es) {
+                                  size_t cache_rows, int es) {
     const int t = blockIdx.x;
     const size_t crow = (size_t)t + (size_t)tok_row[t] * G;
+    if (!ZO_DCHECK(crow < cache_rows, ZO_DBG_KV_SLOT)) return;     // (debug build)
     copy_row(qkv + ((size_t)t * ld_qkv + q_dim) * es, cache + crow * kv2 * es, kv2, es);
 }
 
@@ -54,11 +57,12 @@ __global__ void decode_prep_kernel(const int* __restrict__ gen_tok, int G, int g
 
 __global__ void kv_append_kernel(const char* __restrict__ qkv, int ld_qkv, int q_dim, int kv2,
                                  const int* __restrict__ cu, const int* __restrict__ lens, int g,
-                                 int G, char* __restrict__ cache, int es) {
+                                 int G, char* __restrict__ cache, size_t cache_rows, int es) {
     grid_dep_wait();                    // launched as a programmatic dependent
     grid_dep_launch();
     const int r = blockIdx.x;
     const size_t crow = (size_t)cu[r] + (size_t)r * G + lens[r] + g;
+    if (!ZO_DCHECK(crow < cache_rows, ZO_DBG_KV_SLOT)) return;     // (debug build)
     copy_row(qkv + ((size_t)r * ld_qkv + q_dim) * es, cache + crow * kv2 * es, kv2, es);
 }
 
@@ -420,10 +424,10 @@ __global__ void gen_objective_kernel(const float* __restrict__ logprob, int R, i
 }  // namespace
 
 void launch_kv_scatter(const void* qkv, int ld_qkv, int q_dim, int kv2, const int* tok_row,
-                       int T, int G, void* cache, int dtype, cudaStream_t st) {
+                       int T, int G, void* cache, size_t cache_rows, int dtype, cudaStream_t st) {
     if (T == 0) return;
     kv_scatter_kernel<<<T, 128, 0, st>>>(static_cast<const char*>(qkv), ld_qkv, q_dim, kv2,
-                                         tok_row, G, static_cast<char*>(cache),
+                                         tok_row, G, static_cast<char*>(cache), cache_rows,
                                          dtype == E_F32 ? 4 : 2);
 }
 
@@ -435,11 +439,12 @@ void launch_decode_prep(const int* gen_tok, int G, int g, const int* lens, int R
 }
 
 void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int* cu,
-                      const int* lens, int R, int g, int G, void* cache, int dtype,
-                      cudaStream_t st) {
+                      const int* lens, int R, int g, int G, void* cache, size_t cache_rows,
+                      int dtype, cudaStream_t st) {
     if (R == 0) return;
     launch_pdl(kv_append_kernel, dim3(R), dim3(128), 0, st, static_cast<const char*>(qkv), ld_qkv,
-               q_dim, kv2, cu, lens, g, G, static_cast<char*>(cache), dtype == E_F32 ? 4 : 2);
+               q_dim, kv2, cu, lens, g, G, static_cast<char*>(cache), cache_rows,
+               dtype == E_F32 ? 4 : 2);
 }
 
 template <int HD, int NR>

@@ -20,6 +20,8 @@
 
 namespace zo {
 
+ZO_DEBUG_WORD(debug_word_reduce)
+
 // One warp per scored position; lanes take tiles lane, lane+32, ... and the
 // lane results are combined by a fixed xor tree.
 __global__ void lse_merge_kernel(const float* __restrict__ pmax, const float* __restrict__ psum,
@@ -82,10 +84,13 @@ void launch_lse_argmax_merge(const float* part_max, const float* part_sum, const
 
 __global__ void row_objective_kernel(const float* __restrict__ logprob,
                                      const int* __restrict__ score_off, int R, int B,
-                                     double* __restrict__ L_row, float* L_plus, float* L_minus) {
+                                     long long S, double* __restrict__ L_row, float* L_plus,
+                                     float* L_minus) {
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= R) return;
-    const int a = score_off[r], b = score_off[r + 1];
+    int a = score_off[r], b = score_off[r + 1];
+    // (debug build) a span outside [0, S) is not read: an empty span gives L = NaN
+    if (!ZO_DCHECK(a >= 0 && a <= b && b <= S, ZO_DBG_SCORE_SPAN)) a = b = 0;
     double s = 0.0;
     for (int i = a; i < b; ++i) s += (double)logprob[i];
     const double L = -s / (double)(b - a);
@@ -94,10 +99,10 @@ __global__ void row_objective_kernel(const float* __restrict__ logprob,
     else if (r >= B && r < 2 * B && L_minus) L_minus[r - B] = (float)L;
 }
 
-void launch_row_objective(const float* logprob, const int* score_off, int R, int B,
+void launch_row_objective(const float* logprob, const int* score_off, int R, int B, long long S,
                           double* L_row, float* L_plus, float* L_minus, cudaStream_t st) {
     if (R == 0) return;
-    row_objective_kernel<<<cdiv(R, 128), 128, 0, st>>>(logprob, score_off, R, B, L_row, L_plus,
+    row_objective_kernel<<<cdiv(R, 128), 128, 0, st>>>(logprob, score_off, R, B, S, L_row, L_plus,
                                                        L_minus);
 }
 

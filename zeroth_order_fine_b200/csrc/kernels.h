@@ -142,6 +142,7 @@ struct AttnArgs {
     int H, Hkv, hd;
     float scale;
     int n_tokens;                   // T: rows of qkv (the tensor-core kernel's TMA extent)
+    int n_rows;                     // R: entries of cu_seqlens minus one (debug bounds checks)
 };
 // (Qwen3's q/k RMSNorm and rotary positions are applied to the q|k|v rows before
 // attention by launch_qk_norm_rope; the attention kernels take q and k as they are.)
@@ -164,14 +165,15 @@ void launch_lse_argmax_merge(const float* part_max, const float* part_sum, const
 // Cache layout per layer: [rows of (k | v)], row r's tokens at cu[r] + r * G + p, where cu
 // are the prompt offsets and G the new tokens per row; a cache row is 2 * kv_dim wide.
 // Prefill: copy each token's k|v columns of the packed q|k|v rows into the cache.
+// cache_rows: rows of one layer's cache (the debug build checks every row index against it).
 void launch_kv_scatter(const void* qkv, int ld_qkv, int q_dim, int kv2, const int* tok_row,
-                       int T, int G, void* cache, int dtype, cudaStream_t st);
+                       int T, int G, void* cache, size_t cache_rows, int dtype, cudaStream_t st);
 // Decode step g (g >= 0): row r's new token sits at prompt length + g.
 void launch_decode_prep(const int* gen_tok, int G, int g, const int* lens, int R, int B,
                         int* tok_id, int* tok_pos, int* tok_sign, int* tok_row, cudaStream_t st);
 void launch_kv_append(const void* qkv, int ld_qkv, int q_dim, int kv2, const int* cu,
-                      const int* lens, int R, int g, int G, void* cache, int dtype,
-                      cudaStream_t st);
+                      const int* lens, int R, int g, int G, void* cache, size_t cache_rows,
+                      int dtype, cudaStream_t st);
 // One query per row (its q heads in qkv row r) against the row's n = lens[r] + g + 1 cached
 // keys; softmax(q k^T * scale) v into out [R x H*hd].  CUDA cores (memory-bound).  false
 // when H / Hkv > 8 or hd is not 32, 64, 128 or 256.
@@ -202,7 +204,8 @@ void launch_last_tokens(const int* cu, int R, int* out, int* lens, cudaStream_t 
 void launch_gen_objective(const float* logprob, int R, int B, int G, double* L_row,
                           float* L_plus, float* L_minus, cudaStream_t st);
 // per row L = -mean(logprob over its span) (fp64); L+/L- copies for the probe rows.
-void launch_row_objective(const float* logprob, const int* score_off, int R, int B,
+// S: scored positions in logprob (the debug build checks each span against it).
+void launch_row_objective(const float* logprob, const int* score_off, int R, int B, long long S,
                           double* L_row, float* L_plus, float* L_minus, cudaStream_t st);
 // sums[0] = sum_i (L_row[i] - L_row[B+i]) in a fixed order, sums[1] = B.
 void launch_objective_sums(const double* L_row, int B, double* sums, cudaStream_t st);
@@ -226,5 +229,17 @@ void launch_bank_update(const UpdateJob* jobs, int n_jobs, int max_pairs, const 
                         const int* flag, float lr, uint64_t run_seed, uint64_t step,
                         const uint64_t* step_dev, uint64_t nu, float scale, int apply_scale,
                         long long replay_from, float* coef_hist, cudaStream_t st);
+
+// Debug build (ZO_DEBUG): the device bounds-check words of the translation units that check
+// (bits ZO_DBG_*), read and optionally cleared; always 0 in the release build.
+enum : unsigned {
+    ZO_DBG_ATTN_TILE = 1u,      // an attention work item names a row or query tile that is not there
+    ZO_DBG_KV_SLOT = 2u,        // a key/value cache row index past the cache
+    ZO_DBG_SCORE_SPAN = 4u,     // a row's scored span outside the scored positions
+};
+unsigned debug_word_attention_tc(bool clear);
+unsigned debug_word_attention(bool clear);
+unsigned debug_word_decode(bool clear);
+unsigned debug_word_reduce(bool clear);
 
 }  // namespace zo

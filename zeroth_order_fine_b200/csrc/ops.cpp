@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <algorithm>
 #include <string>
@@ -191,6 +192,13 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     if (tc)
         std::stable_sort(tiles.begin(), tiles.end(),
                          [](int x, int y) { return (x & 0xFFFF) > (y & 0xFFFF); });
+#ifdef ZO_DEBUG
+    // test hook of the debug build: ZO_DEBUG_PLANT=attention_tile makes the last work tile
+    // name a row past the batch; the kernels' bounds checks must report it and skip it
+    if (const char* plant = std::getenv("ZO_DEBUG_PLANT"))
+        if (!std::strcmp(plant, "attention_tile") && !tiles.empty())
+            tiles.back() = (n_rows << 16) | (tiles.back() & 0xFFFF);
+#endif
     const size_t need = (meta.size() + tiles.size()) * 4;
     if (!workspace || workspace_bytes < need) return ZO_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -211,6 +219,7 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     a.H = n_heads; a.Hkv = n_kv_heads; a.hd = head_dim;
     a.scale = (float)(1.0 / std::sqrt((double)head_dim));
     a.n_tokens = meta[n_rows];
+    a.n_rows = n_rows;
     if (tc && attention_tc_supported(a)) {
         if (!launch_attention_tc(a, st)) return op_fail("tensor-core attention setup failed");
     } else if (impl == ZO_IMPL_TENSOR_CORES) {
@@ -287,6 +296,19 @@ int zo_op_error_word(void) {
     const int w = attention_tc_error_word();
     if (v < 0 || w < 0) return -1;
     return v | w;
+}
+
+int zo_debug_build(void) {
+#ifdef ZO_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+uint32_t zo_debug_word(int32_t clear) {
+    return debug_word_attention_tc(clear != 0) | debug_word_attention(clear != 0) |
+           debug_word_decode(clear != 0) | debug_word_reduce(clear != 0);
 }
 
 const char* zo_op_last_error(void) { return t_op_err.c_str(); }

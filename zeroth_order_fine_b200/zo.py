@@ -17,7 +17,9 @@ import torch
 from . import workload as wl
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libzo_b200.so")
+# ZO_LIB=debug loads the debug build (device bounds checks, see zo_ops.h zo_debug_word)
+LIB_PATH = os.path.join(_HERE, "libzo_b200_debug.so" if os.environ.get("ZO_LIB") == "debug"
+                        else "libzo_b200.so")
 
 ZO_OK, ZO_ERR_ARG, ZO_ERR_STATE, ZO_ERR_CUDA, ZO_ERR_OOM, ZO_ERR_NONFINITE, ZO_ERR_TIMEOUT, \
     ZO_ERR_UNSUPPORTED = range(8)
@@ -101,6 +103,8 @@ _SIGS = {
     "zo_destroy": (None, [c_void_p]),
     "zo_last_error": (ctypes.c_char_p, [c_void_p]),
     "zo_op_last_error": (ctypes.c_char_p, []),
+    "zo_debug_build": (ctypes.c_int, []),
+    "zo_debug_word": (ctypes.c_uint32, [ctypes.c_int32]),
     "zo_probe_plan": (c_int32, [c_void_p, c_uint64, c_int32, ctypes.c_float,
                                 ctypes.POINTER(zo_targets), ctypes.POINTER(c_void_p)]),
     "zo_score": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -160,7 +164,8 @@ def lib() -> ctypes.CDLL:
     if _LIB is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                               "`python -m zeroth_order_fine_b200.build` (needs nvcc)")
+                               "`python -m zeroth_order_fine_b200.build` (--debug for the debug "
+                               "build; needs nvcc)")
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in _SIGS.items():
             fn = getattr(L, name)
@@ -559,11 +564,16 @@ def zo_op_lm_head_logprob(h: torch.Tensor, E: torch.Tensor, targets: torch.Tenso
 
 
 def zo_op_attention(qkv: torch.Tensor, seq_lens, n_heads: int, n_kv_heads: int,
-                    head_dim: int, impl: int = IMPL_AUTO) -> torch.Tensor:
+                    head_dim: int, impl: int = IMPL_AUTO,
+                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
     sl = _i32(seq_lens)
     T = qkv.shape[0]
     dtype = wl.DTYPE_BF16 if qkv.dtype == torch.bfloat16 else wl.DTYPE_FP32
-    out = torch.empty(T, n_heads * head_dim, dtype=qkv.dtype, device=qkv.device)
+    if out is None:
+        out = torch.empty(T, n_heads * head_dim, dtype=qkv.dtype, device=qkv.device)
+    elif (out.shape != (T, n_heads * head_dim) or out.dtype != qkv.dtype or not out.is_cuda
+          or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous CUDA tensor [T x n_heads*head_dim] of qkv's dtype")
     ws = torch.empty(4 * (2 * len(sl) + 2 + T // 64 + 1) + 256, dtype=torch.uint8, device=qkv.device)
     _check_op(lib().zo_op_attention(_ptr(qkv), _ptr(out), _ptr(sl), len(sl), n_heads, n_kv_heads,
                                  head_dim, dtype, _ptr(ws), ws.numel(), impl, _stream()))
