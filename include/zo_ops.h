@@ -166,7 +166,7 @@ int zo_op_lm_head_logprob(const void* h, const void* E, const int32_t* targets, 
  *   out      dev [T x H*hd] dtype
  *   seq_lens host int32 [n_rows], rows back to back in qkv
  *   workspace dev >= 4*(n_rows + 1 + T/64 + n_rows + 1) bytes (row offsets and tiles)
- *   impl     ZO_IMPL_TENSOR_CORES needs bf16 and head_dim 128; AUTO picks them then.
+ *   impl     ZO_IMPL_TENSOR_CORES needs bf16 and head_dim 64 or 128; AUTO picks them then.
  * The call copies the row offsets from the host and synchronises the stream. */
 int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t n_rows,
                     int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t dtype,

@@ -91,10 +91,13 @@ def test_qwen3_fp8_generation_matches_oracle():
 
 def test_opt_width_fp8_generation_matches_oracle():
     """E4M3 q|k|v and fc1 at OPT-1.3B width: the decode steps run them on the swapped
-    single-SM kernel with kind::f8f6f4 main blocks and the bf16 bank extension."""
+    single-SM kernel with kind::f8f6f4 main blocks and the bf16 bank extension.  The prefill's
+    attention (head_dim 64) runs on the tensor cores with P rounded to bf16; where that moves
+    a value of the next layer's input across an E4M3 code boundary (codes 12.5 % apart) a
+    token's log-prob moves by a few 1e-2, so the log-prob bound is the logit bound, 5e-2."""
     w = wl.WORKLOADS["opt-1.3b-b16"]
     w = dataclasses.replace(w, shape=wl.shrink_shape(w.shape, n_layers=2), batch=4, len_hi=48)
-    _check_against_oracle(w, True, 5e-2, 3e-2, 2e-2)
+    _check_against_oracle(w, True, 5e-2, 5e-2, 2e-2)
 
 
 @pytest.mark.parametrize("heads,kv_heads", [(6, 2), (8, 1)], ids=["group3", "group8"])

@@ -165,7 +165,11 @@ def test_lm_head_logprob(S, V, d, dtype, impl):
     # several items per persistent CTA, 1-5 key chunks each, in mixed order
     ([int(x) for x in np.random.default_rng(5).integers(1, 600, 40)], 8, 2, 128,
      torch.bfloat16, 2),
-    ([200, 1, 64], 8, 2, 64, torch.float32, 1)])
+    ([200, 1, 64], 8, 2, 64, torch.float32, 1),
+    # head_dim 64 on the tensor cores (OPT-1.3B's heads): one 64-column atom per tile
+    ([1, 5, 64, 65, 130, 300], 32, 32, 64, torch.bfloat16, 2),
+    ([int(x) for x in np.random.default_rng(6).integers(1, 400, 30)], 8, 2, 64,
+     torch.bfloat16, 2)])
 def test_attention_matches_oracle(lens, H, Hkv, hd, dtype, impl):
     from oracle import model as om
     from zeroth_order_fine_b200 import zo

@@ -133,6 +133,18 @@ def test_opt_13b_width_layer_full_batch_64_bf16_same_state_parity():
     _bf16_same_state_parity(w, shape, batch, pre_steps=1)
 
 
+def test_opt_6_7b_width_layer_full_batch_64_spans_bf16_same_state_parity():
+    """One full-width OPT-6.7B layer (d = 4096, FFN 16384, vocab 50272) over the whole seeded
+    batch of that workload: 64 prompts of 32-256 tokens, each scored on a 1-8-token span at
+    its end, LoZO r = 4 on q and v; L+- against the oracle at step 0 and after the oracle's
+    first update (its bank loaded)."""
+    w = wl.WORKLOADS["opt-6.7b-b64"]
+    shape = wl.shrink_shape(w.shape, n_layers=1)
+    batch = wl.make_batch(w)
+    assert batch.target_lens.max() > 1 and w.rank == 4
+    _bf16_same_state_parity(w, shape, batch, pre_steps=1)
+
+
 def test_tiny_bf16_many_rows_parity_and_cobatching():
     """160 physical rows of ~62 tokens (~9900 tokens, more 128-row tiles than CTA pairs): the
     bank shrink's CTA pairs each take a second tile, handing the split halves over twice;

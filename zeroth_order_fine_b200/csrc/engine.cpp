@@ -937,7 +937,7 @@ int prepare_batch(zo_handle* h, int B, const int32_t* lens, const int32_t* tls,
     int fo = 0;
     int r = 0, nt = 0;
     // attention tiles: 128 queries for the tensor-core kernel, 64 for the CUDA-core one
-    const bool tc_attn = h->use_tc && h->dt == E_BF16 && d.head_dim == 128;
+    const bool tc_attn = h->use_tc && h->dt == E_BF16 && (d.head_dim == 64 || d.head_dim == 128);
     const int qtile = tc_attn ? 128 : 64;
     for (int pass = 0; pass < 3; ++pass) {
         const int n = pass < 2 ? B : F;
@@ -1092,7 +1092,7 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
     const zo_model_desc& d = h->desc;
     const int R = bp.R, nt = bp.nt;
     const long long T = bp.T, S = bp.S;
-    const bool tc_attn = h->use_tc && h->dt == E_BF16 && d.head_dim == 128;
+    const bool tc_attn = h->use_tc && h->dt == E_BF16 && (d.head_dim == 64 || d.head_dim == 128);
     RowMeta m;
     m.cu_seqlens = md;
     m.row_src = md + (R + 1);
@@ -1219,7 +1219,7 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
     const size_t layer_elems = h->kv_rows * (size_t)kv2;
     const size_t es = esize(h->dt);
     auto cache = [&](int l) { return static_cast<char*>(h->kv_cache) + (size_t)l * layer_elems * es; };
-    const bool tc_attn = h->use_tc && h->dt == E_BF16 && d.head_dim == 128;
+    const bool tc_attn = h->use_tc && h->dt == E_BF16 && (d.head_dim == 64 || d.head_dim == 128);
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;
     const float scale = (float)(1.0 / std::sqrt((double)d.head_dim));
 

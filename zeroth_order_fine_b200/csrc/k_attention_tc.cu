@@ -1,4 +1,5 @@
-// Packed variable-length causal attention on the 5th-generation tensor cores.
+// Packed variable-length causal attention on the 5th-generation tensor cores (head_dim 64
+// or 128).
 //
 // Work items are (128-query tile of one row, head) pairs.  One persistent CTA per
 // SM walks its items in turn with its warps specialised:
@@ -31,9 +32,10 @@ ZO_DEBUG_WORD(debug_word_attention_tc)
 
 namespace {
 
-constexpr int TQ = 128, TK = 128, HD = 128;
+constexpr int TQ = 128, TK = 128;              // head_dim HD = 64 or 128 (template)
 constexpr int ATOM = TQ * 128;                  // bytes of one 64-column swizzle atom block
-constexpr int BUF = 2 * ATOM;                   // one [128 x 128] bf16 operand
+constexpr int BUF = 2 * ATOM;                   // one [128 x 128] bf16 operand (P is always
+                                                // 128 keys wide; Q, K, V fill HD / 64 atoms)
 // Q[3] K[2] V[2] buffers, then 23 mbarriers, the TMEM base and the abort flag
 constexpr int SMEM = 7 * BUF + 1024 + 256;
 constexpr int NTHREADS = 224;                   // Q/K producer, MMA issuer, 4 softmax warps,
@@ -158,10 +160,11 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                  : "memory");
 }
 
-// S = Q K^T: 8 MMAs (K = 128 = 2 swizzle atoms x 4 steps of 16) into TMEM at d_tmem.
+// S = Q K^T: HD / 16 MMAs (K = HD = HD / 64 swizzle atoms x 4 steps of 16) into TMEM at d_tmem.
+template <int HD>
 __device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint32_t q, uint32_t k) {
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
+    for (int kk = 0; kk < HD / 16; ++kk) {
         const uint32_t off = (kk >> 2) * ATOM + (kk & 3) * 32;
         const uint32_t acc = kk > 0 ? 1u : 0u;
         asm volatile(
@@ -183,8 +186,11 @@ __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
     d |= (uint64_t)2u << 61;
     return d;
 }
-// P.V: A = P (K-major, keys contiguous), B = V as loaded ([keys x dims], MN-major)
-constexpr uint32_t kIdescPV = kIdesc | (1u << 16);
+// P.V: A = P (K-major, keys contiguous), B = V as loaded ([keys x dims], MN-major); N = HD
+template <int HD>
+constexpr uint32_t idesc_pv() {
+    return (kIdesc & ~(0x3Fu << 17)) | ((uint32_t)(HD >> 3) << 17) | (1u << 16);
+}
 
 __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x,
                                         int y) {
@@ -287,7 +293,8 @@ __device__ __forceinline__ float ex2_ftz(float x) {
 }
 
 // O (+)= P V: A = P (K-major, keys contiguous) over the chunk's K buffer, B = V as loaded
-// ([keys x dims], MN-major); 8 MMAs of K = 16 keys.
+// ([keys x dims], MN-major); 8 MMAs of K = 16 keys, N = HD.
+template <int HD>
 __device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t pb, uint32_t vb, bool accum) {
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
@@ -297,7 +304,7 @@ __device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t pb, uint32_t vb
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-            "l"(ad), "l"(bd), "r"(kIdescPV), "r"(acc)
+            "l"(ad), "l"(bd), "r"(idesc_pv<HD>()), "r"(acc)
             : "memory");
     }
 }
@@ -306,8 +313,12 @@ __device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t pb, uint32_t vb
 // Chunks are numbered g = 0, 1, ... across the CTA's items: chunk g uses K/V stage g & 1
 // and S buffer g & 1; item k uses Q buffer and O buffer k & 1.  Phases follow from the
 // counters: the n-th use of a two-slot resource waits parity (n >> 1) & 1.
+template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
+    static_assert(HD == 64 || HD == 128, "head_dim");
+    constexpr int NATOM = HD / 64;              // swizzle atoms of a Q, K or V tile
+    constexpr uint32_t TILE_BYTES = TQ * HD * 2;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -387,8 +398,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!vk) {
                     const int qs = k % 3;
                     if (!wait_bar(q_empty(qs), ((k / 3) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
-                    bar_expect_tx(q_full(qs), BUF);
-                    for (int half = 0; half < 2; ++half)
+                    bar_expect_tx(q_full(qs), TILE_BYTES);
+                    for (int half = 0; half < NATOM; ++half)
                         tma_box(Qb(qs) + half * ATOM, &tm, q_full(qs), it.h * HD + half * 64,
                                 it.start + it.q0);
                     ++gq;
@@ -399,8 +410,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const uint32_t e = vk ? v_empty(st) : k_empty(st);
                     const uint32_t f = vk ? v_full(st) : k_full(st);
                     if (!wait_bar(e, ((gc >> 1) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
-                    bar_expect_tx(f, BUF);
-                    for (int half = 0; half < 2; ++half)
+                    bar_expect_tx(f, TILE_BYTES);
+                    for (int half = 0; half < NATOM; ++half)
                         tma_box((vk ? Vb(st) : Kb(st)) + half * ATOM, &tm, f, col + half * 64,
                                 it.start + c * TK);
                     ++gc;
@@ -425,7 +436,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (s_more && gs <= gp + 1 && (sc > 0 || bar_test(q_full(sk % 3), (sk / 3) & 1)) &&
                     bar_test(k_full(gs & 1), (gs >> 1) & 1)) {
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                    mma_qk(t_s(gs & 1), Qb(sk % 3), Kb(gs & 1));
+                    mma_qk<HD>(t_s(gs & 1), Qb(sk % 3), Kb(gs & 1));
                     tc_commit(s_full(gs & 1));
                     // the item's last chunk keeps its P in the Q buffer: its K is free now
                     if (sc == s_feed.cur.n_chunks - 1) tc_commit(k_empty(gs & 1));
@@ -443,7 +454,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     (pc > 0 || bar_test(o_free(pk & 1), ((pk >> 1) & 1) ^ 1u))) {
                     const bool last = pc == p_feed.cur.n_chunks - 1;
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                    mma_pv(t_o(pk & 1), last ? Qb(pk % 3) : Kb(gp & 1), Vb(gp & 1), pc > 0);
+                    mma_pv<HD>(t_o(pk & 1), last ? Qb(pk % 3) : Kb(gp & 1), Vb(gp & 1), pc > 0);
                     tc_commit(v_empty(gp & 1));          // V of the chunk is free
                     if (!last) tc_commit(k_empty(gp & 1));   // and its K buffer (held P)
                     issued = progress = true;
@@ -493,7 +504,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                                  (size_t)it.h * HD);
             const bool store = row < it.nq;
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < HD / 32; ++cc) {
                 float v[32];
                 tmem_ld32(t_o(os) + lane_addr + cc * 32, v);     // warp-collective: every lane
                 if (store) {
@@ -588,7 +599,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!wait_bar(v_empty(pv & 1), (pv >> 1) & 1, abort_f, err)) { ok = false; break; }
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll 1
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 0; cc < HD / 32; ++cc) {
                         float v[32];
                         tmem_ld32(t_o(os) + lane_addr + cc * 32, v);
 #pragma unroll
@@ -650,7 +661,8 @@ EncodeTiledFn attn_encode_fn() {
 }  // namespace
 
 bool attention_tc_supported(const AttnArgs& a) {
-    return a.dtype == E_BF16 && a.hd == HD && a.ld_qkv % 8 == 0 && a.ld_out % 8 == 0 &&
+    return a.dtype == E_BF16 && (a.hd == 64 || a.hd == 128) && a.ld_qkv % 8 == 0 &&
+           a.ld_out % 8 == 0 &&
            a.n_tokens > 0 && attn_encode_fn() != nullptr &&
            (reinterpret_cast<uintptr_t>(a.qkv) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
@@ -658,11 +670,15 @@ bool attention_tc_supported(const AttnArgs& a) {
 
 bool launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
     if (a.n_tiles == 0 || a.n_tokens <= 0) return true;
-    static cudaError_t attr = cudaErrorNotReady;
-    if (attr == cudaErrorNotReady)
-        attr = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    SMEM);
-    if (attr != cudaSuccess) return false;
+    if (a.hd != 64 && a.hd != 128) return false;
+    static cudaError_t attr[2] = {cudaErrorNotReady, cudaErrorNotReady};
+    cudaError_t& at = attr[a.hd == 128];
+    if (at == cudaErrorNotReady)
+        at = a.hd == 128 ? cudaFuncSetAttribute(attention_tc_kernel<128>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM)
+                         : cudaFuncSetAttribute(attention_tc_kernel<64>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (at != cudaSuccess) return false;
     // one map over the packed [T x ld_qkv] q|k|v rows: 64-column x 128-row boxes,
     // 128-byte swizzle, rows past T read as zero
     CUtensorMap tm;
@@ -686,7 +702,10 @@ bool launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
             sms = 148;
     }
     const unsigned grid = (unsigned)(items < sms ? items : sms);
-    attention_tc_kernel<<<grid, NTHREADS, SMEM, st>>>(tm, a);
+    if (a.hd == 128)
+        attention_tc_kernel<128><<<grid, NTHREADS, SMEM, st>>>(tm, a);
+    else
+        attention_tc_kernel<64><<<grid, NTHREADS, SMEM, st>>>(tm, a);
     return true;
 }
 

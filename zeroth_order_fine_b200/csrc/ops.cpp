@@ -179,7 +179,7 @@ int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t
     if (n_rows >= 32768) return ZO_ERR_ARG;
     std::vector<int> meta(n_rows + 1);
     meta[0] = 0;
-    const bool tc = use_tc(impl, dtype) && head_dim == 128;
+    const bool tc = use_tc(impl, dtype) && (head_dim == 64 || head_dim == 128);
     if (impl == ZO_IMPL_TENSOR_CORES && !tc) return ZO_ERR_UNSUPPORTED;
     const int qtile = tc ? 128 : 64;
     std::vector<int> tiles;
