@@ -169,7 +169,10 @@ def test_lm_head_logprob(S, V, d, dtype, impl):
     # head_dim 64 on the tensor cores (OPT-1.3B's heads): one 64-column atom per tile
     ([1, 5, 64, 65, 130, 300], 32, 32, 64, torch.bfloat16, 2),
     ([int(x) for x in np.random.default_rng(6).integers(1, 400, 30)], 8, 2, 64,
-     torch.bfloat16, 2)])
+     torch.bfloat16, 2),
+    # rows at OPT's longest position (2048 tokens: 16 query tiles of up to 16 key chunks)
+    ([2048, 1, 1500], 4, 2, 128, torch.bfloat16, 2),
+    ([2048, 700], 4, 4, 64, torch.bfloat16, 2)])
 def test_attention_matches_oracle(lens, H, Hkv, hd, dtype, impl):
     from oracle import model as om
     from zeroth_order_fine_b200 import zo
