@@ -252,7 +252,9 @@ int zo_score_cobatch(zo_plan* plan, const int32_t* packed_tokens, int32_t n_prom
                      const int32_t* fg_seq_lens, const int32_t* fg_target_lens,
                      float* fg_tok_logprob);
 
-/* Foreground rows alone under theta_t (the "scored alone" counterpart). */
+/* Foreground rows alone under theta_t (the "scored alone" counterpart).  It
+ * may run between a plan's scoring and its zo_step: the plan's objectives,
+ * and so the step's c, are left as they were. */
 int zo_score_foreground(zo_handle* h, const int32_t* fg_tokens, int32_t n_fg,
                         const int32_t* fg_seq_lens, const int32_t* fg_target_lens,
                         float* fg_tok_logprob);

@@ -165,6 +165,28 @@ def test_tiny_bf16_many_rows_parity_and_cobatching():
         h.zo_step(w.lr)
 
 
+@pytest.mark.parametrize("wk", ["tiny", "tiny-bf16"])
+def test_foreground_scoring_between_score_and_step_leaves_the_step_alone(wk):
+    """A serving-style zo_score_foreground between a plan's scoring and its zo_step must not
+    touch the plan's objectives: c and the bank equal those of a handle that never served."""
+    w = dataclasses.replace(TINY if wk == "tiny" else TINY_BF16, fg_rows=4)
+    batch = wl.make_batch(w)
+    toks, ftoks = dev_tokens(batch), dev_fg_tokens(batch)
+    _, ha = gpu_handle(w, fg=4)
+    _, hb = gpu_handle(w, fg=4)
+    for t in range(3):
+        cs = []
+        for h, serve in ((ha, True), (hb, False)):
+            h.zo_probe_plan(t, w.eps)
+            h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, ftoks,
+                               batch.fg_seq_lens, batch.fg_target_lens)
+            if serve:
+                h.zo_score_foreground(ftoks, batch.fg_seq_lens, batch.fg_target_lens)
+            cs.append(h.zo_step(w.lr))
+        assert cs[0] == cs[1], (t, cs)
+    assert ha.zo_save_state() == hb.zo_save_state()
+
+
 def test_qwen3_bf16_same_state_parity():
     shape = dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16)
     w = dataclasses.replace(QWEN_SMALL, shape=shape, fg_rows=0)

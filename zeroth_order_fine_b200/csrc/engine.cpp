@@ -1329,8 +1329,12 @@ static int score_common(zo_plan* plan, zo_handle* h, const int32_t* ptok, int32_
     long long Sp = 0, Sf = 0;
     for (int i = 0; i < B; ++i) Sp += tls[i];
     for (int i = 0; i < F; ++i) Sf += ftls[i];
-    launch_row_objective(h->logprob, soff_d, R, B, 2 * Sp + Sf, h->L_row, Lp, Lm, h->st);
-    h->stats.kernel_launches++;
+    // the row objectives feed the estimate of a scored plan; a foreground-only call has none,
+    // and must leave those of a plan scored earlier for its zo_step
+    if (B > 0) {
+        launch_row_objective(h->logprob, soff_d, R, B, 2 * Sp + Sf, h->L_row, Lp, Lm, h->st);
+        h->stats.kernel_launches++;
+    }
     if (tok_lp && Sp)
         CK(h, cudaMemcpyAsync(tok_lp, h->logprob, 2 * Sp * 4, cudaMemcpyDeviceToDevice, h->st));
     if (fg_lp && Sf)
