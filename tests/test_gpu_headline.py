@@ -1,10 +1,12 @@
-"""The headline configuration at its full size, through the calls bench.py times.
+"""The headline configuration at its full size, through the calls bench.py times, and the
+OPT-6.7B batch-64 configuration beside it.
 
 OPT-13B shape (40 layers, d = 5120, vocab 50272, bf16, random init drawn on the device), the
-seeded batch of 64 ragged prompts (128 physical rows, 9196 tokens), LoZO r = 2 on q and v.
-The float64 oracle cannot hold this model (13 B parameters), so the full-size checks are
-properties that fix the result at any size; the oracle itself checks one full-width layer
-over this same batch (test_gpu_step.py):
+seeded batch of 64 ragged prompts (128 physical rows, 9196 tokens), LoZO r = 2 on q and v;
+OPT-6.7B shape (32 layers, d = 4096) on its batch of 64 prompts of 32-256 tokens, each scored
+on a 1-8-token span, LoZO r = 4.  The float64 oracle cannot hold these models, so the
+full-size checks are properties that fix the result at any size; the oracle itself checks
+one full-width layer of each over the same batch (test_gpu_step.py):
 
 * eps = 0 makes every + row and its - row the same computation: L+ == L- bit for bit;
 * the step is deterministic: the same plan scored twice gives the same bits;
@@ -24,13 +26,13 @@ from gpu_util import dev_fg_tokens, dev_tokens, needs_gpu
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
-W = wl.WORKLOADS["opt-13b-b64"]
 FG = 8
 
 
-@pytest.fixture(scope="module")
-def headline():
+@pytest.fixture(scope="module", params=["opt-13b-b64", "opt-6.7b-b64"])
+def headline(request):
     from zeroth_order_fine_b200 import zo
+    W = wl.WORKLOADS[request.param]
     batch = wl.make_batch(W)
     assert batch.n_tokens_physical == sum(2 * len(p) for p in batch.prompts) > 9000
     model = zo.DeviceModel(W.shape, W.weight_seed)
@@ -39,15 +41,16 @@ def headline():
     fg_tokens = int(sum(len(p) for p in batch.prompts[:FG]))
     h = zo.Handle(model, W.run_seed, W.nu, W.rank, tg,
                   max_tokens=batch.n_tokens_physical + fg_tokens + 64, max_rows=2 * B + FG,
-                  max_scored=2 * int(batch.target_lens.sum()) + FG, max_slots=4)
-    yield batch, h
+                  max_scored=2 * int(batch.target_lens.sum()) + int(batch.target_lens[:FG].sum()),
+                  max_slots=4)
+    yield W, batch, h
     h.close()
     del model
     torch.cuda.empty_cache()
 
 
 def test_eps_zero_rows_are_bitwise_equal_and_scoring_is_deterministic(headline):
-    batch, h = headline
+    W, batch, h = headline
     toks = dev_tokens(batch)
     h.zo_probe_plan(0, 0.0)
     Lp, Lm, lp = h.zo_score(toks, batch.seq_lens, batch.target_lens, want_logprob=True)
@@ -62,7 +65,7 @@ def test_eps_zero_rows_are_bitwise_equal_and_scoring_is_deterministic(headline):
 
 
 def test_estimate_and_first_two_bank_updates_at_full_size(headline):
-    batch, h = headline
+    W, batch, h = headline
     toks = dev_tokens(batch)
     state0 = h.zo_save_state()
     coefs = []
@@ -96,7 +99,7 @@ def test_estimate_and_first_two_bank_updates_at_full_size(headline):
 
 
 def test_cobatched_foreground_rows_are_bitwise_alone_at_full_size(headline):
-    batch, h = headline
+    W, batch, h = headline
     toks = dev_tokens(batch)
     fg = wl.Batch(batch.prompts, batch.target_lens, list(batch.prompts[:FG]),
                   np.asarray(batch.target_lens[:FG], dtype=np.int32))
