@@ -147,3 +147,55 @@ def test_out_of_range_token_ids_are_rejected_on_the_device(bad):
     c = h.zo_step(w.lr)
     assert np.isfinite(c)
     h.close()
+
+
+def test_capacity_limits_are_refused_and_leave_no_trace():
+    """Batches past the handle's sizes (rows, tokens, scored positions), rows too short to
+    score and an empty batch are refused with ZO_ERR_ARG before any launch; the handle then
+    steps exactly like a fresh one."""
+    from zeroth_order_fine_b200 import zo
+    from gpu_util import dev_tokens, gpu_handle
+    w = wl.WORKLOADS["tiny"]
+    batch = wl.make_batch(w)
+    B = len(batch.prompts)
+    T = int(batch.seq_lens.sum())
+    model = zo.DeviceModel(w.shape, w.weight_seed)
+    tg = zo.make_targets(w.shape.n_layers, w.matrices, w.scale_mode)
+
+    def handle():
+        return zo.Handle(model, w.run_seed, w.nu, w.rank, tg, max_tokens=2 * T, max_rows=2 * B,
+                         max_scored=2 * int(batch.target_lens.sum()))
+
+    h, ref = handle(), handle()
+    toks = dev_tokens(batch)
+    h.zo_probe_plan(0, w.eps)
+    rng = np.random.default_rng(3)
+    cases = {
+        "more rows than max_rows": list(batch.prompts) + [batch.prompts[0]],
+        # rows of max_pos tokens: twice the physical tokens the handle was sized for
+        "more tokens than max_tokens": [np.concatenate([p, p]) for p in batch.prompts],
+    }
+    for msg, prompts in cases.items():
+        b = wl.Batch(prompts, np.ones(len(prompts), np.int32), [], np.zeros(0, np.int32))
+        with pytest.raises(zo.ZoError) as e:
+            h.zo_score(dev_tokens(b), b.seq_lens, b.target_lens)
+        assert e.value.code == zo.ZO_ERR_ARG and msg in str(e.value), str(e.value)
+    wide = batch.target_lens.copy() + 1                       # one more scored position each
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_score(toks, batch.seq_lens, np.minimum(wide + 4, batch.seq_lens - 1))
+    assert e.value.code == zo.ZO_ERR_ARG and "max_scored" in str(e.value)
+    short = wl.Batch([rng.integers(0, w.shape.vocab, 1).astype(np.int32)], np.ones(1, np.int32),
+                     [], np.zeros(0, np.int32))
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_score(dev_tokens(short), short.seq_lens, short.target_lens)
+    assert e.value.code == zo.ZO_ERR_ARG
+    with pytest.raises(zo.ZoError) as e:
+        h.zo_score(toks[:0], np.zeros(0, np.int32), np.zeros(0, np.int32))
+    assert e.value.code == zo.ZO_ERR_ARG
+    for hh in (h, ref):
+        hh.zo_probe_plan(0, w.eps)
+        hh.zo_score(toks, batch.seq_lens, batch.target_lens)
+    assert h.zo_step(w.lr) == ref.zo_step(w.lr)
+    assert h.zo_save_state() == ref.zo_save_state()
+    h.close()
+    ref.close()
