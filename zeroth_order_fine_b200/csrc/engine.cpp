@@ -22,6 +22,7 @@
 // "The System Reorganization"; "Inference-Native Zeroth-Order Optimization",
 // abstract: factorised side states, persistent banks, frozen base weights).
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>   // header-only: ranges cost nothing unless a profiler is attached
 
 #include <algorithm>
 #include <cmath>
@@ -72,6 +73,7 @@ struct PhaseTimer {
     int head = 0, tail = 0;   // [tail, head) pending
     double total_ms = 0.0;
     bool init = false;
+    nvtxRangeId_t range = 0;  // the phase's open NVTX range
 };
 
 // Per-launch GEMM timing (options.profile): event pairs in a ring, harvested
@@ -301,8 +303,12 @@ void prof_harvest(GemmProfiler& p, bool wait) {
 int prof_begin(zo_handle* h);
 void prof_end(zo_handle* h, int slot, double flops, bool tc);
 
+// Each phase (plan, score, step) is also an NVTX range, so a timeline profiler shows the
+// step's structure on the host thread.
 void timer_begin(zo_handle* h, int ph) {
+    static const char* const kPhase[3] = {"zo_probe_plan", "zo_score", "zo_step"};
     PhaseTimer& t = h->tm[ph];
+    t.range = nvtxRangeStartA(kPhase[ph]);   // start/end pairs: an error return leaves no stack
     if (!t.init) {
         for (int i = 0; i < PhaseTimer::kRing; ++i) {
             cudaEventCreate(&t.a[i]);
@@ -319,6 +325,7 @@ void timer_end(zo_handle* h, int ph) {
     PhaseTimer& t = h->tm[ph];
     cudaEventRecord(t.b[t.head % PhaseTimer::kRing], h->st);
     t.head++;
+    nvtxRangeEnd(t.range);
 }
 
 int prof_begin(zo_handle* h) {
