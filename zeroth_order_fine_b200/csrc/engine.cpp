@@ -983,12 +983,18 @@ int prepare_batch(zo_handle* h, int B, const int32_t* lens, const int32_t* tls,
 // it can be captured into a CUDA graph.
 // One fused GEMM group of a layer over Ti token rows: the bank shrink (when the group
 // carries targets) and the base GEMM with the extension K blocks, epilogue epi.
+// nn (decode steps, EPI_RESID): the norm of the updated residual rows that comes next; it runs
+// fused into the split reduction when that path is taken, else right after the GEMM.
 int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc, int ctype,
-               int Ti, float eps, const Layer* Lq = nullptr, bool decode = false) {
+               int Ti, float eps, const Layer* Lq = nullptr, bool decode = false,
+               const NormNext* nn = nullptr) {
     const zo_model_desc& d = h->desc;
     const int r_ = h->opt.rank;
     GemmArgs g;
     memset(&g, 0, sizeof(g));
+    int norm_done = 0;
+    g.norm_next = nn;
+    g.norm_done = &norm_done;
     if (epi == EPI_QKNR) {
         g.tok_pos = h->tok_pos; g.qn = Lq->w.q_norm; g.kn = Lq->w.k_norm;
         g.rope_cos = h->rope_cos; g.rope_sin = h->rope_sin; g.norm_eps = d.norm_eps;
@@ -1052,7 +1058,12 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
     // algorithmic work: the base GEMM plus, per target, its own expand columns
     double fl = 2.0 * Ti * (double)G.N * G.K;
     for (int t = 0; t < G.n_t; ++t) fl += 2.0 * Ti * (double)G.d_out[t] * r_ * (1 + h->n_slots);
-    return run_gemm(h, g, fl);
+    const int rc = run_gemm(h, g, fl);
+    if (rc || !nn || norm_done) return rc;
+    launch_norm(static_cast<const float*>(C), nullptr, Ti, G.N, nn->kind, nn->w, nn->b, nn->eps,
+                nn->out, nn->out_type, h->st, nn->q8, nn->s8, decode);
+    h->stats.kernel_launches++;
+    return ZO_OK;
 }
 
 // Every decoder layer over the Ti token rows whose ids, positions, signs and embeddings are
@@ -1062,10 +1073,13 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
                    bool decode = false) {
     const zo_model_desc& d = h->desc;
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
+    // decode steps: each residual GEMM also applies the norm that follows it (ln2 after o, the
+    // next layer's ln1 or the final norm after the FFN), fused into its split reduction
     for (int l = 0; l < d.n_layers; ++l) {
         Layer& L = h->layers[l];
-        launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps, h->xn,
-                    h->dt, h->st, h->xq, h->sx, decode);
+        if (!decode || l == 0)
+            launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps,
+                        h->xn, h->dt, h->st, h->xq, h->sx, decode);
         int rc = group_gemm(h, L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
                             h->n_qkv, h->dt, Ti, eps, &L, decode);
         if (rc) return rc;
@@ -1075,10 +1089,13 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
                                 h->rope_sin, h->st);
         rc = attn(l);
         if (rc) return rc;
-        rc = group_gemm(h, L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr, decode);
+        const NormNext ln2 = {L.w.ln2_w, L.w.ln2_b, nk, d.norm_eps, h->xn, h->dt, h->xq, h->sx};
+        rc = group_gemm(h, L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr,
+                        decode, decode ? &ln2 : nullptr);
         if (rc) return rc;
-        launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps, h->xn,
-                    h->dt, h->st, h->xq, h->sx, decode);
+        if (!decode)
+            launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln2_w, L.w.ln2_b, d.norm_eps,
+                        h->xn, h->dt, h->st, h->xq, h->sx);
         if (d.arch == ZO_ARCH_OPT) {
             rc = group_gemm(h, L.g[G_IN], h->xn, EPI_STORE_RELU, h->act, d.d_ffn, h->dt, Ti, eps, nullptr, decode);
         } else if (h->swiglu_fused) {
@@ -1088,7 +1105,15 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
             if (!rc) launch_swiglu(h->gu, Ti, d.d_ffn, h->act, h->dt, h->st);
         }
         if (rc) return rc;
-        rc = group_gemm(h, L.g[G_OUT], h->act, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr, decode);
+        NormNext next;
+        if (l + 1 < d.n_layers) {
+            const Layer& N1 = h->layers[l + 1];
+            next = {N1.w.ln1_w, N1.w.ln1_b, nk, d.norm_eps, h->xn, h->dt, h->xq, h->sx};
+        } else {
+            next = {h->wts.final_w, h->wts.final_b, nk, d.norm_eps, h->hs, h->dt, nullptr, nullptr};
+        }
+        rc = group_gemm(h, L.g[G_OUT], h->act, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr,
+                        decode, decode ? &next : nullptr);
         if (rc) return rc;
     }
     return ZO_OK;
@@ -1290,8 +1315,7 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
             return ZO_OK;
         }, true);
         if (rc) return rc;
-        launch_norm(h->resid, nullptr, R, d.d_model, nk, h->wts.final_w, h->wts.final_b,
-                    d.norm_eps, h->hs, h->dt, h->st);
+        // (the final norm of the R rows into hs ran with the last layer's FFN reduction)
         rc = lm_head_greedy(h, R, h->gen_tok + g + 1, h->gen_lp + g + 1, G);
         if (rc) return rc;
         h->stats.kernel_launches += 3 + (uint64_t)d.n_layers * (2 + (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused) +

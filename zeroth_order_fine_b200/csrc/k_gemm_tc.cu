@@ -1729,6 +1729,12 @@ int launch_split_reduce(const GemmArgs& g, const TcParams& p, int ks, cudaStream
         const long long warps = (long long)g.M * (g.N / 128);
         go(splitk_qknr_kernel, dim3((unsigned)((warps + 3) / 4)), (const float*)g.ws, ks, g.M, g.N,
            p, static_cast<__nv_bfloat16*>(g.C), g.ldc);
+    } else if (g.epi == EPI_RESID && g.norm_next &&
+               launch_splitk_resid_norm(g.ws, ks, g.M, g.N, g.bias, static_cast<float*>(g.C),
+                                        g.ldc, *g.norm_next, st, pdl)) {
+        // the residual rows and the next norm in one pass
+        e = cudaGetLastError();
+        if (g.norm_done) *g.norm_done = 1;
     } else {
         go(splitk_epilogue_kernel, dim3((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M),
            (const float*)g.ws, ks, g.M, g.N, g.bias, g.epi, g.C, g.ldc);

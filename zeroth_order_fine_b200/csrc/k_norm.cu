@@ -132,30 +132,20 @@ __global__ void __launch_bounds__(256) norm_kernel(const float* __restrict__ x,
 // (VPT float4 per thread), 16-byte loads, 8-byte bf16 stores.
 // With q8: the bf16 output row is also quantised to E4M3 with one scale per row
 // (amax / 448), from the bf16-rounded values, for the FP8 base GEMMs.
+// Normalise one row held by the CTA's 256 threads as float4s (v[i] = elements 4j..4j+3, j =
+// threadIdx.x + 256 i; s = their per-thread partial sum, or sum of squares for RMSNorm) and
+// write output row t: LayerNorm (x - mean) / sqrt(var + eps) * w + b (kind 0) or RMSNorm
+// x / sqrt(mean(x^2) + eps) * w (kind 1), statistics in fp32 with a two-pass variance, then
+// (q8) the E4M3 codes and scale of the bf16-rounded row.  Shared by the norm kernel and the
+// residual reduction that fuses the next norm, so both give the same bits.
 template <int VPT>
-__global__ void __launch_bounds__(256) norm_vec_kernel(const float* __restrict__ x,
-                                                       const int* __restrict__ rows, int d,
-                                                       int kind, const float* __restrict__ w,
-                                                       const float* __restrict__ b, float eps,
-                                                       void* __restrict__ out, int out_type,
-                                                       uint8_t* __restrict__ q8,
-                                                       float* __restrict__ s8) {
-    grid_dep_wait();                    // a no-op unless launched as a programmatic dependent
-    grid_dep_launch();
-    __shared__ float red[32];
-    const int t = blockIdx.x;
-    const int src = rows ? rows[t] : t;
-    const float4* xr = reinterpret_cast<const float4*>(x + (size_t)src * d);
+__device__ __forceinline__ void norm_row_finish(float4 (&v)[VPT], float s, int t, int d, int kind,
+                                                const float* __restrict__ w,
+                                                const float* __restrict__ b, float eps,
+                                                void* __restrict__ out, int out_type,
+                                                uint8_t* __restrict__ q8, float* __restrict__ s8,
+                                                float* red) {
     const int n4 = d >> 2;
-    float4 v[VPT];
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        const int j = threadIdx.x + i * 256;
-        v[i] = j < n4 ? xr[j] : make_float4(0.f, 0.f, 0.f, 0.f);
-        s += kind == 0 ? (v[i].x + v[i].y) + (v[i].z + v[i].w)
-                       : (v[i].x * v[i].x + v[i].y * v[i].y) + (v[i].z * v[i].z + v[i].w * v[i].w);
-    }
     s = block_sum(s, red);
     float mean = 0.f, rstd;
     if (kind == 0) {
@@ -226,6 +216,84 @@ __global__ void __launch_bounds__(256) norm_vec_kernel(const float* __restrict__
     }
 }
 
+template <int VPT>
+__global__ void __launch_bounds__(256) norm_vec_kernel(const float* __restrict__ x,
+                                                       const int* __restrict__ rows, int d,
+                                                       int kind, const float* __restrict__ w,
+                                                       const float* __restrict__ b, float eps,
+                                                       void* __restrict__ out, int out_type,
+                                                       uint8_t* __restrict__ q8,
+                                                       float* __restrict__ s8) {
+    grid_dep_wait();                    // a no-op unless launched as a programmatic dependent
+    grid_dep_launch();
+    __shared__ float red[32];
+    const int t = blockIdx.x;
+    const int src = rows ? rows[t] : t;
+    const float4* xr = reinterpret_cast<const float4*>(x + (size_t)src * d);
+    const int n4 = d >> 2;
+    float4 v[VPT];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int j = threadIdx.x + i * 256;
+        v[i] = j < n4 ? xr[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+        s += kind == 0 ? (v[i].x + v[i].y) + (v[i].z + v[i].w)
+                       : (v[i].x * v[i].x + v[i].y * v[i].y) + (v[i].z * v[i].z + v[i].w * v[i].w);
+    }
+    norm_row_finish<VPT>(v, s, t, d, kind, w, b, eps, out, out_type, q8, s8, red);
+}
+
+// Residual reduction of a split-K GEMM with the next norm fused: row m of C (the fp32
+// residual) gains sum_s slice_s[m] + bias, added slice by slice in split order exactly as the
+// plain reduction adds them, and the updated row, still in registers, is normalised into the
+// norm's output row m.  One CTA per row, 256 threads.
+template <int VPT>
+__global__ void __launch_bounds__(256) splitk_resid_norm_kernel(
+    const float* __restrict__ ws, int ks, int M, int N, const float* __restrict__ bias,
+    float* __restrict__ C, int ldc, const float* __restrict__ w, const float* __restrict__ b,
+    int kind, float eps, void* __restrict__ out, int out_type, uint8_t* __restrict__ q8,
+    float* __restrict__ s8) {
+    grid_dep_wait();                    // a no-op unless launched as a programmatic dependent
+    grid_dep_launch();
+    __shared__ float red[32];
+    const int m = blockIdx.x;
+    const int n4 = N >> 2;
+    float4* crow = reinterpret_cast<float4*>(C + (size_t)m * ldc);
+    const float4* b4 = reinterpret_cast<const float4*>(bias);
+    float4 v[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    // slices in split order; each slice's VPT loads per thread are independent, so they (and,
+    // unrolled, those of the next slices) are in flight together
+#pragma unroll 2
+    for (int sl = 0; sl < ks; ++sl) {
+        const float4* p4 = reinterpret_cast<const float4*>(ws + ((size_t)sl * M + m) * N);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int j = threadIdx.x + i * 256;
+            if (j < n4) {
+                const float4 p = p4[j];
+                v[i].x += p.x; v[i].y += p.y; v[i].z += p.z; v[i].w += p.w;
+            }
+        }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int j = threadIdx.x + i * 256;
+        if (j < n4) {
+            const float4 bb = bias ? b4[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 c = crow[j];
+            c.x += v[i].x + bb.x; c.y += v[i].y + bb.y; c.z += v[i].z + bb.z; c.w += v[i].w + bb.w;
+            crow[j] = c;
+            v[i] = c;
+        }
+        s += kind == 0 ? (v[i].x + v[i].y) + (v[i].z + v[i].w)
+                       : (v[i].x * v[i].x + v[i].y * v[i].y) + (v[i].z * v[i].z + v[i].w * v[i].w);
+    }
+    norm_row_finish<VPT>(v, s, m, N, kind, w, b, eps, out, out_type, q8, s8, red);
+}
+
 // One CTA per row: amax, then the codes (used for the frozen weights at set-up).
 __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const void* __restrict__ x,
                                                               int x_type, int cols, size_t ldx,
@@ -265,6 +333,39 @@ void norm_vec_go(bool pdl, int T, cudaStream_t st, const float* x, const int* ro
                    out, out_type, q8, s8);
     else
         norm_vec_kernel<VPT><<<T, 256, 0, st>>>(x, rows, d, kind, w, b, eps, out, out_type, q8, s8);
+}
+
+template <int VPT>
+void resid_norm_go(bool pdl, const float* ws, int ks, int M, int N, const float* bias, float* C,
+                   int ldc, const NormNext& nn, cudaStream_t st) {
+    if (pdl)
+        launch_pdl(splitk_resid_norm_kernel<VPT>, dim3(M), dim3(256), 0, st, ws, ks, M, N, bias, C,
+                   ldc, nn.w, nn.b, nn.kind, nn.eps, nn.out, nn.out_type, nn.q8, nn.s8);
+    else
+        splitk_resid_norm_kernel<VPT><<<M, 256, 0, st>>>(ws, ks, M, N, bias, C, ldc, nn.w, nn.b,
+                                                         nn.kind, nn.eps, nn.out, nn.out_type,
+                                                         nn.q8, nn.s8);
+}
+
+bool launch_splitk_resid_norm(const float* ws, int ks, int M, int N, const float* bias, float* C,
+                              int ldc, const NormNext& nn, cudaStream_t st, bool pdl) {
+    if (M == 0) return true;
+    const int vpt = (N / 4 + 255) / 256;
+    auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (N % 4 || ldc % 4 || vpt > 8 || !al16(ws) || !al16(C) || !al16(nn.w) ||
+        (nn.b && !al16(nn.b)) || (bias && !al16(bias)) || !al16(nn.out))
+        return false;
+    switch (vpt) {
+        case 1: resid_norm_go<1>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+        case 2: resid_norm_go<2>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+        case 3: resid_norm_go<3>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+        case 4: resid_norm_go<4>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+        case 5: resid_norm_go<5>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+        case 6: resid_norm_go<6>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+        case 7: resid_norm_go<7>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+        default: resid_norm_go<8>(pdl, ws, ks, M, N, bias, C, ldc, nn, st); break;
+    }
+    return true;
 }
 
 void launch_norm(const float* x, const int* rows, int T, int d, int kind, const float* w,

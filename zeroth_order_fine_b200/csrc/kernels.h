@@ -88,6 +88,14 @@ enum Epi : int {
                          // rotary positions from the tables; v heads are stored as they are
 };
 
+// The norm that follows a residual GEMM (decode steps): fused into its split-K reduction.
+struct NormNext {
+    const float* w; const float* b;         // norm weight, bias (LayerNorm) or NULL
+    int kind; float eps;                    // 0 LayerNorm, 1 RMSNorm
+    void* out; int out_type;                // normalised rows [M x N]
+    uint8_t* q8; float* s8;                 // optional E4M3 rows and scales of the output
+};
+
 struct GemmArgs {
     const void* A; int lda; int a_type;     // [M x K], K contiguous
     const void* B; int ldb; int b_type;     // [N x K], K contiguous
@@ -118,7 +126,14 @@ struct GemmArgs {
     // reduction sums the slices in order and applies the epilogue.  Callers give at least
     // M x N floats (one slice); more room allows more splits.
     float* ws; size_t ws_floats;
+    // EPI_RESID with a split reduction: the reduction may also apply norm_next to each updated
+    // row of C (the fp32 residual); it then sets *norm_done = 1 (else the caller runs the norm)
+    const NormNext* norm_next; int* norm_done;
 };
+// Split-K residual reduction with the next norm fused (see NormNext); false when the shape or
+// alignment is outside the vectorised form (nothing launched).
+bool launch_splitk_resid_norm(const float* ws, int ks, int M, int N, const float* bias, float* C,
+                              int ldc, const NormNext& nn, cudaStream_t st, bool pdl);
 
 void gemm_simt(const GemmArgs& g, cudaStream_t st);
 // tcgen05 / TMEM / TMA path; returns false when the shape is outside its limits.
