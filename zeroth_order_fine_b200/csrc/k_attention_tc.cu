@@ -3,18 +3,21 @@
 //
 // Work items are (128-query tile of one row, head) pairs.  One persistent CTA per
 // SM walks its items in turn with its warps specialised:
-//   warp 0      TMA producer: Q of an item, then K and V of each 128-key chunk,
-//               into two stages of 128-byte-swizzled shared-memory buffers
+//   warp 0      TMA producer of Q (three buffers, one per item in flight) and of K
+//               (two stages, one per 128-key chunk), 128-byte-swizzled
+//   warp 6      TMA producer of V (two stages)
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
-//                 S = Q K^T      M=128 N=128 K=128 into one of two TMEM S buffers
-//                 O (+)= P V     into one of two TMEM O buffers (one per item in flight)
+//                 S = Q K^T      M=128 N=128 K=HD into one of two TMEM S buffers
+//                 O (+)= P V     N=HD into one of two TMEM O buffers (one per item in flight)
 //               S of the next chunk is issued while the softmax works on this one
 //   warps 2..5  softmax and epilogue, one query row per thread (= its TMEM lane):
 //               P = exp(S*scale - m) with the causal and row-end masks, written as
-//               bf16 over the chunk's K buffer in the swizzled K-major layout; across
-//               chunks the softmax is online (running max and sum in registers, the
-//               output rescaled in TMEM); at the item's end O / l goes to memory
-// So the next item's loads and its Q K^T overlap this item's softmax and store.
+//               bf16 in the swizzled K-major layout over the chunk's K buffer, or over
+//               the item's Q buffer for its last chunk (so that K buffer frees once S
+//               retires); across chunks the softmax is online (running max and sum in
+//               registers, the output rescaled in TMEM); an item's O / l goes to memory
+//               after the next item's softmax (the item's own P V runs meanwhile)
+// So the next items' loads and Q K^T overlap this item's softmax and the last item's store.
 // Queries, keys and values arrive by TMA straight from the packed q|k|v rows (Qwen3's
 // q/k norm and rotary positions were applied beforehand).  Keys past the row's end
 // get zero probability, so a query's result depends only on its own row: packing
@@ -311,7 +314,7 @@ __device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t pb, uint32_t vb
 
 // Persistent: CTA b takes items b, b + gridDim.x, ... (dealt longest first by the host).
 // Chunks are numbered g = 0, 1, ... across the CTA's items: chunk g uses K/V stage g & 1
-// and S buffer g & 1; item k uses Q buffer and O buffer k & 1.  Phases follow from the
+// and S buffer g & 1; item k uses Q buffer k % 3 and O buffer k & 1.  Phases follow from the
 // counters: the n-th use of a two-slot resource waits parity (n >> 1) & 1.
 template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
