@@ -187,6 +187,29 @@ def test_foreground_scoring_between_score_and_step_leaves_the_step_alone(wk):
     assert ha.zo_save_state() == hb.zo_save_state()
 
 
+def test_qwen3_head_dim_64_bf16_same_state_parity_and_cobatching():
+    """A Qwen3-family model with 64-wide heads (8 query / 4 kv heads over d = 512): the q/k
+    norm and rotary positions run as their own kernel (the fused epilogue takes 128-wide
+    heads) and attention on the tensor cores' head_dim-64 form; L+- against the oracle on
+    the same state, and co-batched foreground rows bit-identical to alone."""
+    shape = wl.ModelShape("qwen3-hd64", wl.ARCH_QWEN3, 2, 512, 8, 4, 64, 1024, 1000, 4096, 1e-6,
+                          1e6, wl.DTYPE_BF16, False)
+    w = dataclasses.replace(QWEN_SMALL, shape=shape, fg_rows=0)
+    _bf16_same_state_parity(w, shape, wl.make_batch(w, fg_rows=0), pre_steps=3)
+    wf = dataclasses.replace(QWEN_SMALL, shape=shape, fg_rows=4)
+    batch = wl.make_batch(wf)
+    _, h = gpu_handle(wf, shape=shape, fg=4)
+    toks, ftoks = dev_tokens(batch), dev_fg_tokens(batch)
+    for t in range(2):
+        h.zo_probe_plan(t, wf.eps)
+        _, _, _, flp = h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, ftoks,
+                                          batch.fg_seq_lens, batch.fg_target_lens)
+        assert torch.equal(flp, h.zo_score_foreground(ftoks, batch.fg_seq_lens,
+                                                      batch.fg_target_lens))
+        h.zo_step(wf.lr)
+    assert h.zo_stats()["cuda_core_gemm_launches"] == 0
+
+
 def test_qwen3_bf16_same_state_parity():
     shape = dataclasses.replace(Q3_SMALL, dtype=wl.DTYPE_BF16)
     w = dataclasses.replace(QWEN_SMALL, shape=shape, fg_rows=0)
