@@ -127,3 +127,22 @@ def test_debug_build_exports_the_same_symbols_and_says_so(built_lib):
     missing = [n for n in sorted(declared_functions()) if not hasattr(dbg, n)]
     assert not missing, missing
     assert dbg.zo_debug_build() == 1 and built_lib.zo_debug_build() == 0
+
+
+def test_op_wrappers_refuse_host_tensors_before_any_launch():
+    """The ops take raw device pointers: host tensors (or wrong shapes / dtypes) are refused
+    in the binding, so nothing reaches a kernel."""
+    import torch
+    from zeroth_order_fine_b200 import zo
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    W = torch.zeros(32, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        zo.zo_op_linear(x, W)
+    with pytest.raises(ValueError, match="CUDA"):
+        zo.zo_op_linear_decode(x, W)
+    with pytest.raises(ValueError, match="CUDA"):
+        zo.zo_op_lm_head_logprob(x, W, torch.zeros(4, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA"):
+        zo.zo_op_attention(torch.zeros(10, 3 * 128, dtype=torch.bfloat16), [10], 1, 1, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        zo.zo_op_quantize_rows_e4m3(x)

@@ -351,6 +351,9 @@ class Handle:
                  target_ids: Optional[torch.Tensor] = None, want_logprob: bool = False):
         sl, tl = _i32(seq_lens), _i32(target_lens)
         B = len(sl)
+        _cuda_args({"tokens": (int(sl.sum()),), "target_ids": (int(tl.sum()),)},
+                   {"tokens": (torch.int32,), "target_ids": (torch.int32,)},
+                   tokens=tokens, target_ids=target_ids)
         dev = tokens.device
         Lp = torch.empty(B, dtype=torch.float32, device=dev)
         Lm = torch.empty(B, dtype=torch.float32, device=dev)
@@ -365,6 +368,9 @@ class Handle:
         sl, tl = _i32(seq_lens), _i32(target_lens)
         fsl, ftl = _i32(fg_seq_lens), _i32(fg_target_lens)
         B, F = len(sl), len(fsl)
+        _cuda_args({"tokens": (int(sl.sum()),), "fg_tokens": (int(fsl.sum()),)},
+                   {"tokens": (torch.int32,), "fg_tokens": (torch.int32,)},
+                   tokens=tokens, fg_tokens=fg_tokens)
         dev = tokens.device
         Lp = torch.empty(B, dtype=torch.float32, device=dev)
         Lm = torch.empty(B, dtype=torch.float32, device=dev)
@@ -379,6 +385,7 @@ class Handle:
     def zo_generate(self, tokens, seq_lens, n_new: int):
         sl = _i32(seq_lens)
         B = len(sl)
+        _cuda_args({"tokens": (int(sl.sum()),)}, {"tokens": (torch.int32,)}, tokens=tokens)
         dev = tokens.device
         Lp = torch.empty(B, dtype=torch.float32, device=dev)
         Lm = torch.empty(B, dtype=torch.float32, device=dev)
@@ -391,6 +398,8 @@ class Handle:
     # zo_score_foreground
     def zo_score_foreground(self, fg_tokens, fg_seq_lens, fg_target_lens):
         fsl, ftl = _i32(fg_seq_lens), _i32(fg_target_lens)
+        _cuda_args({"fg_tokens": (int(fsl.sum()),)}, {"fg_tokens": (torch.int32,)},
+                   fg_tokens=fg_tokens)
         flp = torch.empty(int(ftl.sum()), dtype=torch.float32, device=fg_tokens.device)
         _check(lib().zo_score_foreground(self.h, _ptr(fg_tokens), len(fsl), _ptr(fsl), _ptr(ftl),
                                          _ptr(flp)), self.h)
@@ -408,6 +417,7 @@ class Handle:
     def zo_step_graph(self, tokens, seq_lens, target_lens, eps: float, lr: float):
         sl, tl = _i32(seq_lens), _i32(target_lens)
         B = len(sl)
+        _cuda_args({"tokens": (int(sl.sum()),)}, {"tokens": (torch.int32,)}, tokens=tokens)
         bufs = self.__dict__.setdefault("_graph_out", {})
         if B not in bufs:
             bufs[B] = (torch.empty(B, dtype=torch.float32, device=tokens.device),
@@ -418,9 +428,11 @@ class Handle:
         return Lp, Lm
 
     def zo_objective_sums(self, dev_sums: torch.Tensor) -> None:
+        _cuda_args({"dev_sums": (2,)}, {"dev_sums": (torch.float64,)}, dev_sums=dev_sums)
         _check(lib().zo_objective_sums(self.h, _ptr(dev_sums)), self.h)
 
     def zo_step_from_sums(self, lr: float, dev_sums: torch.Tensor, want_c: bool = True):
+        _cuda_args({"dev_sums": (2,)}, {"dev_sums": (torch.float64,)}, dev_sums=dev_sums)
         c = ctypes.c_double(0.0)
         _check(lib().zo_step_from_sums(self.h, lr, _ptr(dev_sums),
                                        ctypes.byref(c) if want_c else None), self.h)
@@ -458,6 +470,32 @@ class Handle:
 
 # ---- kernel-level ops -----------------------------------------------------------------
 
+def _cuda_args(shapes: dict, dtypes: dict = None, **tensors) -> None:
+    """The library takes raw device pointers: every tensor it reads or writes must be a
+    contiguous CUDA tensor on one device, with the shape (a tuple, None entries free) and
+    dtype the op expects; a wrong one raises here instead of reaching a kernel."""
+    dev = None
+    dtypes = dtypes or {}
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other arguments on {dev}")
+        want = shapes.get(name)
+        if want is not None and (t.dim() != len(want) or
+                                 any(w is not None and w != n for w, n in zip(want, t.shape))):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want}")
+        if name in dtypes and t.dtype not in dtypes[name]:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes[name]}")
+
+
+_FLOATS = (torch.float32, torch.bfloat16)
+
+
 def zo_op_linear(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None, act: int = 0, accumulate: bool = False,
                  impl: int = IMPL_AUTO) -> torch.Tensor:
@@ -466,6 +504,9 @@ def zo_op_linear(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] 
     dtype = wl.DTYPE_BF16 if x.dtype == torch.bfloat16 else wl.DTYPE_FP32
     if out is None:
         out = torch.empty(M, N, dtype=torch.float32 if accumulate else x.dtype, device=x.device)
+    _cuda_args({"W": (N, K), "bias": (N,), "out": (M, N)},
+               {"x": _FLOATS, "W": (x.dtype,), "bias": (torch.float32,),
+                "out": (torch.float32,) if accumulate else (x.dtype,)}, x=x, W=W, bias=bias, out=out)
     _check_op(lib().zo_op_linear(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, dtype, act,
                               int(accumulate), impl, _stream()))
     return out
@@ -481,6 +522,10 @@ def zo_op_linear_decode(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.T
         out = torch.empty(M, N, dtype=torch.float32 if accumulate else x.dtype, device=x.device)
     if ws is None:
         ws = torch.empty(max(1, 16 * M * N), dtype=torch.float32, device=x.device)
+    _cuda_args({"W": (N, K), "bias": (N,), "out": (M, N)},
+               {"x": (torch.bfloat16,), "W": (torch.bfloat16,), "bias": (torch.float32,),
+                "out": (torch.float32,) if accumulate else (torch.bfloat16,), "ws": (torch.float32,)},
+               x=x, W=W, bias=bias, out=out, ws=ws)
     _check_op(lib().zo_op_linear_decode(_ptr(x), _ptr(W), _ptr(bias), _ptr(out), M, N, K, act,
                                      int(accumulate), _ptr(ws), ws.numel(), _stream()))
     return out
@@ -504,8 +549,18 @@ def zo_op_linear_ext(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tens
         cols = N // 2 if epi == EPI_SWIGLU else N
         out = torch.empty(M, cols, dtype=torch.float32 if epi == EPI_RESID else torch.bfloat16,
                           device=x.device)
+    _cuda_args({"W": (N, K), "bias": (N,), "x2": (M, K2), "W2": (N, K2)},
+               {"x": (torch.bfloat16,), "W": (torch.bfloat16,), "bias": (torch.float32,),
+                "x2": (torch.bfloat16,), "W2": (torch.bfloat16,)},
+               x=x, W=W, bias=bias, x2=x2, W2=W2)
+    if out.device != x.device or not out.is_cuda or out.stride(1) != 1 or out.shape[0] != M:
+        raise ValueError("out must be a CUDA tensor with unit column stride and M rows")
+    if out.dtype != (torch.float32 if epi == EPI_RESID else torch.bfloat16):
+        raise ValueError("out must be float32 for the residual epilogue, else bfloat16")
     args = None
     if qk is not None:
+        _cuda_args({}, {"tok_pos": (torch.int32,)}, tok_pos=qk["tok_pos"], q_norm=qk["q_norm"],
+                   k_norm=qk["k_norm"], rope_cos=qk["rope_cos"], rope_sin=qk["rope_sin"], x=x)
         args = zo_qk_norm_rope_args(_ptr(qk["tok_pos"]), _ptr(qk["q_norm"]), _ptr(qk["k_norm"]),
                                     _ptr(qk["rope_cos"]), _ptr(qk["rope_sin"]), qk["eps"],
                                     qk["n_q_heads"], qk["n_kv_heads"])
@@ -533,6 +588,7 @@ def zo_op_quantize_rows_e4m3(x: torch.Tensor):
     """(codes uint8 [rows, cols], scale float [rows]) of the E4M3 row quantiser."""
     rows, cols = x.shape
     dtype = wl.DTYPE_BF16 if x.dtype == torch.bfloat16 else wl.DTYPE_FP32
+    _cuda_args({}, {"x": _FLOATS}, x=x)
     q = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
     sc = torch.empty(rows, dtype=torch.float32, device=x.device)
     _check_op(lib().zo_op_quantize_rows_e4m3(_ptr(x), dtype, rows, cols, _ptr(q), _ptr(sc),
@@ -544,6 +600,10 @@ def zo_op_linear_fp8(xq: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: t
                      bias: Optional[torch.Tensor] = None, act: int = 0) -> torch.Tensor:
     M, K = xq.shape
     N = wq.shape[0]
+    _cuda_args({"sx": (M,), "wq": (N, K), "sw": (N,), "bias": (N,)},
+               {"xq": (torch.uint8,), "wq": (torch.uint8,), "sx": (torch.float32,),
+                "sw": (torch.float32,), "bias": (torch.float32,)},
+               xq=xq, sx=sx, wq=wq, sw=sw, bias=bias)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
     _check_op(lib().zo_op_linear_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y),
                                   M, N, K, act, _stream()))
@@ -554,6 +614,8 @@ def zo_op_lm_head_logprob(h: torch.Tensor, E: torch.Tensor, targets: torch.Tenso
                           impl: int = IMPL_AUTO) -> torch.Tensor:
     S, d = h.shape
     V = E.shape[0]
+    _cuda_args({"E": (V, d), "targets": (S,)},
+               {"h": _FLOATS, "E": (h.dtype,), "targets": (torch.int32,)}, h=h, E=E, targets=targets)
     dtype = wl.DTYPE_BF16 if h.dtype == torch.bfloat16 else wl.DTYPE_FP32
     ws_bytes = lib().zo_op_lm_head_workspace(S, V, impl)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=h.device)
@@ -568,6 +630,8 @@ def zo_op_attention(qkv: torch.Tensor, seq_lens, n_heads: int, n_kv_heads: int,
                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
     sl = _i32(seq_lens)
     T = qkv.shape[0]
+    _cuda_args({"qkv": (int(sl.sum()), (n_heads + 2 * n_kv_heads) * head_dim)}, {"qkv": _FLOATS},
+               qkv=qkv)
     dtype = wl.DTYPE_BF16 if qkv.dtype == torch.bfloat16 else wl.DTYPE_FP32
     if out is None:
         out = torch.empty(T, n_heads * head_dim, dtype=qkv.dtype, device=qkv.device)
