@@ -145,6 +145,45 @@ def test_opt_6_7b_width_layer_full_batch_64_spans_bf16_same_state_parity():
     _bf16_same_state_parity(w, shape, batch, pre_steps=1)
 
 
+def test_qwen3_8b_width_layer_full_cobatch_step_bf16_same_state_parity():
+    """One full-width Qwen3-8B layer (d = 4096, 32 / 8 heads, SwiGLU 12288, vocab 151936) over
+    the whole seeded co-batching step: 16 prompts as 32 probe rows plus 32 foreground rows,
+    64-512 tokens, MeZO r = 64 on all seven matrices.  L+- and the foreground rows' mean
+    log-probs against the oracle at step 0 and after the oracle's first update (its bank
+    loaded)."""
+    from gpu_util import oracle_state_blob
+    w = wl.WORKLOADS["qwen3-8b-cobatch"]
+    shape = wl.shrink_shape(w.shape, n_layers=1)
+    batch = wl.make_batch(w)
+    assert len(batch.fg_prompts) == 32 and batch.n_tokens_physical > 12000
+    _, h = gpu_handle(w, shape=shape, fg=len(batch.fg_prompts))
+    orc = oracle_run(w, shape=shape)
+    toks, ftoks = dev_tokens(batch), dev_fg_tokens(batch)
+    fsplit = np.cumsum(batch.fg_target_lens)[:-1]
+
+    def compare():
+        Lp, Lm, _, flp = h.zo_score_cobatch(toks, batch.seq_lens, batch.target_lens, ftoks,
+                                            batch.fg_seq_lens, batch.fg_target_lens)
+        ref = orc.score(batch.prompts, batch.target_lens, batch.fg_prompts, batch.fg_target_lens)
+        fg_mean = np.array([x.mean() for x in np.split(flp.cpu().numpy(), fsplit)])
+        fg_ref = np.array([np.asarray(x).mean() for x in ref.fg_logprob])
+        return max(np.max(np.abs(Lp.cpu().numpy() - ref.L_plus)),
+                   np.max(np.abs(Lm.cpu().numpy() - ref.L_minus)),
+                   np.max(np.abs(fg_mean - fg_ref)))
+
+    errs = []
+    h.zo_probe_plan(0, w.eps)
+    orc.plan(0, w.eps)
+    errs.append(compare())
+    orc.step(w.lr)
+    h.zo_load_state(oracle_state_blob(orc, w, shape))
+    h.zo_probe_plan(orc.t, w.eps)
+    orc.plan(orc.t, w.eps)
+    errs.append(compare())
+    h.close()
+    assert max(errs) <= 2e-2, errs
+
+
 def test_tiny_bf16_many_rows_parity_and_cobatching():
     """160 physical rows of ~62 tokens (~9900 tokens, more 128-row tiles than CTA pairs): the
     bank shrink's CTA pairs each take a second tile, handing the split halves over twice;
