@@ -985,9 +985,12 @@ int prepare_batch(zo_handle* h, int B, const int32_t* lens, const int32_t* tls,
 // carries targets) and the base GEMM with the extension K blocks, epilogue epi.
 // nn (decode steps, EPI_RESID): the norm of the updated residual rows that comes next; it runs
 // fused into the split reduction when that path is taken, else right after the GEMM.
+// kv (decode steps, the q|k|v group): the reduction also appends k|v to the cache when it can;
+// *kv_done reports whether it did.
 int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc, int ctype,
                int Ti, float eps, const Layer* Lq = nullptr, bool decode = false,
-               const NormNext* nn = nullptr) {
+               const NormNext* nn = nullptr, const KvAppend* kv = nullptr,
+               int* kv_done = nullptr) {
     const zo_model_desc& d = h->desc;
     const int r_ = h->opt.rank;
     GemmArgs g;
@@ -995,6 +998,8 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
     int norm_done = 0;
     g.norm_next = nn;
     g.norm_done = &norm_done;
+    g.kv_append = kv;
+    g.kv_done = kv_done;
     if (epi == EPI_QKNR) {
         g.tok_pos = h->tok_pos; g.qn = Lq->w.q_norm; g.kn = Lq->w.k_norm;
         g.rope_cos = h->rope_cos; g.rope_sin = h->rope_sin; g.norm_eps = d.norm_eps;
@@ -1069,8 +1074,9 @@ int group_gemm(zo_handle* h, Group& G, const void* X, int epi, void* C, int ldc,
 // Every decoder layer over the Ti token rows whose ids, positions, signs and embeddings are
 // in place (h->tok_*, h->resid).  attn(l) enqueues layer l's attention: it reads the q|k|v
 // rows in h->qkv (q/k normalised and rotated for Qwen3) and writes h->att.
-int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)>& attn,
-                   bool decode = false) {
+int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int, bool)>& attn,
+                   bool decode = false,
+                   const std::function<const KvAppend*(int)>& kv_of = nullptr) {
     const zo_model_desc& d = h->desc;
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
     // decode steps: each residual GEMM also applies the norm that follows it (ln2 after o, the
@@ -1080,14 +1086,18 @@ int decoder_layers(zo_handle* h, int Ti, float eps, const std::function<int(int)
         if (!decode || l == 0)
             launch_norm(h->resid, nullptr, Ti, d.d_model, nk, L.w.ln1_w, L.w.ln1_b, d.norm_eps,
                         h->xn, h->dt, h->st, h->xq, h->sx, decode);
+        // decode steps: k|v go to the cache from the q|k|v reduction when the rows it stores
+        // are final (OPT, or Qwen3 with the q/k norm fused into that reduction)
+        int kv_done = 0;
+        const KvAppend* kv = kv_of && (d.arch == ZO_ARCH_OPT || h->qknr_fused) ? kv_of(l) : nullptr;
         int rc = group_gemm(h, L.g[G_QKV], h->xn, h->qknr_fused ? EPI_QKNR : EPI_STORE, h->qkv,
-                            h->n_qkv, h->dt, Ti, eps, &L, decode);
+                            h->n_qkv, h->dt, Ti, eps, &L, decode, nullptr, kv, &kv_done);
         if (rc) return rc;
         if (d.arch == ZO_ARCH_QWEN3 && !h->qknr_fused)
             launch_qk_norm_rope(h->qkv, h->n_qkv, h->dt, h->tok_pos, Ti, d.n_heads, d.n_kv_heads,
                                 d.head_dim, L.w.q_norm, L.w.k_norm, d.norm_eps, h->rope_cos,
                                 h->rope_sin, h->st);
-        rc = attn(l);
+        rc = attn(l, kv_done != 0);
         if (rc) return rc;
         const NormNext ln2 = {L.w.ln2_w, L.w.ln2_b, nk, d.norm_eps, h->xn, h->dt, h->xq, h->sx};
         rc = group_gemm(h, L.g[G_O], h->att, EPI_RESID, h->resid, d.d_model, E_F32, Ti, eps, nullptr,
@@ -1147,7 +1157,7 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
                  d.d_model, h->st);
 
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
-    int rc = decoder_layers(h, Ti, eps, [&](int l) -> int {
+    int rc = decoder_layers(h, Ti, eps, [&](int l, bool) -> int {
             AttnArgs a;
             memset(&a, 0, sizeof(a));
             a.qkv = h->qkv; a.ld_qkv = h->n_qkv;
@@ -1262,7 +1272,7 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
     launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
                  d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, Ti,
                  d.d_model, h->st);
-    rc = decoder_layers(h, Ti, eps, [&](int l) -> int {
+    rc = decoder_layers(h, Ti, eps, [&](int l, bool) -> int {
         launch_kv_scatter(h->qkv, h->n_qkv, h->q_dim, kv2, h->tok_row, Ti, G, cache(l),
                           h->kv_rows, h->dt, h->st);
         AttnArgs a;
@@ -1303,9 +1313,11 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
         launch_embed(h->tok_id, h->tok_pos, h->wts.tok_embed,
                      d.arch == ZO_ARCH_OPT ? h->wts.pos_embed : nullptr, h->dt, h->resid, R,
                      d.d_model, h->st);
-        rc = decoder_layers(h, R, eps, [&](int l) -> int {
-            launch_kv_append(h->qkv, h->n_qkv, h->q_dim, kv2, md, h->gen_lens, R, g, G, cache(l),
-                             h->kv_rows, h->dt, h->st);
+        KvAppend kva;
+        rc = decoder_layers(h, R, eps, [&](int l, bool kv_in_cache) -> int {
+            if (!kv_in_cache)
+                launch_kv_append(h->qkv, h->n_qkv, h->q_dim, kv2, md, h->gen_lens, R, g, G,
+                                 cache(l), h->kv_rows, h->dt, h->st);
             if (!launch_decode_attention(h->qkv, h->n_qkv, cache(l), kv2, md, h->gen_lens, R, g, G,
                                          d.n_heads, d.n_kv_heads, d.head_dim, scale, h->att,
                                          h->q_dim, h->dt, max_len + g + 1, h->splitk_ws,
@@ -1313,7 +1325,10 @@ int generate_impl(zo_handle* h, float eps, const int32_t* ptok, int B, const int
                 FAIL(h, ZO_ERR_UNSUPPORTED, "decode attention: more than 8 query heads per kv head");
             h->stats.kernel_launches += 2;
             return ZO_OK;
-        }, true);
+        }, true, [&](int l) -> const KvAppend* {
+            kva = {cache(l), h->kv_rows, md, h->gen_lens, g, G, h->q_dim, kv2};
+            return h->dt == E_BF16 ? &kva : nullptr;
+        });
         if (rc) return rc;
         // (the final norm of the R rows into hs ran with the last layer's FFN reduction)
         rc = lm_head_greedy(h, R, h->gen_tok + g + 1, h->gen_lp + g + 1, G);

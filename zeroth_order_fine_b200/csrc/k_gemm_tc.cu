@@ -33,6 +33,8 @@
 
 namespace zo {
 
+ZO_DEBUG_WORD(debug_word_gemm)
+
 namespace {
 
 constexpr int BM = 128, BK = 64, BN = 256;
@@ -1599,8 +1601,23 @@ namespace {
 
 // y[m, n] = sum_s ws[s, m, n] (in s order) + bias[n], then the epilogue: bf16 store / ReLU,
 // or the fp32 residual add.  One thread per 4 columns.
+// (kv.cache: the k|v columns of each row also go to its key/value cache row.)  Four
+// consecutive bf16 outputs n..n+3 of row m (n a multiple of 4, as q_dim and kv2 are), one
+// 8-byte store when they are k|v columns.
+__device__ __forceinline__ uint32_t bf16_pair_bits(__nv_bfloat16 a, __nv_bfloat16 b) {
+    return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+}
+__device__ __forceinline__ void kv_put4(const KvAppend& kv, int m, int n, uint2 v4) {
+    const int c = n - kv.q_dim;
+    if (c < 0 || c >= kv.kv2) return;
+    const size_t crow = (size_t)kv.cu[m] + (size_t)m * kv.G + kv.lens[m] + kv.g;
+    if (!ZO_DCHECK(crow < kv.cache_rows, ZO_DBG_KV_SLOT)) return;     // (debug build)
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(kv.cache) + crow * kv.kv2 + c) = v4;
+}
+
 __global__ void splitk_epilogue_kernel(const float* __restrict__ ws, int ks, int M, int N,
-                                       const float* __restrict__ bias, int epi, void* C, int ldc) {
+                                       const float* __restrict__ bias, int epi, void* C, int ldc,
+                                       KvAppend kv) {
     grid_dep_wait();
     const int m = blockIdx.y;
     const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
@@ -1614,6 +1631,7 @@ __global__ void splitk_epilogue_kernel(const float* __restrict__ ws, int ks, int
         for (int j = 0; j < 4; ++j)
             if (n + j < N) y[j] += w[j];
     }
+    __nv_bfloat16 hv[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         if (n + j >= N) break;
@@ -1622,9 +1640,12 @@ __global__ void splitk_epilogue_kernel(const float* __restrict__ ws, int ks, int
             static_cast<float*>(C)[(size_t)m * ldc + n + j] += v;
         } else {
             if (epi == EPI_STORE_RELU) v = fmaxf(v, 0.f);
-            static_cast<__nv_bfloat16*>(C)[(size_t)m * ldc + n + j] = __float2bfloat16_rn(v);
+            hv[j] = __float2bfloat16_rn(v);
+            static_cast<__nv_bfloat16*>(C)[(size_t)m * ldc + n + j] = hv[j];
         }
     }
+    if (kv.cache && n + 4 <= N)
+        kv_put4(kv, m, n, make_uint2(bf16_pair_bits(hv[0], hv[1]), bf16_pair_bits(hv[2], hv[3])));
 }
 
 // SwiGLU from the split slices: gate/up rows interleaved in 128-row blocks, so output f
@@ -1655,7 +1676,7 @@ __global__ void splitk_swiglu_kernel(const float* __restrict__ ws, int ks, int M
 // pairs (i, i + 64) at the token's position; lane l holds columns 4l..4l+3, its partner
 // columns sit in lane l ^ 16.
 __global__ void splitk_qknr_kernel(const float* __restrict__ ws, int ks, int M, int N, TcParams p,
-                                   __nv_bfloat16* C, int ldc) {
+                                   __nv_bfloat16* C, int ldc, KvAppend kv) {
     grid_dep_wait();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int heads = N / 128;
@@ -1689,8 +1710,14 @@ __global__ void splitk_qknr_kernel(const float* __restrict__ ws, int ks, int M, 
             x[e] = lane < 16 ? x[e] * cs - partner[e] * sn : x[e] * cs + partner[e] * sn;
         }
     }
+    __nv_bfloat16 hv[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) C[(size_t)m * ldc + c0 + e] = __float2bfloat16_rn(x[e]);
+    for (int e = 0; e < 4; ++e) {
+        hv[e] = __float2bfloat16_rn(x[e]);
+        C[(size_t)m * ldc + c0 + e] = hv[e];
+    }
+    if (kv.cache)
+        kv_put4(kv, m, c0, make_uint2(bf16_pair_bits(hv[0], hv[1]), bf16_pair_bits(hv[2], hv[3])));
 }
 
 // [ks][M][N] fp32 workspace, 32 x 32 boxes (128-byte rows, 128-byte swizzle)
@@ -1710,6 +1737,11 @@ bool make_map_ws(CUtensorMap* m, const float* ws, int ks, int M, int N) {
 // launched as a programmatic dependent of the GEMM that wrote the slices.
 int launch_split_reduce(const GemmArgs& g, const TcParams& p, int ks, cudaStream_t st, bool pdl) {
     cudaError_t e = cudaSuccess;
+    // k|v to the cache from the bf16 store or q/k-norm reduction (bf16 models only)
+    KvAppend kv;
+    memset(&kv, 0, sizeof(kv));
+    if (g.kv_append && (g.epi == EPI_STORE || g.epi == EPI_QKNR) && g.c_type == E_BF16)
+        kv = *g.kv_append;
     auto go = [&](auto kernel, dim3 grid, auto... args) {
         if (pdl) {
             e = launch_pdl(kernel, grid, dim3(128), 0, st, args...);
@@ -1728,7 +1760,8 @@ int launch_split_reduce(const GemmArgs& g, const TcParams& p, int ks, cudaStream
     } else if (g.epi == EPI_QKNR) {
         const long long warps = (long long)g.M * (g.N / 128);
         go(splitk_qknr_kernel, dim3((unsigned)((warps + 3) / 4)), (const float*)g.ws, ks, g.M, g.N,
-           p, static_cast<__nv_bfloat16*>(g.C), g.ldc);
+           p, static_cast<__nv_bfloat16*>(g.C), g.ldc, kv);
+        if (kv.cache && g.kv_done) *g.kv_done = 1;
     } else if (g.epi == EPI_RESID && g.norm_next &&
                launch_splitk_resid_norm(g.ws, ks, g.M, g.N, g.bias, static_cast<float*>(g.C),
                                         g.ldc, *g.norm_next, st, pdl)) {
@@ -1737,7 +1770,8 @@ int launch_split_reduce(const GemmArgs& g, const TcParams& p, int ks, cudaStream
         if (g.norm_done) *g.norm_done = 1;
     } else {
         go(splitk_epilogue_kernel, dim3((unsigned)((g.N / 4 + 127) / 128), (unsigned)g.M),
-           (const float*)g.ws, ks, g.M, g.N, g.bias, g.epi, g.C, g.ldc);
+           (const float*)g.ws, ks, g.M, g.N, g.bias, g.epi, g.C, g.ldc, kv);
+        if (kv.cache && g.kv_done) *g.kv_done = 1;
     }
     return e == cudaSuccess ? 0 : 1;
 }

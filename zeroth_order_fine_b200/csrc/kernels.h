@@ -96,6 +96,14 @@ struct NormNext {
     uint8_t* q8; float* s8;                 // optional E4M3 rows and scales of the output
 };
 
+// Decode steps: the q|k|v split reduction also writes each row's k|v columns into the key/value
+// cache (row r's new token at cache row cu[r] + r * G + lens[r] + g, kv2 elements wide).
+struct KvAppend {
+    void* cache; size_t cache_rows;
+    const int* cu; const int* lens; int g, G;
+    int q_dim, kv2;
+};
+
 struct GemmArgs {
     const void* A; int lda; int a_type;     // [M x K], K contiguous
     const void* B; int ldb; int b_type;     // [N x K], K contiguous
@@ -129,6 +137,9 @@ struct GemmArgs {
     // EPI_RESID with a split reduction: the reduction may also apply norm_next to each updated
     // row of C (the fp32 residual); it then sets *norm_done = 1 (else the caller runs the norm)
     const NormNext* norm_next; int* norm_done;
+    // EPI_STORE / EPI_QKNR with a split reduction: the reduction may also append the k|v
+    // columns to the cache (sets *kv_done = 1; else the caller copies them)
+    const KvAppend* kv_append; int* kv_done;
 };
 // Split-K residual reduction with the next norm fused (see NormNext); false when the shape or
 // alignment is outside the vectorised form (nothing launched).
@@ -256,5 +267,6 @@ unsigned debug_word_attention_tc(bool clear);
 unsigned debug_word_attention(bool clear);
 unsigned debug_word_decode(bool clear);
 unsigned debug_word_reduce(bool clear);
+unsigned debug_word_gemm(bool clear);
 
 }  // namespace zo

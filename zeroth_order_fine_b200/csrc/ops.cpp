@@ -308,7 +308,8 @@ int zo_debug_build(void) {
 
 uint32_t zo_debug_word(int32_t clear) {
     return debug_word_attention_tc(clear != 0) | debug_word_attention(clear != 0) |
-           debug_word_decode(clear != 0) | debug_word_reduce(clear != 0);
+           debug_word_decode(clear != 0) | debug_word_reduce(clear != 0) |
+           debug_word_gemm(clear != 0);
 }
 
 const char* zo_op_last_error(void) { return t_op_err.c_str(); }
