@@ -80,3 +80,41 @@ def test_random_batch_shapes_match_the_oracle(seed):
             assert abs(c - c_ref) <= 1e-2 * max(abs(c_ref), 1.0), (seed, t, c, c_ref)
     assert h.zo_stats()["last_error_code"] == 0
     h.close()
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_generation_shapes_match_the_oracle(seed):
+    """Generation queries on random shapes: 1-6 prompts of 2-150 tokens, 1-6 new tokens,
+    OPT or Qwen3 in fp32 or bf16.  Every generated token is a largest logit of the oracle
+    teacher-forced on the GPU's own prefix (within the precision's bound, so near-ties may
+    go either way), its log-prob matches, and so do L+-."""
+    from oracle import model as om
+    rng = np.random.default_rng(5000 + seed)
+    w = _case(seed)
+    w = dataclasses.replace(w, batch=int(rng.integers(1, 7)), len_hi=150, fg_rows=0)
+    G = int(rng.integers(1, 7))
+    fp32 = w.shape.dtype == wl.DTYPE_FP32
+    logit_tol, lp_tol, L_tol = (1e-4, 1e-4, 1e-4) if fp32 else (5e-2, 3e-2, 2e-2)
+    batch = wl.make_batch(w)
+    B = len(batch.prompts)
+    _, h = gpu_handle(w, max_new=G)
+    h.zo_probe_plan(0, w.eps)
+    Lp, Lm, gt, gl = h.zo_generate(dev_tokens(batch), batch.seq_lens, G)
+    gt, gl = gt.cpu().numpy(), gl.cpu().numpy()
+    orc = oracle_run(w)
+    orc.plan(0, w.eps)
+    rows = [np.concatenate([p, gt[r]]).astype(np.int64)
+            for r, p in enumerate(list(batch.prompts) * 2)]
+    hs = om.hidden_states(orc.w, rows, [1.0] * B + [-1.0] * B, orc.eps, orc.perturbation())
+    logits = om.span_logits(orc.w, hs, rows, [G] * (2 * B))
+    ref_lp = om.token_logprobs(orc.w, hs, rows, [G] * (2 * B))
+    for r in range(2 * B):
+        lg = logits[r].numpy()
+        chosen = lg[np.arange(G), gt[r]]
+        assert np.all(chosen >= lg.max(axis=1) - logit_tol), (seed, r)
+        assert np.max(np.abs(gl[r] - ref_lp[r].numpy())) <= lp_tol, (seed, r)
+    ref_L = np.array([-x.numpy().mean() for x in ref_lp])
+    assert np.max(np.abs(Lp.cpu().numpy() - ref_L[:B])) <= L_tol
+    assert np.max(np.abs(Lm.cpu().numpy() - ref_L[B:])) <= L_tol
+    assert np.isfinite(h.zo_step(w.lr))
+    h.close()
