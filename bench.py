@@ -497,7 +497,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="opt-13b-b64", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-prompts", type=int, default=2)
+    # prompts in the oracle's timing sample of the larger workloads: the reference arm's
+    # per-step sample (about 4 s of CPU work for OPT-13B b64), and the one cpu_baseline
+    # sample of the default line (about 10 s)
+    ap.add_argument("--ref-prompts", type=int, default=16)
+    ap.add_argument("--baseline-prompts", type=int, default=40)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the whole-step CUDA graph leg")
@@ -806,7 +810,7 @@ def main():
         torch.cuda.empty_cache()
         line["cobatch"] = cobatch_leg(args.steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample(w, n_prompts=args.ref_prompts)
+        cb = oracle_sample(w, n_prompts=args.baseline_prompts)
         line["cpu_baseline"] = {"value": cb["tokens_per_s"], "unit": "scored tokens/s",
                                 "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"],
                                 "extrapolated": cb["extrapolated"],
