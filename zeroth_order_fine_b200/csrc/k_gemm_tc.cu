@@ -38,6 +38,9 @@ ZO_DEBUG_WORD(debug_word_gemm)
 namespace {
 
 constexpr int BM = 128, BK = 64, BN = 256;
+// lm_head log-sum-exp tiles: 128 vocabulary columns, so that the ~400 tiles of a 50k-151k
+// vocabulary fill the SMs' waves evenly (256-column tiles left OPT's second wave a third full)
+constexpr int BN_LSE = 128;
 constexpr int BK8 = 128;                    // E4M3 K block: the same 128-byte rows
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int TMEM_COLS = 512;              // two BN-wide fp32 accumulators
@@ -1527,10 +1530,11 @@ int launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2
 }
 
 // N tile of the single-SM kernel: the narrowest of 64/128/256 that covers N, for
-// the epilogues that work column chunk by column chunk; the LSE partials and the
-// SwiGLU gate/up interleave are laid out in 256-column tiles.
+// the epilogues that work column chunk by column chunk; the LSE partials are laid out in
+// BN_LSE-column tiles and the SwiGLU gate/up interleave in 256-column tiles.
 int tile1_width(const GemmArgs& g) {
-    if (g.epi == EPI_LSE || g.epi == EPI_SWIGLU) return BN;
+    if (g.epi == EPI_LSE) return BN_LSE;
+    if (g.epi == EPI_SWIGLU) return BN;
     return g.N <= 64 ? 64 : (g.N <= 128 ? 128 : 256);
 }
 
@@ -1910,7 +1914,7 @@ bool gemm_tc_supported(const GemmArgs& g) {
     }
 }
 
-int gemm_tc_col_tiles(int N) { return (N + BN - 1) / BN; }
+int gemm_tc_col_tiles(int N) { return (N + BN_LSE - 1) / BN_LSE; }
 
 int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     // Decoder GEMMs run on SM pairs, the LSE and shrink forms on single SMs.  The
@@ -2021,7 +2025,7 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
         case EPI_STORE: return launch_epi_w<EPI_STORE>(bnt, a, b, a2, b2, p, st);
         case EPI_STORE_RELU: return launch_epi_w<EPI_STORE_RELU>(bnt, a, b, a2, b2, p, st);
         case EPI_RESID: return launch_epi_w<EPI_RESID>(bnt, a, b, a2, b2, p, st);
-        case EPI_LSE: return launch_epi<EPI_LSE, BN>(a, b, a2, b2, p, st);
+        case EPI_LSE: return launch_epi<EPI_LSE, BN_LSE>(a, b, a2, b2, p, st);
         case EPI_SHRINK: return launch_epi_w<EPI_SHRINK>(bnt, a, b, a2, b2, p, st);
         case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, BN>(a, b, a2, b2, p, st);
         default: return 1;
