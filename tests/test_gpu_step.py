@@ -300,8 +300,11 @@ def test_tiny_bf16_loss_trajectory_100_steps():
 
 def test_opt_1_3b_width_slice_bf16_loss_trajectory_100_steps():
     """bf16 mode: 100 steps of two full-width OPT-1.3B layers (d = 2048, vocab 50272,
-    q and v targets, eta = 1e-4 as configured), trajectory within 2 % of the oracle's."""
-    w = wl.WORKLOADS["opt-1.3b-b16"]
+    q and v targets, eta = 1e-4 as configured), trajectory within 2 % of the oracle's.
+    eps = 1e-2, as for the tiny trajectory: on this slice an objective error of 1e-3 (the
+    bf16 rounding of L) moves the oracle's own 100-step trajectory by up to 1.9 % at
+    eps = 1e-3 but by 0.17 % at eps = 1e-2, where the oracle still falls by 20 %."""
+    w = dataclasses.replace(wl.WORKLOADS["opt-1.3b-b16"], eps=1e-2)
     shape = wl.shrink_shape(w.shape, n_layers=2)
     _check_trajectory(*_trajectory_vs_oracle(w, shape, wl.make_batch(w, batch=4, len_hi=64)))
 
