@@ -147,7 +147,7 @@ struct zo_handle {
     GenJob* genU32_d = nullptr;   // bf16 models: fp32 U jobs, run only by zo_read_factors
     // bank update: coefficients of the current slot since replay_from (its opening step), or
     // replay_from = -1 when the slot must be read-modify-written (loaded state, or replay
-    // judged too costly for the factor sizes: replay_enabled)
+    // too costly for the factor sizes: replay_enabled)
     float* coef_hist = nullptr;
     long long replay_from = -1;
     bool replay_enabled = false;
