@@ -18,6 +18,8 @@
 //               registers, the output rescaled in TMEM); an item's O / l goes to memory
 //               after the next item's softmax (the item's own P V runs meanwhile)
 // So the next items' loads and Q K^T overlap this item's softmax and the last item's store.
+// A CTA's items (up to 40) are decoded once into a shared-memory table at the start, so
+// no role walks the item order and the row offsets in global memory per item.
 // Queries, keys and values arrive by TMA straight from the packed q|k|v rows (Qwen3's
 // q/k norm and rotary positions were applied beforehand).  Keys past the row's end
 // get zero probability, so a query's result depends only on its own row: packing
@@ -39,8 +41,10 @@ constexpr int TQ = 128, TK = 128;              // head_dim HD = 64 or 128 (templ
 constexpr int ATOM = TQ * 128;                  // bytes of one 64-column swizzle atom block
 constexpr int BUF = 2 * ATOM;                   // one [128 x 128] bf16 operand (P is always
                                                 // 128 keys wide; Q, K, V fill HD / 64 atoms)
-// Q[3] K[2] V[2] buffers, then 23 mbarriers, the TMEM base and the abort flag
-constexpr int SMEM = 7 * BUF + 1024 + 256;
+// Q[3] K[2] V[2] buffers, then 23 mbarriers, the TMEM base, the abort flag and the CTA's
+// decoded work items (when they fit)
+constexpr int ITEM_CACHE = 40;                  // items of a CTA decoded into shared memory
+constexpr int SMEM = 7 * BUF + 1024 + 256 + ITEM_CACHE * 32;
 constexpr int NTHREADS = 224;                   // Q/K producer, MMA issuer, 4 softmax warps,
                                                 // V producer
 constexpr long long WAIT_CYCLES = 4000000000ll;
@@ -208,6 +212,7 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, ui
 struct Item {
     int start, len, q0, nq, kend, n_chunks, h, kvh;
 };
+static_assert(sizeof(Item) == 32, "item cache slots are 32 bytes");
 __device__ __forceinline__ Item make_item(const AttnArgs& a, int i, int tile, int start, int end) {
     Item it;
     const int qt = tile & 0xFFFF;
@@ -250,6 +255,8 @@ __device__ __forceinline__ Item get_item(const AttnArgs& a, int i) {
 // loaded while item k is being worked on, so no role waits on the dependent loads
 // (tile, then the row's offsets) when it moves to its next item.
 struct ItemFeed {
+    const Item* cache;          // the CTA's items decoded in shared memory, or NULL
+    int n_mine;                 // this CTA's item count
     const int* tiles;
     const int* cu;
     AttnArgs shape;             // only H, Hkv and n_rows are read
@@ -260,7 +267,15 @@ struct ItemFeed {
     int tile1, s1, e1;          // item k + 1: tile and row offsets (valid when k + 1 exists)
     int tile2;                  // item k + 2: tile
     __device__ __forceinline__ int idx(int kk) const { return blockIdx.x + kk * gridDim.x; }
-    __device__ __forceinline__ void init(const AttnArgs& args, int n) {
+    __device__ __forceinline__ void init(const AttnArgs& args, int n, const Item* decoded) {
+        n_mine = (int)blockIdx.x < n ? (n - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+        cache = n_mine <= ITEM_CACHE ? decoded : nullptr;
+        if (cache) {
+            k = 0;
+            has = n_mine > 0;
+            if (has) cur = cache[0];
+            return;
+        }
         tiles = args.tiles;
         cu = args.cu_seqlens;
         shape.H = args.H;
@@ -278,6 +293,12 @@ struct ItemFeed {
         if (idx(2) < n) tile2 = tiles[idx(2) / shape.H];
     }
     __device__ __forceinline__ void advance() {
+        if (cache) {
+            ++k;
+            has = k < n_mine;
+            if (has) cur = cache[k];
+            return;
+        }
         ++k;
         has = idx(k) < n_items;
         if (has) cur = make_item(shape, idx(k), tile1, s1, e1);   // loaded an item ago
@@ -343,6 +364,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t drain = bar0 + 8u * 22;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(g + 7 * BUF + 192);
     volatile int* abort_f = reinterpret_cast<volatile int*>(g + 7 * BUF + 200);
+    Item* items = reinterpret_cast<Item*>(g + 7 * BUF + 256);   // ITEM_CACHE decoded items
     // P of a chunk goes over its K buffer, except for an item's last chunk: over the item's
     // Q buffer, whose last reader (that chunk's S) has retired by then.  So the K buffer of an
     // item's last chunk is free as soon as its S retires, and the next K load overlaps the
@@ -373,6 +395,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
+    {
+        // the CTA's work items (blockIdx.x + k * gridDim.x) decoded once, when they all fit:
+        // each role then reads an item from shared memory instead of the tile -> row-offset
+        // loads and the divisions by the head counts
+        const int mine = (int)blockIdx.x < n_items
+                             ? (n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+        if (mine <= ITEM_CACHE)
+            for (int kk = tid; kk < mine; kk += NTHREADS)
+                items[kk] = get_item(a, (int)blockIdx.x + kk * (int)gridDim.x);
+    }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                          smem_u32(tslot))
@@ -395,7 +427,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int& gc = gcl;
             bool ok = true;
             ItemFeed feed;
-            feed.init(a, n_items);
+            feed.init(a, n_items, items);
             for (int k = 0; ok && feed.has; ++k, feed.advance()) {
                 const Item it = feed.cur;
                 if (!vk) {
@@ -429,8 +461,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int sk = 0, sc = 0, gs = 0;          // next S: item counter, chunk, global chunk
             int pk = 0, pc = 0, gp = 0;          // next P V
             ItemFeed s_feed, p_feed;             // the items of the next S and the next P V
-            s_feed.init(a, n_items);
-            p_feed.init(a, n_items);
+            s_feed.init(a, n_items, items);
+            p_feed.init(a, n_items, items);
             bool s_more = s_feed.has, p_more = p_feed.has;
             bool ok = true, issued = false;
             long long t0 = clock64();
@@ -530,7 +562,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int gc = 0;
         bool ok = true;
         ItemFeed feed;
-        feed.init(a, n_items);
+        feed.init(a, n_items, items);
         for (int k = 0; ok && feed.has; ++k, feed.advance()) {
             const Item it = feed.cur;
             const int q = it.q0 + row;
