@@ -20,10 +20,11 @@
 // So the next items' loads and Q K^T overlap this item's softmax and the last item's store.
 // A CTA's items (up to 40) are decoded once into a shared-memory table at the start, so
 // no role walks the item order and the row offsets in global memory per item.
-// Queries, keys and values arrive by TMA straight from the packed q|k|v rows (Qwen3's
-// q/k norm and rotary positions were applied beforehand).  Keys past the row's end
-// get zero probability, so a query's result depends only on its own row: packing
-// never changes a bit.  Every wait is bounded; on expiry the kernel records the error
+// Queries, keys and values arrive by TMA straight from the packed q|k|v rows, each tile
+// with the shortest box (32, 64, 96 or 128 rows) that covers it (Qwen3's q/k norm and
+// rotary positions were applied beforehand).  Keys past the row's end get zero
+// probability, so a query's result depends only on its own row: packing never changes a
+// bit.  Every wait is bounded; on expiry the kernel records the error
 // word, drains what it issued, frees its tensor memory and returns.
 #include <cuda.h>
 #include <float.h>
@@ -208,6 +209,19 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, ui
         : "memory");
 }
 
+// Maps over the packed q|k|v rows with boxes of 64 columns and 32, 64, 96 or 128 rows: a
+// tile is fetched with the shortest box that holds its rows (queries of the tile, keys of
+// the chunk), so a short row does not pull its neighbours' rows through L2.  Rows of a
+// buffer past the box keep older contents: query rows there are never stored, key columns
+// there are masked before the exponential, and the value rows there meet probability 0
+// (the value buffers start zeroed and only ever hold value rows, so they stay finite).
+struct AttnMaps {
+    CUtensorMap box[4];
+};
+__device__ __forceinline__ int box_of(int rows) {   // rows 1..128 -> box 0..3
+    return rows <= 32 ? 0 : rows <= 64 ? 1 : rows <= 96 ? 2 : 3;
+}
+
 // One (query tile, head) work item.
 struct Item {
     int start, len, q0, nq, kend, n_chunks, h, kvh;
@@ -339,10 +353,10 @@ __device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t pb, uint32_t vb
 // counters: the n-th use of a two-slot resource waits parity (n >> 1) & 1.
 template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnArgs a) {
+    attention_tc_kernel(const __grid_constant__ AttnMaps tm, AttnArgs a) {
     static_assert(HD == 64 || HD == 128, "head_dim");
     constexpr int NATOM = HD / 64;              // swizzle atoms of a Q, K or V tile
-    constexpr uint32_t TILE_BYTES = TQ * HD * 2;
+    constexpr uint32_t BOX_BYTES = 32 * HD * 2;   // bytes of 32 rows of a Q, K or V tile
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -404,6 +418,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (mine <= ITEM_CACHE)
             for (int kk = tid; kk < mine; kk += NTHREADS)
                 items[kk] = get_item(a, (int)blockIdx.x + kk * (int)gridDim.x);
+        // value buffers start at zero: rows a short box leaves untouched are finite
+        uint4* vz = reinterpret_cast<uint4*>(g + 5 * BUF);
+        for (int i = tid; i < 2 * BUF / 16; i += NTHREADS) vz[i] = make_uint4(0u, 0u, 0u, 0u);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // before the TMA writes
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
@@ -433,10 +451,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!vk) {
                     const int qs = k % 3;
                     if (!wait_bar(q_empty(qs), ((k / 3) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
-                    bar_expect_tx(q_full(qs), TILE_BYTES);
+                    const int qb = box_of(it.nq);
+                    bar_expect_tx(q_full(qs), (uint32_t)(qb + 1) * BOX_BYTES);
                     for (int half = 0; half < NATOM; ++half)
-                        tma_box(Qb(qs) + half * ATOM, &tm, q_full(qs), it.h * HD + half * 64,
-                                it.start + it.q0);
+                        tma_box(Qb(qs) + half * ATOM, &tm.box[qb], q_full(qs),
+                                it.h * HD + half * 64, it.start + it.q0);
                     ++gq;
                 }
                 const int col = vk ? q_dim + kv_dim + it.kvh * HD : q_dim + it.kvh * HD;
@@ -445,10 +464,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const uint32_t e = vk ? v_empty(st) : k_empty(st);
                     const uint32_t f = vk ? v_full(st) : k_full(st);
                     if (!wait_bar(e, ((gc >> 1) & 1) ^ 1u, abort_f, err)) { ok = false; break; }
-                    bar_expect_tx(f, TILE_BYTES);
+                    const int kb = box_of(min(TK, it.kend - c * TK));
+                    bar_expect_tx(f, (uint32_t)(kb + 1) * BOX_BYTES);
                     for (int half = 0; half < NATOM; ++half)
-                        tma_box((vk ? Vb(st) : Kb(st)) + half * ATOM, &tm, f, col + half * 64,
-                                it.start + c * TK);
+                        tma_box((vk ? Vb(st) : Kb(st)) + half * ATOM, &tm.box[kb], f,
+                                col + half * 64, it.start + c * TK);
                     ++gc;
                 }
             }
@@ -714,19 +734,21 @@ bool launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
                          : cudaFuncSetAttribute(attention_tc_kernel<64>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (at != cudaSuccess) return false;
-    // one map over the packed [T x ld_qkv] q|k|v rows: 64-column x 128-row boxes,
-    // 128-byte swizzle, rows past T read as zero
-    CUtensorMap tm;
+    // maps over the packed [T x ld_qkv] q|k|v rows: 64-column boxes of 32, 64, 96 and 128
+    // rows, 128-byte swizzle, rows past T read as zero
+    AttnMaps tm;
     EncodeTiledFn fn = attn_encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)a.ld_qkv, (cuuint64_t)a.n_tokens};
     const cuuint64_t strides[1] = {(cuuint64_t)a.ld_qkv * 2};
-    const cuuint32_t box[2] = {64, 128};
     const cuuint32_t es[2] = {1, 1};
-    if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.qkv), dims, strides, box,
-           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return false;
+    for (int b = 0; b < 4; ++b) {
+        const cuuint32_t box[2] = {64, (cuuint32_t)(32 * (b + 1))};
+        if (fn(&tm.box[b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.qkv), dims,
+               strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
     const long long items = (long long)a.n_tiles * a.H;
     if (items > 0x7fffffffLL) return false;
     static int sms = 0;
