@@ -111,6 +111,15 @@ __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 32 contiguous bytes to global memory in one instruction (the address is 32-byte aligned)
+__device__ __forceinline__ void st_global_32b(void* p, uint32_t w0, uint32_t w1, uint32_t w2,
+                                              uint32_t w3, uint32_t w4, uint32_t w5, uint32_t w6,
+                                              uint32_t w7) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w0), "r"(w1),
+                 "r"(w2), "r"(w3), "r"(w4), "r"(w5), "r"(w6), "r"(w7)
+                 : "memory");
+}
+
 __device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -548,6 +557,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int row = wq * 32 + lane;          // query row of the tile = TMEM lane
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sl2 = a.scale * 1.4426950408889634f;
+        // output rows start on 32-byte boundaries: 32-byte stores (one sector each)
+        const bool st32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0 && a.ld_out % 16 == 0;
         // epilogue of item ke: O / l of this thread's query row, once its last P V retired
         auto store_item = [&](int ke, const Item& it, float l) -> bool {
             const int os = ke & 1;
@@ -562,13 +573,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int cc = 0; cc < HD / 32; ++cc) {
                 float v[32];
                 tmem_ld32(t_o(os) + lane_addr + cc * 32, v);     // warp-collective: every lane
-                if (store) {
+                auto w = [&](int j) { return pack_bf2(v[2 * j] * inv, v[2 * j + 1] * inv); };
+                if (store && st32) {
+#pragma unroll
+                    for (int k8 = 0; k8 < 2; ++k8)
+                        st_global_32b(o4 + cc * 4 + k8 * 2, w(8 * k8), w(8 * k8 + 1), w(8 * k8 + 2),
+                                      w(8 * k8 + 3), w(8 * k8 + 4), w(8 * k8 + 5), w(8 * k8 + 6),
+                                      w(8 * k8 + 7));
+                } else if (store) {
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                        o4[cc * 4 + k4] = make_uint4(pack_bf2(v[8 * k4] * inv, v[8 * k4 + 1] * inv),
-                                                     pack_bf2(v[8 * k4 + 2] * inv, v[8 * k4 + 3] * inv),
-                                                     pack_bf2(v[8 * k4 + 4] * inv, v[8 * k4 + 5] * inv),
-                                                     pack_bf2(v[8 * k4 + 6] * inv, v[8 * k4 + 7] * inv));
+                        o4[cc * 4 + k4] = make_uint4(w(4 * k4), w(4 * k4 + 1), w(4 * k4 + 2),
+                                                     w(4 * k4 + 3));
                 }
             }
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
