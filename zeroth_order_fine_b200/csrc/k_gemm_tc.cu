@@ -1203,10 +1203,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 // epilogue.  The split is the same for every M, so a row's bits never depend on the batch.
 template <int BNT>
 struct TileS {
-    static_assert(BNT == 64 || BNT == 128, "shrink N tile");
+    static_assert(BNT == 32 || BNT == 64 || BNT == 128, "shrink N tile");
     static constexpr int B_BYTES = BNT * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // multiple of 1024
-    static constexpr int STAGES = BNT == 64 ? 7 : 4;
+    // as many stages as fit beside the partial-sum buffer: each CTA's streaming rate is set
+    // by the bytes of x it keeps in flight
+    static constexpr int STAGES = BNT == 32 ? 10 : BNT == 64 ? 7 : 4;
     static constexpr int PART_LD = BNT + 4;                      // padded rows: no bank clash
     static constexpr int PART_BYTES = BM * PART_LD * 4;          // the odd CTA's accumulator
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + PART_BYTES + 1024 + 256;
@@ -1975,7 +1977,14 @@ int gemm_tc(const GemmArgs& g, cudaStream_t st) {
     p.wait_cycles = g_wait_cycles;
     if (g.epi == EPI_SHRINK && !g.ws && !f8 && g.K2 == 0 && bnt <= 128 && p.kb_main >= 2) {
         // the bank shrink of a scoring batch: K split over a CTA pair so that every SM streams
-        // rows of x (chosen by N and K only, never by M)
+        // rows of x (chosen by N and K only, never by M); up to 32 bank columns take a
+        // 32-wide N tile, whose smaller stages leave room for more of them in flight
+        if (g.N <= 32) {
+            if (!make_map(&b, g.B, g.N, g.K, g.ldb, 32u)) return 1;
+            p.n_n_blk = 1;
+            p.n_tiles = p.n_m_blk;
+            return launch_shrink_pair<32>(a, b, p, st);
+        }
         return bnt == 64 ? launch_shrink_pair<64>(a, b, p, st) : launch_shrink_pair<128>(a, b, p, st);
     }
     if (pair && g.ws && !f8 && g.N % 4 == 0 &&
