@@ -189,3 +189,30 @@ def test_attention_matches_oracle(lens, H, Hkv, hd, dtype, impl):
         ref = om.causal_attention(q[off:off + L], k[off:off + L], v[off:off + L], H // Hkv)
         assert torch.max((out[off:off + L] - ref).abs()) < tol
         off += L
+
+
+@pytest.mark.parametrize("out_offset", [0, 8])
+def test_attention_many_items_per_cta_and_output_alignment(out_offset):
+    """220 short rows x 32 heads = 7040 (query tile, head) items, more than 40 per persistent
+    CTA on 148 SMs: each role then decodes its items from the tile list instead of the
+    shared-memory item table.  With out_offset = 8 the output starts 16 bytes past a 32-byte
+    boundary, so its rows are written with 16-byte stores instead of 32-byte ones."""
+    from oracle import model as om
+    from zeroth_order_fine_b200 import zo
+    lens = [int(x) for x in np.random.default_rng(7).integers(1, 25, 220)]
+    H, Hkv, hd = 32, 8, 64
+    T = sum(lens)
+    qkv = _rand((T, (H + 2 * Hkv) * hd), torch.bfloat16, 17)
+    buf = torch.empty(out_offset + T * H * hd, dtype=torch.bfloat16, device="cuda")
+    out = buf[out_offset:].view(T, H * hd)
+    zo.zo_op_attention(qkv.cuda(), lens, H, Hkv, hd, impl=2, out=out)
+    assert zo.zo_op_error_word() == 0
+    got = out.double().cpu()
+    q = qkv.double()[:, :H * hd].reshape(T, H, hd)
+    k = qkv.double()[:, H * hd:(H + Hkv) * hd].reshape(T, Hkv, hd)
+    v = qkv.double()[:, (H + Hkv) * hd:].reshape(T, Hkv, hd)
+    off = 0
+    for L in lens:
+        ref = om.causal_attention(q[off:off + L], k[off:off + L], v[off:off + L], H // Hkv)
+        assert torch.max((got[off:off + L] - ref).abs()) < 2e-2
+        off += L

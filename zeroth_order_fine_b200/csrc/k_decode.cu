@@ -110,8 +110,13 @@ inline int dec_tile_keys(int hd, int es) { return std::min(DEC_KT_MAX, 65536 / (
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// wait until at most N of this thread's committed copy groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // 8 consecutive elements of a shared-memory row (bf16 or fp32)
@@ -172,14 +177,22 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_attention_kernel(
     const uint32_t vs_addr = static_cast<uint32_t>(__cvta_generic_to_shared(Vs));
     for (int t0 = kbeg; t0 < kend; t0 += kt) {
         const int nt = min(kt, kend - t0);
-        // 0. the tile's k and v rows of this head
+        // 0. the tile's k rows, then its v rows, of this head: two copy groups, so that the
+        //    scores and the softmax run while the v rows are still landing
         for (int c = threadIdx.x; c < nt * chunks; c += DEC_THREADS) {
             const int row = c / chunks, pc = c - row * chunks;
-            const char* src = cbase + ((base + t0 + row) * kv2 + (size_t)kvh * HD) * es + pc * 16;
-            cp_async16(ks_addr + row * row_bytes + pc * 16, src);
-            cp_async16(vs_addr + row * row_bytes + pc * 16, src + (size_t)kv_dim * es);
+            cp_async16(ks_addr + row * row_bytes + pc * 16,
+                       cbase + ((base + t0 + row) * kv2 + (size_t)kvh * HD) * es + pc * 16);
         }
-        cp_async_wait_all();
+        cp_async_commit();
+        for (int c = threadIdx.x; c < nt * chunks; c += DEC_THREADS) {
+            const int row = c / chunks, pc = c - row * chunks;
+            cp_async16(vs_addr + row * row_bytes + pc * 16,
+                       cbase + ((base + t0 + row) * kv2 + (size_t)kv_dim + (size_t)kvh * HD) * es +
+                           pc * 16);
+        }
+        cp_async_commit();
+        cp_async_wait<1>();                            // this thread's k copies have landed
         __syncthreads();
         // 1. scores; the loop bounds are uniform over the warp (the shuffles need every lane)
         for (int i0 = warp * KPW; i0 < nt; i0 += U * SLOTS) {
@@ -230,6 +243,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_attention_kernel(
                 s_l[h] = s_l[h] * alpha + sum;
             }
         }
+        cp_async_wait<0>();                            // and its v copies
         __syncthreads();
         // 3. o = alpha * o + P V
 #pragma unroll
