@@ -167,6 +167,8 @@ int zo_op_lm_head_logprob(const void* h, const void* E, const int32_t* targets, 
  *   seq_lens host int32 [n_rows], rows back to back in qkv
  *   workspace dev >= 4*(n_rows + 1 + T/64 + n_rows + 1) bytes (row offsets and tiles)
  *   impl     ZO_IMPL_TENSOR_CORES needs bf16 and head_dim 64 or 128; AUTO picks them then.
+ * The tensor-core form also needs qkv and out 16-byte aligned; when out is 32-byte
+ * aligned its rows are written with 32-byte stores (same values either way).
  * The call copies the row offsets from the host and synchronises the stream. */
 int zo_op_attention(const void* qkv, void* out, const int32_t* seq_lens, int32_t n_rows,
                     int32_t n_heads, int32_t n_kv_heads, int32_t head_dim, int32_t dtype,
