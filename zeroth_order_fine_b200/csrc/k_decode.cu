@@ -106,10 +106,6 @@ constexpr int DEC_MAX_REP = 8;
 
 // keys per tile: the tile's k and v rows fill 64 KB of shared memory, at most DEC_KT_MAX
 inline int dec_tile_keys(int hd, int es) { return std::min(DEC_KT_MAX, 65536 / (2 * hd * es)); }
-// keys per tile when 9 CTAs share an SM: k and v rows in 24 KB, a multiple of 16 keys
-inline int dec_tile_keys_9(int hd, int es) {
-    return std::max(16, std::min(DEC_KT_MAX, 24576 / (2 * hd * es)) / 16 * 16);
-}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -134,10 +130,8 @@ __device__ __forceinline__ void smem8(const uint8_t* p, int es, float* v) {
     }
 }
 
-// One query head per kv head: capped at 56 registers so that 9 CTAs fit on an SM (with the
-// 24 KB tiles the host picks then), e.g. OPT-13B's 32 rows x 40 heads in one wave.
 template <int HD, int NREP>
-__global__ void __launch_bounds__(DEC_THREADS, NREP == 1 ? 9 : 1) decode_attention_kernel(
+__global__ void __launch_bounds__(DEC_THREADS) decode_attention_kernel(
     const void* __restrict__ qkv, int ld_qkv, const void* __restrict__ cache, int kv2,
     const int* __restrict__ cu, const int* __restrict__ lens, int g, int G, int Hkv, int n_rep,
     float scale, void* __restrict__ out, int ld_out, int dtype, int kps, int kt,
@@ -507,7 +501,6 @@ bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
     const int n_rep = H / Hkv;
     const int es = dtype == E_F32 ? 4 : 2;
     int kt = dec_tile_keys(hd, es);
-    const int nrep_p = n_rep == 1 ? 1 : n_rep == 2 ? 2 : n_rep <= 4 ? 4 : 8;
     // with fewer than ~4 (row, kv head) CTAs per SM, split the keys into tiles so enough
     // copies stay in flight; the splits' partial softmaxes are combined in order by the merge
     // kernel.  Without a split a CTA walks its keys in half-size tiles: twice the CTAs fit on
@@ -516,9 +509,10 @@ bool launch_decode_attention(const void* qkv, int ld_qkv, const void* cache, int
     int S = many ? 1 : (max_n + kt - 1) / kt;
     if (S < 1) S = 1;
     if ((size_t)R * Hkv * S * n_rep * (hd + 2) > ws_floats) S = 1;
-    if (S == 1) kt = nrep_p == 1 ? dec_tile_keys_9(hd, es) : std::max(16, kt / 2);
+    if (S == 1) kt = std::max(16, kt / 2);
     const int kps = S == 1 ? max_n : kt;
     float* part = S > 1 ? ws : nullptr;
+    const int nrep_p = n_rep == 1 ? 1 : n_rep == 2 ? 2 : n_rep <= 4 ? 4 : 8;
     const size_t slots_bytes = (size_t)(1024 / hd) * nrep_p * hd * 4;
     const size_t smem = std::max((size_t)2 * kt * hd * es, slots_bytes) + (size_t)nrep_p * kt * 4;
     dim3 grid(R, Hkv, S);
