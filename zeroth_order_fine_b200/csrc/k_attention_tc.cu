@@ -23,9 +23,10 @@
 // Queries, keys and values arrive by TMA straight from the packed q|k|v rows, each tile
 // with the shortest box (32, 64, 96 or 128 rows) that covers it (Qwen3's q/k norm and
 // rotary positions were applied beforehand).  Keys past the row's end get zero
-// probability, so a query's result depends only on its own row: packing never changes a
-// bit.  Every wait is bounded; on expiry the kernel records the error
-// word, drains what it issued, frees its tensor memory and returns.
+// probability (the value rows they meet are finite: other rows' values, or zeros), so a
+// query's result depends only on its own row: packing never changes a bit.  Every wait is
+// bounded; on expiry the kernel records the error word, drains what it issued, frees its
+// tensor memory and returns.
 #include <cuda.h>
 #include <float.h>
 
