@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
         }
     }
 
-    if (EPI == EPI_LSE) {
+    if constexpr (EPI == EPI_LSE) {
         // per row: max and sum of exp over this tile's valid columns; the 16
         // threads of a row sit in one half-warp
 #pragma unroll
@@ -99,31 +99,31 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
             }
         }
         return;
-    }
-
+    } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int m = m0 + ty * 4 + i;
-        if (m >= g.M) continue;
-        float rs = 1.f;
-        if (EPI == EPI_SHRINK) rs = (float)g.row_sign[m] * g.eps;
+        for (int i = 0; i < 4; ++i) {
+            const int m = m0 + ty * 4 + i;
+            if (m >= g.M) continue;
+            float rs = 1.f;
+            if (EPI == EPI_SHRINK) rs = (float)g.row_sign[m] * g.eps;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int n = n0 + tx * 4 + j;
-            if (n >= g.N) continue;
-            float v = acc[i][j];
-            const size_t ci = (size_t)m * g.ldc + n;
-            if (EPI == EPI_SHRINK) {
-                if (n < g.scale_cols) v *= rs;
-                st_elem(g.C, ci, g.c_type, v);
-            } else if (EPI == EPI_RESID) {
-                if (g.bias) v += g.bias[n];
-                float* C = static_cast<float*>(g.C);
-                C[ci] += v;
-            } else {
-                if (g.bias) v += g.bias[n];
-                if (EPI == EPI_STORE_RELU) v = fmaxf(v, 0.f);
-                st_elem(g.C, ci, g.c_type, v);
+            for (int j = 0; j < 4; ++j) {
+                const int n = n0 + tx * 4 + j;
+                if (n >= g.N) continue;
+                float v = acc[i][j];
+                const size_t ci = (size_t)m * g.ldc + n;
+                if (EPI == EPI_SHRINK) {
+                    if (n < g.scale_cols) v *= rs;
+                    st_elem(g.C, ci, g.c_type, v);
+                } else if (EPI == EPI_RESID) {
+                    if (g.bias) v += g.bias[n];
+                    float* C = static_cast<float*>(g.C);
+                    C[ci] += v;
+                } else {
+                    if (g.bias) v += g.bias[n];
+                    if (EPI == EPI_STORE_RELU) v = fmaxf(v, 0.f);
+                    st_elem(g.C, ci, g.c_type, v);
+                }
             }
         }
     }
