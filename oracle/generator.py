@@ -4,7 +4,7 @@ The pages name a "random-direction stream" that the reorganised runtime keeps
 unchanged ("Zeroth-Order Fine-Tuning Was an Inference Workload All Along",
 section "The System Reorganization"), and LoZO's factors U, V of rank r
 ("Why ZO Fine-Tuning Is Really Scoring").  They do not say how the stream is
-drawn; this build fixes one counter-based definition that the CUDA library
+drawn; this library fixes one counter-based definition that the CUDA code
 and this oracle implement independently and must agree on bit for bit:
 
 * splitmix64 (Steele, Lea, Flood 2014; Vigna's public-domain finaliser):
@@ -16,7 +16,7 @@ and this oracle implement independently and must agree on bit for bit:
 * Box-Muller on the 64-bit word b: u1 = ((b >> 40) + 1) * 2^-24 in (0, 1],
   u2 = (b & 0xFFFFFF) * 2^-24; z0 = sqrt(-2 ln u1) cos(2 pi u2),
   z1 = sqrt(-2 ln u1) sin(2 pi u2).
-* ln, sin and cos are this build's own, written from their series so that
+* ln, sin and cos are this library's own, written from their series so that
   both sides reproduce them exactly with +, -, *, / and sqrt alone (no fused
   multiply-add anywhere): ln m = 2 atanh((m-1)/(m+1)) on m in [sqrt(1/2),
   sqrt(2)); sin/cos by their Taylor series on [-pi/4, pi/4] after an exact
