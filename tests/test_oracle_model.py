@@ -155,3 +155,21 @@ def test_bf16_mode_rounds_weights():
     W = w.layers[0]["W0"]
     assert torch.equal(W, W.to(torch.bfloat16).to(torch.float64))
     assert not torch.equal(w.layers[0]["b0"], w.layers[0]["b0"].to(torch.bfloat16).double())
+
+
+@pytest.mark.parametrize("L,H,Hkv,hd", [(1, 4, 4, 8), (7, 8, 2, 16), (33, 6, 3, 32), (64, 4, 1, 128)])
+def test_causal_attention_matches_library_attention_per_head(L, H, Hkv, hd):
+    """The oracle's row attention against torch's scaled-dot-product attention (a library
+    routine, causal), called once per query head h with kv head h // (H / Hkv): pins the
+    1/sqrt(hd) scale, the causal mask, the softmax axis and the grouped-query head mapping
+    (query heads sharing a kv head are consecutive)."""
+    g = torch.Generator().manual_seed(L * 1000 + H)
+    q = torch.randn(L, H, hd, generator=g, dtype=torch.float64)
+    k = torch.randn(L, Hkv, hd, generator=g, dtype=torch.float64)
+    v = torch.randn(L, Hkv, hd, generator=g, dtype=torch.float64)
+    got = om.causal_attention(q, k, v, H // Hkv).reshape(L, H, hd)
+    for h in range(H):
+        kv = h // (H // Hkv)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[:, h][None, None], k[:, kv][None, None], v[:, kv][None, None], is_causal=True)[0, 0]
+        assert torch.allclose(got[:, h], ref, atol=1e-12, rtol=1e-10), h
