@@ -173,3 +173,42 @@ def test_causal_attention_matches_library_attention_per_head(L, H, Hkv, hd):
         ref = torch.nn.functional.scaled_dot_product_attention(
             q[:, h][None, None], k[:, kv][None, None], v[:, kv][None, None], is_causal=True)[0, 0]
         assert torch.allclose(got[:, h], ref, atol=1e-12, rtol=1e-10), h
+
+
+def test_rope_is_a_rotation_whose_dot_products_depend_on_the_offset_only():
+    """Rotary positions (Qwen3's q/k) by their defining properties: position 0 is the
+    identity, each (i, i + hd/2) pair keeps its length, and q(m).k(n) depends on m - n only;
+    the lowest pair turns by exactly m radians at position m (frequency theta^0 = 1)."""
+    hd, theta = 16, 1e6
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(1, 1, hd, generator=g, dtype=torch.float64)
+    k = torch.randn(1, 1, hd, generator=g, dtype=torch.float64)
+    at = lambda x, p: om.rope(x, torch.tensor([p]), theta)  # noqa: E731
+    assert torch.equal(at(q, 0), q)
+    half = hd // 2
+    r = at(q, 37)
+    assert torch.allclose(r[..., :half] ** 2 + r[..., half:] ** 2,
+                          q[..., :half] ** 2 + q[..., half:] ** 2, atol=1e-12)
+    dots = [float((at(q, m) * at(k, m - 5)).sum()) for m in (5, 11, 40, 300)]
+    assert max(dots) - min(dots) < 1e-9, dots
+    a0 = torch.atan2(q[0, 0, half], q[0, 0, 0])
+    a1 = torch.atan2(r[0, 0, half], r[0, 0, 0])
+    turn = float((a1 - a0) % (2 * np.pi))
+    assert abs(turn - 37 % (2 * np.pi)) < 1e-9, turn
+
+
+def test_norms_by_definition():
+    """LayerNorm gives zero mean and unit variance before its affine terms; RMSNorm unit
+    root-mean-square; both scale per feature by w (and LayerNorm shifts by b)."""
+    g = torch.Generator().manual_seed(4)
+    x = torch.randn(5, 24, generator=g, dtype=torch.float64) * 3 + 2
+    one, zero = torch.ones(24, dtype=torch.float64), torch.zeros(24, dtype=torch.float64)
+    y = om.layer_norm(x, one, zero, 0.0)
+    assert torch.allclose(y.mean(-1), torch.zeros(5, dtype=torch.float64), atol=1e-12)
+    assert torch.allclose((y * y).mean(-1), torch.ones(5, dtype=torch.float64), atol=1e-12)
+    z = om.rms_norm(x, one, 0.0)
+    assert torch.allclose((z * z).mean(-1), torch.ones(5, dtype=torch.float64), atol=1e-12)
+    w = torch.randn(24, generator=g, dtype=torch.float64)
+    b = torch.randn(24, generator=g, dtype=torch.float64)
+    assert torch.allclose(om.layer_norm(x, w, b, 0.0), y * w + b, atol=1e-12)
+    assert torch.allclose(om.rms_norm(x, w, 0.0), z * w, atol=1e-12)
