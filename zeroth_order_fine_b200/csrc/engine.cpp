@@ -1157,7 +1157,7 @@ int launch_batch(zo_handle* h, float eps, const int* md, const BatchPlan& bp,
                  d.d_model, h->st);
 
     const int nk = d.arch == ZO_ARCH_OPT ? 0 : 1;   // norm kind
-    int rc = decoder_layers(h, Ti, eps, [&](int l, bool) -> int {
+    int rc = decoder_layers(h, Ti, eps, [&](int, bool) -> int {
             AttnArgs a;
             memset(&a, 0, sizeof(a));
             a.qkv = h->qkv; a.ld_qkv = h->n_qkv;
